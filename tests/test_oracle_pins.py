@@ -1,0 +1,278 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Each test names the passage or the mathematical fact it checks.  Together
+they are chosen so that a plausible slip in the oracle (a dropped gain or
+eps, a wrong sign or pairing in RoPE, a transposed or swapped FFN operand,
+a missing mask, a post-norm ordering, a missing parameter tensor) fails at
+least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import expit
+
+import oracle
+from synth.workloads import TINY, ModelShape
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- RMSNorm
+
+def test_rmsnorm_worked_example_and_centred_identity():
+    """Printed demo: [1,2,3,4] -> x/sqrt(7.5); centred vector equals LayerNorm."""
+    g = _golden("rmsnorm_worked_example.json")
+    for case in g["cases"]:
+        x = np.array(case["x"])
+        y = oracle.rms_norm(x, eps=0.0)
+        assert np.round(y, g["digits"]).tolist() == case["rms_norm"]
+        if "rms_norm_mean" in case:
+            assert round(float(y.mean()), 4) == case["rms_norm_mean"]
+    # the centred case: RMSNorm output equals the printed LayerNorm output
+    c = g["cases"][1]
+    y = oracle.rms_norm(np.array(c["x"]), eps=0.0)
+    assert np.round(y, 4).tolist() == c["layer_norm"]
+
+
+def test_rmsnorm_zeros_eps():
+    """0/0 is NaN with eps = 0; eps = 1e-5 gives zeros (printed)."""
+    z = np.zeros(4)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        assert np.isnan(oracle.rms_norm(z, eps=0.0)).all()
+    assert (oracle.rms_norm(z, eps=1e-5) == 0.0).all()
+
+
+def test_rmsnorm_closed_forms():
+    """eps sits inside the square root; the gain multiplies elementwise; the
+    output has unit root-mean-square and is scale invariant (eps = 0)."""
+    ones = np.ones(8)
+    assert oracle.rms_norm(ones, eps=3.0) == pytest.approx(np.full(8, 0.5), abs=0, rel=1e-15)
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((3, 16))
+    y = oracle.rms_norm(x, eps=0.0)
+    assert np.allclose(np.sqrt((y ** 2).mean(-1)), 1.0, atol=1e-14)
+    assert np.allclose(oracle.rms_norm(37.5 * x, eps=0.0), y, atol=1e-14)
+    gain = rng.standard_normal(16)
+    assert np.allclose(oracle.rms_norm(x, gain, eps=0.0), y * gain, atol=1e-14)
+    # no mean subtraction: a constant vector maps to sign(c) * 1
+    assert np.allclose(oracle.rms_norm(np.full(5, -2.0), eps=0.0), -1.0)
+
+
+# ---------------------------------------------------------------- SiLU / SwiGLU
+
+def test_silu_closed_forms():
+    assert oracle.silu(np.array(0.0)) == 0.0
+    assert oracle.silu(np.array(1.0)) == pytest.approx(1.0 / (1.0 + math.exp(-1.0)), rel=1e-15)
+    u = np.linspace(-30, 30, 601)
+    assert np.allclose(oracle.silu(u), u * expit(u), rtol=1e-13, atol=1e-300)
+    assert oracle.silu(np.array(40.0)) == pytest.approx(40.0, rel=1e-15)
+    s = oracle.silu(np.array(-20.0))
+    assert s < 0 and abs(s) < 1e-7
+    # exact zeros only at 0 (the 0.0% exactly-off units of the SwiGLU demo)
+    r = np.random.default_rng(2).standard_normal(100000)
+    assert np.count_nonzero(oracle.silu(r) == 0.0) == np.count_nonzero(r == 0.0)
+
+
+def test_swiglu_brute_force():
+    """(SiLU(z Wg) * (z Wu)) Wd, every sum written out as a Python loop."""
+    rng = np.random.default_rng(3)
+    n, d, h = 3, 4, 5
+    z = rng.standard_normal((n, d))
+    W = {"wg": rng.standard_normal((d, h)), "wu": rng.standard_normal((d, h)),
+         "wd": rng.standard_normal((h, d))}
+    ref = np.zeros((n, d))
+    for i in range(n):
+        for j in range(d):
+            acc = 0.0
+            for k in range(h):
+                g = sum(z[i, m] * W["wg"][m, k] for m in range(d))
+                u = sum(z[i, m] * W["wu"][m, k] for m in range(d))
+                acc += (g / (1.0 + math.exp(-g))) * u * W["wd"][k, j]
+            ref[i, j] = acc
+    assert np.allclose(oracle.swiglu_ffn(z, W), ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- hidden size, parameter counts
+
+def test_hidden_size_rule():
+    """Size table: 4096->11008, 5120->13824, 6656->17920, 8192->22016 (not 10923)."""
+    for s in _golden("llama_shapes.json")["sizes"]:
+        assert oracle.llama_hidden(s["dim"]) == s["ffn"]
+    assert oracle.llama_hidden(128) == 512
+    assert TINY.ffn_hidden == oracle.llama_hidden(TINY.d_model)
+
+
+def _shape(dim, layers, ffn, vocab):
+    return ModelShape("t", layers, dim, dim // 128, 128, ffn, vocab)
+
+
+def test_parameter_counts_from_allocated_shapes():
+    """count_params column of the size table, summed over every tensor the
+    oracle builds, and the bias=True break (+1,622,016 for 7B)."""
+    g = _golden("llama_shapes.json")
+    for s in g["sizes"]:
+        assert oracle.count_params(_shape(s["dim"], s["layers"], s["ffn"], g["vocab"])) == s["count_params"]
+    s7 = _shape(4096, 32, 11008, g["vocab"])
+    assert oracle.count_params(s7, bias=True) == g["bias_7b"]["count_params"]
+    assert oracle.count_params(s7, bias=True) - oracle.count_params(s7) == g["bias_7b"]["delta"]
+    f = g["ffn_d4096"]
+    d = 4096
+    assert 3 * d * oracle.llama_hidden(d) == f["swiglu_params"]
+    assert 3 * d * 4 * d == f["swiglu_4d_params"]
+    assert 2 * d * 4 * d == f["relu_4d_params"]
+    # inference ~ 2N FLOPs per token
+    assert 2 * oracle.count_params(s7) == pytest.approx(g["inference_flops_per_token_7b"], rel=0.005)
+    assert oracle.count_params(TINY) == 780928
+
+
+# ---------------------------------------------------------------- RoPE
+
+def test_rope_special_cases():
+    """Pair i = (x[2i], x[2i+1]) turns by p * 10000^(-2i/d): with d = 4 the
+    first pair turns by p, the second by p/100; interleaved, not half-split."""
+    p = 0.7
+    out = oracle.rope(np.array([[1.0, 0.0, 0.0, 0.0]]), np.array([p]))
+    assert np.allclose(out, [[math.cos(p), math.sin(p), 0, 0]], atol=1e-15)
+    out = oracle.rope(np.array([[0.0, 1.0, 0.0, 0.0]]), np.array([p]))
+    assert np.allclose(out, [[-math.sin(p), math.cos(p), 0, 0]], atol=1e-15)
+    out = oracle.rope(np.array([[0.0, 0.0, 1.0, 0.0]]), np.array([p]))
+    assert np.allclose(out, [[0, 0, math.cos(p / 100), math.sin(p / 100)]], atol=1e-15)
+    x = np.random.default_rng(4).standard_normal((3, 6, 32))
+    assert np.array_equal(oracle.rope(x, np.zeros(6)), x)          # position 0 = identity
+
+
+def test_rope_preserves_norm_and_depends_on_offset_only():
+    """Each pair is a 2-D rotation (norm preserved); (R_m q).(R_n k) depends
+    only on n - m ([NAR] relative-offset identity), and equals q^T R_{n-m} k."""
+    rng = np.random.default_rng(5)
+    d = 128
+    x = rng.standard_normal((7, d))
+    pos = np.array([0, 1, 5, 100, 1000, 2047, 4096])
+    assert np.allclose(np.linalg.norm(oracle.rope(x, pos), axis=-1), np.linalg.norm(x, axis=-1),
+                       rtol=1e-13)
+    q, k = rng.standard_normal(d), rng.standard_normal(d)
+
+    def score(m, n):
+        return float(oracle.rope(q[None], np.array([m]))[0] @ oracle.rope(k[None], np.array([n]))[0])
+
+    for m, n in [(3, 1), (1, 3), (10, 17), (2000, 5)]:
+        assert score(m, n) == pytest.approx(score(m + 91, n + 91), abs=1e-10)
+        # q^T R_{n-m} k with R built as a block-diagonal rotation matrix
+        theta = 10000.0 ** (-np.arange(0, d, 2) / d)
+        R = np.zeros((d, d))
+        for i, t in enumerate(theta):
+            a = (n - m) * t
+            R[2 * i:2 * i + 2, 2 * i:2 * i + 2] = [[math.cos(a), -math.sin(a)], [math.sin(a), math.cos(a)]]
+        assert score(m, n) == pytest.approx(float(q @ R @ k), abs=1e-10)
+    assert score(3, 1) != pytest.approx(score(3, 0), abs=1e-6)
+
+
+# ---------------------------------------------------------------- attention
+
+def _attention_loops(q, k, v):
+    n, dh = q.shape
+    out = np.zeros_like(v)
+    for t in range(n):
+        s = [sum(q[t, c] * k[j, c] for c in range(dh)) / math.sqrt(dh) for j in range(t + 1)]
+        m = max(s)
+        w = [math.exp(x - m) for x in s]
+        tot = sum(w)
+        for c in range(v.shape[1]):
+            out[t, c] = sum(w[j] * v[j, c] for j in range(t + 1)) / tot
+    return out
+
+
+def test_attention_brute_force():
+    rng = np.random.default_rng(6)
+    for n, dh in [(1, 4), (5, 4), (9, 8)]:
+        q, k, v = (rng.standard_normal((n, dh)) for _ in range(3))
+        assert np.allclose(oracle.causal_attention(q, k, v), _attention_loops(q, k, v),
+                           rtol=1e-12, atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(7)
+    n, dh = 6, 8
+    q, k, v = (rng.standard_normal((n, dh)) for _ in range(3))
+    out = oracle.causal_attention(q, k, v)
+    assert np.array_equal(out[0], v[0])                                   # row 0 sees only key 0
+    same_k = np.tile(k[:1], (n, 1))                                       # equal keys: running mean
+    out2 = oracle.causal_attention(q, same_k, v)
+    assert np.allclose(out2, np.cumsum(v, 0) / np.arange(1, n + 1)[:, None], atol=1e-14)
+    # causality: later q/k/v rows do not move earlier outputs
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    q2[4:] += 3.0
+    k2[4:] -= 2.0
+    v2[4:] *= 5.0
+    assert np.allclose(oracle.causal_attention(q2, k2, v2)[:4], out[:4], atol=1e-15)
+
+
+# ---------------------------------------------------------------- block and model
+
+def _small_shape(layers=2):
+    return ModelShape("s", layers, 64, 4, 16, oracle.llama_hidden(64), 97, dtype="f32")
+
+
+def test_pre_norm_block_identity_when_branches_add_nothing():
+    """Pre-norm: the trunk is only ever added to.  With Wo = Wd = 0 the block
+    returns x exactly (a post-norm block would return norm(x))."""
+    s = _small_shape()
+    W = oracle.layer_weights(s, 0)
+    W["wo"] = np.zeros_like(W["wo"])
+    W["wd"] = np.zeros_like(W["wd"])
+    x = np.random.default_rng(8).standard_normal((5, s.d_model)) * 3.0
+    assert np.array_equal(oracle.block_forward(s, x, weights=W), x)
+
+
+def test_single_token_attention_reduces_to_value_path():
+    """One token: RoPE at position 0 is the identity and the softmax over one
+    key is 1, so the attention branch is RMSNorm(x) Wv Wo (not Wq or Wk)."""
+    s = _small_shape()
+    W = oracle.layer_weights(s, 0)
+    W["wd"] = np.zeros_like(W["wd"])
+    x = np.random.default_rng(9).standard_normal((1, s.d_model))
+    z = x / np.sqrt((x ** 2).mean() + s.norm_eps)
+    expect = x + z @ W["wv"] @ W["wo"]
+    assert np.allclose(oracle.block_forward(s, x, weights=W), expect, atol=1e-13)
+
+
+def test_model_invariants_causality_prefix_decode():
+    s = _small_shape()
+    rng = np.random.default_rng(10)
+    tok = rng.integers(0, s.vocab, size=(2, 12))
+    lg, cache = oracle.prefill(s, tok, return_cache=True)
+    # causality: perturbing tokens after t leaves rows <= t unchanged
+    tok2 = tok.copy()
+    tok2[:, 7:] = (tok2[:, 7:] + 5) % s.vocab
+    assert np.allclose(oracle.prefill(s, tok2)[:, :7], lg[:, :7], atol=1e-12)
+    assert not np.allclose(oracle.prefill(s, tok2)[:, 7:], lg[:, 7:])
+    # prefix truncation
+    assert np.allclose(oracle.prefill(s, tok[:, :5]), lg[:, :5], atol=1e-12)
+    # decode (one token at a time with a KV cache) == prefill row
+    lg9, c9 = oracle.prefill(s, tok[:, :9], return_cache=True)
+    for t in range(9, 12):
+        logits, nxt, c9 = oracle.decode_step(s, c9, tok[:, t])
+        assert np.allclose(logits, lg[:, t], atol=1e-12)
+        assert (nxt == np.argmax(lg[:, t], -1)).all()
+    assert c9[0][0].shape == cache[0][0].shape
+    assert np.allclose(c9[1][0], cache[1][0], atol=1e-12)
+
+
+def test_no_position_signal_at_the_bottom():
+    """Zero blocks: logits = RMSNorm(E[tok]) Whead; the embedding alone, the
+    same token at two positions gives the same logits."""
+    s = _small_shape(layers=0)
+    tok = np.array([[3, 3, 50]])
+    lg = oracle.prefill(s, tok)
+    assert np.array_equal(lg[0, 0], lg[0, 1])
+    E, Wh = oracle.embed_table(s), oracle.head_matrix(s)
+    ref = (E[3] / np.sqrt((E[3] ** 2).mean() + s.norm_eps)) @ Wh
+    assert np.allclose(lg[0, 0], ref, atol=1e-14)
