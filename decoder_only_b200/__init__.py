@@ -1,0 +1,242 @@
+"""Python binding of libllama_b200.so: argument marshalling only.
+
+Every step of the forward pass runs in the library's CUDA kernels; PyTorch
+supplies device memory (one arena tensor per model) and the current stream.
+Importing this package without the built library raises ImportError: there
+is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libllama_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "llama_b200.h")
+
+F32, BF16 = 0, 1
+STATUS = {0: "ok", -1: "invalid argument", -2: "arena or workspace too small", -3: "CUDA error",
+          -4: "bounded device wait expired", -5: "call out of order"}
+
+
+class LlamaError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({code})")
+        self.code = code
+
+
+class LlamaConfig(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int32), ("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("ffn_hidden", ctypes.c_int32), ("vocab", ctypes.c_int32),
+                ("norm_eps", ctypes.c_float), ("rope_theta", ctypes.c_float), ("dtype", ctypes.c_int32),
+                ("max_batch", ctypes.c_int32), ("max_seq", ctypes.c_int32)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m decoder_only_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, U64, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_float
+    sig = {
+        "llama_model_bytes": [P, P],
+        "llama_init_weights": [P, ctypes.c_uint32, P, U64, P, P],
+        "llama_prefill": [P, P, I, I, P, P],
+        "llama_prefill_trunk": [P, P, I, I, P, P],
+        "llama_decode_step": [P, P, P, P, P],
+        "llama_generate": [P, P, I, P, P],
+        "llama_position": [P],
+        "llama_model_tensor": [P, ctypes.c_char_p, I, P, P],
+        "llama_last_error": [P],
+        "llama_free": [P],
+        "llama_status_str": [ctypes.c_int],
+        "llama_op_rmsnorm": [I, P, P, P, I, I, F, P],
+        "llama_op_gemm": [I, P, P, P, I, I, I, I, P],
+        "llama_op_attention_prefill": [I, P, P, P, P, I, I, I, I, I, P],
+        "llama_op_attention_decode": [I, P, P, P, P, I, I, I, I, I, P, U64, P],
+        "llama_op_attention_decode_work_bytes": [I, I, I, I],
+        "llama_op_argmax": [P, I, I, P, P],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    lib.llama_free.restype = None
+    lib.llama_status_str.restype = ctypes.c_char_p
+    lib.llama_op_attention_decode_work_bytes.restype = U64
+    return lib
+
+
+lib = _load()
+
+
+def header_symbols() -> list[str]:
+    """Names of the entry points include/llama_b200.h declares."""
+    with open(HEADER_PATH) as f:
+        return re.findall(r"^LLAMA_API\s+[\w\s\*]+?\b(llama_\w+)\s*\(", f.read(), flags=re.M)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise LlamaError(rc, what)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def make_config(shape, max_batch: int, max_seq: int) -> LlamaConfig:
+    """`shape`: any object with n_layers, d_model, n_heads, head_dim,
+    ffn_hidden, vocab, dtype ('bf16' | 'f32'), norm_eps, rope_theta."""
+    return LlamaConfig(shape.n_layers, shape.d_model, shape.n_heads, shape.head_dim, shape.ffn_hidden,
+                       shape.vocab, shape.norm_eps, shape.rope_theta, BF16 if shape.dtype == "bf16" else F32,
+                       max_batch, max_seq)
+
+
+def model_bytes(cfg: LlamaConfig) -> int:
+    n = ctypes.c_uint64()
+    _check(lib.llama_model_bytes(ctypes.byref(cfg), ctypes.byref(n)), "llama_model_bytes")
+    return n.value
+
+
+class Model:
+    """One model in one device arena.  Weights are generated on the device."""
+
+    def __init__(self, shape, max_batch: int, max_seq: int, seed: int = 0):
+        self.shape = shape
+        self.cfg = make_config(shape, max_batch, max_seq)
+        nbytes = model_bytes(self.cfg)
+        self.arena = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        h = ctypes.c_void_p()
+        _check(lib.llama_init_weights(ctypes.byref(self.cfg), seed, _ptr(self.arena), nbytes, _stream(),
+                                      ctypes.byref(h)), "llama_init_weights")
+        self.h = h
+        self.wdtype = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+
+    def close(self):
+        if self.h:
+            lib.llama_free(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def position(self) -> int:
+        return lib.llama_position(self.h)
+
+    def prefill(self, tokens: torch.Tensor, logits: bool = True):
+        """tokens int32 [B, S] on the device -> logits fp32 [B, S, V] (or None)."""
+        B, S = tokens.shape
+        tokens = tokens.contiguous()
+        out = torch.empty(B, S, self.cfg.vocab, dtype=torch.float32, device="cuda") if logits else None
+        _check(lib.llama_prefill(self.h, _ptr(tokens), B, S, _ptr(out), _stream()), "llama_prefill")
+        return out
+
+    def prefill_trunk(self, x: torch.Tensor, out: torch.Tensor | None = None):
+        """x fp32 [B, S, d] -> trunk after the blocks, fp32 [B, S, d]."""
+        B, S, _ = x.shape
+        x = x.contiguous()
+        y = torch.empty_like(x) if out is None else out
+        _check(lib.llama_prefill_trunk(self.h, _ptr(x), B, S, _ptr(y), _stream()), "llama_prefill_trunk")
+        return y
+
+    def decode_step(self, tokens: torch.Tensor, logits: bool = True):
+        B = tokens.shape[0]
+        nxt = torch.empty(B, dtype=torch.int32, device="cuda")
+        lg = torch.empty(B, self.cfg.vocab, dtype=torch.float32, device="cuda") if logits else None
+        _check(lib.llama_decode_step(self.h, _ptr(tokens.contiguous()), _ptr(nxt), _ptr(lg), _stream()),
+               "llama_decode_step")
+        return nxt, lg
+
+    def generate(self, first: torch.Tensor, n_steps: int, out: torch.Tensor | None = None):
+        B = first.shape[0]
+        out = torch.empty(n_steps, B, dtype=torch.int32, device="cuda") if out is None else out
+        _check(lib.llama_generate(self.h, _ptr(first.contiguous()), n_steps, _ptr(out), _stream()),
+               "llama_generate")
+        return out
+
+    def tensor(self, name: str, layer: int = 0, dtype=None, shape=None) -> torch.Tensor:
+        """A view of an internal buffer (see llama_model_tensor)."""
+        p, n = ctypes.c_void_p(), ctypes.c_uint64()
+        _check(lib.llama_model_tensor(self.h, name.encode(), layer, ctypes.byref(p), ctypes.byref(n)),
+               "llama_model_tensor")
+        off = p.value - self.arena.data_ptr()
+        t = self.arena[off:off + n.value]
+        if dtype is not None:
+            t = t.view(dtype)
+        if shape is not None:
+            t = t[: int(torch.Size(shape).numel())].view(shape)
+        return t
+
+    def last_error(self) -> int:
+        return lib.llama_last_error(self.h)
+
+
+# ----------------------------------------------------------------- single ops
+
+def rmsnorm(x: torch.Tensor, g: torch.Tensor, eps: float, out_dtype=torch.bfloat16) -> torch.Tensor:
+    rows, d = x.shape
+    y = torch.empty(rows, d, dtype=out_dtype, device=x.device)
+    _check(lib.llama_op_rmsnorm(_dt(y), _ptr(x.contiguous()), _ptr(g.contiguous()), _ptr(y), rows, d, eps,
+                                _stream()), "llama_op_rmsnorm")
+    return y
+
+
+def gemm(A: torch.Tensor, W: torch.Tensor, C: torch.Tensor | None = None, accumulate: bool = False):
+    """C (+)= A W^T, A [M, K], W [N, K] (same dtype), C fp32 [M, N]."""
+    M, K = A.shape
+    N = W.shape[0]
+    if C is None:
+        C = torch.empty(M, N, dtype=torch.float32, device=A.device)
+    _check(lib.llama_op_gemm(_dt(A), _ptr(A.contiguous()), _ptr(W.contiguous()), _ptr(C), M, N, K,
+                             1 if accumulate else 0, _stream()), "llama_op_gemm")
+    return C
+
+
+def attention_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> torch.Tensor:
+    """q [B, H, S, hd]; k, v [B, H, kv_stride, hd] -> o [B*S, H*hd]."""
+    B, H, S, hd = q.shape
+    kv_stride = k.shape[2]
+    o = torch.empty(B * S, H * hd, dtype=q.dtype, device=q.device)
+    _check(lib.llama_op_attention_prefill(_dt(q), _ptr(q.contiguous()), _ptr(k.contiguous()), _ptr(v.contiguous()),
+                                          _ptr(o), B, H, S, hd, kv_stride, _stream()), "llama_op_attention_prefill")
+    return o
+
+
+def attention_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, length: int,
+                     work: torch.Tensor | None = None) -> torch.Tensor:
+    """q [B, H*hd]; k, v [B, H, kv_stride, hd]; keys 0..length-1 -> o [B, H*hd]."""
+    B, H, kv_stride, hd = k.shape
+    nbytes = lib.llama_op_attention_decode_work_bytes(B, H, length, hd)
+    if work is None:
+        work = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    o = torch.empty(B, H * hd, dtype=q.dtype, device=q.device)
+    _check(lib.llama_op_attention_decode(_dt(q), _ptr(q.contiguous()), _ptr(k.contiguous()), _ptr(v.contiguous()),
+                                         _ptr(o), B, H, length, hd, kv_stride, _ptr(work), work.numel(),
+                                         _stream()), "llama_op_attention_decode")
+    return o
+
+
+def argmax(logits: torch.Tensor) -> torch.Tensor:
+    rows, n = logits.shape
+    out = torch.empty(rows, dtype=torch.int32, device=logits.device)
+    _check(lib.llama_op_argmax(_ptr(logits.contiguous()), rows, n, _ptr(out), _stream()), "llama_op_argmax")
+    return out

@@ -1,0 +1,250 @@
+// Decode-side kernels: split-sequence attention over the contiguous KV cache
+// and the split-K reduction that finishes the decode GEMMs.
+//
+// Decode attention ("GQA Was Not an Original LLaMA Feature": every step
+// reads the keys and values of all previous tokens) is HBM-bound: each
+// (sequence, head) streams len * head_dim * 2 elements once.  The sequence
+// is cut into chunks of 256 keys so that B*H*chunks CTAs cover the SMs; each
+// chunk leaves (max, sum, unnormalised output) in the workspace and a second
+// pass merges the chunks (the online-softmax merge rule).
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "kernels.h"
+
+constexpr int DEC_CHUNK = 256;   // keys per CTA
+constexpr int DEC_WARPS = 4;
+
+template <typename T> struct Vec16;                      // 16 bytes of T
+template <> struct Vec16<bf16> { static constexpr int N = 8; };
+template <> struct Vec16<float> { static constexpr int N = 4; };
+
+template <typename T>
+__device__ __forceinline__ void load16(const T* p, float* out);
+template <>
+__device__ __forceinline__ void load16<bf16>(const bf16* p, float* out) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
+    float2 f;
+    f = unpack_bf16x2(w.x); out[0] = f.x; out[1] = f.y;
+    f = unpack_bf16x2(w.y); out[2] = f.x; out[3] = f.y;
+    f = unpack_bf16x2(w.z); out[4] = f.x; out[5] = f.y;
+    f = unpack_bf16x2(w.w); out[6] = f.x; out[7] = f.y;
+}
+template <>
+__device__ __forceinline__ void load16<float>(const float* p, float* out) {
+    const float4 w = __ldg(reinterpret_cast<const float4*>(p));
+    out[0] = w.x; out[1] = w.y; out[2] = w.z; out[3] = w.w;
+}
+
+// Eight lanes share one key: lane (g*8 + r) holds dims [r*DPL, (r+1)*DPL).
+template <typename T, int HD>
+__global__ void __launch_bounds__(DEC_WARPS * 32) attn_decode_partial_kernel(
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, int H, int len_static,
+    const int* __restrict__ d_len_minus1, int kv_stride, float scale, float* __restrict__ work, int n_chunks) {
+    constexpr int DPL = HD / 8;                 // dims per lane
+    constexpr int VPL = DPL / Vec16<T>::N;      // 16-byte loads per lane per row
+    const int len = d_len_minus1 ? (*d_len_minus1 + 1) : len_static;
+    const int chunk = blockIdx.x;
+    const int bh = blockIdx.y;                  // b*H + h
+    const int b = bh / H, h = bh - b * H;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 3, r = lane & 7;
+    const int k_begin = chunk * DEC_CHUNK;
+    const int k_stop = min(len, k_begin + DEC_CHUNK);
+
+    float qv[DPL];
+    {
+        const T* qp = q + ((size_t)b * H + h) * HD + r * DPL;
+#pragma unroll
+        for (int u = 0; u < VPL; ++u) load16<T>(qp + u * Vec16<T>::N, qv + u * Vec16<T>::N);
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) qv[j] *= scale;
+    }
+    float m = -INFINITY, l = 0.f, o[DPL];
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) o[j] = 0.f;
+
+    const size_t head_off = ((size_t)b * H + h) * (size_t)kv_stride * HD;
+    const T* kh = k + head_off + r * DPL;
+    const T* vh = v + head_off + r * DPL;
+    // The warp walks keys jb + g (g = 0..3) with jb warp-uniform, so every
+    // lane takes part in the shuffles; a group past the end skips the update.
+    for (int jb = k_begin + warp * 4; jb < k_stop; jb += DEC_WARPS * 4) {
+        const int j = jb + g;
+        const bool valid = j < k_stop;
+        float kk[DPL], vv[DPL];
+        if (valid) {
+#pragma unroll
+            for (int u = 0; u < VPL; ++u) {
+                load16<T>(kh + (size_t)j * HD + u * Vec16<T>::N, kk + u * Vec16<T>::N);
+                load16<T>(vh + (size_t)j * HD + u * Vec16<T>::N, vv + u * Vec16<T>::N);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) kk[e] = vv[e] = 0.f;
+        }
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) s = fmaf(qv[e], kk[e], s);
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        if (valid) {
+            const float m_new = fmaxf(m, s);
+            const float corr = __expf(m - m_new);
+            const float p = __expf(s - m_new);
+            l = l * corr + p;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) o[e] = fmaf(o[e], corr, p * vv[e]);
+            m = m_new;
+        }
+    }
+    // merge the 16 key groups (4 per warp x 4 warps) through shared memory
+    __shared__ float sm_m[DEC_WARPS * 4], sm_l[DEC_WARPS * 4];
+    __shared__ float sm_o[DEC_WARPS * 4][HD];
+    const int grp = warp * 4 + g;
+    if (r == 0) {
+        sm_m[grp] = m;
+        sm_l[grp] = l;
+    }
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) sm_o[grp][r * DPL + e] = o[e];
+    __syncthreads();
+    float M = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < DEC_WARPS * 4; ++t) M = fmaxf(M, sm_m[t]);
+    float* wp = work + ((size_t)bh * n_chunks + chunk) * (HD + 2);
+    for (int c = threadIdx.x; c < HD; c += blockDim.x) {
+        float acc = 0.f;
+#pragma unroll
+        for (int t = 0; t < DEC_WARPS * 4; ++t)
+            if (sm_m[t] != -INFINITY) acc += sm_o[t][c] * __expf(sm_m[t] - M);
+        wp[2 + c] = acc;
+    }
+    if (threadIdx.x == 0) {
+        float L = 0.f;
+#pragma unroll
+        for (int t = 0; t < DEC_WARPS * 4; ++t)
+            if (sm_m[t] != -INFINITY) L += sm_l[t] * __expf(sm_m[t] - M);
+        wp[0] = M;
+        wp[1] = L;
+    }
+}
+
+template <typename T, int HD>
+__global__ void attn_decode_combine_kernel(const float* __restrict__ work, int n_chunks, int len_static,
+                                           const int* __restrict__ d_len_minus1, int H, T* __restrict__ o) {
+    const int len = d_len_minus1 ? (*d_len_minus1 + 1) : len_static;
+    const int used = min(n_chunks, (len + DEC_CHUNK - 1) / DEC_CHUNK);
+    const int bh = blockIdx.x;
+    const float* wp = work + (size_t)bh * n_chunks * (HD + 2);
+    float M = -INFINITY;
+    for (int c = 0; c < used; ++c) M = fmaxf(M, wp[(size_t)c * (HD + 2)]);
+    for (int e = threadIdx.x; e < HD; e += blockDim.x) {
+        float L = 0.f, acc = 0.f;
+        for (int c = 0; c < used; ++c) {
+            const float mc = wp[(size_t)c * (HD + 2)];
+            if (mc == -INFINITY) continue;
+            const float w = __expf(mc - M);
+            L += wp[(size_t)c * (HD + 2) + 1] * w;
+            acc += wp[(size_t)c * (HD + 2) + 2 + e] * w;
+        }
+        o[(size_t)bh * HD + e] = from_f32<T>(acc / L);
+    }
+}
+
+uint64_t attention_decode_work_bytes(int B, int H, int max_len, int hd) {
+    const int n_chunks = (max_len + DEC_CHUNK - 1) / DEC_CHUNK;
+    return (uint64_t)B * H * n_chunks * (hd + 2) * sizeof(float);
+}
+
+template <typename T, int HD>
+static int launch_dec_t(const void* q, const void* k, const void* v, void* o, int B, int H, int len,
+                        const int* d_len_minus1, int kv_stride, float* work, cudaStream_t st) {
+    // With a device-side length, size the grid for the largest length the
+    // cache can hold; chunks past the live length exit at once.
+    const int grid_len = d_len_minus1 ? kv_stride : len;
+    const int n_chunks = (grid_len + DEC_CHUNK - 1) / DEC_CHUNK;
+    dim3 grid(n_chunks, B * H);
+    attn_decode_partial_kernel<T, HD><<<grid, DEC_WARPS * 32, 0, st>>>(
+        (const T*)q, (const T*)k, (const T*)v, H, len, d_len_minus1, kv_stride, 1.0f / sqrtf((float)HD), work,
+        n_chunks);
+    LLAMA_LAUNCH_CHECK();
+    attn_decode_combine_kernel<T, HD><<<B * H, HD, 0, st>>>(work, n_chunks, len, d_len_minus1, H, (T*)o);
+    LLAMA_LAUNCH_CHECK();
+    return LLAMA_OK;
+}
+
+int launch_attention_decode(int dtype, const void* q, const void* k, const void* v, void* o, int B, int H,
+                            int len, const int* d_len_minus1, int hd, int kv_stride, float* work,
+                            cudaStream_t st) {
+    if (B <= 0) return LLAMA_OK;
+#define DEC_CASE(TT, HH) return launch_dec_t<TT, HH>(q, k, v, o, B, H, len, d_len_minus1, kv_stride, work, st)
+    if (dtype == LLAMA_BF16) {
+        if (hd == 128) DEC_CASE(bf16, 128);
+        if (hd == 64) DEC_CASE(bf16, 64);
+    } else {
+        if (hd == 128) DEC_CASE(float, 128);
+        if (hd == 64) DEC_CASE(float, 64);
+        if (hd == 32) DEC_CASE(float, 32);
+    }
+#undef DEC_CASE
+    return LLAMA_ERR_INVALID_ARG;
+}
+
+// ---------------------------------------------------------------------------
+// Split-K reduction of the decode GEMMs, then the epilogue.
+// partial: fp32 [splits][M][N] (M = batch rows, N = output features).
+template <typename T, int MODE>
+__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int splits, EpiArgs a) {
+    const int chunks = (MODE == EPI_SWIGLU ? a.hidden : a.N) / 32;
+    const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)a.M * chunks) return;
+    const int m = (int)(idx / chunks);
+    const int c = (int)(idx - (int64_t)m * chunks);
+    const size_t plane = (size_t)a.M * a.N;
+    if (MODE == EPI_SWIGLU) {
+        const int j0 = c * 32;
+        const int ng = (j0 / 128) * 256 + (j0 % 128);
+        float g[32], u[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) g[j] = u[j] = 0.f;
+        for (int s = 0; s < splits; ++s) {
+            const float* row = partial + s * plane + (size_t)m * a.N;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                g[j] += row[ng + j];
+                u[j] += row[ng + 128 + j];
+            }
+        }
+        epi_swiglu32<T>(a, m, j0, g, u);
+    } else {
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        const int n0 = c * 32;
+        for (int s = 0; s < splits; ++s) {
+            const float* row = partial + s * plane + (size_t)m * a.N + n0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += row[j];
+        }
+        if (MODE == EPI_QKV) epi_qkv32<T>(a, m, n0, v);
+        else if (MODE == EPI_RESID) epi_resid32(a, m, n0, v);
+        else epi_f32_32(a, m, n0, v);
+    }
+}
+
+int launch_splitk_reduce(int mode, const float* partial, int splits, const EpiArgs& a, cudaStream_t st) {
+    const int chunks = (mode == EPI_SWIGLU ? a.hidden : a.N) / 32;
+    const int64_t total = (int64_t)a.M * chunks;
+    if (total == 0) return LLAMA_OK;
+    const int blocks = (int)((total + 63) / 64);
+    switch (mode) {
+        case EPI_SWIGLU: splitk_reduce_kernel<bf16, EPI_SWIGLU><<<blocks, 64, 0, st>>>(partial, splits, a); break;
+        case EPI_QKV: splitk_reduce_kernel<bf16, EPI_QKV><<<blocks, 64, 0, st>>>(partial, splits, a); break;
+        case EPI_RESID: splitk_reduce_kernel<bf16, EPI_RESID><<<blocks, 64, 0, st>>>(partial, splits, a); break;
+        case EPI_F32: splitk_reduce_kernel<bf16, EPI_F32><<<blocks, 64, 0, st>>>(partial, splits, a); break;
+        default: return LLAMA_ERR_INVALID_ARG;
+    }
+    LLAMA_LAUNCH_CHECK();
+    return LLAMA_OK;
+}

@@ -1,0 +1,526 @@
+// bf16 tensor-core GEMM for sm_100a: tcgen05.mma with fp32 accumulators in
+// tensor memory, operands staged by TMA, fused epilogues.
+//
+// Computes D[r, c] = sum_k A[r, k] * B[c, k] for the projections of the
+// block ("The one formula"): Q/K/V (+RoPE), O (+residual), gate/up
+// (+SwiGLU), down (+residual) and the output head.  Both operands are
+// K-major bf16; A supplies the 128 rows that map onto the 128 TMEM lanes.
+//
+//   prefill (swap = 0): A = activations [tokens, K], B = weights [N, K],
+//                       tile 128 x 256, fused epilogue on the output tile.
+//   decode  (swap = 1): A = weights [N, K], B = activations [batch, K]
+//                       (batch <= 32, zero-filled to 16 or 32 rows by TMA),
+//                       tile 128 x {16, 32}, split over K; fp32 partial
+//                       tiles go to a workspace and a reduction applies the
+//                       epilogue.  Weight streaming is HBM-bound: deep TMA
+//                       ring, grid sized to the SM count.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over tiles):
+//   warp 0      TMA producer (one elected lane): stage ring of S slots
+//   warp 1      TMEM allocator + MMA issuer (one lane): 4 x K=16 per stage
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns per warp,
+//               TMEM accumulators double-buffered so the epilogue of
+//               tile i overlaps the mainloop of tile i+1.
+// Every mbarrier wait is bounded (~2 s); on expiry the CTA records
+// LLAMA_DEVERR_TIMEOUT in the error word, drains its own TMA copies, frees
+// its TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "kernels.h"
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                 // 64 bf16 = one 128-byte swizzle row
+constexpr int NTHREADS = 192;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_timer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait; false when this CTA is aborting (timeout here or elsewhere).
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_timer() - t0 > WAIT_LIMIT_NS) {
+            *abort_flag = 1;
+            atomicOr(err, LLAMA_DEVERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+        "[%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major tile, rows of 128 bytes with the
+// 128-byte swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);   // start address
+    d |= (uint64_t)1 << 16;                      // leading byte offset (unused for this layout)
+    d |= (uint64_t)(1024 >> 4) << 32;            // stride byte offset
+    d |= (uint64_t)1 << 46;                      // descriptor version
+    d |= (uint64_t)2 << 61;                      // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+#define TMEM_LD_X16(taddr, r)                                                                          \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+                 "%15}, [%16];"                                                                        \
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),  \
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),         \
+                   "=r"(r[13]), "=r"(r[14]), "=r"(r[15])                                               \
+                 : "r"(taddr))
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[16];
+    TMEM_LD_X16(taddr, r);
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+#pragma unroll
+    for (int i = 16; i < 32; ++i) v[i] = 0.f;
+}
+
+template <int BN>
+struct Cfg {
+    static constexpr int A_BYTES = BM * BK * 2;            // 16 KB
+    static constexpr int B_BYTES = BN * BK * 2;            // BN * 128 B
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = (BN >= 256) ? 4 : 8;
+    static constexpr int TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;   // two accumulators, power of 2
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+struct TileSched {
+    int m_blocks, n_blocks, splits, kb_total, group;
+    __device__ __forceinline__ int num_tiles() const { return m_blocks * n_blocks * splits; }
+    // prefill: grouped raster (group m-blocks, n fastest inside a group); decode: m fastest
+    __device__ __forceinline__ void get(int t, int& mb, int& nb, int& sp, int& kb0, int& kb1) const {
+        if (splits > 1 || n_blocks == 1) {
+            mb = t % m_blocks;
+            const int rest = t / m_blocks;
+            nb = rest % n_blocks;
+            sp = rest / n_blocks;
+        } else {
+            const int per_group = group * n_blocks;
+            const int g = t / per_group;
+            const int w = t - g * per_group;
+            const int gm = min(group, m_blocks - g * group);
+            mb = g * group + w % gm;
+            nb = w / gm;
+            sp = 0;
+        }
+        const int per = (kb_total + splits - 1) / splits;
+        kb0 = sp * per;
+        kb1 = min(kb_total, kb0 + per);
+    }
+};
+
+template <int BN, int MODE>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TileSched ts,
+                   EpiArgs ep, int* err) {
+    using C = Cfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    const uint32_t sA = base;                                   // STAGES x A tile
+    const uint32_t sB = base + C::STAGES * C::A_BYTES;          // STAGES x B tile
+    const uint32_t bars = base + C::STAGES * C::STAGE_BYTES;    // barrier block
+    const uint32_t full_bar = bars;                             // [STAGES]
+    const uint32_t empty_bar = bars + 8 * C::STAGES;            // [STAGES]
+    const uint32_t tfull_bar = bars + 16 * C::STAGES;           // [2]
+    const uint32_t tempty_bar = tfull_bar + 16;                 // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::STAGES * C::STAGE_BYTES + 16 * C::STAGES + 32);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(full_bar + 8 * s, 1);
+            mbar_init(empty_bar + 8 * s, 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(tfull_bar + 8 * i, 1);
+            mbar_init(tempty_bar + 8 * i, 128);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int n_tiles = ts.num_tiles();
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t filled = 0, fill_phase = 0;   // per-stage: filled at least once / parity of last fill
+            bool ok = true;
+            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+                int mb, nb, sp, kb0, kb1;
+                ts.get(t, mb, nb, sp, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(empty_bar + 8 * stage, phase ^ 1u, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(full_bar + 8 * stage, C::STAGE_BYTES);
+                    tma_load_2d(sA + stage * C::A_BYTES, &tmA, full_bar + 8 * stage, kb * BK, mb * BM);
+                    tma_load_2d(sB + stage * C::B_BYTES, &tmB, full_bar + 8 * stage, kb * BK, nb * BN);
+                    filled |= 1u << stage;
+                    fill_phase = (fill_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // drain: wait (bounded) for the copies this thread issued
+                for (int s = 0; s < C::STAGES; ++s) {
+                    if (!(filled >> s & 1u)) continue;
+                    const uint64_t t0 = global_timer();
+                    while (!mbar_try_wait(full_bar + 8 * s, (fill_phase >> s) & 1u) &&
+                           global_timer() - t0 < WAIT_LIMIT_NS / 4) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC = idesc_bf16(BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+                int mb, nb, sp, kb0, kb1;
+                ts.get(t, mb, nb, sp, kb0, kb1);
+                if (!mbar_wait(tempty_bar + 8 * acc, acc_phase ^ 1u, abort_flag, err)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(full_bar + 8 * stage, phase, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t da = sw128_desc(sA + stage * C::A_BYTES);
+                    const uint64_t db = sw128_desc(sB + stage * C::B_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)   // +32 bytes along K per step (encoded >> 4)
+                        umma_bf16(d_tmem, da + 2 * k, db + 2 * k, IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
+                    umma_commit(empty_bar + 8 * stage);
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(tfull_bar + 8 * acc);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue warps 2..5
+        const int quarter = warp & 3;                    // TMEM lanes [32*quarter, 32*quarter + 32)
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+            int mb, nb, sp, kb0, kb1;
+            ts.get(t, mb, nb, sp, kb0, kb1);
+            if (!mbar_wait(tfull_bar + 8 * acc, acc_phase, abort_flag, err)) break;
+            tc_fence_after();
+            const uint32_t tacc = tmem_base + lane_addr + (uint32_t)(acc * BN);
+            const int row = mb * BM + quarter * 32 + lane;   // row of operand A
+            if constexpr (MODE == EPI_PARTIAL) {
+                // row = output feature n; columns = batch rows
+                float v[32];
+                if constexpr (BN == 16) tmem_ld16(tacc, v);
+                else tmem_ld32(tacc, v);
+                if (row < ep.N) {
+                    float* dst = ep.out + (size_t)sp * ep.M * ep.N + row;
+#pragma unroll
+                    for (int b = 0; b < BN; ++b)
+                        if (b < ep.M) dst[(size_t)b * ep.N] = v[b];
+                }
+            } else if constexpr (MODE == EPI_SWIGLU) {
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float g[32], u[32];
+                    tmem_ld32(tacc + c * 32, g);
+                    tmem_ld32(tacc + 128 + c * 32, u);
+                    if (row < ep.M) epi_swiglu32<bf16>(ep, row, nb * 128 + c * 32, g, u);
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(tacc + c * 32, v);
+                    const int n0 = nb * BN + c * 32;
+                    if (row < ep.M && n0 < ep.N) {
+                        if constexpr (MODE == EPI_F32) epi_f32_32(ep, row, n0, v);
+                        else if constexpr (MODE == EPI_RESID) epi_resid32(ep, row, n0, v);
+                        else epi_qkv32<bf16>(ep, row, n0, v);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(tempty_bar + 8 * acc);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D K-major bf16 map: dims (K, rows), box (64, box_rows), 128-byte swizzle,
+// out-of-range rows read as zero.
+int make_map(CUtensorMap* map, const void* ptr, int rows, int K, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return LLAMA_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <int BN, int MODE>
+int ensure_attr() {
+    static bool attr = false;
+    if (!attr) {
+        LLAMA_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            Cfg<BN>::SMEM));
+        attr = true;
+    }
+    return LLAMA_OK;
+}
+
+template <int BN, int MODE>
+int run(const CUtensorMap& ma, const CUtensorMap& mb, const TileSched& ts, const EpiArgs& a, int* err,
+        cudaStream_t st) {
+    using C = Cfg<BN>;
+    int rc = ensure_attr<BN, MODE>();
+    if (rc) return rc;
+    const int tiles = ts.m_blocks * ts.n_blocks * ts.splits;
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    gemm_tc_kernel<BN, MODE><<<grid, NTHREADS, C::SMEM, st>>>(ma, mb, ts, a, err);
+    LLAMA_LAUNCH_CHECK();
+    return LLAMA_OK;
+}
+
+}  // namespace
+
+int gemm_tc_prepare() {
+    if (!encode_fn()) return LLAMA_ERR_CUDA;
+    num_sms();
+    int rc;
+    if ((rc = ensure_attr<256, EPI_F32>())) return rc;
+    if ((rc = ensure_attr<256, EPI_RESID>())) return rc;
+    if ((rc = ensure_attr<256, EPI_SWIGLU>())) return rc;
+    if ((rc = ensure_attr<256, EPI_QKV>())) return rc;
+    if ((rc = ensure_attr<16, EPI_PARTIAL>())) return rc;
+    return ensure_attr<32, EPI_PARTIAL>();
+}
+
+int gemm_tc_pick_splits(int rowsA, int K) {
+    const int m_blocks = (rowsA + BM - 1) / BM;
+    const int kb = K / BK;
+    const int sms = num_sms();
+    int best = 1;
+    double best_eff = 0.0;
+    for (int s = 1; s <= 16 && s <= kb / 2; ++s) {
+        const int per = (kb + s - 1) / s;
+        if ((s - 1) * per >= kb) continue;        // the last split would own no k-block
+        const int tiles = m_blocks * s;
+        const int waves = (tiles + sms - 1) / sms;
+        double eff = (double)tiles / (double)(waves * sms);
+        if (tiles < sms) eff *= 0.5;              // leaves SMs idle
+        eff -= 0.004 * s;                         // partial-sum traffic and reduction work
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best = s;
+        }
+    }
+    return best;
+}
+
+int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaStream_t st) {
+    if (g.K % BK != 0 || g.K <= 0 || g.rowsA <= 0 || g.rowsB <= 0) return LLAMA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(g.A) | reinterpret_cast<uintptr_t>(g.B)) & 15u) return LLAMA_ERR_INVALID_ARG;
+    CUtensorMap ma, mb;
+    TileSched ts;
+    ts.kb_total = g.K / BK;
+    ts.group = 16;
+    if (mode == EPI_PARTIAL) {
+        if (g.rowsB > 32) return LLAMA_ERR_INVALID_ARG;
+        const int bn = g.rowsB <= 16 ? 16 : 32;
+        ts.m_blocks = (g.rowsA + BM - 1) / BM;
+        ts.n_blocks = 1;
+        ts.splits = g.splits < 1 ? 1 : (g.splits > ts.kb_total ? ts.kb_total : g.splits);
+        // every split must own at least one k-block
+        while (ts.splits > 1 && (ts.splits - 1) * ((ts.kb_total + ts.splits - 1) / ts.splits) >= ts.kb_total)
+            --ts.splits;
+        if (ts.splits != g.splits) return LLAMA_ERR_INVALID_ARG;
+        int rc = make_map(&ma, g.A, g.rowsA, g.K, BM);
+        if (rc) return rc;
+        rc = make_map(&mb, g.B, g.rowsB, g.K, bn);
+        if (rc) return rc;
+        if (bn == 16) return run<16, EPI_PARTIAL>(ma, mb, ts, a, err, st);
+        return run<32, EPI_PARTIAL>(ma, mb, ts, a, err, st);
+    }
+    constexpr int BN = 256;
+    ts.m_blocks = (g.rowsA + BM - 1) / BM;
+    ts.n_blocks = (g.rowsB + BN - 1) / BN;
+    ts.splits = 1;
+    if (mode == EPI_SWIGLU && g.rowsB % 256 != 0) return LLAMA_ERR_INVALID_ARG;
+    if ((mode == EPI_RESID || mode == EPI_QKV) && g.rowsB % 32 != 0) return LLAMA_ERR_INVALID_ARG;
+    int rc = make_map(&ma, g.A, g.rowsA, g.K, BM);
+    if (rc) return rc;
+    rc = make_map(&mb, g.B, g.rowsB, g.K, BN);
+    if (rc) return rc;
+    switch (mode) {
+        case EPI_F32: return run<BN, EPI_F32>(ma, mb, ts, a, err, st);
+        case EPI_RESID: return run<BN, EPI_RESID>(ma, mb, ts, a, err, st);
+        case EPI_SWIGLU: return run<BN, EPI_SWIGLU>(ma, mb, ts, a, err, st);
+        case EPI_QKV: return run<BN, EPI_QKV>(ma, mb, ts, a, err, st);
+        default: return LLAMA_ERR_INVALID_ARG;
+    }
+}

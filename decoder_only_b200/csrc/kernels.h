@@ -1,0 +1,50 @@
+// Internal launchers of the llama_b200 kernels (host side).  Every function
+// queues work on `st` and returns a llama_status.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "llama_b200.h"
+
+struct EpiArgs;
+
+// init.cu
+int launch_init_matrix(int dtype, void* dst, int K, int N_log, int blk, int blk_stride, int row_off,
+                       int rowmajor_nk, uint32_t seed, uint32_t tensor_id, double scale, cudaStream_t st);
+int launch_fill_f32(float* dst, float v, int64_t n, cudaStream_t st);
+
+// norm.cu
+int launch_rmsnorm(int dtype, const float* x, const float* g, void* y, int rows, int d, float eps,
+                   cudaStream_t st);
+int launch_embed(int dtype, const int32_t* tok, const void* E, float* x, int rows, int d, int vocab, int* err,
+                 cudaStream_t st);
+int launch_argmax(const float* logits, int rows, int n, int32_t* out, cudaStream_t st);
+
+// simt.cu  (fp32 storage path and shared epilogue passes)
+int launch_gemm_simt(int dtype, const void* A, const void* W, float* C, int M, int N, int K, int accumulate,
+                     cudaStream_t st);
+int launch_epilogue_from_f32(int dtype, int mode, const float* C, int ldc, const EpiArgs& a, cudaStream_t st);
+int launch_attention_prefill_simt(int dtype, const void* q, const void* k, const void* v, void* o, int B,
+                                  int H, int S, int hd, int kv_stride, cudaStream_t st);
+int attention_prepare();  // sets kernel attributes; call before any stream capture
+
+// decode.cu
+uint64_t attention_decode_work_bytes(int B, int H, int max_len, int hd);
+int launch_attention_decode(int dtype, const void* q, const void* k, const void* v, void* o, int B, int H,
+                            int len, const int* d_len_minus1, int hd, int kv_stride, float* work,
+                            cudaStream_t st);
+int launch_splitk_reduce(int mode, const float* partial, int splits, const EpiArgs& a, cudaStream_t st);
+
+// gemm_tc.cu  (bf16 tcgen05 GEMM)
+struct TcGemm {
+    // C-tile roles: rows of the 128-row operand "A" map to TMEM lanes.
+    const void* A;  // bf16 [rowsA, K]
+    const void* B;  // bf16 [rowsB, K]
+    int rowsA, rowsB, K;
+    int splits;     // split-K factor (EPI_PARTIAL only)
+    int swap;       // 0: A = tokens, B = weights; 1: A = weights, B = tokens (decode)
+};
+int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaStream_t st);
+int gemm_tc_pick_splits(int rowsA, int K);
+int gemm_tc_prepare();  // sets kernel attributes; call before any stream capture

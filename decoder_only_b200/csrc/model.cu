@@ -1,0 +1,629 @@
+// The model: arena layout, weight initialisation, prefill and decode launch
+// sequences, the C ABI of include/llama_b200.h.
+//
+// Per block ("The one formula"; "Pre-norm: the norm goes on the branch, not
+// the trunk"):
+//   xn    = RMSNorm(trunk) * g_attn                       rmsnorm kernel
+//   Q,K,V = xn [Wq Wk Wv]; RoPE(Q), RoPE(K); K,V -> cache  GEMM + QKV epilogue
+//   attn  = causal softmax(Q K^T / sqrt(hd)) V per head     attention kernel
+//   trunk += attn Wo                                        GEMM + residual epilogue
+//   xn    = RMSNorm(trunk) * g_ffn                          rmsnorm kernel
+//   act   = SiLU(xn Wg) * (xn Wu)                           GEMM + SwiGLU epilogue
+//   trunk += act Wd                                         GEMM + residual epilogue
+// then logits = RMSNorm(trunk) * g_final Whead.
+#include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "kernels.h"
+
+namespace {
+
+constexpr uint32_t TID_EMBED = 1, TID_HEAD = 2;
+inline uint32_t layer_tid(int l, int m) { return 16u + 8u * (uint32_t)l + (uint32_t)m; }
+constexpr int MAX_DEC_SPLITS = 16;
+
+struct Layer {
+    void *wqkv, *wo, *wgu, *wd;
+    float *g_attn, *g_ffn;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+// Error word of the standalone ops (the model has its own in its arena).
+__device__ int g_op_err_word;
+
+namespace {
+int op_error_word(int** p) {
+    static int* addr = nullptr;
+    if (!addr) LLAMA_CUDA_TRY(cudaGetSymbolAddress((void**)&addr, g_op_err_word));
+    *p = addr;
+    return LLAMA_OK;
+}
+}  // namespace
+
+struct llama_model {
+    llama_config cfg;
+    int esz;                 // bytes per stored element
+    uint8_t* arena;
+    uint64_t arena_bytes;
+    void* embed;
+    std::vector<Layer> layers;
+    float* g_final;
+    void* head;
+    float2* rope;
+    void* kv;
+    size_t kv_layer_elems;   // elements of one of K or V for one layer
+    float* trunk;
+    void *xn, *q, *attn, *act;
+    float* gemm_c;           // fp32 GEMM result for the fp32 path
+    float* logits_dec;       // [max_batch, vocab]
+    float* partial;          // split-K partials
+    size_t partial_elems;
+    float* attn_work;
+    uint64_t attn_work_bytes;
+    int32_t* tok_cur;        // decode input tokens; argmax writes the next ones here
+    int* d_pos;              // decode position
+    int* d_err;              // sticky device error word
+    int B;                   // batch of the last prefill (0: none)
+    int cur_len;             // host mirror of *d_pos
+    int splits_qkv, splits_o, splits_gu, splits_d, splits_head;
+    cudaStream_t cap_stream;
+    cudaGraphExec_t graph;
+    int graph_B;
+};
+
+namespace {
+
+int validate(const llama_config* c) {
+    if (!c) return LLAMA_ERR_INVALID_ARG;
+    if (c->n_layers < 0 || c->d_model <= 0 || c->n_heads <= 0 || c->vocab <= 0) return LLAMA_ERR_INVALID_ARG;
+    if (c->head_dim * c->n_heads != c->d_model) return LLAMA_ERR_INVALID_ARG;
+    if (c->dtype != LLAMA_F32 && c->dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+    if (c->max_batch <= 0 || c->max_seq <= 0) return LLAMA_ERR_INVALID_ARG;
+    if (!(c->norm_eps >= 0.f) || !(c->rope_theta > 0.f)) return LLAMA_ERR_INVALID_ARG;
+    if (c->d_model % 32 != 0 || c->d_model > 8192) return LLAMA_ERR_INVALID_ARG;
+    if (c->ffn_hidden < 0 || c->ffn_hidden % 128 != 0) return LLAMA_ERR_INVALID_ARG;
+    if (c->dtype == LLAMA_BF16) {
+        if (c->head_dim != 64 && c->head_dim != 128) return LLAMA_ERR_INVALID_ARG;
+        if (c->d_model % 256 != 0) return LLAMA_ERR_INVALID_ARG;
+        if (c->max_batch > 32) return LLAMA_ERR_INVALID_ARG;
+        if (c->vocab % 4 != 0) return LLAMA_ERR_INVALID_ARG;
+    } else {
+        if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return LLAMA_ERR_INVALID_ARG;
+    }
+    return LLAMA_OK;
+}
+
+int hidden_of(const llama_config* c) {
+    if (c->ffn_hidden > 0) return c->ffn_hidden;
+    const int two_thirds = (8 * c->d_model) / 3;
+    return 256 * ((two_thirds + 255) / 256);
+}
+
+// Walks the arena layout; with m != NULL assigns the pointers.
+uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
+    const int esz = c->dtype == LLAMA_BF16 ? 2 : 4;
+    const size_t d = c->d_model, h = hidden_of(c), V = c->vocab, L = c->n_layers;
+    const size_t nmax = (size_t)c->max_batch * c->max_seq;
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> void* {
+        void* p = base ? base + off : nullptr;
+        off += align256(bytes);
+        return p;
+    };
+    void* embed = take(V * d * esz);
+    if (m) {
+        m->embed = embed;
+        m->layers.resize(L);
+    }
+    for (size_t l = 0; l < L; ++l) {
+        Layer ly;
+        ly.wqkv = take(3 * d * d * esz);
+        ly.wo = take(d * d * esz);
+        ly.wgu = take(2 * h * d * esz);
+        ly.wd = take(d * h * esz);
+        ly.g_attn = (float*)take(d * 4);
+        ly.g_ffn = (float*)take(d * 4);
+        if (m) m->layers[l] = ly;
+    }
+    float* g_final = (float*)take(d * 4);
+    void* head = take(V * d * esz);
+    float2* rope = (float2*)take((size_t)c->max_seq * (c->head_dim / 2) * sizeof(float2));
+    const size_t kv_layer = (size_t)c->max_batch * c->n_heads * c->max_seq * c->head_dim;
+    void* kv = take(2 * L * kv_layer * esz);
+    float* trunk = (float*)take(nmax * d * 4);
+    void* xn = take(nmax * d * esz);
+    void* q = take(nmax * d * esz);
+    void* attn = take(nmax * d * esz);
+    void* act = take(nmax * h * esz);
+    const size_t cmax = std::max(3 * d, 2 * h);
+    float* gemm_c = (float*)take(c->dtype == LLAMA_F32 ? nmax * std::max(cmax, V) * 4 : 0);
+    float* logits_dec = (float*)take((size_t)c->max_batch * V * 4);
+    const size_t pmax = (size_t)MAX_DEC_SPLITS * c->max_batch * std::max(cmax, V);
+    float* partial = (float*)take(c->dtype == LLAMA_BF16 ? pmax * 4 : 0);
+    const uint64_t awb = attention_decode_work_bytes(c->max_batch, c->n_heads, c->max_seq, c->head_dim);
+    float* attn_work = (float*)take(awb);
+    int32_t* tok_cur = (int32_t*)take((size_t)c->max_batch * 4);
+    int* small = (int*)take(256);
+    if (m) {
+        m->g_final = g_final;
+        m->head = head;
+        m->rope = rope;
+        m->kv = kv;
+        m->kv_layer_elems = kv_layer;
+        m->trunk = trunk;
+        m->xn = xn;
+        m->q = q;
+        m->attn = attn;
+        m->act = act;
+        m->gemm_c = gemm_c;
+        m->logits_dec = logits_dec;
+        m->partial = partial;
+        m->partial_elems = pmax;
+        m->attn_work = attn_work;
+        m->attn_work_bytes = awb;
+        m->tok_cur = tok_cur;
+        m->d_pos = small;
+        m->d_err = small + 1;
+    }
+    return off;
+}
+
+inline void* kcache(llama_model* m, int l) {
+    return (uint8_t*)m->kv + (size_t)(2 * l) * m->kv_layer_elems * m->esz;
+}
+inline void* vcache(llama_model* m, int l) {
+    return (uint8_t*)m->kv + (size_t)(2 * l + 1) * m->kv_layer_elems * m->esz;
+}
+
+__global__ void pos_set_kernel(int* pos, int v) { *pos = v; }
+__global__ void pos_advance_kernel(int* pos) { *pos += 1; }
+
+EpiArgs base_args(llama_model* m, int M, int N) {
+    EpiArgs a;
+    memset(&a, 0, sizeof(a));
+    a.M = M;
+    a.N = N;
+    a.H = m->cfg.n_heads;
+    a.hd = m->cfg.head_dim;
+    a.d = m->cfg.d_model;
+    a.smax = m->cfg.max_seq;
+    a.rope = m->rope;
+    a.hidden = hidden_of(&m->cfg);
+    return a;
+}
+
+// One projection: out-op(A [M, K] . W [N, K]^T).  mode in EPI_*.
+// Prefill (decode = false): tcgen05 GEMM with the fused epilogue (bf16) or
+// SIMT GEMM + epilogue pass (fp32).  Decode: split-K swap-AB tcgen05 GEMM
+// into partials + reduction with the epilogue (bf16); SIMT for fp32.
+int project(llama_model* m, int mode, const void* A, const void* W, int M, int N, int K, int splits,
+            const EpiArgs& a, bool decode, cudaStream_t st) {
+    const int dt = m->cfg.dtype;
+    if (dt == LLAMA_BF16) {
+        TcGemm g;
+        if (!decode) {
+            g.A = A;
+            g.B = W;
+            g.rowsA = M;
+            g.rowsB = N;
+            g.K = K;
+            g.splits = 1;
+            g.swap = 0;
+            return launch_gemm_tc(g, mode, a, m->d_err, st);
+        }
+        g.A = W;
+        g.B = A;
+        g.rowsA = N;
+        g.rowsB = M;
+        g.K = K;
+        g.splits = splits;
+        g.swap = 1;
+        EpiArgs pa = a;
+        pa.out = m->partial;
+        int rc = launch_gemm_tc(g, EPI_PARTIAL, pa, m->d_err, st);
+        if (rc) return rc;
+        return launch_splitk_reduce(mode, m->partial, splits, a, st);
+    }
+    // fp32 storage: SIMT GEMM
+    if (mode == EPI_RESID) return launch_gemm_simt(dt, A, W, a.out, M, N, K, 1, st);
+    if (mode == EPI_F32) return launch_gemm_simt(dt, A, W, a.out, M, N, K, 0, st);
+    int rc = launch_gemm_simt(dt, A, W, m->gemm_c, M, N, K, 0, st);
+    if (rc) return rc;
+    return launch_epilogue_from_f32(dt, mode, m->gemm_c, N, a, st);
+}
+
+// The L blocks on the trunk [B*S, d] (prefill) or [B, d] (decode).
+int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
+    const llama_config& c = m->cfg;
+    const int d = c.d_model, h = hidden_of(&c);
+    const int n = decode ? B : B * S;
+    const int dt = c.dtype;
+    int rc;
+    for (int l = 0; l < c.n_layers; ++l) {
+        const Layer& ly = m->layers[l];
+        // attention sublayer
+        if ((rc = launch_rmsnorm(dt, m->trunk, ly.g_attn, m->xn, n, d, c.norm_eps, st))) return rc;
+        EpiArgs qa = base_args(m, n, 3 * d);
+        qa.q = m->q;
+        qa.kc = kcache(m, l);
+        qa.vc = vcache(m, l);
+        qa.S = decode ? 1 : S;
+        qa.d_pos = decode ? m->d_pos : nullptr;
+        if ((rc = project(m, EPI_QKV, m->xn, ly.wqkv, n, 3 * d, d, m->splits_qkv, qa, decode, st))) return rc;
+        if (decode) {
+            if ((rc = launch_attention_decode(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, 0,
+                                              m->d_pos, c.head_dim, c.max_seq, m->attn_work, st)))
+                return rc;
+        } else {
+            if ((rc = launch_attention_prefill_simt(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, S,
+                                                    c.head_dim, c.max_seq, st)))
+                return rc;
+        }
+        EpiArgs ra = base_args(m, n, d);
+        ra.out = m->trunk;
+        ra.ld_out = d;
+        if ((rc = project(m, EPI_RESID, m->attn, ly.wo, n, d, d, m->splits_o, ra, decode, st))) return rc;
+        // feed-forward sublayer
+        if ((rc = launch_rmsnorm(dt, m->trunk, ly.g_ffn, m->xn, n, d, c.norm_eps, st))) return rc;
+        EpiArgs sa = base_args(m, n, 2 * h);
+        sa.act = m->act;
+        if ((rc = project(m, EPI_SWIGLU, m->xn, ly.wgu, n, 2 * h, d, m->splits_gu, sa, decode, st))) return rc;
+        if ((rc = project(m, EPI_RESID, m->act, ly.wd, n, d, h, m->splits_d, ra, decode, st))) return rc;
+    }
+    return LLAMA_OK;
+}
+
+int run_head(llama_model* m, int n, float* logits, bool decode, cudaStream_t st) {
+    const llama_config& c = m->cfg;
+    int rc = launch_rmsnorm(c.dtype, m->trunk, m->g_final, m->xn, n, c.d_model, c.norm_eps, st);
+    if (rc) return rc;
+    EpiArgs a = base_args(m, n, c.vocab);
+    a.out = logits;
+    a.ld_out = c.vocab;
+    return project(m, EPI_F32, m->xn, m->head, n, c.vocab, c.d_model, m->splits_head, a, decode, st);
+}
+
+// Body of one decode step on the internal buffers: tok_cur -> tok_cur.
+int decode_body(llama_model* m, cudaStream_t st) {
+    const llama_config& c = m->cfg;
+    int rc = launch_embed(c.dtype, m->tok_cur, m->embed, m->trunk, m->B, c.d_model, c.vocab, m->d_err, st);
+    if (rc) return rc;
+    if ((rc = run_blocks(m, m->B, 1, true, st))) return rc;
+    if ((rc = run_head(m, m->B, m->logits_dec, true, st))) return rc;
+    if ((rc = launch_argmax(m->logits_dec, m->B, c.vocab, m->tok_cur, st))) return rc;
+    pos_advance_kernel<<<1, 1, 0, st>>>(m->d_pos);
+    LLAMA_LAUNCH_CHECK();
+    return LLAMA_OK;
+}
+
+int ensure_graph(llama_model* m) {
+    if (m->graph && m->graph_B == m->B) return LLAMA_OK;
+    if (m->graph) {
+        cudaGraphExecDestroy(m->graph);
+        m->graph = nullptr;
+    }
+    cudaGraph_t g = nullptr;
+    LLAMA_CUDA_TRY(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
+    int rc = decode_body(m, m->cap_stream);
+    cudaError_t e = cudaStreamEndCapture(m->cap_stream, &g);
+    if (rc) {
+        if (g) cudaGraphDestroy(g);
+        return rc;
+    }
+    if (e != cudaSuccess) return LLAMA_ERR_CUDA;
+    e = cudaGraphInstantiate(&m->graph, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) {
+        m->graph = nullptr;
+        return LLAMA_ERR_CUDA;
+    }
+    m->graph_B = m->B;
+    return LLAMA_OK;
+}
+
+void pick_decode_splits(llama_model* m) {
+    const llama_config& c = m->cfg;
+    const int d = c.d_model, h = hidden_of(&c);
+    if (c.dtype != LLAMA_BF16) {
+        m->splits_qkv = m->splits_o = m->splits_gu = m->splits_d = m->splits_head = 1;
+        return;
+    }
+    m->splits_qkv = gemm_tc_pick_splits(3 * d, d);
+    m->splits_o = gemm_tc_pick_splits(d, d);
+    m->splits_gu = gemm_tc_pick_splits(2 * h, d);
+    m->splits_d = gemm_tc_pick_splits(d, h);
+    m->splits_head = gemm_tc_pick_splits(c.vocab, d);
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+const char* llama_status_str(int s) {
+    switch (s) {
+        case LLAMA_OK: return "ok";
+        case LLAMA_ERR_INVALID_ARG: return "invalid argument";
+        case LLAMA_ERR_OOM: return "arena or workspace too small";
+        case LLAMA_ERR_CUDA: return "CUDA error";
+        case LLAMA_ERR_TIMEOUT: return "bounded device wait expired";
+        case LLAMA_ERR_STATE: return "call out of order";
+        default: return "unknown status";
+    }
+}
+
+int llama_model_bytes(const llama_config* cfg, uint64_t* bytes_out) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if (!bytes_out) return LLAMA_ERR_INVALID_ARG;
+    *bytes_out = layout(cfg, nullptr, nullptr);
+    return LLAMA_OK;
+}
+
+int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, uint64_t arena_bytes, void* stream,
+                       llama_model** out) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if (!out || !d_arena || (reinterpret_cast<uintptr_t>(d_arena) & 255u)) return LLAMA_ERR_INVALID_ARG;
+    const uint64_t need = layout(cfg, nullptr, nullptr);
+    if (arena_bytes < need) return LLAMA_ERR_OOM;
+    cudaStream_t st = (cudaStream_t)stream;
+    llama_model* m = new llama_model();
+    m->cfg = *cfg;
+    m->cfg.ffn_hidden = hidden_of(cfg);
+    m->esz = cfg->dtype == LLAMA_BF16 ? 2 : 4;
+    m->arena = (uint8_t*)d_arena;
+    m->arena_bytes = arena_bytes;
+    layout(&m->cfg, m, m->arena);
+    m->B = 0;
+    m->cur_len = 0;
+    m->graph = nullptr;
+    m->graph_B = 0;
+    if (cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
+        delete m;
+        return LLAMA_ERR_CUDA;
+    }
+    const int dt = cfg->dtype;
+    const int d = cfg->d_model, h = m->cfg.ffn_hidden, V = cfg->vocab;
+    const double sc = 0.02;
+#define TRY(x)                  \
+    do {                        \
+        if ((rc = (x))) {       \
+            llama_free(m);      \
+            return rc;          \
+        }                       \
+    } while (0)
+    TRY(launch_init_matrix(dt, m->embed, d, V, V, 0, 0, 1, seed, TID_EMBED, sc, st));
+    TRY(launch_init_matrix(dt, m->head, d, V, V, 0, 0, 0, seed, TID_HEAD, sc, st));
+    TRY(launch_fill_f32(m->g_final, 1.0f, d, st));
+    for (int l = 0; l < cfg->n_layers; ++l) {
+        const Layer& ly = m->layers[l];
+        TRY(launch_init_matrix(dt, ly.wqkv, d, d, d, 0, 0, 0, seed, layer_tid(l, 0), sc, st));
+        TRY(launch_init_matrix(dt, ly.wqkv, d, d, d, 0, d, 0, seed, layer_tid(l, 1), sc, st));
+        TRY(launch_init_matrix(dt, ly.wqkv, d, d, d, 0, 2 * d, 0, seed, layer_tid(l, 2), sc, st));
+        TRY(launch_init_matrix(dt, ly.wo, d, d, d, 0, 0, 0, seed, layer_tid(l, 3), sc, st));
+        TRY(launch_init_matrix(dt, ly.wgu, d, h, 128, 256, 0, 0, seed, layer_tid(l, 4), sc, st));
+        TRY(launch_init_matrix(dt, ly.wgu, d, h, 128, 256, 128, 0, seed, layer_tid(l, 5), sc, st));
+        TRY(launch_init_matrix(dt, ly.wd, h, d, d, 0, 0, 0, seed, layer_tid(l, 6), sc, st));
+        TRY(launch_fill_f32(ly.g_attn, 1.0f, d, st));
+        TRY(launch_fill_f32(ly.g_ffn, 1.0f, d, st));
+    }
+    // RoPE table: angle = pos * theta^(-2i/hd), cos and sin in fp64, stored fp32
+    const int hp = cfg->head_dim / 2;
+    std::vector<float2> tab((size_t)cfg->max_seq * hp);
+    for (int p = 0; p < cfg->max_seq; ++p)
+        for (int i = 0; i < hp; ++i) {
+            const double ang = (double)p * pow((double)cfg->rope_theta, -(2.0 * i) / (double)cfg->head_dim);
+            tab[(size_t)p * hp + i] = make_float2((float)cos(ang), (float)sin(ang));
+        }
+    if (cudaMemcpyAsync(m->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice, st) !=
+        cudaSuccess) {
+        llama_free(m);
+        return LLAMA_ERR_CUDA;
+    }
+    if (cudaMemsetAsync(m->d_pos, 0, 256, st) != cudaSuccess) {
+        llama_free(m);
+        return LLAMA_ERR_CUDA;
+    }
+    pick_decode_splits(m);
+    if ((rc = gemm_tc_prepare()) || (rc = attention_prepare())) {
+        llama_free(m);
+        return rc;
+    }
+    if (cudaStreamSynchronize(st) != cudaSuccess) {
+        llama_free(m);
+        return LLAMA_ERR_CUDA;
+    }
+#undef TRY
+    *out = m;
+    return LLAMA_OK;
+}
+
+int llama_prefill(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S, float* d_logits, void* stream) {
+    if (!m || !d_tokens || B <= 0 || S <= 0 || B > m->cfg.max_batch || S > m->cfg.max_seq)
+        return LLAMA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int n = B * S;
+    int rc = launch_embed(m->cfg.dtype, d_tokens, m->embed, m->trunk, n, m->cfg.d_model, m->cfg.vocab, m->d_err, st);
+    if (rc) return rc;
+    if ((rc = run_blocks(m, B, S, false, st))) return rc;
+    if (d_logits && (rc = run_head(m, n, d_logits, false, st))) return rc;
+    pos_set_kernel<<<1, 1, 0, st>>>(m->d_pos, S);
+    LLAMA_LAUNCH_CHECK();
+    m->B = B;
+    m->cur_len = S;
+    return LLAMA_OK;
+}
+
+int llama_prefill_trunk(llama_model* m, const float* d_x, int32_t B, int32_t S, float* d_y, void* stream) {
+    if (!m || !d_x || !d_y || B <= 0 || S <= 0 || B > m->cfg.max_batch || S > m->cfg.max_seq)
+        return LLAMA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t bytes = (size_t)B * S * m->cfg.d_model * 4;
+    if (d_x != m->trunk) LLAMA_CUDA_TRY(cudaMemcpyAsync(m->trunk, d_x, bytes, cudaMemcpyDeviceToDevice, st));
+    int rc = run_blocks(m, B, S, false, st);
+    if (rc) return rc;
+    if (d_y != m->trunk) LLAMA_CUDA_TRY(cudaMemcpyAsync(d_y, m->trunk, bytes, cudaMemcpyDeviceToDevice, st));
+    pos_set_kernel<<<1, 1, 0, st>>>(m->d_pos, S);
+    LLAMA_LAUNCH_CHECK();
+    m->B = B;
+    m->cur_len = S;
+    return LLAMA_OK;
+}
+
+int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t* d_next, float* d_logits, void* stream) {
+    if (!m || !d_tokens) return LLAMA_ERR_INVALID_ARG;
+    if (m->B <= 0 || m->cur_len >= m->cfg.max_seq) return LLAMA_ERR_STATE;
+    cudaStream_t st = (cudaStream_t)stream;
+    int rc = ensure_graph(m);
+    if (rc) return rc;
+    LLAMA_CUDA_TRY(cudaMemcpyAsync(m->tok_cur, d_tokens, (size_t)m->B * 4, cudaMemcpyDeviceToDevice, st));
+    LLAMA_CUDA_TRY(cudaGraphLaunch(m->graph, st));
+    if (d_next) LLAMA_CUDA_TRY(cudaMemcpyAsync(d_next, m->tok_cur, (size_t)m->B * 4, cudaMemcpyDeviceToDevice, st));
+    if (d_logits)
+        LLAMA_CUDA_TRY(cudaMemcpyAsync(d_logits, m->logits_dec, (size_t)m->B * m->cfg.vocab * 4,
+                                       cudaMemcpyDeviceToDevice, st));
+    m->cur_len += 1;
+    return LLAMA_OK;
+}
+
+int llama_generate(llama_model* m, const int32_t* d_first, int32_t n_steps, int32_t* d_out, void* stream) {
+    if (!m || !d_first || !d_out || n_steps < 0) return LLAMA_ERR_INVALID_ARG;
+    if (m->B <= 0 || m->cur_len + n_steps > m->cfg.max_seq) return LLAMA_ERR_STATE;
+    cudaStream_t st = (cudaStream_t)stream;
+    int rc = ensure_graph(m);
+    if (rc) return rc;
+    LLAMA_CUDA_TRY(cudaMemcpyAsync(m->tok_cur, d_first, (size_t)m->B * 4, cudaMemcpyDeviceToDevice, st));
+    for (int i = 0; i < n_steps; ++i) {
+        LLAMA_CUDA_TRY(cudaGraphLaunch(m->graph, st));
+        LLAMA_CUDA_TRY(cudaMemcpyAsync(d_out + (size_t)i * m->B, m->tok_cur, (size_t)m->B * 4,
+                                       cudaMemcpyDeviceToDevice, st));
+        m->cur_len += 1;
+    }
+    return LLAMA_OK;
+}
+
+int llama_position(const llama_model* m) { return m ? m->cur_len : LLAMA_ERR_INVALID_ARG; }
+
+int llama_model_tensor(const llama_model* m, const char* name, int32_t layer, void** d_ptr, uint64_t* bytes) {
+    if (!m || !name || !d_ptr || !bytes) return LLAMA_ERR_INVALID_ARG;
+    const llama_config& c = m->cfg;
+    const size_t d = c.d_model, h = c.ffn_hidden, V = c.vocab, es = m->esz;
+    const size_t nmax = (size_t)c.max_batch * c.max_seq;
+    auto lay = [&](int l) -> const Layer* { return (l >= 0 && l < c.n_layers) ? &m->layers[l] : nullptr; };
+    if (!strcmp(name, "kv")) { *d_ptr = m->kv; *bytes = 2 * (size_t)c.n_layers * m->kv_layer_elems * es; }
+    else if (!strcmp(name, "trunk")) { *d_ptr = m->trunk; *bytes = nmax * d * 4; }
+    else if (!strcmp(name, "q")) { *d_ptr = m->q; *bytes = nmax * d * es; }
+    else if (!strcmp(name, "attn")) { *d_ptr = m->attn; *bytes = nmax * d * es; }
+    else if (!strcmp(name, "xn")) { *d_ptr = m->xn; *bytes = nmax * d * es; }
+    else if (!strcmp(name, "act")) { *d_ptr = m->act; *bytes = nmax * h * es; }
+    else if (!strcmp(name, "embed")) { *d_ptr = m->embed; *bytes = V * d * es; }
+    else if (!strcmp(name, "head")) { *d_ptr = m->head; *bytes = V * d * es; }
+    else if (!strcmp(name, "logits_dec")) { *d_ptr = m->logits_dec; *bytes = (size_t)c.max_batch * V * 4; }
+    else {
+        const Layer* ly = lay(layer);
+        if (!ly) return LLAMA_ERR_INVALID_ARG;
+        if (!strcmp(name, "wqkv")) { *d_ptr = ly->wqkv; *bytes = 3 * d * d * es; }
+        else if (!strcmp(name, "wo")) { *d_ptr = ly->wo; *bytes = d * d * es; }
+        else if (!strcmp(name, "wgu")) { *d_ptr = ly->wgu; *bytes = 2 * h * d * es; }
+        else if (!strcmp(name, "wd")) { *d_ptr = ly->wd; *bytes = d * h * es; }
+        else return LLAMA_ERR_INVALID_ARG;
+    }
+    return LLAMA_OK;
+}
+
+int llama_last_error(llama_model* m) {
+    if (!m) return LLAMA_ERR_INVALID_ARG;
+    int e = 0;
+    LLAMA_CUDA_TRY(cudaMemcpy(&e, m->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+    LLAMA_CUDA_TRY(cudaMemset(m->d_err, 0, sizeof(int)));
+    if (e & LLAMA_DEVERR_TIMEOUT) return LLAMA_ERR_TIMEOUT;
+    if (e) return LLAMA_ERR_INVALID_ARG;
+    return LLAMA_OK;
+}
+
+void llama_free(llama_model* m) {
+    if (!m) return;
+    if (m->graph) cudaGraphExecDestroy(m->graph);
+    if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
+    delete m;
+}
+
+// ------------------------------------------------------------ single ops
+
+int llama_op_rmsnorm(int32_t dtype, const float* d_x, const float* d_g, void* d_y, int32_t rows, int32_t d,
+                     float eps, void* stream) {
+    if (!d_x || !d_g || !d_y || rows < 0 || d <= 0 || d % 4 != 0 || d > 8192) return LLAMA_ERR_INVALID_ARG;
+    if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+    return launch_rmsnorm(dtype, d_x, d_g, d_y, rows, d, eps, (cudaStream_t)stream);
+}
+
+int llama_op_gemm(int32_t dtype, const void* d_A, const void* d_W, float* d_C, int32_t M, int32_t N, int32_t K,
+                  int32_t accumulate, void* stream) {
+    if (!d_A || !d_W || !d_C || M <= 0 || N <= 0 || K <= 0) return LLAMA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == LLAMA_F32) return launch_gemm_simt(dtype, d_A, d_W, d_C, M, N, K, accumulate ? 1 : 0, st);
+    if (dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+    if (K % 64 != 0 || N % 16 != 0 || (reinterpret_cast<uintptr_t>(d_C) & 15u)) return LLAMA_ERR_INVALID_ARG;
+    if (accumulate && N % 32 != 0) return LLAMA_ERR_INVALID_ARG;
+    TcGemm g;
+    g.A = d_A;
+    g.B = d_W;
+    g.rowsA = M;
+    g.rowsB = N;
+    g.K = K;
+    g.splits = 1;
+    g.swap = 0;
+    EpiArgs a;
+    memset(&a, 0, sizeof(a));
+    a.M = M;
+    a.N = N;
+    a.out = d_C;
+    a.ld_out = N;
+    int* err = nullptr;
+    int rc = op_error_word(&err);
+    if (rc) return rc;
+    return launch_gemm_tc(g, accumulate ? EPI_RESID : EPI_F32, a, err, st);
+}
+
+int llama_op_attention_prefill(int32_t dtype, const void* d_q, const void* d_k, const void* d_v, void* d_o,
+                               int32_t B, int32_t H, int32_t S, int32_t head_dim, int32_t kv_stride, void* stream) {
+    if (!d_q || !d_k || !d_v || !d_o || B <= 0 || H <= 0 || S <= 0 || kv_stride < S) return LLAMA_ERR_INVALID_ARG;
+    if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+    return launch_attention_prefill_simt(dtype, d_q, d_k, d_v, d_o, B, H, S, head_dim, kv_stride,
+                                         (cudaStream_t)stream);
+}
+
+uint64_t llama_op_attention_decode_work_bytes(int32_t B, int32_t H, int32_t max_len, int32_t head_dim) {
+    if (B <= 0 || H <= 0 || max_len <= 0 || head_dim <= 0) return 0;
+    return attention_decode_work_bytes(B, H, max_len, head_dim);
+}
+
+int llama_op_attention_decode(int32_t dtype, const void* d_q, const void* d_k, const void* d_v, void* d_o, int32_t B,
+                              int32_t H, int32_t len, int32_t head_dim, int32_t kv_stride, void* d_work,
+                              uint64_t work_bytes, void* stream) {
+    if (!d_q || !d_k || !d_v || !d_o || !d_work || B <= 0 || H <= 0 || len <= 0 || kv_stride < len)
+        return LLAMA_ERR_INVALID_ARG;
+    if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+    if (work_bytes < attention_decode_work_bytes(B, H, len, head_dim)) return LLAMA_ERR_OOM;
+    return launch_attention_decode(dtype, d_q, d_k, d_v, d_o, B, H, len, nullptr, head_dim, kv_stride,
+                                   (float*)d_work, (cudaStream_t)stream);
+}
+
+int llama_op_argmax(const float* d_logits, int32_t rows, int32_t n, int32_t* d_out, void* stream) {
+    if (!d_logits || !d_out || rows < 0 || n <= 0) return LLAMA_ERR_INVALID_ARG;
+    return launch_argmax(d_logits, rows, n, d_out, (cudaStream_t)stream);
+}
+
+}  // extern "C"

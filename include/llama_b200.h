@@ -1,0 +1,196 @@
+/*
+ * llama_b200.h -- C ABI of the B200 (sm_100a) forward pass of the LLaMA
+ * pre-norm decoder stack.
+ *
+ * What is computed (the pages, cited by title and section):
+ *   [PFD] "LLaMA: Open and Efficient Foundation Language Models"
+ *         (paperfordummies.in), section "The one formula":
+ *             h = x + Attn(RMSNorm(x))
+ *             y = h + Wdown(SiLU(Wgate RMSNorm(h)) (.) Wup RMSNorm(h))
+ *         stacked L times, then one final RMSNorm and an untied output head
+ *         producing (n, vocab) logits; no bias anywhere; no position signal
+ *         at the bottom.
+ *   [PFD] "RMSNorm: LayerNorm minus the mean"; [NAR] "LLaMA: No
+ *         Architecture Revolution, Yet It Became the Open-Model
+ *         Foundation", section "An Architecture Recipe Without an Invention
+ *         Myth": RMSNorm(x) = x / sqrt(mean(x^2) + eps) (.) g.
+ *   [PFD] "RoPE: rotate Q and K, leave V alone": Q and K rotated per head,
+ *         pair (2i, 2i+1) by angle pos * theta^(-2i/head_dim); V untouched.
+ *   [PFD] "SwiGLU: a gate in the FFN, paid for with a narrower hidden
+ *         layer": hidden = 2/3 * 4d rounded up to a multiple of 256.
+ *   [NAR] "GQA Was Not an Original LLaMA Feature": the KV cache read by
+ *         autoregressive decoding.
+ *
+ * Conventions for every entry point below
+ *   - Pointers named d_* are DEVICE pointers; h_* are HOST pointers.  The
+ *     caller owns every buffer it passes and keeps it alive until the work
+ *     queued on `stream` has finished.  The library never calls cudaMalloc:
+ *     the model lives in one caller-allocated device arena.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it unless stated otherwise; outputs are valid once the
+ *     stream has been synchronised.
+ *   - Return value: LLAMA_OK (0) or a negative llama_status.  Arguments are
+ *     validated on the host before anything is queued; an invalid call
+ *     queues nothing.  A failed CUDA launch returns LLAMA_ERR_CUDA.
+ *   - Row-major layouts.  Weights are stored "K-major": a matrix the pages
+ *     apply as x @ W with W of shape (d_in, d_out) is stored as (d_out, d_in).
+ *   - Not thread-safe per model handle: one host thread drives one model.
+ */
+#ifndef LLAMA_B200_H
+#define LLAMA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LLAMA_API __attribute__((visibility("default")))
+#else
+#define LLAMA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum llama_status {
+    LLAMA_OK = 0,
+    LLAMA_ERR_INVALID_ARG = -1, /* shape or argument outside what is supported */
+    LLAMA_ERR_OOM = -2,         /* arena / workspace smaller than required */
+    LLAMA_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
+    LLAMA_ERR_TIMEOUT = -4,     /* a bounded device-side wait expired */
+    LLAMA_ERR_STATE = -5        /* call out of order (decode before prefill, cache full) */
+} llama_status;
+
+typedef enum llama_dtype {
+    LLAMA_F32 = 0,  /* weights and activations fp32, SIMT fp32 GEMMs */
+    LLAMA_BF16 = 1  /* weights and GEMM operands bf16, fp32 accumulate and trunk */
+} llama_dtype;
+
+typedef struct llama_config {
+    int32_t n_layers;
+    int32_t d_model;
+    int32_t n_heads;
+    int32_t head_dim;    /* d_model == n_heads * head_dim; head_dim in {32, 64, 128} */
+    int32_t ffn_hidden;  /* 0 => 256 * ceil(floor(8 d / 3) / 256) */
+    int32_t vocab;
+    float norm_eps;      /* RMSNorm eps (1e-6 in every workload) */
+    float rope_theta;    /* RoPE base (10000) */
+    int32_t dtype;       /* llama_dtype */
+    int32_t max_batch;   /* largest B passed to prefill / decode */
+    int32_t max_seq;     /* prompt length + decode steps, per sequence */
+} llama_config;
+
+typedef struct llama_model llama_model; /* opaque host handle */
+
+/* ------------------------------------------------------------------ model */
+
+/* Device bytes the model arena must hold for `cfg`: weights, RoPE table,
+ * KV cache [L][2][max_batch][H][max_seq][head_dim], activations and
+ * workspace.  Host-only; queues nothing. */
+LLAMA_API int llama_model_bytes(const llama_config* cfg, uint64_t* bytes_out);
+
+/* Carve the model out of `d_arena` (>= llama_model_bytes, 256-byte aligned)
+ * and fill the weights on the device from the counter-based generator
+ * (Philox4x32-10 keyed by (seed, tensor id), Box-Muller, N(0, 0.02^2),
+ * rounded to nearest-even into the storage type; RMSNorm gains 1).  Builds
+ * the RoPE cos/sin table on the host in fp64 and copies it.  Synchronises
+ * `stream` before returning.  *out receives a host handle freed by
+ * llama_free; the arena stays owned by the caller. */
+LLAMA_API int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena,
+                       uint64_t arena_bytes, void* stream, llama_model** out);
+
+/* Causal prefill of B sequences of S tokens each (B <= max_batch,
+ * 1 <= S <= max_seq).  d_tokens: int32 [B*S], row b*S + s.  Resets the KV
+ * cache and sets the decode position to S.  d_logits: fp32 [B*S, vocab]
+ * logits of every position, or NULL to skip the final norm and head. */
+LLAMA_API int llama_prefill(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S,
+                  float* d_logits, void* stream);
+
+/* The blocks alone, on a given fp32 trunk: d_x [B*S, d_model] in,
+ * d_y [B*S, d_model] out (the trunk after the last block, before the final
+ * norm).  Positions 0..S-1 per sequence.  d_x and d_y may alias. */
+LLAMA_API int llama_prefill_trunk(llama_model* m, const float* d_x, int32_t B, int32_t S,
+                        float* d_y, void* stream);
+
+/* One greedy decoding step for the B sequences of the last prefill: token
+ * d_tokens[b] (int32 [B]) sits at the current position p; its K and V are
+ * appended at p; attention spans 0..p.  d_next (int32 [B], may be NULL):
+ * argmax of the logits, lowest id on ties.  d_logits: fp32 [B, vocab] or
+ * NULL.  Advances p by one.  LLAMA_ERR_STATE before a prefill or when
+ * p == max_seq. */
+LLAMA_API int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t* d_next,
+                      float* d_logits, void* stream);
+
+/* n_steps greedy steps fed back on the device: step 0 consumes
+ * d_first [B]; step i consumes the token step i-1 chose.  d_out:
+ * int32 [n_steps, B].  Replays one captured CUDA graph per step. */
+LLAMA_API int llama_generate(llama_model* m, const int32_t* d_first, int32_t n_steps,
+                   int32_t* d_out, void* stream);
+
+/* Current decode position (tokens held per sequence in the KV cache). */
+LLAMA_API int llama_position(const llama_model* m);
+
+/* Device pointer and byte size of an internal buffer, for inspection:
+ * name in {"kv" (the whole cache), "trunk", "q", "attn", "act", "xn",
+ * "embed", "head", "wqkv", "wo", "wgu", "wd"}; `layer` selects the layer for
+ * per-layer weights.  Layouts are those of the arena described above. */
+LLAMA_API int llama_model_tensor(const llama_model* m, const char* name, int32_t layer,
+                       void** d_ptr, uint64_t* bytes);
+
+/* Reads (synchronously) and clears the sticky device error word that
+ * bounded device waits set; returns LLAMA_OK or LLAMA_ERR_TIMEOUT. */
+LLAMA_API int llama_last_error(llama_model* m);
+
+/* Releases the host handle (and its captured graphs).  The arena is the
+ * caller's to free afterwards. */
+LLAMA_API void llama_free(llama_model* m);
+
+LLAMA_API const char* llama_status_str(int status);
+
+/* ------------------------------------------------------------ single ops
+ * The kernels the model runs, exposed one by one on caller buffers.  dtype
+ * selects fp32 or bf16 storage of the T-typed operands. */
+
+/* y[r, :] = x[r, :] / sqrt(mean(x[r, :]^2) + eps) * g, r < rows.
+ * x fp32 [rows, d]; g fp32 [d]; y dtype-typed [rows, d]; d % 4 == 0,
+ * d <= 8192.  [PFD] "RMSNorm: LayerNorm minus the mean". */
+LLAMA_API int llama_op_rmsnorm(int32_t dtype, const float* d_x, const float* d_g, void* d_y,
+                     int32_t rows, int32_t d, float eps, void* stream);
+
+/* C = A W^T, or C += A W^T when accumulate != 0.  A dtype-typed [M, K],
+ * W dtype-typed [N, K] (K-major), C fp32 [M, N].  bf16: tcgen05 tensor-core
+ * GEMM, K % 64 == 0, N % 16 == 0, pointers 16-byte aligned; fp32: SIMT. */
+LLAMA_API int llama_op_gemm(int32_t dtype, const void* d_A, const void* d_W, float* d_C,
+                  int32_t M, int32_t N, int32_t K, int32_t accumulate, void* stream);
+
+/* Causal attention, heads independent.  q, k, v dtype-typed with layout
+ * [B][H][*][head_dim]; q has S rows per head, k/v have kv_stride rows per
+ * head (>= S; the first S are used).  o dtype-typed [B*S, H*head_dim]:
+ * row b*S + t, columns of head h at [h*head_dim, (h+1)*head_dim).
+ * Scale 1/sqrt(head_dim); key j is visible to query t iff j <= t. */
+LLAMA_API int llama_op_attention_prefill(int32_t dtype, const void* d_q, const void* d_k,
+                               const void* d_v, void* d_o, int32_t B, int32_t H,
+                               int32_t S, int32_t head_dim, int32_t kv_stride,
+                               void* stream);
+
+/* Decode attention: one query per (b, h) against keys/values 0..len-1.
+ * q dtype-typed [B, H*head_dim]; k, v [B][H][kv_stride][head_dim];
+ * o dtype-typed [B, H*head_dim].  Split over the sequence into chunks whose
+ * partial results go to d_work (fp32, llama_op_attention_decode_work_bytes
+ * bytes), then combined. */
+LLAMA_API int llama_op_attention_decode(int32_t dtype, const void* d_q, const void* d_k,
+                              const void* d_v, void* d_o, int32_t B, int32_t H,
+                              int32_t len, int32_t head_dim, int32_t kv_stride,
+                              void* d_work, uint64_t work_bytes, void* stream);
+LLAMA_API uint64_t llama_op_attention_decode_work_bytes(int32_t B, int32_t H, int32_t max_len,
+                                              int32_t head_dim);
+
+/* out[r] = argmax_j logits[r, j] (lowest j on ties), r < rows. */
+LLAMA_API int llama_op_argmax(const float* d_logits, int32_t rows, int32_t n, int32_t* d_out,
+                    void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLAMA_B200_H */
