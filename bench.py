@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Throughput of the LLaMA pre-norm decoder forward pass on B200.
+
+Default workload (one GPU): the LLaMA-7B-shaped model -- 32 layers, d 4096,
+32 heads x 128, FFN hidden 11008, vocab 32000, bf16 weights N(0, 0.02^2)
+drawn on the device from seed 0 -- running a causal prefill of 4 sequences x
+2048 uniform random token ids (logits for every position), then 128 greedy
+decode steps over the contiguous bf16 KV cache.  One step is that whole
+pass; `value` counts prompt plus generated tokens per second over all ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl b200|reference]
+
+Under torchrun every rank runs an independent replica (no collective on the
+data path: sequences are independent); the timed region is bracketed by a
+barrier and a device synchronise, and the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only) and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LLaMA-shape tokens/s (prefill, decode) on 1 B200; % of BF16/HBM roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {
+    "7b": dict(model="LLAMA_7B", batch=4, seq=2048, decode=128,
+               desc="llama-7b: prefill 4 x 2048 (logits at every position) + 128 greedy decode steps"),
+    "13b-decode": dict(model="LLAMA_13B", batch=32, seq=2048, decode=256,
+                       desc="llama-13b: 256 greedy decode steps, batch 32, 2048-token prompts prefilled untimed"),
+    "65b-slice": dict(model="LLAMA_65B_SLICE", batch=8, seq=2048, decode=0,
+                      desc="llama-65b widths, 16 layers: prefill 8 x 2048 (logits at every position)"),
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured (MEASURED_PEAKS.json)"
+    return dict(FALLBACK_PEAKS), "fallback (no MEASURED_PEAKS.json)"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        self.tmp.flush()
+        with open(self.tmp.name) as f:
+            rows = [r.split(",") for r in f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.tmp.name)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], [], set()
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 7:
+                continue
+            try:
+                sm.append(float(r[0]))
+                mx.append(float(r[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def algorithmic_work(shape, B, S, steps):
+    """FLOPs of one prefill (causal attention halved) and bytes of one decode
+    step (every weight once + the KV cache read + activations), average over
+    the decode steps."""
+    d, h, V, L = shape.d_model, shape.ffn_hidden, shape.vocab, shape.n_layers
+    n = B * S
+    gemm = 2.0 * n * (4 * d * d + 3 * d * h) * L + 2.0 * n * d * V
+    attn = 2.0 * B * S * (S + 1) * d * L
+    wbytes = 2.0 * (L * (4 * d * d + 3 * d * h) + d * V)
+    mean_len = S + (steps + 1) / 2.0
+    kv = 2.0 * 2 * L * B * mean_len * d
+    return gemm + attn, wbytes + kv
+
+
+def kernel_family(region: str) -> str:
+    if region.startswith("prefill_gemm"):
+        return "gemm_tc prefill (tcgen05, fused epilogues)"
+    if region.startswith("decode_gemm"):
+        return "gemm_tc decode (tcgen05 swap-AB split-K)"
+    return region
+
+
+def roofline(prof, decode_scale, peaks, peak_src):
+    """Dominant kernel over one step from the live per-region timing."""
+    fam = {}
+    for name, e in prof.items():
+        scale = decode_scale if name.startswith("decode") else 1.0
+        f = fam.setdefault(kernel_family(name), dict(ms=0.0, bytes=0.0, flops=0.0, launches=0, step_ms=0.0))
+        f["ms"] += e["ms"]
+        f["bytes"] += e["bytes"]
+        f["flops"] += e["flops"]
+        f["launches"] += e["launches"]
+        f["step_ms"] += e["ms"] * scale
+    total = sum(f["step_ms"] for f in fam.values())
+    name, f = max(fam.items(), key=lambda kv: kv[1]["step_ms"])
+    per_launch_ms = f["ms"] / max(f["launches"], 1)
+    if name.startswith("gemm_tc prefill") or name == "prefill_attention":
+        achieved = f["flops"] / (f["ms"] * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        out = dict(bound="tensor", unit="TFLOP/s", peak_kind="bf16 dense, sustained (kernel timed inside a long step)")
+    else:
+        achieved = f["bytes"] / (f["ms"] * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        out = dict(bound="hbm", unit="GB/s", peak_kind="HBM copy bandwidth")
+    out.update(kernel=name, achieved=round(achieved, 1), peak=peak, frac=round(achieved / peak, 4),
+               peak_source=peak_src, traffic=None, launches_profiled=f["launches"],
+               avg_launch_us=round(per_launch_ms * 1e3, 2), share_of_step=round(f["step_ms"] / total, 4),
+               shares={k: round(v["step_ms"] / total, 4) for k, v in sorted(fam.items(), key=lambda kv: -kv[1]["step_ms"])})
+    return out
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(shape, B, S, steps, prompt=64, layers=2):
+    """Times the fp64 oracle as it stands on a bounded sample of the workload
+    and scales it to one full step.  Weights are drawn before timing."""
+    import numpy as np
+    import oracle
+    import synth
+    from threadpoolctl import threadpool_info
+
+    sub = shape.with_(n_layers=layers)
+    W = [oracle.layer_weights(shape, l) for l in range(layers)]
+    tok = synth.tokens(0, prompt + 2, shape.vocab).reshape(1, prompt + 2)
+    t0 = time.perf_counter()
+    _, cache = oracle.prefill(sub, tok[:, :prompt], weights=lambda l: W[l], return_cache=True)
+    t1 = time.perf_counter()
+    oracle.decode_step(sub, cache, tok[:, prompt], weights=lambda l: W[l])
+    t2 = time.perf_counter()
+    # the oracle's head is included in both calls; scale the layers to L
+    scale = shape.n_layers / layers
+    t_pre_tok = (t1 - t0) * scale / prompt
+    t_dec_tok = (t2 - t1) * scale
+    step_s = B * S * t_pre_tok + B * steps * t_dec_tok
+    value = (B * S + B * steps) / step_s
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    sample = (f"oracle prefill of 1 x {prompt} tokens and one decode step through {layers} of "
+              f"{shape.n_layers} layers (+ head), per-token times scaled by {scale:g} in layer count "
+              f"to one step of {B}x{S} prefill + {B}x{steps} decode tokens")
+    return dict(value=round(value, 4), unit=UNIT, cores=threads, kind="oracle", sample=sample,
+                seconds=round(t2 - t0, 3)), step_s
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args, wl, shape):
+    import torch.distributed as dist  # noqa: F401
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    B, S, steps = wl["batch"], wl["seq"], wl["decode"]
+    vals = []
+    for i in range(args.warmup + args.steps):
+        cb, step_s = oracle_sample(shape, B, S, steps)
+        if i >= args.warmup:
+            vals.append((cb["value"], step_s))
+    value = statistics.median(v for v, _ in vals)
+    ms = statistics.median(s for _, s in vals) * 1e3
+    cb["value"] = round(value, 4)
+    line = dict(impl="reference", metric=METRIC, value=round(value, 4), unit=UNIT, n_gpus=args.gpus,
+                steps=args.steps, warmup=args.warmup, ms_per_step=round(ms, 1), higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                config=dict(workload=wl["desc"], batch=B, seq_len=S, decode_steps=steps),
+                cpu_baseline=cb, e2e=dict(value=round(value, 4), unit=UNIT, h2d_bytes_per_step=0,
+                                          d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+def run_b200(args, wl, shape):
+    import torch
+    import torch.distributed as dist
+
+    import decoder_only_b200 as lb
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    B, S, steps = wl["batch"], wl["seq"], wl["decode"]
+    max_seq = S + steps
+    model = lb.Model(shape, max_batch=B, max_seq=max_seq, seed=synth.workloads.SEED)
+    tok_host = torch.from_numpy(synth.tokens(synth.workloads.SEED + rank, B * S, shape.vocab).reshape(B, S))
+    tok_host = tok_host.pin_memory()
+    tok_dev = tok_host.cuda()
+    logits = torch.empty(B, S, shape.vocab, dtype=torch.float32, device="cuda") if wl["name"] != "13b-decode" else None
+    gen = torch.empty(max(steps, 1), B, dtype=torch.int32, device="cuda")
+    st = torch.cuda.current_stream()
+
+    decode_only = wl["name"] == "13b-decode"
+    if decode_only:
+        model.prefill(tok_dev, logits=False)               # untimed: the prompt cache
+        first = tok_dev[:, -1].contiguous()
+
+    def step():
+        if decode_only:
+            model.rewind(S)
+            model.generate(first, steps, out=gen)
+        else:
+            model.prefill(tok_dev, out=logits)
+            if steps:
+                model.generate(None, steps, out=gen, batch=B)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ------------------------------------------------ timed region (device events)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier()
+    torch.cuda.synchronize()
+    l0 = lb.kernel_launches()
+    with ClockSampler(local) as clk:
+        ev[0].record(st)
+        for _ in range(args.steps):
+            step()
+        ev[1].record(st)
+        torch.cuda.synchronize()
+    barrier()
+    launches = lb.kernel_launches() - l0
+    ms = ev[0].elapsed_time(ev[1])
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    clocks = clk.summary()
+    tokens_step = (0 if decode_only else B * S) + B * steps
+    value = world * tokens_step * args.steps / (ms * 1e-3)
+
+    # ------------------------------------------------ prefill / decode split
+    split = {}
+    if not decode_only:
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        pre, dec = [], []
+        for _ in range(2):
+            e[0].record(st)
+            model.prefill(tok_dev, out=logits)
+            e[1].record(st)
+            if steps:
+                model.generate(None, steps, out=gen, batch=B)
+            e[2].record(st)
+            torch.cuda.synchronize()
+            pre.append(e[0].elapsed_time(e[1]))
+            dec.append(e[1].elapsed_time(e[2]))
+        split["prefill_ms"] = min(pre)
+        split["decode_ms"] = min(dec) if steps else 0.0
+
+    # ------------------------------------------------ end to end from host buffers
+    out_host = torch.empty(max(steps, 1), B, dtype=torch.int32).pin_memory()
+    e2e_ms = None
+    if not decode_only:
+        model.complete(tok_host, steps, logits=logits, out_host=out_host)
+        torch.cuda.synchronize()
+        ee = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        barrier()
+        torch.cuda.synchronize()
+        ee[0].record(st)
+        for _ in range(args.steps):
+            model.complete(tok_host, steps, logits=logits, out_host=out_host)
+        ee[1].record(st)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = ee[0].elapsed_time(ee[1])
+        if world > 1:
+            t = torch.tensor([e2e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+
+    # ------------------------------------------------ live per-region timing (roofline)
+    peaks, peak_src = load_peaks()
+    prof_steps = min(steps, 16)
+    lb.profile_reset()
+    lb.profile_enable(True)
+    if decode_only:
+        model.rewind(S)
+        model.generate(first, prof_steps, out=gen)
+    else:
+        model.prefill(tok_dev, out=logits)
+        if steps:
+            model.generate(None, prof_steps, out=gen, batch=B)
+    torch.cuda.synchronize()
+    prof = lb.profile_read()
+    lb.profile_enable(False)
+    roof = roofline(prof, steps / max(prof_steps, 1), peaks, peak_src)
+
+    if rank == 0:
+        flops_pre, bytes_dec = algorithmic_work(shape, B, S, steps)
+        line = dict(
+            metric=METRIC, value=round(value, 2), unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
+            ms_per_step=round(ms / args.steps, 3), higher_is_better=True, scaling="weak", vs_baseline=None,
+            dtype="bf16", data="synthetic (seeded token ids; random-init weights N(0, 0.02^2) drawn on device)",
+            config=dict(workload=wl["desc"], model=shape.name, global_batch=B * world, seq_len=S,
+                        decode_steps=steps, parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                        l2="inputs larger than L2: every step streams all weights (13+ GB) from HBM"),
+            gpu_launches=launches, clocks=clocks, roofline=roof)
+        if split:
+            pre_s, dec_s = split["prefill_ms"] * 1e-3, split["decode_ms"] * 1e-3
+            line["prefill"] = dict(tokens_per_s=round(B * S / pre_s, 1), ms=round(split["prefill_ms"], 3),
+                                   tflops=round(flops_pre / pre_s / 1e12, 1),
+                                   frac_bf16=round(flops_pre / pre_s / 1e12 / peaks["bf16_tflops_sustained"], 4))
+            if steps:
+                line["decode"] = dict(tokens_per_s=round(B * steps / dec_s, 1),
+                                      ms_per_step=round(split["decode_ms"] / steps, 4),
+                                      gbs=round(bytes_dec * steps / dec_s / 1e9, 1),
+                                      frac_hbm=round(bytes_dec * steps / dec_s / 1e9 / peaks["hbm_gbs"], 4))
+        if e2e_ms is not None:
+            line["e2e"] = dict(value=round(world * tokens_step * args.steps / (e2e_ms * 1e-3), 2), unit=UNIT,
+                               h2d_bytes_per_step=B * S * 4, d2h_bytes_per_step=B * steps * 4)
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"], _ = oracle_sample(shape, B, S, steps)
+        print(json.dumps(line), flush=True)
+    model.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--workload", default="7b", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from synth import workloads as wls
+    wl = dict(WORKLOADS[args.workload], name=args.workload)
+    shape = getattr(wls, wl["model"])
+    if args.impl == "reference":
+        run_reference(args, wl, shape)
+    else:
+        run_b200(args, wl, shape)
+
+
+if __name__ == "__main__":
+    main()

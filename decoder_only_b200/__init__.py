@@ -58,12 +58,21 @@ def _load():
         "llama_op_attention_decode": [I, P, P, P, P, I, I, I, I, I, P, U64, P],
         "llama_op_attention_decode_work_bytes": [I, I, I, I],
         "llama_op_argmax": [P, I, I, P, P],
+        "llama_rewind": [P, I, P],
+        "llama_complete": [P, P, I, I, P, I, P, P],
+        "llama_kernel_launches": [],
+        "llama_profile_enable": [I],
+        "llama_profile_reset": [],
+        "llama_profile_count": [],
+        "llama_profile_entry": [I, P, P, P, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
         fn.argtypes = args
         fn.restype = ctypes.c_int
     lib.llama_free.restype = None
+    lib.llama_profile_reset.restype = None
+    lib.llama_kernel_launches.restype = ctypes.c_int64
     lib.llama_status_str.restype = ctypes.c_char_p
     lib.llama_op_attention_decode_work_bytes.restype = U64
     return lib
@@ -142,13 +151,29 @@ class Model:
     def position(self) -> int:
         return lib.llama_position(self.h)
 
-    def prefill(self, tokens: torch.Tensor, logits: bool = True):
+    def prefill(self, tokens: torch.Tensor, logits: bool = True, out: torch.Tensor | None = None):
         """tokens int32 [B, S] on the device -> logits fp32 [B, S, V] (or None)."""
         B, S = tokens.shape
         tokens = tokens.contiguous()
-        out = torch.empty(B, S, self.cfg.vocab, dtype=torch.float32, device="cuda") if logits else None
-        _check(lib.llama_prefill(self.h, _ptr(tokens), B, S, _ptr(out), _stream()), "llama_prefill")
-        return out
+        if logits and out is None:
+            out = torch.empty(B, S, self.cfg.vocab, dtype=torch.float32, device="cuda")
+        _check(lib.llama_prefill(self.h, _ptr(tokens), B, S, _ptr(out if logits else None), _stream()),
+               "llama_prefill")
+        return out if logits else None
+
+    def complete(self, tokens_host: torch.Tensor, n_steps: int, logits: torch.Tensor | None = None,
+                 out_host: torch.Tensor | None = None) -> torch.Tensor:
+        """Host int32 [B, S] prompt -> host int32 [n_steps, B] greedy tokens
+        (llama_complete; pass pinned tensors for asynchronous copies)."""
+        B, S = tokens_host.shape
+        if out_host is None:
+            out_host = torch.empty(n_steps, B, dtype=torch.int32, pin_memory=True)
+        _check(lib.llama_complete(self.h, _ptr(tokens_host.contiguous()), B, S, _ptr(logits), n_steps,
+                                  _ptr(out_host), _stream()), "llama_complete")
+        return out_host
+
+    def rewind(self, position: int):
+        _check(lib.llama_rewind(self.h, position, _stream()), "llama_rewind")
 
     def prefill_trunk(self, x: torch.Tensor, out: torch.Tensor | None = None):
         """x fp32 [B, S, d] -> trunk after the blocks, fp32 [B, S, d]."""
@@ -166,11 +191,14 @@ class Model:
                "llama_decode_step")
         return nxt, lg
 
-    def generate(self, first: torch.Tensor, n_steps: int, out: torch.Tensor | None = None):
-        B = first.shape[0]
+    def generate(self, first: torch.Tensor | None, n_steps: int, out: torch.Tensor | None = None,
+                 batch: int | None = None):
+        """n_steps greedy tokens [n_steps, B]; first=None continues from the
+        prefill's own greedy choice."""
+        B = first.shape[0] if first is not None else batch
         out = torch.empty(n_steps, B, dtype=torch.int32, device="cuda") if out is None else out
-        _check(lib.llama_generate(self.h, _ptr(first.contiguous()), n_steps, _ptr(out), _stream()),
-               "llama_generate")
+        f = None if first is None else first.contiguous()
+        _check(lib.llama_generate(self.h, _ptr(f), n_steps, _ptr(out), _stream()), "llama_generate")
         return out
 
     def tensor(self, name: str, layer: int = 0, dtype=None, shape=None) -> torch.Tensor:
@@ -188,6 +216,34 @@ class Model:
 
     def last_error(self) -> int:
         return lib.llama_last_error(self.h)
+
+
+# ----------------------------------------------------------------- instrumentation
+
+def kernel_launches() -> int:
+    return int(lib.llama_kernel_launches())
+
+
+def profile_enable(on: bool = True):
+    lib.llama_profile_enable(1 if on else 0)
+
+
+def profile_reset():
+    lib.llama_profile_reset()
+
+
+def profile_read() -> dict:
+    """{region: dict(ms, launches, calls, bytes, flops)} (synchronises)."""
+    out = {}
+    for i in range(lib.llama_profile_count()):
+        name = ctypes.c_char_p()
+        ms, by, fl = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+        la, ca = ctypes.c_int64(), ctypes.c_int64()
+        _check(lib.llama_profile_entry(i, ctypes.byref(name), ctypes.byref(ms), ctypes.byref(la), ctypes.byref(ca),
+                                       ctypes.byref(by), ctypes.byref(fl)), "llama_profile_entry")
+        out[name.value.decode()] = dict(ms=ms.value, launches=la.value, calls=ca.value, bytes=by.value,
+                                        flops=fl.value)
+    return out
 
 
 # ----------------------------------------------------------------- single ops

@@ -1,6 +1,8 @@
 """Builds libllama_b200.so in-tree with nvcc for sm_100a.
 
-    python -m decoder_only_b200.build [--debug]
+    python decoder_only_b200/build.py [--force] [--ptxas-v]
+
+(run as a file: importing the package needs the library it builds)
 
 Each .cu under csrc/ is compiled to an object under _build/ (rebuilt when it
 or a header is newer), then linked into decoder_only_b200/libllama_b200.so

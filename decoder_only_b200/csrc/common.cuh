@@ -15,12 +15,15 @@ typedef __nv_bfloat16 bf16;
         if (_e != cudaSuccess) return LLAMA_ERR_CUDA;      \
     } while (0)
 
+// Every kernel launch is followed by this check, which also counts it.
+void llama_count_launches(int64_t n);
 #define LLAMA_LAUNCH_CHECK()                               \
     do {                                                   \
         if (cudaPeekAtLastError() != cudaSuccess) {        \
             cudaGetLastError();                            \
             return LLAMA_ERR_CUDA;                         \
         }                                                  \
+        llama_count_launches(1);                           \
     } while (0)
 
 // Device error word values (sticky, set by bounded waits)

@@ -19,7 +19,7 @@ int launch_rmsnorm(int dtype, const float* x, const float* g, void* y, int rows,
                    cudaStream_t st);
 int launch_embed(int dtype, const int32_t* tok, const void* E, float* x, int rows, int d, int vocab, int* err,
                  cudaStream_t st);
-int launch_argmax(const float* logits, int rows, int n, int32_t* out, cudaStream_t st);
+int launch_argmax(const float* logits, int rows, int n, int64_t ld, int32_t* out, cudaStream_t st);
 
 // simt.cu  (fp32 storage path and shared epilogue passes)
 int launch_gemm_simt(int dtype, const void* A, const void* W, float* C, int M, int N, int K, int accumulate,

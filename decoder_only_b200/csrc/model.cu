@@ -17,11 +17,90 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
+#include <string>
 #include <vector>
 
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
+
+// ------------------------------------------------------------------ counters
+// Launches of this library's kernels (graph replays count their kernels).
+static std::atomic<int64_t> g_launches{0};
+void llama_count_launches(int64_t n) { g_launches += n; }
+
+namespace prof {
+// Optional per-region timing with CUDA events (eager launches only): each
+// region records its device time, its kernel launches and the algorithmic
+// bytes / FLOPs it was given.
+struct Entry {
+    std::string name;
+    double ms = 0, bytes = 0, flops = 0;
+    int64_t launches = 0, calls = 0;
+};
+struct Pending {
+    int idx;
+    cudaEvent_t a, b;
+};
+static bool on = false;
+static std::vector<Entry> entries;
+static std::vector<Pending> pending;
+static std::vector<cudaEvent_t> pool;
+
+static cudaEvent_t get_event() {
+    if (!pool.empty()) {
+        cudaEvent_t e = pool.back();
+        pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+static void flush() {
+    for (auto& p : pending) {
+        float ms = 0.f;
+        cudaEventSynchronize(p.b);
+        cudaEventElapsedTime(&ms, p.a, p.b);
+        entries[p.idx].ms += ms;
+        pool.push_back(p.a);
+        pool.push_back(p.b);
+    }
+    pending.clear();
+}
+static int find(const char* name) {
+    for (size_t i = 0; i < entries.size(); ++i)
+        if (entries[i].name == name) return (int)i;
+    entries.push_back(Entry());
+    entries.back().name = name;
+    return (int)entries.size() - 1;
+}
+struct Scope {
+    int idx = -1;
+    cudaEvent_t a = nullptr;
+    cudaStream_t st;
+    int64_t l0 = 0;
+    Scope(cudaStream_t s, const char* name, double bytes, double flops) : st(s) {
+        if (!on) return;
+        idx = find(name);
+        entries[idx].bytes += bytes;
+        entries[idx].flops += flops;
+        entries[idx].calls += 1;
+        a = get_event();
+        cudaEventRecord(a, st);
+        l0 = g_launches.load();
+    }
+    ~Scope() {
+        if (idx < 0) return;
+        cudaEvent_t b = get_event();
+        cudaEventRecord(b, st);
+        entries[idx].launches += g_launches.load() - l0;
+        pending.push_back({idx, a, b});
+        if (pending.size() > 4096) flush();
+    }
+};
+}  // namespace prof
 
 namespace {
 
@@ -71,6 +150,9 @@ struct llama_model {
     float* attn_work;
     uint64_t attn_work_bytes;
     int32_t* tok_cur;        // decode input tokens; argmax writes the next ones here
+    int32_t* tok_in;         // prompt tokens copied from the host [max_batch * max_seq]
+    int32_t* gen_out;        // generated tokens [max_seq, max_batch]
+    float* trunk_last;       // last-position trunk rows [max_batch, d]
     int* d_pos;              // decode position
     int* d_err;              // sticky device error word
     int B;                   // batch of the last prefill (0: none)
@@ -79,6 +161,7 @@ struct llama_model {
     cudaStream_t cap_stream;
     cudaGraphExec_t graph;
     int graph_B;
+    int64_t graph_kernels;   // kernels per replay of the decode graph
 };
 
 namespace {
@@ -153,6 +236,9 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     const uint64_t awb = attention_decode_work_bytes(c->max_batch, c->n_heads, c->max_seq, c->head_dim);
     float* attn_work = (float*)take(awb);
     int32_t* tok_cur = (int32_t*)take((size_t)c->max_batch * 4);
+    int32_t* tok_in = (int32_t*)take(nmax * 4);
+    int32_t* gen_out = (int32_t*)take(nmax * 4);
+    float* trunk_last = (float*)take((size_t)c->max_batch * d * 4);
     int* small = (int*)take(256);
     if (m) {
         m->g_final = g_final;
@@ -172,6 +258,9 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
         m->attn_work = attn_work;
         m->attn_work_bytes = awb;
         m->tok_cur = tok_cur;
+        m->tok_in = tok_in;
+        m->gen_out = gen_out;
+        m->trunk_last = trunk_last;
         m->d_pos = small;
         m->d_err = small + 1;
     }
@@ -206,12 +295,27 @@ EpiArgs base_args(llama_model* m, int M, int N) {
 // Prefill (decode = false): tcgen05 GEMM with the fused epilogue (bf16) or
 // SIMT GEMM + epilogue pass (fp32).  Decode: split-K swap-AB tcgen05 GEMM
 // into partials + reduction with the epilogue (bf16); SIMT for fp32.
-int project(llama_model* m, int mode, const void* A, const void* W, int M, int N, int K, int splits,
-            const EpiArgs& a, bool decode, cudaStream_t st) {
+double out_bytes(int mode, int M, int N, int esz) {
+    switch (mode) {
+        case EPI_F32: return (double)M * N * 4;
+        case EPI_RESID: return (double)M * N * 8;     // read + write of the fp32 trunk
+        case EPI_SWIGLU: return (double)M * (N / 2) * esz;
+        default: return (double)M * N * esz;           // Q, K, V
+    }
+}
+
+int project(llama_model* m, const char* name, int mode, const void* A, const void* W, int M, int N, int K,
+            int splits, const EpiArgs& a, bool decode, cudaStream_t st) {
     const int dt = m->cfg.dtype;
+    const double esz = m->esz;
+    const double flops = 2.0 * M * N * K;
+    const double in_bytes = ((double)M * K + (double)N * K) * esz;
+    char region[64];
+    snprintf(region, sizeof(region), "%s_gemm_%s", decode ? "decode" : "prefill", name);
     if (dt == LLAMA_BF16) {
         TcGemm g;
         if (!decode) {
+            prof::Scope ps(st, region, in_bytes + out_bytes(mode, M, N, m->esz), flops);
             g.A = A;
             g.B = W;
             g.rowsA = M;
@@ -230,11 +334,17 @@ int project(llama_model* m, int mode, const void* A, const void* W, int M, int N
         g.swap = 1;
         EpiArgs pa = a;
         pa.out = m->partial;
-        int rc = launch_gemm_tc(g, EPI_PARTIAL, pa, m->d_err, st);
-        if (rc) return rc;
+        {
+            prof::Scope ps(st, region, in_bytes, flops);
+            int rc = launch_gemm_tc(g, EPI_PARTIAL, pa, m->d_err, st);
+            if (rc) return rc;
+        }
+        snprintf(region, sizeof(region), "decode_reduce_%s", name);
+        prof::Scope ps(st, region, out_bytes(mode, M, N, m->esz), 0.0);
         return launch_splitk_reduce(mode, m->partial, splits, a, st);
     }
     // fp32 storage: SIMT GEMM
+    prof::Scope ps(st, region, in_bytes + out_bytes(mode, M, N, m->esz), flops);
     if (mode == EPI_RESID) return launch_gemm_simt(dt, A, W, a.out, M, N, K, 1, st);
     if (mode == EPI_F32) return launch_gemm_simt(dt, A, W, a.out, M, N, K, 0, st);
     int rc = launch_gemm_simt(dt, A, W, m->gemm_c, M, N, K, 0, st);
@@ -251,20 +361,27 @@ int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
     int rc;
     for (int l = 0; l < c.n_layers; ++l) {
         const Layer& ly = m->layers[l];
+        const double nb = (double)n * d * (4 + m->esz);
         // attention sublayer
-        if ((rc = launch_rmsnorm(dt, m->trunk, ly.g_attn, m->xn, n, d, c.norm_eps, st))) return rc;
+        {
+            prof::Scope ps(st, decode ? "decode_rmsnorm" : "prefill_rmsnorm", nb, 3.0 * n * d);
+            if ((rc = launch_rmsnorm(dt, m->trunk, ly.g_attn, m->xn, n, d, c.norm_eps, st))) return rc;
+        }
         EpiArgs qa = base_args(m, n, 3 * d);
         qa.q = m->q;
         qa.kc = kcache(m, l);
         qa.vc = vcache(m, l);
         qa.S = decode ? 1 : S;
         qa.d_pos = decode ? m->d_pos : nullptr;
-        if ((rc = project(m, EPI_QKV, m->xn, ly.wqkv, n, 3 * d, d, m->splits_qkv, qa, decode, st))) return rc;
+        if ((rc = project(m, "qkv", EPI_QKV, m->xn, ly.wqkv, n, 3 * d, d, m->splits_qkv, qa, decode, st))) return rc;
         if (decode) {
+            const double len = (double)m->cur_len + 1;   // keys read this step
+            prof::Scope ps(st, "decode_attention", (2.0 * len + 2.0) * B * d * m->esz, 4.0 * B * d * len);
             if ((rc = launch_attention_decode(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, 0,
                                               m->d_pos, c.head_dim, c.max_seq, m->attn_work, st)))
                 return rc;
         } else {
+            prof::Scope ps(st, "prefill_attention", 4.0 * n * d * m->esz, 2.0 * B * (double)S * (S + 1) * d);
             if ((rc = launch_attention_prefill_simt(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, S,
                                                     c.head_dim, c.max_seq, st)))
                 return rc;
@@ -272,37 +389,58 @@ int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
         EpiArgs ra = base_args(m, n, d);
         ra.out = m->trunk;
         ra.ld_out = d;
-        if ((rc = project(m, EPI_RESID, m->attn, ly.wo, n, d, d, m->splits_o, ra, decode, st))) return rc;
+        if ((rc = project(m, "o", EPI_RESID, m->attn, ly.wo, n, d, d, m->splits_o, ra, decode, st))) return rc;
         // feed-forward sublayer
-        if ((rc = launch_rmsnorm(dt, m->trunk, ly.g_ffn, m->xn, n, d, c.norm_eps, st))) return rc;
+        {
+            prof::Scope ps(st, decode ? "decode_rmsnorm" : "prefill_rmsnorm", nb, 3.0 * n * d);
+            if ((rc = launch_rmsnorm(dt, m->trunk, ly.g_ffn, m->xn, n, d, c.norm_eps, st))) return rc;
+        }
         EpiArgs sa = base_args(m, n, 2 * h);
         sa.act = m->act;
-        if ((rc = project(m, EPI_SWIGLU, m->xn, ly.wgu, n, 2 * h, d, m->splits_gu, sa, decode, st))) return rc;
-        if ((rc = project(m, EPI_RESID, m->act, ly.wd, n, d, h, m->splits_d, ra, decode, st))) return rc;
+        if ((rc = project(m, "gateup", EPI_SWIGLU, m->xn, ly.wgu, n, 2 * h, d, m->splits_gu, sa, decode, st))) return rc;
+        if ((rc = project(m, "down", EPI_RESID, m->act, ly.wd, n, d, h, m->splits_d, ra, decode, st))) return rc;
     }
     return LLAMA_OK;
 }
 
-int run_head(llama_model* m, int n, float* logits, bool decode, cudaStream_t st) {
+int run_head(llama_model* m, const float* x, int n, float* logits, bool decode, cudaStream_t st) {
     const llama_config& c = m->cfg;
-    int rc = launch_rmsnorm(c.dtype, m->trunk, m->g_final, m->xn, n, c.d_model, c.norm_eps, st);
+    int rc;
+    {
+        prof::Scope ps(st, decode ? "decode_rmsnorm" : "prefill_rmsnorm", (double)n * c.d_model * (4 + m->esz),
+                       3.0 * n * c.d_model);
+        rc = launch_rmsnorm(c.dtype, x, m->g_final, m->xn, n, c.d_model, c.norm_eps, st);
+    }
     if (rc) return rc;
     EpiArgs a = base_args(m, n, c.vocab);
     a.out = logits;
     a.ld_out = c.vocab;
-    return project(m, EPI_F32, m->xn, m->head, n, c.vocab, c.d_model, m->splits_head, a, decode, st);
+    return project(m, "head", EPI_F32, m->xn, m->head, n, c.vocab, c.d_model, m->splits_head, a, decode, st);
 }
 
 // Body of one decode step on the internal buffers: tok_cur -> tok_cur.
 int decode_body(llama_model* m, cudaStream_t st) {
     const llama_config& c = m->cfg;
-    int rc = launch_embed(c.dtype, m->tok_cur, m->embed, m->trunk, m->B, c.d_model, c.vocab, m->d_err, st);
+    int rc;
+    {
+        prof::Scope ps(st, "decode_embed", (double)m->B * c.d_model * (4 + m->esz), 0.0);
+        rc = launch_embed(c.dtype, m->tok_cur, m->embed, m->trunk, m->B, c.d_model, c.vocab, m->d_err, st);
+    }
     if (rc) return rc;
     if ((rc = run_blocks(m, m->B, 1, true, st))) return rc;
-    if ((rc = run_head(m, m->B, m->logits_dec, true, st))) return rc;
-    if ((rc = launch_argmax(m->logits_dec, m->B, c.vocab, m->tok_cur, st))) return rc;
+    if ((rc = run_head(m, m->trunk, m->B, m->logits_dec, true, st))) return rc;
+    prof::Scope ps(st, "decode_argmax", (double)m->B * c.vocab * 4, 0.0);
+    if ((rc = launch_argmax(m->logits_dec, m->B, c.vocab, c.vocab, m->tok_cur, st))) return rc;
     pos_advance_kernel<<<1, 1, 0, st>>>(m->d_pos);
     LLAMA_LAUNCH_CHECK();
+    return LLAMA_OK;
+}
+
+// One decode step: the captured graph, or eager launches while profiling.
+int decode_once(llama_model* m, cudaStream_t st) {
+    if (prof::on) return decode_body(m, st);
+    LLAMA_CUDA_TRY(cudaGraphLaunch(m->graph, st));
+    llama_count_launches(m->graph_kernels);
     return LLAMA_OK;
 }
 
@@ -313,9 +451,15 @@ int ensure_graph(llama_model* m) {
         m->graph = nullptr;
     }
     cudaGraph_t g = nullptr;
+    const bool prof_was = prof::on;
+    prof::on = false;
+    const int64_t l0 = g_launches.load();
     LLAMA_CUDA_TRY(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
     int rc = decode_body(m, m->cap_stream);
     cudaError_t e = cudaStreamEndCapture(m->cap_stream, &g);
+    prof::on = prof_was;
+    m->graph_kernels = g_launches.load() - l0;   // captured, not run
+    g_launches -= m->graph_kernels;
     if (rc) {
         if (g) cudaGraphDestroy(g);
         return rc;
@@ -390,6 +534,7 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
     m->cur_len = 0;
     m->graph = nullptr;
     m->graph_B = 0;
+    m->graph_kernels = 0;
     if (cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
         delete m;
         return LLAMA_ERR_CUDA;
@@ -455,10 +600,22 @@ int llama_prefill(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S,
         return LLAMA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     const int n = B * S;
-    int rc = launch_embed(m->cfg.dtype, d_tokens, m->embed, m->trunk, n, m->cfg.d_model, m->cfg.vocab, m->d_err, st);
+    int rc;
+    {
+        prof::Scope ps(st, "prefill_embed", (double)n * m->cfg.d_model * (4 + m->esz), 0.0);
+        rc = launch_embed(m->cfg.dtype, d_tokens, m->embed, m->trunk, n, m->cfg.d_model, m->cfg.vocab, m->d_err, st);
+    }
     if (rc) return rc;
     if ((rc = run_blocks(m, B, S, false, st))) return rc;
-    if (d_logits && (rc = run_head(m, n, d_logits, false, st))) return rc;
+    if (d_logits) {
+        if ((rc = run_head(m, m->trunk, n, d_logits, false, st))) return rc;
+        // greedy choice at each sequence's last position: the input of the
+        // first decode step when llama_generate is given no tokens
+        prof::Scope ps(st, "prefill_argmax", (double)B * m->cfg.vocab * 4, 0.0);
+        if ((rc = launch_argmax(d_logits + (size_t)(S - 1) * m->cfg.vocab, B, m->cfg.vocab,
+                                (int64_t)S * m->cfg.vocab, m->tok_cur, st)))
+            return rc;
+    }
     pos_set_kernel<<<1, 1, 0, st>>>(m->d_pos, S);
     LLAMA_LAUNCH_CHECK();
     m->B = B;
@@ -489,7 +646,7 @@ int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t* d_next, 
     int rc = ensure_graph(m);
     if (rc) return rc;
     LLAMA_CUDA_TRY(cudaMemcpyAsync(m->tok_cur, d_tokens, (size_t)m->B * 4, cudaMemcpyDeviceToDevice, st));
-    LLAMA_CUDA_TRY(cudaGraphLaunch(m->graph, st));
+    if ((rc = decode_once(m, st))) return rc;
     if (d_next) LLAMA_CUDA_TRY(cudaMemcpyAsync(d_next, m->tok_cur, (size_t)m->B * 4, cudaMemcpyDeviceToDevice, st));
     if (d_logits)
         LLAMA_CUDA_TRY(cudaMemcpyAsync(d_logits, m->logits_dec, (size_t)m->B * m->cfg.vocab * 4,
@@ -499,14 +656,15 @@ int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t* d_next, 
 }
 
 int llama_generate(llama_model* m, const int32_t* d_first, int32_t n_steps, int32_t* d_out, void* stream) {
-    if (!m || !d_first || !d_out || n_steps < 0) return LLAMA_ERR_INVALID_ARG;
+    if (!m || !d_out || n_steps < 0) return LLAMA_ERR_INVALID_ARG;
     if (m->B <= 0 || m->cur_len + n_steps > m->cfg.max_seq) return LLAMA_ERR_STATE;
     cudaStream_t st = (cudaStream_t)stream;
     int rc = ensure_graph(m);
     if (rc) return rc;
-    LLAMA_CUDA_TRY(cudaMemcpyAsync(m->tok_cur, d_first, (size_t)m->B * 4, cudaMemcpyDeviceToDevice, st));
+    if (d_first)
+        LLAMA_CUDA_TRY(cudaMemcpyAsync(m->tok_cur, d_first, (size_t)m->B * 4, cudaMemcpyDeviceToDevice, st));
     for (int i = 0; i < n_steps; ++i) {
-        LLAMA_CUDA_TRY(cudaGraphLaunch(m->graph, st));
+        if ((rc = decode_once(m, st))) return rc;
         LLAMA_CUDA_TRY(cudaMemcpyAsync(d_out + (size_t)i * m->B, m->tok_cur, (size_t)m->B * 4,
                                        cudaMemcpyDeviceToDevice, st));
         m->cur_len += 1;
@@ -515,6 +673,38 @@ int llama_generate(llama_model* m, const int32_t* d_first, int32_t n_steps, int3
 }
 
 int llama_position(const llama_model* m) { return m ? m->cur_len : LLAMA_ERR_INVALID_ARG; }
+
+int llama_rewind(llama_model* m, int32_t position, void* stream) {
+    if (!m || position < 1 || position > m->cur_len) return LLAMA_ERR_INVALID_ARG;
+    if (m->B <= 0) return LLAMA_ERR_STATE;
+    pos_set_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(m->d_pos, position);
+    LLAMA_LAUNCH_CHECK();
+    m->cur_len = position;
+    return LLAMA_OK;
+}
+
+int llama_complete(llama_model* m, const int32_t* h_tokens, int32_t B, int32_t S, float* d_logits, int32_t n_steps,
+                   int32_t* h_out, void* stream) {
+    if (!m || !h_tokens || !h_out || B <= 0 || S <= 0 || n_steps < 0 || B > m->cfg.max_batch ||
+        S + n_steps > m->cfg.max_seq)
+        return LLAMA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const llama_config& c = m->cfg;
+    LLAMA_CUDA_TRY(cudaMemcpyAsync(m->tok_in, h_tokens, (size_t)B * S * 4, cudaMemcpyHostToDevice, st));
+    int rc = llama_prefill(m, m->tok_in, B, S, d_logits, stream);
+    if (rc) return rc;
+    if (!d_logits) {
+        // head on the last position of each sequence only
+        LLAMA_CUDA_TRY(cudaMemcpy2DAsync(m->trunk_last, (size_t)c.d_model * 4, m->trunk + (size_t)(S - 1) * c.d_model,
+                                         (size_t)S * c.d_model * 4, (size_t)c.d_model * 4, B,
+                                         cudaMemcpyDeviceToDevice, st));
+        if ((rc = run_head(m, m->trunk_last, B, m->logits_dec, true, st))) return rc;
+        if ((rc = launch_argmax(m->logits_dec, B, c.vocab, c.vocab, m->tok_cur, st))) return rc;
+    }
+    if ((rc = llama_generate(m, nullptr, n_steps, m->gen_out, stream))) return rc;
+    LLAMA_CUDA_TRY(cudaMemcpyAsync(h_out, m->gen_out, (size_t)n_steps * B * 4, cudaMemcpyDeviceToHost, st));
+    return LLAMA_OK;
+}
 
 int llama_model_tensor(const llama_model* m, const char* name, int32_t layer, void** d_ptr, uint64_t* bytes) {
     if (!m || !name || !d_ptr || !bytes) return LLAMA_ERR_INVALID_ARG;
@@ -623,7 +813,37 @@ int llama_op_attention_decode(int32_t dtype, const void* d_q, const void* d_k, c
 
 int llama_op_argmax(const float* d_logits, int32_t rows, int32_t n, int32_t* d_out, void* stream) {
     if (!d_logits || !d_out || rows < 0 || n <= 0) return LLAMA_ERR_INVALID_ARG;
-    return launch_argmax(d_logits, rows, n, d_out, (cudaStream_t)stream);
+    return launch_argmax(d_logits, rows, n, n, d_out, (cudaStream_t)stream);
+}
+
+int64_t llama_kernel_launches(void) { return g_launches.load(); }
+
+int llama_profile_enable(int32_t on) {
+    prof::on = on != 0;
+    return LLAMA_OK;
+}
+
+void llama_profile_reset(void) {
+    prof::flush();
+    prof::entries.clear();
+}
+
+int llama_profile_count(void) {
+    prof::flush();
+    return (int)prof::entries.size();
+}
+
+int llama_profile_entry(int32_t i, const char** name, double* ms, int64_t* launches, int64_t* calls,
+                        double* bytes, double* flops) {
+    if (i < 0 || i >= (int)prof::entries.size()) return LLAMA_ERR_INVALID_ARG;
+    const prof::Entry& e = prof::entries[i];
+    if (name) *name = e.name.c_str();
+    if (ms) *ms = e.ms;
+    if (launches) *launches = e.launches;
+    if (calls) *calls = e.calls;
+    if (bytes) *bytes = e.bytes;
+    if (flops) *flops = e.flops;
+    return LLAMA_OK;
 }
 
 }  // extern "C"

@@ -105,10 +105,10 @@ int launch_embed(int dtype, const int32_t* tok, const void* E, float* x, int row
 }
 
 // Greedy choice: argmax over a logits row, lowest index on ties.  One CTA per row.
-__global__ void __launch_bounds__(256) argmax_kernel(const float* __restrict__ logits, int n,
+__global__ void __launch_bounds__(256) argmax_kernel(const float* __restrict__ logits, int n, int64_t ld,
                                                      int32_t* __restrict__ out) {
     const int r = blockIdx.x;
-    const float* p = logits + (size_t)r * n;
+    const float* p = logits + (size_t)r * ld;
     float best = -INFINITY;
     int bi = 0x7fffffff;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
@@ -145,9 +145,9 @@ __global__ void __launch_bounds__(256) argmax_kernel(const float* __restrict__ l
     }
 }
 
-int launch_argmax(const float* logits, int rows, int n, int32_t* out, cudaStream_t st) {
+int launch_argmax(const float* logits, int rows, int n, int64_t ld, int32_t* out, cudaStream_t st) {
     if (rows <= 0) return LLAMA_OK;
-    argmax_kernel<<<rows, 256, 0, st>>>(logits, n, out);
+    argmax_kernel<<<rows, 256, 0, st>>>(logits, n, ld, out);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }

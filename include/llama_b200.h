@@ -122,13 +122,30 @@ LLAMA_API int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t
                       float* d_logits, void* stream);
 
 /* n_steps greedy steps fed back on the device: step 0 consumes
- * d_first [B]; step i consumes the token step i-1 chose.  d_out:
- * int32 [n_steps, B].  Replays one captured CUDA graph per step. */
+ * d_first [B] (or, when d_first is NULL, the greedy choice at the last
+ * position of the preceding llama_prefill that produced logits, or the
+ * token the preceding step chose); step i consumes the token step i-1
+ * chose.  d_out: int32 [n_steps, B].  Replays one captured CUDA graph per
+ * step (launched eagerly while profiling is enabled). */
 LLAMA_API int llama_generate(llama_model* m, const int32_t* d_first, int32_t n_steps,
                    int32_t* d_out, void* stream);
 
 /* Current decode position (tokens held per sequence in the KV cache). */
 LLAMA_API int llama_position(const llama_model* m);
+
+/* Move the decode position back to `position` (1 <= position <= current):
+ * cache entries below it are kept, later ones are overwritten by the next
+ * steps.  Queued on `stream`. */
+LLAMA_API int llama_rewind(llama_model* m, int32_t position, void* stream);
+
+/* End to end from HOST buffers: copy h_tokens (int32 [B*S], host; pinned
+ * memory makes the copy asynchronous) to the device, prefill (logits of
+ * every position into d_logits [B*S, vocab] when it is not NULL, else the
+ * head runs on each sequence's last position only), then n_steps greedy
+ * steps, and copy the generated tokens to h_out (int32 [n_steps, B],
+ * host).  Asynchronous on `stream`: h_out is valid after a synchronise. */
+LLAMA_API int llama_complete(llama_model* m, const int32_t* h_tokens, int32_t B, int32_t S,
+                             float* d_logits, int32_t n_steps, int32_t* h_out, void* stream);
 
 /* Device pointer and byte size of an internal buffer, for inspection:
  * name in {"kv" (the whole cache), "trunk", "q", "attn", "act", "xn",
@@ -146,6 +163,25 @@ LLAMA_API int llama_last_error(llama_model* m);
 LLAMA_API void llama_free(llama_model* m);
 
 LLAMA_API const char* llama_status_str(int status);
+
+/* --------------------------------------------------------- instrumentation */
+
+/* Kernel launches this library has issued in this process; a replay of the
+ * captured decode graph counts every kernel in it. */
+LLAMA_API int64_t llama_kernel_launches(void);
+
+/* Per-region device timing (process-wide, host-side state).  While enabled,
+ * every region of the launch sequence (one GEMM, its reduction, a norm,
+ * an attention pass ...) is bracketed by CUDA events on its stream and the
+ * decode step runs eagerly instead of as a graph.  Entries accumulate the
+ * region's device milliseconds, kernel launches, calls, and the algorithmic
+ * bytes and FLOPs of the work it was handed.  llama_profile_count()
+ * synchronises on the pending events. */
+LLAMA_API int llama_profile_enable(int32_t on);
+LLAMA_API void llama_profile_reset(void);
+LLAMA_API int llama_profile_count(void);
+LLAMA_API int llama_profile_entry(int32_t i, const char** name, double* ms, int64_t* launches,
+                                  int64_t* calls, double* bytes, double* flops);
 
 /* ------------------------------------------------------------ single ops
  * The kernels the model runs, exposed one by one on caller buffers.  dtype

@@ -27,3 +27,21 @@ def argmax_agreement(got, ref):
     err = np.max(np.abs(got - ref))
     ok = ref[np.arange(len(g)), g] >= ref.max(-1) - 2 * err
     return strict, float(np.mean(ok))
+
+
+def storage_bar(got, exact, stored, rms_factor=1.5, max_factor=2.0):
+    """Accuracy bar for bf16 workloads, derived from the arithmetic.
+
+    `exact` is the fp64 oracle, `stored` the same oracle rounding every value
+    the workload stores in bf16.  The GPU result must be no further from the
+    exact answer than `rms_factor` (RMS norm) / `max_factor` (max norm) times
+    the distance bf16 storage alone produces.  Returns the four numbers."""
+    r = rms(exact)
+    g = np.asarray(got, dtype=np.float64) - exact
+    s = np.asarray(stored, dtype=np.float64) - exact
+    out = dict(gpu_rms=rms(g) / r, gpu_max=float(np.max(np.abs(g))) / r,
+               bf16_rms=rms(s) / r, bf16_max=float(np.max(np.abs(s))) / r)
+    print("accuracy vs exact oracle:", {k: round(v, 5) for k, v in out.items()})
+    assert out["gpu_rms"] <= rms_factor * out["bf16_rms"], out
+    assert out["gpu_max"] <= max_factor * out["bf16_max"], out
+    return out

@@ -1,6 +1,14 @@
 """Parity of the bf16 7B-shaped paths at their full sizes.
 
- * one 7B block on an N(0,1) fp32 trunk, 1 x 2048 (y and y - x at 2e-2 RMS);
+Accuracy bar (derived from the arithmetic; see tests/_parity.storage_bar):
+the GPU must be no further from the exact fp64 oracle than bf16 storage of
+the values the workload stores in bf16 moves the oracle itself (x1.5 RMS,
+x2 max), and its greedy choices must agree on >= 99% of positions.  A fixed
+2e-2 RMS max-norm bound is unreachable at 32 layers with a bf16 KV cache
+(tests/test_oracle_pins.py::test_bf16_kv_cache_alone_moves_deep_logits_past_2e2).
+
+ * one 7B block on an N(0,1) fp32 trunk, 1 x 2048 (y and the block's
+   increment y - x);
  * the 32-layer model, prefill 4 x 2048: sampled rows (whole rows of two
    sequences, positions 0..99) against the oracle -- exact by causality;
  * greedy decode against the oracle (prompt 96, teacher-forced steps 96..99);
@@ -16,10 +24,9 @@ import decoder_only_b200 as lb
 import oracle
 import synth
 from synth.workloads import BLOCK_7B, LLAMA_7B, SEED
-from _parity import rel_max_err, argmax_agreement, rms
+from _parity import rel_max_err, argmax_agreement, rms, storage_bar
 
 pytestmark = pytest.mark.gpu
-TOL = 2e-2
 B, S, STEPS = 4, 2048, 128
 
 
@@ -31,9 +38,11 @@ def test_single_block_7b():
     finally:
         m.close()
     x64 = x.astype(np.float64)
-    ref = oracle.block_forward(BLOCK_7B, x64)
-    assert rel_max_err(y, ref) <= TOL
-    assert rel_max_err(y - x64, ref - x64) <= TOL
+    W = oracle.layer_weights(BLOCK_7B, 0)
+    ref = oracle.block_forward(BLOCK_7B, x64, weights=W)
+    ref16 = oracle.block_forward(BLOCK_7B, x64, weights=W, storage="bf16")
+    storage_bar(y, ref, ref16)
+    storage_bar(y - x64, ref - x64, ref16 - x64)
 
 
 @pytest.fixture(scope="module")
@@ -51,19 +60,31 @@ def tokens():
 
 @pytest.fixture(scope="module")
 def oracle_rows(tokens):
-    """Oracle logits of sequences 0 and 3, positions 0..99."""
-    return oracle.prefill(LLAMA_7B, tokens[[0, 3], :100])
+    """Oracle logits of sequences 0 and 3, positions 0..99: exact, and with
+    bf16 storage of the values the workload stores in bf16."""
+    cache = {}
+
+    def w(l):
+        if l not in cache:
+            cache.clear()
+            cache[l] = oracle.layer_weights(LLAMA_7B, l)
+        return cache[l]
+
+    exact = oracle.prefill(LLAMA_7B, tokens[[0, 3], :100], weights=w)
+    stored = oracle.prefill(LLAMA_7B, tokens[[0, 3], :100], weights=w, storage="bf16")
+    return exact, stored
 
 
 def test_prefill_full_size_sampled_rows(model, tokens, oracle_rows):
     lg = model.prefill(torch.from_numpy(tokens[:, :S].copy()).cuda())
     got = lg[[0, 3], :100].cpu().numpy()
-    assert rel_max_err(got, oracle_rows) <= TOL
-    assert argmax_agreement(got, oracle_rows)[1] >= 0.99
+    exact, stored = oracle_rows
+    storage_bar(got, exact, stored)
+    assert argmax_agreement(got, exact)[1] >= 0.99
     # every row is finite and on the oracle's scale
     r = lg.float()
     assert torch.isfinite(r).all()
-    assert abs(float(r.std()) / rms(oracle_rows) - 1.0) < 0.1
+    assert abs(float(r.std()) / rms(exact) - 1.0) < 0.1
 
 
 def test_greedy_decode_against_oracle(model, tokens, oracle_rows):
@@ -73,11 +94,12 @@ def test_greedy_decode_against_oracle(model, tokens, oracle_rows):
         _, lg = model.decode_step(torch.from_numpy(tokens[:, t].copy()).cuda())
         got.append(lg[[0, 3]].cpu().numpy())
     got = np.stack(got, axis=1)
-    assert rel_max_err(got, oracle_rows[:, 96:100]) <= TOL
-    assert argmax_agreement(got, oracle_rows[:, 96:100])[1] >= 0.99
+    exact, stored = oracle_rows
+    storage_bar(got, exact[:, 96:100], stored[:, 96:100])
+    assert argmax_agreement(got, exact[:, 96:100])[1] >= 0.99
 
 
-def test_full_length_decode_equals_prefill_rows(model, tokens):
+def test_full_length_decode_equals_prefill_rows(model, tokens, oracle_rows):
     tk = torch.from_numpy(tokens).cuda()
     model.prefill(tk[:, :S].contiguous(), logits=False)
     dec = []
@@ -86,7 +108,17 @@ def test_full_length_decode_equals_prefill_rows(model, tokens):
         dec.append(lg.cpu().numpy())
     dec = np.stack(dec, axis=1)
     ref = model.prefill(tk[:, :S + 4].contiguous())[:, S:S + 4].cpu().numpy()
-    assert rel_max_err(dec, ref) <= TOL
+    # two bf16 computations of the same rows (split-K decode GEMMs and decode
+    # attention vs prefill kernels): each within the storage bar of the exact
+    # answer, so their difference within twice it
+    exact, stored = oracle_rows
+    r = rms(exact)
+    bar_rms = rms(stored - exact) / r
+    bar_max = float(np.max(np.abs(stored - exact))) / r
+    diff = dec - ref
+    print("decode vs prefill:", rms(diff) / rms(ref), np.max(np.abs(diff)) / rms(ref), bar_rms, bar_max)
+    assert rms(diff) / rms(ref) <= 2 * 1.5 * bar_rms
+    assert np.max(np.abs(diff)) / rms(ref) <= 2 * 2.0 * bar_max
     assert argmax_agreement(dec, ref)[1] >= 0.99
 
 
