@@ -159,7 +159,8 @@ def roofline(prof, decode_scale, peaks, peak_src):
     out.update(kernel=name, achieved=round(achieved, 1), peak=peak, frac=round(achieved / peak, 4),
                peak_source=peak_src, traffic=None, launches_profiled=f["launches"],
                avg_launch_us=round(per_launch_ms * 1e3, 2), share_of_step=round(f["step_ms"] / total, 4),
-               shares={k: round(v["step_ms"] / total, 4) for k, v in sorted(fam.items(), key=lambda kv: -kv[1]["step_ms"])})
+               shares={k: round(v["step_ms"] / total, 4) for k, v in sorted(fam.items(), key=lambda kv: -kv[1]["step_ms"])},
+               est_ms_per_step={k: round(v["step_ms"], 2) for k, v in sorted(fam.items(), key=lambda kv: -kv[1]["step_ms"])})
     return out
 
 
@@ -265,6 +266,14 @@ def run_b200(args, wl, shape):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    if args.ncu:
+        for _ in range(args.steps):
+            torch.cuda.nvtx.range_push("timed_step")
+            step()
+            torch.cuda.nvtx.range_pop()
+        torch.cuda.synchronize()
+        model.close()
+        return
 
     # ------------------------------------------------ timed region (device events)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -376,6 +385,36 @@ def run_b200(args, wl, shape):
         dist.destroy_process_group()
 
 
+def summarize_ncu(path):
+    """Per-kernel launches, total device time and share from an ncu
+    `--metrics gpu__time_duration.sum --csv` launch list."""
+    import csv
+    import re
+    with open(path) as f:
+        lines = f.read().splitlines()
+    start = next(i for i, l in enumerate(lines) if l.startswith('"ID"'))
+    rows = list(csv.DictReader(lines[start:]))
+    agg = {}
+    for r in rows:
+        if r.get("Metric Name") != "gpu__time_duration.sum":
+            continue
+        name = r["Kernel Name"]
+        name = re.sub(r"\(.*", "", name)
+        m = re.search(r"(gemm_tc_kernel|attn_\w+|\w+_kernel)(<[^>]*>)?", r["Kernel Name"])
+        key = m.group(0) if m else name
+        v = float(r["Metric Value"].replace(",", ""))
+        unit = r.get("Metric Unit", "nsecond")
+        scale = {"nsecond": 1e-3, "usecond": 1.0, "msecond": 1e3, "second": 1e6}.get(unit, 1e-3)
+        a = agg.setdefault(key, [0, 0.0])
+        a[0] += 1
+        a[1] += v * scale
+    total = sum(v[1] for v in agg.values())
+    print(f"{'kernel':70s} {'launches':>9s} {'total_ms':>10s} {'avg_us':>9s} {'share':>7s}")
+    for k, (n, us) in sorted(agg.items(), key=lambda kv: -kv[1][1]):
+        print(f"{k[:70]:70s} {n:9d} {us / 1e3:10.3f} {us / n:9.2f} {us / total:7.4f}")
+    print(f"{'total':70s} {sum(v[0] for v in agg.values()):9d} {total / 1e3:10.3f}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -384,7 +423,15 @@ def main():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--workload", default="7b", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu", action="store_true",
+                    help="only the warm-up and timed steps, each timed step in an NVTX range 'timed_step' "
+                         "(for: ncu --nvtx --nvtx-include timed_step/ ...); prints no JSON")
+    ap.add_argument("--summarize-ncu", metavar="CSV",
+                    help="print the per-kernel launches / time / share table of an ncu --csv launch list")
     args = ap.parse_args()
+    if args.summarize_ncu:
+        summarize_ncu(args.summarize_ncu)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from synth import workloads as wls
