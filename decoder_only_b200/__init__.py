@@ -57,6 +57,7 @@ def _load():
         "llama_op_attention_prefill": [I, P, P, P, P, I, I, I, I, I, P],
         "llama_op_attention_decode": [I, P, P, P, P, I, I, I, I, I, P, U64, P],
         "llama_op_attention_decode_work_bytes": [I, I, I, I],
+        "llama_op_attention_decode_noalloc": [I, P, P, P, P, I, I, I, I, I, P],
         "llama_op_argmax": [P, I, I, P, P],
         "llama_rewind": [P, I, P],
         "llama_complete": [P, P, I, I, P, I, P, P],
@@ -288,6 +289,17 @@ def attention_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, length: 
     _check(lib.llama_op_attention_decode(_dt(q), _ptr(q.contiguous()), _ptr(k.contiguous()), _ptr(v.contiguous()),
                                          _ptr(o), B, H, length, hd, kv_stride, _ptr(work), work.numel(),
                                          _stream()), "llama_op_attention_decode")
+    return o
+
+
+def attention_decode_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, length: int) -> torch.Tensor:
+    """attention_decode with the workspace in the library's fixed device
+    array: no allocation by the library (see the header for the limit)."""
+    B, H, kv_stride, hd = k.shape
+    o = torch.empty(B, H * hd, dtype=q.dtype, device=q.device)
+    _check(lib.llama_op_attention_decode_noalloc(_dt(q), _ptr(q.contiguous()), _ptr(k.contiguous()),
+                                                 _ptr(v.contiguous()), _ptr(o), B, H, length, hd, kv_stride,
+                                                 _stream()), "llama_op_attention_decode_noalloc")
     return o
 
 

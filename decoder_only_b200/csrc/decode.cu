@@ -7,6 +7,8 @@
 // is cut into chunks of 256 keys so that B*H*chunks CTAs cover the SMs; each
 // chunk leaves (max, sum, unnormalised output) in the workspace and a second
 // pass merges the chunks (the online-softmax merge rule).
+#include <mutex>
+
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
@@ -247,4 +249,68 @@ int launch_splitk_reduce(int mode, const float* partial, int splits, const EpiAr
     }
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Decode attention with no allocation at all.
+//
+// Some callers cannot call cudaMalloc (or hand us an allocator) when they
+// run a decode step: runtimes that plan every byte of device memory up
+// front and forbid allocation once serving starts, code that must not
+// allocate while it is being captured into a CUDA graph, or embedders that
+// have no device allocator to give us.  For them the split-sequence
+// workspace lives in a fixed array in this library's own device memory,
+// loaded with the library on every GPU that uses it and held until exit.
+//
+// Limit: 8 MiB of workspace, i.e. B * H * ceil(len / 256) * (head_dim + 2)
+// <= 2,097,152 floats (LLaMA-13B shapes at batch 32 and 2304 positions need
+// 1,497,600).  Larger calls are rejected with LLAMA_ERR_OOM before anything
+// is queued.  Every call shares the one array, so calls that overlap on the
+// GPU (other streams, other host threads) race; each call writes every
+// workspace slot it later reads, so nothing has to start at zero.
+constexpr size_t NOALLOC_SCRATCH_FLOATS = (size_t)2 << 20;
+static __device__ __align__(256) float g_decode_scratch[NOALLOC_SCRATCH_FLOATS];
+
+namespace {
+constexpr int MAX_DEVICES = 64;
+float* g_scratch_addr[MAX_DEVICES];
+std::mutex g_scratch_mu;
+
+// Device address of the array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and kept.
+int noalloc_scratch(float** out) {
+    int dev = -1;
+    LLAMA_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= MAX_DEVICES) return LLAMA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+        if (e != cudaSuccess || !p) {
+            cudaGetLastError();
+            return LLAMA_ERR_CUDA;
+        }
+        g_scratch_addr[dev] = static_cast<float*>(p);
+    }
+    *out = g_scratch_addr[dev];
+    return LLAMA_OK;
+}
+}  // namespace
+
+extern "C" LLAMA_API int llama_op_attention_decode_noalloc(int32_t dtype, const void* d_q, const void* d_k,
+                                                           const void* d_v, void* d_o, int32_t B, int32_t H,
+                                                           int32_t len, int32_t head_dim, int32_t kv_stride,
+                                                           void* stream) {
+    if (!d_q || !d_k || !d_v || !d_o || B <= 0 || H <= 0 || len <= 0 || kv_stride < len)
+        return LLAMA_ERR_INVALID_ARG;
+    if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+    if (head_dim != 32 && head_dim != 64 && head_dim != 128) return LLAMA_ERR_INVALID_ARG;
+    if (attention_decode_work_bytes(B, H, len, head_dim) > sizeof(float) * NOALLOC_SCRATCH_FLOATS)
+        return LLAMA_ERR_OOM;
+    float* work = nullptr;
+    const int rc = noalloc_scratch(&work);
+    if (rc) return rc;
+    return launch_attention_decode(dtype, d_q, d_k, d_v, d_o, B, H, len, nullptr, head_dim, kv_stride, work,
+                                   (cudaStream_t)stream);
 }

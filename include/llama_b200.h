@@ -221,6 +221,28 @@ LLAMA_API int llama_op_attention_decode(int32_t dtype, const void* d_q, const vo
 LLAMA_API uint64_t llama_op_attention_decode_work_bytes(int32_t B, int32_t H, int32_t max_len,
                                               int32_t head_dim);
 
+/* The same decode attention for callers that cannot allocate device
+ * memory when they call it (runtimes that plan all device memory up front,
+ * code being captured into a CUDA graph that must not allocate, embedders
+ * without a device allocator).  The pages have no counterpart: this is an
+ * integration variant.  The split-sequence workspace is a fixed 8 MiB array
+ * in the library's own device memory, held on every GPU that loads the
+ * library until the process exits; this call allocates nothing.
+ *   - B * H * ceil(len / 256) * (head_dim + 2) must be <= 2,097,152
+ *     (floats of workspace); larger calls return LLAMA_ERR_OOM and queue
+ *     nothing.  head_dim in {32, 64, 128}.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first
+ *     call before any stream capture.
+ *   - All calls share the array: calls that overlap on the GPU (different
+ *     streams or host threads) race.  Each call writes every workspace slot
+ *     it reads, so no clearing is needed between calls.
+ * Arguments and layouts as llama_op_attention_decode. */
+LLAMA_API int llama_op_attention_decode_noalloc(int32_t dtype, const void* d_q, const void* d_k,
+                                                const void* d_v, void* d_o, int32_t B, int32_t H,
+                                                int32_t len, int32_t head_dim, int32_t kv_stride,
+                                                void* stream);
+
 /* out[r] = argmax_j logits[r, j] (lowest j on ties), r < rows. */
 LLAMA_API int llama_op_argmax(const float* d_logits, int32_t rows, int32_t n, int32_t* d_out,
                     void* stream);
