@@ -1,0 +1,396 @@
+// Causal flash attention for prefill on the sm_100a tensor cores.
+//
+// Per head: O = softmax(Q K^T / sqrt(hd) + causal mask) V ("LLaMA is a pull
+// request against the 2017 transformer": attention untouched, causal mask;
+// "RoPE: rotate Q and K, leave V alone": Q and K arrive rotated).  The
+// fully masked key tiles above the diagonal are never computed, and the
+// (S x S) score matrix is never written to memory -- the two ideas the
+// knowledge note credits to the xFormers attention of the training system.
+//
+// One CTA per (128-query tile, head, sequence), longest tiles first.
+//   warp 0      TMA: Q once, then K_j and V_j tiles (2-stage ring).  3-D
+//               tensor maps (hd, position, head) make rows >= S read as 0.
+//   warp 1      TMEM allocator + MMA issuer:
+//                 S_j = Q K_j^T   (M 128, N 128, K hd)  -> TMEM S[j % 2]
+//                 O_j = P_j V_j   (M 128, N hd, K 128)  -> TMEM O[j % 2]
+//               V is the MN-major B operand (hd contiguous), so the cache
+//               layout [position][hd] is used as is.
+//   warps 2..5  one query row per thread: row max of S_j (pass 1), then
+//               p = 2^((s - m) log2e / sqrt(hd)) rounded to bf16 into the
+//               shared P tile (128-byte swizzled, K-major) and the row sum
+//               (pass 2); one tile later O_{j-1} is read from TMEM and
+//               folded into the fp32 running output with the online-softmax
+//               correction exp(m_old - m_new).
+// All mbarrier waits are bounded (see tcgen05.cuh).
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tcgen05.cuh"
+
+namespace {
+
+using namespace tc;
+
+constexpr int BQ = 128;         // queries per tile
+constexpr int BKV = 128;        // keys per tile
+constexpr int NTHREADS = 192;
+
+template <int HD>
+struct ACfg {
+    static constexpr int REG = 128 * 128;                    // one [128 rows][64 bf16] swizzled region, bytes
+    static constexpr int NREG = HD / 64;                     // regions per Q / K / V tile
+    static constexpr int TILE = NREG * REG;                  // Q, K or V tile bytes
+    static constexpr int P_TILE = 2 * REG;                   // P: [128 q][128 keys] bf16
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + TILE;               // [2]
+    static constexpr int OFF_V = OFF_K + 2 * TILE;           // [2]
+    static constexpr int OFF_P = OFF_V + 2 * TILE;           // [2]
+    static constexpr int OFF_BAR = OFF_P + 2 * P_TILE;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;               // S[2] at 0, 128; O[2] at 256, 384
+};
+
+// P tile position of 8 consecutive keys (one 16-byte chunk) of query row t:
+// region by key half, 128-byte row t, chunk index XOR (t % 8).
+__device__ __forceinline__ uint32_t p_chunk_addr(uint32_t base, int t, int chunk16) {
+    const int region = chunk16 >> 3;
+    const int c = chunk16 & 7;
+    return base + region * (128 * 128) + t * 128 + ((c ^ (t & 7)) << 4);
+}
+
+template <int HD>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ out, int H, int S,
+                           float scale_log2, int* err) {
+    using C = ACfg<HD>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    const uint32_t sQ = base + C::OFF_Q, sK = base + C::OFF_K, sV = base + C::OFF_V, sP = base + C::OFF_P;
+    const uint32_t bars = base + C::OFF_BAR;
+    const uint32_t q_full = bars;
+    const uint32_t k_full = bars + 8;        // [2]
+    const uint32_t v_full = bars + 24;       // [2]
+    const uint32_t kv_empty = bars + 40;     // [2]
+    const uint32_t s_full = bars + 56;       // [2]
+    const uint32_t s_empty = bars + 72;      // [2]
+    const uint32_t p_full = bars + 88;       // [2]
+    const uint32_t o_full = bars + 104;      // [2]
+    const uint32_t o_empty = bars + 120;     // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 160);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int qt = (int)(gridDim.x - 1 - blockIdx.x);     // longest (most key tiles) first
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int head = b * H + h;
+    const int q0 = qt * BQ;
+    const int n_kv = qt + 1;                              // key tiles 0..qt (causal)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(k_full + 8 * i, 1);
+            mbar_init(v_full + 8 * i, 1);
+            mbar_init(kv_empty + 8 * i, 1);
+            mbar_init(s_full + 8 * i, 1);
+            mbar_init(s_empty + 8 * i, 128);
+            mbar_init(p_full + 8 * i, 128);
+            mbar_init(o_full + 8 * i, 1);
+            mbar_init(o_empty + 8 * i, 128);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            mbar_expect_tx(q_full, C::TILE);
+            for (int r = 0; r < C::NREG; ++r) tma_load_3d(sQ + r * C::REG, &tmQ, q_full, 64 * r, q0, head);
+            int issued = 0;
+            for (int j = 0; j < n_kv && ok; ++j) {
+                const int st = j & 1;
+                if (!mbar_wait(kv_empty + 8 * st, ((j >> 1) & 1) ^ 1u, abort_flag, err)) {
+                    ok = false;
+                    break;
+                }
+                mbar_expect_tx(k_full + 8 * st, C::TILE);
+                for (int r = 0; r < C::NREG; ++r)
+                    tma_load_3d(sK + st * C::TILE + r * C::REG, &tmK, k_full + 8 * st, 64 * r, j * BKV, head);
+                mbar_expect_tx(v_full + 8 * st, C::TILE);
+                for (int r = 0; r < C::NREG; ++r)
+                    tma_load_3d(sV + st * C::TILE + r * C::REG, &tmV, v_full + 8 * st, 64 * r, j * BKV, head);
+                issued = j + 1;
+            }
+            if (!ok) {
+                // drain (bounded) the copies this thread issued
+                const uint64_t t0 = global_timer();
+                while (!mbar_try_wait(q_full, 0) && global_timer() - t0 < WAIT_LIMIT_NS / 4) {
+                }
+                for (int j = issued > 2 ? issued - 2 : 0; j < issued; ++j) {
+                    const int st = j & 1;
+                    const uint32_t par = (j >> 1) & 1;
+                    while (!(mbar_try_wait(k_full + 8 * st, par) && mbar_try_wait(v_full + 8 * st, par)) &&
+                           global_timer() - t0 < WAIT_LIMIT_NS / 2) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_QK = idesc_bf16(BKV);                 // K-major A and B
+            constexpr uint32_t IDESC_PV = idesc_bf16(HD) | (1u << 16);      // B (V) MN-major
+            bool ok = mbar_wait(q_full, 0, abort_flag, err);
+            tc_fence_after();
+            for (int j = 0; j <= n_kv && ok; ++j) {
+                if (j < n_kv) {
+                    const int st = j & 1;
+                    const uint32_t par = (j >> 1) & 1;
+                    if (!mbar_wait(k_full + 8 * st, par, abort_flag, err) ||
+                        !mbar_wait(s_empty + 8 * st, par ^ 1u, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_s = tmem + (uint32_t)(st * 128);
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * C::REG + (kk & 3) * 32;
+                        umma_bf16(d_s, sw128_desc(sQ + off), sw128_desc(sK + st * C::TILE + off), IDESC_QK,
+                                  kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(s_full + 8 * st);
+                }
+                if (j > 0) {
+                    const int jj = j - 1, st = jj & 1;
+                    const uint32_t par = (jj >> 1) & 1;
+                    if (!mbar_wait(p_full + 8 * st, par, abort_flag, err) ||
+                        !mbar_wait(v_full + 8 * st, par, abort_flag, err) ||
+                        !mbar_wait(o_empty + 8 * st, par ^ 1u, abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_o = tmem + 256u + (uint32_t)(st * 128);
+#pragma unroll
+                    for (int kk = 0; kk < BKV / 16; ++kk) {
+                        // A = P (K-major, keys contiguous); B = V (MN-major): 16 keys = 2 groups of 8 rows
+                        const uint32_t poff = (kk >> 2) * C::REG + (kk & 3) * 32;
+                        uint64_t vd = sw128_desc(sV + st * C::TILE + kk * 2048);
+                        vd = (vd & ~(((uint64_t)0x3FFF) << 16)) | ((uint64_t)(C::REG >> 4) << 16);   // LBO: next 64 hd
+                        umma_bf16(d_o, sw128_desc(sP + st * C::P_TILE + poff), vd, IDESC_PV, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(o_full + 8 * st);
+                    umma_commit(kv_empty + 8 * st);
+                }
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- softmax + output (warps 2..5)
+        const int quarter = warp & 3;
+        const int t = quarter * 32 + lane;               // query row within the tile
+        const int q = q0 + t;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        float o[HD];
+#pragma unroll
+        for (int i = 0; i < HD; ++i) o[i] = 0.f;
+        float m = -INFINITY, l = 0.f, corr_prev = 0.f;
+        bool ok = true;
+        for (int j = 0; j <= n_kv; ++j) {
+            float corr = 0.f;
+            if (j < n_kv) {
+                const int st = j & 1;
+                const uint32_t par = (j >> 1) & 1;
+                if (!mbar_wait(s_full + 8 * st, par, abort_flag, err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t s_addr = tmem + lane_addr + (uint32_t)(st * 128);
+                const bool diag = (j == n_kv - 1);
+                const int k0 = j * BKV;
+                // pass 1: row maximum over the visible keys
+                float mx = -INFINITY;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float sv[32];
+                    tmem_ld32(s_addr + c * 32, sv);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int key = k0 + c * 32 + i;
+                        const bool vis = !diag || (key <= q && key < S);
+                        mx = fmaxf(mx, vis ? sv[i] : -INFINITY);
+                    }
+                }
+                const float m_new = fmaxf(m, mx);
+                corr = (m == -INFINITY) ? 0.f : exp2f((m - m_new) * scale_log2);
+                const float mo = m_new * scale_log2;
+                // pass 2: probabilities (bf16) into the P tile, row sum from the rounded values
+                float rs = 0.f;
+                const uint32_t pbase = sP + st * C::P_TILE;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float sv[32];
+                    tmem_ld32(s_addr + c * 32, sv);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int key = k0 + c * 32 + 2 * i;
+                        const bool v0 = !diag || (key <= q && key < S);
+                        const bool v1 = !diag || (key + 1 <= q && key + 1 < S);
+                        const float p0 = v0 ? exp2f(fmaf(sv[2 * i], scale_log2, -mo)) : 0.f;
+                        const float p1 = v1 ? exp2f(fmaf(sv[2 * i + 1], scale_log2, -mo)) : 0.f;
+                        pk[i] = pack_bf16x2(p0, p1);
+                        const float2 r = unpack_bf16x2(pk[i]);
+                        rs += r.x + r.y;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t addr = p_chunk_addr(pbase, t, c * 4 + u);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * u]),
+                                     "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
+                                     : "memory");
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(s_empty + 8 * st);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(p_full + 8 * st);
+                l = l * corr + rs;
+                m = m_new;
+            }
+            if (j > 0) {
+                const int jj = j - 1, st = jj & 1;
+                const uint32_t par = (jj >> 1) & 1;
+                if (!mbar_wait(o_full + 8 * st, par, abort_flag, err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t o_addr = tmem + lane_addr + 256u + (uint32_t)(st * 128);
+#pragma unroll
+                for (int c = 0; c < HD / 32; ++c) {
+                    float ov[32];
+                    tmem_ld32(o_addr + c * 32, ov);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], corr_prev, ov[i]);
+                }
+                tc_fence_before();
+                mbar_arrive(o_empty + 8 * st);
+            }
+            corr_prev = corr;
+        }
+        if (ok && q < S) {
+            const float inv = 1.f / l;
+            bf16* dst = out + ((size_t)b * S + q) * ((size_t)H * HD) + (size_t)h * HD;
+#pragma unroll
+            for (int c = 0; c < HD / 8; ++c) {
+                uint4 w = make_uint4(pack_bf16x2(o[8 * c] * inv, o[8 * c + 1] * inv),
+                                     pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
+                                     pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
+                                     pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
+                *reinterpret_cast<uint4*>(dst + 8 * c) = w;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn_attn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 3-D map over [heads][rows][hd] bf16 with `rows` valid rows per head
+// (rows past them read as zero), `stride_rows` rows apart; box (64, 128, 1).
+int make_head_map(CUtensorMap* map, const void* ptr, int hd, int rows, int stride_rows, int heads) {
+    auto fn = encode_fn_attn();
+    if (!fn) return LLAMA_ERR_CUDA;
+    cuuint64_t dims[3] = {(cuuint64_t)hd, (cuuint64_t)rows, (cuuint64_t)heads};
+    cuuint64_t strides[2] = {(cuuint64_t)hd * 2, (cuuint64_t)stride_rows * hd * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+template <int HD>
+int attn_attr() {
+    static bool done = false;
+    if (!done) {
+        LLAMA_CUDA_TRY(cudaFuncSetAttribute(attn_prefill_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            ACfg<HD>::SMEM));
+        done = true;
+    }
+    return LLAMA_OK;
+}
+
+}  // namespace
+
+int attention_tc_prepare() {
+    if (!encode_fn_attn()) return LLAMA_ERR_CUDA;
+    int rc = attn_attr<128>();
+    if (rc) return rc;
+    return attn_attr<64>();
+}
+
+int launch_attention_prefill_tc(const void* q, const void* k, const void* v, void* o, int B, int H, int S, int hd,
+                                int kv_stride, int* err, cudaStream_t st) {
+    if (B <= 0 || S <= 0) return LLAMA_OK;
+    if (hd != 64 && hd != 128) return LLAMA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
+         reinterpret_cast<uintptr_t>(o)) & 15u)
+        return LLAMA_ERR_INVALID_ARG;
+    CUtensorMap mq, mk, mv;
+    int rc;
+    if ((rc = make_head_map(&mq, q, hd, S, S, B * H))) return rc;
+    if ((rc = make_head_map(&mk, k, hd, S, kv_stride, B * H))) return rc;
+    if ((rc = make_head_map(&mv, v, hd, S, kv_stride, B * H))) return rc;
+    const float scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
+    dim3 grid((S + BQ - 1) / BQ, H, B);
+    if (hd == 128) {
+        if ((rc = attn_attr<128>())) return rc;
+        attn_prefill_tc_kernel<128><<<grid, NTHREADS, ACfg<128>::SMEM, st>>>(mq, mk, mv, (bf16*)o, H, S, scale_log2,
+                                                                             err);
+    } else {
+        if ((rc = attn_attr<64>())) return rc;
+        attn_prefill_tc_kernel<64><<<grid, NTHREADS, ACfg<64>::SMEM, st>>>(mq, mk, mv, (bf16*)o, H, S, scale_log2,
+                                                                           err);
+    }
+    LLAMA_LAUNCH_CHECK();
+    return LLAMA_OK;
+}

@@ -1,5 +1,5 @@
-// Decode-side kernels: split-sequence attention over the contiguous KV cache
-// and the split-K reduction that finishes the decode GEMMs.
+// Decode-side attention: split-sequence attention over the contiguous KV
+// cache.
 //
 // Decode attention ("GQA Was Not an Original LLaMA Feature": every step
 // reads the keys and values of all previous tokens) is HBM-bound: each
@@ -68,35 +68,47 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) attn_decode_partial_kernel(
     const size_t head_off = ((size_t)b * H + h) * (size_t)kv_stride * HD;
     const T* kh = k + head_off + r * DPL;
     const T* vh = v + head_off + r * DPL;
-    // The warp walks keys jb + g (g = 0..3) with jb warp-uniform, so every
-    // lane takes part in the shuffles; a group past the end skips the update.
-    for (int jb = k_begin + warp * 4; jb < k_stop; jb += DEC_WARPS * 4) {
-        const int j = jb + g;
-        const bool valid = j < k_stop;
-        float kk[DPL], vv[DPL];
-        if (valid) {
+    // Warp w walks keys [k_begin + 64 w, k_begin + 64 w + 64) eight at a time:
+    // lane group g takes keys jb + g and jb + 4 + g, so each lane has four
+    // 16-byte-per-row loads (two K rows, two V rows) in flight per round.
+    // jb is warp-uniform, so every lane takes part in the shuffles.
+    const int seg_end = min(k_stop, k_begin + (warp + 1) * (DEC_CHUNK / DEC_WARPS));
+    for (int jb = k_begin + warp * (DEC_CHUNK / DEC_WARPS); jb < seg_end; jb += 8) {
+        const int j0 = jb + g, j1 = jb + 4 + g;
+        const bool ok0 = j0 < seg_end, ok1 = j1 < seg_end;
+        float k0[DPL], k1[DPL], x0[DPL], x1[DPL];
 #pragma unroll
-            for (int u = 0; u < VPL; ++u) {
-                load16<T>(kh + (size_t)j * HD + u * Vec16<T>::N, kk + u * Vec16<T>::N);
-                load16<T>(vh + (size_t)j * HD + u * Vec16<T>::N, vv + u * Vec16<T>::N);
+        for (int u = 0; u < VPL; ++u) {
+            if (ok0) {
+                load16<T>(kh + (size_t)j0 * HD + u * Vec16<T>::N, k0 + u * Vec16<T>::N);
+                load16<T>(vh + (size_t)j0 * HD + u * Vec16<T>::N, x0 + u * Vec16<T>::N);
             }
-        } else {
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) kk[e] = vv[e] = 0.f;
+            if (ok1) {
+                load16<T>(kh + (size_t)j1 * HD + u * Vec16<T>::N, k1 + u * Vec16<T>::N);
+                load16<T>(vh + (size_t)j1 * HD + u * Vec16<T>::N, x1 + u * Vec16<T>::N);
+            }
         }
-        float s = 0.f;
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) s = fmaf(qv[e], kk[e], s);
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        s += __shfl_xor_sync(0xffffffffu, s, 4);
-        if (valid) {
-            const float m_new = fmaxf(m, s);
+        for (int e = 0; e < DPL; ++e) {
+            s0 = fmaf(qv[e], ok0 ? k0[e] : 0.f, s0);
+            s1 = fmaf(qv[e], ok1 ? k1[e] : 0.f, s1);
+        }
+#pragma unroll
+        for (int o2 = 1; o2 < 8; o2 <<= 1) {
+            s0 += __shfl_xor_sync(0xffffffffu, s0, o2);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, o2);
+        }
+        if (!ok0) s0 = -INFINITY;
+        if (!ok1) s1 = -INFINITY;
+        const float m_new = fmaxf(m, fmaxf(s0, s1));
+        if (m_new != -INFINITY) {
             const float corr = __expf(m - m_new);
-            const float p = __expf(s - m_new);
-            l = l * corr + p;
+            const float p0 = __expf(s0 - m_new), p1 = __expf(s1 - m_new);
+            l = l * corr + p0 + p1;
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) o[e] = fmaf(o[e], corr, p * vv[e]);
+            for (int e = 0; e < DPL; ++e)
+                o[e] = fmaf(o[e], corr, fmaf(p0, ok0 ? x0[e] : 0.f, p1 * (ok1 ? x1[e] : 0.f)));
             m = m_new;
         }
     }
@@ -191,64 +203,6 @@ int launch_attention_decode(int dtype, const void* q, const void* k, const void*
     }
 #undef DEC_CASE
     return LLAMA_ERR_INVALID_ARG;
-}
-
-// ---------------------------------------------------------------------------
-// Split-K reduction of the decode GEMMs, then the epilogue.
-// partial: fp32 [splits][M][N] (M = batch rows, N = output features).
-template <typename T, int MODE>
-__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int splits, EpiArgs a) {
-    const int chunks = (MODE == EPI_SWIGLU ? a.hidden : a.N) / 32;
-    const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (idx >= (int64_t)a.M * chunks) return;
-    const int m = (int)(idx / chunks);
-    const int c = (int)(idx - (int64_t)m * chunks);
-    const size_t plane = (size_t)a.M * a.N;
-    if (MODE == EPI_SWIGLU) {
-        const int j0 = c * 32;
-        const int ng = (j0 / 128) * 256 + (j0 % 128);
-        float g[32], u[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) g[j] = u[j] = 0.f;
-        for (int s = 0; s < splits; ++s) {
-            const float* row = partial + s * plane + (size_t)m * a.N;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                g[j] += row[ng + j];
-                u[j] += row[ng + 128 + j];
-            }
-        }
-        epi_swiglu32<T>(a, m, j0, g, u);
-    } else {
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = 0.f;
-        const int n0 = c * 32;
-        for (int s = 0; s < splits; ++s) {
-            const float* row = partial + s * plane + (size_t)m * a.N + n0;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] += row[j];
-        }
-        if (MODE == EPI_QKV) epi_qkv32<T>(a, m, n0, v);
-        else if (MODE == EPI_RESID) epi_resid32(a, m, n0, v);
-        else epi_f32_32(a, m, n0, v);
-    }
-}
-
-int launch_splitk_reduce(int mode, const float* partial, int splits, const EpiArgs& a, cudaStream_t st) {
-    const int chunks = (mode == EPI_SWIGLU ? a.hidden : a.N) / 32;
-    const int64_t total = (int64_t)a.M * chunks;
-    if (total == 0) return LLAMA_OK;
-    const int blocks = (int)((total + 63) / 64);
-    switch (mode) {
-        case EPI_SWIGLU: splitk_reduce_kernel<bf16, EPI_SWIGLU><<<blocks, 64, 0, st>>>(partial, splits, a); break;
-        case EPI_QKV: splitk_reduce_kernel<bf16, EPI_QKV><<<blocks, 64, 0, st>>>(partial, splits, a); break;
-        case EPI_RESID: splitk_reduce_kernel<bf16, EPI_RESID><<<blocks, 64, 0, st>>>(partial, splits, a); break;
-        case EPI_F32: splitk_reduce_kernel<bf16, EPI_F32><<<blocks, 64, 0, st>>>(partial, splits, a); break;
-        default: return LLAMA_ERR_INVALID_ARG;
-    }
-    LLAMA_LAUNCH_CHECK();
-    return LLAMA_OK;
 }
 
 // ---------------------------------------------------------------------------

@@ -17,12 +17,14 @@
 
 #include "common.cuh"
 
-enum EpiMode { EPI_F32 = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_QKV = 3, EPI_PARTIAL = 4 };
+enum EpiMode { EPI_F32 = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_QKV = 3 };
 
 struct EpiArgs {
     int M, N;             // logical output rows (tokens) and columns
-    float* out;           // EPI_F32 / EPI_RESID: fp32 [M, ld_out]; EPI_PARTIAL: fp32 [splits][M][N]
+    float* out;           // EPI_F32 / EPI_RESID: fp32 [M, ld_out]
     int ld_out;
+    float* partial;       // decode split-K workspace: fp32 [splits][M][N]
+    int* counters;        // decode split-K arrival counters (zero between launches)
     void* act;            // EPI_SWIGLU: T [M, hidden]
     int hidden;
     void* q;              // EPI_QKV: T [B][H][S][hd]  (decode: [B][H][1][hd])

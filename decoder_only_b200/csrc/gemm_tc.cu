@@ -10,10 +10,15 @@
 //                       tile 128 x 256, fused epilogue on the output tile.
 //   decode  (swap = 1): A = weights [N, K], B = activations [batch, K]
 //                       (batch <= 32, zero-filled to 16 or 32 rows by TMA),
-//                       tile 128 x {16, 32}, split over K; fp32 partial
-//                       tiles go to a workspace and a reduction applies the
-//                       epilogue.  Weight streaming is HBM-bound: deep TMA
-//                       ring, grid sized to the SM count.
+//                       tile 128 x {16, 32}, split over K to fill the SMs.
+//                       Each split leaves its fp32 partial tile in a
+//                       workspace and bumps a per-tile counter; the CTA that
+//                       arrives last sums the partials in split order
+//                       (deterministic) and applies the epilogue, so no
+//                       second kernel runs.  Gate and up tiles of the same
+//                       128 SwiGLU units share one counter.  Weight
+//                       streaming is HBM-bound: deep TMA ring, grid sized to
+//                       the SM count.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer (one elected lane): stage ring of S slots
@@ -30,136 +35,15 @@
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "tcgen05.cuh"
 
 namespace {
+
+using namespace tc;
 
 constexpr int BM = 128;
 constexpr int BK = 64;                 // 64 bf16 = one 128-byte swizzle row
 constexpr int NTHREADS = 192;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t global_timer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait; false when this CTA is aborting (timeout here or elsewhere).
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (global_timer() - t0 > WAIT_LIMIT_NS) {
-            *abort_flag = 1;
-            atomicOr(err, LLAMA_DEVERR_TIMEOUT);
-            return false;
-        }
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-        "[%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-        : "memory");
-}
-
-// Shared-memory matrix descriptor: K-major tile, rows of 128 bytes with the
-// 128-byte swizzle, 8-row groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);   // start address
-    d |= (uint64_t)1 << 16;                      // leading byte offset (unused for this layout)
-    d |= (uint64_t)(1024 >> 4) << 32;            // stride byte offset
-    d |= (uint64_t)1 << 46;                      // descriptor version
-    d |= (uint64_t)2 << 61;                      // 128-byte swizzle
-    return d;
-}
-
-// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128, N = n.
-__host__ __device__ constexpr uint32_t idesc_bf16(int n) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accum) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
-        : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-#define TMEM_LD_X16(taddr, r)                                                                          \
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
-                 "%15}, [%16];"                                                                        \
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),  \
-                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),         \
-                   "=r"(r[13]), "=r"(r[14]), "=r"(r[15])                                               \
-                 : "r"(taddr))
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
-        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[16];
-    TMEM_LD_X16(taddr, r);
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-#pragma unroll
-    for (int i = 16; i < 32; ++i) v[i] = 0.f;
-}
-
 template <int BN>
 struct Cfg {
     static constexpr int A_BYTES = BM * BK * 2;            // 16 KB
@@ -167,7 +51,24 @@ struct Cfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = (BN >= 256) ? 4 : 8;
     static constexpr int TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;   // two accumulators, power of 2
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr int XLD = BM + 1;                                // transpose buffer row (decode)
+    static constexpr int XBUF_BYTES = (BN < 256) ? 32 * XLD * 4 : 0;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + XBUF_BYTES;
+};
+
+// Bounded barrier of the 128 epilogue threads (an mbarrier with 128
+// arrivals): false when the CTA is aborting.
+struct EpiSync {
+    uint32_t bar;
+    uint32_t phase;
+    volatile int* abort_flag;
+    int* err;
+    __device__ __forceinline__ bool sync() {
+        mbar_arrive(bar);
+        const bool ok = mbar_wait(bar, phase, abort_flag, err);
+        phase ^= 1u;
+        return ok;
+    }
 };
 
 struct TileSched {
@@ -195,7 +96,95 @@ struct TileSched {
     }
 };
 
+// Decode epilogue of one 128-feature tile (thread et owns feature
+// mb*128 + et for every batch row): write the split's partial, let the last
+// split to arrive finish the tile.  Runs on the 128 epilogue threads only.
 template <int BN, int MODE>
+__device__ __forceinline__ bool epilogue_swap(const EpiArgs& ep, const TileSched& ts, int mb, int sp, int et,
+                                              const float (&v)[32], float* xbuf, volatile int* last_flag,
+                                              EpiSync& es) {
+    constexpr bool PAIR = (MODE == EPI_SWIGLU);      // gate tile 2j and up tile 2j+1 finish together
+    const int n = mb * BM + et;
+    const int M = ep.M, N = ep.N;
+    const bool direct = (ts.splits == 1) && !PAIR;
+    if (!direct) {
+        if (n < N) {
+            float* dst = ep.partial + (size_t)sp * M * N + n;
+#pragma unroll
+            for (int b = 0; b < BN; ++b)
+                if (b < M) dst[(size_t)b * N] = v[b];
+        }
+        __threadfence();
+        if (!es.sync()) return false;
+        if (et == 0) {
+            const int cidx = PAIR ? (mb >> 1) : mb;
+            const int target = PAIR ? 2 * ts.splits : ts.splits;
+            const int prev = atomicAdd(ep.counters + cidx, 1);
+            const int last = (prev == target - 1);
+            if (last) ep.counters[cidx] = 0;     // ready for the next launch
+            *last_flag = last;
+        }
+        if (!es.sync()) return false;
+        const int last = *last_flag;
+        if (!es.sync()) return false;            // everyone has read the flag
+        if (!last) return true;
+        __threadfence();
+    }
+    if constexpr (PAIR) {
+        // hidden units 128j + et from gate row 256j + et and up row 256j + 128 + et
+        const int j = mb >> 1;
+        const float* pg = ep.partial + 256 * j + et;
+        const float* pu = pg + 128;
+        for (int b = 0; b < M; ++b) {
+            float g = 0.f, u = 0.f;
+            for (int s = 0; s < ts.splits; ++s) {
+                g += __ldcg(pg + (size_t)s * M * N + (size_t)b * N);
+                u += __ldcg(pu + (size_t)s * M * N + (size_t)b * N);
+            }
+            reinterpret_cast<bf16*>(ep.act)[(size_t)b * ep.hidden + 128 * j + et] = __float2bfloat16_rn(silu_f(g) * u);
+        }
+    } else {
+        float sum[32];
+#pragma unroll
+        for (int b = 0; b < 32; ++b) sum[b] = direct ? v[b] : 0.f;
+        if (!direct && n < N) {
+            for (int s = 0; s < ts.splits; ++s) {
+                const float* p = ep.partial + (size_t)s * M * N + n;
+#pragma unroll
+                for (int b = 0; b < BN; ++b)
+                    if (b < M) sum[b] += __ldcg(p + (size_t)b * N);
+            }
+        }
+        if constexpr (MODE == EPI_RESID || MODE == EPI_F32) {
+            if (n < N) {
+#pragma unroll
+                for (int b = 0; b < BN; ++b) {
+                    if (b < M) {
+                        float* o = ep.out + (size_t)b * ep.ld_out + n;
+                        if constexpr (MODE == EPI_RESID) *o += sum[b];
+                        else *o = sum[b];
+                    }
+                }
+            }
+        } else {
+            // Q/K/V: 32-feature chunks of one token row through shared memory
+#pragma unroll
+            for (int b = 0; b < BN; ++b) xbuf[b * Cfg<BN>::XLD + et] = sum[b];
+            if (!es.sync()) return false;
+            if (et < 4 * M) {
+                const int b = et >> 2, c = et & 3;
+                float w[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w[i] = xbuf[b * Cfg<BN>::XLD + c * 32 + i];
+                epi_qkv32<bf16>(ep, b, mb * BM + c * 32, w);
+            }
+            if (!es.sync()) return false;
+        }
+    }
+    return true;
+}
+
+template <int BN, int MODE, bool SWAP>
 __global__ void __launch_bounds__(NTHREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TileSched ts,
                    EpiArgs ep, int* err) {
@@ -213,6 +202,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tempty_bar = tfull_bar + 16;                 // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::STAGES * C::STAGE_BYTES + 16 * C::STAGES + 32);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+    const uint32_t epi_bar_addr = tempty_bar + 32;                  // 128-thread epilogue barrier
+    float* xbuf = reinterpret_cast<float*>(gbase + C::STAGES * C::STAGE_BYTES + 256);   // [32][XLD] (decode)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -225,6 +217,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(tfull_bar + 8 * i, 1);
             mbar_init(tempty_bar + 8 * i, 128);
         }
+        mbar_init(epi_bar_addr, 128);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
@@ -325,6 +318,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         int acc = 0;
         uint32_t acc_phase = 0;
+        EpiSync es{epi_bar_addr, 0u, abort_flag, err};
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
             int mb, nb, sp, kb0, kb1;
             ts.get(t, mb, nb, sp, kb0, kb1);
@@ -332,17 +326,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc_fence_after();
             const uint32_t tacc = tmem_base + lane_addr + (uint32_t)(acc * BN);
             const int row = mb * BM + quarter * 32 + lane;   // row of operand A
-            if constexpr (MODE == EPI_PARTIAL) {
-                // row = output feature n; columns = batch rows
+            if constexpr (SWAP) {
+                // row = output feature; TMEM columns = batch rows
                 float v[32];
                 if constexpr (BN == 16) tmem_ld16(tacc, v);
                 else tmem_ld32(tacc, v);
-                if (row < ep.N) {
-                    float* dst = ep.out + (size_t)sp * ep.M * ep.N + row;
-#pragma unroll
-                    for (int b = 0; b < BN; ++b)
-                        if (b < ep.M) dst[(size_t)b * ep.N] = v[b];
+                tc_fence_before();
+                mbar_arrive(tempty_bar + 8 * acc);       // accumulator free for the next tile
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
                 }
+                if (!epilogue_swap<BN, MODE>(ep, ts, mb, sp, threadIdx.x - 64, v, xbuf, last_flag, es)) break;
+                continue;
             } else if constexpr (MODE == EPI_SWIGLU) {
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
@@ -422,26 +418,26 @@ int num_sms() {
     return n;
 }
 
-template <int BN, int MODE>
+template <int BN, int MODE, bool SWAP>
 int ensure_attr() {
     static bool attr = false;
     if (!attr) {
-        LLAMA_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            Cfg<BN>::SMEM));
+        LLAMA_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, MODE, SWAP>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::SMEM));
         attr = true;
     }
     return LLAMA_OK;
 }
 
-template <int BN, int MODE>
+template <int BN, int MODE, bool SWAP>
 int run(const CUtensorMap& ma, const CUtensorMap& mb, const TileSched& ts, const EpiArgs& a, int* err,
         cudaStream_t st) {
     using C = Cfg<BN>;
-    int rc = ensure_attr<BN, MODE>();
+    int rc = ensure_attr<BN, MODE, SWAP>();
     if (rc) return rc;
     const int tiles = ts.m_blocks * ts.n_blocks * ts.splits;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    gemm_tc_kernel<BN, MODE><<<grid, NTHREADS, C::SMEM, st>>>(ma, mb, ts, a, err);
+    gemm_tc_kernel<BN, MODE, SWAP><<<grid, NTHREADS, C::SMEM, st>>>(ma, mb, ts, a, err);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }
@@ -452,12 +448,18 @@ int gemm_tc_prepare() {
     if (!encode_fn()) return LLAMA_ERR_CUDA;
     num_sms();
     int rc;
-    if ((rc = ensure_attr<256, EPI_F32>())) return rc;
-    if ((rc = ensure_attr<256, EPI_RESID>())) return rc;
-    if ((rc = ensure_attr<256, EPI_SWIGLU>())) return rc;
-    if ((rc = ensure_attr<256, EPI_QKV>())) return rc;
-    if ((rc = ensure_attr<16, EPI_PARTIAL>())) return rc;
-    return ensure_attr<32, EPI_PARTIAL>();
+    if ((rc = ensure_attr<256, EPI_F32, false>())) return rc;
+    if ((rc = ensure_attr<256, EPI_RESID, false>())) return rc;
+    if ((rc = ensure_attr<256, EPI_SWIGLU, false>())) return rc;
+    if ((rc = ensure_attr<256, EPI_QKV, false>())) return rc;
+    if ((rc = ensure_attr<16, EPI_F32, true>())) return rc;
+    if ((rc = ensure_attr<16, EPI_RESID, true>())) return rc;
+    if ((rc = ensure_attr<16, EPI_SWIGLU, true>())) return rc;
+    if ((rc = ensure_attr<16, EPI_QKV, true>())) return rc;
+    if ((rc = ensure_attr<32, EPI_F32, true>())) return rc;
+    if ((rc = ensure_attr<32, EPI_RESID, true>())) return rc;
+    if ((rc = ensure_attr<32, EPI_SWIGLU, true>())) return rc;
+    return ensure_attr<32, EPI_QKV, true>();
 }
 
 int gemm_tc_pick_splits(int rowsA, int K) {
@@ -489,8 +491,10 @@ int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaSt
     TileSched ts;
     ts.kb_total = g.K / BK;
     ts.group = 16;
-    if (mode == EPI_PARTIAL) {
+    if (g.swap) {
         if (g.rowsB > 32) return LLAMA_ERR_INVALID_ARG;
+        if ((g.splits > 1 || mode == EPI_SWIGLU) && (!a.partial || !a.counters)) return LLAMA_ERR_INVALID_ARG;
+        if (g.rowsA % BM != 0) return LLAMA_ERR_INVALID_ARG;   // whole 128-feature tiles
         const int bn = g.rowsB <= 16 ? 16 : 32;
         ts.m_blocks = (g.rowsA + BM - 1) / BM;
         ts.n_blocks = 1;
@@ -503,8 +507,17 @@ int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaSt
         if (rc) return rc;
         rc = make_map(&mb, g.B, g.rowsB, g.K, bn);
         if (rc) return rc;
-        if (bn == 16) return run<16, EPI_PARTIAL>(ma, mb, ts, a, err, st);
-        return run<32, EPI_PARTIAL>(ma, mb, ts, a, err, st);
+#define SWAP_CASE(BNV)                                                      \
+    switch (mode) {                                                         \
+        case EPI_F32: return run<BNV, EPI_F32, true>(ma, mb, ts, a, err, st);       \
+        case EPI_RESID: return run<BNV, EPI_RESID, true>(ma, mb, ts, a, err, st);   \
+        case EPI_SWIGLU: return run<BNV, EPI_SWIGLU, true>(ma, mb, ts, a, err, st); \
+        case EPI_QKV: return run<BNV, EPI_QKV, true>(ma, mb, ts, a, err, st);       \
+        default: return LLAMA_ERR_INVALID_ARG;                              \
+    }
+        if (bn == 16) SWAP_CASE(16);
+        SWAP_CASE(32);
+#undef SWAP_CASE
     }
     constexpr int BN = 256;
     ts.m_blocks = (g.rowsA + BM - 1) / BM;
@@ -517,10 +530,10 @@ int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaSt
     rc = make_map(&mb, g.B, g.rowsB, g.K, BN);
     if (rc) return rc;
     switch (mode) {
-        case EPI_F32: return run<BN, EPI_F32>(ma, mb, ts, a, err, st);
-        case EPI_RESID: return run<BN, EPI_RESID>(ma, mb, ts, a, err, st);
-        case EPI_SWIGLU: return run<BN, EPI_SWIGLU>(ma, mb, ts, a, err, st);
-        case EPI_QKV: return run<BN, EPI_QKV>(ma, mb, ts, a, err, st);
+        case EPI_F32: return run<BN, EPI_F32, false>(ma, mb, ts, a, err, st);
+        case EPI_RESID: return run<BN, EPI_RESID, false>(ma, mb, ts, a, err, st);
+        case EPI_SWIGLU: return run<BN, EPI_SWIGLU, false>(ma, mb, ts, a, err, st);
+        case EPI_QKV: return run<BN, EPI_QKV, false>(ma, mb, ts, a, err, st);
         default: return LLAMA_ERR_INVALID_ARG;
     }
 }

@@ -20,6 +20,10 @@ int launch_rmsnorm(int dtype, const float* x, const float* g, void* y, int rows,
 int launch_embed(int dtype, const int32_t* tok, const void* E, float* x, int rows, int d, int vocab, int* err,
                  cudaStream_t st);
 int launch_argmax(const float* logits, int rows, int n, int64_t ld, int32_t* out, cudaStream_t st);
+int argmax_split_chunks(int n);
+// part: int2 [rows][argmax_split_chunks(n)]; counters: int [rows], zero between launches
+int launch_argmax_split(const float* logits, int rows, int n, int64_t ld, int32_t* out, int2* part, int* counters,
+                        cudaStream_t st);
 
 // simt.cu  (fp32 storage path and shared epilogue passes)
 int launch_gemm_simt(int dtype, const void* A, const void* W, float* C, int M, int N, int K, int accumulate,
@@ -29,12 +33,16 @@ int launch_attention_prefill_simt(int dtype, const void* q, const void* k, const
                                   int H, int S, int hd, int kv_stride, cudaStream_t st);
 int attention_prepare();  // sets kernel attributes; call before any stream capture
 
+// attn_tc.cu  (bf16 tcgen05 causal flash attention, head_dim 64 or 128)
+int launch_attention_prefill_tc(const void* q, const void* k, const void* v, void* o, int B, int H, int S, int hd,
+                                int kv_stride, int* err, cudaStream_t st);
+int attention_tc_prepare();
+
 // decode.cu
 uint64_t attention_decode_work_bytes(int B, int H, int max_len, int hd);
 int launch_attention_decode(int dtype, const void* q, const void* k, const void* v, void* o, int B, int H,
                             int len, const int* d_len_minus1, int hd, int kv_stride, float* work,
                             cudaStream_t st);
-int launch_splitk_reduce(int mode, const float* partial, int splits, const EpiArgs& a, cudaStream_t st);
 
 // gemm_tc.cu  (bf16 tcgen05 GEMM)
 struct TcGemm {
@@ -42,7 +50,7 @@ struct TcGemm {
     const void* A;  // bf16 [rowsA, K]
     const void* B;  // bf16 [rowsB, K]
     int rowsA, rowsB, K;
-    int splits;     // split-K factor (EPI_PARTIAL only)
+    int splits;     // split-K factor (decode only)
     int swap;       // 0: A = tokens, B = weights; 1: A = weights, B = tokens (decode)
 };
 int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaStream_t st);

@@ -107,6 +107,7 @@ namespace {
 constexpr uint32_t TID_EMBED = 1, TID_HEAD = 2;
 inline uint32_t layer_tid(int l, int m) { return 16u + 8u * (uint32_t)l + (uint32_t)m; }
 constexpr int MAX_DEC_SPLITS = 16;
+constexpr int MAX_COUNTERS = 4096;
 
 struct Layer {
     void *wqkv, *wo, *wgu, *wd;
@@ -147,6 +148,9 @@ struct llama_model {
     float* logits_dec;       // [max_batch, vocab]
     float* partial;          // split-K partials
     size_t partial_elems;
+    int* counters;           // split-K arrival counters (zero between launches)
+    int2* amax_part;         // greedy-choice chunk results [max_batch][chunks]
+    int* amax_cnt;           // and their arrival counters [max_batch]
     float* attn_work;
     uint64_t attn_work_bytes;
     int32_t* tok_cur;        // decode input tokens; argmax writes the next ones here
@@ -233,6 +237,9 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     float* logits_dec = (float*)take((size_t)c->max_batch * V * 4);
     const size_t pmax = (size_t)MAX_DEC_SPLITS * c->max_batch * std::max(cmax, V);
     float* partial = (float*)take(c->dtype == LLAMA_BF16 ? pmax * 4 : 0);
+    int* counters = (int*)take(MAX_COUNTERS * 4);
+    int2* amax_part = (int2*)take((size_t)c->max_batch * argmax_split_chunks(c->vocab) * sizeof(int2));
+    int* amax_cnt = (int*)take((size_t)c->max_batch * 4);
     const uint64_t awb = attention_decode_work_bytes(c->max_batch, c->n_heads, c->max_seq, c->head_dim);
     float* attn_work = (float*)take(awb);
     int32_t* tok_cur = (int32_t*)take((size_t)c->max_batch * 4);
@@ -255,6 +262,9 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
         m->logits_dec = logits_dec;
         m->partial = partial;
         m->partial_elems = pmax;
+        m->counters = counters;
+        m->amax_part = amax_part;
+        m->amax_cnt = amax_cnt;
         m->attn_work = attn_work;
         m->attn_work_bytes = awb;
         m->tok_cur = tok_cur;
@@ -333,15 +343,10 @@ int project(llama_model* m, const char* name, int mode, const void* A, const voi
         g.splits = splits;
         g.swap = 1;
         EpiArgs pa = a;
-        pa.out = m->partial;
-        {
-            prof::Scope ps(st, region, in_bytes, flops);
-            int rc = launch_gemm_tc(g, EPI_PARTIAL, pa, m->d_err, st);
-            if (rc) return rc;
-        }
-        snprintf(region, sizeof(region), "decode_reduce_%s", name);
-        prof::Scope ps(st, region, out_bytes(mode, M, N, m->esz), 0.0);
-        return launch_splitk_reduce(mode, m->partial, splits, a, st);
+        pa.partial = m->partial;
+        pa.counters = m->counters;
+        prof::Scope ps(st, region, in_bytes + out_bytes(mode, M, N, m->esz), flops);
+        return launch_gemm_tc(g, mode, pa, m->d_err, st);
     }
     // fp32 storage: SIMT GEMM
     prof::Scope ps(st, region, in_bytes + out_bytes(mode, M, N, m->esz), flops);
@@ -382,9 +387,13 @@ int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
                 return rc;
         } else {
             prof::Scope ps(st, "prefill_attention", 4.0 * n * d * m->esz, 2.0 * B * (double)S * (S + 1) * d);
-            if ((rc = launch_attention_prefill_simt(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, S,
-                                                    c.head_dim, c.max_seq, st)))
-                return rc;
+            if (dt == LLAMA_BF16)
+                rc = launch_attention_prefill_tc(m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, S,
+                                                 c.head_dim, c.max_seq, m->d_err, st);
+            else
+                rc = launch_attention_prefill_simt(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, S,
+                                                   c.head_dim, c.max_seq, st);
+            if (rc) return rc;
         }
         EpiArgs ra = base_args(m, n, d);
         ra.out = m->trunk;
@@ -430,7 +439,8 @@ int decode_body(llama_model* m, cudaStream_t st) {
     if ((rc = run_blocks(m, m->B, 1, true, st))) return rc;
     if ((rc = run_head(m, m->trunk, m->B, m->logits_dec, true, st))) return rc;
     prof::Scope ps(st, "decode_argmax", (double)m->B * c.vocab * 4, 0.0);
-    if ((rc = launch_argmax(m->logits_dec, m->B, c.vocab, c.vocab, m->tok_cur, st))) return rc;
+    if ((rc = launch_argmax_split(m->logits_dec, m->B, c.vocab, c.vocab, m->tok_cur, m->amax_part, m->amax_cnt, st)))
+        return rc;
     pos_advance_kernel<<<1, 1, 0, st>>>(m->d_pos);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
@@ -577,12 +587,14 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
         llama_free(m);
         return LLAMA_ERR_CUDA;
     }
-    if (cudaMemsetAsync(m->d_pos, 0, 256, st) != cudaSuccess) {
+    if (cudaMemsetAsync(m->counters, 0, MAX_COUNTERS * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(m->amax_cnt, 0, (size_t)cfg->max_batch * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(m->d_pos, 0, 256, st) != cudaSuccess) {
         llama_free(m);
         return LLAMA_ERR_CUDA;
     }
     pick_decode_splits(m);
-    if ((rc = gemm_tc_prepare()) || (rc = attention_prepare())) {
+    if ((rc = gemm_tc_prepare()) || (rc = attention_prepare()) || (rc = attention_tc_prepare())) {
         llama_free(m);
         return rc;
     }
@@ -612,8 +624,8 @@ int llama_prefill(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S,
         // greedy choice at each sequence's last position: the input of the
         // first decode step when llama_generate is given no tokens
         prof::Scope ps(st, "prefill_argmax", (double)B * m->cfg.vocab * 4, 0.0);
-        if ((rc = launch_argmax(d_logits + (size_t)(S - 1) * m->cfg.vocab, B, m->cfg.vocab,
-                                (int64_t)S * m->cfg.vocab, m->tok_cur, st)))
+        if ((rc = launch_argmax_split(d_logits + (size_t)(S - 1) * m->cfg.vocab, B, m->cfg.vocab,
+                                      (int64_t)S * m->cfg.vocab, m->tok_cur, m->amax_part, m->amax_cnt, st)))
             return rc;
     }
     pos_set_kernel<<<1, 1, 0, st>>>(m->d_pos, S);
@@ -699,7 +711,9 @@ int llama_complete(llama_model* m, const int32_t* h_tokens, int32_t B, int32_t S
                                          (size_t)S * c.d_model * 4, (size_t)c.d_model * 4, B,
                                          cudaMemcpyDeviceToDevice, st));
         if ((rc = run_head(m, m->trunk_last, B, m->logits_dec, true, st))) return rc;
-        if ((rc = launch_argmax(m->logits_dec, B, c.vocab, c.vocab, m->tok_cur, st))) return rc;
+        if ((rc = launch_argmax_split(m->logits_dec, B, c.vocab, c.vocab, m->tok_cur, m->amax_part, m->amax_cnt,
+                                      st)))
+            return rc;
     }
     if ((rc = llama_generate(m, nullptr, n_steps, m->gen_out, stream))) return rc;
     LLAMA_CUDA_TRY(cudaMemcpyAsync(h_out, m->gen_out, (size_t)n_steps * B * 4, cudaMemcpyDeviceToHost, st));
@@ -790,9 +804,14 @@ int llama_op_gemm(int32_t dtype, const void* d_A, const void* d_W, float* d_C, i
 int llama_op_attention_prefill(int32_t dtype, const void* d_q, const void* d_k, const void* d_v, void* d_o,
                                int32_t B, int32_t H, int32_t S, int32_t head_dim, int32_t kv_stride, void* stream) {
     if (!d_q || !d_k || !d_v || !d_o || B <= 0 || H <= 0 || S <= 0 || kv_stride < S) return LLAMA_ERR_INVALID_ARG;
-    if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
-    return launch_attention_prefill_simt(dtype, d_q, d_k, d_v, d_o, B, H, S, head_dim, kv_stride,
-                                         (cudaStream_t)stream);
+    if (dtype == LLAMA_F32)
+        return launch_attention_prefill_simt(dtype, d_q, d_k, d_v, d_o, B, H, S, head_dim, kv_stride,
+                                             (cudaStream_t)stream);
+    if (dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+    int* err = nullptr;
+    int rc = op_error_word(&err);
+    if (rc) return rc;
+    return launch_attention_prefill_tc(d_q, d_k, d_v, d_o, B, H, S, head_dim, kv_stride, err, (cudaStream_t)stream);
 }
 
 uint64_t llama_op_attention_decode_work_bytes(int32_t B, int32_t H, int32_t max_len, int32_t head_dim) {

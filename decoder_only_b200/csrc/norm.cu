@@ -151,3 +151,85 @@ int launch_argmax(const float* logits, int rows, int n, int64_t ld, int32_t* out
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }
+
+// Greedy choice over long rows: the row is cut into chunks of AMX_CHUNK
+// logits, one CTA each; every CTA leaves its (max, lowest index) in the
+// workspace and bumps the row's counter; the CTA that arrives last merges
+// the chunks in index order (so ties still go to the lowest id) and resets
+// the counter for the next launch.
+constexpr int AMX_CHUNK = 2048;
+
+__device__ __forceinline__ bool amx_better(float v, int i, float bv, int bi) {
+    return v > bv || (v == bv && i < bi);
+}
+
+__global__ void __launch_bounds__(256) argmax_split_kernel(const float* __restrict__ logits, int n, int64_t ld,
+                                                           int32_t* __restrict__ out, int2* __restrict__ part,
+                                                           int* __restrict__ counters, int chunks) {
+    const int r = blockIdx.y, c = blockIdx.x;
+    const float* p = logits + (size_t)r * ld;
+    const int i0 = c * AMX_CHUNK, i1 = min(n, i0 + AMX_CHUNK);
+    float best = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
+        const float v = p[i];
+        if (amx_better(v, i, best, bi)) {
+            best = v;
+            bi = i;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (amx_better(ov, oi, best, bi)) {
+            best = ov;
+            bi = oi;
+        }
+    }
+    __shared__ float sb[8];
+    __shared__ int si[8];
+    __shared__ int last;
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    if (l == 0) {
+        sb[w] = best;
+        si[w] = bi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int k = 1; k < (int)(blockDim.x >> 5); ++k)
+            if (amx_better(sb[k], si[k], best, bi)) {
+                best = sb[k];
+                bi = si[k];
+            }
+        part[(size_t)r * chunks + c] = make_int2(__float_as_int(best), bi);
+        __threadfence();
+        const int prev = atomicAdd(counters + r, 1);
+        last = (prev == chunks - 1);
+        if (last) {
+            counters[r] = 0;
+            __threadfence();
+            float fb = -INFINITY;
+            int fi = 0x7fffffff;
+            for (int k = 0; k < chunks; ++k) {
+                const int2 e = __ldcg(part + (size_t)r * chunks + k);
+                if (amx_better(__int_as_float(e.x), e.y, fb, fi)) {
+                    fb = __int_as_float(e.x);
+                    fi = e.y;
+                }
+            }
+            out[r] = (fi == 0x7fffffff) ? 0 : fi;
+        }
+    }
+}
+
+int argmax_split_chunks(int n) { return (n + AMX_CHUNK - 1) / AMX_CHUNK; }
+
+int launch_argmax_split(const float* logits, int rows, int n, int64_t ld, int32_t* out, int2* part, int* counters,
+                        cudaStream_t st) {
+    if (rows <= 0) return LLAMA_OK;
+    const int chunks = argmax_split_chunks(n);
+    argmax_split_kernel<<<dim3(chunks, rows), 256, 0, st>>>(logits, n, ld, out, part, counters, chunks);
+    LLAMA_LAUNCH_CHECK();
+    return LLAMA_OK;
+}

@@ -1,4 +1,4 @@
-// SIMT kernels: the fp32 GEMM of the fp32 workload, epilogue passes over an
+// SIMT kernels of the fp32 workload: the fp32 GEMM, epilogue passes over an
 // fp32 GEMM result, and a CUDA-core causal flash attention.
 //
 // The fp32 workload is compared at 1e-4 RMS, which rules out TF32 tensor
@@ -242,9 +242,6 @@ static size_t attn_simt_smem() {
 
 int attention_prepare() {
     int rc;
-    if ((rc = attn_simt_attr<bf16, 128>(attn_simt_smem<bf16, 128>()))) return rc;
-    if ((rc = attn_simt_attr<bf16, 64>(attn_simt_smem<bf16, 64>()))) return rc;
-    if ((rc = attn_simt_attr<bf16, 32>(attn_simt_smem<bf16, 32>()))) return rc;
     if ((rc = attn_simt_attr<float, 128>(attn_simt_smem<float, 128>()))) return rc;
     if ((rc = attn_simt_attr<float, 64>(attn_simt_smem<float, 64>()))) return rc;
     return attn_simt_attr<float, 32>(attn_simt_smem<float, 32>());
@@ -266,14 +263,9 @@ static int launch_attn_simt_t(const void* q, const void* k, const void* v, void*
 int launch_attention_prefill_simt(int dtype, const void* q, const void* k, const void* v, void* o, int B,
                                   int H, int S, int hd, int kv_stride, cudaStream_t st) {
     if (B <= 0 || S <= 0) return LLAMA_OK;
-    if (dtype == LLAMA_BF16) {
-        if (hd == 128) return launch_attn_simt_t<bf16, 128>(q, k, v, o, B, H, S, kv_stride, st);
-        if (hd == 64) return launch_attn_simt_t<bf16, 64>(q, k, v, o, B, H, S, kv_stride, st);
-        if (hd == 32) return launch_attn_simt_t<bf16, 32>(q, k, v, o, B, H, S, kv_stride, st);
-    } else {
-        if (hd == 128) return launch_attn_simt_t<float, 128>(q, k, v, o, B, H, S, kv_stride, st);
-        if (hd == 64) return launch_attn_simt_t<float, 64>(q, k, v, o, B, H, S, kv_stride, st);
-        if (hd == 32) return launch_attn_simt_t<float, 32>(q, k, v, o, B, H, S, kv_stride, st);
-    }
+    if (dtype != LLAMA_F32) return LLAMA_ERR_INVALID_ARG;   // bf16 runs on the tensor cores (attn_tc.cu)
+    if (hd == 128) return launch_attn_simt_t<float, 128>(q, k, v, o, B, H, S, kv_stride, st);
+    if (hd == 64) return launch_attn_simt_t<float, 64>(q, k, v, o, B, H, S, kv_stride, st);
+    if (hd == 32) return launch_attn_simt_t<float, 32>(q, k, v, o, B, H, S, kv_stride, st);
     return LLAMA_ERR_INVALID_ARG;
 }
