@@ -96,9 +96,10 @@ struct TileSched {
     }
 };
 
-// Decode epilogue of one 128-feature tile (thread et owns feature
-// mb*128 + et for every batch row): write the split's partial, let the last
-// split to arrive finish the tile.  Runs on the 128 epilogue threads only.
+// Decode epilogue of one 128-feature tile (et = the TMEM lane the thread
+// read, so it owns feature mb*128 + et for every batch row): write the
+// split's partial, let the last split to arrive finish the tile.  Runs on
+// the 128 epilogue threads only.
 template <int BN, int MODE>
 __device__ __forceinline__ bool epilogue_swap(const EpiArgs& ep, const TileSched& ts, int mb, int sp, int et,
                                               const float (&v)[32], float* xbuf, volatile int* last_flag,
@@ -337,7 +338,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     acc = 0;
                     acc_phase ^= 1u;
                 }
-                if (!epilogue_swap<BN, MODE>(ep, ts, mb, sp, threadIdx.x - 64, v, xbuf, last_flag, es)) break;
+                // feature within the tile = the TMEM lane this thread read
+                if (!epilogue_swap<BN, MODE>(ep, ts, mb, sp, quarter * 32 + lane, v, xbuf, last_flag, es)) break;
                 continue;
             } else if constexpr (MODE == EPI_SWIGLU) {
 #pragma unroll 1
