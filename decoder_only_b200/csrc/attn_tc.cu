@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int q0 = qt * BQ;
     const int n_kv = qt + 1;                              // key tiles 0..qt (causal)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -115,6 +116,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();   // Q, K, V come from the projection kernel before this one
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
@@ -384,12 +386,12 @@ int launch_attention_prefill_tc(const void* q, const void* k, const void* v, voi
     dim3 grid((S + BQ - 1) / BQ, H, B);
     if (hd == 128) {
         if ((rc = attn_attr<128>())) return rc;
-        attn_prefill_tc_kernel<128><<<grid, NTHREADS, ACfg<128>::SMEM, st>>>(mq, mk, mv, (bf16*)o, H, S, scale_log2,
-                                                                             err);
+        launch_pdl(attn_prefill_tc_kernel<128>, grid, dim3(NTHREADS), ACfg<128>::SMEM, st, mq, mk, mv, (bf16*)o, H, S,
+                   scale_log2, err);
     } else {
         if ((rc = attn_attr<64>())) return rc;
-        attn_prefill_tc_kernel<64><<<grid, NTHREADS, ACfg<64>::SMEM, st>>>(mq, mk, mv, (bf16*)o, H, S, scale_log2,
-                                                                           err);
+        launch_pdl(attn_prefill_tc_kernel<64>, grid, dim3(NTHREADS), ACfg<64>::SMEM, st, mq, mk, mv, (bf16*)o, H, S,
+                   scale_log2, err);
     }
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;

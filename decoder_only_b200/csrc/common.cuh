@@ -26,6 +26,34 @@ void llama_count_launches(int64_t n);
         llama_count_launches(1);                           \
     } while (0)
 
+// Programmatic dependent launch.  Kernels on the hot path are launched with
+// programmatic stream serialisation: each one lets its successor launch
+// early (pdl_launch_dependents) and waits for its predecessor's memory
+// (pdl_wait) only before it reads or writes data the predecessor touches.
+// Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+extern bool g_llama_pdl;   // launch with the attribute (default on; LLAMA_B200_NO_PDL=1 turns it off)
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = g_llama_pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Device error word values (sticky, set by bounded waits)
 #define LLAMA_DEVERR_TIMEOUT 1
 

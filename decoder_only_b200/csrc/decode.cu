@@ -44,6 +44,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) attn_decode_partial_kernel(
     const int* __restrict__ d_len_minus1, int kv_stride, float scale, float* __restrict__ work, int n_chunks) {
     constexpr int DPL = HD / 8;                 // dims per lane
     constexpr int VPL = DPL / Vec16<T>::N;      // 16-byte loads per lane per row
+    pdl_launch_dependents();
+    pdl_wait();
     const int len = d_len_minus1 ? (*d_len_minus1 + 1) : len_static;
     const int chunk = blockIdx.x;
     const int bh = blockIdx.y;                  // b*H + h
@@ -147,6 +149,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) attn_decode_partial_kernel(
 template <typename T, int HD>
 __global__ void attn_decode_combine_kernel(const float* __restrict__ work, int n_chunks, int len_static,
                                            const int* __restrict__ d_len_minus1, int H, T* __restrict__ o) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int len = d_len_minus1 ? (*d_len_minus1 + 1) : len_static;
     const int used = min(n_chunks, (len + DEC_CHUNK - 1) / DEC_CHUNK);
     const int bh = blockIdx.x;
@@ -179,11 +183,11 @@ static int launch_dec_t(const void* q, const void* k, const void* v, void* o, in
     const int grid_len = d_len_minus1 ? kv_stride : len;
     const int n_chunks = (grid_len + DEC_CHUNK - 1) / DEC_CHUNK;
     dim3 grid(n_chunks, B * H);
-    attn_decode_partial_kernel<T, HD><<<grid, DEC_WARPS * 32, 0, st>>>(
-        (const T*)q, (const T*)k, (const T*)v, H, len, d_len_minus1, kv_stride, 1.0f / sqrtf((float)HD), work,
-        n_chunks);
+    launch_pdl(attn_decode_partial_kernel<T, HD>, grid, dim3(DEC_WARPS * 32), 0, st, (const T*)q, (const T*)k,
+               (const T*)v, H, len, d_len_minus1, kv_stride, 1.0f / sqrtf((float)HD), work, n_chunks);
     LLAMA_LAUNCH_CHECK();
-    attn_decode_combine_kernel<T, HD><<<B * H, HD, 0, st>>>(work, n_chunks, len, d_len_minus1, H, (T*)o);
+    launch_pdl(attn_decode_combine_kernel<T, HD>, dim3(B * H), dim3(HD), 0, st, (const float*)work, n_chunks, len,
+               d_len_minus1, H, (T*)o);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }

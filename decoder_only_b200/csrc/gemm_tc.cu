@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     float* xbuf = reinterpret_cast<float*>(gbase + C::STAGES * C::STAGE_BYTES + 256);   // [32][XLD] (decode)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -238,22 +239,50 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
+        // The weight operand (A in decode, B in prefill) does not depend on
+        // the kernels before this one: the weight tiles of the first stages
+        // are requested before waiting for the predecessor, the activation
+        // tiles after it.
         if (lane == 0) {
+            const CUtensorMap* w_map = SWAP ? &tmA : &tmB;
+            const CUtensorMap* x_map = SWAP ? &tmB : &tmA;
+            const uint32_t w_base = SWAP ? sA : sB;
+            const uint32_t x_base = SWAP ? sB : sA;
+            const int w_bytes = SWAP ? C::A_BYTES : C::B_BYTES;
+            const int x_bytes = SWAP ? C::B_BYTES : C::A_BYTES;
             int stage = 0;
             uint32_t phase = 0;
             uint32_t filled = 0, fill_phase = 0;   // per-stage: filled at least once / parity of last fill
             bool ok = true;
+            int pre = 0;                           // k-blocks of the first tile whose weights are in flight
+            if ((int)blockIdx.x < n_tiles) {
+                int mb, nb, sp, kb0, kb1;
+                ts.get(blockIdx.x, mb, nb, sp, kb0, kb1);
+                pre = min(C::STAGES, kb1 - kb0);
+                const int w_row = SWAP ? mb * BM : nb * BN;
+                for (int i = 0; i < pre; ++i) {    // fresh ring: every stage starts empty
+                    mbar_expect_tx(full_bar + 8 * i, C::STAGE_BYTES);
+                    tma_load_2d(w_base + i * w_bytes, w_map, full_bar + 8 * i, (kb0 + i) * BK, w_row);
+                    filled |= 1u << i;
+                }
+            }
+            pdl_wait();
+            int it = 0;
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
                 int mb, nb, sp, kb0, kb1;
                 ts.get(t, mb, nb, sp, kb0, kb1);
-                for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!mbar_wait(empty_bar + 8 * stage, phase ^ 1u, abort_flag, err)) {
-                        ok = false;
-                        break;
+                const int w_row = SWAP ? mb * BM : nb * BN;
+                const int x_row = SWAP ? nb * BN : mb * BM;
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    if (it >= pre) {
+                        if (!mbar_wait(empty_bar + 8 * stage, phase ^ 1u, abort_flag, err)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_expect_tx(full_bar + 8 * stage, C::STAGE_BYTES);
+                        tma_load_2d(w_base + stage * w_bytes, w_map, full_bar + 8 * stage, kb * BK, w_row);
                     }
-                    mbar_expect_tx(full_bar + 8 * stage, C::STAGE_BYTES);
-                    tma_load_2d(sA + stage * C::A_BYTES, &tmA, full_bar + 8 * stage, kb * BK, mb * BM);
-                    tma_load_2d(sB + stage * C::B_BYTES, &tmB, full_bar + 8 * stage, kb * BK, nb * BN);
+                    tma_load_2d(x_base + stage * x_bytes, x_map, full_bar + 8 * stage, kb * BK, x_row);
                     filled |= 1u << stage;
                     fill_phase = (fill_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == C::STAGES) {
@@ -320,6 +349,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         EpiSync es{epi_bar_addr, 0u, abort_flag, err};
+        pdl_wait();
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
             int mb, nb, sp, kb0, kb1;
             ts.get(t, mb, nb, sp, kb0, kb1);
@@ -439,7 +469,7 @@ int run(const CUtensorMap& ma, const CUtensorMap& mb, const TileSched& ts, const
     if (rc) return rc;
     const int tiles = ts.m_blocks * ts.n_blocks * ts.splits;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    gemm_tc_kernel<BN, MODE, SWAP><<<grid, NTHREADS, C::SMEM, st>>>(ma, mb, ts, a, err);
+    launch_pdl(gemm_tc_kernel<BN, MODE, SWAP>, dim3(grid), dim3(NTHREADS), C::SMEM, st, ma, mb, ts, a, err);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }

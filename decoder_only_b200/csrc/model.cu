@@ -25,6 +25,12 @@
 #include "epilogue.cuh"
 #include "kernels.h"
 
+// Programmatic dependent launch on the hot path (LLAMA_B200_NO_PDL=1: off).
+bool g_llama_pdl = [] {
+    const char* e = getenv("LLAMA_B200_NO_PDL");
+    return !(e && e[0] == '1');
+}();
+
 // ------------------------------------------------------------------ counters
 // Launches of this library's kernels (graph replays count their kernels).
 static std::atomic<int64_t> g_launches{0};
@@ -284,8 +290,16 @@ inline void* vcache(llama_model* m, int l) {
     return (uint8_t*)m->kv + (size_t)(2 * l + 1) * m->kv_layer_elems * m->esz;
 }
 
-__global__ void pos_set_kernel(int* pos, int v) { *pos = v; }
-__global__ void pos_advance_kernel(int* pos) { *pos += 1; }
+__global__ void pos_set_kernel(int* pos, int v) {
+    pdl_launch_dependents();
+    pdl_wait();
+    *pos = v;
+}
+__global__ void pos_advance_kernel(int* pos) {
+    pdl_launch_dependents();
+    pdl_wait();
+    *pos += 1;
+}
 
 EpiArgs base_args(llama_model* m, int M, int N) {
     EpiArgs a;
@@ -441,7 +455,7 @@ int decode_body(llama_model* m, cudaStream_t st) {
     prof::Scope ps(st, "decode_argmax", (double)m->B * c.vocab * 4, 0.0);
     if ((rc = launch_argmax_split(m->logits_dec, m->B, c.vocab, c.vocab, m->tok_cur, m->amax_part, m->amax_cnt, st)))
         return rc;
-    pos_advance_kernel<<<1, 1, 0, st>>>(m->d_pos);
+    launch_pdl(pos_advance_kernel, dim3(1), dim3(1), 0, st, m->d_pos);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }
@@ -628,7 +642,7 @@ int llama_prefill(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S,
                                       (int64_t)S * m->cfg.vocab, m->tok_cur, m->amax_part, m->amax_cnt, st)))
             return rc;
     }
-    pos_set_kernel<<<1, 1, 0, st>>>(m->d_pos, S);
+    launch_pdl(pos_set_kernel, dim3(1), dim3(1), 0, st, m->d_pos, (int)S);
     LLAMA_LAUNCH_CHECK();
     m->B = B;
     m->cur_len = S;
@@ -644,7 +658,7 @@ int llama_prefill_trunk(llama_model* m, const float* d_x, int32_t B, int32_t S, 
     int rc = run_blocks(m, B, S, false, st);
     if (rc) return rc;
     if (d_y != m->trunk) LLAMA_CUDA_TRY(cudaMemcpyAsync(d_y, m->trunk, bytes, cudaMemcpyDeviceToDevice, st));
-    pos_set_kernel<<<1, 1, 0, st>>>(m->d_pos, S);
+    launch_pdl(pos_set_kernel, dim3(1), dim3(1), 0, st, m->d_pos, (int)S);
     LLAMA_LAUNCH_CHECK();
     m->B = B;
     m->cur_len = S;
@@ -689,7 +703,7 @@ int llama_position(const llama_model* m) { return m ? m->cur_len : LLAMA_ERR_INV
 int llama_rewind(llama_model* m, int32_t position, void* stream) {
     if (!m || position < 1 || position > m->cur_len) return LLAMA_ERR_INVALID_ARG;
     if (m->B <= 0) return LLAMA_ERR_STATE;
-    pos_set_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(m->d_pos, position);
+    launch_pdl(pos_set_kernel, dim3(1), dim3(1), 0, (cudaStream_t)stream, m->d_pos, (int)position);
     LLAMA_LAUNCH_CHECK();
     m->cur_len = position;
     return LLAMA_OK;

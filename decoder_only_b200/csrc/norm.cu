@@ -12,6 +12,8 @@
 template <typename T>
 __global__ void embed_kernel(const int32_t* __restrict__ tok, const T* __restrict__ E, float* __restrict__ x,
                              int d, int vocab, int* __restrict__ err) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int r = blockIdx.x;
     int t = tok[r];
     if (t < 0 || t >= vocab) {   // out-of-range id: flag it, read row 0 instead
@@ -39,6 +41,8 @@ constexpr int RMS_MAXV = 8;   // float4 per thread held in registers: d <= 8 * 4
 template <typename TO>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ g,
                                                       TO* __restrict__ y, int d, float eps) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int r = blockIdx.x;
     const int nv = d >> 2;
     const float4* xr = reinterpret_cast<const float4*>(x + (size_t)r * d);
@@ -86,9 +90,9 @@ int launch_rmsnorm(int dtype, const float* x, const float* g, void* y, int rows,
     if (threads > 256) threads = 256;
     if (nv > RMS_MAXV * threads) return LLAMA_ERR_INVALID_ARG;
     if (dtype == LLAMA_BF16)
-        rmsnorm_kernel<bf16><<<rows, threads, 0, st>>>(x, g, (bf16*)y, d, eps);
+        launch_pdl(rmsnorm_kernel<bf16>, dim3(rows), dim3(threads), 0, st, x, g, (bf16*)y, d, eps);
     else
-        rmsnorm_kernel<float><<<rows, threads, 0, st>>>(x, g, (float*)y, d, eps);
+        launch_pdl(rmsnorm_kernel<float>, dim3(rows), dim3(threads), 0, st, x, g, (float*)y, d, eps);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }
@@ -97,9 +101,9 @@ int launch_embed(int dtype, const int32_t* tok, const void* E, float* x, int row
                  cudaStream_t st) {
     if (rows <= 0) return LLAMA_OK;
     if (dtype == LLAMA_BF16)
-        embed_kernel<bf16><<<rows, 256, 0, st>>>(tok, (const bf16*)E, x, d, vocab, err);
+        launch_pdl(embed_kernel<bf16>, dim3(rows), dim3(256), 0, st, tok, (const bf16*)E, x, d, vocab, err);
     else
-        embed_kernel<float><<<rows, 256, 0, st>>>(tok, (const float*)E, x, d, vocab, err);
+        launch_pdl(embed_kernel<float>, dim3(rows), dim3(256), 0, st, tok, (const float*)E, x, d, vocab, err);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }
@@ -166,6 +170,8 @@ __device__ __forceinline__ bool amx_better(float v, int i, float bv, int bi) {
 __global__ void __launch_bounds__(256) argmax_split_kernel(const float* __restrict__ logits, int n, int64_t ld,
                                                            int32_t* __restrict__ out, int2* __restrict__ part,
                                                            int* __restrict__ counters, int chunks) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int r = blockIdx.y, c = blockIdx.x;
     const float* p = logits + (size_t)r * ld;
     const int i0 = c * AMX_CHUNK, i1 = min(n, i0 + AMX_CHUNK);
@@ -229,7 +235,7 @@ int launch_argmax_split(const float* logits, int rows, int n, int64_t ld, int32_
                         cudaStream_t st) {
     if (rows <= 0) return LLAMA_OK;
     const int chunks = argmax_split_chunks(n);
-    argmax_split_kernel<<<dim3(chunks, rows), 256, 0, st>>>(logits, n, ld, out, part, counters, chunks);
+    launch_pdl(argmax_split_kernel, dim3(chunks, rows), dim3(256), 0, st, logits, n, ld, out, part, counters, chunks);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }

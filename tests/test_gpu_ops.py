@@ -133,7 +133,15 @@ def test_attention_prefill(B, H, S, hd, dtype):
             if dtype == torch.float32:
                 assert np.max(np.abs(got - ref)) <= 1e-5 * max(_rms(ref), 1e-3)
             else:
-                assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 2e-3 * _rms(ref))
+                assert np.all(np.abs(got - ref) <= _bf16_attn_bound(ref, v64[b, h, :S]))
+
+
+def _bf16_attn_bound(ref, v):
+    """Per-element bound of the bf16 attention: the probabilities are rounded
+    to bf16 before P.V (relative 2^-9 each), which moves a weighted average
+    by at most 2^-9 * sum_j w_j |v_j - o| <= 2^-8 max_j |v_j|; the output is
+    rounded once more (2^-9 |o|); fp32 accumulation adds far less."""
+    return 2.0 ** -8 * np.abs(ref) + 2.0 ** -8 * np.max(np.abs(v), axis=0)[None, :] + 1e-6
 
 
 def test_attention_prefill_full_length_sampled_heads():
@@ -142,7 +150,9 @@ def test_attention_prefill_full_length_sampled_heads():
     o = lb.attention_prefill(q, k, v).float().cpu().numpy().reshape(B, S, H, hd)
     for h in (0, 17, 31):
         ref = oracle.causal_attention(q64[0, h], k64[0, h], v64[0, h])
-        assert np.all(np.abs(o[0, :, h] - ref) <= 2.0 ** -8 * np.abs(ref) + 2e-3 * _rms(ref))
+        assert np.all(np.abs(o[0, :, h] - ref) <= _bf16_attn_bound(ref, v64[0, h]))
+        # and far inside it on average
+        assert _rms(o[0, :, h] - ref) <= 2e-3 * _rms(ref) + 2.0 ** -12
 
 
 @pytest.mark.parametrize("B,H,length,hd,dtype", [
