@@ -49,7 +49,9 @@ struct Cfg {
     static constexpr int A_BYTES = BM * BK * 2;            // 16 KB
     static constexpr int B_BYTES = BN * BK * 2;            // BN * 128 B
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = (BN >= 256) ? 4 : 8;
+    // decode tiles (BN 16 / 32) keep their footprint under half an SM so a
+    // second decode GEMM can be resident and prefetch its weights early
+    static constexpr int STAGES = (BN >= 256) ? 4 : (BN == 16 ? 5 : 4);
     static constexpr int TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;   // two accumulators, power of 2
     static constexpr int XLD = BM + 1;                                // transpose buffer row (decode)
     static constexpr int XBUF_BYTES = (BN < 256) ? 32 * XLD * 4 : 0;

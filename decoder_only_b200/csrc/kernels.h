@@ -40,9 +40,14 @@ int attention_tc_prepare();
 
 // decode.cu
 uint64_t attention_decode_work_bytes(int B, int H, int max_len, int hd);
+// counters: int [B*H], zero before the launch (each launch leaves them zero)
 int launch_attention_decode(int dtype, const void* q, const void* k, const void* v, void* o, int B, int H,
-                            int len, const int* d_len_minus1, int hd, int kv_stride, float* work,
-                            cudaStream_t st);
+                            int len, const int* d_len_minus1, int hd, int kv_stride, float* work, int* counters,
+                            int* err, cudaStream_t st);
+int* attention_decode_counters(float* work, int B, int H, int max_len, int hd);
+int attention_decode_clear(float* work, int B, int H, int len, int hd, cudaStream_t st);
+int attention_decode_prepare();
+int op_error_word(int** p);   // error word of the standalone ops
 
 // gemm_tc.cu  (bf16 tcgen05 GEMM)
 struct TcGemm {

@@ -127,14 +127,12 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // Error word of the standalone ops (the model has its own in its arena).
 __device__ int g_op_err_word;
 
-namespace {
 int op_error_word(int** p) {
     static int* addr = nullptr;
     if (!addr) LLAMA_CUDA_TRY(cudaGetSymbolAddress((void**)&addr, g_op_err_word));
     *p = addr;
     return LLAMA_OK;
 }
-}  // namespace
 
 struct llama_model {
     llama_config cfg;
@@ -155,6 +153,7 @@ struct llama_model {
     float* partial;          // split-K partials
     size_t partial_elems;
     int* counters;           // split-K arrival counters (zero between launches)
+    int* attn_cnt;           // decode-attention arrival counters [max_batch * H]
     int2* amax_part;         // greedy-choice chunk results [max_batch][chunks]
     int* amax_cnt;           // and their arrival counters [max_batch]
     float* attn_work;
@@ -244,6 +243,7 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     const size_t pmax = (size_t)MAX_DEC_SPLITS * c->max_batch * std::max(cmax, V);
     float* partial = (float*)take(c->dtype == LLAMA_BF16 ? pmax * 4 : 0);
     int* counters = (int*)take(MAX_COUNTERS * 4);
+    int* attn_cnt = (int*)take((size_t)c->max_batch * c->n_heads * 4);
     int2* amax_part = (int2*)take((size_t)c->max_batch * argmax_split_chunks(c->vocab) * sizeof(int2));
     int* amax_cnt = (int*)take((size_t)c->max_batch * 4);
     const uint64_t awb = attention_decode_work_bytes(c->max_batch, c->n_heads, c->max_seq, c->head_dim);
@@ -270,6 +270,7 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
         m->partial_elems = pmax;
         m->counters = counters;
         m->amax_part = amax_part;
+        m->attn_cnt = attn_cnt;
         m->amax_cnt = amax_cnt;
         m->attn_work = attn_work;
         m->attn_work_bytes = awb;
@@ -397,7 +398,8 @@ int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
             const double len = (double)m->cur_len + 1;   // keys read this step
             prof::Scope ps(st, "decode_attention", (2.0 * len + 2.0) * B * d * m->esz, 4.0 * B * d * len);
             if ((rc = launch_attention_decode(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, 0,
-                                              m->d_pos, c.head_dim, c.max_seq, m->attn_work, st)))
+                                              m->d_pos, c.head_dim, c.max_seq, m->attn_work, m->attn_cnt, m->d_err,
+                                              st)))
                 return rc;
         } else {
             prof::Scope ps(st, "prefill_attention", 4.0 * n * d * m->esz, 2.0 * B * (double)S * (S + 1) * d);
@@ -603,12 +605,14 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
     }
     if (cudaMemsetAsync(m->counters, 0, MAX_COUNTERS * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->amax_cnt, 0, (size_t)cfg->max_batch * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(m->attn_cnt, 0, (size_t)cfg->max_batch * cfg->n_heads * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->d_pos, 0, 256, st) != cudaSuccess) {
         llama_free(m);
         return LLAMA_ERR_CUDA;
     }
     pick_decode_splits(m);
-    if ((rc = gemm_tc_prepare()) || (rc = attention_prepare()) || (rc = attention_tc_prepare())) {
+    if ((rc = gemm_tc_prepare()) || (rc = attention_prepare()) || (rc = attention_tc_prepare()) ||
+        (rc = attention_decode_prepare())) {
         llama_free(m);
         return rc;
     }
@@ -840,8 +844,13 @@ int llama_op_attention_decode(int32_t dtype, const void* d_q, const void* d_k, c
         return LLAMA_ERR_INVALID_ARG;
     if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
     if (work_bytes < attention_decode_work_bytes(B, H, len, head_dim)) return LLAMA_ERR_OOM;
+    int* err = nullptr;
+    int rc = op_error_word(&err);
+    if (rc) return rc;
+    if ((rc = attention_decode_clear((float*)d_work, B, H, len, head_dim, (cudaStream_t)stream))) return rc;
     return launch_attention_decode(dtype, d_q, d_k, d_v, d_o, B, H, len, nullptr, head_dim, kv_stride,
-                                   (float*)d_work, (cudaStream_t)stream);
+                                   (float*)d_work, attention_decode_counters((float*)d_work, B, H, len, head_dim),
+                                   err, (cudaStream_t)stream);
 }
 
 int llama_op_argmax(const float* d_logits, int32_t rows, int32_t n, int32_t* d_out, void* stream) {

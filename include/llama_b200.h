@@ -211,9 +211,10 @@ LLAMA_API int llama_op_attention_prefill(int32_t dtype, const void* d_q, const v
 
 /* Decode attention: one query per (b, h) against keys/values 0..len-1.
  * q dtype-typed [B, H*head_dim]; k, v [B][H][kv_stride][head_dim];
- * o dtype-typed [B, H*head_dim].  Split over the sequence into chunks whose
- * partial results go to d_work (fp32, llama_op_attention_decode_work_bytes
- * bytes), then combined. */
+ * o dtype-typed [B, H*head_dim].  Split over the sequence into chunks of 128
+ * keys whose partial results go to d_work (llama_op_attention_decode_work_bytes
+ * bytes: fp32 partials, then int arrival counters the call clears first);
+ * the last chunk of each (b, h) to finish merges them. */
 LLAMA_API int llama_op_attention_decode(int32_t dtype, const void* d_q, const void* d_k,
                               const void* d_v, void* d_o, int32_t B, int32_t H,
                               int32_t len, int32_t head_dim, int32_t kv_stride,
@@ -228,15 +229,17 @@ LLAMA_API uint64_t llama_op_attention_decode_work_bytes(int32_t B, int32_t H, in
  * integration variant.  The split-sequence workspace is a fixed 8 MiB array
  * in the library's own device memory, held on every GPU that loads the
  * library until the process exits; this call allocates nothing.
- *   - B * H * ceil(len / 256) * (head_dim + 2) must be <= 2,097,152
- *     (floats of workspace); larger calls return LLAMA_ERR_OOM and queue
- *     nothing.  head_dim in {32, 64, 128}.
+ *   - llama_op_attention_decode_work_bytes(B, H, len, head_dim) =
+ *     4 * B * H * ceil(len / 128) * (head_dim + 2) (rounded up to 16) +
+ *     4 * B * H must be <= 8 MiB; larger calls return LLAMA_ERR_OOM and
+ *     queue nothing.  head_dim in {32, 64, 128}.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first
  *     call before any stream capture.
  *   - All calls share the array: calls that overlap on the GPU (different
- *     streams or host threads) race.  Each call writes every workspace slot
- *     it reads, so no clearing is needed between calls.
+ *     streams or host threads) race.  Each call clears the array's
+ *     arrival counters (a memset on `stream`) before its kernel; every
+ *     other slot it reads it writes first.
  * Arguments and layouts as llama_op_attention_decode. */
 LLAMA_API int llama_op_attention_decode_noalloc(int32_t dtype, const void* d_q, const void* d_k,
                                                 const void* d_v, void* d_o, int32_t B, int32_t H,

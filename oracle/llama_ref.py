@@ -283,30 +283,41 @@ def prefill(shape, tokens: np.ndarray, seed: int = 0, weights=None, return_cache
     ``weights``: optional callable layer -> dict (else drawn from ``synth``).
     With ``return_cache`` the per-layer (K after RoPE, V) of every sequence is
     returned as cache[l] = (K, V), each (B, H, S, d_head).
+    ``storage`` may be a tuple of storage modes: the forward pass then runs
+    once per mode on the same weights (each layer drawn once) and a list of
+    logits, one per mode, is returned.
     """
+    multi = isinstance(storage, (tuple, list))
+    modes = list(storage) if multi else [storage]
     tokens = np.asarray(tokens)
     B, S = tokens.shape
     E = embed_table(shape, seed)
     get_w = weights if weights is not None else (lambda l: layer_weights(shape, l, seed))
-    xs = [E[tokens[b]].copy() for b in range(B)]
+    xs = [[E[tokens[b]].copy() for b in range(B)] for _ in modes]
     positions = np.arange(S)
     cache = [] if return_cache else None
     for l in range(shape.n_layers):
         W = get_w(l)
-        kv = []
-        for b in range(B):
-            xs[b] = pre_norm_block(xs[b], W, positions, shape, kv if return_cache else None, storage)
-        if return_cache:
-            cache.append((np.stack([k for k, _ in kv]), np.stack([v for _, v in kv])))
+        for mi, mode in enumerate(modes):
+            kv = []
+            for b in range(B):
+                xs[mi][b] = pre_norm_block(xs[mi][b], W, positions, shape,
+                                           kv if (return_cache and mi == 0) else None, mode)
+            if return_cache and mi == 0:
+                cache.append((np.stack([k for k, _ in kv]), np.stack([v for _, v in kv])))
         del W
-    trunk = np.stack(xs)
     Wh = head_matrix(shape, seed)
-    logits = _storer(storage)(rms_norm(trunk, np.ones(shape.d_model), shape.norm_eps)) @ Wh
-    out = [logits]
+    logits_all = []
+    for mi, mode in enumerate(modes):
+        trunk = np.stack(xs[mi])
+        logits_all.append(_storer(mode)(rms_norm(trunk, np.ones(shape.d_model), shape.norm_eps)) @ Wh)
+    if multi:
+        return logits_all
+    out = [logits_all[0]]
     if return_cache:
         out.append(cache)
     if return_trunk:
-        out.append(trunk)
+        out.append(np.stack(xs[0]))
     return out[0] if len(out) == 1 else tuple(out)
 
 

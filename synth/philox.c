@@ -102,20 +102,51 @@ static inline uint16_t f64_to_bf16_rne(double x) {
 
 uint16_t synth_f64_to_bf16(double x) { return f64_to_bf16_rne(x); }
 
+/* Elements [first, first+count) computed four at a time: one Philox call and
+ * one (u1 -> R) per pair of lanes serve all four; every element still gets
+ * exactly the value normal_at(e) defines. */
+static inline void normals_block(uint32_t seed, uint32_t tensor_id, uint64_t e4, double out[4]) {
+    uint32_t ctr[4] = {(uint32_t)e4, (uint32_t)(e4 >> 32), 0u, 0u};
+    uint32_t key[2] = {seed, tensor_id};
+    uint32_t r[4];
+    synth_philox4x32_10(ctr, key, r);
+    for (int p = 0; p < 2; ++p) {
+        double u1 = ((double)r[2 * p] + 1.0) * 2.3283064365386963e-10;
+        double u2 = (double)r[2 * p + 1] * 2.3283064365386963e-10;
+        double R = sqrt(-2.0 * log(u1));
+        double t = 2.0 * 3.141592653589793 * u2;
+        out[2 * p] = R * cos(t);
+        out[2 * p + 1] = R * sin(t);
+    }
+}
+
+static inline void normals_range(uint32_t seed, uint32_t tensor_id, uint64_t first, uint64_t count, double scale,
+                                 double* out) {
+    const int64_t b0 = (int64_t)(first >> 2), b1 = (int64_t)((first + count + 3) >> 2);
+#pragma omp parallel for schedule(static)
+    for (int64_t blk = b0; blk < b1; ++blk) {
+        double z[4];
+        normals_block(seed, tensor_id, (uint64_t)blk, z);
+        for (int j = 0; j < 4; ++j) {
+            const uint64_t e = ((uint64_t)blk << 2) + (uint64_t)j;
+            if (e >= first && e < first + count) out[e - first] = scale * z[j];
+        }
+    }
+}
+
 /* out[i] = scale * z_{first+i}, fp64, unrounded */
 void synth_normal_f64(uint32_t seed, uint32_t tensor_id, uint64_t first, uint64_t count,
                       double scale, double* out) {
-#pragma omp parallel for schedule(static)
-    for (int64_t i = 0; i < (int64_t)count; ++i)
-        out[i] = scale * normal_at(seed, tensor_id, first + (uint64_t)i);
+    normals_range(seed, tensor_id, first, count, scale, out);
 }
 
 /* rounded to the storage type, returned as fp64 values (exactly representable) */
 void synth_normal_stored_f64(uint32_t seed, uint32_t tensor_id, uint64_t first, uint64_t count,
                              double scale, int dtype_bf16, double* out) {
+    normals_range(seed, tensor_id, first, count, scale, out);
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < (int64_t)count; ++i) {
-        double v = scale * normal_at(seed, tensor_id, first + (uint64_t)i);
+        double v = out[i];
         if (dtype_bf16) {
             uint32_t b = (uint32_t)f64_to_bf16_rne(v) << 16;
             float f;

@@ -1,0 +1,67 @@
+"""Parity of the LLaMA-13B-shaped decode workload (40 layers, d 5120,
+batch 32: the 32-row decode GEMMs) and of the LLaMA-65B-width slice (16
+layers, d 8192, hidden 22016, batch 8).  Same bar as the 7B tests: no
+further from the exact fp64 oracle than bf16 storage alone moves it, and
+>= 99 % greedy agreement (tests/_parity.py)."""
+import numpy as np
+import pytest
+import torch
+
+import decoder_only_b200 as lb
+import oracle
+import synth
+from synth.workloads import LLAMA_13B, LLAMA_65B_SLICE, SEED
+from _parity import argmax_agreement, rms, storage_bar
+
+pytestmark = pytest.mark.gpu
+
+
+def test_13b_batch32_prefill_and_decode():
+    B, S, P = 32, 2048, 64
+    tok = synth.tokens(SEED, B * (S + 4), LLAMA_13B.vocab).reshape(B, S + 4)
+    m = lb.Model(LLAMA_13B, max_batch=B, max_seq=S + 256)
+    try:
+        tk = torch.from_numpy(tok).cuda()
+        # short prompts: prefill rows 0..P-1 and four teacher-forced decode
+        # steps at positions P..P+3, against the oracle on sequences 0 and 31
+        lg = m.prefill(tk[:, :P].contiguous())[[0, 31]].cpu().numpy()
+        dec = []
+        for t in range(P, P + 4):
+            _, l = m.decode_step(tk[:, t].contiguous())
+            dec.append(l[[0, 31]].cpu().numpy())
+        dec = np.stack(dec, axis=1)
+        # full-length prompts: decode at positions 2048.. equals prefill rows
+        m.prefill(tk[:, :S].contiguous(), logits=False)
+        full = []
+        for t in range(S, S + 2):
+            _, l = m.decode_step(tk[:, t].contiguous())
+            full.append(l.cpu().numpy())
+        full = np.stack(full, axis=1)
+        ref_full = m.prefill(tk[:, :S + 2].contiguous())[:, S:S + 2].cpu().numpy()
+    finally:
+        m.close()
+        torch.cuda.empty_cache()
+    exact, stored = oracle.prefill(LLAMA_13B, tok[[0, 31], :P + 4], storage=(None, "bf16"))
+    storage_bar(lg, exact[:, :P], stored[:, :P])
+    storage_bar(dec, exact[:, P:P + 4], stored[:, P:P + 4])
+    assert argmax_agreement(np.concatenate([lg, dec], 1), exact)[1] >= 0.99
+    bar_rms = rms(stored - exact) / rms(exact)
+    assert rms(full - ref_full) / rms(ref_full) <= 2 * 1.5 * bar_rms
+    assert argmax_agreement(full, ref_full)[1] >= 0.99
+
+
+def test_65b_slice_prefill_8x2048():
+    B, S, P = 8, 2048, 64
+    tok = synth.tokens(SEED, B * S, LLAMA_65B_SLICE.vocab).reshape(B, S)
+    m = lb.Model(LLAMA_65B_SLICE, max_batch=B, max_seq=S)
+    try:
+        lg = m.prefill(torch.from_numpy(tok).cuda())
+        got = lg[[0, 7], :P].cpu().numpy()
+        assert torch.isfinite(lg).all()
+    finally:
+        m.close()
+        del lg
+        torch.cuda.empty_cache()
+    exact, stored = oracle.prefill(LLAMA_65B_SLICE, tok[[0, 7], :P], storage=(None, "bf16"))
+    storage_bar(got, exact, stored)
+    assert argmax_agreement(got, exact)[1] >= 0.99
