@@ -43,6 +43,9 @@ WORKLOADS = {
                        desc="llama-13b: 256 greedy decode steps, batch 32, 2048-token prompts prefilled untimed"),
     "65b-slice": dict(model="LLAMA_65B_SLICE", batch=8, seq=2048, decode=0,
                       desc="llama-65b widths, 16 layers: prefill 8 x 2048 (logits at every position)"),
+    # small case of the 7B kernels (same shapes per launch) for ncu captures
+    "7b-2layer": dict(model="LLAMA_7B", layers=2, batch=4, seq=2048, decode=128,
+                      desc="llama-7b widths, 2 layers: prefill 4 x 2048 + 128 greedy decode steps"),
 }
 
 
@@ -437,6 +440,8 @@ def main():
     from synth import workloads as wls
     wl = dict(WORKLOADS[args.workload], name=args.workload)
     shape = getattr(wls, wl["model"])
+    if "layers" in wl:
+        shape = shape.with_(n_layers=wl["layers"], name=f"{shape.name}-{wl['layers']}layer")
     if args.impl == "reference":
         run_reference(args, wl, shape)
     else:
