@@ -1,0 +1,884 @@
+// The greedy decode step of a bf16 model as one persistent kernel.
+//
+// One decode step ([PFD] "The one formula" applied to the B newest tokens,
+// keys and values of all earlier positions read from the cache ([NAR] "GQA
+// Was Not an Original LLaMA Feature")) is a chain of small, HBM-bound
+// phases:
+//   embed + RMSNorm
+//   per layer:  QKV projection (+RoPE, append K and V at the position)
+//               attention over the cache
+//               O projection (+residual, then RMSNorm of the updated trunk)
+//               gate/up projection (+SwiGLU)
+//               down projection (+residual, then the next RMSNorm)
+//   head projection (fp32 logits), greedy argmax, position + 1.
+// Launched one kernel per phase, fixed costs dominate (launch, set-up,
+// pipeline fill, tails).  Here one cooperative launch of one CTA per SM runs
+// all phases, separated by a grid-wide barrier; the weights -- which do not
+// depend on any phase -- stream continuously: the TMA producer requests the
+// weight tile of the next projection as soon as a ring slot frees, and only
+// the activation tile of each stage waits for the barrier that makes that
+// activation visible.
+//
+// Warp roles (192 threads):
+//   warp 0     TMA producer, all projections of the step in order
+//   warp 1     TMEM owner and tcgen05.mma issuer (swap-AB: 128 weight rows on
+//              the TMEM lanes, the B <= 32 tokens as N = 16 or 32 columns)
+//   warps 2-5  everything else: projection epilogues (split-K partials, the
+//              last split to arrive finishes the tile), attention, norms,
+//              greedy choice, and the arrivals at the grid barrier.
+// Every wait is bounded (2 s): a CTA that gives up records
+// LLAMA_DEVERR_TIMEOUT and leaves; the others then give up at the next grid
+// barrier.  Named barriers among the 128 epilogue threads follow a
+// collective OR of each thread's wait result, so they leave together.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "kernels.h"
+#include "tcgen05.cuh"
+
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128;      // weight rows per tile (TMEM lanes)
+constexpr int BK = 64;       // K per stage (one 128-byte swizzle row)
+constexpr int NT = 192;
+constexpr int ACH = 64;      // keys per attention item
+constexpr int ANB = 3;       // attention items in flight per CTA
+constexpr int AMX = 2048;    // logits per greedy-choice item
+
+enum PhaseType { PH_EMBED = 0, PH_QKV = 1, PH_ATTN = 2, PH_O = 3, PH_GU = 4, PH_DOWN = 5, PH_HEAD = 6, PH_ARGMAX = 7 };
+
+template <int BN, int HD>
+struct SCfg {
+    static constexpr int STAGES = (BN == 16) ? 5 : 4;
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_ATT = OFF_B + STAGES * B_BYTES;             // [ANB][2][ACH][HD] bf16
+    static constexpr int ATT_BUF = 2 * ACH * HD * 2;
+    static constexpr int OFF_X = OFF_ATT + ANB * ATT_BUF;               // [32][XLD] floats
+    static constexpr int XLD = BM + 1;
+    static constexpr int OFF_SO = OFF_X + 32 * XLD * 4;                   // [16][HD] floats
+    static constexpr int OFF_SML = OFF_SO + 16 * HD * 4;                  // m[16], l[16], red[16]
+    static constexpr int OFF_BAR = OFF_SML + 256;
+    static constexpr int SMEM = OFF_BAR + 512 + 1024;
+    static constexpr uint32_t TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
+};
+
+__device__ __forceinline__ int phase_count(const StepArgs& a) { return 3 + 5 * a.L; }
+
+__device__ __forceinline__ int phase_type(const StepArgs& a, int p, int& layer) {
+    if (p == 0) {
+        layer = 0;
+        return PH_EMBED;
+    }
+    const int q = p - 1;
+    if (q < 5 * a.L) {
+        layer = q / 5;
+        return PH_QKV + q % 5;
+    }
+    layer = a.L;
+    return q == 5 * a.L ? PH_HEAD : PH_ARGMAX;
+}
+
+struct GemmPh {
+    int map_a, map_b, rowsA, K, splits, mode;
+};
+
+__device__ __forceinline__ bool gemm_of(const StepArgs& a, int type, int l, GemmPh& g) {
+    const int L = a.L;
+    switch (type) {
+        case PH_QKV: g = GemmPh{4 * l + 0, 4 * L + 1, 3 * a.d, a.d, a.splits[0], EPI_QKV}; return true;
+        case PH_O: g = GemmPh{4 * l + 1, 4 * L + 2, a.d, a.d, a.splits[1], EPI_RESID}; return true;
+        case PH_GU: g = GemmPh{4 * l + 2, 4 * L + 1, 2 * a.h, a.d, a.splits[2], EPI_SWIGLU}; return true;
+        case PH_DOWN: g = GemmPh{4 * l + 3, 4 * L + 3, a.d, a.h, a.splits[3], EPI_RESID}; return true;
+        case PH_HEAD: g = GemmPh{4 * L, 4 * L + 1, a.V, a.d, a.splits[4], EPI_F32}; return true;
+        default: return false;
+    }
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Bounded wait until the grid barrier generation reaches `target`.
+__device__ bool wait_gen(const unsigned* gen, unsigned target, volatile int* abort_flag, int* err) {
+    if ((int)(ld_acquire_u32(gen) - target) >= 0) return true;
+    const uint64_t t0 = global_timer();
+    while (true) {
+        if ((int)(ld_acquire_u32(gen) - target) >= 0) return true;
+        if (*abort_flag) return false;
+        if (global_timer() - t0 > WAIT_LIMIT_NS) {
+            *abort_flag = 1;
+            atomicOr(err, LLAMA_DEVERR_TIMEOUT);
+            return false;
+        }
+        __nanosleep(32);
+    }
+}
+
+// One arrival per CTA; the last one resets the count and publishes the next
+// generation.
+__device__ void grid_arrive(unsigned* bar, unsigned next_gen) {
+    __threadfence();
+    const unsigned prev = atomicAdd(bar, 1u);
+    if (prev == gridDim.x - 1) {
+        atomicExch(bar, 0u);
+        __threadfence();
+        atomicExch(bar + 1, next_gen);
+    }
+}
+
+// Named barrier of the 128 epilogue threads
+__device__ __forceinline__ void esync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// ... that also returns whether any of them failed (all leave together)
+__device__ __forceinline__ bool esync_any(bool fail) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, 1, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)fail)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ float esum(float v, float* red, int tid) {
+    v = warp_sum(v);
+    if ((tid & 31) == 0) red[tid >> 5] = v;
+    esync();
+    const float s = red[0] + red[1] + red[2] + red[3];
+    esync();
+    return s;
+}
+
+// RMSNorm of the B trunk rows into xn (bf16), by the 128 epilogue threads
+// of one CTA ("RMSNorm: LayerNorm minus the mean"; gain g).
+__device__ void norm_rows(const StepArgs& a, const float* g, float* red, int tid) {
+    const int d = a.d;
+    for (int b = 0; b < a.B; ++b) {
+        const float* x = a.trunk + (size_t)b * d;
+        float ss = 0.f;
+        for (int i = tid * 4; i < d; i += 512) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(x + i));
+            ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+        }
+        const float inv = rsqrtf(esum(ss, red, tid) / (float)d + a.eps);
+        for (int i = tid * 4; i < d; i += 512) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(x + i));
+            const float4 gg = *reinterpret_cast<const float4*>(g + i);
+            *reinterpret_cast<uint2*>(a.xn + (size_t)b * d + i) =
+                make_uint2(pack_bf16x2(v.x * inv * gg.x, v.y * inv * gg.y), pack_bf16x2(v.z * inv * gg.z, v.w * inv * gg.w));
+        }
+    }
+}
+
+template <int BN, int HD>
+struct Smem {
+    uint32_t sA, sB;
+    uint32_t full, empty, tfull, tempty, abar;
+    uint8_t* att;        // generic pointer to the attention buffers
+    float* xbuf;
+    float* so;
+    float* sm;           // [16] maxima
+    float* sl;           // [16] sums
+    float* red;          // [16] reduction scratch
+    volatile int* flag;
+};
+
+// ---------------------------------------------------------------- projection epilogue
+// One finished 128-feature tile (et = TMEM lane = feature within the tile).
+template <int BN, int HD, int MODE>
+__device__ bool tile_epilogue(const StepArgs& a, const EpiArgs& ep, const GemmPh& g, int l, int type, int mb,
+                              int sp, int et, int tid, const float (&v)[32], const Smem<BN, HD>& sm) {
+    constexpr bool PAIR = (MODE == EPI_SWIGLU);
+    const int n = mb * BM + et;
+    const int M = a.B, N = g.rowsA;
+    const bool direct = (g.splits == 1) && !PAIR;
+    if (!direct) {
+        float* dst = a.partial + (size_t)sp * M * N + n;
+#pragma unroll
+        for (int b = 0; b < BN; ++b)
+            if (b < M) dst[(size_t)b * N] = v[b];
+        __threadfence();
+        esync();
+        if (tid == 0) {
+            const int cidx = PAIR ? (mb >> 1) : mb;
+            const int target = PAIR ? 2 * g.splits : g.splits;
+            const int prev = atomicAdd(a.counters + cidx, 1);
+            const int last = (prev == target - 1);
+            if (last) a.counters[cidx] = 0;
+            *sm.flag = last;
+        }
+        esync();
+        const int last = *sm.flag;
+        esync();
+        if (!last) return true;
+        __threadfence();
+    }
+    if constexpr (PAIR) {
+        const int j = mb >> 1;
+        const float* pg = a.partial + 256 * j + et;
+        const float* pu = pg + 128;
+        for (int b = 0; b < M; ++b) {
+            float gsum = 0.f, usum = 0.f;
+            for (int s = 0; s < g.splits; ++s) {
+                gsum += __ldcg(pg + (size_t)s * M * N + (size_t)b * N);
+                usum += __ldcg(pu + (size_t)s * M * N + (size_t)b * N);
+            }
+            a.act[(size_t)b * a.h + 128 * j + et] = __float2bfloat16_rn(silu_f(gsum) * usum);
+        }
+        return true;
+    } else {
+        float sum[32];
+#pragma unroll
+        for (int b = 0; b < 32; ++b) sum[b] = direct ? v[b] : 0.f;
+        if (!direct) {
+            for (int s = 0; s < g.splits; ++s) {
+                const float* p = a.partial + (size_t)s * M * N + n;
+#pragma unroll
+                for (int b = 0; b < BN; ++b)
+                    if (b < M) sum[b] += __ldcg(p + (size_t)b * N);
+            }
+        }
+        if constexpr (MODE == EPI_RESID || MODE == EPI_F32) {
+#pragma unroll
+            for (int b = 0; b < BN; ++b) {
+                if (b < M) {
+                    float* o = ep.out + (size_t)b * ep.ld_out + n;
+                    if constexpr (MODE == EPI_RESID) *o += sum[b];
+                    else *o = sum[b];
+                }
+            }
+            if constexpr (MODE == EPI_RESID) {
+                // the CTA that finishes the phase's last tile normalises the trunk
+                __threadfence();
+                esync();
+                if (tid == 0) {
+                    const int prev = atomicAdd(a.tiles_done, 1);
+                    const int last = (prev == g.rowsA / BM - 1);
+                    if (last) *a.tiles_done = 0;
+                    *sm.flag = last;
+                }
+                esync();
+                const int last = *sm.flag;
+                esync();
+                if (last) {
+                    __threadfence();
+                    const float* gain = (type == PH_O) ? a.gains[2 * l + 1] : a.gains[2 * (l + 1)];
+                    norm_rows(a, gain, sm.red, tid);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int b = 0; b < BN; ++b) sm.xbuf[b * SCfg<BN, HD>::XLD + et] = sum[b];
+            esync();
+            if (tid < 4 * M) {
+                const int b = tid >> 2, c = tid & 3;
+                float w[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w[i] = sm.xbuf[b * SCfg<BN, HD>::XLD + c * 32 + i];
+                epi_qkv32<bf16>(ep, b, mb * BM + c * 32, w);
+            }
+            esync();
+        }
+        return true;
+    }
+}
+
+// ---------------------------------------------------------------- attention phase
+template <int BN, int HD>
+__device__ void issue_attn(const StepArgs& a, int l, int item, int nch, int len, int buf, const Smem<BN, HD>& sm) {
+    const int chunk = item % nch, bh = item / nch;
+    const int b = bh / a.H, h = bh - b * a.H;
+    const int k0 = chunk * ACH;
+    const int nkeys = min(len - k0, ACH);
+    const bf16* kc = a.kv + (size_t)(2 * l) * a.kv_layer;
+    const bf16* vc = kc + a.kv_layer;
+    const size_t off = (((size_t)b * a.H + h) * a.smax + k0) * HD;
+    const uint32_t bytes = (uint32_t)(nkeys * HD * 2);
+    const uint32_t bar = sm.abar + 8 * buf;
+    const uint32_t dk = smem_u32(sm.att + (size_t)buf * SCfg<BN, HD>::ATT_BUF);
+    const uint32_t dv = dk + ACH * HD * 2;
+    mbar_expect_tx(bar, 2 * bytes);
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dk),
+                 "l"(kc + off), "r"(bytes), "r"(bar)
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dv),
+                 "l"(vc + off), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+template <int BN, int HD>
+__device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>& sm, uint32_t* uses,
+                           volatile int* abort_flag) {
+    constexpr int DPL = HD / 8;      // dims per lane: 16-byte vectors u = 0.., dims (u*8 + r)*8 ..
+    constexpr int NV = DPL / 8;
+    const int len = *a.d_pos + 1;
+    const int nch = (len + ACH - 1) / ACH;
+    const int nchmax = (a.smax + ACH - 1) / ACH;
+    const int nitems = nch * a.B * a.H;
+    int count = 0;
+    for (int i = blockIdx.x; i < nitems; i += gridDim.x) ++count;
+    if (tid == 0)
+        for (int j = 0; j < min(ANB, count); ++j) issue_attn<BN, HD>(a, l, blockIdx.x + j * gridDim.x, nch, len, j, sm);
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 3, r = lane & 7;
+    const float scale = rsqrtf((float)HD);
+    for (int j = 0; j < count; ++j) {
+        const int item = blockIdx.x + j * gridDim.x;
+        const int buf = j % ANB;
+        const int chunk = item % nch, bh = item / nch;
+        const int b = bh / a.H, h = bh - b * a.H;
+        const int nkeys = min(len - chunk * ACH, ACH);
+        // wait for this item's K and V rows
+        const uint32_t bar = sm.abar + 8 * buf;
+        bool ok = false;
+        {
+            const uint64_t t0 = global_timer();
+            while (true) {
+                if (mbar_try_wait(bar, uses[buf] & 1u)) {
+                    ok = true;
+                    break;
+                }
+                if (*abort_flag || global_timer() - t0 > WAIT_LIMIT_NS) break;
+            }
+        }
+        uses[buf]++;
+        if (esync_any(!ok)) {
+            if (tid == 0) {
+                *abort_flag = 1;
+                atomicOr(a.err, LLAMA_DEVERR_TIMEOUT);
+            }
+            return false;
+        }
+        const bf16* sk = reinterpret_cast<const bf16*>(sm.att + (size_t)buf * SCfg<BN, HD>::ATT_BUF);
+        const bf16* sv = sk + ACH * HD;
+        float qv[DPL];
+        {
+            const bf16* qp = a.q + ((size_t)b * a.H + h) * HD;
+#pragma unroll
+            for (int u = 0; u < NV; ++u) {
+                const uint4 w = __ldcg(reinterpret_cast<const uint4*>(qp + (u * 8 + r) * 8));
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const float2 f = unpack_bf16x2(ws[t]);
+                    qv[u * 8 + 2 * t] = f.x * scale;
+                    qv[u * 8 + 2 * t + 1] = f.y * scale;
+                }
+            }
+        }
+        float m = -INFINITY, lsum = 0.f, acc[DPL];
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int i = 0; i < ACH / 16; ++i) {
+            const int key = warp * (ACH / 4) + 4 * i + g;
+            const bool valid = key < nkeys;
+            const int kr = valid ? key : 0;
+            float kk[DPL], vv[DPL];
+#pragma unroll
+            for (int u = 0; u < NV; ++u) {
+                const uint4 wk = *reinterpret_cast<const uint4*>(sk + (size_t)kr * HD + (u * 8 + r) * 8);
+                const uint4 wv = *reinterpret_cast<const uint4*>(sv + (size_t)kr * HD + (u * 8 + r) * 8);
+                const uint32_t k4[4] = {wk.x, wk.y, wk.z, wk.w}, v4[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const float2 fk = unpack_bf16x2(k4[t]), fv = unpack_bf16x2(v4[t]);
+                    kk[u * 8 + 2 * t] = fk.x;
+                    kk[u * 8 + 2 * t + 1] = fk.y;
+                    vv[u * 8 + 2 * t] = fv.x;
+                    vv[u * 8 + 2 * t + 1] = fv.y;
+                }
+            }
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) s = fmaf(qv[e], kk[e], s);
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            s += __shfl_xor_sync(0xffffffffu, s, 2);
+            s += __shfl_xor_sync(0xffffffffu, s, 4);
+            if (valid) {
+                const float m_new = fmaxf(m, s);
+                const float corr = __expf(m - m_new);
+                const float p = __expf(s - m_new);
+                lsum = lsum * corr + p;
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) acc[e] = fmaf(acc[e], corr, p * vv[e]);
+                m = m_new;
+            }
+        }
+        // merge the 16 groups of this item into the chunk's partial
+        const int grp = warp * 4 + g;
+        if (r == 0) {
+            sm.sm[grp] = m;
+            sm.sl[grp] = lsum;
+        }
+#pragma unroll
+        for (int u = 0; u < NV; ++u)
+#pragma unroll
+            for (int t = 0; t < 8; ++t) sm.so[grp * HD + (u * 8 + r) * 8 + t] = acc[u * 8 + t];
+        esync();
+        // the buffer has been read: refill it with the item ANB places ahead
+        if (tid == 0 && j + ANB < count) issue_attn<BN, HD>(a, l, blockIdx.x + (j + ANB) * gridDim.x, nch, len, buf, sm);
+        float M = -INFINITY;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) M = fmaxf(M, sm.sm[t]);
+        float* wp = a.attn_work + ((size_t)bh * nchmax + chunk) * (HD + 2);
+        for (int c = tid; c < HD; c += 128) {
+            float s = 0.f;
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+                if (sm.sm[t] != -INFINITY) s += sm.so[t * HD + c] * __expf(sm.sm[t] - M);
+            wp[2 + c] = s;
+        }
+        if (tid == 0) {
+            float L = 0.f;
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+                if (sm.sm[t] != -INFINITY) L += sm.sl[t] * __expf(sm.sm[t] - M);
+            wp[0] = M;
+            wp[1] = L;
+        }
+        __threadfence();
+        esync();
+        if (tid == 0) {
+            const int prev = atomicAdd(a.attn_cnt + bh, 1);
+            const int last = (prev == nch - 1);
+            if (last) a.attn_cnt[bh] = 0;
+            *sm.flag = last;
+        }
+        esync();
+        const int last = *sm.flag;
+        esync();
+        if (last) {
+            __threadfence();
+            const float* wb = a.attn_work + (size_t)bh * nchmax * (HD + 2);
+            float Mall = -INFINITY;
+            for (int c = 0; c < nch; ++c) Mall = fmaxf(Mall, __ldcg(wb + (size_t)c * (HD + 2)));
+            for (int e = tid; e < HD; e += 128) {
+                float L = 0.f, s = 0.f;
+                for (int c = 0; c < nch; ++c) {
+                    const float mc = __ldcg(wb + (size_t)c * (HD + 2));
+                    if (mc == -INFINITY) continue;
+                    const float w = __expf(mc - Mall);
+                    L += __ldcg(wb + (size_t)c * (HD + 2) + 1) * w;
+                    s += __ldcg(wb + (size_t)c * (HD + 2) + 2 + e) * w;
+                }
+                a.attn[(size_t)b * a.d + (size_t)h * HD + e] = __float2bfloat16_rn(s / L);
+            }
+        }
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------- greedy choice
+__device__ bool amx_better(float v, int i, float bv, int bi) { return v > bv || (v == bv && i < bi); }
+
+template <int BN, int HD>
+__device__ void phase_argmax(const StepArgs& a, int tid, const Smem<BN, HD>& sm) {
+    const int nc = (a.V + AMX - 1) / AMX;
+    const int nitems = a.B * nc;
+    int* sidx = reinterpret_cast<int*>(sm.red + 8);
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+        const int b = item / nc, c = item - b * nc;
+        const float* p = a.logits + (size_t)b * a.V;
+        float best = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int i = c * AMX + tid; i < min(a.V, (c + 1) * AMX); i += 128) {
+            const float v = __ldcg(p + i);
+            if (amx_better(v, i, best, bi)) {
+                best = v;
+                bi = i;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (amx_better(ov, oi, best, bi)) {
+                best = ov;
+                bi = oi;
+            }
+        }
+        if ((tid & 31) == 0) {
+            sm.red[tid >> 5] = best;
+            sidx[tid >> 5] = bi;
+        }
+        esync();
+        if (tid == 0) {
+            for (int k = 1; k < 4; ++k)
+                if (amx_better(sm.red[k], sidx[k], best, bi)) {
+                    best = sm.red[k];
+                    bi = sidx[k];
+                }
+            a.amax_part[(size_t)b * nc + c] = make_int2(__float_as_int(best), bi);
+            __threadfence();
+            const int prev = atomicAdd(a.amax_cnt + b, 1);
+            if (prev == nc - 1) {
+                a.amax_cnt[b] = 0;
+                __threadfence();
+                float fb = -INFINITY;
+                int fi = 0x7fffffff;
+                for (int k = 0; k < nc; ++k) {
+                    const int2 e = __ldcg(a.amax_part + (size_t)b * nc + k);
+                    if (amx_better(__int_as_float(e.x), e.y, fb, fi)) {
+                        fb = __int_as_float(e.x);
+                        fi = e.y;
+                    }
+                }
+                a.tok[b] = (fi == 0x7fffffff) ? 0 : fi;
+                // the last row to finish advances the position
+                __threadfence();
+                const int rows = atomicAdd(a.amax_cnt + a.B, 1);
+                if (rows == a.B - 1) {
+                    a.amax_cnt[a.B] = 0;
+                    *a.d_pos += 1;
+                }
+            }
+        }
+        esync();
+    }
+}
+
+// ---------------------------------------------------------------- the kernel
+template <int BN, int HD>
+__global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
+    using C = SCfg<BN, HD>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base_s = (raw + 1023u) & ~1023u;
+    uint8_t* gb = smem_raw + (base_s - raw);
+    Smem<BN, HD> sm;
+    sm.sA = base_s + C::OFF_A;
+    sm.sB = base_s + C::OFF_B;
+    sm.att = gb + C::OFF_ATT;
+    sm.xbuf = reinterpret_cast<float*>(gb + C::OFF_X);
+    sm.so = reinterpret_cast<float*>(gb + C::OFF_SO);
+    sm.sm = reinterpret_cast<float*>(gb + C::OFF_SML);
+    sm.sl = sm.sm + 16;
+    sm.red = sm.sm + 32;
+    const uint32_t bars = base_s + C::OFF_BAR;
+    sm.full = bars;
+    sm.empty = bars + 8 * C::STAGES;
+    sm.tfull = bars + 16 * C::STAGES;
+    sm.tempty = sm.tfull + 16;
+    sm.abar = sm.tempty + 16;                                       // [ANB]
+    uint32_t* misc = reinterpret_cast<uint32_t*>(gb + C::OFF_BAR + 16 * C::STAGES + 32 + 8 * ANB);
+    uint32_t* tmem_slot = misc;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+    sm.flag = reinterpret_cast<volatile int*>(misc + 2);
+    volatile unsigned* base_gen = reinterpret_cast<volatile unsigned*>(misc + 3);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int P = phase_count(a);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(sm.full + 8 * s, 1);
+            mbar_init(sm.empty + 8 * s, 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(sm.tfull + 8 * i, 1);
+            mbar_init(sm.tempty + 8 * i, 128);
+        }
+        for (int i = 0; i < ANB; ++i) mbar_init(sm.abar + 8 * i, 1);
+        *abort_flag = 0;
+        // no barrier of this launch can complete before every CTA arrives,
+        // so all CTAs read the same starting generation here
+        *base_gen = ld_acquire_u32(a.bar + 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const unsigned gen0 = *base_gen;
+
+    if (warp == 0) {
+        // -------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t ph = 0;
+            int ready = -1;
+            bool ok = true;
+            for (int p = 0; p < P && ok; ++p) {
+                int l;
+                const int type = phase_type(a, p, l);
+                GemmPh g;
+                if (!gemm_of(a, type, l, g)) continue;
+                const int mblk = g.rowsA / BM, kbt = g.K / BK, per = (kbt + g.splits - 1) / g.splits;
+                const int tiles = mblk * g.splits;
+                for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                    const int mb = t % mblk, sp = t / mblk;
+                    const int kb0 = sp * per, kb1 = min(kbt, kb0 + per);
+                    for (int kb = kb0; kb < kb1; ++kb) {
+                        if (!mbar_wait(sm.empty + 8 * stage, ph ^ 1u, abort_flag, a.err)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_expect_tx(sm.full + 8 * stage, C::STAGE_BYTES);
+                        tma_load_2d(sm.sA + stage * C::A_BYTES, a.maps + g.map_a, sm.full + 8 * stage, kb * BK,
+                                    mb * BM);
+                        if (ready < p) {
+                            if (!wait_gen(a.bar + 1, gen0 + (unsigned)p, abort_flag, a.err)) {
+                                ok = false;
+                                break;
+                            }
+                            asm volatile("fence.proxy.async.global;" ::: "memory");
+                            ready = p;
+                        }
+                        tma_load_2d(sm.sB + stage * C::B_BYTES, a.maps + g.map_b, sm.full + 8 * stage, kb * BK, 0);
+                        if (++stage == C::STAGES) {
+                            stage = 0;
+                            ph ^= 1u;
+                        }
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC = idesc_bf16(BN);
+            int stage = 0;
+            uint32_t ph = 0;
+            int acc = 0;
+            uint32_t acc_ph = 0;
+            bool ok = true;
+            for (int p = 0; p < P && ok; ++p) {
+                int l;
+                const int type = phase_type(a, p, l);
+                GemmPh g;
+                if (!gemm_of(a, type, l, g)) continue;
+                const int mblk = g.rowsA / BM, kbt = g.K / BK, per = (kbt + g.splits - 1) / g.splits;
+                const int tiles = mblk * g.splits;
+                for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                    const int sp = t / mblk;
+                    const int kb0 = sp * per, kb1 = min(kbt, kb0 + per);
+                    if (!mbar_wait(sm.tempty + 8 * acc, acc_ph ^ 1u, abort_flag, a.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+                    for (int kb = kb0; kb < kb1; ++kb) {
+                        if (!mbar_wait(sm.full + 8 * stage, ph, abort_flag, a.err)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t da = sw128_desc(sm.sA + stage * C::A_BYTES);
+                        const uint64_t db = sw128_desc(sm.sB + stage * C::B_BYTES);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k)
+                            umma_bf16(d_tmem, da + 2 * k, db + 2 * k, IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
+                        umma_commit(sm.empty + 8 * stage);
+                        if (++stage == C::STAGES) {
+                            stage = 0;
+                            ph ^= 1u;
+                        }
+                    }
+                    if (!ok) break;
+                    umma_commit(sm.tfull + 8 * acc);
+                    if (++acc == 2) {
+                        acc = 0;
+                        acc_ph ^= 1u;
+                    }
+                }
+            }
+        }
+    } else {
+        // -------------------------------------------------------- epilogue warps 2..5
+        const int tid = threadIdx.x - 64;
+        const int quarter = warp & 3;
+        const int et = quarter * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        int acc = 0;
+        uint32_t acc_ph = 0;
+        uint32_t uses[ANB];
+#pragma unroll
+        for (int i = 0; i < ANB; ++i) uses[i] = 0;
+        for (int p = 0; p < P; ++p) {
+            int l;
+            const int type = phase_type(a, p, l);
+            if (p > 0) {
+                const bool ok = wait_gen(a.bar + 1, gen0 + (unsigned)p, abort_flag, a.err);
+                if (esync_any(!ok)) break;
+            }
+            bool fail = false;
+            if (type == PH_EMBED) {
+                if ((int)blockIdx.x < a.B) {
+                    const int b = blockIdx.x;
+                    int t = a.tok[b];
+                    if (t < 0 || t >= a.V) {
+                        if (tid == 0) atomicOr(a.err, 2);
+                        t = 0;
+                    }
+                    const bf16* e = a.embed + (size_t)t * a.d;
+                    float* x = a.trunk + (size_t)b * a.d;
+                    for (int i = tid; i < a.d; i += 128) x[i] = __bfloat162float(e[i]);
+                    __threadfence_block();
+                    esync();
+                    // RMSNorm of this row with layer 0's attention gain
+                    float ss = 0.f;
+                    for (int i = tid * 4; i < a.d; i += 512) {
+                        const float4 v = *reinterpret_cast<const float4*>(x + i);
+                        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+                    }
+                    const float inv = rsqrtf(esum(ss, sm.red, tid) / (float)a.d + a.eps);
+                    const float* gg = a.gains[0];
+                    for (int i = tid * 4; i < a.d; i += 512) {
+                        const float4 v = *reinterpret_cast<const float4*>(x + i);
+                        const float4 gv = *reinterpret_cast<const float4*>(gg + i);
+                        *reinterpret_cast<uint2*>(a.xn + (size_t)b * a.d + i) = make_uint2(
+                            pack_bf16x2(v.x * inv * gv.x, v.y * inv * gv.y), pack_bf16x2(v.z * inv * gv.z, v.w * inv * gv.w));
+                    }
+                }
+            } else if (type == PH_ATTN) {
+                fail = !phase_attn<BN, HD>(a, l, tid, sm, uses, abort_flag);
+            } else if (type == PH_ARGMAX) {
+                phase_argmax<BN, HD>(a, tid, sm);
+            } else {
+                GemmPh g;
+                gemm_of(a, type, l, g);
+                EpiArgs ep;
+                ep.M = a.B;
+                ep.N = g.rowsA;
+                ep.out = (type == PH_HEAD) ? a.logits : a.trunk;
+                ep.ld_out = (type == PH_HEAD) ? a.V : a.d;
+                ep.partial = a.partial;
+                ep.counters = a.counters;
+                ep.act = a.act;
+                ep.hidden = a.h;
+                ep.q = a.q;
+                ep.kc = a.kv + (size_t)(2 * l) * a.kv_layer;
+                ep.vc = a.kv + (size_t)(2 * l + 1) * a.kv_layer;
+                ep.rope = a.rope;
+                ep.d_pos = a.d_pos;
+                ep.S = 1;
+                ep.H = a.H;
+                ep.hd = a.hd;
+                ep.d = a.d;
+                ep.smax = a.smax;
+                const int mblk = g.rowsA / BM;
+                const int tiles = mblk * g.splits;
+                for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+                    const int mb = t % mblk, sp = t / mblk;
+                    const bool ok = mbar_wait(sm.tfull + 8 * acc, acc_ph, abort_flag, a.err);
+                    if (esync_any(!ok)) {
+                        fail = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    float v[32];
+                    const uint32_t tacc = tmem + lane_addr + (uint32_t)(acc * BN);
+                    if constexpr (BN == 16) tmem_ld16(tacc, v);
+                    else tmem_ld32(tacc, v);
+                    tc_fence_before();
+                    mbar_arrive(sm.tempty + 8 * acc);
+                    if (++acc == 2) {
+                        acc = 0;
+                        acc_ph ^= 1u;
+                    }
+                    switch (g.mode) {
+                        case EPI_QKV: tile_epilogue<BN, HD, EPI_QKV>(a, ep, g, l, type, mb, sp, et, tid, v, sm); break;
+                        case EPI_RESID: tile_epilogue<BN, HD, EPI_RESID>(a, ep, g, l, type, mb, sp, et, tid, v, sm); break;
+                        case EPI_SWIGLU: tile_epilogue<BN, HD, EPI_SWIGLU>(a, ep, g, l, type, mb, sp, et, tid, v, sm); break;
+                        default: tile_epilogue<BN, HD, EPI_F32>(a, ep, g, l, type, mb, sp, et, tid, v, sm); break;
+                    }
+                }
+            }
+            if (esync_any(fail)) break;
+            if (p + 1 < P && tid == 0) grid_arrive(a.bar, gen0 + (unsigned)p + 1u);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+}
+
+template <int BN, int HD>
+int launch_step_t(const StepArgs& a, cudaStream_t st) {
+    using C = SCfg<BN, HD>;
+    static bool attr = false;
+    if (!attr) {
+        LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<BN, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            C::SMEM));
+        attr = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(tc_num_sms());
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr_c[1];
+    attr_c[0].id = cudaLaunchAttributeCooperative;
+    attr_c[0].val.cooperative = 1;
+    cfg.attrs = attr_c;
+    cfg.numAttrs = 1;
+    LLAMA_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_step_kernel<BN, HD>, a));
+    llama_count_launches(1);
+    return LLAMA_OK;
+}
+
+}  // namespace
+
+int decode_step_prepare() {
+    int n = 0;
+    LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        SCfg<16, 128>::SMEM));
+    LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<32, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        SCfg<32, 128>::SMEM));
+    LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<16, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        SCfg<16, 64>::SMEM));
+    LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<32, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        SCfg<32, 64>::SMEM));
+    // one CTA per SM must fit for the cooperative launch
+    LLAMA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_step_kernel<32, 128>, NT,
+                                                                 SCfg<32, 128>::SMEM));
+    return n >= 1 ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int launch_decode_step(const StepArgs& a, cudaStream_t st) {
+    if (a.B <= 0 || a.B > 32) return LLAMA_ERR_INVALID_ARG;
+    if (a.hd == 128) return a.B <= 16 ? launch_step_t<16, 128>(a, st) : launch_step_t<32, 128>(a, st);
+    if (a.hd == 64) return a.B <= 16 ? launch_step_t<16, 64>(a, st) : launch_step_t<32, 64>(a, st);
+    return LLAMA_ERR_INVALID_ARG;
+}
+
+// Tensor-map table for the decode step: 4 per layer (W_qkv, W_o, W_gu, W_d),
+// the head, then the activation buffers xn, attn, act with `B` rows.
+int decode_step_maps(CUtensorMap* host_maps, const void* const* w, int L, const void* head, const void* xn,
+                     const void* attn, const void* act, int B, int d, int h, int V) {
+    int rc;
+    const int bn = B <= 16 ? 16 : 32;
+    for (int l = 0; l < L; ++l) {
+        if ((rc = tc_make_map_2d(&host_maps[4 * l + 0], w[4 * l + 0], 3 * d, d, BM))) return rc;
+        if ((rc = tc_make_map_2d(&host_maps[4 * l + 1], w[4 * l + 1], d, d, BM))) return rc;
+        if ((rc = tc_make_map_2d(&host_maps[4 * l + 2], w[4 * l + 2], 2 * h, d, BM))) return rc;
+        if ((rc = tc_make_map_2d(&host_maps[4 * l + 3], w[4 * l + 3], d, h, BM))) return rc;
+    }
+    if ((rc = tc_make_map_2d(&host_maps[4 * L + 0], head, V, d, BM))) return rc;
+    if ((rc = tc_make_map_2d(&host_maps[4 * L + 1], xn, B, d, bn))) return rc;
+    if ((rc = tc_make_map_2d(&host_maps[4 * L + 2], attn, B, d, bn))) return rc;
+    return tc_make_map_2d(&host_maps[4 * L + 3], act, B, h, bn);
+}

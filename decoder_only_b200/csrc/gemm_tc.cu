@@ -8,17 +8,8 @@
 //
 //   prefill (swap = 0): A = activations [tokens, K], B = weights [N, K],
 //                       tile 128 x 256, fused epilogue on the output tile.
-//   decode  (swap = 1): A = weights [N, K], B = activations [batch, K]
-//                       (batch <= 32, zero-filled to 16 or 32 rows by TMA),
-//                       tile 128 x {16, 32}, split over K to fill the SMs.
-//                       Each split leaves its fp32 partial tile in a
-//                       workspace and bumps a per-tile counter; the CTA that
-//                       arrives last sums the partials in split order
-//                       (deterministic) and applies the epilogue, so no
-//                       second kernel runs.  Gate and up tiles of the same
-//                       128 SwiGLU units share one counter.  Weight
-//                       streaming is HBM-bound: deep TMA ring, grid sized to
-//                       the SM count.
+//   (the decode projections, with the batch as N, run inside the fused
+//   decode step of decode_step.cu)
 //
 // Warp roles (192 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer (one elected lane): stage ring of S slots
@@ -49,28 +40,9 @@ struct Cfg {
     static constexpr int A_BYTES = BM * BK * 2;            // 16 KB
     static constexpr int B_BYTES = BN * BK * 2;            // BN * 128 B
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    // decode tiles (BN 16 / 32) keep their footprint under half an SM so a
-    // second decode GEMM can be resident and prefetch its weights early
-    static constexpr int STAGES = (BN >= 256) ? 4 : (BN == 16 ? 5 : 4);
-    static constexpr int TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;   // two accumulators, power of 2
-    static constexpr int XLD = BM + 1;                                // transpose buffer row (decode)
-    static constexpr int XBUF_BYTES = (BN < 256) ? 32 * XLD * 4 : 0;
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + XBUF_BYTES;
-};
-
-// Bounded barrier of the 128 epilogue threads (an mbarrier with 128
-// arrivals): false when the CTA is aborting.
-struct EpiSync {
-    uint32_t bar;
-    uint32_t phase;
-    volatile int* abort_flag;
-    int* err;
-    __device__ __forceinline__ bool sync() {
-        mbar_arrive(bar);
-        const bool ok = mbar_wait(bar, phase, abort_flag, err);
-        phase ^= 1u;
-        return ok;
-    }
+    static constexpr int STAGES = 4;
+    static constexpr int TMEM_COLS = 2 * BN;                          // two accumulators
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
 
 struct TileSched {
@@ -98,96 +70,7 @@ struct TileSched {
     }
 };
 
-// Decode epilogue of one 128-feature tile (et = the TMEM lane the thread
-// read, so it owns feature mb*128 + et for every batch row): write the
-// split's partial, let the last split to arrive finish the tile.  Runs on
-// the 128 epilogue threads only.
 template <int BN, int MODE>
-__device__ __forceinline__ bool epilogue_swap(const EpiArgs& ep, const TileSched& ts, int mb, int sp, int et,
-                                              const float (&v)[32], float* xbuf, volatile int* last_flag,
-                                              EpiSync& es) {
-    constexpr bool PAIR = (MODE == EPI_SWIGLU);      // gate tile 2j and up tile 2j+1 finish together
-    const int n = mb * BM + et;
-    const int M = ep.M, N = ep.N;
-    const bool direct = (ts.splits == 1) && !PAIR;
-    if (!direct) {
-        if (n < N) {
-            float* dst = ep.partial + (size_t)sp * M * N + n;
-#pragma unroll
-            for (int b = 0; b < BN; ++b)
-                if (b < M) dst[(size_t)b * N] = v[b];
-        }
-        __threadfence();
-        if (!es.sync()) return false;
-        if (et == 0) {
-            const int cidx = PAIR ? (mb >> 1) : mb;
-            const int target = PAIR ? 2 * ts.splits : ts.splits;
-            const int prev = atomicAdd(ep.counters + cidx, 1);
-            const int last = (prev == target - 1);
-            if (last) ep.counters[cidx] = 0;     // ready for the next launch
-            *last_flag = last;
-        }
-        if (!es.sync()) return false;
-        const int last = *last_flag;
-        if (!es.sync()) return false;            // everyone has read the flag
-        if (!last) return true;
-        __threadfence();
-    }
-    if constexpr (PAIR) {
-        // hidden units 128j + et from gate row 256j + et and up row 256j + 128 + et
-        const int j = mb >> 1;
-        const float* pg = ep.partial + 256 * j + et;
-        const float* pu = pg + 128;
-        for (int b = 0; b < M; ++b) {
-            float g = 0.f, u = 0.f;
-            for (int s = 0; s < ts.splits; ++s) {
-                g += __ldcg(pg + (size_t)s * M * N + (size_t)b * N);
-                u += __ldcg(pu + (size_t)s * M * N + (size_t)b * N);
-            }
-            reinterpret_cast<bf16*>(ep.act)[(size_t)b * ep.hidden + 128 * j + et] = __float2bfloat16_rn(silu_f(g) * u);
-        }
-    } else {
-        float sum[32];
-#pragma unroll
-        for (int b = 0; b < 32; ++b) sum[b] = direct ? v[b] : 0.f;
-        if (!direct && n < N) {
-            for (int s = 0; s < ts.splits; ++s) {
-                const float* p = ep.partial + (size_t)s * M * N + n;
-#pragma unroll
-                for (int b = 0; b < BN; ++b)
-                    if (b < M) sum[b] += __ldcg(p + (size_t)b * N);
-            }
-        }
-        if constexpr (MODE == EPI_RESID || MODE == EPI_F32) {
-            if (n < N) {
-#pragma unroll
-                for (int b = 0; b < BN; ++b) {
-                    if (b < M) {
-                        float* o = ep.out + (size_t)b * ep.ld_out + n;
-                        if constexpr (MODE == EPI_RESID) *o += sum[b];
-                        else *o = sum[b];
-                    }
-                }
-            }
-        } else {
-            // Q/K/V: 32-feature chunks of one token row through shared memory
-#pragma unroll
-            for (int b = 0; b < BN; ++b) xbuf[b * Cfg<BN>::XLD + et] = sum[b];
-            if (!es.sync()) return false;
-            if (et < 4 * M) {
-                const int b = et >> 2, c = et & 3;
-                float w[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) w[i] = xbuf[b * Cfg<BN>::XLD + c * 32 + i];
-                epi_qkv32<bf16>(ep, b, mb * BM + c * 32, w);
-            }
-            if (!es.sync()) return false;
-        }
-    }
-    return true;
-}
-
-template <int BN, int MODE, bool SWAP>
 __global__ void __launch_bounds__(NTHREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TileSched ts,
                    EpiArgs ep, int* err) {
@@ -205,9 +88,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tempty_bar = tfull_bar + 16;                 // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::STAGES * C::STAGE_BYTES + 16 * C::STAGES + 32);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
-    const uint32_t epi_bar_addr = tempty_bar + 32;                  // 128-thread epilogue barrier
-    float* xbuf = reinterpret_cast<float*>(gbase + C::STAGES * C::STAGE_BYTES + 256);   // [32][XLD] (decode)
+
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_launch_dependents();
@@ -221,7 +102,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(tfull_bar + 8 * i, 1);
             mbar_init(tempty_bar + 8 * i, 128);
         }
-        mbar_init(epi_bar_addr, 128);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
@@ -241,17 +121,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        // The weight operand (A in decode, B in prefill) does not depend on
-        // the kernels before this one: the weight tiles of the first stages
-        // are requested before waiting for the predecessor, the activation
-        // tiles after it.
+        // The weight operand (B) does not depend on the kernels before this
+        // one: the weight tiles of the first stages are requested before
+        // waiting for the predecessor, the activation tiles after it.
         if (lane == 0) {
-            const CUtensorMap* w_map = SWAP ? &tmA : &tmB;
-            const CUtensorMap* x_map = SWAP ? &tmB : &tmA;
-            const uint32_t w_base = SWAP ? sA : sB;
-            const uint32_t x_base = SWAP ? sB : sA;
-            const int w_bytes = SWAP ? C::A_BYTES : C::B_BYTES;
-            const int x_bytes = SWAP ? C::B_BYTES : C::A_BYTES;
+            const CUtensorMap* w_map = &tmB;     // weights
+            const CUtensorMap* x_map = &tmA;     // activations
+            const uint32_t w_base = sB;
+            const uint32_t x_base = sA;
+            const int w_bytes = C::B_BYTES;
+            const int x_bytes = C::A_BYTES;
             int stage = 0;
             uint32_t phase = 0;
             uint32_t filled = 0, fill_phase = 0;   // per-stage: filled at least once / parity of last fill
@@ -261,7 +140,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 int mb, nb, sp, kb0, kb1;
                 ts.get(blockIdx.x, mb, nb, sp, kb0, kb1);
                 pre = min(C::STAGES, kb1 - kb0);
-                const int w_row = SWAP ? mb * BM : nb * BN;
+                const int w_row = nb * BN;
                 for (int i = 0; i < pre; ++i) {    // fresh ring: every stage starts empty
                     mbar_expect_tx(full_bar + 8 * i, C::STAGE_BYTES);
                     tma_load_2d(w_base + i * w_bytes, w_map, full_bar + 8 * i, (kb0 + i) * BK, w_row);
@@ -273,8 +152,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
                 int mb, nb, sp, kb0, kb1;
                 ts.get(t, mb, nb, sp, kb0, kb1);
-                const int w_row = SWAP ? mb * BM : nb * BN;
-                const int x_row = SWAP ? nb * BN : mb * BM;
+                const int w_row = nb * BN;
+                const int x_row = mb * BM;
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     if (it >= pre) {
                         if (!mbar_wait(empty_bar + 8 * stage, phase ^ 1u, abort_flag, err)) {
@@ -350,7 +229,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         int acc = 0;
         uint32_t acc_phase = 0;
-        EpiSync es{epi_bar_addr, 0u, abort_flag, err};
         pdl_wait();
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
             int mb, nb, sp, kb0, kb1;
@@ -359,21 +237,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc_fence_after();
             const uint32_t tacc = tmem_base + lane_addr + (uint32_t)(acc * BN);
             const int row = mb * BM + quarter * 32 + lane;   // row of operand A
-            if constexpr (SWAP) {
-                // row = output feature; TMEM columns = batch rows
-                float v[32];
-                if constexpr (BN == 16) tmem_ld16(tacc, v);
-                else tmem_ld32(tacc, v);
-                tc_fence_before();
-                mbar_arrive(tempty_bar + 8 * acc);       // accumulator free for the next tile
-                if (++acc == 2) {
-                    acc = 0;
-                    acc_phase ^= 1u;
-                }
-                // feature within the tile = the TMEM lane this thread read
-                if (!epilogue_swap<BN, MODE>(ep, ts, mb, sp, quarter * 32 + lane, v, xbuf, last_flag, es)) break;
-                continue;
-            } else if constexpr (MODE == EPI_SWIGLU) {
+            if constexpr (MODE == EPI_SWIGLU) {
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     float g[32], u[32];
@@ -452,26 +316,26 @@ int num_sms() {
     return n;
 }
 
-template <int BN, int MODE, bool SWAP>
+template <int BN, int MODE>
 int ensure_attr() {
     static bool attr = false;
     if (!attr) {
-        LLAMA_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, MODE, SWAP>,
+        LLAMA_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, MODE>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::SMEM));
         attr = true;
     }
     return LLAMA_OK;
 }
 
-template <int BN, int MODE, bool SWAP>
+template <int BN, int MODE>
 int run(const CUtensorMap& ma, const CUtensorMap& mb, const TileSched& ts, const EpiArgs& a, int* err,
         cudaStream_t st) {
     using C = Cfg<BN>;
-    int rc = ensure_attr<BN, MODE, SWAP>();
+    int rc = ensure_attr<BN, MODE>();
     if (rc) return rc;
     const int tiles = ts.m_blocks * ts.n_blocks * ts.splits;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    launch_pdl(gemm_tc_kernel<BN, MODE, SWAP>, dim3(grid), dim3(NTHREADS), C::SMEM, st, ma, mb, ts, a, err);
+    launch_pdl(gemm_tc_kernel<BN, MODE>, dim3(grid), dim3(NTHREADS), C::SMEM, st, ma, mb, ts, a, err);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }
@@ -482,18 +346,10 @@ int gemm_tc_prepare() {
     if (!encode_fn()) return LLAMA_ERR_CUDA;
     num_sms();
     int rc;
-    if ((rc = ensure_attr<256, EPI_F32, false>())) return rc;
-    if ((rc = ensure_attr<256, EPI_RESID, false>())) return rc;
-    if ((rc = ensure_attr<256, EPI_SWIGLU, false>())) return rc;
-    if ((rc = ensure_attr<256, EPI_QKV, false>())) return rc;
-    if ((rc = ensure_attr<16, EPI_F32, true>())) return rc;
-    if ((rc = ensure_attr<16, EPI_RESID, true>())) return rc;
-    if ((rc = ensure_attr<16, EPI_SWIGLU, true>())) return rc;
-    if ((rc = ensure_attr<16, EPI_QKV, true>())) return rc;
-    if ((rc = ensure_attr<32, EPI_F32, true>())) return rc;
-    if ((rc = ensure_attr<32, EPI_RESID, true>())) return rc;
-    if ((rc = ensure_attr<32, EPI_SWIGLU, true>())) return rc;
-    return ensure_attr<32, EPI_QKV, true>();
+    if ((rc = ensure_attr<256, EPI_F32>())) return rc;
+    if ((rc = ensure_attr<256, EPI_RESID>())) return rc;
+    if ((rc = ensure_attr<256, EPI_SWIGLU>())) return rc;
+    return ensure_attr<256, EPI_QKV>();
 }
 
 int gemm_tc_pick_splits(int rowsA, int K) {
@@ -525,34 +381,7 @@ int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaSt
     TileSched ts;
     ts.kb_total = g.K / BK;
     ts.group = 16;
-    if (g.swap) {
-        if (g.rowsB > 32) return LLAMA_ERR_INVALID_ARG;
-        if ((g.splits > 1 || mode == EPI_SWIGLU) && (!a.partial || !a.counters)) return LLAMA_ERR_INVALID_ARG;
-        if (g.rowsA % BM != 0) return LLAMA_ERR_INVALID_ARG;   // whole 128-feature tiles
-        const int bn = g.rowsB <= 16 ? 16 : 32;
-        ts.m_blocks = (g.rowsA + BM - 1) / BM;
-        ts.n_blocks = 1;
-        ts.splits = g.splits < 1 ? 1 : (g.splits > ts.kb_total ? ts.kb_total : g.splits);
-        // every split must own at least one k-block
-        while (ts.splits > 1 && (ts.splits - 1) * ((ts.kb_total + ts.splits - 1) / ts.splits) >= ts.kb_total)
-            --ts.splits;
-        if (ts.splits != g.splits) return LLAMA_ERR_INVALID_ARG;
-        int rc = make_map(&ma, g.A, g.rowsA, g.K, BM);
-        if (rc) return rc;
-        rc = make_map(&mb, g.B, g.rowsB, g.K, bn);
-        if (rc) return rc;
-#define SWAP_CASE(BNV)                                                      \
-    switch (mode) {                                                         \
-        case EPI_F32: return run<BNV, EPI_F32, true>(ma, mb, ts, a, err, st);       \
-        case EPI_RESID: return run<BNV, EPI_RESID, true>(ma, mb, ts, a, err, st);   \
-        case EPI_SWIGLU: return run<BNV, EPI_SWIGLU, true>(ma, mb, ts, a, err, st); \
-        case EPI_QKV: return run<BNV, EPI_QKV, true>(ma, mb, ts, a, err, st);       \
-        default: return LLAMA_ERR_INVALID_ARG;                              \
-    }
-        if (bn == 16) SWAP_CASE(16);
-        SWAP_CASE(32);
-#undef SWAP_CASE
-    }
+    if (g.swap) return LLAMA_ERR_INVALID_ARG;   // decode projections run in decode_step.cu
     constexpr int BN = 256;
     ts.m_blocks = (g.rowsA + BM - 1) / BM;
     ts.n_blocks = (g.rowsB + BN - 1) / BN;
@@ -564,10 +393,16 @@ int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaSt
     rc = make_map(&mb, g.B, g.rowsB, g.K, BN);
     if (rc) return rc;
     switch (mode) {
-        case EPI_F32: return run<BN, EPI_F32, false>(ma, mb, ts, a, err, st);
-        case EPI_RESID: return run<BN, EPI_RESID, false>(ma, mb, ts, a, err, st);
-        case EPI_SWIGLU: return run<BN, EPI_SWIGLU, false>(ma, mb, ts, a, err, st);
-        case EPI_QKV: return run<BN, EPI_QKV, false>(ma, mb, ts, a, err, st);
+        case EPI_F32: return run<BN, EPI_F32>(ma, mb, ts, a, err, st);
+        case EPI_RESID: return run<BN, EPI_RESID>(ma, mb, ts, a, err, st);
+        case EPI_SWIGLU: return run<BN, EPI_SWIGLU>(ma, mb, ts, a, err, st);
+        case EPI_QKV: return run<BN, EPI_QKV>(ma, mb, ts, a, err, st);
         default: return LLAMA_ERR_INVALID_ARG;
     }
 }
+
+int tc_make_map_2d(CUtensorMap* map, const void* ptr, int rows, int K, int box_rows) {
+    return make_map(map, ptr, rows, K, box_rows);
+}
+
+int tc_num_sms() { return num_sms(); }

@@ -2,6 +2,8 @@
 // queues work on `st` and returns a llama_status.
 #pragma once
 
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -60,4 +62,38 @@ struct TcGemm {
 };
 int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaStream_t st);
 int gemm_tc_pick_splits(int rowsA, int K);
+
+// decode_step.cu  (one cooperative kernel per greedy decode step, bf16)
+struct StepArgs {
+    const CUtensorMap* maps;      // device table: 4 per layer (W_qkv, W_o, W_gu, W_d), head, xn, attn, act
+    const float* const* gains;    // device table [2L + 1]: g_attn[l], g_ffn[l], ..., g_final
+    const __nv_bfloat16* embed;
+    __nv_bfloat16* kv;            // layer l: K at kv + 2l * kv_layer, V at kv + (2l + 1) * kv_layer
+    size_t kv_layer;
+    float* trunk;
+    __nv_bfloat16 *xn, *q, *attn, *act;
+    float* logits;
+    float* partial;               // split-K partials
+    int* counters;                // split-K arrival counters
+    int* tiles_done;              // finished tiles of a residual projection
+    float* attn_work;             // attention chunk partials [B*H][ceil(smax/64)][hd + 2]
+    int* attn_cnt;                // [B*H]
+    int2* amax_part;              // [B][ceil(V/2048)]
+    int* amax_cnt;                // [B + 1]
+    int32_t* tok;
+    int* d_pos;
+    int* err;
+    unsigned int* bar;            // grid barrier: [0] arrivals, [1] generation
+    const float2* rope;
+    int L, d, h, V, H, hd, B, smax;
+    float eps;
+    int splits[5];                // qkv, o, gate/up, down, head
+};
+int decode_step_prepare();
+int launch_decode_step(const StepArgs& a, cudaStream_t st);
+int decode_step_maps(CUtensorMap* host_maps, const void* const* w, int L, const void* head, const void* xn,
+                     const void* attn, const void* act, int B, int d, int h, int V);
+// 2-D K-major bf16 tensor map, box (64, box_rows), 128-byte swizzle, zero fill
+int tc_make_map_2d(CUtensorMap* map, const void* ptr, int rows, int K, int box_rows);
+int tc_num_sms();
 int gemm_tc_prepare();  // sets kernel attributes; call before any stream capture

@@ -154,6 +154,11 @@ struct llama_model {
     size_t partial_elems;
     int* counters;           // split-K arrival counters (zero between launches)
     int* attn_cnt;           // decode-attention arrival counters [max_batch * H]
+    CUtensorMap* step_maps;  // decode-step tensor-map table (device) [4L + 4]
+    const float** step_gains;  // decode-step gain table (device) [2L + 1]
+    unsigned int* step_bar;  // decode-step grid barrier [2]
+    int* tiles_done;         // decode-step finished residual tiles
+    float* step_attn_work;   // decode-step attention partials
     int2* amax_part;         // greedy-choice chunk results [max_batch][chunks]
     int* amax_cnt;           // and their arrival counters [max_batch]
     float* attn_work;
@@ -188,7 +193,7 @@ int validate(const llama_config* c) {
         if (c->head_dim != 64 && c->head_dim != 128) return LLAMA_ERR_INVALID_ARG;
         if (c->d_model % 256 != 0) return LLAMA_ERR_INVALID_ARG;
         if (c->max_batch > 32) return LLAMA_ERR_INVALID_ARG;
-        if (c->vocab % 4 != 0) return LLAMA_ERR_INVALID_ARG;
+        if (c->vocab % 128 != 0) return LLAMA_ERR_INVALID_ARG;   // whole 128-row head tiles
     } else {
         if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return LLAMA_ERR_INVALID_ARG;
     }
@@ -244,8 +249,14 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     float* partial = (float*)take(c->dtype == LLAMA_BF16 ? pmax * 4 : 0);
     int* counters = (int*)take(MAX_COUNTERS * 4);
     int* attn_cnt = (int*)take((size_t)c->max_batch * c->n_heads * 4);
+    CUtensorMap* step_maps = (CUtensorMap*)take((size_t)(4 * L + 4) * sizeof(CUtensorMap));
+    const float** step_gains = (const float**)take((size_t)(2 * L + 1) * sizeof(float*));
+    unsigned int* step_bar = (unsigned int*)take(256);
+    int* tiles_done = (int*)take(256);
+    float* step_attn_work = (float*)take((size_t)c->max_batch * c->n_heads * ((c->max_seq + 63) / 64) *
+                                         (c->head_dim + 2) * 4);
     int2* amax_part = (int2*)take((size_t)c->max_batch * argmax_split_chunks(c->vocab) * sizeof(int2));
-    int* amax_cnt = (int*)take((size_t)c->max_batch * 4);
+    int* amax_cnt = (int*)take((size_t)(c->max_batch + 1) * 4);
     const uint64_t awb = attention_decode_work_bytes(c->max_batch, c->n_heads, c->max_seq, c->head_dim);
     float* attn_work = (float*)take(awb);
     int32_t* tok_cur = (int32_t*)take((size_t)c->max_batch * 4);
@@ -271,6 +282,11 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
         m->counters = counters;
         m->amax_part = amax_part;
         m->attn_cnt = attn_cnt;
+        m->step_maps = step_maps;
+        m->step_gains = step_gains;
+        m->step_bar = step_bar;
+        m->tiles_done = tiles_done;
+        m->step_attn_work = step_attn_work;
         m->amax_cnt = amax_cnt;
         m->attn_work = attn_work;
         m->attn_work_bytes = awb;
@@ -317,9 +333,9 @@ EpiArgs base_args(llama_model* m, int M, int N) {
 }
 
 // One projection: out-op(A [M, K] . W [N, K]^T).  mode in EPI_*.
-// Prefill (decode = false): tcgen05 GEMM with the fused epilogue (bf16) or
-// SIMT GEMM + epilogue pass (fp32).  Decode: split-K swap-AB tcgen05 GEMM
-// into partials + reduction with the epilogue (bf16); SIMT for fp32.
+// bf16: tcgen05 GEMM with the fused epilogue (prefill; the bf16 decode step
+// is one fused kernel).  fp32: SIMT GEMM + epilogue pass (prefill and
+// decode).
 double out_bytes(int mode, int M, int N, int esz) {
     switch (mode) {
         case EPI_F32: return (double)M * N * 4;
@@ -350,18 +366,7 @@ int project(llama_model* m, const char* name, int mode, const void* A, const voi
             g.swap = 0;
             return launch_gemm_tc(g, mode, a, m->d_err, st);
         }
-        g.A = W;
-        g.B = A;
-        g.rowsA = N;
-        g.rowsB = M;
-        g.K = K;
-        g.splits = splits;
-        g.swap = 1;
-        EpiArgs pa = a;
-        pa.partial = m->partial;
-        pa.counters = m->counters;
-        prof::Scope ps(st, region, in_bytes + out_bytes(mode, M, N, m->esz), flops);
-        return launch_gemm_tc(g, mode, pa, m->d_err, st);
+        return LLAMA_ERR_INVALID_ARG;   // bf16 decode runs as one fused step (decode_step.cu)
     }
     // fp32 storage: SIMT GEMM
     prof::Scope ps(st, region, in_bytes + out_bytes(mode, M, N, m->esz), flops);
@@ -444,9 +449,90 @@ int run_head(llama_model* m, const float* x, int n, float* logits, bool decode, 
 }
 
 // Body of one decode step on the internal buffers: tok_cur -> tok_cur.
+// Arguments of the fused bf16 decode step for the current batch.
+StepArgs step_args(llama_model* m) {
+    const llama_config& c = m->cfg;
+    StepArgs a;
+    memset(&a, 0, sizeof(a));
+    a.maps = m->step_maps;
+    a.gains = m->step_gains;
+    a.embed = (const bf16*)m->embed;
+    a.kv = (bf16*)m->kv;
+    a.kv_layer = m->kv_layer_elems;
+    a.trunk = m->trunk;
+    a.xn = (bf16*)m->xn;
+    a.q = (bf16*)m->q;
+    a.attn = (bf16*)m->attn;
+    a.act = (bf16*)m->act;
+    a.logits = m->logits_dec;
+    a.partial = m->partial;
+    a.counters = m->counters;
+    a.tiles_done = m->tiles_done;
+    a.attn_work = m->step_attn_work;
+    a.attn_cnt = m->attn_cnt;
+    a.amax_part = m->amax_part;
+    a.amax_cnt = m->amax_cnt;
+    a.tok = m->tok_cur;
+    a.d_pos = m->d_pos;
+    a.err = m->d_err;
+    a.bar = m->step_bar;
+    a.rope = m->rope;
+    a.L = c.n_layers;
+    a.d = c.d_model;
+    a.h = c.ffn_hidden;
+    a.V = c.vocab;
+    a.H = c.n_heads;
+    a.hd = c.head_dim;
+    a.B = m->B;
+    a.smax = c.max_seq;
+    a.eps = c.norm_eps;
+    a.splits[0] = m->splits_qkv;
+    a.splits[1] = m->splits_o;
+    a.splits[2] = m->splits_gu;
+    a.splits[3] = m->splits_d;
+    a.splits[4] = m->splits_head;
+    return a;
+}
+
+// Tensor maps and gain pointers of the fused decode step (synchronous copy
+// into the arena; done before the step graph is captured).
+int step_tables(llama_model* m) {
+    const llama_config& c = m->cfg;
+    const int L = c.n_layers;
+    std::vector<CUtensorMap> maps((size_t)4 * L + 4);
+    std::vector<const void*> w((size_t)4 * L);
+    for (int l = 0; l < L; ++l) {
+        w[4 * l + 0] = m->layers[l].wqkv;
+        w[4 * l + 1] = m->layers[l].wo;
+        w[4 * l + 2] = m->layers[l].wgu;
+        w[4 * l + 3] = m->layers[l].wd;
+    }
+    int rc = decode_step_maps(maps.data(), w.data(), L, m->head, m->xn, m->attn, m->act, m->B, c.d_model,
+                              c.ffn_hidden, c.vocab);
+    if (rc) return rc;
+    std::vector<const float*> gains((size_t)2 * L + 1);
+    for (int l = 0; l < L; ++l) {
+        gains[2 * l] = m->layers[l].g_attn;
+        gains[2 * l + 1] = m->layers[l].g_ffn;
+    }
+    gains[2 * L] = m->g_final;
+    LLAMA_CUDA_TRY(cudaMemcpy(m->step_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
+    LLAMA_CUDA_TRY(cudaMemcpy(m->step_gains, gains.data(), gains.size() * sizeof(float*), cudaMemcpyHostToDevice));
+    return LLAMA_OK;
+}
+
 int decode_body(llama_model* m, cudaStream_t st) {
     const llama_config& c = m->cfg;
     int rc;
+    if (c.dtype == LLAMA_BF16) {
+        // weights + KV cache read + activations, once per step
+        const double d = c.d_model, h = c.ffn_hidden, L = c.n_layers, V = c.vocab;
+        const double wbytes = 2.0 * (L * (4 * d * d + 3 * d * h) + d * V);
+        const double kvbytes = 2.0 * 2.0 * L * m->B * (m->cur_len + 1) * d;
+        const double flops = 2.0 * m->B * (L * (4 * d * d + 3 * d * h) + d * V) + 4.0 * L * m->B * (m->cur_len + 1) * d;
+        prof::Scope ps(st, "decode_step", wbytes + kvbytes, flops);
+        return launch_decode_step(step_args(m), st);
+    }
     {
         prof::Scope ps(st, "decode_embed", (double)m->B * c.d_model * (4 + m->esz), 0.0);
         rc = launch_embed(c.dtype, m->tok_cur, m->embed, m->trunk, m->B, c.d_model, c.vocab, m->d_err, st);
@@ -472,6 +558,10 @@ int decode_once(llama_model* m, cudaStream_t st) {
 
 int ensure_graph(llama_model* m) {
     if (m->graph && m->graph_B == m->B) return LLAMA_OK;
+    if (m->cfg.dtype == LLAMA_BF16) {
+        int rc = step_tables(m);
+        if (rc) return rc;
+    }
     if (m->graph) {
         cudaGraphExecDestroy(m->graph);
         m->graph = nullptr;
@@ -604,7 +694,8 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
         return LLAMA_ERR_CUDA;
     }
     if (cudaMemsetAsync(m->counters, 0, MAX_COUNTERS * 4, st) != cudaSuccess ||
-        cudaMemsetAsync(m->amax_cnt, 0, (size_t)cfg->max_batch * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(m->amax_cnt, 0, (size_t)(cfg->max_batch + 1) * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(m->step_bar, 0, 256, st) != cudaSuccess || cudaMemsetAsync(m->tiles_done, 0, 256, st) != cudaSuccess ||
         cudaMemsetAsync(m->attn_cnt, 0, (size_t)cfg->max_batch * cfg->n_heads * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->d_pos, 0, 256, st) != cudaSuccess) {
         llama_free(m);
@@ -612,7 +703,7 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
     }
     pick_decode_splits(m);
     if ((rc = gemm_tc_prepare()) || (rc = attention_prepare()) || (rc = attention_tc_prepare()) ||
-        (rc = attention_decode_prepare())) {
+        (rc = attention_decode_prepare()) || (cfg->dtype == LLAMA_BF16 && (rc = decode_step_prepare()))) {
         llama_free(m);
         return rc;
     }
