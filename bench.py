@@ -129,6 +129,36 @@ def algorithmic_work(shape, B, S, steps):
     return gemm + attn, wbytes + kv
 
 
+PHASE_NAMES = ["embed", "qkv", "attention", "o_proj", "gate_up", "down", "head", "argmax"]
+
+
+def step_phases(tl, n_layers):
+    """Per phase type of the fused decode step: summed critical-path time
+    (first start to last end over the CTAs) and the barrier gaps after each
+    phase (last end to the next phase's first start), in microseconds."""
+    import numpy as np
+    start = tl[:, :, 0].astype(np.float64)
+    end = tl[:, :, 1].astype(np.float64)
+    P = tl.shape[1]
+    s0, e1 = start.min(0), end.max(0)
+    out = {n: 0.0 for n in PHASE_NAMES}
+    gaps = 0.0
+    for p in range(P):
+        if p == 0:
+            name = "embed"
+        elif p - 1 < 5 * n_layers:
+            name = PHASE_NAMES[1 + (p - 1) % 5]
+        else:
+            name = "head" if p - 1 == 5 * n_layers else "argmax"
+        out[name] += (e1[p] - s0[p]) / 1e3
+        if p + 1 < P:
+            gaps += (s0[p + 1] - e1[p]) / 1e3
+    res = {k: round(v, 1) for k, v in out.items()}
+    res["barrier_gaps"] = round(gaps, 1)
+    res["total"] = round((e1[-1] - s0[0]) / 1e3, 1)
+    return res
+
+
 def kernel_family(region: str) -> str:
     if region.startswith("prefill_gemm"):
         return "gemm_tc prefill (tcgen05, fused epilogues)"
@@ -355,6 +385,9 @@ def run_b200(args, wl, shape):
     prof = lb.profile_read()
     lb.profile_enable(False)
     roof = roofline(prof, steps / max(prof_steps, 1), peaks, peak_src)
+    phases = None
+    if shape.dtype == "bf16" and steps:
+        phases = step_phases(model.step_timeline(), shape.n_layers)
 
     if rank == 0:
         flops_pre, bytes_dec = algorithmic_work(shape, B, S, steps)
@@ -376,6 +409,8 @@ def run_b200(args, wl, shape):
                                       ms_per_step=round(split["decode_ms"] / steps, 4),
                                       gbs=round(bytes_dec * steps / dec_s / 1e9, 1),
                                       frac_hbm=round(bytes_dec * steps / dec_s / 1e9 / peaks["hbm_gbs"], 4))
+        if phases:
+            line["decode_step_phases_us"] = phases
         if e2e_ms is not None:
             line["e2e"] = dict(value=round(world * tokens_step * args.steps / (e2e_ms * 1e-3), 2), unit=UNIT,
                                h2d_bytes_per_step=B * S * 4, d2h_bytes_per_step=B * steps * 4)

@@ -62,6 +62,7 @@ def _load():
         "llama_rewind": [P, I, P],
         "llama_complete": [P, P, I, I, P, I, P, P],
         "llama_kernel_launches": [],
+        "llama_step_timeline": [P, P, ctypes.c_int64, P, P],
         "llama_profile_enable": [I],
         "llama_profile_reset": [],
         "llama_profile_count": [],
@@ -214,6 +215,17 @@ class Model:
         if shape is not None:
             t = t[: int(torch.Size(shape).numel())].view(shape)
         return t
+
+    def step_timeline(self):
+        """[ctas, phases, 2] ns stamps of the last decode step run while
+        profiling was enabled (bf16 models)."""
+        import numpy as np
+        c, p = ctypes.c_int32(), ctypes.c_int32()
+        _check(lib.llama_step_timeline(self.h, None, 0, ctypes.byref(c), ctypes.byref(p)), "llama_step_timeline")
+        out = np.zeros((c.value, p.value, 2), dtype=np.uint64)
+        _check(lib.llama_step_timeline(self.h, ctypes.c_void_p(out.ctypes.data), out.size, None, None),
+               "llama_step_timeline")
+        return out
 
     def last_error(self) -> int:
         return lib.llama_last_error(self.h)

@@ -44,8 +44,9 @@ using namespace tc;
 constexpr int BM = 128;      // weight rows per tile (TMEM lanes)
 constexpr int BK = 64;       // K per stage (one 128-byte swizzle row)
 constexpr int NT = 192;
-constexpr int ACH = 64;      // keys per attention item
-constexpr int ANB = 3;       // attention items in flight per CTA
+constexpr int ACH = 32;      // keys per attention chunk (one bulk copy of K rows, one of V rows)
+constexpr int SEG = 4;       // chunks per attention item: one warp, 128 keys of one (sequence, head)
+constexpr int SEGK = ACH * SEG;
 constexpr int AMX = 2048;    // logits per greedy-choice item
 
 enum PhaseType { PH_EMBED = 0, PH_QKV = 1, PH_ATTN = 2, PH_O = 3, PH_GU = 4, PH_DOWN = 5, PH_HEAD = 6, PH_ARGMAX = 7 };
@@ -58,12 +59,14 @@ struct SCfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-    static constexpr int OFF_ATT = OFF_B + STAGES * B_BYTES;             // [ANB][2][ACH][HD] bf16
+    // attention: per epilogue warp two chunk buffers (K rows then V rows);
+    // the Q/K/V transpose buffer of the QKV epilogue shares the region
     static constexpr int ATT_BUF = 2 * ACH * HD * 2;
-    static constexpr int OFF_X = OFF_ATT + ANB * ATT_BUF;               // [32][XLD] floats
+    static constexpr int OFF_ATT = OFF_B + STAGES * B_BYTES;             // [4 warps][2][ATT_BUF]
+    static constexpr int OFF_X = OFF_ATT;                                 // [32][XLD] floats
     static constexpr int XLD = BM + 1;
-    static constexpr int OFF_SO = OFF_X + 32 * XLD * 4;                   // [16][HD] floats
-    static constexpr int OFF_SML = OFF_SO + 16 * HD * 4;                  // m[16], l[16], red[16]
+    static constexpr int ATT_BYTES = 4 * 2 * ATT_BUF > 32 * XLD * 4 ? 4 * 2 * ATT_BUF : 32 * XLD * 4;
+    static constexpr int OFF_SML = OFF_ATT + ATT_BYTES;                   // reduction scratch
     static constexpr int OFF_BAR = OFF_SML + 256;
     static constexpr int SMEM = OFF_BAR + 512 + 1024;
     static constexpr uint32_t TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
@@ -107,34 +110,6 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     return v;
 }
 
-// Bounded wait until the grid barrier generation reaches `target`.
-__device__ bool wait_gen(const unsigned* gen, unsigned target, volatile int* abort_flag, int* err) {
-    if ((int)(ld_acquire_u32(gen) - target) >= 0) return true;
-    const uint64_t t0 = global_timer();
-    while (true) {
-        if ((int)(ld_acquire_u32(gen) - target) >= 0) return true;
-        if (*abort_flag) return false;
-        if (global_timer() - t0 > WAIT_LIMIT_NS) {
-            *abort_flag = 1;
-            atomicOr(err, LLAMA_DEVERR_TIMEOUT);
-            return false;
-        }
-        __nanosleep(32);
-    }
-}
-
-// One arrival per CTA; the last one resets the count and publishes the next
-// generation.
-__device__ void grid_arrive(unsigned* bar, unsigned next_gen) {
-    __threadfence();
-    const unsigned prev = atomicAdd(bar, 1u);
-    if (prev == gridDim.x - 1) {
-        atomicExch(bar, 0u);
-        __threadfence();
-        atomicExch(bar + 1, next_gen);
-    }
-}
-
 // Named barrier of the 128 epilogue threads
 __device__ __forceinline__ void esync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 // ... that also returns whether any of them failed (all leave together)
@@ -149,6 +124,48 @@ __device__ __forceinline__ bool esync_any(bool fail) {
         : "r"((uint32_t)fail)
         : "memory");
     return r != 0;
+}
+
+// Grid barrier state: bar[0] counts arrivals; CTA i polls its own release
+// flag bar[32 + 32 i] (a 128-byte line of its own), which the last CTA to
+// arrive sets to the next generation.
+__device__ __forceinline__ unsigned* bar_flag(unsigned* bar, int cta) { return bar + 32 + 32 * cta; }
+
+// Bounded wait until this CTA's release flag reaches generation `target`.
+__device__ bool wait_gen(const unsigned* flag, unsigned target, volatile int* abort_flag, int* err) {
+    if ((int)(ld_acquire_u32(flag) - target) >= 0) return true;
+    const uint64_t t0 = global_timer();
+    while (true) {
+        if ((int)(ld_acquire_u32(flag) - target) >= 0) return true;
+        if (*abort_flag) return false;
+        if (global_timer() - t0 > WAIT_LIMIT_NS) {
+            *abort_flag = 1;
+            atomicOr(err, LLAMA_DEVERR_TIMEOUT);
+            return false;
+        }
+        __nanosleep(20);
+    }
+}
+
+// Arrival of this CTA (all 128 epilogue threads call it after their work);
+// the last CTA to arrive resets the count and releases every CTA's flag.
+__device__ void grid_arrive(unsigned* bar, unsigned next_gen, int tid, volatile int* last_flag) {
+    if (tid == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(bar, 1u);
+        const int last = (prev == gridDim.x - 1);
+        if (last) {
+            atomicExch(bar, 0u);
+            __threadfence();
+        }
+        *last_flag = last;
+    }
+    esync();
+    if (*last_flag) {
+        for (int i = tid; i < (int)gridDim.x; i += 128)
+            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(bar_flag(bar, i)), "r"(next_gen) : "memory");
+    }
+    esync();
 }
 
 __device__ __forceinline__ float esum(float v, float* red, int tid) {
@@ -187,9 +204,6 @@ struct Smem {
     uint32_t full, empty, tfull, tempty, abar;
     uint8_t* att;        // generic pointer to the attention buffers
     float* xbuf;
-    float* so;
-    float* sm;           // [16] maxima
-    float* sl;           // [16] sums
     float* red;          // [16] reduction scratch
     volatile int* flag;
 };
@@ -295,24 +309,33 @@ __device__ bool tile_epilogue(const StepArgs& a, const EpiArgs& ep, const GemmPh
 }
 
 // ---------------------------------------------------------------- attention phase
+// Each epilogue warp works alone: an item is 128 keys (4 chunks of 32) of
+// one (sequence b, head h); the warp streams its chunks through two shared
+// buffers of its own (bulk copies, the next chunk in flight while one is
+// computed), keeps the online-softmax state across the item, merges its four
+// lane groups with shuffles and leaves the item's (max, sum, output) in the
+// workspace; the warp that finishes the last item of (b, h) merges them.
+struct AttnCursor {
+    int j, c;   // item ordinal of this warp, chunk within the item
+};
+
 template <int BN, int HD>
-__device__ void issue_attn(const StepArgs& a, int l, int item, int nch, int len, int buf, const Smem<BN, HD>& sm) {
-    const int chunk = item % nch, bh = item / nch;
+__device__ __forceinline__ void attn_issue(const StepArgs& a, int l, int item, int c, int nseg, int len,
+                                           uint32_t dst, uint32_t bar) {
+    const int seg = item % nseg, bh = item / nseg;
     const int b = bh / a.H, h = bh - b * a.H;
-    const int k0 = chunk * ACH;
+    const int k0 = seg * SEGK + c * ACH;
     const int nkeys = min(len - k0, ACH);
     const bf16* kc = a.kv + (size_t)(2 * l) * a.kv_layer;
     const bf16* vc = kc + a.kv_layer;
     const size_t off = (((size_t)b * a.H + h) * a.smax + k0) * HD;
     const uint32_t bytes = (uint32_t)(nkeys * HD * 2);
-    const uint32_t bar = sm.abar + 8 * buf;
-    const uint32_t dk = smem_u32(sm.att + (size_t)buf * SCfg<BN, HD>::ATT_BUF);
-    const uint32_t dv = dk + ACH * HD * 2;
     mbar_expect_tx(bar, 2 * bytes);
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dk),
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(kc + off), "r"(bytes), "r"(bar)
                  : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dv),
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst + ACH * HD * 2),
                  "l"(vc + off), "r"(bytes), "r"(bar)
                  : "memory");
 }
@@ -320,49 +343,43 @@ __device__ void issue_attn(const StepArgs& a, int l, int item, int nch, int len,
 template <int BN, int HD>
 __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>& sm, uint32_t* uses,
                            volatile int* abort_flag) {
-    constexpr int DPL = HD / 8;      // dims per lane: 16-byte vectors u = 0.., dims (u*8 + r)*8 ..
+    constexpr int DPL = HD / 8;      // dims per lane: 16-byte vectors u, dims (u*8 + r)*8 ..
     constexpr int NV = DPL / 8;
-    const int len = *a.d_pos + 1;
-    const int nch = (len + ACH - 1) / ACH;
-    const int nchmax = (a.smax + ACH - 1) / ACH;
-    const int nitems = nch * a.B * a.H;
-    int count = 0;
-    for (int i = blockIdx.x; i < nitems; i += gridDim.x) ++count;
-    if (tid == 0)
-        for (int j = 0; j < min(ANB, count); ++j) issue_attn<BN, HD>(a, l, blockIdx.x + j * gridDim.x, nch, len, j, sm);
+    constexpr int DPW = HD / 32;     // dims per lane in the final merge
     const int warp = tid >> 5, lane = tid & 31, g = lane >> 3, r = lane & 7;
+    const int len = *a.d_pos + 1;
+    const int nseg = (len + SEGK - 1) / SEGK;
+    const int nsegmax = (a.smax + SEGK - 1) / SEGK;
+    const int nitems = nseg * a.B * a.H;
+    const int gw = blockIdx.x * 4 + warp, nw = gridDim.x * 4;
+    auto item_of = [&](int j) { return gw + j * nw; };
+    auto chunks_of = [&](int it) {
+        const int seg = it % nseg;
+        return (min(SEGK, len - seg * SEGK) + ACH - 1) / ACH;
+    };
+    const uint32_t wbuf = smem_u32(sm.att) + warp * 2 * SCfg<BN, HD>::ATT_BUF;
+    const uint32_t wbar = sm.abar + warp * 16;
+    // issue the first two chunks
+    AttnCursor is{0, 0};
+    int issued = 0;
+    for (; issued < 2 && item_of(is.j) < nitems; ++issued) {
+        if (lane == 0)
+            attn_issue<BN, HD>(a, l, item_of(is.j), is.c, nseg, len, wbuf + (issued & 1) * SCfg<BN, HD>::ATT_BUF,
+                               wbar + 8 * (issued & 1));
+        if (++is.c == chunks_of(item_of(is.j))) {
+            ++is.j;
+            is.c = 0;
+        }
+    }
     const float scale = rsqrtf((float)HD);
-    for (int j = 0; j < count; ++j) {
-        const int item = blockIdx.x + j * gridDim.x;
-        const int buf = j % ANB;
-        const int chunk = item % nch, bh = item / nch;
+    float m = -INFINITY, lsum = 0.f, acc[DPL], qv[DPL];
+    int k = 0;
+    for (AttnCursor cur{0, 0}; item_of(cur.j) < nitems; ++k) {
+        const int item = item_of(cur.j);
+        const int seg = item % nseg, bh = item / nseg;
         const int b = bh / a.H, h = bh - b * a.H;
-        const int nkeys = min(len - chunk * ACH, ACH);
-        // wait for this item's K and V rows
-        const uint32_t bar = sm.abar + 8 * buf;
-        bool ok = false;
-        {
-            const uint64_t t0 = global_timer();
-            while (true) {
-                if (mbar_try_wait(bar, uses[buf] & 1u)) {
-                    ok = true;
-                    break;
-                }
-                if (*abort_flag || global_timer() - t0 > WAIT_LIMIT_NS) break;
-            }
-        }
-        uses[buf]++;
-        if (esync_any(!ok)) {
-            if (tid == 0) {
-                *abort_flag = 1;
-                atomicOr(a.err, LLAMA_DEVERR_TIMEOUT);
-            }
-            return false;
-        }
-        const bf16* sk = reinterpret_cast<const bf16*>(sm.att + (size_t)buf * SCfg<BN, HD>::ATT_BUF);
-        const bf16* sv = sk + ACH * HD;
-        float qv[DPL];
-        {
+        const int nkeys = min(len - (seg * SEGK + cur.c * ACH), ACH);
+        if (cur.c == 0) {    // a new item: its query and a fresh state
             const bf16* qp = a.q + ((size_t)b * a.H + h) * HD;
 #pragma unroll
             for (int u = 0; u < NV; ++u) {
@@ -375,13 +392,37 @@ __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>
                     qv[u * 8 + 2 * t + 1] = f.y * scale;
                 }
             }
+            m = -INFINITY;
+            lsum = 0.f;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
         }
-        float m = -INFINITY, lsum = 0.f, acc[DPL];
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-#pragma unroll
-        for (int i = 0; i < ACH / 16; ++i) {
-            const int key = warp * (ACH / 4) + 4 * i + g;
+        const int buf = k & 1;
+        const uint32_t bar = wbar + 8 * buf;
+        bool ok = false;
+        {
+            const uint64_t t0 = global_timer();
+            while (true) {
+                if (mbar_try_wait(bar, uses[buf] & 1u)) {
+                    ok = true;
+                    break;
+                }
+                if (*abort_flag || global_timer() - t0 > WAIT_LIMIT_NS) break;
+            }
+        }
+        uses[buf]++;
+        if (__any_sync(0xffffffffu, !ok)) {
+            if (lane == 0) {
+                *abort_flag = 1;
+                atomicOr(a.err, LLAMA_DEVERR_TIMEOUT);
+            }
+            return false;
+        }
+        const bf16* sk = reinterpret_cast<const bf16*>(sm.att + (size_t)(warp * 2 + buf) * SCfg<BN, HD>::ATT_BUF);
+        const bf16* sv = sk + ACH * HD;
+#pragma unroll 2
+        for (int i = 0; i < ACH / 4; ++i) {
+            const int key = 4 * i + g;
             const bool valid = key < nkeys;
             const int kr = valid ? key : 0;
             float kk[DPL], vv[DPL];
@@ -415,65 +456,78 @@ __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>
                 m = m_new;
             }
         }
-        // merge the 16 groups of this item into the chunk's partial
-        const int grp = warp * 4 + g;
-        if (r == 0) {
-            sm.sm[grp] = m;
-            sm.sl[grp] = lsum;
+        __syncwarp();
+        // the buffer is free: put the chunk two places ahead in flight
+        if (item_of(is.j) < nitems) {
+            if (lane == 0)
+                attn_issue<BN, HD>(a, l, item_of(is.j), is.c, nseg, len, wbuf + buf * SCfg<BN, HD>::ATT_BUF, bar);
+            if (++is.c == chunks_of(item_of(is.j))) {
+                ++is.j;
+                is.c = 0;
+            }
         }
-#pragma unroll
-        for (int u = 0; u < NV; ++u)
-#pragma unroll
-            for (int t = 0; t < 8; ++t) sm.so[grp * HD + (u * 8 + r) * 8 + t] = acc[u * 8 + t];
-        esync();
-        // the buffer has been read: refill it with the item ANB places ahead
-        if (tid == 0 && j + ANB < count) issue_attn<BN, HD>(a, l, blockIdx.x + (j + ANB) * gridDim.x, nch, len, buf, sm);
-        float M = -INFINITY;
-#pragma unroll
-        for (int t = 0; t < 16; ++t) M = fmaxf(M, sm.sm[t]);
-        float* wp = a.attn_work + ((size_t)bh * nchmax + chunk) * (HD + 2);
-        for (int c = tid; c < HD; c += 128) {
-            float s = 0.f;
-#pragma unroll
-            for (int t = 0; t < 16; ++t)
-                if (sm.sm[t] != -INFINITY) s += sm.so[t * HD + c] * __expf(sm.sm[t] - M);
-            wp[2 + c] = s;
+        const bool item_done = (cur.c + 1 == chunks_of(item));
+        if (++cur.c == chunks_of(item)) {
+            ++cur.j;
+            cur.c = 0;
         }
-        if (tid == 0) {
-            float L = 0.f;
+        if (!item_done) continue;
+        // merge the four lane groups (each covers every 4th key)
 #pragma unroll
-            for (int t = 0; t < 16; ++t)
-                if (sm.sm[t] != -INFINITY) L += sm.sl[t] * __expf(sm.sm[t] - M);
-            wp[0] = M;
-            wp[1] = L;
+        for (int off = 8; off <= 16; off <<= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+            const float l2 = __shfl_xor_sync(0xffffffffu, lsum, off);
+            const float M = fmaxf(m, m2);
+            const float c1 = (m == -INFINITY) ? 0.f : __expf(m - M);
+            const float c2 = (m2 == -INFINITY) ? 0.f : __expf(m2 - M);
+            lsum = lsum * c1 + l2 * c2;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) {
+                const float o2 = __shfl_xor_sync(0xffffffffu, acc[e], off);
+                acc[e] = acc[e] * c1 + o2 * c2;
+            }
+            m = M;
+        }
+        float* wp = a.attn_work + ((size_t)bh * nsegmax + seg) * (HD + 2);
+        if (g == 0) {
+#pragma unroll
+            for (int u = 0; u < NV; ++u)
+#pragma unroll
+                for (int t = 0; t < 8; ++t) wp[2 + (u * 8 + r) * 8 + t] = acc[u * 8 + t];
+            if (r == 0) {
+                wp[0] = m;
+                wp[1] = lsum;
+            }
         }
         __threadfence();
-        esync();
-        if (tid == 0) {
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
             const int prev = atomicAdd(a.attn_cnt + bh, 1);
-            const int last = (prev == nch - 1);
+            last = (prev == nseg - 1);
             if (last) a.attn_cnt[bh] = 0;
-            *sm.flag = last;
         }
-        esync();
-        const int last = *sm.flag;
-        esync();
+        last = __shfl_sync(0xffffffffu, last, 0);
         if (last) {
             __threadfence();
-            const float* wb = a.attn_work + (size_t)bh * nchmax * (HD + 2);
+            const float* wb = a.attn_work + (size_t)bh * nsegmax * (HD + 2);
             float Mall = -INFINITY;
-            for (int c = 0; c < nch; ++c) Mall = fmaxf(Mall, __ldcg(wb + (size_t)c * (HD + 2)));
-            for (int e = tid; e < HD; e += 128) {
-                float L = 0.f, s = 0.f;
-                for (int c = 0; c < nch; ++c) {
-                    const float mc = __ldcg(wb + (size_t)c * (HD + 2));
-                    if (mc == -INFINITY) continue;
-                    const float w = __expf(mc - Mall);
-                    L += __ldcg(wb + (size_t)c * (HD + 2) + 1) * w;
-                    s += __ldcg(wb + (size_t)c * (HD + 2) + 2 + e) * w;
-                }
-                a.attn[(size_t)b * a.d + (size_t)h * HD + e] = __float2bfloat16_rn(s / L);
+            for (int c = 0; c < nseg; ++c) Mall = fmaxf(Mall, __ldcg(wb + (size_t)c * (HD + 2)));
+            float L = 0.f, o[DPW];
+#pragma unroll
+            for (int e = 0; e < DPW; ++e) o[e] = 0.f;
+            for (int c = 0; c < nseg; ++c) {
+                const float* pc = wb + (size_t)c * (HD + 2);
+                const float mc = __ldcg(pc);
+                const float w = (mc == -INFINITY) ? 0.f : __expf(mc - Mall);
+                L += __ldcg(pc + 1) * w;
+#pragma unroll
+                for (int e = 0; e < DPW; ++e) o[e] += __ldcg(pc + 2 + lane * DPW + e) * w;
             }
+            const float inv = 1.f / L;
+            bf16* dst = a.attn + (size_t)b * a.d + (size_t)h * HD + lane * DPW;
+#pragma unroll
+            for (int e = 0; e < DPW; ++e) dst[e] = __float2bfloat16_rn(o[e] * inv);
         }
     }
     return true;
@@ -561,17 +615,14 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
     sm.sB = base_s + C::OFF_B;
     sm.att = gb + C::OFF_ATT;
     sm.xbuf = reinterpret_cast<float*>(gb + C::OFF_X);
-    sm.so = reinterpret_cast<float*>(gb + C::OFF_SO);
-    sm.sm = reinterpret_cast<float*>(gb + C::OFF_SML);
-    sm.sl = sm.sm + 16;
-    sm.red = sm.sm + 32;
+    sm.red = reinterpret_cast<float*>(gb + C::OFF_SML);
     const uint32_t bars = base_s + C::OFF_BAR;
     sm.full = bars;
     sm.empty = bars + 8 * C::STAGES;
     sm.tfull = bars + 16 * C::STAGES;
     sm.tempty = sm.tfull + 16;
-    sm.abar = sm.tempty + 16;                                       // [ANB]
-    uint32_t* misc = reinterpret_cast<uint32_t*>(gb + C::OFF_BAR + 16 * C::STAGES + 32 + 8 * ANB);
+    sm.abar = sm.tempty + 16;                                       // [4 warps][2]
+    uint32_t* misc = reinterpret_cast<uint32_t*>(gb + C::OFF_BAR + 16 * C::STAGES + 32 + 64);
     uint32_t* tmem_slot = misc;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
     sm.flag = reinterpret_cast<volatile int*>(misc + 2);
@@ -588,11 +639,11 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
             mbar_init(sm.tfull + 8 * i, 1);
             mbar_init(sm.tempty + 8 * i, 128);
         }
-        for (int i = 0; i < ANB; ++i) mbar_init(sm.abar + 8 * i, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(sm.abar + 8 * i, 1);
         *abort_flag = 0;
         // no barrier of this launch can complete before every CTA arrives,
         // so all CTAs read the same starting generation here
-        *base_gen = ld_acquire_u32(a.bar + 1);
+        *base_gen = ld_acquire_u32(bar_flag(a.bar, blockIdx.x));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -633,7 +684,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                         tma_load_2d(sm.sA + stage * C::A_BYTES, a.maps + g.map_a, sm.full + 8 * stage, kb * BK,
                                     mb * BM);
                         if (ready < p) {
-                            if (!wait_gen(a.bar + 1, gen0 + (unsigned)p, abort_flag, a.err)) {
+                            if (!wait_gen(bar_flag(a.bar, blockIdx.x), gen0 + (unsigned)p, abort_flag, a.err)) {
                                 ok = false;
                                 break;
                             }
@@ -708,16 +759,17 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         int acc = 0;
         uint32_t acc_ph = 0;
-        uint32_t uses[ANB];
-#pragma unroll
-        for (int i = 0; i < ANB; ++i) uses[i] = 0;
+        uint32_t uses[2] = {0u, 0u};
+        unsigned long long* tl = a.timeline ? a.timeline + (size_t)blockIdx.x * P * 2 : nullptr;
         for (int p = 0; p < P; ++p) {
             int l;
             const int type = phase_type(a, p, l);
             if (p > 0) {
-                const bool ok = wait_gen(a.bar + 1, gen0 + (unsigned)p, abort_flag, a.err);
+                bool ok = true;
+                if (tid == 0) ok = wait_gen(bar_flag(a.bar, blockIdx.x), gen0 + (unsigned)p, abort_flag, a.err);
                 if (esync_any(!ok)) break;
             }
+            if (tl && tid == 0) tl[2 * p] = global_timer();
             bool fail = false;
             if (type == PH_EMBED) {
                 if ((int)blockIdx.x < a.B) {
@@ -802,7 +854,8 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                 }
             }
             if (esync_any(fail)) break;
-            if (p + 1 < P && tid == 0) grid_arrive(a.bar, gen0 + (unsigned)p + 1u);
+            if (tl && tid == 0) tl[2 * p + 1] = global_timer();
+            if (p + 1 < P) grid_arrive(a.bar, gen0 + (unsigned)p + 1u, tid, sm.flag);
         }
     }
 

@@ -83,7 +83,8 @@ struct StepArgs {
     int32_t* tok;
     int* d_pos;
     int* err;
-    unsigned int* bar;            // grid barrier: [0] arrivals, [1] generation
+    unsigned int* bar;            // grid barrier: [0] arrivals, [32 + 32 i] release flag of CTA i
+    unsigned long long* timeline; // optional: per CTA and phase, start / end %globaltimer stamps
     const float2* rope;
     int L, d, h, V, H, hd, B, smax;
     float eps;

@@ -159,6 +159,7 @@ struct llama_model {
     unsigned int* step_bar;  // decode-step grid barrier [2]
     int* tiles_done;         // decode-step finished residual tiles
     float* step_attn_work;   // decode-step attention partials
+    unsigned long long* step_timeline;   // decode-step phase stamps (while profiling)
     int2* amax_part;         // greedy-choice chunk results [max_batch][chunks]
     int* amax_cnt;           // and their arrival counters [max_batch]
     float* attn_work;
@@ -251,10 +252,12 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     int* attn_cnt = (int*)take((size_t)c->max_batch * c->n_heads * 4);
     CUtensorMap* step_maps = (CUtensorMap*)take((size_t)(4 * L + 4) * sizeof(CUtensorMap));
     const float** step_gains = (const float**)take((size_t)(2 * L + 1) * sizeof(float*));
-    unsigned int* step_bar = (unsigned int*)take(256);
+    unsigned int* step_bar = (unsigned int*)take(32 * 1024);   // arrivals + one 128-byte flag per CTA
     int* tiles_done = (int*)take(256);
-    float* step_attn_work = (float*)take((size_t)c->max_batch * c->n_heads * ((c->max_seq + 63) / 64) *
+    float* step_attn_work = (float*)take((size_t)c->max_batch * c->n_heads * ((c->max_seq + 127) / 128) *
                                          (c->head_dim + 2) * 4);
+    // per-phase timestamps of the fused decode step (profiling): 2 per CTA per phase
+    unsigned long long* step_timeline = (unsigned long long*)take((size_t)1024 * (3 + 5 * L) * 2 * 8);
     int2* amax_part = (int2*)take((size_t)c->max_batch * argmax_split_chunks(c->vocab) * sizeof(int2));
     int* amax_cnt = (int*)take((size_t)(c->max_batch + 1) * 4);
     const uint64_t awb = attention_decode_work_bytes(c->max_batch, c->n_heads, c->max_seq, c->head_dim);
@@ -287,6 +290,7 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
         m->step_bar = step_bar;
         m->tiles_done = tiles_done;
         m->step_attn_work = step_attn_work;
+        m->step_timeline = step_timeline;
         m->amax_cnt = amax_cnt;
         m->attn_work = attn_work;
         m->attn_work_bytes = awb;
@@ -531,7 +535,9 @@ int decode_body(llama_model* m, cudaStream_t st) {
         const double kvbytes = 2.0 * 2.0 * L * m->B * (m->cur_len + 1) * d;
         const double flops = 2.0 * m->B * (L * (4 * d * d + 3 * d * h) + d * V) + 4.0 * L * m->B * (m->cur_len + 1) * d;
         prof::Scope ps(st, "decode_step", wbytes + kvbytes, flops);
-        return launch_decode_step(step_args(m), st);
+        StepArgs sa = step_args(m);
+        if (prof::on) sa.timeline = m->step_timeline;
+        return launch_decode_step(sa, st);
     }
     {
         prof::Scope ps(st, "decode_embed", (double)m->B * c.d_model * (4 + m->esz), 0.0);
@@ -695,7 +701,8 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
     }
     if (cudaMemsetAsync(m->counters, 0, MAX_COUNTERS * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->amax_cnt, 0, (size_t)(cfg->max_batch + 1) * 4, st) != cudaSuccess ||
-        cudaMemsetAsync(m->step_bar, 0, 256, st) != cudaSuccess || cudaMemsetAsync(m->tiles_done, 0, 256, st) != cudaSuccess ||
+        cudaMemsetAsync(m->step_bar, 0, 32 * 1024, st) != cudaSuccess ||
+        cudaMemsetAsync(m->tiles_done, 0, 256, st) != cudaSuccess ||
         cudaMemsetAsync(m->attn_cnt, 0, (size_t)cfg->max_batch * cfg->n_heads * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->d_pos, 0, 256, st) != cudaSuccess) {
         llama_free(m);
@@ -950,6 +957,18 @@ int llama_op_argmax(const float* d_logits, int32_t rows, int32_t n, int32_t* d_o
 }
 
 int64_t llama_kernel_launches(void) { return g_launches.load(); }
+
+int llama_step_timeline(llama_model* m, uint64_t* h_out, int64_t n, int32_t* ctas, int32_t* phases) {
+    if (!m || m->cfg.dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+    const int P = 3 + 5 * m->cfg.n_layers, G = tc_num_sms();
+    if (ctas) *ctas = G;
+    if (phases) *phases = P;
+    const int64_t need = (int64_t)G * P * 2;
+    if (!h_out) return LLAMA_OK;
+    if (n < need) return LLAMA_ERR_INVALID_ARG;
+    LLAMA_CUDA_TRY(cudaMemcpy(h_out, m->step_timeline, (size_t)need * 8, cudaMemcpyDeviceToHost));
+    return LLAMA_OK;
+}
 
 int llama_profile_enable(int32_t on) {
     prof::on = on != 0;

@@ -183,6 +183,14 @@ LLAMA_API int llama_profile_count(void);
 LLAMA_API int llama_profile_entry(int32_t i, const char** name, double* ms, int64_t* launches,
                                   int64_t* calls, double* bytes, double* flops);
 
+/* Phase timestamps of the last bf16 decode step run while profiling was
+ * enabled: h_out (host) receives ctas * phases * 2 %globaltimer values
+ * (ns), [cta][phase][start, end]; phases run embed, then per layer QKV,
+ * attention, O, gate/up, down, then head and greedy choice.  With
+ * h_out == NULL only *ctas and *phases are filled.  Synchronous. */
+LLAMA_API int llama_step_timeline(llama_model* m, uint64_t* h_out, int64_t n, int32_t* ctas,
+                                  int32_t* phases);
+
 /* ------------------------------------------------------------ single ops
  * The kernels the model runs, exposed one by one on caller buffers.  dtype
  * selects fp32 or bf16 storage of the T-typed operands. */
