@@ -178,18 +178,18 @@ __device__ __forceinline__ float esum(float v, float* red, int tid) {
 }
 
 // RMSNorm of the B trunk rows into xn (bf16), by the 128 epilogue threads
-// of one CTA ("RMSNorm: LayerNorm minus the mean"; gain g).
-__device__ void norm_rows(const StepArgs& a, const float* g, float* red, int tid) {
-    const int d = a.d;
-    for (int b = 0; b < a.B; ++b) {
+// of one CTA, one warp per row ("RMSNorm: LayerNorm minus the mean"; gain g).
+__device__ void norm_rows(const StepArgs& a, const float* g, int tid) {
+    const int d = a.d, warp = tid >> 5, lane = tid & 31;
+    for (int b = warp; b < a.B; b += 4) {
         const float* x = a.trunk + (size_t)b * d;
         float ss = 0.f;
-        for (int i = tid * 4; i < d; i += 512) {
+        for (int i = lane * 4; i < d; i += 128) {
             const float4 v = __ldcg(reinterpret_cast<const float4*>(x + i));
             ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
         }
-        const float inv = rsqrtf(esum(ss, red, tid) / (float)d + a.eps);
-        for (int i = tid * 4; i < d; i += 512) {
+        const float inv = rsqrtf(warp_sum(ss) / (float)d + a.eps);
+        for (int i = lane * 4; i < d; i += 128) {
             const float4 v = __ldcg(reinterpret_cast<const float4*>(x + i));
             const float4 gg = *reinterpret_cast<const float4*>(g + i);
             *reinterpret_cast<uint2*>(a.xn + (size_t)b * d + i) =
@@ -209,19 +209,59 @@ struct Smem {
 };
 
 // ---------------------------------------------------------------- projection epilogue
+// Sum of one feature's split-K partials, stored contiguously [split][Mp]:
+// every load is independent, issued four splits at a time, summed in split
+// order (deterministic).
+template <int BN>
+__device__ __forceinline__ void splitk_sum(const float* p, int splits, int M, int Mp, float (&out)[BN]) {
+    constexpr int U = BN <= 16 ? 4 : 2;   // splits in flight per round (register budget)
+#pragma unroll
+    for (int b = 0; b < BN; ++b) out[b] = 0.f;
+    int s = 0;
+    for (; s + U <= splits; s += U) {
+        float4 w[U][BN / 4];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int q = 0; q < BN / 4; ++q)
+                w[u][q] = (4 * q < M) ? __ldcg(reinterpret_cast<const float4*>(p + (size_t)(s + u) * Mp + 4 * q))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int q = 0; q < BN / 4; ++q) {
+                out[4 * q] += w[u][q].x;
+                out[4 * q + 1] += w[u][q].y;
+                out[4 * q + 2] += w[u][q].z;
+                out[4 * q + 3] += w[u][q].w;
+            }
+    }
+    for (; s < splits; ++s)
+#pragma unroll
+        for (int q = 0; q < BN / 4; ++q)
+            if (4 * q < M) {
+                const float4 w = __ldcg(reinterpret_cast<const float4*>(p + (size_t)s * Mp + 4 * q));
+                out[4 * q] += w.x;
+                out[4 * q + 1] += w.y;
+                out[4 * q + 2] += w.z;
+                out[4 * q + 3] += w.w;
+            }
+}
+
 // One finished 128-feature tile (et = TMEM lane = feature within the tile).
 template <int BN, int HD, int MODE>
 __device__ bool tile_epilogue(const StepArgs& a, const EpiArgs& ep, const GemmPh& g, int l, int type, int mb,
                               int sp, int et, int tid, const float (&v)[32], const Smem<BN, HD>& sm) {
     constexpr bool PAIR = (MODE == EPI_SWIGLU);
     const int n = mb * BM + et;
-    const int M = a.B, N = g.rowsA;
+    const int M = a.B;
+    const int Mp = (M + 3) & ~3;             // partials: [feature][split][Mp], read back as float4
     const bool direct = (g.splits == 1) && !PAIR;
     if (!direct) {
-        float* dst = a.partial + (size_t)sp * M * N + n;
+        float* dst = a.partial + ((size_t)n * g.splits + sp) * Mp;
 #pragma unroll
-        for (int b = 0; b < BN; ++b)
-            if (b < M) dst[(size_t)b * N] = v[b];
+        for (int b = 0; b < BN; b += 4)
+            if (b < M) *reinterpret_cast<float4*>(dst + b) = make_float4(v[b], v[b + 1], v[b + 2], v[b + 3]);
         __threadfence();
         esync();
         if (tid == 0) {
@@ -239,29 +279,22 @@ __device__ bool tile_epilogue(const StepArgs& a, const EpiArgs& ep, const GemmPh
         __threadfence();
     }
     if constexpr (PAIR) {
+        // hidden units 128j + et from gate feature 256j + et and up feature 256j + 128 + et
         const int j = mb >> 1;
-        const float* pg = a.partial + 256 * j + et;
-        const float* pu = pg + 128;
-        for (int b = 0; b < M; ++b) {
-            float gsum = 0.f, usum = 0.f;
-            for (int s = 0; s < g.splits; ++s) {
-                gsum += __ldcg(pg + (size_t)s * M * N + (size_t)b * N);
-                usum += __ldcg(pu + (size_t)s * M * N + (size_t)b * N);
-            }
-            a.act[(size_t)b * a.h + 128 * j + et] = __float2bfloat16_rn(silu_f(gsum) * usum);
-        }
+        float gs[BN], us[BN];
+        splitk_sum<BN>(a.partial + (size_t)(256 * j + et) * g.splits * Mp, g.splits, M, Mp, gs);
+        splitk_sum<BN>(a.partial + (size_t)(256 * j + 128 + et) * g.splits * Mp, g.splits, M, Mp, us);
+#pragma unroll
+        for (int b = 0; b < BN; ++b)
+            if (b < M) a.act[(size_t)b * a.h + 128 * j + et] = __float2bfloat16_rn(silu_f(gs[b]) * us[b]);
         return true;
     } else {
-        float sum[32];
+        float sum[BN];
+        if (direct) {
 #pragma unroll
-        for (int b = 0; b < 32; ++b) sum[b] = direct ? v[b] : 0.f;
-        if (!direct) {
-            for (int s = 0; s < g.splits; ++s) {
-                const float* p = a.partial + (size_t)s * M * N + n;
-#pragma unroll
-                for (int b = 0; b < BN; ++b)
-                    if (b < M) sum[b] += __ldcg(p + (size_t)b * N);
-            }
+            for (int b = 0; b < BN; ++b) sum[b] = v[b];
+        } else {
+            splitk_sum<BN>(a.partial + (size_t)n * g.splits * Mp, g.splits, M, Mp, sum);
         }
         if constexpr (MODE == EPI_RESID || MODE == EPI_F32) {
 #pragma unroll
@@ -288,7 +321,7 @@ __device__ bool tile_epilogue(const StepArgs& a, const EpiArgs& ep, const GemmPh
                 if (last) {
                     __threadfence();
                     const float* gain = (type == PH_O) ? a.gains[2 * l + 1] : a.gains[2 * (l + 1)];
-                    norm_rows(a, gain, sm.red, tid);
+                    norm_rows(a, gain, tid);
                 }
             }
         } else {
@@ -511,19 +544,31 @@ __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>
         if (last) {
             __threadfence();
             const float* wb = a.attn_work + (size_t)bh * nsegmax * (HD + 2);
+            // lane c owns segment c (and c + 32, ...): maxima and weighted sums by shuffles
             float Mall = -INFINITY;
-            for (int c = 0; c < nseg; ++c) Mall = fmaxf(Mall, __ldcg(wb + (size_t)c * (HD + 2)));
+            for (int c = lane; c < nseg; c += 32) Mall = fmaxf(Mall, __ldcg(wb + (size_t)c * (HD + 2)));
+            Mall = warp_max(Mall);
             float L = 0.f, o[DPW];
 #pragma unroll
             for (int e = 0; e < DPW; ++e) o[e] = 0.f;
-            for (int c = 0; c < nseg; ++c) {
-                const float* pc = wb + (size_t)c * (HD + 2);
-                const float mc = __ldcg(pc);
-                const float w = (mc == -INFINITY) ? 0.f : __expf(mc - Mall);
-                L += __ldcg(pc + 1) * w;
+            for (int c0 = 0; c0 < nseg; c0 += 32) {
+                const int c = c0 + lane;
+                float w = 0.f;
+                if (c < nseg) {
+                    const float mc = __ldcg(wb + (size_t)c * (HD + 2));
+                    w = (mc == -INFINITY) ? 0.f : __expf(mc - Mall);
+                    L += __ldcg(wb + (size_t)c * (HD + 2) + 1) * w;
+                }
+                const int cn = min(32, nseg - c0);
+#pragma unroll 4
+                for (int t = 0; t < cn; ++t) {
+                    const float wt = __shfl_sync(0xffffffffu, w, t);
+                    const float* pc = wb + (size_t)(c0 + t) * (HD + 2) + 2 + lane * DPW;
 #pragma unroll
-                for (int e = 0; e < DPW; ++e) o[e] += __ldcg(pc + 2 + lane * DPW + e) * w;
+                    for (int e = 0; e < DPW; ++e) o[e] = fmaf(__ldcg(pc + e), wt, o[e]);
+                }
             }
+            L = warp_sum(L);
             const float inv = 1.f / L;
             bf16* dst = a.attn + (size_t)b * a.d + (size_t)h * HD + lane * DPW;
 #pragma unroll

@@ -246,7 +246,7 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     const size_t cmax = std::max(3 * d, 2 * h);
     float* gemm_c = (float*)take(c->dtype == LLAMA_F32 ? nmax * std::max(cmax, V) * 4 : 0);
     float* logits_dec = (float*)take((size_t)c->max_batch * V * 4);
-    const size_t pmax = (size_t)MAX_DEC_SPLITS * c->max_batch * std::max(cmax, V);
+    const size_t pmax = (size_t)MAX_DEC_SPLITS * ((c->max_batch + 3) & ~3) * std::max(cmax, V);
     float* partial = (float*)take(c->dtype == LLAMA_BF16 ? pmax * 4 : 0);
     int* counters = (int*)take(MAX_COUNTERS * 4);
     int* attn_cnt = (int*)take((size_t)c->max_batch * c->n_heads * 4);
