@@ -63,6 +63,7 @@ def _load():
         "llama_complete": [P, P, I, I, P, I, P, P],
         "llama_kernel_launches": [],
         "llama_step_timeline": [P, P, ctypes.c_int64, P, P],
+        "llama_debug_gemm_timeout": [P],
         "llama_profile_enable": [I],
         "llama_profile_reset": [],
         "llama_profile_count": [],

@@ -47,6 +47,7 @@ struct Cfg {
 
 struct TileSched {
     int m_blocks, n_blocks, splits, kb_total, group;
+    int skip_first_load;   // test hook: leave the first activation tile unrequested (its wait must expire)
     __device__ __forceinline__ int num_tiles() const { return m_blocks * n_blocks * splits; }
     // prefill: grouped raster (group m-blocks, n fastest inside a group); decode: m fastest
     __device__ __forceinline__ void get(int t, int& mb, int& nb, int& sp, int& kb0, int& kb1) const {
@@ -163,7 +164,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         mbar_expect_tx(full_bar + 8 * stage, C::STAGE_BYTES);
                         tma_load_2d(w_base + stage * w_bytes, w_map, full_bar + 8 * stage, kb * BK, w_row);
                     }
-                    tma_load_2d(x_base + stage * x_bytes, x_map, full_bar + 8 * stage, kb * BK, x_row);
+                    if (!(ts.skip_first_load && it == 0))
+                        tma_load_2d(x_base + stage * x_bytes, x_map, full_bar + 8 * stage, kb * BK, x_row);
                     filled |= 1u << stage;
                     fill_phase = (fill_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == C::STAGES) {
@@ -379,6 +381,7 @@ int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaSt
     if ((reinterpret_cast<uintptr_t>(g.A) | reinterpret_cast<uintptr_t>(g.B)) & 15u) return LLAMA_ERR_INVALID_ARG;
     CUtensorMap ma, mb;
     TileSched ts;
+    ts.skip_first_load = g.test_skip_load;
     ts.kb_total = g.K / BK;
     ts.group = 16;
     if (g.swap) return LLAMA_ERR_INVALID_ARG;   // decode projections run in decode_step.cu

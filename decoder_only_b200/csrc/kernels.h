@@ -58,7 +58,8 @@ struct TcGemm {
     const void* B;  // bf16 [rowsB, K]
     int rowsA, rowsB, K;
     int splits;     // split-K factor (decode only)
-    int swap;       // 0: A = tokens, B = weights; 1: A = weights, B = tokens (decode)
+    int swap;       // must be 0 (decode projections run in decode_step.cu)
+    int test_skip_load = 0;   // test hook (llama_debug_gemm_timeout)
 };
 int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaStream_t st);
 int gemm_tc_pick_splits(int rowsA, int K);

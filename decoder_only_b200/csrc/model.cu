@@ -951,6 +951,46 @@ int llama_op_attention_decode(int32_t dtype, const void* d_q, const void* d_k, c
                                    err, (cudaStream_t)stream);
 }
 
+int llama_debug_gemm_timeout(void* stream) {
+    // 128 x 256 x 64 GEMM whose only activation tile is never requested: the
+    // MMA warp's bounded wait on it must expire and the kernel must leave
+    // cleanly with LLAMA_DEVERR_TIMEOUT in the error word.
+    cudaStream_t st = (cudaStream_t)stream;
+    int* err = nullptr;
+    int rc = op_error_word(&err);
+    if (rc) return rc;
+    const size_t a_bytes = 128 * 64 * 2, w_bytes = 256 * 64 * 2, c_bytes = 128 * 256 * 4;
+    // operands of the self-test (zeros)
+    void* buf = nullptr;
+    LLAMA_CUDA_TRY(cudaMallocAsync(&buf, a_bytes + w_bytes + c_bytes, st));
+    LLAMA_CUDA_TRY(cudaMemsetAsync(buf, 0, a_bytes + w_bytes + c_bytes, st));
+    LLAMA_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(int), st));
+    TcGemm g;
+    g.A = buf;
+    g.B = (uint8_t*)buf + a_bytes;
+    g.rowsA = 128;
+    g.rowsB = 256;
+    g.K = 64;
+    g.splits = 1;
+    g.swap = 0;
+    g.test_skip_load = 1;
+    EpiArgs a;
+    memset(&a, 0, sizeof(a));
+    a.M = 128;
+    a.N = 256;
+    a.out = (float*)((uint8_t*)buf + a_bytes + w_bytes);
+    a.ld_out = 256;
+    rc = launch_gemm_tc(g, EPI_F32, a, err, st);
+    int e = 0;
+    LLAMA_CUDA_TRY(cudaMemcpyAsync(&e, err, sizeof(int), cudaMemcpyDeviceToHost, st));
+    LLAMA_CUDA_TRY(cudaStreamSynchronize(st));
+    LLAMA_CUDA_TRY(cudaFreeAsync(buf, st));
+    LLAMA_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(int), st));
+    LLAMA_CUDA_TRY(cudaStreamSynchronize(st));
+    if (rc) return rc;
+    return (e & LLAMA_DEVERR_TIMEOUT) ? LLAMA_ERR_TIMEOUT : LLAMA_OK;
+}
+
 int llama_op_argmax(const float* d_logits, int32_t rows, int32_t n, int32_t* d_out, void* stream) {
     if (!d_logits || !d_out || rows < 0 || n <= 0) return LLAMA_ERR_INVALID_ARG;
     return launch_argmax(d_logits, rows, n, n, d_out, (cudaStream_t)stream);

@@ -191,6 +191,14 @@ LLAMA_API int llama_profile_entry(int32_t i, const char** name, double* ms, int6
 LLAMA_API int llama_step_timeline(llama_model* m, uint64_t* h_out, int64_t n, int32_t* ctas,
                                   int32_t* phases);
 
+/* Failure-detection self-test (synchronous): runs one small tensor-core
+ * GEMM whose activation tile is never requested, so the kernel's bounded
+ * wait for it expires (about 2 s); the kernel records the timeout, frees
+ * its tensor memory and exits.  Returns LLAMA_ERR_TIMEOUT when the
+ * mechanism works (the CUDA context stays usable).  Allocates and frees its
+ * own 80 KB with cudaMallocAsync. */
+LLAMA_API int llama_debug_gemm_timeout(void* stream);
+
 /* ------------------------------------------------------------ single ops
  * The kernels the model runs, exposed one by one on caller buffers.  dtype
  * selects fp32 or bf16 storage of the T-typed operands. */

@@ -184,3 +184,15 @@ def test_argmax_lowest_index_on_ties():
     assert lb.argmax(x).tolist() == [5, 7, 0]
     y = torch.randn(16, 32000, device="cuda")
     assert torch.equal(lb.argmax(y).long(), torch.argmax(y, dim=-1))
+
+
+def test_bounded_wait_expires_and_the_context_survives():
+    """Failure detection: a GEMM whose activation tile is never requested
+    must give up after its bounded wait, report LLAMA_ERR_TIMEOUT, and leave
+    the context usable (a normal GEMM right after is correct)."""
+    assert lb.lib.llama_debug_gemm_timeout(lb._stream()) == -4
+    A, a64 = _normal_bf16(31, (256, 512))
+    W, w64 = _normal_bf16(32, (256, 512), 0.02)
+    C = lb.gemm(A, W)
+    ref = a64 @ w64.T
+    assert np.max(np.abs(C.cpu().numpy() - ref)) <= _acc_bound(512) * _rms(ref)
