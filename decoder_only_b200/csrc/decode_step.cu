@@ -4,33 +4,50 @@
 // keys and values of all earlier positions read from the cache ([NAR] "GQA
 // Was Not an Original LLaMA Feature")) is a chain of small, HBM-bound
 // phases:
-//   embed + RMSNorm
+//   embed (+ the first norm's inputs)
 //   per layer:  QKV projection (+RoPE, append K and V at the position)
 //               attention over the cache
-//               O projection (+residual, then RMSNorm of the updated trunk)
+//               O projection (+residual, + the FFN norm's inputs)
 //               gate/up projection (+SwiGLU)
-//               down projection (+residual, then the next RMSNorm)
+//               down projection (+residual, + the next norm's inputs)
 //   head projection (fp32 logits), greedy argmax, position + 1.
 // Launched one kernel per phase, fixed costs dominate (launch, set-up,
 // pipeline fill, tails).  Here one cooperative launch of one CTA per SM runs
 // all phases, separated by a grid-wide barrier; the weights -- which do not
-// depend on any phase -- stream continuously: the TMA producer requests the
-// weight tile of the next projection as soon as a ring slot frees, and only
-// the activation tile of each stage waits for the barrier that makes that
+// depend on any phase -- stream continuously: the TMA producer keeps its
+// ring of weight tiles full across phase boundaries, and only the
+// activation tile of each stage waits for the barrier that makes that
 // activation visible.
+//
+// Work split of a projection: its (128-row block, 64-wide k-block)
+// iterations, block-major, are cut into gridDim.x equal contiguous ranges
+// (stream-K), so every CTA streams the same number of weight bytes and
+// finishes at most a few accumulators per phase.  A block touched by one
+// range is finished directly from the accumulator; otherwise each range
+// leaves a partial sum and the last range to arrive adds them in range
+// order (deterministic) and finishes the block.
+//
+// RMSNorm ([PFD] "RMSNorm: LayerNorm minus the mean") enters a projection as
+// W (g * x / rms(x)).  1/rms(x) is one scalar per token, so it commutes with
+// W: the code that finishes a 128-feature block of the trunk x writes
+// bf16(g * x) and the block's sum of squares; the projection consuming the
+// norm multiplies its fp32 result by rsqrt(sum of the block sums / d + eps),
+// the block sums added in a fixed order.  No phase waits on a separate
+// normalisation pass over the whole trunk.
 //
 // Warp roles (192 threads):
 //   warp 0     TMA producer, all projections of the step in order
 //   warp 1     TMEM owner and tcgen05.mma issuer (swap-AB: 128 weight rows on
 //              the TMEM lanes, the B <= 32 tokens as N = 16 or 32 columns)
-//   warps 2-5  everything else: projection epilogues (split-K partials, the
-//              last split to arrive finishes the tile), attention, norms,
-//              greedy choice, and the arrivals at the grid barrier.
+//   warps 2-5  everything else: projection epilogues, attention, greedy
+//              choice, and the arrivals at the grid barrier.
 // Every wait is bounded (2 s): a CTA that gives up records
 // LLAMA_DEVERR_TIMEOUT and leaves; the others then give up at the next grid
 // barrier.  Named barriers among the 128 epilogue threads follow a
 // collective OR of each thread's wait result, so they leave together.
 #include <cuda.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "epilogue.cuh"
@@ -48,6 +65,7 @@ constexpr int ACH = 32;      // keys per attention chunk (one bulk copy of K row
 constexpr int SEG = 4;       // chunks per attention item: one warp, 128 keys of one (sequence, head)
 constexpr int SEGK = ACH * SEG;
 constexpr int AMX = 2048;    // logits per greedy-choice item
+constexpr int SSQ_BLOCKS = 64;   // 128-feature blocks of one norm's sums of squares (d <= 8192)
 
 enum PhaseType { PH_EMBED = 0, PH_QKV = 1, PH_ATTN = 2, PH_O = 3, PH_GU = 4, PH_DOWN = 5, PH_HEAD = 6, PH_ARGMAX = 7 };
 
@@ -60,14 +78,14 @@ struct SCfg {
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     // attention: per epilogue warp two chunk buffers (K rows then V rows);
-    // the Q/K/V transpose buffer of the QKV epilogue shares the region
+    // the transpose buffer of the projection epilogues shares the region
     static constexpr int ATT_BUF = 2 * ACH * HD * 2;
     static constexpr int OFF_ATT = OFF_B + STAGES * B_BYTES;             // [4 warps][2][ATT_BUF]
     static constexpr int OFF_X = OFF_ATT;                                 // [32][XLD] floats
     static constexpr int XLD = BM + 1;
     static constexpr int ATT_BYTES = 4 * 2 * ATT_BUF > 32 * XLD * 4 ? 4 * 2 * ATT_BUF : 32 * XLD * 4;
-    static constexpr int OFF_SML = OFF_ATT + ATT_BYTES;                   // reduction scratch
-    static constexpr int OFF_BAR = OFF_SML + 256;
+    static constexpr int OFF_SML = OFF_ATT + ATT_BYTES;                   // 1/rms [32], reduction scratch
+    static constexpr int OFF_BAR = OFF_SML + 1024;
     static constexpr int SMEM = OFF_BAR + 512 + 1024;
     static constexpr uint32_t TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
 };
@@ -88,20 +106,76 @@ __device__ __forceinline__ int phase_type(const StepArgs& a, int p, int& layer) 
     return q == 5 * a.L ? PH_HEAD : PH_ARGMAX;
 }
 
+// One projection: weight map, activation map, output rows, K, epilogue and
+// its kind (index of its partial / counter region)
 struct GemmPh {
-    int map_a, map_b, rowsA, K, splits, mode;
+    int map_a, map_b, rowsA, K, mode, kind;
 };
 
 __device__ __forceinline__ bool gemm_of(const StepArgs& a, int type, int l, GemmPh& g) {
     const int L = a.L;
     switch (type) {
-        case PH_QKV: g = GemmPh{4 * l + 0, 4 * L + 1, 3 * a.d, a.d, a.splits[0], EPI_QKV}; return true;
-        case PH_O: g = GemmPh{4 * l + 1, 4 * L + 2, a.d, a.d, a.splits[1], EPI_RESID}; return true;
-        case PH_GU: g = GemmPh{4 * l + 2, 4 * L + 1, 2 * a.h, a.d, a.splits[2], EPI_SWIGLU}; return true;
-        case PH_DOWN: g = GemmPh{4 * l + 3, 4 * L + 3, a.d, a.h, a.splits[3], EPI_RESID}; return true;
-        case PH_HEAD: g = GemmPh{4 * L, 4 * L + 1, a.V, a.d, a.splits[4], EPI_F32}; return true;
+        case PH_QKV: g = GemmPh{4 * l + 0, 4 * L + 1, 3 * a.d, a.d, EPI_QKV, 0}; return true;
+        case PH_O: g = GemmPh{4 * l + 1, 4 * L + 2, a.d, a.d, EPI_RESID, 1}; return true;
+        case PH_GU: g = GemmPh{4 * l + 2, 4 * L + 4, 2 * a.h, a.d, EPI_SWIGLU, 2}; return true;
+        case PH_DOWN: g = GemmPh{4 * l + 3, 4 * L + 3, a.d, a.h, EPI_RESID, 3}; return true;
+        case PH_HEAD: g = GemmPh{4 * L, 4 * L + 1, a.V, a.d, EPI_F32, 4}; return true;
         default: return false;
     }
+}
+
+// This CTA's stream-K range [s, e) of a projection's T = mblk * kbt
+// iterations (iteration i: block i / kbt, k-block i % kbt), cut into
+// G = min(gridDim.x, T) equal ranges so that none is empty; CTAs from G on
+// have no work in this projection.
+struct Work {
+    GemmPh g;
+    int mblk, kbt, s, e, G;
+    long long T;
+};
+
+__device__ __forceinline__ bool work_of(const StepArgs& a, int type, int l, Work& w) {
+    if (!gemm_of(a, type, l, w.g)) return false;
+    w.mblk = w.g.rowsA / BM;
+    w.kbt = w.g.K / BK;
+    w.T = (long long)w.mblk * w.kbt;
+    w.G = (int)min((long long)gridDim.x, w.T);
+    const int c = blockIdx.x;
+    w.s = c < w.G ? (int)(w.T * c / w.G) : 0;
+    w.e = c < w.G ? (int)(w.T * (c + 1) / w.G) : 0;
+    return true;
+}
+
+// The CTA whose range holds iteration i: the largest c with c*T/G <= i
+__device__ __forceinline__ int owner_of(long long i, const Work& w) { return (int)(((i + 1) * w.G - 1) / w.T); }
+
+// Walk over this CTA's projection iterations of the whole step, in order.
+struct Cursor {
+    int p, i, e, kbt, map_a, map_b;
+    bool valid;
+};
+
+__device__ void cursor_seek(const StepArgs& a, int P, Cursor& c, int p0) {
+    for (int p = p0; p < P; ++p) {
+        int l;
+        const int type = phase_type(a, p, l);
+        Work w;
+        if (!work_of(a, type, l, w) || w.s >= w.e) continue;
+        c.p = p;
+        c.i = w.s;
+        c.e = w.e;
+        c.kbt = w.kbt;
+        c.map_a = w.g.map_a;
+        c.map_b = w.g.map_b;
+        c.valid = true;
+        return;
+    }
+    c.valid = false;
+}
+
+__device__ __forceinline__ void cursor_next(const StepArgs& a, int P, Cursor& c) {
+    if (++c.i < c.e) return;
+    cursor_seek(a, P, c, c.p + 1);
 }
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
@@ -110,10 +184,23 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     return v;
 }
 
+// Non-blocking probe of an mbarrier phase
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Named barrier of the 128 epilogue threads
 __device__ __forceinline__ void esync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-// ... that also returns whether any of them failed (all leave together)
-__device__ __forceinline__ bool esync_any(bool fail) {
+// ... that also returns whether any of them passed true (all leave together)
+__device__ __forceinline__ bool esync_any(bool pred) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
@@ -121,7 +208,7 @@ __device__ __forceinline__ bool esync_any(bool fail) {
         "bar.red.or.pred p, 1, 128, q;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(r)
-        : "r"((uint32_t)fail)
+        : "r"((uint32_t)pred)
         : "memory");
     return r != 0;
 }
@@ -168,57 +255,42 @@ __device__ void grid_arrive(unsigned* bar, unsigned next_gen, int tid, volatile 
     esync();
 }
 
-__device__ __forceinline__ float esum(float v, float* red, int tid) {
-    v = warp_sum(v);
-    if ((tid & 31) == 0) red[tid >> 5] = v;
-    esync();
-    const float s = red[0] + red[1] + red[2] + red[3];
-    esync();
-    return s;
-}
-
-// RMSNorm of the B trunk rows into xn (bf16), by the 128 epilogue threads
-// of one CTA, one warp per row ("RMSNorm: LayerNorm minus the mean"; gain g).
-__device__ void norm_rows(const StepArgs& a, const float* g, int tid) {
-    const int d = a.d, warp = tid >> 5, lane = tid & 31;
-    for (int b = warp; b < a.B; b += 4) {
-        const float* x = a.trunk + (size_t)b * d;
-        float ss = 0.f;
-        for (int i = lane * 4; i < d; i += 128) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(x + i));
-            ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-        }
-        const float inv = rsqrtf(warp_sum(ss) / (float)d + a.eps);
-        for (int i = lane * 4; i < d; i += 128) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(x + i));
-            const float4 gg = *reinterpret_cast<const float4*>(g + i);
-            *reinterpret_cast<uint2*>(a.xn + (size_t)b * d + i) =
-                make_uint2(pack_bf16x2(v.x * inv * gg.x, v.y * inv * gg.y), pack_bf16x2(v.z * inv * gg.z, v.w * inv * gg.w));
-        }
-    }
-}
-
 template <int BN, int HD>
 struct Smem {
     uint32_t sA, sB;
     uint32_t full, empty, tfull, tempty, abar;
     uint8_t* att;        // generic pointer to the attention buffers
-    float* xbuf;
-    float* red;          // [16] reduction scratch
+    float* xbuf;         // [32][XLD] transpose buffer
+    float* sinv;         // [32] 1/rms of the B rows for the current projection
+    float* red;          // [128] reduction scratch
     volatile int* flag;
 };
 
+// 1/rms of each of the B rows from a norm's 128-feature block sums of
+// squares (added in block order by lane, then across the warp: the same
+// order in every CTA), into sinv.
+__device__ void load_inv(const StepArgs& a, const float* ssq, float* sinv, int tid) {
+    const int warp = tid >> 5, lane = tid & 31, nblk = a.d / BM;
+    for (int b = warp; b < a.B; b += 4) {
+        float s = 0.f;
+        for (int k = lane; k < nblk; k += 32) s += __ldcg(ssq + k * 32 + b);
+        s = warp_sum(s);
+        if (lane == 0) sinv[b] = rsqrtf(s / (float)a.d + a.eps);
+    }
+    esync();
+}
+
 // ---------------------------------------------------------------- projection epilogue
-// Sum of one feature's split-K partials, stored contiguously [split][Mp]:
-// every load is independent, issued four splits at a time, summed in split
-// order (deterministic).
+// Sum of one feature's partials, stored contiguously [slot][Mp]: every load
+// is independent, issued four slots at a time, summed in slot order
+// (deterministic).
 template <int BN>
-__device__ __forceinline__ void splitk_sum(const float* p, int splits, int M, int Mp, float (&out)[BN]) {
-    constexpr int U = BN <= 16 ? 4 : 2;   // splits in flight per round (register budget)
+__device__ __forceinline__ void splitk_sum(const float* p, int slots, int M, int Mp, float (&out)[BN]) {
+    constexpr int U = BN <= 16 ? 4 : 2;   // slots in flight per round (register budget)
 #pragma unroll
     for (int b = 0; b < BN; ++b) out[b] = 0.f;
     int s = 0;
-    for (; s + U <= splits; s += U) {
+    for (; s + U <= slots; s += U) {
         float4 w[U][BN / 4];
 #pragma unroll
         for (int u = 0; u < U; ++u)
@@ -236,7 +308,7 @@ __device__ __forceinline__ void splitk_sum(const float* p, int splits, int M, in
                 out[4 * q + 3] += w[u][q].w;
             }
     }
-    for (; s < splits; ++s)
+    for (; s < slots; ++s)
 #pragma unroll
         for (int q = 0; q < BN / 4; ++q)
             if (4 * q < M) {
@@ -248,96 +320,104 @@ __device__ __forceinline__ void splitk_sum(const float* p, int splits, int M, in
             }
 }
 
-// One finished 128-feature tile (et = TMEM lane = feature within the tile).
+// The accumulator of this CTA's range over block mb (et = TMEM lane =
+// feature within the block): leave it as a partial, or finish the block.
 template <int BN, int HD, int MODE>
-__device__ bool tile_epilogue(const StepArgs& a, const EpiArgs& ep, const GemmPh& g, int l, int type, int mb,
-                              int sp, int et, int tid, const float (&v)[32], const Smem<BN, HD>& sm) {
+__device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& w, int l, int type, int mb, int et,
+                              int tid, const float (&v)[32], const Smem<BN, HD>& sm) {
     constexpr bool PAIR = (MODE == EPI_SWIGLU);
-    const int n = mb * BM + et;
+    constexpr int XLD = SCfg<BN, HD>::XLD;
     const int M = a.B;
-    const int Mp = (M + 3) & ~3;             // partials: [feature][split][Mp], read back as float4
-    const bool direct = (g.splits == 1) && !PAIR;
+    const int Mp = (M + 3) & ~3;             // partials: [feature][slot][Mp], read back as float4
+    const int ns = step_slots(w.mblk, w.G);
+    auto first_of = [&](int m) { return owner_of((long long)m * w.kbt, w); };
+    auto nseg_of = [&](int m) { return owner_of((long long)(m + 1) * w.kbt - 1, w) - first_of(m) + 1; };
+    const int nseg = nseg_of(mb);
+    const int n = mb * BM + et;
+    float* part = a.partial + a.part_off[w.g.kind];
+    const bool direct = (nseg == 1) && !PAIR;
     if (!direct) {
-        float* dst = a.partial + ((size_t)n * g.splits + sp) * Mp;
+        float* dst = part + ((size_t)n * ns + ((int)blockIdx.x - first_of(mb))) * Mp;
 #pragma unroll
         for (int b = 0; b < BN; b += 4)
             if (b < M) *reinterpret_cast<float4*>(dst + b) = make_float4(v[b], v[b + 1], v[b + 2], v[b + 3]);
-        __threadfence();
         esync();
+        int last = 0;
         if (tid == 0) {
-            const int cidx = PAIR ? (mb >> 1) : mb;
-            const int target = PAIR ? 2 * g.splits : g.splits;
-            const int prev = atomicAdd(a.counters + cidx, 1);
-            const int last = (prev == target - 1);
-            if (last) a.counters[cidx] = 0;
-            *sm.flag = last;
+            int* cnt = a.counters + a.cnt_off[w.g.kind] + (PAIR ? (mb >> 1) : mb);
+            const int target = PAIR ? nseg_of(mb & ~1) + nseg_of(mb | 1) : nseg;
+            __threadfence();
+            const int prev = atomicAdd(cnt, 1);
+            last = (prev == target - 1);
+            if (last) {
+                *cnt = 0;
+                __threadfence();
+            }
         }
-        esync();
-        const int last = *sm.flag;
-        esync();
-        if (!last) return true;
-        __threadfence();
+        if (!esync_any(last)) return;
     }
     if constexpr (PAIR) {
         // hidden units 128j + et from gate feature 256j + et and up feature 256j + 128 + et
         const int j = mb >> 1;
         float gs[BN], us[BN];
-        splitk_sum<BN>(a.partial + (size_t)(256 * j + et) * g.splits * Mp, g.splits, M, Mp, gs);
-        splitk_sum<BN>(a.partial + (size_t)(256 * j + 128 + et) * g.splits * Mp, g.splits, M, Mp, us);
+        splitk_sum<BN>(part + (size_t)(256 * j + et) * ns * Mp, nseg_of(2 * j), M, Mp, gs);
+        splitk_sum<BN>(part + (size_t)(256 * j + 128 + et) * ns * Mp, nseg_of(2 * j + 1), M, Mp, us);
 #pragma unroll
         for (int b = 0; b < BN; ++b)
-            if (b < M) a.act[(size_t)b * a.h + 128 * j + et] = __float2bfloat16_rn(silu_f(gs[b]) * us[b]);
-        return true;
+            if (b < M) {
+                const float inv = sm.sinv[b];
+                a.act[(size_t)b * a.h + 128 * j + et] = __float2bfloat16_rn(silu_f(gs[b] * inv) * (us[b] * inv));
+            }
     } else {
         float sum[BN];
         if (direct) {
 #pragma unroll
             for (int b = 0; b < BN; ++b) sum[b] = v[b];
         } else {
-            splitk_sum<BN>(a.partial + (size_t)n * g.splits * Mp, g.splits, M, Mp, sum);
+            splitk_sum<BN>(part + (size_t)n * ns * Mp, nseg, M, Mp, sum);
         }
-        if constexpr (MODE == EPI_RESID || MODE == EPI_F32) {
+        if constexpr (MODE == EPI_F32) {
 #pragma unroll
-            for (int b = 0; b < BN; ++b) {
+            for (int b = 0; b < BN; ++b)
+                if (b < M) ep.out[(size_t)b * ep.ld_out + n] = sum[b] * sm.sinv[b];
+        } else if constexpr (MODE == EPI_RESID) {
+            // trunk += the block's sum; then the next norm's inputs: bf16(g * x)
+            // and the block's sum of squares per row
+            const bool to_ffn = (type == PH_O);
+            const float gn = (to_ffn ? a.gains[2 * l + 1] : a.gains[2 * (l + 1)])[n];
+            bf16* xg = to_ffn ? a.xg2 : a.xg;
+#pragma unroll
+            for (int b = 0; b < BN; ++b)
                 if (b < M) {
-                    float* o = ep.out + (size_t)b * ep.ld_out + n;
-                    if constexpr (MODE == EPI_RESID) *o += sum[b];
-                    else *o = sum[b];
+                    float* o = a.trunk + (size_t)b * a.d + n;
+                    const float x = __ldcg(o) + sum[b];
+                    *o = x;
+                    xg[(size_t)b * a.d + n] = __float2bfloat16_rn(x * gn);
+                    sm.xbuf[b * XLD + et] = x * x;
                 }
+            esync();
+            const int warp = tid >> 5, lane = tid & 31;
+            float* ssq = a.ssq + (to_ffn ? SSQ_BLOCKS * 32 : 0);
+            for (int b = warp; b < M; b += 4) {
+                const float* r = sm.xbuf + b * XLD;
+                const float s = warp_sum((r[lane] + r[lane + 32]) + (r[lane + 64] + r[lane + 96]));
+                if (lane == 0) ssq[mb * 32 + b] = s;
             }
-            if constexpr (MODE == EPI_RESID) {
-                // the CTA that finishes the phase's last tile normalises the trunk
-                __threadfence();
-                esync();
-                if (tid == 0) {
-                    const int prev = atomicAdd(a.tiles_done, 1);
-                    const int last = (prev == g.rowsA / BM - 1);
-                    if (last) *a.tiles_done = 0;
-                    *sm.flag = last;
-                }
-                esync();
-                const int last = *sm.flag;
-                esync();
-                if (last) {
-                    __threadfence();
-                    const float* gain = (type == PH_O) ? a.gains[2 * l + 1] : a.gains[2 * (l + 1)];
-                    norm_rows(a, gain, tid);
-                }
-            }
-        } else {
+            esync();
+        } else {   // EPI_QKV: 1/rms, then RoPE and the cache append on 32-column rows
 #pragma unroll
-            for (int b = 0; b < BN; ++b) sm.xbuf[b * SCfg<BN, HD>::XLD + et] = sum[b];
+            for (int b = 0; b < BN; ++b)
+                if (b < M) sm.xbuf[b * XLD + et] = sum[b] * sm.sinv[b];
             esync();
             if (tid < 4 * M) {
                 const int b = tid >> 2, c = tid & 3;
-                float w[32];
+                float x[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) w[i] = sm.xbuf[b * SCfg<BN, HD>::XLD + c * 32 + i];
-                epi_qkv32<bf16>(ep, b, mb * BM + c * 32, w);
+                for (int i = 0; i < 32; ++i) x[i] = sm.xbuf[b * XLD + c * 32 + i];
+                epi_qkv32<bf16>(ep, b, mb * BM + c * 32, x);
             }
             esync();
         }
-        return true;
     }
 }
 
@@ -345,9 +425,12 @@ __device__ bool tile_epilogue(const StepArgs& a, const EpiArgs& ep, const GemmPh
 // Each epilogue warp works alone: an item is 128 keys (4 chunks of 32) of
 // one (sequence b, head h); the warp streams its chunks through two shared
 // buffers of its own (bulk copies, the next chunk in flight while one is
-// computed), keeps the online-softmax state across the item, merges its four
-// lane groups with shuffles and leaves the item's (max, sum, output) in the
-// workspace; the warp that finishes the last item of (b, h) merges them.
+// computed).  Within a chunk each group of 8 lanes takes every 4th key: all
+// its scores first (independent dot products), then one rescale of the
+// running state by the chunk maximum, then the weighted values.  At the end
+// of an item the four groups merge with shuffles and leave the item's
+// (max, sum, output) in the workspace; the warp that finishes the last item
+// of (b, h) merges them.
 struct AttnCursor {
     int j, c;   // item ordinal of this warp, chunk within the item
 };
@@ -378,6 +461,7 @@ __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>
                            volatile int* abort_flag) {
     constexpr int DPL = HD / 8;      // dims per lane: 16-byte vectors u, dims (u*8 + r)*8 ..
     constexpr int NV = DPL / 8;
+    constexpr int KPG = ACH / 4;     // keys of a chunk per lane group
     constexpr int DPW = HD / 32;     // dims per lane in the final merge
     const int warp = tid >> 5, lane = tid & 31, g = lane >> 3, r = lane & 7;
     const int len = *a.d_pos + 1;
@@ -392,6 +476,11 @@ __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>
     };
     const uint32_t wbuf = smem_u32(sm.att) + warp * 2 * SCfg<BN, HD>::ATT_BUF;
     const uint32_t wbar = sm.abar + warp * 16;
+    // the cache rows of this position were stored by other CTAs (generic
+    // proxy) before the grid barrier; the bulk copies read them through the
+    // async proxy, and overwrite shared memory last written by generic stores
+    if (lane == 0) asm volatile("fence.proxy.async.global;\n\tfence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
     // issue the first two chunks
     AttnCursor is{0, 0};
     int issued = 0;
@@ -453,41 +542,63 @@ __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>
         }
         const bf16* sk = reinterpret_cast<const bf16*>(sm.att + (size_t)(warp * 2 + buf) * SCfg<BN, HD>::ATT_BUF);
         const bf16* sv = sk + ACH * HD;
-#pragma unroll 2
-        for (int i = 0; i < ACH / 4; ++i) {
+        // scores of this group's keys 4i + g (row 0 stands in for a missing key)
+        float s[KPG];
+#pragma unroll
+        for (int i = 0; i < KPG; ++i) {
             const int key = 4 * i + g;
-            const bool valid = key < nkeys;
-            const int kr = valid ? key : 0;
-            float kk[DPL], vv[DPL];
+            const int kr = key < nkeys ? key : 0;
+            float d0 = 0.f, d1 = 0.f;
 #pragma unroll
             for (int u = 0; u < NV; ++u) {
                 const uint4 wk = *reinterpret_cast<const uint4*>(sk + (size_t)kr * HD + (u * 8 + r) * 8);
-                const uint4 wv = *reinterpret_cast<const uint4*>(sv + (size_t)kr * HD + (u * 8 + r) * 8);
-                const uint32_t k4[4] = {wk.x, wk.y, wk.z, wk.w}, v4[4] = {wv.x, wv.y, wv.z, wv.w};
+                const uint32_t k4[4] = {wk.x, wk.y, wk.z, wk.w};
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
-                    const float2 fk = unpack_bf16x2(k4[t]), fv = unpack_bf16x2(v4[t]);
-                    kk[u * 8 + 2 * t] = fk.x;
-                    kk[u * 8 + 2 * t + 1] = fk.y;
-                    vv[u * 8 + 2 * t] = fv.x;
-                    vv[u * 8 + 2 * t + 1] = fv.y;
+                    const float2 fk = unpack_bf16x2(k4[t]);
+                    d0 = fmaf(qv[u * 8 + 2 * t], fk.x, d0);
+                    d1 = fmaf(qv[u * 8 + 2 * t + 1], fk.y, d1);
                 }
             }
-            float s = 0.f;
+            s[i] = d0 + d1;
+        }
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) s = fmaf(qv[e], kk[e], s);
-            s += __shfl_xor_sync(0xffffffffu, s, 1);
-            s += __shfl_xor_sync(0xffffffffu, s, 2);
-            s += __shfl_xor_sync(0xffffffffu, s, 4);
-            if (valid) {
-                const float m_new = fmaxf(m, s);
-                const float corr = __expf(m - m_new);
-                const float p = __expf(s - m_new);
-                lsum = lsum * corr + p;
+        for (int off = 1; off <= 4; off <<= 1)
 #pragma unroll
-                for (int e = 0; e < DPL; ++e) acc[e] = fmaf(acc[e], corr, p * vv[e]);
-                m = m_new;
+            for (int i = 0; i < KPG; ++i) s[i] += __shfl_xor_sync(0xffffffffu, s[i], off);
+        float cmax = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < KPG; ++i)
+            if (4 * i + g < nkeys) cmax = fmaxf(cmax, s[i]);
+        const float m_new = fmaxf(m, cmax);
+        if (m_new != -INFINITY) {   // this group holds at least one key so far
+            const float corr = __expf(m - m_new);
+            float p[KPG], psum = 0.f;
+#pragma unroll
+            for (int i = 0; i < KPG; ++i) {
+                p[i] = (4 * i + g < nkeys) ? __expf(s[i] - m_new) : 0.f;
+                psum += p[i];
             }
+            lsum = lsum * corr + psum;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[e] *= corr;
+#pragma unroll
+            for (int i = 0; i < KPG; ++i) {
+                const int key = 4 * i + g;
+                const int kr = key < nkeys ? key : 0;
+#pragma unroll
+                for (int u = 0; u < NV; ++u) {
+                    const uint4 wv = *reinterpret_cast<const uint4*>(sv + (size_t)kr * HD + (u * 8 + r) * 8);
+                    const uint32_t v4[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float2 fv = unpack_bf16x2(v4[t]);
+                        acc[u * 8 + 2 * t] = fmaf(p[i], fv.x, acc[u * 8 + 2 * t]);
+                        acc[u * 8 + 2 * t + 1] = fmaf(p[i], fv.y, acc[u * 8 + 2 * t + 1]);
+                    }
+                }
+            }
+            m = m_new;
         }
         __syncwarp();
         // the buffer is free: put the chunk two places ahead in flight
@@ -647,6 +758,7 @@ __device__ void phase_argmax(const StepArgs& a, int tid, const Smem<BN, HD>& sm)
     }
 }
 
+
 // ---------------------------------------------------------------- the kernel
 template <int BN, int HD>
 __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
@@ -660,7 +772,8 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
     sm.sB = base_s + C::OFF_B;
     sm.att = gb + C::OFF_ATT;
     sm.xbuf = reinterpret_cast<float*>(gb + C::OFF_X);
-    sm.red = reinterpret_cast<float*>(gb + C::OFF_SML);
+    sm.sinv = reinterpret_cast<float*>(gb + C::OFF_SML);
+    sm.red = sm.sinv + 32;
     const uint32_t bars = base_s + C::OFF_BAR;
     sm.full = bars;
     sm.empty = bars + 8 * C::STAGES;
@@ -705,43 +818,69 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
 
     if (warp == 0) {
         // -------------------------------------------------------- TMA producer
+        // Two cursors over the same stage sequence: weight tiles are requested
+        // as soon as a ring slot frees; the activation tile of a stage only
+        // once the grid barrier before its phase has released this CTA.
         if (lane == 0) {
-            int stage = 0;
-            uint32_t ph = 0;
-            int ready = -1;
-            bool ok = true;
-            for (int p = 0; p < P && ok; ++p) {
-                int l;
-                const int type = phase_type(a, p, l);
-                GemmPh g;
-                if (!gemm_of(a, type, l, g)) continue;
-                const int mblk = g.rowsA / BM, kbt = g.K / BK, per = (kbt + g.splits - 1) / g.splits;
-                const int tiles = mblk * g.splits;
-                for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-                    const int mb = t % mblk, sp = t / mblk;
-                    const int kb0 = sp * per, kb1 = min(kbt, kb0 + per);
-                    for (int kb = kb0; kb < kb1; ++kb) {
-                        if (!mbar_wait(sm.empty + 8 * stage, ph ^ 1u, abort_flag, a.err)) {
-                            ok = false;
-                            break;
-                        }
-                        mbar_expect_tx(sm.full + 8 * stage, C::STAGE_BYTES);
-                        tma_load_2d(sm.sA + stage * C::A_BYTES, a.maps + g.map_a, sm.full + 8 * stage, kb * BK,
-                                    mb * BM);
-                        if (ready < p) {
-                            if (!wait_gen(bar_flag(a.bar, blockIdx.x), gen0 + (unsigned)p, abort_flag, a.err)) {
-                                ok = false;
-                                break;
-                            }
-                            asm volatile("fence.proxy.async.global;" ::: "memory");
-                            ready = p;
-                        }
-                        tma_load_2d(sm.sB + stage * C::B_BYTES, a.maps + g.map_b, sm.full + 8 * stage, kb * BK, 0);
-                        if (++stage == C::STAGES) {
-                            stage = 0;
-                            ph ^= 1u;
-                        }
+            Cursor wc, xc;
+            cursor_seek(a, P, wc, 0);
+            xc = wc;
+            int wn = 0, xn = 0, ready = -1;
+            const unsigned* myflag = bar_flag(a.bar, blockIdx.x);
+            uint64_t t_last = global_timer();
+            while (xc.valid) {
+                bool prog = false;
+                if (wc.valid && wn - xn < C::STAGES) {
+                    const int slot = wn % C::STAGES;
+                    if (mbar_test(sm.empty + 8 * slot, ((wn / C::STAGES) & 1) ^ 1)) {
+                        const int mb = wc.i / wc.kbt, kb = wc.i - mb * wc.kbt;
+                        mbar_expect_tx(sm.full + 8 * slot, C::STAGE_BYTES);
+                        tma_load_2d(sm.sA + slot * C::A_BYTES, a.maps + wc.map_a, sm.full + 8 * slot, kb * BK, mb * BM);
+                        ++wn;
+                        cursor_next(a, P, wc);
+                        prog = true;
                     }
+                }
+                if (xn < wn) {
+                    if (ready < xc.p && (int)(ld_acquire_u32(myflag) - (gen0 + (unsigned)xc.p)) >= 0) {
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                        ready = xc.p;
+                    }
+                    if (ready >= xc.p) {
+                        const int slot = xn % C::STAGES;
+                        tma_load_2d(sm.sB + slot * C::B_BYTES, a.maps + xc.map_b, sm.full + 8 * slot,
+                                    (xc.i % xc.kbt) * BK, 0);
+                        ++xn;
+                        cursor_next(a, P, xc);
+                        prog = true;
+                    }
+                }
+                if (prog) {
+                    t_last = global_timer();
+                    continue;
+                }
+                if (*abort_flag) break;
+                if (global_timer() - t_last > WAIT_LIMIT_NS) {
+                    *abort_flag = 1;
+                    atomicOr(a.err, LLAMA_DEVERR_TIMEOUT);
+                    break;
+                }
+                __nanosleep(32);   // leave issue slots to the epilogue warp on this sub-partition
+            }
+            // Leave no copy in flight: complete every stage whose weight tile
+            // was requested (its activation tile too, stale or not, so that its
+            // barrier can complete), then wait -- bounded -- for the last ring
+            // of stages to land.
+            while (xn < wn) {
+                const int slot = xn % C::STAGES;
+                tma_load_2d(sm.sB + slot * C::B_BYTES, a.maps + xc.map_b, sm.full + 8 * slot, (xc.i % xc.kbt) * BK, 0);
+                ++xn;
+                cursor_next(a, P, xc);
+            }
+            for (int u = max(0, wn - C::STAGES); u < wn; ++u) {
+                const uint64_t t0 = global_timer();
+                while (!mbar_test(sm.full + 8 * (u % C::STAGES), (u / C::STAGES) & 1) &&
+                       global_timer() - t0 < WAIT_LIMIT_NS / 4) {
                 }
             }
         }
@@ -757,20 +896,17 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
             for (int p = 0; p < P && ok; ++p) {
                 int l;
                 const int type = phase_type(a, p, l);
-                GemmPh g;
-                if (!gemm_of(a, type, l, g)) continue;
-                const int mblk = g.rowsA / BM, kbt = g.K / BK, per = (kbt + g.splits - 1) / g.splits;
-                const int tiles = mblk * g.splits;
-                for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-                    const int sp = t / mblk;
-                    const int kb0 = sp * per, kb1 = min(kbt, kb0 + per);
+                Work w;
+                if (!work_of(a, type, l, w)) continue;
+                for (int i = w.s; i < w.e && ok;) {
+                    const int se = min(w.e, (i / w.kbt + 1) * w.kbt);   // end of this block's run
                     if (!mbar_wait(sm.tempty + 8 * acc, acc_ph ^ 1u, abort_flag, a.err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
-                    for (int kb = kb0; kb < kb1; ++kb) {
+                    for (int it = i; it < se; ++it) {
                         if (!mbar_wait(sm.full + 8 * stage, ph, abort_flag, a.err)) {
                             ok = false;
                             break;
@@ -780,7 +916,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                         const uint64_t db = sw128_desc(sm.sB + stage * C::B_BYTES);
 #pragma unroll
                         for (int k = 0; k < BK / 16; ++k)
-                            umma_bf16(d_tmem, da + 2 * k, db + 2 * k, IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
+                            umma_bf16(d_tmem, da + 2 * k, db + 2 * k, IDESC, (it > i || k > 0) ? 1u : 0u);
                         umma_commit(sm.empty + 8 * stage);
                         if (++stage == C::STAGES) {
                             stage = 0;
@@ -793,6 +929,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                         acc = 0;
                         acc_ph ^= 1u;
                     }
+                    i = se;
                 }
             }
         }
@@ -817,6 +954,9 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
             if (tl && tid == 0) tl[2 * p] = global_timer();
             bool fail = false;
             if (type == PH_EMBED) {
+                // trunk row b = embedding of its token; bf16(g * x) of the
+                // first attention norm and the 128-feature block sums of
+                // squares (one warp per block: 32 lanes x 4 features)
                 if ((int)blockIdx.x < a.B) {
                     const int b = blockIdx.x;
                     int t = a.tok[b];
@@ -826,22 +966,16 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                     }
                     const bf16* e = a.embed + (size_t)t * a.d;
                     float* x = a.trunk + (size_t)b * a.d;
-                    for (int i = tid; i < a.d; i += 128) x[i] = __bfloat162float(e[i]);
-                    __threadfence_block();
-                    esync();
-                    // RMSNorm of this row with layer 0's attention gain
-                    float ss = 0.f;
-                    for (int i = tid * 4; i < a.d; i += 512) {
-                        const float4 v = *reinterpret_cast<const float4*>(x + i);
-                        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-                    }
-                    const float inv = rsqrtf(esum(ss, sm.red, tid) / (float)a.d + a.eps);
-                    const float* gg = a.gains[0];
-                    for (int i = tid * 4; i < a.d; i += 512) {
-                        const float4 v = *reinterpret_cast<const float4*>(x + i);
-                        const float4 gv = *reinterpret_cast<const float4*>(gg + i);
-                        *reinterpret_cast<uint2*>(a.xn + (size_t)b * a.d + i) = make_uint2(
-                            pack_bf16x2(v.x * inv * gv.x, v.y * inv * gv.y), pack_bf16x2(v.z * inv * gv.z, v.w * inv * gv.w));
+                    const float* g0 = a.gains[0];
+                    for (int i = 4 * tid; i < a.d; i += 512) {
+                        const uint2 w = *reinterpret_cast<const uint2*>(e + i);
+                        const float2 v01 = unpack_bf16x2(w.x), v23 = unpack_bf16x2(w.y);
+                        const float4 gg = *reinterpret_cast<const float4*>(g0 + i);
+                        *reinterpret_cast<float4*>(x + i) = make_float4(v01.x, v01.y, v23.x, v23.y);
+                        *reinterpret_cast<uint2*>(a.xg + (size_t)b * a.d + i) =
+                            make_uint2(pack_bf16x2(v01.x * gg.x, v01.y * gg.y), pack_bf16x2(v23.x * gg.z, v23.y * gg.w));
+                        const float s = warp_sum((v01.x * v01.x + v01.y * v01.y) + (v23.x * v23.x + v23.y * v23.y));
+                        if (lane == 0) a.ssq[(i >> 7) * 32 + b] = s;
                     }
                 }
             } else if (type == PH_ATTN) {
@@ -849,11 +983,13 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
             } else if (type == PH_ARGMAX) {
                 phase_argmax<BN, HD>(a, tid, sm);
             } else {
-                GemmPh g;
-                gemm_of(a, type, l, g);
+                Work w;
+                work_of(a, type, l, w);
+                if (type == PH_QKV || type == PH_HEAD) load_inv(a, a.ssq, sm.sinv, tid);
+                else if (type == PH_GU) load_inv(a, a.ssq + SSQ_BLOCKS * 32, sm.sinv, tid);
                 EpiArgs ep;
                 ep.M = a.B;
-                ep.N = g.rowsA;
+                ep.N = w.g.rowsA;
                 ep.out = (type == PH_HEAD) ? a.logits : a.trunk;
                 ep.ld_out = (type == PH_HEAD) ? a.V : a.d;
                 ep.partial = a.partial;
@@ -870,10 +1006,8 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                 ep.hd = a.hd;
                 ep.d = a.d;
                 ep.smax = a.smax;
-                const int mblk = g.rowsA / BM;
-                const int tiles = mblk * g.splits;
-                for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-                    const int mb = t % mblk, sp = t / mblk;
+                for (int i = w.s; i < w.e;) {
+                    const int mb = i / w.kbt;
                     const bool ok = mbar_wait(sm.tfull + 8 * acc, acc_ph, abort_flag, a.err);
                     if (esync_any(!ok)) {
                         fail = true;
@@ -890,12 +1024,13 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                         acc = 0;
                         acc_ph ^= 1u;
                     }
-                    switch (g.mode) {
-                        case EPI_QKV: tile_epilogue<BN, HD, EPI_QKV>(a, ep, g, l, type, mb, sp, et, tid, v, sm); break;
-                        case EPI_RESID: tile_epilogue<BN, HD, EPI_RESID>(a, ep, g, l, type, mb, sp, et, tid, v, sm); break;
-                        case EPI_SWIGLU: tile_epilogue<BN, HD, EPI_SWIGLU>(a, ep, g, l, type, mb, sp, et, tid, v, sm); break;
-                        default: tile_epilogue<BN, HD, EPI_F32>(a, ep, g, l, type, mb, sp, et, tid, v, sm); break;
+                    switch (w.g.mode) {
+                        case EPI_QKV: tile_epilogue<BN, HD, EPI_QKV>(a, ep, w, l, type, mb, et, tid, v, sm); break;
+                        case EPI_RESID: tile_epilogue<BN, HD, EPI_RESID>(a, ep, w, l, type, mb, et, tid, v, sm); break;
+                        case EPI_SWIGLU: tile_epilogue<BN, HD, EPI_SWIGLU>(a, ep, w, l, type, mb, et, tid, v, sm); break;
+                        default: tile_epilogue<BN, HD, EPI_F32>(a, ep, w, l, type, mb, et, tid, v, sm); break;
                     }
+                    i = min(w.e, (mb + 1) * w.kbt);
                 }
             }
             if (esync_any(fail)) break;
@@ -924,7 +1059,7 @@ int launch_step_t(const StepArgs& a, cudaStream_t st) {
         attr = true;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(tc_num_sms());
+    cfg.gridDim = dim3(decode_step_ctas());
     cfg.blockDim = dim3(NT);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
@@ -940,6 +1075,26 @@ int launch_step_t(const StepArgs& a, cudaStream_t st) {
 
 }  // namespace
 
+int decode_step_ctas() { return std::min(tc_num_sms(), STEP_MAX_CTAS); }
+
+// Partial-sum and counter regions of the five projection kinds (qkv, o,
+// gate/up, down, head) for `ctas` CTAs and batch B; returns the floats of
+// all partial regions.
+long long decode_step_layout(int ctas, int d, int h, int V, int B, long long part_off[5], int cnt_off[5]) {
+    const int rows[5] = {3 * d, d, 2 * h, d, V};
+    const long long Mp = (B + 3) & ~3;
+    long long off = 0;
+    int coff = 0;
+    for (int t = 0; t < 5; ++t) {
+        const int mblk = rows[t] / BM;
+        part_off[t] = off;
+        off += (long long)rows[t] * step_slots(mblk, ctas) * Mp;
+        cnt_off[t] = coff;
+        coff += (t == 2) ? mblk / 2 : mblk;
+    }
+    return off;
+}
+
 int decode_step_prepare() {
     int n = 0;
     LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -951,8 +1106,8 @@ int decode_step_prepare() {
     LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<32, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         SCfg<32, 64>::SMEM));
     // one CTA per SM must fit for the cooperative launch
-    LLAMA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_step_kernel<32, 128>, NT,
-                                                                 SCfg<32, 128>::SMEM));
+    LLAMA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_step_kernel<16, 128>, NT,
+                                                                 SCfg<16, 128>::SMEM));
     return n >= 1 ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
@@ -964,9 +1119,9 @@ int launch_decode_step(const StepArgs& a, cudaStream_t st) {
 }
 
 // Tensor-map table for the decode step: 4 per layer (W_qkv, W_o, W_gu, W_d),
-// the head, then the activation buffers xn, attn, act with `B` rows.
-int decode_step_maps(CUtensorMap* host_maps, const void* const* w, int L, const void* head, const void* xn,
-                     const void* attn, const void* act, int B, int d, int h, int V) {
+// the head, then the activation buffers xg, attn, act, xg2 with `B` rows.
+int decode_step_maps(CUtensorMap* host_maps, const void* const* w, int L, const void* head, const void* xg,
+                     const void* attn, const void* act, const void* xg2, int B, int d, int h, int V) {
     int rc;
     const int bn = B <= 16 ? 16 : 32;
     for (int l = 0; l < L; ++l) {
@@ -976,7 +1131,8 @@ int decode_step_maps(CUtensorMap* host_maps, const void* const* w, int L, const 
         if ((rc = tc_make_map_2d(&host_maps[4 * l + 3], w[4 * l + 3], d, h, BM))) return rc;
     }
     if ((rc = tc_make_map_2d(&host_maps[4 * L + 0], head, V, d, BM))) return rc;
-    if ((rc = tc_make_map_2d(&host_maps[4 * L + 1], xn, B, d, bn))) return rc;
+    if ((rc = tc_make_map_2d(&host_maps[4 * L + 1], xg, B, d, bn))) return rc;
     if ((rc = tc_make_map_2d(&host_maps[4 * L + 2], attn, B, d, bn))) return rc;
-    return tc_make_map_2d(&host_maps[4 * L + 3], act, B, h, bn);
+    if ((rc = tc_make_map_2d(&host_maps[4 * L + 3], act, B, h, bn))) return rc;
+    return tc_make_map_2d(&host_maps[4 * L + 4], xg2, B, d, bn);
 }

@@ -65,19 +65,30 @@ int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaSt
 int gemm_tc_pick_splits(int rowsA, int K);
 
 // decode_step.cu  (one cooperative kernel per greedy decode step, bf16)
+// At most this many CTAs run the fused decode step (one per SM).
+constexpr int STEP_MAX_CTAS = 160;
+// Partial-sum slots per output feature of a projection with `mblk` 128-row
+// blocks when its (block, k-block) iterations are cut into `ctas` equal
+// contiguous ranges: no block is touched by more ranges than this.
+__host__ __device__ inline int step_slots(int mblk, int ctas) { return (ctas + mblk - 1) / mblk + 1; }
+
 struct StepArgs {
-    const CUtensorMap* maps;      // device table: 4 per layer (W_qkv, W_o, W_gu, W_d), head, xn, attn, act
+    const CUtensorMap* maps;      // device table: 4 per layer (W_qkv, W_o, W_gu, W_d), head, xg, attn, act, xg2
     const float* const* gains;    // device table [2L + 1]: g_attn[l], g_ffn[l], ..., g_final
     const __nv_bfloat16* embed;
     __nv_bfloat16* kv;            // layer l: K at kv + 2l * kv_layer, V at kv + (2l + 1) * kv_layer
     size_t kv_layer;
     float* trunk;
-    __nv_bfloat16 *xn, *q, *attn, *act;
+    __nv_bfloat16* xg;            // g (.) x of the attention / final norm, bf16 [B][d]
+    __nv_bfloat16* xg2;           // g (.) x of the FFN norm, bf16 [B][d]
+    float* ssq;                   // [2][64][32] per 128-feature block sums of squares (attention, FFN norm)
+    __nv_bfloat16 *q, *attn, *act;
     float* logits;
-    float* partial;               // split-K partials
-    int* counters;                // split-K arrival counters
-    int* tiles_done;              // finished tiles of a residual projection
-    float* attn_work;             // attention chunk partials [B*H][ceil(smax/64)][hd + 2]
+    float* partial;               // split-K partials, one region per projection kind
+    long long part_off[5];        // qkv, o, gate/up, down, head (floats)
+    int* counters;                // arrival counters, one region per projection kind
+    int cnt_off[5];
+    float* attn_work;             // attention chunk partials [B*H][ceil(smax/128)][hd + 2]
     int* attn_cnt;                // [B*H]
     int2* amax_part;              // [B][ceil(V/2048)]
     int* amax_cnt;                // [B + 1]
@@ -89,12 +100,14 @@ struct StepArgs {
     const float2* rope;
     int L, d, h, V, H, hd, B, smax;
     float eps;
-    int splits[5];                // qkv, o, gate/up, down, head
 };
 int decode_step_prepare();
 int launch_decode_step(const StepArgs& a, cudaStream_t st);
-int decode_step_maps(CUtensorMap* host_maps, const void* const* w, int L, const void* head, const void* xn,
-                     const void* attn, const void* act, int B, int d, int h, int V);
+int decode_step_maps(CUtensorMap* host_maps, const void* const* w, int L, const void* head, const void* xg,
+                     const void* attn, const void* act, const void* xg2, int B, int d, int h, int V);
+// Grid of the fused decode step, and the partial / counter regions for batch B
+int decode_step_ctas();
+long long decode_step_layout(int ctas, int d, int h, int V, int B, long long part_off[5], int cnt_off[5]);
 // 2-D K-major bf16 tensor map, box (64, box_rows), 128-byte swizzle, zero fill
 int tc_make_map_2d(CUtensorMap* map, const void* ptr, int rows, int K, int box_rows);
 int tc_num_sms();

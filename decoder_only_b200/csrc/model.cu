@@ -154,10 +154,11 @@ struct llama_model {
     size_t partial_elems;
     int* counters;           // split-K arrival counters (zero between launches)
     int* attn_cnt;           // decode-attention arrival counters [max_batch * H]
-    CUtensorMap* step_maps;  // decode-step tensor-map table (device) [4L + 4]
+    CUtensorMap* step_maps;  // decode-step tensor-map table (device) [4L + 5]
     const float** step_gains;  // decode-step gain table (device) [2L + 1]
     unsigned int* step_bar;  // decode-step grid barrier [2]
-    int* tiles_done;         // decode-step finished residual tiles
+    void* step_xg2;          // decode-step FFN-norm input g * x, bf16 [max_batch, d]
+    float* step_ssq;         // decode-step block sums of squares [2][64][32]
     float* step_attn_work;   // decode-step attention partials
     unsigned long long* step_timeline;   // decode-step phase stamps (while profiling)
     int2* amax_part;         // greedy-choice chunk results [max_batch][chunks]
@@ -181,6 +182,8 @@ struct llama_model {
 
 namespace {
 
+int hidden_of(const llama_config* c);
+
 int validate(const llama_config* c) {
     if (!c) return LLAMA_ERR_INVALID_ARG;
     if (c->n_layers < 0 || c->d_model <= 0 || c->n_heads <= 0 || c->vocab <= 0) return LLAMA_ERR_INVALID_ARG;
@@ -195,6 +198,8 @@ int validate(const llama_config* c) {
         if (c->d_model % 256 != 0) return LLAMA_ERR_INVALID_ARG;
         if (c->max_batch > 32) return LLAMA_ERR_INVALID_ARG;
         if (c->vocab % 128 != 0) return LLAMA_ERR_INVALID_ARG;   // whole 128-row head tiles
+        // arrival counters of the fused decode step: one per 128-row block
+        if ((5 * (int64_t)c->d_model + hidden_of(c) + c->vocab) / 128 > MAX_COUNTERS) return LLAMA_ERR_INVALID_ARG;
     } else {
         if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return LLAMA_ERR_INVALID_ARG;
     }
@@ -246,14 +251,18 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     const size_t cmax = std::max(3 * d, 2 * h);
     float* gemm_c = (float*)take(c->dtype == LLAMA_F32 ? nmax * std::max(cmax, V) * 4 : 0);
     float* logits_dec = (float*)take((size_t)c->max_batch * V * 4);
-    const size_t pmax = (size_t)MAX_DEC_SPLITS * ((c->max_batch + 3) & ~3) * std::max(cmax, V);
+    long long part_off[5];
+    int cnt_off[5];
+    const size_t pmax = (size_t)decode_step_layout(STEP_MAX_CTAS, (int)d, (int)h, (int)V, c->max_batch, part_off,
+                                                   cnt_off);
     float* partial = (float*)take(c->dtype == LLAMA_BF16 ? pmax * 4 : 0);
     int* counters = (int*)take(MAX_COUNTERS * 4);
     int* attn_cnt = (int*)take((size_t)c->max_batch * c->n_heads * 4);
-    CUtensorMap* step_maps = (CUtensorMap*)take((size_t)(4 * L + 4) * sizeof(CUtensorMap));
+    CUtensorMap* step_maps = (CUtensorMap*)take((size_t)(4 * L + 5) * sizeof(CUtensorMap));
     const float** step_gains = (const float**)take((size_t)(2 * L + 1) * sizeof(float*));
     unsigned int* step_bar = (unsigned int*)take(32 * 1024);   // arrivals + one 128-byte flag per CTA
-    int* tiles_done = (int*)take(256);
+    void* step_xg2 = take((size_t)c->max_batch * d * esz);
+    float* step_ssq = (float*)take(2 * 64 * 32 * 4);
     float* step_attn_work = (float*)take((size_t)c->max_batch * c->n_heads * ((c->max_seq + 127) / 128) *
                                          (c->head_dim + 2) * 4);
     // per-phase timestamps of the fused decode step (profiling): 2 per CTA per phase
@@ -288,7 +297,8 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
         m->step_maps = step_maps;
         m->step_gains = step_gains;
         m->step_bar = step_bar;
-        m->tiles_done = tiles_done;
+        m->step_xg2 = step_xg2;
+        m->step_ssq = step_ssq;
         m->step_attn_work = step_attn_work;
         m->step_timeline = step_timeline;
         m->amax_cnt = amax_cnt;
@@ -464,14 +474,16 @@ StepArgs step_args(llama_model* m) {
     a.kv = (bf16*)m->kv;
     a.kv_layer = m->kv_layer_elems;
     a.trunk = m->trunk;
-    a.xn = (bf16*)m->xn;
+    a.xg = (bf16*)m->xn;
+    a.xg2 = (bf16*)m->step_xg2;
+    a.ssq = m->step_ssq;
     a.q = (bf16*)m->q;
     a.attn = (bf16*)m->attn;
     a.act = (bf16*)m->act;
     a.logits = m->logits_dec;
     a.partial = m->partial;
     a.counters = m->counters;
-    a.tiles_done = m->tiles_done;
+    decode_step_layout(decode_step_ctas(), c.d_model, c.ffn_hidden, c.vocab, m->B, a.part_off, a.cnt_off);
     a.attn_work = m->step_attn_work;
     a.attn_cnt = m->attn_cnt;
     a.amax_part = m->amax_part;
@@ -490,11 +502,6 @@ StepArgs step_args(llama_model* m) {
     a.B = m->B;
     a.smax = c.max_seq;
     a.eps = c.norm_eps;
-    a.splits[0] = m->splits_qkv;
-    a.splits[1] = m->splits_o;
-    a.splits[2] = m->splits_gu;
-    a.splits[3] = m->splits_d;
-    a.splits[4] = m->splits_head;
     return a;
 }
 
@@ -503,7 +510,7 @@ StepArgs step_args(llama_model* m) {
 int step_tables(llama_model* m) {
     const llama_config& c = m->cfg;
     const int L = c.n_layers;
-    std::vector<CUtensorMap> maps((size_t)4 * L + 4);
+    std::vector<CUtensorMap> maps((size_t)4 * L + 5);
     std::vector<const void*> w((size_t)4 * L);
     for (int l = 0; l < L; ++l) {
         w[4 * l + 0] = m->layers[l].wqkv;
@@ -511,8 +518,8 @@ int step_tables(llama_model* m) {
         w[4 * l + 2] = m->layers[l].wgu;
         w[4 * l + 3] = m->layers[l].wd;
     }
-    int rc = decode_step_maps(maps.data(), w.data(), L, m->head, m->xn, m->attn, m->act, m->B, c.d_model,
-                              c.ffn_hidden, c.vocab);
+    int rc = decode_step_maps(maps.data(), w.data(), L, m->head, m->xn, m->attn, m->act, m->step_xg2, m->B,
+                              c.d_model, c.ffn_hidden, c.vocab);
     if (rc) return rc;
     std::vector<const float*> gains((size_t)2 * L + 1);
     for (int l = 0; l < L; ++l) {
@@ -702,7 +709,6 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
     if (cudaMemsetAsync(m->counters, 0, MAX_COUNTERS * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->amax_cnt, 0, (size_t)(cfg->max_batch + 1) * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->step_bar, 0, 32 * 1024, st) != cudaSuccess ||
-        cudaMemsetAsync(m->tiles_done, 0, 256, st) != cudaSuccess ||
         cudaMemsetAsync(m->attn_cnt, 0, (size_t)cfg->max_batch * cfg->n_heads * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->d_pos, 0, 256, st) != cudaSuccess) {
         llama_free(m);
