@@ -60,10 +60,10 @@ using namespace tc;
 
 constexpr int BM = 128;      // weight rows per tile (TMEM lanes)
 constexpr int BK = 64;       // K per stage (one 128-byte swizzle row)
-constexpr int NT = 192;
-constexpr int ACH = 32;      // keys per attention chunk (one bulk copy of K rows, one of V rows)
-constexpr int SEG = 4;       // chunks per attention item: one warp, 128 keys of one (sequence, head)
-constexpr int SEGK = ACH * SEG;
+constexpr int NT = 256;      // warps 0-3 epilogue, 4 TMA producer, 5 MMA, 6-7 attention
+constexpr int NAW = STEP_ATTN_WARPS;   // attention warps per CTA: the four epilogue warps and warps 6, 7
+static_assert(NAW == 6, "warp roles");
+constexpr int ACH = 16;      // keys per attention chunk (one bulk copy of K rows, one of V rows)
 constexpr int AMX = 2048;    // logits per greedy-choice item
 constexpr int SSQ_BLOCKS = 64;   // 128-feature blocks of one norm's sums of squares (d <= 8192)
 
@@ -77,16 +77,20 @@ struct SCfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-    // attention: per epilogue warp two chunk buffers (K rows then V rows);
-    // the transpose buffer of the projection epilogues shares the region
-    static constexpr int ATT_BUF = 2 * ACH * HD * 2;
-    static constexpr int OFF_ATT = OFF_B + STAGES * B_BYTES;             // [4 warps][2][ATT_BUF]
+    // attention: per attention warp two chunk buffers (K rows, V rows, and
+    // the query of a pair whose first chunk it is); the transpose buffer of
+    // the projection epilogues shares the region
+    static constexpr int ATT_Q = 2 * ACH * HD * 2;                        // offset of the query
+    static constexpr int ATT_BUF = ATT_Q + HD * 2;
+    static constexpr int OFF_ATT = OFF_B + STAGES * B_BYTES;             // [NAW warps][2][ATT_BUF]
     static constexpr int OFF_X = OFF_ATT;                                 // [32][XLD] floats
     static constexpr int XLD = BM + 1;
-    static constexpr int ATT_BYTES = 4 * 2 * ATT_BUF > 32 * XLD * 4 ? 4 * 2 * ATT_BUF : 32 * XLD * 4;
+    static constexpr int ATT_BYTES = NAW * 2 * ATT_BUF > 32 * XLD * 4 ? NAW * 2 * ATT_BUF : 32 * XLD * 4;
     static constexpr int OFF_SML = OFF_ATT + ATT_BYTES;                   // 1/rms [32], reduction scratch
-    static constexpr int OFF_BAR = OFF_SML + 1024;
+    static constexpr int OFF_BAR = OFF_SML + 1024;                       // mbarriers, then misc words
+    static constexpr int OFF_MISC = OFF_BAR + 8 * (2 * STAGES + 4 + 2 * NAW);
     static constexpr int SMEM = OFF_BAR + 512 + 1024;
+    static_assert(OFF_MISC + 16 <= OFF_BAR + 512, "mbarrier region");
     static constexpr uint32_t TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
 };
 
@@ -422,104 +426,90 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
 }
 
 // ---------------------------------------------------------------- attention phase
-// Each epilogue warp works alone: an item is 128 keys (4 chunks of 32) of
-// one (sequence b, head h); the warp streams its chunks through two shared
-// buffers of its own (bulk copies, the next chunk in flight while one is
-// computed).  Within a chunk each group of 8 lanes takes every 4th key: all
-// its scores first (independent dot products), then one rescale of the
-// running state by the chunk maximum, then the weighted values.  At the end
-// of an item the four groups merge with shuffles and leave the item's
-// (max, sum, output) in the workspace; the warp that finishes the last item
-// of (b, h) merges them.
-struct AttnCursor {
-    int j, c;   // item ordinal of this warp, chunk within the item
-};
-
+// Work split: the (pair = (sequence b, head h), 16-key chunk) units of all
+// pairs, pair-major, are cut into equal contiguous ranges, one per
+// attention warp of the grid (stream-K, as for the projections), so every
+// warp reads the same number of cache bytes.  A warp streams its chunks
+// through two shared buffers of its own (bulk copies; the next chunk in
+// flight while one is computed; the first chunk of each pair brings the
+// pair's query along).  Within a chunk each group of 8 lanes takes every 4th
+// key: all its scores first (independent dot products), then one rescale of
+// the running (max, sum, output) by the chunk maximum, then the weighted
+// values.  Where a warp's range leaves a pair, the four groups merge with
+// shuffles; a pair inside one range is written directly, otherwise each
+// range leaves its (max, sum, output) in the workspace and the last range to
+// arrive merges them in range order.
 template <int BN, int HD>
-__device__ __forceinline__ void attn_issue(const StepArgs& a, int l, int item, int c, int nseg, int len,
+__device__ __forceinline__ void attn_issue(const StepArgs& a, int l, int pr, int kc, bool with_q, int len,
                                            uint32_t dst, uint32_t bar) {
-    const int seg = item % nseg, bh = item / nseg;
-    const int b = bh / a.H, h = bh - b * a.H;
-    const int k0 = seg * SEGK + c * ACH;
+    const int k0 = kc * ACH;
     const int nkeys = min(len - k0, ACH);
-    const bf16* kc = a.kv + (size_t)(2 * l) * a.kv_layer;
-    const bf16* vc = kc + a.kv_layer;
-    const size_t off = (((size_t)b * a.H + h) * a.smax + k0) * HD;
+    const bf16* kc_ = a.kv + (size_t)(2 * l) * a.kv_layer;
+    const bf16* vc = kc_ + a.kv_layer;
+    const size_t off = ((size_t)pr * a.smax + k0) * HD;     // pair pr = b * H + h
     const uint32_t bytes = (uint32_t)(nkeys * HD * 2);
-    mbar_expect_tx(bar, 2 * bytes);
+    mbar_expect_tx(bar, 2 * bytes + (with_q ? HD * 2 : 0));
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(kc + off), "r"(bytes), "r"(bar)
+                 "l"(kc_ + off), "r"(bytes), "r"(bar)
                  : "memory");
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                      dst + ACH * HD * 2),
                  "l"(vc + off), "r"(bytes), "r"(bar)
                  : "memory");
+    if (with_q)
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                         dst + SCfg<BN, HD>::ATT_Q),
+                     "l"(a.q + (size_t)pr * HD), "r"((uint32_t)(HD * 2)), "r"(bar)
+                     : "memory");
 }
 
+// Attention of layer l for attention warp aw of this CTA (0..NAW-1).
 template <int BN, int HD>
-__device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>& sm, uint32_t* uses,
+__device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Smem<BN, HD>& sm, uint32_t* uses,
                            volatile int* abort_flag) {
+    using C = SCfg<BN, HD>;
     constexpr int DPL = HD / 8;      // dims per lane: 16-byte vectors u, dims (u*8 + r)*8 ..
     constexpr int NV = DPL / 8;
     constexpr int KPG = ACH / 4;     // keys of a chunk per lane group
     constexpr int DPW = HD / 32;     // dims per lane in the final merge
-    const int warp = tid >> 5, lane = tid & 31, g = lane >> 3, r = lane & 7;
+    const int g = lane >> 3, r = lane & 7;
     const int len = *a.d_pos + 1;
-    const int nseg = (len + SEGK - 1) / SEGK;
-    const int nsegmax = (a.smax + SEGK - 1) / SEGK;
-    const int nitems = nseg * a.B * a.H;
-    const int gw = blockIdx.x * 4 + warp, nw = gridDim.x * 4;
-    auto item_of = [&](int j) { return gw + j * nw; };
-    auto chunks_of = [&](int it) {
-        const int seg = it % nseg;
-        return (min(SEGK, len - seg * SEGK) + ACH - 1) / ACH;
-    };
-    const uint32_t wbuf = smem_u32(sm.att) + warp * 2 * SCfg<BN, HD>::ATT_BUF;
-    const uint32_t wbar = sm.abar + warp * 16;
-    // the cache rows of this position were stored by other CTAs (generic
-    // proxy) before the grid barrier; the bulk copies read them through the
-    // async proxy, and overwrite shared memory last written by generic stores
+    const int nch = (len + ACH - 1) / ACH;
+    const int pairs = a.B * a.H;
+    const long long Ctot = (long long)pairs * nch;
+    const int Wp = (int)min((long long)gridDim.x * NAW, Ctot);
+    const int gw = blockIdx.x * NAW + aw;
+    if (gw >= Wp) return true;
+    const long long cs = Ctot * gw / Wp, ce = Ctot * (gw + 1) / Wp;
+    auto owner = [&](long long i) { return (int)(((i + 1) * Wp - 1) / Ctot); };
+    const int PM = (Wp + pairs - 1) / pairs + 1;    // ranges that can touch one pair
+    const uint32_t wbuf = smem_u32(sm.att) + aw * 2 * C::ATT_BUF;
+    const uint32_t wbar = sm.abar + aw * 16;
+    // the cache rows and queries of this step were stored by other CTAs
+    // (generic proxy) before the grid barrier; the bulk copies read them
+    // through the async proxy, and overwrite shared memory that generic
+    // stores wrote before
     if (lane == 0) asm volatile("fence.proxy.async.global;\n\tfence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
-    // issue the first two chunks
-    AttnCursor is{0, 0};
-    int issued = 0;
-    for (; issued < 2 && item_of(is.j) < nitems; ++issued) {
+    // issue cursor: chunk ic = (pair ip, chunk kc_i of the pair)
+    long long ic = cs;
+    int ip = (int)(cs / nch), ikc = (int)(cs - (long long)ip * nch);
+    auto issue = [&](int buf) {
         if (lane == 0)
-            attn_issue<BN, HD>(a, l, item_of(is.j), is.c, nseg, len, wbuf + (issued & 1) * SCfg<BN, HD>::ATT_BUF,
-                               wbar + 8 * (issued & 1));
-        if (++is.c == chunks_of(item_of(is.j))) {
-            ++is.j;
-            is.c = 0;
+            attn_issue<BN, HD>(a, l, ip, ikc, ic == cs || ikc == 0, len, wbuf + buf * C::ATT_BUF, wbar + 8 * buf);
+        ++ic;
+        if (++ikc == nch) {
+            ikc = 0;
+            ++ip;
         }
-    }
+    };
+    issue(0);
+    if (ic < ce) issue(1);
     const float scale = rsqrtf((float)HD);
     float m = -INFINITY, lsum = 0.f, acc[DPL], qv[DPL];
-    int k = 0;
-    for (AttnCursor cur{0, 0}; item_of(cur.j) < nitems; ++k) {
-        const int item = item_of(cur.j);
-        const int seg = item % nseg, bh = item / nseg;
-        const int b = bh / a.H, h = bh - b * a.H;
-        const int nkeys = min(len - (seg * SEGK + cur.c * ACH), ACH);
-        if (cur.c == 0) {    // a new item: its query and a fresh state
-            const bf16* qp = a.q + ((size_t)b * a.H + h) * HD;
-#pragma unroll
-            for (int u = 0; u < NV; ++u) {
-                const uint4 w = __ldcg(reinterpret_cast<const uint4*>(qp + (u * 8 + r) * 8));
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const float2 f = unpack_bf16x2(ws[t]);
-                    qv[u * 8 + 2 * t] = f.x * scale;
-                    qv[u * 8 + 2 * t + 1] = f.y * scale;
-                }
-            }
-            m = -INFINITY;
-            lsum = 0.f;
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-        }
-        const int buf = k & 1;
+    int p = (int)(cs / nch), kc = (int)(cs - (long long)p * nch);
+    for (long long c = cs; c < ce; ++c) {
+        const int k = (int)(c - cs), buf = k & 1;
         const uint32_t bar = wbar + 8 * buf;
         bool ok = false;
         {
@@ -540,8 +530,28 @@ __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>
             }
             return false;
         }
-        const bf16* sk = reinterpret_cast<const bf16*>(sm.att + (size_t)(warp * 2 + buf) * SCfg<BN, HD>::ATT_BUF);
+        const uint8_t* bp = sm.att + (size_t)(aw * 2 + buf) * C::ATT_BUF;
+        const bf16* sk = reinterpret_cast<const bf16*>(bp);
         const bf16* sv = sk + ACH * HD;
+        if (c == cs || kc == 0) {    // a new pair: its query (in this buffer) and a fresh state
+            const bf16* qp = reinterpret_cast<const bf16*>(bp + C::ATT_Q);
+#pragma unroll
+            for (int u = 0; u < NV; ++u) {
+                const uint4 w = *reinterpret_cast<const uint4*>(qp + (u * 8 + r) * 8);
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const float2 f = unpack_bf16x2(ws[t]);
+                    qv[u * 8 + 2 * t] = f.x * scale;
+                    qv[u * 8 + 2 * t + 1] = f.y * scale;
+                }
+            }
+            m = -INFINITY;
+            lsum = 0.f;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+        }
+        const int nkeys = min(len - kc * ACH, ACH);
         // scores of this group's keys 4i + g (row 0 stands in for a missing key)
         float s[KPG];
 #pragma unroll
@@ -573,11 +583,11 @@ __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>
         const float m_new = fmaxf(m, cmax);
         if (m_new != -INFINITY) {   // this group holds at least one key so far
             const float corr = __expf(m - m_new);
-            float p[KPG], psum = 0.f;
+            float pk[KPG], psum = 0.f;
 #pragma unroll
             for (int i = 0; i < KPG; ++i) {
-                p[i] = (4 * i + g < nkeys) ? __expf(s[i] - m_new) : 0.f;
-                psum += p[i];
+                pk[i] = (4 * i + g < nkeys) ? __expf(s[i] - m_new) : 0.f;
+                psum += pk[i];
             }
             lsum = lsum * corr + psum;
 #pragma unroll
@@ -593,8 +603,8 @@ __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
                         const float2 fv = unpack_bf16x2(v4[t]);
-                        acc[u * 8 + 2 * t] = fmaf(p[i], fv.x, acc[u * 8 + 2 * t]);
-                        acc[u * 8 + 2 * t + 1] = fmaf(p[i], fv.y, acc[u * 8 + 2 * t + 1]);
+                        acc[u * 8 + 2 * t] = fmaf(pk[i], fv.x, acc[u * 8 + 2 * t]);
+                        acc[u * 8 + 2 * t + 1] = fmaf(pk[i], fv.y, acc[u * 8 + 2 * t + 1]);
                     }
                 }
             }
@@ -602,20 +612,14 @@ __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>
         }
         __syncwarp();
         // the buffer is free: put the chunk two places ahead in flight
-        if (item_of(is.j) < nitems) {
-            if (lane == 0)
-                attn_issue<BN, HD>(a, l, item_of(is.j), is.c, nseg, len, wbuf + buf * SCfg<BN, HD>::ATT_BUF, bar);
-            if (++is.c == chunks_of(item_of(is.j))) {
-                ++is.j;
-                is.c = 0;
-            }
+        if (ic < ce) issue(buf);
+        const int pr = p;
+        const bool pair_done = (c + 1 == ce) || (kc + 1 == nch);
+        if (++kc == nch) {
+            kc = 0;
+            ++p;
         }
-        const bool item_done = (cur.c + 1 == chunks_of(item));
-        if (++cur.c == chunks_of(item)) {
-            ++cur.j;
-            cur.c = 0;
-        }
-        if (!item_done) continue;
+        if (!pair_done) continue;
         // merge the four lane groups (each covers every 4th key)
 #pragma unroll
         for (int off = 8; off <= 16; off <<= 1) {
@@ -632,7 +636,26 @@ __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>
             }
             m = M;
         }
-        float* wp = a.attn_work + ((size_t)bh * nsegmax + seg) * (HD + 2);
+        const int b = pr / a.H, h = pr - b * a.H;
+        const long long pc0 = (long long)pr * nch;
+        const int first = owner(pc0), nparts = owner(pc0 + nch - 1) - first + 1;
+        bf16* dst = a.attn + (size_t)b * a.d + (size_t)h * HD;
+        if (nparts == 1) {    // the whole pair in this range
+            const float inv = 1.f / lsum;
+            if (g == 0) {
+#pragma unroll
+                for (int u = 0; u < NV; ++u) {
+                    uint4 o;
+                    o.x = pack_bf16x2(acc[u * 8 + 0] * inv, acc[u * 8 + 1] * inv);
+                    o.y = pack_bf16x2(acc[u * 8 + 2] * inv, acc[u * 8 + 3] * inv);
+                    o.z = pack_bf16x2(acc[u * 8 + 4] * inv, acc[u * 8 + 5] * inv);
+                    o.w = pack_bf16x2(acc[u * 8 + 6] * inv, acc[u * 8 + 7] * inv);
+                    *reinterpret_cast<uint4*>(dst + (u * 8 + r) * 8) = o;
+                }
+            }
+            continue;
+        }
+        float* wp = a.attn_work + ((size_t)pr * PM + (gw - first)) * (HD + 2);
         if (g == 0) {
 #pragma unroll
             for (int u = 0; u < NV; ++u)
@@ -643,48 +666,48 @@ __device__ bool phase_attn(const StepArgs& a, int l, int tid, const Smem<BN, HD>
                 wp[1] = lsum;
             }
         }
-        __threadfence();
         __syncwarp();
         int last = 0;
         if (lane == 0) {
-            const int prev = atomicAdd(a.attn_cnt + bh, 1);
-            last = (prev == nseg - 1);
-            if (last) a.attn_cnt[bh] = 0;
+            __threadfence();
+            const int prev = atomicAdd(a.attn_cnt + pr, 1);
+            last = (prev == nparts - 1);
+            if (last) {
+                a.attn_cnt[pr] = 0;
+                __threadfence();
+            }
         }
         last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-            __threadfence();
-            const float* wb = a.attn_work + (size_t)bh * nsegmax * (HD + 2);
-            // lane c owns segment c (and c + 32, ...): maxima and weighted sums by shuffles
-            float Mall = -INFINITY;
-            for (int c = lane; c < nseg; c += 32) Mall = fmaxf(Mall, __ldcg(wb + (size_t)c * (HD + 2)));
-            Mall = warp_max(Mall);
-            float L = 0.f, o[DPW];
+        if (!last) continue;
+        const float* wb = a.attn_work + (size_t)pr * PM * (HD + 2);
+        // lane j owns range j (and j + 32, ...): maxima and weighted sums by shuffles
+        float Mall = -INFINITY;
+        for (int j = lane; j < nparts; j += 32) Mall = fmaxf(Mall, __ldcg(wb + (size_t)j * (HD + 2)));
+        Mall = warp_max(Mall);
+        float L = 0.f, o[DPW];
 #pragma unroll
-            for (int e = 0; e < DPW; ++e) o[e] = 0.f;
-            for (int c0 = 0; c0 < nseg; c0 += 32) {
-                const int c = c0 + lane;
-                float w = 0.f;
-                if (c < nseg) {
-                    const float mc = __ldcg(wb + (size_t)c * (HD + 2));
-                    w = (mc == -INFINITY) ? 0.f : __expf(mc - Mall);
-                    L += __ldcg(wb + (size_t)c * (HD + 2) + 1) * w;
-                }
-                const int cn = min(32, nseg - c0);
-#pragma unroll 4
-                for (int t = 0; t < cn; ++t) {
-                    const float wt = __shfl_sync(0xffffffffu, w, t);
-                    const float* pc = wb + (size_t)(c0 + t) * (HD + 2) + 2 + lane * DPW;
-#pragma unroll
-                    for (int e = 0; e < DPW; ++e) o[e] = fmaf(__ldcg(pc + e), wt, o[e]);
-                }
+        for (int e = 0; e < DPW; ++e) o[e] = 0.f;
+        for (int j0 = 0; j0 < nparts; j0 += 32) {
+            const int j = j0 + lane;
+            float w = 0.f;
+            if (j < nparts) {
+                const float mj = __ldcg(wb + (size_t)j * (HD + 2));
+                w = (mj == -INFINITY) ? 0.f : __expf(mj - Mall);
+                L += __ldcg(wb + (size_t)j * (HD + 2) + 1) * w;
             }
-            L = warp_sum(L);
-            const float inv = 1.f / L;
-            bf16* dst = a.attn + (size_t)b * a.d + (size_t)h * HD + lane * DPW;
+            const int jn = min(32, nparts - j0);
+#pragma unroll 4
+            for (int t = 0; t < jn; ++t) {
+                const float wt = __shfl_sync(0xffffffffu, w, t);
+                const float* pc = wb + (size_t)(j0 + t) * (HD + 2) + 2 + lane * DPW;
 #pragma unroll
-            for (int e = 0; e < DPW; ++e) dst[e] = __float2bfloat16_rn(o[e] * inv);
+                for (int e = 0; e < DPW; ++e) o[e] = fmaf(__ldcg(pc + e), wt, o[e]);
+            }
         }
+        L = warp_sum(L);
+        const float inv = 1.f / L;
+#pragma unroll
+        for (int e = 0; e < DPW; ++e) dst[lane * DPW + e] = __float2bfloat16_rn(o[e] * inv);
     }
     return true;
 }
@@ -779,8 +802,8 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
     sm.empty = bars + 8 * C::STAGES;
     sm.tfull = bars + 16 * C::STAGES;
     sm.tempty = sm.tfull + 16;
-    sm.abar = sm.tempty + 16;                                       // [4 warps][2]
-    uint32_t* misc = reinterpret_cast<uint32_t*>(gb + C::OFF_BAR + 16 * C::STAGES + 32 + 64);
+    sm.abar = sm.tempty + 16;                                       // [NAW warps][2]
+    uint32_t* misc = reinterpret_cast<uint32_t*>(gb + C::OFF_MISC);
     uint32_t* tmem_slot = misc;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
     sm.flag = reinterpret_cast<volatile int*>(misc + 2);
@@ -797,14 +820,14 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
             mbar_init(sm.tfull + 8 * i, 1);
             mbar_init(sm.tempty + 8 * i, 128);
         }
-        for (int i = 0; i < 8; ++i) mbar_init(sm.abar + 8 * i, 1);
+        for (int i = 0; i < 2 * NAW; ++i) mbar_init(sm.abar + 8 * i, 1);
         *abort_flag = 0;
         // no barrier of this launch can complete before every CTA arrives,
         // so all CTAs read the same starting generation here
         *base_gen = ld_acquire_u32(bar_flag(a.bar, blockIdx.x));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 1) {
+    if (warp == 5) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(C::TMEM_COLS)
                      : "memory");
@@ -816,7 +839,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
     const uint32_t tmem = *tmem_slot;
     const unsigned gen0 = *base_gen;
 
-    if (warp == 0) {
+    if (warp == 4) {
         // -------------------------------------------------------- TMA producer
         // Two cursors over the same stage sequence: weight tiles are requested
         // as soon as a ring slot frees; the activation tile of a stage only
@@ -884,7 +907,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                 }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 5) {
         // -------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t IDESC = idesc_bf16(BN);
@@ -933,10 +956,10 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                 }
             }
         }
-    } else {
-        // -------------------------------------------------------- epilogue warps 2..5
-        const int tid = threadIdx.x - 64;
-        const int quarter = warp & 3;
+    } else if (warp < 4) {
+        // -------------------------------------------------------- epilogue warps 0..3
+        const int tid = threadIdx.x;
+        const int quarter = warp;
         const int et = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         int acc = 0;
@@ -979,7 +1002,8 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                     }
                 }
             } else if (type == PH_ATTN) {
-                fail = !phase_attn<BN, HD>(a, l, tid, sm, uses, abort_flag);
+                fail = !phase_attn<BN, HD>(a, l, warp, lane, sm, uses, abort_flag);
+                asm volatile("bar.sync 2, 192;" ::: "memory");   // with attention warps 6, 7
             } else if (type == PH_ARGMAX) {
                 phase_argmax<BN, HD>(a, tid, sm);
             } else {
@@ -1037,11 +1061,30 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
             if (tl && tid == 0) tl[2 * p + 1] = global_timer();
             if (p + 1 < P) grid_arrive(a.bar, gen0 + (unsigned)p + 1u, tid, sm.flag);
         }
+    } else {
+        // -------------------------------------------------------- attention warps 6, 7
+        // They join the epilogue warps in each attention phase: wait for the
+        // barrier that opens it, take their share, and arrive at the named
+        // barrier the epilogue warps pass before they leave the phase (once
+        // per layer, also after a failure, so that nobody waits for them).
+        uint32_t uses[2] = {0u, 0u};
+        bool ok = true;
+        for (int l = 0; l < a.L; ++l) {
+            const int p = 2 + 5 * l;      // embed, then per layer QKV, attention, ...
+            if (ok) {
+                int w = 1;
+                if (lane == 0) w = wait_gen(bar_flag(a.bar, blockIdx.x), gen0 + (unsigned)p, abort_flag, a.err);
+                ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+                if (ok) ok = phase_attn<BN, HD>(a, l, warp - 2, lane, sm, uses, abort_flag);
+            }
+            __syncwarp();
+            asm volatile("bar.arrive 2, 192;" ::: "memory");
+        }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 5) {
         __syncwarp();
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)

@@ -65,8 +65,10 @@ int launch_gemm_tc(const TcGemm& g, int mode, const EpiArgs& a, int* err, cudaSt
 int gemm_tc_pick_splits(int rowsA, int K);
 
 // decode_step.cu  (one cooperative kernel per greedy decode step, bf16)
-// At most this many CTAs run the fused decode step (one per SM).
+// At most this many CTAs run the fused decode step (one per SM), each with
+// this many warps working on attention.
 constexpr int STEP_MAX_CTAS = 160;
+constexpr int STEP_ATTN_WARPS = 6;
 // Partial-sum slots per output feature of a projection with `mblk` 128-row
 // blocks when its (block, k-block) iterations are cut into `ctas` equal
 // contiguous ranges: no block is touched by more ranges than this.
@@ -88,7 +90,7 @@ struct StepArgs {
     long long part_off[5];        // qkv, o, gate/up, down, head (floats)
     int* counters;                // arrival counters, one region per projection kind
     int cnt_off[5];
-    float* attn_work;             // attention chunk partials [B*H][ceil(smax/128)][hd + 2]
+    float* attn_work;             // attention partials [B*H][ranges per pair][hd + 2]
     int* attn_cnt;                // [B*H]
     int2* amax_part;              // [B][ceil(V/2048)]
     int* amax_cnt;                // [B + 1]

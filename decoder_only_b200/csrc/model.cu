@@ -263,8 +263,10 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     unsigned int* step_bar = (unsigned int*)take(32 * 1024);   // arrivals + one 128-byte flag per CTA
     void* step_xg2 = take((size_t)c->max_batch * d * esz);
     float* step_ssq = (float*)take(2 * 64 * 32 * 4);
-    float* step_attn_work = (float*)take((size_t)c->max_batch * c->n_heads * ((c->max_seq + 127) / 128) *
-                                         (c->head_dim + 2) * 4);
+    // attention partials of the fused decode step: pairs * (ranges per pair)
+    // <= pairs * (ceil(W / pairs) + 1) <= W + 2 * pairs for W attention warps
+    float* step_attn_work = (float*)take(((size_t)STEP_MAX_CTAS * STEP_ATTN_WARPS + 2 * (size_t)c->max_batch *
+                                          c->n_heads) * (c->head_dim + 2) * 4);
     // per-phase timestamps of the fused decode step (profiling): 2 per CTA per phase
     unsigned long long* step_timeline = (unsigned long long*)take((size_t)1024 * (3 + 5 * L) * 2 * 8);
     int2* amax_part = (int2*)take((size_t)c->max_batch * argmax_split_chunks(c->vocab) * sizeof(int2));
@@ -1006,7 +1008,7 @@ int64_t llama_kernel_launches(void) { return g_launches.load(); }
 
 int llama_step_timeline(llama_model* m, uint64_t* h_out, int64_t n, int32_t* ctas, int32_t* phases) {
     if (!m || m->cfg.dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
-    const int P = 3 + 5 * m->cfg.n_layers, G = tc_num_sms();
+    const int P = 3 + 5 * m->cfg.n_layers, G = decode_step_ctas();
     if (ctas) *ctas = G;
     if (phases) *phases = P;
     const int64_t need = (int64_t)G * P * 2;
