@@ -448,14 +448,19 @@ __device__ __forceinline__ void attn_issue(const StepArgs& a, int l, int pr, int
     const bf16* vc = kc_ + a.kv_layer;
     const size_t off = ((size_t)pr * a.smax + k0) * HD;     // pair pr = b * H + h
     const uint32_t bytes = (uint32_t)(nkeys * HD * 2);
+    // cache rows are read once per step: first out of L2
+    const uint64_t pol = l2_evict_first();
     mbar_expect_tx(bar, 2 * bytes + (with_q ? HD * 2 : 0));
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(kc_ + off), "r"(bytes), "r"(bar)
-                 : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     dst + ACH * HD * 2),
-                 "l"(vc + off), "r"(bytes), "r"(bar)
-                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+            "r"(dst),
+        "l"(kc_ + off), "r"(bytes), "r"(bar), "l"(pol)
+        : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+            "r"(dst + ACH * HD * 2),
+        "l"(vc + off), "r"(bytes), "r"(bar), "l"(pol)
+        : "memory");
     if (with_q)
         asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                          dst + SCfg<BN, HD>::ATT_Q),
@@ -849,6 +854,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
             cursor_seek(a, P, wc, 0);
             xc = wc;
             int wn = 0, xn = 0, ready = -1;
+            const uint64_t wpol = l2_evict_first();   // a weight tile is read once per step
             const unsigned* myflag = bar_flag(a.bar, blockIdx.x);
             uint64_t t_last = global_timer();
             while (xc.valid) {
@@ -858,7 +864,8 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                     if (mbar_test(sm.empty + 8 * slot, ((wn / C::STAGES) & 1) ^ 1)) {
                         const int mb = wc.i / wc.kbt, kb = wc.i - mb * wc.kbt;
                         mbar_expect_tx(sm.full + 8 * slot, C::STAGE_BYTES);
-                        tma_load_2d(sm.sA + slot * C::A_BYTES, a.maps + wc.map_a, sm.full + 8 * slot, kb * BK, mb * BM);
+                        tma_load_2d_hint(sm.sA + slot * C::A_BYTES, a.maps + wc.map_a, sm.full + 8 * slot, kb * BK,
+                                         mb * BM, wpol);
                         ++wn;
                         cursor_next(a, P, wc);
                         prog = true;
