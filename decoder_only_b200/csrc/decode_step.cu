@@ -217,46 +217,66 @@ __device__ __forceinline__ bool esync_any(bool pred) {
     return r != 0;
 }
 
-// Grid barrier state: bar[0] counts arrivals; CTA i polls its own release
-// flag bar[32 + 32 i] (a 128-byte line of its own), which the last CTA to
-// arrive sets to the next generation.
-__device__ __forceinline__ unsigned* bar_flag(unsigned* bar, int cta) { return bar + 32 + 32 * cta; }
+// Step synchronisation words in a.bar (32-bit words; each group on a
+// 128-byte line of its own).  Phases are not separated by grid barriers:
+// every unit of work that produces an input of a later phase (a finished
+// 128-row block of a projection, a finished attention pair) adds one to its
+// completion count, and a consumer waits until the count it depends on is
+// complete.
+//   [0]                     epoch of the last completed step
+//   [32]                    CTAs that have started the running step
+//   [64]                    epoch whose embedding (and count reset) is done
+//   [96]                    embedded rows of the running step
+//   [128 + 32 (8 l + k)]    completion count of kind k in layer l (l = L: head)
+constexpr int SY_EPOCH = 0, SY_CHECKIN = 32, SY_EMBED = 64, SY_ROWS = 96, SY_DONE = 128;
+enum DoneKind { DK_QKV = 0, DK_ATTN = 1, DK_O = 2, DK_GU = 3, DK_DOWN = 4, DK_HEAD = 0 };
 
-// Bounded wait until this CTA's release flag reaches generation `target`.
-__device__ bool wait_gen(const unsigned* flag, unsigned target, volatile int* abort_flag, int* err) {
-    if ((int)(ld_acquire_u32(flag) - target) >= 0) return true;
+__device__ __forceinline__ unsigned* done_ctr(const StepArgs& a, int l, int k) {
+    return a.bar + SY_DONE + 32 * (8 * l + k);
+}
+
+// Bounded wait until *p >= target (signed difference: epochs wrap)
+__device__ bool wait_at_least(const unsigned* p, unsigned target, volatile int* abort_flag, int* err) {
+    if ((int)(ld_acquire_u32(p) - target) >= 0) return true;
     const uint64_t t0 = global_timer();
     while (true) {
-        if ((int)(ld_acquire_u32(flag) - target) >= 0) return true;
+        if ((int)(ld_acquire_u32(p) - target) >= 0) return true;
         if (*abort_flag) return false;
         if (global_timer() - t0 > WAIT_LIMIT_NS) {
             *abort_flag = 1;
             atomicOr(err, LLAMA_DEVERR_TIMEOUT);
             return false;
         }
-        __nanosleep(20);
+        __nanosleep(64);
     }
 }
 
-// Arrival of this CTA (all 128 epilogue threads call it after their work);
-// the last CTA to arrive resets the count and releases every CTA's flag.
-__device__ void grid_arrive(unsigned* bar, unsigned next_gen, int tid, volatile int* last_flag) {
-    if (tid == 0) {
-        __threadfence();
-        const unsigned prev = atomicAdd(bar, 1u);
-        const int last = (prev == gridDim.x - 1);
-        if (last) {
-            atomicExch(bar, 0u);
-            __threadfence();
-        }
-        *last_flag = last;
+// One finished unit; the caller's fence makes the CTA's writes before it
+// (ordered by a CTA barrier) visible first
+__device__ __forceinline__ void count_done(unsigned* p) {
+    __threadfence();
+    atomicAdd(p, 1u);
+}
+
+// The completion count (and its complete value) that phase `type` of layer
+// l reads its input after; nullptr: the embedding, which every role of
+// every CTA waits for before anything else.
+__device__ __forceinline__ const unsigned* dep_of(const StepArgs& a, int type, int l, unsigned& target) {
+    const unsigned nd = (unsigned)(a.d / BM);
+    switch (type) {
+        case PH_QKV:
+            target = nd;
+            return l == 0 ? nullptr : done_ctr(a, l - 1, DK_DOWN);
+        case PH_ATTN: target = (unsigned)(3 * a.d / BM); return done_ctr(a, l, DK_QKV);
+        case PH_O: target = (unsigned)(a.B * a.H); return done_ctr(a, l, DK_ATTN);
+        case PH_GU: target = nd; return done_ctr(a, l, DK_O);
+        case PH_DOWN: target = (unsigned)(a.h / BM); return done_ctr(a, l, DK_GU);
+        case PH_HEAD:
+            target = nd;
+            return a.L == 0 ? nullptr : done_ctr(a, a.L - 1, DK_DOWN);
+        case PH_ARGMAX: target = (unsigned)(a.V / BM); return done_ctr(a, a.L, DK_HEAD);
+        default: return nullptr;
     }
-    esync();
-    if (*last_flag) {
-        for (int i = tid; i < (int)gridDim.x; i += 128)
-            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(bar_flag(bar, i)), "r"(next_gen) : "memory");
-    }
-    esync();
 }
 
 template <int BN, int HD>
@@ -372,6 +392,8 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
                 const float inv = sm.sinv[b];
                 a.act[(size_t)b * a.h + 128 * j + et] = __float2bfloat16_rn(silu_f(gs[b] * inv) * (us[b] * inv));
             }
+        esync();
+        if (tid == 0) count_done(done_ctr(a, l, DK_GU));
     } else {
         float sum[BN];
         if (direct) {
@@ -384,6 +406,8 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
 #pragma unroll
             for (int b = 0; b < BN; ++b)
                 if (b < M) ep.out[(size_t)b * ep.ld_out + n] = sum[b] * sm.sinv[b];
+            esync();
+            if (tid == 0) count_done(done_ctr(a, a.L, DK_HEAD));
         } else if constexpr (MODE == EPI_RESID) {
             // trunk += the block's sum; then the next norm's inputs: bf16(g * x)
             // and the block's sum of squares per row
@@ -408,6 +432,7 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
                 if (lane == 0) ssq[mb * 32 + b] = s;
             }
             esync();
+            if (tid == 0) count_done(done_ctr(a, l, to_ffn ? DK_O : DK_DOWN));
         } else {   // EPI_QKV: 1/rms, then RoPE and the cache append on 32-column rows
 #pragma unroll
             for (int b = 0; b < BN; ++b)
@@ -421,6 +446,7 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
                 epi_qkv32<bf16>(ep, b, mb * BM + c * 32, x);
             }
             esync();
+            if (tid == 0) count_done(done_ctr(a, l, DK_QKV));
         }
     }
 }
@@ -658,6 +684,8 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
                     *reinterpret_cast<uint4*>(dst + (u * 8 + r) * 8) = o;
                 }
             }
+            __syncwarp();
+            if (lane == 0) count_done(done_ctr(a, l, DK_ATTN));
             continue;
         }
         float* wp = a.attn_work + ((size_t)pr * PM + (gw - first)) * (HD + 2);
@@ -713,6 +741,8 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
         const float inv = 1.f / L;
 #pragma unroll
         for (int e = 0; e < DPW; ++e) dst[lane * DPW + e] = __float2bfloat16_rn(o[e] * inv);
+        __syncwarp();
+        if (lane == 0) count_done(done_ctr(a, l, DK_ATTN));
     }
     return true;
 }
@@ -721,7 +751,7 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
 __device__ bool amx_better(float v, int i, float bv, int bi) { return v > bv || (v == bv && i < bi); }
 
 template <int BN, int HD>
-__device__ void phase_argmax(const StepArgs& a, int tid, const Smem<BN, HD>& sm) {
+__device__ void phase_argmax(const StepArgs& a, int tid, const Smem<BN, HD>& sm, unsigned E, volatile int* abort_flag) {
     const int nc = (a.V + AMX - 1) / AMX;
     const int nitems = a.B * nc;
     int* sidx = reinterpret_cast<int*>(sm.red + 8);
@@ -778,6 +808,11 @@ __device__ void phase_argmax(const StepArgs& a, int tid, const Smem<BN, HD>& sm)
                 const int rows = atomicAdd(a.amax_cnt + a.B, 1);
                 if (rows == a.B - 1) {
                     a.amax_cnt[a.B] = 0;
+                    // close the step once every CTA has started it (and so
+                    // has read its epoch)
+                    wait_at_least(a.bar + SY_CHECKIN, gridDim.x, abort_flag, a.err);
+                    a.bar[SY_CHECKIN] = 0;
+                    a.bar[SY_EPOCH] = E;
                     *a.d_pos += 1;
                 }
             }
@@ -812,7 +847,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
     uint32_t* tmem_slot = misc;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
     sm.flag = reinterpret_cast<volatile int*>(misc + 2);
-    volatile unsigned* base_gen = reinterpret_cast<volatile unsigned*>(misc + 3);
+    volatile unsigned* epoch = reinterpret_cast<volatile unsigned*>(misc + 3);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = phase_count(a);
@@ -827,9 +862,10 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
         }
         for (int i = 0; i < 2 * NAW; ++i) mbar_init(sm.abar + 8 * i, 1);
         *abort_flag = 0;
-        // no barrier of this launch can complete before every CTA arrives,
-        // so all CTAs read the same starting generation here
-        *base_gen = ld_acquire_u32(bar_flag(a.bar, blockIdx.x));
+        // this step's epoch; the step is closed (and the word advanced) only
+        // after every CTA has checked in here
+        *epoch = ld_acquire_u32(a.bar + SY_EPOCH) + 1u;
+        atomicAdd(a.bar + SY_CHECKIN, 1u);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 5) {
@@ -842,22 +878,23 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const unsigned gen0 = *base_gen;
+    const unsigned E = *epoch;
 
     if (warp == 4) {
         // -------------------------------------------------------- TMA producer
         // Two cursors over the same stage sequence: weight tiles are requested
         // as soon as a ring slot frees; the activation tile of a stage only
-        // once the grid barrier before its phase has released this CTA.
+        // once the completion count its phase reads after is complete.
         if (lane == 0) {
             Cursor wc, xc;
             cursor_seek(a, P, wc, 0);
             xc = wc;
             int wn = 0, xn = 0, ready = -1;
             const uint64_t wpol = l2_evict_first();   // a weight tile is read once per step
-            const unsigned* myflag = bar_flag(a.bar, blockIdx.x);
+            // the embedding (and the reset of the completion counts) first
+            bool ok0 = wait_at_least(a.bar + SY_EMBED, E, abort_flag, a.err);
             uint64_t t_last = global_timer();
-            while (xc.valid) {
+            while (xc.valid && ok0) {
                 bool prog = false;
                 if (wc.valid && wn - xn < C::STAGES) {
                     const int slot = wn % C::STAGES;
@@ -872,9 +909,15 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                     }
                 }
                 if (xn < wn) {
-                    if (ready < xc.p && (int)(ld_acquire_u32(myflag) - (gen0 + (unsigned)xc.p)) >= 0) {
-                        asm volatile("fence.proxy.async.global;" ::: "memory");
-                        ready = xc.p;
+                    if (ready < xc.p) {
+                        int l;
+                        const int type = phase_type(a, xc.p, l);
+                        unsigned tgt = 0;
+                        const unsigned* dp = dep_of(a, type, l, tgt);
+                        if (!dp || (int)(ld_acquire_u32(dp) - tgt) >= 0) {
+                            asm volatile("fence.proxy.async.global;" ::: "memory");
+                            ready = xc.p;
+                        }
                     }
                     if (ready >= xc.p) {
                         const int slot = xn % C::STAGES;
@@ -976,17 +1019,28 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
         for (int p = 0; p < P; ++p) {
             int l;
             const int type = phase_type(a, p, l);
-            if (p > 0) {
+            {
+                // wait for this phase's input (its completion count; before
+                // the first projection also the embedding, which zeroes the
+                // counts)
                 bool ok = true;
-                if (tid == 0) ok = wait_gen(bar_flag(a.bar, blockIdx.x), gen0 + (unsigned)p, abort_flag, a.err);
+                if (tid == 0) {
+                    unsigned tgt = 0;
+                    const unsigned* dp = (type == PH_EMBED) ? nullptr : dep_of(a, type, l, tgt);
+                    if (dp) ok = wait_at_least(dp, tgt, abort_flag, a.err);
+                    // the embedding (and the zeroed counts) before anything else
+                    if (ok && p == 1) ok = wait_at_least(a.bar + SY_EMBED, E, abort_flag, a.err);
+                }
                 if (esync_any(!ok)) break;
             }
             if (tl && tid == 0) tl[2 * p] = global_timer();
             bool fail = false;
             if (type == PH_EMBED) {
-                // trunk row b = embedding of its token; bf16(g * x) of the
-                // first attention norm and the 128-feature block sums of
-                // squares (one warp per block: 32 lanes x 4 features)
+                // CTA b < B: the embedding of row b's token, bf16(g * x) of
+                // the first attention norm and the row's 128-feature block
+                // sums of squares (one warp per block: 32 lanes x 4
+                // features).  The last row to finish zeroes the completion
+                // counts of this step and publishes its epoch.
                 if ((int)blockIdx.x < a.B) {
                     const int b = blockIdx.x;
                     int t = a.tok[b];
@@ -1007,12 +1061,29 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                         const float s = warp_sum((v01.x * v01.x + v01.y * v01.y) + (v23.x * v23.x + v23.y * v23.y));
                         if (lane == 0) a.ssq[(i >> 7) * 32 + b] = s;
                     }
+                    esync();
+                    int last = 0;
+                    if (tid == 0) {
+                        __threadfence();
+                        const unsigned prev = atomicAdd(a.bar + SY_ROWS, 1u);
+                        last = (prev == (unsigned)a.B - 1u);
+                        if (last) a.bar[SY_ROWS] = 0u;
+                    }
+                    if (esync_any(last)) {
+                        for (int i = tid; i < 8 * (a.L + 1); i += 128) a.bar[SY_DONE + 32 * i] = 0u;
+                        esync();
+                        if (tid == 0) {
+                            __threadfence();
+                            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a.bar + SY_EMBED), "r"(E)
+                                         : "memory");
+                        }
+                    }
                 }
             } else if (type == PH_ATTN) {
                 fail = !phase_attn<BN, HD>(a, l, warp, lane, sm, uses, abort_flag);
                 asm volatile("bar.sync 2, 192;" ::: "memory");   // with attention warps 6, 7
             } else if (type == PH_ARGMAX) {
-                phase_argmax<BN, HD>(a, tid, sm);
+                phase_argmax<BN, HD>(a, tid, sm, E, abort_flag);
             } else {
                 Work w;
                 work_of(a, type, l, w);
@@ -1066,7 +1137,6 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
             }
             if (esync_any(fail)) break;
             if (tl && tid == 0) tl[2 * p + 1] = global_timer();
-            if (p + 1 < P) grid_arrive(a.bar, gen0 + (unsigned)p + 1u, tid, sm.flag);
         }
     } else {
         // -------------------------------------------------------- attention warps 6, 7
@@ -1075,12 +1145,17 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
         // barrier the epilogue warps pass before they leave the phase (once
         // per layer, also after a failure, so that nobody waits for them).
         uint32_t uses[2] = {0u, 0u};
-        bool ok = true;
+        int w = 1;
+        if (lane == 0) w = wait_at_least(a.bar + SY_EMBED, E, abort_flag, a.err);
+        bool ok = __shfl_sync(0xffffffffu, w, 0) != 0;
         for (int l = 0; l < a.L; ++l) {
-            const int p = 2 + 5 * l;      // embed, then per layer QKV, attention, ...
             if (ok) {
-                int w = 1;
-                if (lane == 0) w = wait_gen(bar_flag(a.bar, blockIdx.x), gen0 + (unsigned)p, abort_flag, a.err);
+                w = 1;
+                if (lane == 0) {
+                    unsigned tgt = 0;
+                    const unsigned* dp = dep_of(a, PH_ATTN, l, tgt);
+                    w = wait_at_least(dp, tgt, abort_flag, a.err);
+                }
                 ok = __shfl_sync(0xffffffffu, w, 0) != 0;
                 if (ok) ok = phase_attn<BN, HD>(a, l, warp - 2, lane, sm, uses, abort_flag);
             }

@@ -97,7 +97,7 @@ struct StepArgs {
     int32_t* tok;
     int* d_pos;
     int* err;
-    unsigned int* bar;            // grid barrier: [0] arrivals, [32 + 32 i] release flag of CTA i
+    unsigned int* bar;            // step synchronisation words [decode_step_sync_words(L)]
     unsigned long long* timeline; // optional: per CTA and phase, start / end %globaltimer stamps
     const float2* rope;
     int L, d, h, V, H, hd, B, smax;
@@ -109,6 +109,7 @@ int decode_step_maps(CUtensorMap* host_maps, const void* const* w, int L, const 
                      const void* attn, const void* act, const void* xg2, int B, int d, int h, int V);
 // Grid of the fused decode step, and the partial / counter regions for batch B
 int decode_step_ctas();
+inline size_t decode_step_sync_words(int L) { return 128 + 256 * (size_t)(L + 1); }
 long long decode_step_layout(int ctas, int d, int h, int V, int B, long long part_off[5], int cnt_off[5]);
 // 2-D K-major bf16 tensor map, box (64, box_rows), 128-byte swizzle, zero fill
 int tc_make_map_2d(CUtensorMap* map, const void* ptr, int rows, int K, int box_rows);

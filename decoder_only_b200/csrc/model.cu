@@ -156,7 +156,7 @@ struct llama_model {
     int* attn_cnt;           // decode-attention arrival counters [max_batch * H]
     CUtensorMap* step_maps;  // decode-step tensor-map table (device) [4L + 5]
     const float** step_gains;  // decode-step gain table (device) [2L + 1]
-    unsigned int* step_bar;  // decode-step grid barrier [2]
+    unsigned int* step_bar;  // decode-step synchronisation words
     void* step_xg2;          // decode-step FFN-norm input g * x, bf16 [max_batch, d]
     float* step_ssq;         // decode-step block sums of squares [2][64][32]
     float* step_attn_work;   // decode-step attention partials
@@ -260,7 +260,7 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     int* attn_cnt = (int*)take((size_t)c->max_batch * c->n_heads * 4);
     CUtensorMap* step_maps = (CUtensorMap*)take((size_t)(4 * L + 5) * sizeof(CUtensorMap));
     const float** step_gains = (const float**)take((size_t)(2 * L + 1) * sizeof(float*));
-    unsigned int* step_bar = (unsigned int*)take(32 * 1024);   // arrivals + one 128-byte flag per CTA
+    unsigned int* step_bar = (unsigned int*)take(decode_step_sync_words((int)L) * 4);
     void* step_xg2 = take((size_t)c->max_batch * d * esz);
     float* step_ssq = (float*)take(2 * 64 * 32 * 4);
     // attention partials of the fused decode step: pairs * (ranges per pair)
@@ -710,7 +710,7 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
     }
     if (cudaMemsetAsync(m->counters, 0, MAX_COUNTERS * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->amax_cnt, 0, (size_t)(cfg->max_batch + 1) * 4, st) != cudaSuccess ||
-        cudaMemsetAsync(m->step_bar, 0, 32 * 1024, st) != cudaSuccess ||
+        cudaMemsetAsync(m->step_bar, 0, decode_step_sync_words(cfg->n_layers) * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->attn_cnt, 0, (size_t)cfg->max_batch * cfg->n_heads * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->d_pos, 0, 256, st) != cudaSuccess) {
         llama_free(m);
