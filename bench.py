@@ -23,6 +23,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -167,6 +168,29 @@ def kernel_family(region: str) -> str:
     return region
 
 
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "decode_step_llama7b_2layer_dram.md")
+STEP_SOURCE = os.path.join(ROOT, "decoder_only_b200", "csrc", "decode_step.cu")
+
+
+def decode_step_traffic_ratio():
+    """DRAM traffic / algorithmic bytes of the fused decode step from the
+    committed ncu summary, or None when the kernel source has changed since
+    the counters were taken."""
+    import hashlib
+    try:
+        with open(TRAFFIC_PROFILE) as f:
+            txt = f.read()
+        with open(STEP_SOURCE, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    ratio = re.search(r"traffic_ratio:\s*([0-9.]+)", txt)
+    src = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", txt)
+    if not ratio or not src or src.group(1) != h:
+        return None
+    return float(ratio.group(1))
+
+
 def roofline(prof, decode_scale, peaks, peak_src):
     """Dominant kernel over one step from the live per-region timing."""
     fam = {}
@@ -189,8 +213,13 @@ def roofline(prof, decode_scale, peaks, peak_src):
         achieved = f["bytes"] / (f["ms"] * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         out = dict(bound="hbm", unit="GB/s", peak_kind="HBM copy bandwidth")
+    traffic = None
+    if name == "decode_step":
+        r = decode_step_traffic_ratio()
+        if r is not None:   # bytes per launch: measured ratio x this launch's algorithmic bytes
+            traffic = round(r * f["bytes"] / max(f["launches"], 1))
     out.update(kernel=name, achieved=round(achieved, 1), peak=peak, frac=round(achieved / peak, 4),
-               peak_source=peak_src, traffic=None, launches_profiled=f["launches"],
+               peak_source=peak_src, traffic=traffic, launches_profiled=f["launches"],
                avg_launch_us=round(per_launch_ms * 1e3, 2), share_of_step=round(f["step_ms"] / total, 4),
                shares={k: round(v["step_ms"] / total, 4) for k, v in sorted(fam.items(), key=lambda kv: -kv[1]["step_ms"])},
                est_ms_per_step={k: round(v["step_ms"], 2) for k, v in sorted(fam.items(), key=lambda kv: -kv[1]["step_ms"])})
