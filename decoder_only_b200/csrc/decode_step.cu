@@ -155,9 +155,13 @@ __device__ __forceinline__ int owner_of(long long i, const Work& w) { return (in
 
 // Walk over this CTA's projection iterations of the whole step, in order.
 struct Cursor {
-    int p, i, e, kbt, map_a, map_b;
+    int p, i, e, kbt, mb, kb, map_a, map_b;
+    const unsigned* dep;   // completion count this phase's activations wait for (nullptr: none)
+    unsigned tgt;
     bool valid;
 };
+
+__device__ const unsigned* dep_of(const StepArgs& a, int type, int l, unsigned& target);
 
 __device__ void cursor_seek(const StepArgs& a, int P, Cursor& c, int p0) {
     for (int p = p0; p < P; ++p) {
@@ -169,16 +173,26 @@ __device__ void cursor_seek(const StepArgs& a, int P, Cursor& c, int p0) {
         c.i = w.s;
         c.e = w.e;
         c.kbt = w.kbt;
+        c.mb = w.s / w.kbt;
+        c.kb = w.s - c.mb * w.kbt;
         c.map_a = w.g.map_a;
         c.map_b = w.g.map_b;
+        c.dep = dep_of(a, type, l, c.tgt);
         c.valid = true;
         return;
     }
     c.valid = false;
 }
 
+// Next iteration: block and k-block advance without a division
 __device__ __forceinline__ void cursor_next(const StepArgs& a, int P, Cursor& c) {
-    if (++c.i < c.e) return;
+    if (++c.i < c.e) {
+        if (++c.kb == c.kbt) {
+            c.kb = 0;
+            ++c.mb;
+        }
+        return;
+    }
     cursor_seek(a, P, c, c.p + 1);
 }
 
@@ -261,7 +275,7 @@ __device__ __forceinline__ void count_done(unsigned* p) {
 // The completion count (and its complete value) that phase `type` of layer
 // l reads its input after; nullptr: the embedding, which every role of
 // every CTA waits for before anything else.
-__device__ __forceinline__ const unsigned* dep_of(const StepArgs& a, int type, int l, unsigned& target) {
+__device__ const unsigned* dep_of(const StepArgs& a, int type, int l, unsigned& target) {
     const unsigned nd = (unsigned)(a.d / BM);
     switch (type) {
         case PH_QKV:
@@ -899,30 +913,22 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                 if (wc.valid && wn - xn < C::STAGES) {
                     const int slot = wn % C::STAGES;
                     if (mbar_test(sm.empty + 8 * slot, ((wn / C::STAGES) & 1) ^ 1)) {
-                        const int mb = wc.i / wc.kbt, kb = wc.i - mb * wc.kbt;
                         mbar_expect_tx(sm.full + 8 * slot, C::STAGE_BYTES);
-                        tma_load_2d_hint(sm.sA + slot * C::A_BYTES, a.maps + wc.map_a, sm.full + 8 * slot, kb * BK,
-                                         mb * BM, wpol);
+                        tma_load_2d_hint(sm.sA + slot * C::A_BYTES, a.maps + wc.map_a, sm.full + 8 * slot, wc.kb * BK,
+                                         wc.mb * BM, wpol);
                         ++wn;
                         cursor_next(a, P, wc);
                         prog = true;
                     }
                 }
                 if (xn < wn) {
-                    if (ready < xc.p) {
-                        int l;
-                        const int type = phase_type(a, xc.p, l);
-                        unsigned tgt = 0;
-                        const unsigned* dp = dep_of(a, type, l, tgt);
-                        if (!dp || (int)(ld_acquire_u32(dp) - tgt) >= 0) {
-                            asm volatile("fence.proxy.async.global;" ::: "memory");
-                            ready = xc.p;
-                        }
+                    if (ready < xc.p && (!xc.dep || (int)(ld_acquire_u32(xc.dep) - xc.tgt) >= 0)) {
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                        ready = xc.p;
                     }
                     if (ready >= xc.p) {
                         const int slot = xn % C::STAGES;
-                        tma_load_2d(sm.sB + slot * C::B_BYTES, a.maps + xc.map_b, sm.full + 8 * slot,
-                                    (xc.i % xc.kbt) * BK, 0);
+                        tma_load_2d(sm.sB + slot * C::B_BYTES, a.maps + xc.map_b, sm.full + 8 * slot, xc.kb * BK, 0);
                         ++xn;
                         cursor_next(a, P, xc);
                         prog = true;
@@ -946,7 +952,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
             // of stages to land.
             while (xn < wn) {
                 const int slot = xn % C::STAGES;
-                tma_load_2d(sm.sB + slot * C::B_BYTES, a.maps + xc.map_b, sm.full + 8 * slot, (xc.i % xc.kbt) * BK, 0);
+                tma_load_2d(sm.sB + slot * C::B_BYTES, a.maps + xc.map_b, sm.full + 8 * slot, xc.kb * BK, 0);
                 ++xn;
                 cursor_next(a, P, xc);
             }
