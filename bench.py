@@ -44,6 +44,8 @@ WORKLOADS = {
                        desc="llama-13b: 256 greedy decode steps, batch 32, 2048-token prompts prefilled untimed"),
     "65b-slice": dict(model="LLAMA_65B_SLICE", batch=8, seq=2048, decode=0,
                       desc="llama-65b widths, 16 layers: prefill 8 x 2048 (logits at every position)"),
+    "33b": dict(model="LLAMA_33B", batch=4, seq=2048, decode=128,
+                desc="llama-33b: prefill 4 x 2048 (logits at every position) + 128 greedy decode steps"),
     # small case of the 7B kernels (same shapes per launch) for ncu captures
     "7b-2layer": dict(model="LLAMA_7B", layers=2, batch=4, seq=2048, decode=128,
                       desc="llama-7b widths, 2 layers: prefill 4 x 2048 + 128 greedy decode steps"),

@@ -40,6 +40,8 @@ BLOCK_7B = ModelShape("llama-7b-block", 1, 4096, 32, 128, 11008, 32000)
 LLAMA_7B = ModelShape("llama-7b", 32, 4096, 32, 128, 11008, 32000)
 # 13B shape: 40 layers.  Decode-heavy: batch 32, 2048-token prompts, 256 steps.
 LLAMA_13B = ModelShape("llama-13b", 40, 5120, 40, 128, 13824, 32000)
+# 33B shape: 60 layers, d 6656 = 52 heads of 128, hidden 17920.
+LLAMA_33B = ModelShape("llama-33b", 60, 6656, 52, 128, 17920, 32000)
 # 65B widths, 16 of 80 layers.  Prefill 8 x 2048 (+ S in {512,1024,2048} x B in {1,8}).
 LLAMA_65B_SLICE = ModelShape("llama-65b-slice16", 16, 8192, 64, 128, 22016, 32000)
 
