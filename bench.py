@@ -260,6 +260,32 @@ def oracle_sample(shape, B, S, steps, prompt=64, layers=2):
                 seconds=round(t2 - t0, 3)), step_s
 
 
+# ----------------------------------------------------------------------------- replicas
+
+def max_over_ranks(x: float, world: int, device="cpu") -> float:
+    """The largest of every rank's value (device time of the same region);
+    every rank takes this collective step."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, tokens_per_step: int, steps: int, ms: float) -> float:
+    """Whole-job tokens/s: every replica processes tokens_per_step per step;
+    the slowest rank's time bounds the job."""
+    return world * tokens_per_step * steps / (ms * 1e-3)
+
+
+def replica_tokens(shape, rank: int, B: int, S: int):
+    """Prompt token ids of one replica: each rank its own seeded draw."""
+    import synth
+    return synth.tokens(synth.workloads.SEED + rank, B * S, shape.vocab).reshape(B, S)
+
+
 # ----------------------------------------------------------------------------- arms
 
 def run_reference(args, wl, shape):
@@ -302,7 +328,7 @@ def run_b200(args, wl, shape):
     B, S, steps = wl["batch"], wl["seq"], wl["decode"]
     max_seq = S + steps
     model = lb.Model(shape, max_batch=B, max_seq=max_seq, seed=synth.workloads.SEED)
-    tok_host = torch.from_numpy(synth.tokens(synth.workloads.SEED + rank, B * S, shape.vocab).reshape(B, S))
+    tok_host = torch.from_numpy(replica_tokens(shape, rank, B, S))
     tok_host = tok_host.pin_memory()
     tok_dev = tok_host.cuda()
     logits = torch.empty(B, S, shape.vocab, dtype=torch.float32, device="cuda") if wl["name"] != "13b-decode" else None
@@ -352,14 +378,10 @@ def run_b200(args, wl, shape):
         torch.cuda.synchronize()
     barrier()
     launches = lb.kernel_launches() - l0
-    ms = ev[0].elapsed_time(ev[1])
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev[0].elapsed_time(ev[1]), world, "cuda")
     clocks = clk.summary()
     tokens_step = (0 if decode_only else B * S) + B * steps
-    value = world * tokens_step * args.steps / (ms * 1e-3)
+    value = replica_throughput(world, tokens_step, args.steps, ms)
 
     # ------------------------------------------------ prefill / decode split
     split = {}
@@ -394,11 +416,7 @@ def run_b200(args, wl, shape):
         ee[1].record(st)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = ee[0].elapsed_time(ee[1])
-        if world > 1:
-            t = torch.tensor([e2e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(ee[0].elapsed_time(ee[1]), world, "cuda")
 
     # ------------------------------------------------ live per-region timing (roofline)
     peaks, peak_src = load_peaks()
@@ -443,7 +461,7 @@ def run_b200(args, wl, shape):
         if phases:
             line["decode_step_phases_us"] = phases
         if e2e_ms is not None:
-            line["e2e"] = dict(value=round(world * tokens_step * args.steps / (e2e_ms * 1e-3), 2), unit=UNIT,
+            line["e2e"] = dict(value=round(replica_throughput(world, tokens_step, args.steps, e2e_ms), 2), unit=UNIT,
                                h2d_bytes_per_step=B * S * 4, d2h_bytes_per_step=B * steps * 4)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"], _ = oracle_sample(shape, B, S, steps)

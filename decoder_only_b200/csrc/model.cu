@@ -112,7 +112,6 @@ namespace {
 
 constexpr uint32_t TID_EMBED = 1, TID_HEAD = 2;
 inline uint32_t layer_tid(int l, int m) { return 16u + 8u * (uint32_t)l + (uint32_t)m; }
-constexpr int MAX_DEC_SPLITS = 16;
 constexpr int MAX_COUNTERS = 4096;
 
 struct Layer {
