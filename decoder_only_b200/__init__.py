@@ -44,6 +44,8 @@ def _load():
         "llama_model_bytes": [P, P],
         "llama_init_weights": [P, ctypes.c_uint32, P, U64, P, P],
         "llama_prefill": [P, P, I, I, P, P],
+        "llama_prefill_ragged": [P, P, I, I, P, P, P],
+        "llama_positions": [P, P, I],
         "llama_prefill_trunk": [P, P, I, I, P, P],
         "llama_decode_step": [P, P, P, P, P],
         "llama_generate": [P, P, I, P, P],
@@ -154,15 +156,30 @@ class Model:
     def position(self) -> int:
         return lib.llama_position(self.h)
 
-    def prefill(self, tokens: torch.Tensor, logits: bool = True, out: torch.Tensor | None = None):
-        """tokens int32 [B, S] on the device -> logits fp32 [B, S, V] (or None)."""
+    def prefill(self, tokens: torch.Tensor, logits: bool = True, out: torch.Tensor | None = None,
+                lens=None):
+        """tokens int32 [B, S] on the device -> logits fp32 [B, S, V] (or None).
+        With ``lens`` (B ints) the batch is ragged: sequence b is its first
+        lens[b] tokens (llama_prefill_ragged)."""
         B, S = tokens.shape
         tokens = tokens.contiguous()
         if logits and out is None:
             out = torch.empty(B, S, self.cfg.vocab, dtype=torch.float32, device="cuda")
-        _check(lib.llama_prefill(self.h, _ptr(tokens), B, S, _ptr(out if logits else None), _stream()),
-               "llama_prefill")
+        if lens is None:
+            _check(lib.llama_prefill(self.h, _ptr(tokens), B, S, _ptr(out if logits else None), _stream()),
+                   "llama_prefill")
+        else:
+            h_lens = (ctypes.c_int32 * B)(*[int(x) for x in lens])
+            _check(lib.llama_prefill_ragged(self.h, _ptr(tokens), B, S, ctypes.cast(h_lens, ctypes.c_void_p),
+                                            _ptr(out if logits else None), _stream()), "llama_prefill_ragged")
         return out if logits else None
+
+    def positions(self):
+        """Each sequence's decode position (host ints)."""
+        buf = (ctypes.c_int32 * 64)()
+        n = lib.llama_positions(self.h, ctypes.cast(buf, ctypes.c_void_p), 64)
+        _check(min(n, 0), "llama_positions")
+        return [buf[i] for i in range(n)]
 
     def complete(self, tokens_host: torch.Tensor, n_steps: int, logits: torch.Tensor | None = None,
                  out_host: torch.Tensor | None = None) -> torch.Tensor:

@@ -68,12 +68,12 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) attn_decode_kernel(
 
     pdl_launch_dependents();
     pdl_wait();   // the newest K/V row and q come from the projection before this kernel
-    const int len = d_len_minus1 ? (*d_len_minus1 + 1) : len_static;
+    const int bh = blockIdx.y;
+    const int b = bh / H, h = bh - b * H;
+    const int len = d_len_minus1 ? (d_len_minus1[b] + 1) : len_static;   // per sequence
     const int used = (len + DEC_CHUNK - 1) / DEC_CHUNK;
     const int chunk = blockIdx.x;
     if (chunk >= used) return;                          // past the live length
-    const int bh = blockIdx.y;
-    const int b = bh / H, h = bh - b * H;
     const int k_begin = chunk * DEC_CHUNK;
     const int nkeys = min(len - k_begin, DEC_CHUNK);
     const size_t head_off = ((size_t)b * H + h) * (size_t)kv_stride * HD;

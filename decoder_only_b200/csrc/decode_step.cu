@@ -518,41 +518,72 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
     constexpr int KPG = ACH / 4;     // keys of a chunk per lane group
     constexpr int DPW = HD / 32;     // dims per lane in the final merge
     const int g = lane >> 3, r = lane & 7;
-    const int len = *a.d_pos + 1;
-    const int nch = (len + ACH - 1) / ACH;
-    const int pairs = a.B * a.H;
-    const long long Ctot = (long long)pairs * nch;
+    // Sequence j (lane j) holds len_j = pos_j + 1 keys in n_j chunks; the
+    // chunks of all pairs, pair-major (pair = j * H + h), form one range of
+    // H * sum_j n_j units whose sequence j starts at H * (n_0 + ... + n_{j-1}).
+    const int Bq = a.B;
+    const int my_len = lane < Bq ? a.d_pos[lane] + 1 : 0;
+    const int my_nch = (my_len + ACH - 1) / ACH;
+    int incl = my_nch;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    const int excl = incl - my_nch;
+    const long long Ctot = (long long)a.H * __shfl_sync(0xffffffffu, incl, Bq - 1);
     const int Wp = (int)min((long long)gridDim.x * NAW, Ctot);
     const int gw = blockIdx.x * NAW + aw;
     if (gw >= Wp) return true;
     const long long cs = Ctot * gw / Wp, ce = Ctot * (gw + 1) / Wp;
     auto owner = [&](long long i) { return (int)(((i + 1) * Wp - 1) / Ctot); };
-    const int PM = (Wp + pairs - 1) / pairs + 1;    // ranges that can touch one pair
+    // unit index -> (sequence b, head h, chunk kc) with b's length and chunk count
+    struct Pos {
+        int b, h, kc, len, nch;
+    };
+    auto locate = [&](long long c) {
+        Pos q;
+        q.b = __popc(__ballot_sync(0xffffffffu, lane < Bq && (long long)a.H * incl <= c));
+        q.len = __shfl_sync(0xffffffffu, my_len, q.b);
+        q.nch = __shfl_sync(0xffffffffu, my_nch, q.b);
+        const long long rem = c - (long long)a.H * __shfl_sync(0xffffffffu, excl, q.b);
+        q.h = (int)(rem / q.nch);
+        q.kc = (int)(rem - (long long)q.h * q.nch);
+        return q;
+    };
+    auto advance = [&](Pos& q) {
+        if (++q.kc < q.nch) return;
+        q.kc = 0;
+        if (++q.h < a.H) return;
+        q.h = 0;
+        ++q.b;
+        const int bb = min(q.b, 31);
+        q.len = __shfl_sync(0xffffffffu, my_len, bb);
+        q.nch = __shfl_sync(0xffffffffu, my_nch, bb);
+    };
     const uint32_t wbuf = smem_u32(sm.att) + aw * 2 * C::ATT_BUF;
     const uint32_t wbar = sm.abar + aw * 16;
     // the cache rows and queries of this step were stored by other CTAs
-    // (generic proxy) before the grid barrier; the bulk copies read them
-    // through the async proxy, and overwrite shared memory that generic
+    // (generic proxy) before their completion counts; the bulk copies read
+    // them through the async proxy, and overwrite shared memory that generic
     // stores wrote before
     if (lane == 0) asm volatile("fence.proxy.async.global;\n\tfence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
-    // issue cursor: chunk ic = (pair ip, chunk kc_i of the pair)
+    // issue cursor
     long long ic = cs;
-    int ip = (int)(cs / nch), ikc = (int)(cs - (long long)ip * nch);
+    Pos iq = locate(cs);
     auto issue = [&](int buf) {
         if (lane == 0)
-            attn_issue<BN, HD>(a, l, ip, ikc, ic == cs || ikc == 0, len, wbuf + buf * C::ATT_BUF, wbar + 8 * buf);
+            attn_issue<BN, HD>(a, l, iq.b * a.H + iq.h, iq.kc, ic == cs || iq.kc == 0, iq.len,
+                               wbuf + buf * C::ATT_BUF, wbar + 8 * buf);
         ++ic;
-        if (++ikc == nch) {
-            ikc = 0;
-            ++ip;
-        }
+        advance(iq);
     };
     issue(0);
     if (ic < ce) issue(1);
     const float scale = rsqrtf((float)HD);
     float m = -INFINITY, lsum = 0.f, acc[DPL], qv[DPL];
-    int p = (int)(cs / nch), kc = (int)(cs - (long long)p * nch);
+    Pos cq = locate(cs);
     for (long long c = cs; c < ce; ++c) {
         const int k = (int)(c - cs), buf = k & 1;
         const uint32_t bar = wbar + 8 * buf;
@@ -578,6 +609,7 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
         const uint8_t* bp = sm.att + (size_t)(aw * 2 + buf) * C::ATT_BUF;
         const bf16* sk = reinterpret_cast<const bf16*>(bp);
         const bf16* sv = sk + ACH * HD;
+        const int kc = cq.kc, nch = cq.nch, len = cq.len;
         if (c == cs || kc == 0) {    // a new pair: its query (in this buffer) and a fresh state
             const bf16* qp = reinterpret_cast<const bf16*>(bp + C::ATT_Q);
 #pragma unroll
@@ -658,12 +690,9 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
         __syncwarp();
         // the buffer is free: put the chunk two places ahead in flight
         if (ic < ce) issue(buf);
-        const int pr = p;
+        const int pb = cq.b, ph = cq.h, pr = pb * a.H + ph;
         const bool pair_done = (c + 1 == ce) || (kc + 1 == nch);
-        if (++kc == nch) {
-            kc = 0;
-            ++p;
-        }
+        advance(cq);
         if (!pair_done) continue;
         // merge the four lane groups (each covers every 4th key)
 #pragma unroll
@@ -681,10 +710,9 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
             }
             m = M;
         }
-        const int b = pr / a.H, h = pr - b * a.H;
-        const long long pc0 = (long long)pr * nch;
+        const long long pc0 = (long long)a.H * __shfl_sync(0xffffffffu, excl, pb) + (long long)ph * nch;
         const int first = owner(pc0), nparts = owner(pc0 + nch - 1) - first + 1;
-        bf16* dst = a.attn + (size_t)b * a.d + (size_t)h * HD;
+        bf16* dst = a.attn + (size_t)pb * a.d + (size_t)ph * HD;
         if (nparts == 1) {    // the whole pair in this range
             const float inv = 1.f / lsum;
             if (g == 0) {
@@ -702,7 +730,7 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
             if (lane == 0) count_done(done_ctr(a, l, DK_ATTN));
             continue;
         }
-        float* wp = a.attn_work + ((size_t)pr * PM + (gw - first)) * (HD + 2);
+        float* wp = a.attn_work + ((size_t)gw + pr) * (HD + 2);
         if (g == 0) {
 #pragma unroll
             for (int u = 0; u < NV; ++u)
@@ -726,7 +754,7 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
         }
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) continue;
-        const float* wb = a.attn_work + (size_t)pr * PM * (HD + 2);
+        const float* wb = a.attn_work + ((size_t)first + pr) * (HD + 2);
         // lane j owns range j (and j + 32, ...): maxima and weighted sums by shuffles
         float Mall = -INFINITY;
         for (int j = lane; j < nparts; j += 32) Mall = fmaxf(Mall, __ldcg(wb + (size_t)j * (HD + 2)));
@@ -827,7 +855,7 @@ __device__ void phase_argmax(const StepArgs& a, int tid, const Smem<BN, HD>& sm,
                     wait_at_least(a.bar + SY_CHECKIN, gridDim.x, abort_flag, a.err);
                     a.bar[SY_CHECKIN] = 0;
                     a.bar[SY_EPOCH] = E;
-                    *a.d_pos += 1;
+                    for (int j = 0; j < a.B; ++j) a.d_pos[j] += 1;
                 }
             }
         }

@@ -31,7 +31,7 @@ struct EpiArgs {
     void* kc;             // EPI_QKV: this layer's K cache T [B][H][smax][hd]
     void* vc;             //          and V cache
     const float2* rope;   // [max_seq][hd/2] (cos, sin)
-    const int* d_pos;     // decode position (device); NULL in prefill
+    const int* d_pos;     // decode: position of each sequence (device, [B]); NULL in prefill
     int S;                // tokens per sequence in this call (prefill), 1 in decode
     int H, hd, d, smax;
 };
@@ -101,10 +101,10 @@ __device__ __forceinline__ void epi_qkv32(const EpiArgs& a, int m, int n0, const
     const int head = c / a.hd;
     const int i0 = c - head * a.hd;      // multiple of 32 within the head
     int b, s, pos;
-    if (a.d_pos) {                       // decode: one token per sequence at the current position
+    if (a.d_pos) {                       // decode: one token per sequence at its own position
         b = m;
         s = 0;
-        pos = *a.d_pos;
+        pos = a.d_pos[m];
     } else {
         b = m / a.S;
         s = m - b * a.S;

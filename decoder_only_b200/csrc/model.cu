@@ -171,7 +171,8 @@ struct llama_model {
     int* d_pos;              // decode position
     int* d_err;              // sticky device error word
     int B;                   // batch of the last prefill (0: none)
-    int cur_len;             // host mirror of *d_pos
+    int cur_len;             // largest position over the sequences (host)
+    std::vector<int> pos_h;  // host mirror of d_pos: each sequence's position (ragged batches)
     int splits_qkv, splits_o, splits_gu, splits_d, splits_head;
     cudaStream_t cap_stream;
     cudaGraphExec_t graph;
@@ -277,6 +278,7 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     int32_t* gen_out = (int32_t*)take(nmax * 4);
     float* trunk_last = (float*)take((size_t)c->max_batch * d * 4);
     int* small = (int*)take(256);
+    int* d_posv = (int*)take((size_t)c->max_batch * 4);
     if (m) {
         m->g_final = g_final;
         m->head = head;
@@ -309,7 +311,7 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
         m->tok_in = tok_in;
         m->gen_out = gen_out;
         m->trunk_last = trunk_last;
-        m->d_pos = small;
+        m->d_pos = d_posv;
         m->d_err = small + 1;
     }
     return off;
@@ -322,15 +324,22 @@ inline void* vcache(llama_model* m, int l) {
     return (uint8_t*)m->kv + (size_t)(2 * l + 1) * m->kv_layer_elems * m->esz;
 }
 
-__global__ void pos_set_kernel(int* pos, int v) {
+__global__ void pos_set_kernel(int* pos, int v, int n) {
     pdl_launch_dependents();
     pdl_wait();
-    *pos = v;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) pos[i] = v;
 }
-__global__ void pos_advance_kernel(int* pos) {
+__global__ void pos_advance_kernel(int* pos, int n) {
     pdl_launch_dependents();
     pdl_wait();
-    *pos += 1;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) pos[i] += 1;
+}
+// Logits row of each sequence's last prompt token (position pos[b] - 1) into dst [B, V]
+__global__ void last_rows_kernel(const float* logits, const int* pos, int S, int V, float* dst) {
+    const int b = blockIdx.y;
+    const float* src = logits + ((size_t)b * S + (pos[b] - 1)) * V;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < V; i += gridDim.x * blockDim.x)
+        dst[(size_t)b * V + i] = src[i];
 }
 
 EpiArgs base_args(llama_model* m, int M, int N) {
@@ -415,7 +424,9 @@ int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
         qa.d_pos = decode ? m->d_pos : nullptr;
         if ((rc = project(m, "qkv", EPI_QKV, m->xn, ly.wqkv, n, 3 * d, d, m->splits_qkv, qa, decode, st))) return rc;
         if (decode) {
-            const double len = (double)m->cur_len + 1;   // keys read this step
+            double len = 0;   // keys read this step, averaged over the sequences
+            for (int b = 0; b < B; ++b) len += m->pos_h[b] + 1;
+            len /= B;
             prof::Scope ps(st, "decode_attention", (2.0 * len + 2.0) * B * d * m->esz, 4.0 * B * d * len);
             if ((rc = launch_attention_decode(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, 0,
                                               m->d_pos, c.head_dim, c.max_seq, m->attn_work, m->attn_cnt, m->d_err,
@@ -540,8 +551,10 @@ int decode_body(llama_model* m, cudaStream_t st) {
         // weights + KV cache read + activations, once per step
         const double d = c.d_model, h = c.ffn_hidden, L = c.n_layers, V = c.vocab;
         const double wbytes = 2.0 * (L * (4 * d * d + 3 * d * h) + d * V);
-        const double kvbytes = 2.0 * 2.0 * L * m->B * (m->cur_len + 1) * d;
-        const double flops = 2.0 * m->B * (L * (4 * d * d + 3 * d * h) + d * V) + 4.0 * L * m->B * (m->cur_len + 1) * d;
+        double keys = 0;   // keys read this step, over the sequences
+        for (int b = 0; b < m->B; ++b) keys += m->pos_h[b] + 1;
+        const double kvbytes = 2.0 * 2.0 * L * keys * d;
+        const double flops = 2.0 * m->B * (L * (4 * d * d + 3 * d * h) + d * V) + 4.0 * L * keys * d;
         prof::Scope ps(st, "decode_step", wbytes + kvbytes, flops);
         StepArgs sa = step_args(m);
         if (prof::on) sa.timeline = m->step_timeline;
@@ -557,7 +570,7 @@ int decode_body(llama_model* m, cudaStream_t st) {
     prof::Scope ps(st, "decode_argmax", (double)m->B * c.vocab * 4, 0.0);
     if ((rc = launch_argmax_split(m->logits_dec, m->B, c.vocab, c.vocab, m->tok_cur, m->amax_part, m->amax_cnt, st)))
         return rc;
-    launch_pdl(pos_advance_kernel, dim3(1), dim3(1), 0, st, m->d_pos);
+    launch_pdl(pos_advance_kernel, dim3(1), dim3(32), 0, st, m->d_pos, m->B);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }
@@ -711,7 +724,8 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
         cudaMemsetAsync(m->amax_cnt, 0, (size_t)(cfg->max_batch + 1) * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->step_bar, 0, decode_step_sync_words(cfg->n_layers) * 4, st) != cudaSuccess ||
         cudaMemsetAsync(m->attn_cnt, 0, (size_t)cfg->max_batch * cfg->n_heads * 4, st) != cudaSuccess ||
-        cudaMemsetAsync(m->d_pos, 0, 256, st) != cudaSuccess) {
+        cudaMemsetAsync(m->d_pos, 0, (size_t)cfg->max_batch * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(m->d_err - 1, 0, 256, st) != cudaSuccess) {
         llama_free(m);
         return LLAMA_ERR_CUDA;
     }
@@ -730,32 +744,64 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
     return LLAMA_OK;
 }
 
-int llama_prefill(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S, float* d_logits, void* stream) {
+// Prefill of B sequences given as a [B, S] token block; with h_lens
+// sequence b holds only its first h_lens[b] tokens (the rest are padding
+// with valid ids, whose rows are computed and ignored: causality keeps
+// them out of every valid row) and continues at position h_lens[b].
+static int prefill_impl(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S, const int32_t* h_lens,
+                        float* d_logits, cudaStream_t st) {
     if (!m || !d_tokens || B <= 0 || S <= 0 || B > m->cfg.max_batch || S > m->cfg.max_seq)
         return LLAMA_ERR_INVALID_ARG;
-    cudaStream_t st = (cudaStream_t)stream;
+    if (h_lens)
+        for (int b = 0; b < B; ++b)
+            if (h_lens[b] < 1 || h_lens[b] > S) return LLAMA_ERR_INVALID_ARG;
     const int n = B * S;
+    const int V = m->cfg.vocab;
     int rc;
     {
         prof::Scope ps(st, "prefill_embed", (double)n * m->cfg.d_model * (4 + m->esz), 0.0);
-        rc = launch_embed(m->cfg.dtype, d_tokens, m->embed, m->trunk, n, m->cfg.d_model, m->cfg.vocab, m->d_err, st);
+        rc = launch_embed(m->cfg.dtype, d_tokens, m->embed, m->trunk, n, m->cfg.d_model, V, m->d_err, st);
     }
     if (rc) return rc;
     if ((rc = run_blocks(m, B, S, false, st))) return rc;
+    // positions: where each sequence continues
+    if (h_lens) {
+        LLAMA_CUDA_TRY(cudaMemcpyAsync(m->d_pos, h_lens, (size_t)B * 4, cudaMemcpyHostToDevice, st));
+    } else {
+        launch_pdl(pos_set_kernel, dim3(1), dim3(32), 0, st, m->d_pos, (int)S, (int)B);
+        LLAMA_LAUNCH_CHECK();
+    }
     if (d_logits) {
         if ((rc = run_head(m, m->trunk, n, d_logits, false, st))) return rc;
-        // greedy choice at each sequence's last position: the input of the
+        // greedy choice at each sequence's last prompt token: the input of the
         // first decode step when llama_generate is given no tokens
-        prof::Scope ps(st, "prefill_argmax", (double)B * m->cfg.vocab * 4, 0.0);
-        if ((rc = launch_argmax_split(d_logits + (size_t)(S - 1) * m->cfg.vocab, B, m->cfg.vocab,
-                                      (int64_t)S * m->cfg.vocab, m->tok_cur, m->amax_part, m->amax_cnt, st)))
-            return rc;
+        prof::Scope ps(st, "prefill_argmax", (double)B * V * 4, 0.0);
+        if (h_lens) {
+            last_rows_kernel<<<dim3((V + 1023) / 1024, B), 256, 0, st>>>(d_logits, m->d_pos, S, V, m->logits_dec);
+            LLAMA_LAUNCH_CHECK();
+            rc = launch_argmax_split(m->logits_dec, B, V, V, m->tok_cur, m->amax_part, m->amax_cnt, st);
+        } else {
+            rc = launch_argmax_split(d_logits + (size_t)(S - 1) * V, B, V, (int64_t)S * V, m->tok_cur, m->amax_part,
+                                     m->amax_cnt, st);
+        }
+        if (rc) return rc;
     }
-    launch_pdl(pos_set_kernel, dim3(1), dim3(1), 0, st, m->d_pos, (int)S);
-    LLAMA_LAUNCH_CHECK();
     m->B = B;
-    m->cur_len = S;
+    m->pos_h.assign(B, S);
+    if (h_lens) m->pos_h.assign(h_lens, h_lens + B);
+    m->cur_len = 0;
+    for (int b = 0; b < B; ++b) m->cur_len = std::max(m->cur_len, m->pos_h[b]);
     return LLAMA_OK;
+}
+
+int llama_prefill(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S, float* d_logits, void* stream) {
+    return prefill_impl(m, d_tokens, B, S, nullptr, d_logits, (cudaStream_t)stream);
+}
+
+int llama_prefill_ragged(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S, const int32_t* h_lens,
+                         float* d_logits, void* stream) {
+    if (!h_lens) return LLAMA_ERR_INVALID_ARG;
+    return prefill_impl(m, d_tokens, B, S, h_lens, d_logits, (cudaStream_t)stream);
 }
 
 int llama_prefill_trunk(llama_model* m, const float* d_x, int32_t B, int32_t S, float* d_y, void* stream) {
@@ -767,10 +813,11 @@ int llama_prefill_trunk(llama_model* m, const float* d_x, int32_t B, int32_t S, 
     int rc = run_blocks(m, B, S, false, st);
     if (rc) return rc;
     if (d_y != m->trunk) LLAMA_CUDA_TRY(cudaMemcpyAsync(d_y, m->trunk, bytes, cudaMemcpyDeviceToDevice, st));
-    launch_pdl(pos_set_kernel, dim3(1), dim3(1), 0, st, m->d_pos, (int)S);
+    launch_pdl(pos_set_kernel, dim3(1), dim3(32), 0, st, m->d_pos, (int)S, (int)B);
     LLAMA_LAUNCH_CHECK();
     m->B = B;
     m->cur_len = S;
+    m->pos_h.assign(B, S);
     return LLAMA_OK;
 }
 
@@ -787,6 +834,7 @@ int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t* d_next, 
         LLAMA_CUDA_TRY(cudaMemcpyAsync(d_logits, m->logits_dec, (size_t)m->B * m->cfg.vocab * 4,
                                        cudaMemcpyDeviceToDevice, st));
     m->cur_len += 1;
+    for (int& p : m->pos_h) p += 1;
     return LLAMA_OK;
 }
 
@@ -803,18 +851,28 @@ int llama_generate(llama_model* m, const int32_t* d_first, int32_t n_steps, int3
         LLAMA_CUDA_TRY(cudaMemcpyAsync(d_out + (size_t)i * m->B, m->tok_cur, (size_t)m->B * 4,
                                        cudaMemcpyDeviceToDevice, st));
         m->cur_len += 1;
+        for (int& p : m->pos_h) p += 1;
     }
     return LLAMA_OK;
 }
 
 int llama_position(const llama_model* m) { return m ? m->cur_len : LLAMA_ERR_INVALID_ARG; }
 
+int llama_positions(const llama_model* m, int32_t* h_out, int32_t n) {
+    if (!m || !h_out || n < m->B) return LLAMA_ERR_INVALID_ARG;
+    for (int b = 0; b < m->B; ++b) h_out[b] = m->pos_h[b];
+    return m->B;
+}
+
 int llama_rewind(llama_model* m, int32_t position, void* stream) {
-    if (!m || position < 1 || position > m->cur_len) return LLAMA_ERR_INVALID_ARG;
+    if (!m || position < 1) return LLAMA_ERR_INVALID_ARG;
     if (m->B <= 0) return LLAMA_ERR_STATE;
-    launch_pdl(pos_set_kernel, dim3(1), dim3(1), 0, (cudaStream_t)stream, m->d_pos, (int)position);
+    for (int b = 0; b < m->B; ++b)
+        if (position > m->pos_h[b]) return LLAMA_ERR_INVALID_ARG;   // every sequence holds `position` keys
+    launch_pdl(pos_set_kernel, dim3(1), dim3(32), 0, (cudaStream_t)stream, m->d_pos, (int)position, m->B);
     LLAMA_LAUNCH_CHECK();
     m->cur_len = position;
+    m->pos_h.assign(m->B, position);
     return LLAMA_OK;
 }
 

@@ -106,6 +106,17 @@ LLAMA_API int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d
 LLAMA_API int llama_prefill(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S,
                   float* d_logits, void* stream);
 
+/* Ragged batch: the same [B, S] token block, but sequence b holds only its
+ * first h_lens[b] tokens (host int32 [B], 1 <= h_lens[b] <= S); the
+ * remaining tokens are padding and must be valid ids (their rows are
+ * computed and ignored: causal attention keeps them out of every valid
+ * row, and decoding overwrites their cache entries).  Sequence b continues
+ * at position h_lens[b]; with d_logits the greedy choice is taken at its
+ * row h_lens[b] - 1.  Rows of padding positions in d_logits are
+ * unspecified.  Copies h_lens to the device on `stream`. */
+LLAMA_API int llama_prefill_ragged(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S,
+                                   const int32_t* h_lens, float* d_logits, void* stream);
+
 /* The blocks alone, on a given fp32 trunk: d_x [B*S, d_model] in,
  * d_y [B*S, d_model] out (the trunk after the last block, before the final
  * norm).  Positions 0..S-1 per sequence.  d_x and d_y may alias. */
@@ -113,11 +124,11 @@ LLAMA_API int llama_prefill_trunk(llama_model* m, const float* d_x, int32_t B, i
                         float* d_y, void* stream);
 
 /* One greedy decoding step for the B sequences of the last prefill: token
- * d_tokens[b] (int32 [B]) sits at the current position p; its K and V are
- * appended at p; attention spans 0..p.  d_next (int32 [B], may be NULL):
- * argmax of the logits, lowest id on ties.  d_logits: fp32 [B, vocab] or
- * NULL.  Advances p by one.  LLAMA_ERR_STATE before a prefill or when
- * p == max_seq. */
+ * d_tokens[b] (int32 [B]) sits at its sequence's current position p_b; its
+ * K and V are appended at p_b; attention spans 0..p_b.  d_next (int32 [B],
+ * may be NULL): argmax of the logits, lowest id on ties.  d_logits: fp32
+ * [B, vocab] or NULL.  Advances every p_b by one.  LLAMA_ERR_STATE before a
+ * prefill or when the largest p_b == max_seq. */
 LLAMA_API int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t* d_next,
                       float* d_logits, void* stream);
 
@@ -130,12 +141,16 @@ LLAMA_API int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t
 LLAMA_API int llama_generate(llama_model* m, const int32_t* d_first, int32_t n_steps,
                    int32_t* d_out, void* stream);
 
-/* Current decode position (tokens held per sequence in the KV cache). */
+/* Current decode position: the largest over the sequences (tokens held
+ * per sequence in the KV cache; all equal unless the batch is ragged). */
 LLAMA_API int llama_position(const llama_model* m);
 
-/* Move the decode position back to `position` (1 <= position <= current):
- * cache entries below it are kept, later ones are overwritten by the next
- * steps.  Queued on `stream`. */
+/* Each sequence's position into h_out (host int32, n >= B); returns B. */
+LLAMA_API int llama_positions(const llama_model* m, int32_t* h_out, int32_t n);
+
+/* Move every sequence's position back to `position` (1 <= position <= the
+ * smallest current position): cache entries below it are kept, later ones
+ * are overwritten by the next steps.  Queued on `stream`. */
 LLAMA_API int llama_rewind(llama_model* m, int32_t position, void* stream);
 
 /* End to end from HOST buffers: copy h_tokens (int32 [B*S], host; pinned
