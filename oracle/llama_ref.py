@@ -26,6 +26,11 @@ Readings taken where the pages are silent (each also listed in the design doc):
   * RoPE acts per head (its d is the head dimension), on interleaved
     (even, odd) channel pairs, angle = position * base^(-2i/d_head).
   * Heads are contiguous blocks of d_head columns of Q, K, V.
+  * Grouped keys and values ([NAR] "GQA Was Not an Original LLaMA
+    Feature"; LLaMA itself has one K/V head per query head): with n_kv
+    key/value heads, K and V have n_kv heads of d_head columns and query
+    head h attends with key/value head floor(h / (H / n_kv)) -- contiguous
+    groups of H / n_kv query heads.  n_kv = H is the original model.
   * Attention scale 1/sqrt(d_head); the causal mask keeps key j <= query t.
   * Prefill returns logits for every position; decoding is greedy with the
     lowest token id winning ties.
@@ -172,16 +177,17 @@ def weight_shapes(shape, bias: bool = False) -> dict:
     shift (the page's bias=True count).
     """
     d, h, V, L = shape.d_model, shape.ffn_hidden, shape.vocab, shape.n_layers
+    kvd = _kv_heads(shape) * shape.head_dim
     out = {"embed": (V, d)}
     for l in range(L):
         out.update({
-            f"{l}.wq": (d, d), f"{l}.wk": (d, d), f"{l}.wv": (d, d), f"{l}.wo": (d, d),
+            f"{l}.wq": (d, d), f"{l}.wk": (d, kvd), f"{l}.wv": (d, kvd), f"{l}.wo": (d, d),
             f"{l}.wg": (d, h), f"{l}.wu": (d, h), f"{l}.wd": (h, d),
             f"{l}.g_attn": (d,), f"{l}.g_ffn": (d,),
         })
         if bias:
             out.update({
-                f"{l}.bq": (d,), f"{l}.bk": (d,), f"{l}.bv": (d,), f"{l}.bo": (d,),
+                f"{l}.bq": (d,), f"{l}.bk": (kvd,), f"{l}.bv": (kvd,), f"{l}.bo": (d,),
                 f"{l}.bg": (h,), f"{l}.bu": (h,), f"{l}.bd": (d,),
                 f"{l}.beta_attn": (d,), f"{l}.beta_ffn": (d,),
             })
@@ -194,6 +200,11 @@ def count_params(shape, bias: bool = False) -> int:
     return int(sum(int(np.prod(s)) for s in weight_shapes(shape, bias).values()))
 
 
+def _kv_heads(shape) -> int:
+    """Key/value heads: n_kv_heads when the shape sets it, else one per query head."""
+    return getattr(shape, "n_kv_heads", 0) or shape.n_heads
+
+
 def _draw(seed, tensor_id, rows, cols, dtype):
     w = synth.normal_stored(seed, tensor_id, rows * cols, synth.WEIGHT_STD, dtype)
     return w.reshape(rows, cols)
@@ -203,7 +214,8 @@ def layer_weights(shape, layer: int, seed: int = 0) -> dict:
     """Random-init weights of one block (fp64 arrays holding values rounded to
     the storage dtype), N(0, 0.02^2), RMSNorm gains 1."""
     d, h = shape.d_model, shape.ffn_hidden
-    dims = {"wq": (d, d), "wk": (d, d), "wv": (d, d), "wo": (d, d),
+    kvd = _kv_heads(shape) * shape.head_dim
+    dims = {"wq": (d, d), "wk": (d, kvd), "wv": (d, kvd), "wo": (d, d),
             "wg": (d, h), "wu": (d, h), "wd": (h, d)}
     W = {name: _draw(seed, synth.layer_tensor_id(layer, name), r, c, shape.dtype)
          for name, (r, c) in dims.items()}
@@ -240,16 +252,17 @@ def attn_sublayer(z, W, positions, shape, kv_out=None, storage=None):
     per head; heads concatenated; times Wo.  [PFD] "RoPE: rotate Q and K,
     leave V alone" (where rope is applied)."""
     st, st_kv = _storer(storage), _storer(storage, kv=True)
-    H = shape.n_heads
+    H, Hkv = shape.n_heads, _kv_heads(shape)
+    G = H // Hkv                                   # query heads per key/value head
     q = split_heads(z @ W["wq"], H)
-    k = split_heads(z @ W["wk"], H)
-    v = split_heads(z @ W["wv"], H)
+    k = split_heads(z @ W["wk"], Hkv)
+    v = split_heads(z @ W["wv"], Hkv)
     q = st(rope(q, positions, shape.rope_theta))
     k = st_kv(rope(k, positions, shape.rope_theta))
     v = st_kv(v)
     if kv_out is not None:
         kv_out.append((k, v))
-    o = np.stack([causal_attention(q[hh], k[hh], v[hh]) for hh in range(H)])
+    o = np.stack([causal_attention(q[hh], k[hh // G], v[hh // G]) for hh in range(H)])
     return st(merge_heads(o)) @ W["wo"]
 
 
@@ -282,7 +295,7 @@ def prefill(shape, tokens: np.ndarray, seed: int = 0, weights=None, return_cache
     output head, (n, 32000)).  No position signal is added at the bottom.
     ``weights``: optional callable layer -> dict (else drawn from ``synth``).
     With ``return_cache`` the per-layer (K after RoPE, V) of every sequence is
-    returned as cache[l] = (K, V), each (B, H, S, d_head).
+    returned as cache[l] = (K, V), each (B, n_kv, S, d_head).
     ``storage`` may be a tuple of storage modes: the forward pass then runs
     once per mode on the same weights (each layer drawn once) and a list of
     logits, one per mode, is returned.
@@ -335,6 +348,8 @@ def decode_step(shape, cache: list, tokens: np.ndarray, seed: int = 0, weights=N
     tokens = np.asarray(tokens)
     B = tokens.shape[0]
     H, dh = shape.n_heads, shape.head_dim
+    Hkv = _kv_heads(shape)
+    G = H // Hkv
     E = embed_table(shape, seed)
     get_w = weights if weights is not None else (lambda l: layer_weights(shape, l, seed))
     p = cache[0][0].shape[2]
@@ -345,19 +360,19 @@ def decode_step(shape, cache: list, tokens: np.ndarray, seed: int = 0, weights=N
         Kc, Vc = cache[l]
         z = rms_norm(x, W["g_attn"], shape.norm_eps)
         q = (z @ W["wq"]).reshape(B, H, dh)
-        k = (z @ W["wk"]).reshape(B, H, dh)
-        v = (z @ W["wv"]).reshape(B, H, dh)
+        k = (z @ W["wk"]).reshape(B, Hkv, dh)
+        v = (z @ W["wv"]).reshape(B, Hkv, dh)
         pos = np.array([p])
         q = rope(q.reshape(B * H, 1, dh), pos, shape.rope_theta).reshape(B, H, dh)
-        k = rope(k.reshape(B * H, 1, dh), pos, shape.rope_theta).reshape(B, H, dh)
+        k = rope(k.reshape(B * Hkv, 1, dh), pos, shape.rope_theta).reshape(B, Hkv, dh)
         Kc = np.concatenate([Kc, k[:, :, None, :]], axis=2)
         Vc = np.concatenate([Vc, v[:, :, None, :]], axis=2)
         o = np.empty((B, H, dh))
         for b in range(B):
             for hh in range(H):
-                s = Kc[b, hh] @ q[b, hh] / math.sqrt(dh)      # (p+1,)
+                s = Kc[b, hh // G] @ q[b, hh] / math.sqrt(dh)      # (p+1,)
                 w = np.exp(s - s.max())
-                o[b, hh] = (w / w.sum()) @ Vc[b, hh]
+                o[b, hh] = (w / w.sum()) @ Vc[b, hh // G]
         x = x + o.reshape(B, H * dh) @ W["wo"]
         z = rms_norm(x, W["g_ffn"], shape.norm_eps)
         x = x + (silu(z @ W["wg"]) * (z @ W["wu"])) @ W["wd"]

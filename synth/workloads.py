@@ -22,6 +22,11 @@ class ModelShape:
     dtype: str = "bf16"          # storage type of weights and GEMM operands: 'bf16' or 'f32'
     norm_eps: float = 1e-6
     rope_theta: float = 10000.0
+    n_kv_heads: int = 0          # key/value heads (GQA / MQA); 0: one per query head
+
+    @property
+    def kv_heads(self) -> int:
+        return self.n_kv_heads or self.n_heads
 
     def as_dict(self):
         return asdict(self)

@@ -311,3 +311,55 @@ def test_bf16_kv_cache_alone_moves_deep_logits_past_2e2():
     rms = np.sqrt(np.mean(exact ** 2))
     assert np.max(np.abs(kv_only - exact)) / rms > 2e-2
     assert np.sqrt(np.mean((kv_only - exact) ** 2)) / rms < 2e-2
+
+
+# ---------------------------------------------------------------- grouped keys and values
+
+def _gqa_shape(n_kv):
+    return ModelShape("gqa", 1, 64, 4, 16, 128, 50, dtype="f32", n_kv_heads=n_kv)
+
+
+@pytest.mark.parametrize("n_kv", [1, 2])
+def test_grouped_kv_equals_mha_with_the_group_columns_repeated(n_kv):
+    """[NAR] "GQA Was Not an Original LLaMA Feature": query heads share K/V
+    heads.  Reading: query head h uses K/V head floor(h / (H / n_kv)).  The
+    same forward pass written as plain multi-head attention, with each query
+    head's K/V columns copied from its group's, must give the same logits;
+    a wrong group map (h mod n_kv, or the groups of another head) does not."""
+    s = _gqa_shape(n_kv)
+    mha = s.with_(n_kv_heads=0)
+    W = oracle.layer_weights(s, 0)
+    G, hd = s.n_heads // n_kv, s.head_dim
+    Wm = dict(W)
+    for name in ("wk", "wv"):
+        Wm[name] = np.concatenate([W[name][:, (h // G) * hd:(h // G + 1) * hd] for h in range(s.n_heads)], axis=1)
+    tok = np.random.default_rng(21).integers(0, s.vocab, size=(2, 9))
+    a = oracle.prefill(s, tok, weights=lambda l: W)
+    b = oracle.prefill(mha, tok, weights=lambda l: Wm)
+    assert np.allclose(a, b, rtol=0, atol=1e-12)
+    # another grouping (h mod n_kv) is a different model unless it coincides
+    if n_kv == 2:
+        Wx = dict(W)
+        for name in ("wk", "wv"):
+            Wx[name] = np.concatenate([W[name][:, (h % n_kv) * hd:(h % n_kv + 1) * hd] for h in range(s.n_heads)],
+                                      axis=1)
+        assert not np.allclose(a, oracle.prefill(mha, tok, weights=lambda l: Wx), atol=1e-6)
+    # the weight shapes count the narrower K and V
+    assert oracle.count_params(s) == oracle.count_params(mha) - 2 * s.d_model * (s.n_heads - n_kv) * hd
+
+
+@pytest.mark.parametrize("n_kv", [1, 2, 4])
+def test_grouped_kv_cache_size_and_decode(n_kv):
+    """The cache holds 2 L S n_kv d_h values per sequence, the page's
+    M_KV = 2 L S n_kv d_h b with b bytes per value; decoding one token at a
+    time over it reproduces the prefill rows."""
+    s = _gqa_shape(n_kv)
+    tok = np.random.default_rng(22).integers(0, s.vocab, size=(3, 10))
+    lg, cache = oracle.prefill(s, tok, return_cache=True)
+    values = sum(k.size + v.size for k, v in cache)
+    assert values == 2 * s.n_layers * 10 * n_kv * s.head_dim * 3
+    lg7, c7 = oracle.prefill(s, tok[:, :7], return_cache=True)
+    for t in range(7, 10):
+        logits, nxt, c7 = oracle.decode_step(s, c7, tok[:, t])
+        assert np.allclose(logits, lg[:, t], atol=1e-12)
+    assert c7[0][0].shape == (3, n_kv, 10, s.head_dim)
