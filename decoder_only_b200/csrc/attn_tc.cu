@@ -63,7 +63,7 @@ template <int HD>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ out, int H, int S,
-                           float scale_log2, int* err) {
+                           int Hkv, float scale_log2, int* err) {
     using C = ACfg<HD>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -86,6 +86,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int qt = (int)(gridDim.x - 1 - blockIdx.x);     // longest (most key tiles) first
     const int h = blockIdx.y, b = blockIdx.z;
     const int head = b * H + h;
+    const int kv_head = b * Hkv + h / (H / Hkv);      // grouped keys and values
     const int q0 = qt * BQ;
     const int n_kv = qt + 1;                              // key tiles 0..qt (causal)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -133,10 +134,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 mbar_expect_tx(k_full + 8 * st, C::TILE);
                 for (int r = 0; r < C::NREG; ++r)
-                    tma_load_3d(sK + st * C::TILE + r * C::REG, &tmK, k_full + 8 * st, 64 * r, j * BKV, head);
+                    tma_load_3d(sK + st * C::TILE + r * C::REG, &tmK, k_full + 8 * st, 64 * r, j * BKV, kv_head);
                 mbar_expect_tx(v_full + 8 * st, C::TILE);
                 for (int r = 0; r < C::NREG; ++r)
-                    tma_load_3d(sV + st * C::TILE + r * C::REG, &tmV, v_full + 8 * st, 64 * r, j * BKV, head);
+                    tma_load_3d(sV + st * C::TILE + r * C::REG, &tmV, v_full + 8 * st, 64 * r, j * BKV, kv_head);
                 issued = j + 1;
             }
             if (!ok) {
@@ -370,28 +371,29 @@ int attention_tc_prepare() {
     return attn_attr<64>();
 }
 
-int launch_attention_prefill_tc(const void* q, const void* k, const void* v, void* o, int B, int H, int S, int hd,
-                                int kv_stride, int* err, cudaStream_t st) {
+int launch_attention_prefill_tc(const void* q, const void* k, const void* v, void* o, int B, int H, int Hkv, int S,
+                                int hd, int kv_stride, int* err, cudaStream_t st) {
     if (B <= 0 || S <= 0) return LLAMA_OK;
     if (hd != 64 && hd != 128) return LLAMA_ERR_INVALID_ARG;
+    if (Hkv <= 0 || H % Hkv != 0) return LLAMA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
          reinterpret_cast<uintptr_t>(o)) & 15u)
         return LLAMA_ERR_INVALID_ARG;
     CUtensorMap mq, mk, mv;
     int rc;
     if ((rc = make_head_map(&mq, q, hd, S, S, B * H))) return rc;
-    if ((rc = make_head_map(&mk, k, hd, S, kv_stride, B * H))) return rc;
-    if ((rc = make_head_map(&mv, v, hd, S, kv_stride, B * H))) return rc;
+    if ((rc = make_head_map(&mk, k, hd, S, kv_stride, B * Hkv))) return rc;
+    if ((rc = make_head_map(&mv, v, hd, S, kv_stride, B * Hkv))) return rc;
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
     dim3 grid((S + BQ - 1) / BQ, H, B);
     if (hd == 128) {
         if ((rc = attn_attr<128>())) return rc;
         launch_pdl(attn_prefill_tc_kernel<128>, grid, dim3(NTHREADS), ACfg<128>::SMEM, st, mq, mk, mv, (bf16*)o, H, S,
-                   scale_log2, err);
+                   Hkv, scale_log2, err);
     } else {
         if ((rc = attn_attr<64>())) return rc;
         launch_pdl(attn_prefill_tc_kernel<64>, grid, dim3(NTHREADS), ACfg<64>::SMEM, st, mq, mk, mv, (bf16*)o, H, S,
-                   scale_log2, err);
+                   Hkv, scale_log2, err);
     }
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;

@@ -52,7 +52,7 @@ template <> struct V16<float> {
 // in order and writes the output row.
 template <typename T, int HD>
 __global__ void __launch_bounds__(DEC_WARPS * 32) attn_decode_kernel(
-    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ o, int H,
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ o, int H, int Hkv,
     int len_static, const int* __restrict__ d_len_minus1, int kv_stride, float scale, float* __restrict__ work,
     int* __restrict__ counters, int n_chunks, int* __restrict__ err) {
     constexpr int VEC = V16<T>::N;
@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) attn_decode_kernel(
     if (chunk >= used) return;                          // past the live length
     const int k_begin = chunk * DEC_CHUNK;
     const int nkeys = min(len - k_begin, DEC_CHUNK);
-    const size_t head_off = ((size_t)b * H + h) * (size_t)kv_stride * HD;
+    const size_t head_off = ((size_t)b * Hkv + h / (H / Hkv)) * (size_t)kv_stride * HD;   // its key/value head
     const uint32_t bar_a = smem_addr(&bar);
 
     if (threadIdx.x == 0) {
@@ -254,7 +254,7 @@ static int dec_attr() {
 }
 
 template <typename T, int HD>
-static int launch_dec_t(const void* q, const void* k, const void* v, void* o, int B, int H, int len,
+static int launch_dec_t(const void* q, const void* k, const void* v, void* o, int B, int H, int Hkv, int len,
                         const int* d_len_minus1, int kv_stride, float* work, int* counters, int* err,
                         cudaStream_t st) {
     // With a device-side length the grid covers every chunk the cache can
@@ -265,7 +265,7 @@ static int launch_dec_t(const void* q, const void* k, const void* v, void* o, in
     int rc = dec_attr<T, HD>();
     if (rc) return rc;
     launch_pdl(attn_decode_kernel<T, HD>, dim3(n_chunks, B * H), dim3(DEC_WARPS * 32), smem, st, (const T*)q,
-               (const T*)k, (const T*)v, (T*)o, H, len, d_len_minus1, kv_stride, 1.0f / sqrtf((float)HD), work,
+               (const T*)k, (const T*)v, (T*)o, H, Hkv, len, d_len_minus1, kv_stride, 1.0f / sqrtf((float)HD), work,
                counters, n_chunks, err);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
@@ -289,11 +289,12 @@ int attention_decode_clear(float* work, int B, int H, int len, int hd, cudaStrea
 }
 
 int launch_attention_decode(int dtype, const void* q, const void* k, const void* v, void* o, int B, int H,
-                            int len, const int* d_len_minus1, int hd, int kv_stride, float* work, int* counters,
-                            int* err, cudaStream_t st) {
+                            int Hkv, int len, const int* d_len_minus1, int hd, int kv_stride, float* work,
+                            int* counters, int* err, cudaStream_t st) {
     if (B <= 0) return LLAMA_OK;
+    if (Hkv <= 0 || H % Hkv != 0) return LLAMA_ERR_INVALID_ARG;
 #define DEC_CASE(TT, HH) \
-    return launch_dec_t<TT, HH>(q, k, v, o, B, H, len, d_len_minus1, kv_stride, work, counters, err, st)
+    return launch_dec_t<TT, HH>(q, k, v, o, B, H, Hkv, len, d_len_minus1, kv_stride, work, counters, err, st)
     if (dtype == LLAMA_BF16) {
         if (hd == 128) DEC_CASE(bf16, 128);
         if (hd == 64) DEC_CASE(bf16, 64);
@@ -372,6 +373,6 @@ extern "C" LLAMA_API int llama_op_attention_decode_noalloc(int32_t dtype, const 
     int* err = nullptr;
     if ((rc = op_error_word(&err))) return rc;
     if ((rc = attention_decode_clear(work, B, H, len, head_dim, (cudaStream_t)stream))) return rc;
-    return launch_attention_decode(dtype, d_q, d_k, d_v, d_o, B, H, len, nullptr, head_dim, kv_stride, work,
+    return launch_attention_decode(dtype, d_q, d_k, d_v, d_o, B, H, H, len, nullptr, head_dim, kv_stride, work,
                                    attention_decode_counters(work, B, H, len, head_dim), err, (cudaStream_t)stream);
 }

@@ -119,7 +119,7 @@ struct GemmPh {
 __device__ __forceinline__ bool gemm_of(const StepArgs& a, int type, int l, GemmPh& g) {
     const int L = a.L;
     switch (type) {
-        case PH_QKV: g = GemmPh{4 * l + 0, 4 * L + 1, 3 * a.d, a.d, EPI_QKV, 0}; return true;
+        case PH_QKV: g = GemmPh{4 * l + 0, 4 * L + 1, a.d + 2 * a.Hkv * a.hd, a.d, EPI_QKV, 0}; return true;
         case PH_O: g = GemmPh{4 * l + 1, 4 * L + 2, a.d, a.d, EPI_RESID, 1}; return true;
         case PH_GU: g = GemmPh{4 * l + 2, 4 * L + 4, 2 * a.h, a.d, EPI_SWIGLU, 2}; return true;
         case PH_DOWN: g = GemmPh{4 * l + 3, 4 * L + 3, a.d, a.h, EPI_RESID, 3}; return true;
@@ -281,7 +281,7 @@ __device__ const unsigned* dep_of(const StepArgs& a, int type, int l, unsigned& 
         case PH_QKV:
             target = nd;
             return l == 0 ? nullptr : done_ctr(a, l - 1, DK_DOWN);
-        case PH_ATTN: target = (unsigned)(3 * a.d / BM); return done_ctr(a, l, DK_QKV);
+        case PH_ATTN: target = (unsigned)((a.d + 2 * a.Hkv * a.hd) / BM); return done_ctr(a, l, DK_QKV);
         case PH_O: target = (unsigned)(a.B * a.H); return done_ctr(a, l, DK_ATTN);
         case PH_GU: target = nd; return done_ctr(a, l, DK_O);
         case PH_DOWN: target = (unsigned)(a.h / BM); return done_ctr(a, l, DK_GU);
@@ -480,15 +480,17 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
 // range leaves its (max, sum, output) in the workspace and the last range to
 // arrive merges them in range order.
 template <int BN, int HD>
-__device__ __forceinline__ void attn_issue(const StepArgs& a, int l, int pr, int kc, bool with_q, int len,
+__device__ __forceinline__ void attn_issue(const StepArgs& a, int l, int b, int h, int kc, bool with_q, int len,
                                            uint32_t dst, uint32_t bar) {
     const int k0 = kc * ACH;
     const int nkeys = min(len - k0, ACH);
     const bf16* kc_ = a.kv + (size_t)(2 * l) * a.kv_layer;
     const bf16* vc = kc_ + a.kv_layer;
-    const size_t off = ((size_t)pr * a.smax + k0) * HD;     // pair pr = b * H + h
+    const int pr = b * a.H + h;                                        // query head h of sequence b ...
+    const size_t kvr = (size_t)b * a.Hkv + h / (a.H / a.Hkv);         // ... reads key/value head h / group
+    const size_t off = (kvr * a.smax + k0) * HD;
     const uint32_t bytes = (uint32_t)(nkeys * HD * 2);
-    // cache rows are read once per step: first out of L2
+    // cache rows are read once per step (per query head of a group): first out of L2
     const uint64_t pol = l2_evict_first();
     mbar_expect_tx(bar, 2 * bytes + (with_q ? HD * 2 : 0));
     asm volatile(
@@ -574,8 +576,8 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
     Pos iq = locate(cs);
     auto issue = [&](int buf) {
         if (lane == 0)
-            attn_issue<BN, HD>(a, l, iq.b * a.H + iq.h, iq.kc, ic == cs || iq.kc == 0, iq.len,
-                               wbuf + buf * C::ATT_BUF, wbar + 8 * buf);
+            attn_issue<BN, HD>(a, l, iq.b, iq.h, iq.kc, ic == cs || iq.kc == 0, iq.len, wbuf + buf * C::ATT_BUF,
+                               wbar + 8 * buf);
         ++ic;
         advance(iq);
     };
@@ -1124,6 +1126,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                 if (type == PH_QKV || type == PH_HEAD) load_inv(a, a.ssq, sm.sinv, tid);
                 else if (type == PH_GU) load_inv(a, a.ssq + SSQ_BLOCKS * 32, sm.sinv, tid);
                 EpiArgs ep;
+                memset(&ep, 0, sizeof(ep));
                 ep.M = a.B;
                 ep.N = w.g.rowsA;
                 ep.out = (type == PH_HEAD) ? a.logits : a.trunk;
@@ -1142,6 +1145,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                 ep.hd = a.hd;
                 ep.d = a.d;
                 ep.smax = a.smax;
+                ep.Hkv = a.Hkv;
                 for (int i = w.s; i < w.e;) {
                     const int mb = i / w.kbt;
                     const bool ok = mbar_wait(sm.tfull + 8 * acc, acc_ph, abort_flag, a.err);
@@ -1239,8 +1243,9 @@ int decode_step_ctas() { return std::min(tc_num_sms(), STEP_MAX_CTAS); }
 // Partial-sum and counter regions of the five projection kinds (qkv, o,
 // gate/up, down, head) for `ctas` CTAs and batch B; returns the floats of
 // all partial regions.
-long long decode_step_layout(int ctas, int d, int h, int V, int B, long long part_off[5], int cnt_off[5]) {
-    const int rows[5] = {3 * d, d, 2 * h, d, V};
+long long decode_step_layout(int ctas, int qkv_rows, int d, int h, int V, int B, long long part_off[5],
+                             int cnt_off[5]) {
+    const int rows[5] = {qkv_rows, d, 2 * h, d, V};
     const long long Mp = (B + 3) & ~3;
     long long off = 0;
     int coff = 0;
@@ -1280,11 +1285,11 @@ int launch_decode_step(const StepArgs& a, cudaStream_t st) {
 // Tensor-map table for the decode step: 4 per layer (W_qkv, W_o, W_gu, W_d),
 // the head, then the activation buffers xg, attn, act, xg2 with `B` rows.
 int decode_step_maps(CUtensorMap* host_maps, const void* const* w, int L, const void* head, const void* xg,
-                     const void* attn, const void* act, const void* xg2, int B, int d, int h, int V) {
+                     const void* attn, const void* act, const void* xg2, int B, int qkv_rows, int d, int h, int V) {
     int rc;
     const int bn = B <= 16 ? 16 : 32;
     for (int l = 0; l < L; ++l) {
-        if ((rc = tc_make_map_2d(&host_maps[4 * l + 0], w[4 * l + 0], 3 * d, d, BM))) return rc;
+        if ((rc = tc_make_map_2d(&host_maps[4 * l + 0], w[4 * l + 0], qkv_rows, d, BM))) return rc;
         if ((rc = tc_make_map_2d(&host_maps[4 * l + 1], w[4 * l + 1], d, d, BM))) return rc;
         if ((rc = tc_make_map_2d(&host_maps[4 * l + 2], w[4 * l + 2], 2 * h, d, BM))) return rc;
         if ((rc = tc_make_map_2d(&host_maps[4 * l + 3], w[4 * l + 3], d, h, BM))) return rc;

@@ -34,6 +34,7 @@ struct EpiArgs {
     const int* d_pos;     // decode: position of each sequence (device, [B]); NULL in prefill
     int S;                // tokens per sequence in this call (prefill), 1 in decode
     int H, hd, d, smax;
+    int Hkv;              // key/value heads: columns [d, d + Hkv hd) are K, then V
 };
 
 __device__ __forceinline__ float silu_f(float u) { return u / (1.0f + __expf(-u)); }
@@ -94,11 +95,13 @@ __device__ __forceinline__ void epi_swiglu32(const EpiArgs& a, int m, int j0, co
 }
 
 // Q/K/V split + RoPE + KV-cache append for columns n0..n0+31 of token row m.
+// Columns: Q [0, d), K [d, d + kvd), V [d + kvd, d + 2 kvd), kvd = Hkv * hd.
 template <typename T>
 __device__ __forceinline__ void epi_qkv32(const EpiArgs& a, int m, int n0, const float (&v)[32]) {
-    const int which = n0 / a.d;          // 0 = Q, 1 = K, 2 = V
-    const int c = n0 - which * a.d;
-    const int head = c / a.hd;
+    const int kvd = a.Hkv * a.hd;
+    const int which = n0 < a.d ? 0 : (n0 < a.d + kvd ? 1 : 2);   // 0 = Q, 1 = K, 2 = V
+    const int c = which == 0 ? n0 : n0 - a.d - (which - 1) * kvd;
+    const int head = c / a.hd;           // query head (Q) or key/value head (K, V)
     const int i0 = c - head * a.hd;      // multiple of 32 within the head
     int b, s, pos;
     if (a.d_pos) {                       // decode: one token per sequence at its own position
@@ -129,7 +132,7 @@ __device__ __forceinline__ void epi_qkv32(const EpiArgs& a, int m, int n0, const
         dst = reinterpret_cast<T*>(a.q) + (((size_t)b * a.H + head) * a.S + s) * a.hd + i0;
     } else {
         T* base = reinterpret_cast<T*>(which == 1 ? a.kc : a.vc);
-        dst = base + (((size_t)b * a.H + head) * a.smax + pos) * a.hd + i0;
+        dst = base + (((size_t)b * a.Hkv + head) * a.smax + pos) * a.hd + i0;
     }
     store32<T>(dst, r);
 }

@@ -32,20 +32,20 @@ int launch_gemm_simt(int dtype, const void* A, const void* W, float* C, int M, i
                      cudaStream_t st);
 int launch_epilogue_from_f32(int dtype, int mode, const float* C, int ldc, const EpiArgs& a, cudaStream_t st);
 int launch_attention_prefill_simt(int dtype, const void* q, const void* k, const void* v, void* o, int B,
-                                  int H, int S, int hd, int kv_stride, cudaStream_t st);
+                                  int H, int Hkv, int S, int hd, int kv_stride, cudaStream_t st);
 int attention_prepare();  // sets kernel attributes; call before any stream capture
 
 // attn_tc.cu  (bf16 tcgen05 causal flash attention, head_dim 64 or 128)
-int launch_attention_prefill_tc(const void* q, const void* k, const void* v, void* o, int B, int H, int S, int hd,
-                                int kv_stride, int* err, cudaStream_t st);
+int launch_attention_prefill_tc(const void* q, const void* k, const void* v, void* o, int B, int H, int Hkv, int S,
+                                int hd, int kv_stride, int* err, cudaStream_t st);
 int attention_tc_prepare();
 
 // decode.cu
 uint64_t attention_decode_work_bytes(int B, int H, int max_len, int hd);
 // counters: int [B*H], zero before the launch (each launch leaves them zero)
 int launch_attention_decode(int dtype, const void* q, const void* k, const void* v, void* o, int B, int H,
-                            int len, const int* d_len_minus1, int hd, int kv_stride, float* work, int* counters,
-                            int* err, cudaStream_t st);
+                            int Hkv, int len, const int* d_len_minus1, int hd, int kv_stride, float* work,
+                            int* counters, int* err, cudaStream_t st);
 int* attention_decode_counters(float* work, int B, int H, int max_len, int hd);
 int attention_decode_clear(float* work, int B, int H, int len, int hd, cudaStream_t st);
 int attention_decode_prepare();
@@ -101,16 +101,18 @@ struct StepArgs {
     unsigned long long* timeline; // optional: per CTA and phase, start / end %globaltimer stamps
     const float2* rope;
     int L, d, h, V, H, hd, B, smax;
+    int Hkv;                      // key/value heads (query head h uses h / (H / Hkv))
     float eps;
 };
 int decode_step_prepare();
 int launch_decode_step(const StepArgs& a, cudaStream_t st);
 int decode_step_maps(CUtensorMap* host_maps, const void* const* w, int L, const void* head, const void* xg,
-                     const void* attn, const void* act, const void* xg2, int B, int d, int h, int V);
+                     const void* attn, const void* act, const void* xg2, int B, int qkv_rows, int d, int h, int V);
 // Grid of the fused decode step, and the partial / counter regions for batch B
 int decode_step_ctas();
 inline size_t decode_step_sync_words(int L) { return 128 + 256 * (size_t)(L + 1); }
-long long decode_step_layout(int ctas, int d, int h, int V, int B, long long part_off[5], int cnt_off[5]);
+long long decode_step_layout(int ctas, int qkv_rows, int d, int h, int V, int B, long long part_off[5],
+                             int cnt_off[5]);
 // 2-D K-major bf16 tensor map, box (64, box_rows), 128-byte swizzle, zero fill
 int tc_make_map_2d(CUtensorMap* map, const void* ptr, int rows, int K, int box_rows);
 int tc_num_sms();

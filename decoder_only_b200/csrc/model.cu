@@ -184,10 +184,14 @@ namespace {
 
 int hidden_of(const llama_config* c);
 
+// Key/value heads (grouped keys and values); 0 in the config means one per query head
+inline int kv_heads(const llama_config* c) { return c->n_kv_heads > 0 ? c->n_kv_heads : c->n_heads; }
+
 int validate(const llama_config* c) {
     if (!c) return LLAMA_ERR_INVALID_ARG;
     if (c->n_layers < 0 || c->d_model <= 0 || c->n_heads <= 0 || c->vocab <= 0) return LLAMA_ERR_INVALID_ARG;
     if (c->head_dim * c->n_heads != c->d_model) return LLAMA_ERR_INVALID_ARG;
+    if (c->n_kv_heads < 0 || c->n_heads % kv_heads(c) != 0) return LLAMA_ERR_INVALID_ARG;
     if (c->dtype != LLAMA_F32 && c->dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
     if (c->max_batch <= 0 || c->max_seq <= 0) return LLAMA_ERR_INVALID_ARG;
     if (!(c->norm_eps >= 0.f) || !(c->rope_theta > 0.f)) return LLAMA_ERR_INVALID_ARG;
@@ -199,7 +203,10 @@ int validate(const llama_config* c) {
         if (c->max_batch > 32) return LLAMA_ERR_INVALID_ARG;
         if (c->vocab % 128 != 0) return LLAMA_ERR_INVALID_ARG;   // whole 128-row head tiles
         // arrival counters of the fused decode step: one per 128-row block
-        if ((5 * (int64_t)c->d_model + hidden_of(c) + c->vocab) / 128 > MAX_COUNTERS) return LLAMA_ERR_INVALID_ARG;
+        const int64_t qkv_rows = c->d_model + 2 * (int64_t)kv_heads(c) * c->head_dim;
+        if (qkv_rows % 128 != 0) return LLAMA_ERR_INVALID_ARG;
+        if ((qkv_rows + 3 * (int64_t)c->d_model + hidden_of(c) + c->vocab) / 128 > MAX_COUNTERS)
+            return LLAMA_ERR_INVALID_ARG;
     } else {
         if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return LLAMA_ERR_INVALID_ARG;
     }
@@ -216,6 +223,7 @@ int hidden_of(const llama_config* c) {
 uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     const int esz = c->dtype == LLAMA_BF16 ? 2 : 4;
     const size_t d = c->d_model, h = hidden_of(c), V = c->vocab, L = c->n_layers;
+    const size_t kvd = (size_t)kv_heads(c) * c->head_dim;
     const size_t nmax = (size_t)c->max_batch * c->max_seq;
     size_t off = 0;
     auto take = [&](size_t bytes) -> void* {
@@ -230,7 +238,7 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     }
     for (size_t l = 0; l < L; ++l) {
         Layer ly;
-        ly.wqkv = take(3 * d * d * esz);
+        ly.wqkv = take((d + 2 * kvd) * d * esz);
         ly.wo = take(d * d * esz);
         ly.wgu = take(2 * h * d * esz);
         ly.wd = take(d * h * esz);
@@ -241,7 +249,7 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     float* g_final = (float*)take(d * 4);
     void* head = take(V * d * esz);
     float2* rope = (float2*)take((size_t)c->max_seq * (c->head_dim / 2) * sizeof(float2));
-    const size_t kv_layer = (size_t)c->max_batch * c->n_heads * c->max_seq * c->head_dim;
+    const size_t kv_layer = (size_t)c->max_batch * kv_heads(c) * c->max_seq * c->head_dim;
     void* kv = take(2 * L * kv_layer * esz);
     float* trunk = (float*)take(nmax * d * 4);
     void* xn = take(nmax * d * esz);
@@ -253,7 +261,8 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     float* logits_dec = (float*)take((size_t)c->max_batch * V * 4);
     long long part_off[5];
     int cnt_off[5];
-    const size_t pmax = (size_t)decode_step_layout(STEP_MAX_CTAS, (int)d, (int)h, (int)V, c->max_batch, part_off,
+    const size_t pmax = (size_t)decode_step_layout(STEP_MAX_CTAS, (int)(d + 2 * kvd), (int)d, (int)h, (int)V,
+                                                   c->max_batch, part_off,
                                                    cnt_off);
     float* partial = (float*)take(c->dtype == LLAMA_BF16 ? pmax * 4 : 0);
     int* counters = (int*)take(MAX_COUNTERS * 4);
@@ -348,6 +357,7 @@ EpiArgs base_args(llama_model* m, int M, int N) {
     a.M = M;
     a.N = N;
     a.H = m->cfg.n_heads;
+    a.Hkv = kv_heads(&m->cfg);
     a.hd = m->cfg.head_dim;
     a.d = m->cfg.d_model;
     a.smax = m->cfg.max_seq;
@@ -405,6 +415,8 @@ int project(llama_model* m, const char* name, int mode, const void* A, const voi
 int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
     const llama_config& c = m->cfg;
     const int d = c.d_model, h = hidden_of(&c);
+    const int nq = d + 2 * kv_heads(&c) * c.head_dim;   // Q, K, V columns
+    const int Hkv = kv_heads(&c);
     const int n = decode ? B : B * S;
     const int dt = c.dtype;
     int rc;
@@ -416,29 +428,29 @@ int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
             prof::Scope ps(st, decode ? "decode_rmsnorm" : "prefill_rmsnorm", nb, 3.0 * n * d);
             if ((rc = launch_rmsnorm(dt, m->trunk, ly.g_attn, m->xn, n, d, c.norm_eps, st))) return rc;
         }
-        EpiArgs qa = base_args(m, n, 3 * d);
+        EpiArgs qa = base_args(m, n, nq);
         qa.q = m->q;
         qa.kc = kcache(m, l);
         qa.vc = vcache(m, l);
         qa.S = decode ? 1 : S;
         qa.d_pos = decode ? m->d_pos : nullptr;
-        if ((rc = project(m, "qkv", EPI_QKV, m->xn, ly.wqkv, n, 3 * d, d, m->splits_qkv, qa, decode, st))) return rc;
+        if ((rc = project(m, "qkv", EPI_QKV, m->xn, ly.wqkv, n, nq, d, m->splits_qkv, qa, decode, st))) return rc;
         if (decode) {
             double len = 0;   // keys read this step, averaged over the sequences
             for (int b = 0; b < B; ++b) len += m->pos_h[b] + 1;
             len /= B;
             prof::Scope ps(st, "decode_attention", (2.0 * len + 2.0) * B * d * m->esz, 4.0 * B * d * len);
-            if ((rc = launch_attention_decode(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, 0,
+            if ((rc = launch_attention_decode(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, Hkv, 0,
                                               m->d_pos, c.head_dim, c.max_seq, m->attn_work, m->attn_cnt, m->d_err,
                                               st)))
                 return rc;
         } else {
             prof::Scope ps(st, "prefill_attention", 4.0 * n * d * m->esz, 2.0 * B * (double)S * (S + 1) * d);
             if (dt == LLAMA_BF16)
-                rc = launch_attention_prefill_tc(m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, S,
+                rc = launch_attention_prefill_tc(m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, Hkv, S,
                                                  c.head_dim, c.max_seq, m->d_err, st);
             else
-                rc = launch_attention_prefill_simt(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, S,
+                rc = launch_attention_prefill_simt(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, Hkv, S,
                                                    c.head_dim, c.max_seq, st);
             if (rc) return rc;
         }
@@ -495,7 +507,8 @@ StepArgs step_args(llama_model* m) {
     a.logits = m->logits_dec;
     a.partial = m->partial;
     a.counters = m->counters;
-    decode_step_layout(decode_step_ctas(), c.d_model, c.ffn_hidden, c.vocab, m->B, a.part_off, a.cnt_off);
+    decode_step_layout(decode_step_ctas(), c.d_model + 2 * kv_heads(&c) * c.head_dim, c.d_model, c.ffn_hidden,
+                       c.vocab, m->B, a.part_off, a.cnt_off);
     a.attn_work = m->step_attn_work;
     a.attn_cnt = m->attn_cnt;
     a.amax_part = m->amax_part;
@@ -510,6 +523,7 @@ StepArgs step_args(llama_model* m) {
     a.h = c.ffn_hidden;
     a.V = c.vocab;
     a.H = c.n_heads;
+    a.Hkv = kv_heads(&c);
     a.hd = c.head_dim;
     a.B = m->B;
     a.smax = c.max_seq;
@@ -531,6 +545,7 @@ int step_tables(llama_model* m) {
         w[4 * l + 3] = m->layers[l].wd;
     }
     int rc = decode_step_maps(maps.data(), w.data(), L, m->head, m->xn, m->attn, m->act, m->step_xg2, m->B,
+                              c.d_model + 2 * kv_heads(&c) * c.head_dim,
                               c.d_model, c.ffn_hidden, c.vocab);
     if (rc) return rc;
     std::vector<const float*> gains((size_t)2 * L + 1);
@@ -550,11 +565,12 @@ int decode_body(llama_model* m, cudaStream_t st) {
     if (c.dtype == LLAMA_BF16) {
         // weights + KV cache read + activations, once per step
         const double d = c.d_model, h = c.ffn_hidden, L = c.n_layers, V = c.vocab;
-        const double wbytes = 2.0 * (L * (4 * d * d + 3 * d * h) + d * V);
+        const double kvd = (double)kv_heads(&c) * c.head_dim;
+        const double wbytes = 2.0 * (L * (2 * d * d + 2 * d * kvd + 3 * d * h) + d * V);
         double keys = 0;   // keys read this step, over the sequences
         for (int b = 0; b < m->B; ++b) keys += m->pos_h[b] + 1;
-        const double kvbytes = 2.0 * 2.0 * L * keys * d;
-        const double flops = 2.0 * m->B * (L * (4 * d * d + 3 * d * h) + d * V) + 4.0 * L * keys * d;
+        const double kvbytes = 2.0 * 2.0 * L * keys * kvd;
+        const double flops = 2.0 * m->B * (L * (2 * d * d + 2 * d * kvd + 3 * d * h) + d * V) + 4.0 * L * keys * d;
         prof::Scope ps(st, "decode_step", wbytes + kvbytes, flops);
         StepArgs sa = step_args(m);
         if (prof::on) sa.timeline = m->step_timeline;
@@ -625,7 +641,7 @@ void pick_decode_splits(llama_model* m) {
         m->splits_qkv = m->splits_o = m->splits_gu = m->splits_d = m->splits_head = 1;
         return;
     }
-    m->splits_qkv = gemm_tc_pick_splits(3 * d, d);
+    m->splits_qkv = gemm_tc_pick_splits(d + 2 * kv_heads(&c) * c.head_dim, d);
     m->splits_o = gemm_tc_pick_splits(d, d);
     m->splits_gu = gemm_tc_pick_splits(2 * h, d);
     m->splits_d = gemm_tc_pick_splits(d, h);
@@ -697,9 +713,10 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
     TRY(launch_fill_f32(m->g_final, 1.0f, d, st));
     for (int l = 0; l < cfg->n_layers; ++l) {
         const Layer& ly = m->layers[l];
+        const int kvd = kv_heads(cfg) * cfg->head_dim;   // K and V rows follow the d rows of Q
         TRY(launch_init_matrix(dt, ly.wqkv, d, d, d, 0, 0, 0, seed, layer_tid(l, 0), sc, st));
-        TRY(launch_init_matrix(dt, ly.wqkv, d, d, d, 0, d, 0, seed, layer_tid(l, 1), sc, st));
-        TRY(launch_init_matrix(dt, ly.wqkv, d, d, d, 0, 2 * d, 0, seed, layer_tid(l, 2), sc, st));
+        TRY(launch_init_matrix(dt, ly.wqkv, d, kvd, kvd, 0, d, 0, seed, layer_tid(l, 1), sc, st));
+        TRY(launch_init_matrix(dt, ly.wqkv, d, kvd, kvd, 0, d + kvd, 0, seed, layer_tid(l, 2), sc, st));
         TRY(launch_init_matrix(dt, ly.wo, d, d, d, 0, 0, 0, seed, layer_tid(l, 3), sc, st));
         TRY(launch_init_matrix(dt, ly.wgu, d, h, 128, 256, 0, 0, seed, layer_tid(l, 4), sc, st));
         TRY(launch_init_matrix(dt, ly.wgu, d, h, 128, 256, 128, 0, seed, layer_tid(l, 5), sc, st));
@@ -919,7 +936,10 @@ int llama_model_tensor(const llama_model* m, const char* name, int32_t layer, vo
     else {
         const Layer* ly = lay(layer);
         if (!ly) return LLAMA_ERR_INVALID_ARG;
-        if (!strcmp(name, "wqkv")) { *d_ptr = ly->wqkv; *bytes = 3 * d * d * es; }
+        if (!strcmp(name, "wqkv")) {
+            *d_ptr = ly->wqkv;
+            *bytes = (d + 2 * (size_t)kv_heads(&c) * c.head_dim) * d * es;
+        }
         else if (!strcmp(name, "wo")) { *d_ptr = ly->wo; *bytes = d * d * es; }
         else if (!strcmp(name, "wgu")) { *d_ptr = ly->wgu; *bytes = 2 * h * d * es; }
         else if (!strcmp(name, "wd")) { *d_ptr = ly->wd; *bytes = d * h * es; }
@@ -986,13 +1006,14 @@ int llama_op_attention_prefill(int32_t dtype, const void* d_q, const void* d_k, 
                                int32_t B, int32_t H, int32_t S, int32_t head_dim, int32_t kv_stride, void* stream) {
     if (!d_q || !d_k || !d_v || !d_o || B <= 0 || H <= 0 || S <= 0 || kv_stride < S) return LLAMA_ERR_INVALID_ARG;
     if (dtype == LLAMA_F32)
-        return launch_attention_prefill_simt(dtype, d_q, d_k, d_v, d_o, B, H, S, head_dim, kv_stride,
+        return launch_attention_prefill_simt(dtype, d_q, d_k, d_v, d_o, B, H, H, S, head_dim, kv_stride,
                                              (cudaStream_t)stream);
     if (dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
     int* err = nullptr;
     int rc = op_error_word(&err);
     if (rc) return rc;
-    return launch_attention_prefill_tc(d_q, d_k, d_v, d_o, B, H, S, head_dim, kv_stride, err, (cudaStream_t)stream);
+    return launch_attention_prefill_tc(d_q, d_k, d_v, d_o, B, H, H, S, head_dim, kv_stride, err,
+                                       (cudaStream_t)stream);
 }
 
 uint64_t llama_op_attention_decode_work_bytes(int32_t B, int32_t H, int32_t max_len, int32_t head_dim) {
@@ -1011,7 +1032,7 @@ int llama_op_attention_decode(int32_t dtype, const void* d_q, const void* d_k, c
     int rc = op_error_word(&err);
     if (rc) return rc;
     if ((rc = attention_decode_clear((float*)d_work, B, H, len, head_dim, (cudaStream_t)stream))) return rc;
-    return launch_attention_decode(dtype, d_q, d_k, d_v, d_o, B, H, len, nullptr, head_dim, kv_stride,
+    return launch_attention_decode(dtype, d_q, d_k, d_v, d_o, B, H, H, len, nullptr, head_dim, kv_stride,
                                    (float*)d_work, attention_decode_counters((float*)d_work, B, H, len, head_dim),
                                    err, (cudaStream_t)stream);
 }

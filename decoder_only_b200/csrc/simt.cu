@@ -113,11 +113,13 @@ int launch_epilogue_from_f32(int dtype, int mode, const float* C, int ldc, const
 // ---------------------------------------------------------------------------
 // CUDA-core causal flash attention (online softmax), one CTA per
 // (64-query tile, head, sequence); key tiles above the diagonal are skipped.
-// q: [B][H][S][HD]; k, v: [B][H][kv_stride][HD]; o: [B*S][H*HD].
+// q: [B][H][S][HD]; k, v: [B][Hkv][kv_stride][HD] (query head h reads key/value
+// head h / (H / Hkv)); o: [B*S][H*HD].
 template <typename T, int HD>
 __global__ void __launch_bounds__(256) attn_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                                 const T* __restrict__ v, T* __restrict__ o,
-                                                                int H, int S, int kv_stride, float scale) {
+                                                                int H, int Hkv, int S, int kv_stride,
+                                                                float scale) {
     constexpr int BQ = 64, BK = 64, LD = HD + 1, CPT = HD / 16;
     extern __shared__ float sm[];
     float* Qs = sm;                 // [BQ][LD]
@@ -129,9 +131,10 @@ __global__ void __launch_bounds__(256) attn_prefill_simt_kernel(const T* __restr
     const int q0 = qt * BQ;
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
     const size_t head = (size_t)b * H + h;
+    const size_t kv_head = (size_t)b * Hkv + h / (H / Hkv);
     const T* qh = q + head * S * HD;
-    const T* kh = k + head * (size_t)kv_stride * HD;
-    const T* vh = v + head * (size_t)kv_stride * HD;
+    const T* kh = k + kv_head * (size_t)kv_stride * HD;
+    const T* vh = v + kv_head * (size_t)kv_stride * HD;
     for (int i = tid; i < BQ * HD; i += 256) {
         const int r = i / HD, c = i % HD;
         Qs[r * LD + c] = (q0 + r < S) ? to_f32(qh[(size_t)(q0 + r) * HD + c]) * scale : 0.f;
@@ -248,24 +251,25 @@ int attention_prepare() {
 }
 
 template <typename T, int HD>
-static int launch_attn_simt_t(const void* q, const void* k, const void* v, void* o, int B, int H, int S,
-                              int kv_stride, cudaStream_t st) {
+static int launch_attn_simt_t(const void* q, const void* k, const void* v, void* o, int B, int H, int Hkv,
+                              int S, int kv_stride, cudaStream_t st) {
     const size_t smem = attn_simt_smem<T, HD>();
     int rc = attn_simt_attr<T, HD>(smem);
     if (rc) return rc;
     dim3 grid(ceil_div(S, 64), H, B);
-    attn_prefill_simt_kernel<T, HD><<<grid, 256, smem, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, H, S,
-                                                             kv_stride, 1.0f / sqrtf((float)HD));
+    attn_prefill_simt_kernel<T, HD><<<grid, 256, smem, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, H, Hkv,
+                                                             S, kv_stride, 1.0f / sqrtf((float)HD));
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }
 
 int launch_attention_prefill_simt(int dtype, const void* q, const void* k, const void* v, void* o, int B,
-                                  int H, int S, int hd, int kv_stride, cudaStream_t st) {
+                                  int H, int Hkv, int S, int hd, int kv_stride, cudaStream_t st) {
     if (B <= 0 || S <= 0) return LLAMA_OK;
+    if (Hkv <= 0 || H % Hkv != 0) return LLAMA_ERR_INVALID_ARG;
     if (dtype != LLAMA_F32) return LLAMA_ERR_INVALID_ARG;   // bf16 runs on the tensor cores (attn_tc.cu)
-    if (hd == 128) return launch_attn_simt_t<float, 128>(q, k, v, o, B, H, S, kv_stride, st);
-    if (hd == 64) return launch_attn_simt_t<float, 64>(q, k, v, o, B, H, S, kv_stride, st);
-    if (hd == 32) return launch_attn_simt_t<float, 32>(q, k, v, o, B, H, S, kv_stride, st);
+    if (hd == 128) return launch_attn_simt_t<float, 128>(q, k, v, o, B, H, Hkv, S, kv_stride, st);
+    if (hd == 64) return launch_attn_simt_t<float, 64>(q, k, v, o, B, H, Hkv, S, kv_stride, st);
+    if (hd == 32) return launch_attn_simt_t<float, 32>(q, k, v, o, B, H, Hkv, S, kv_stride, st);
     return LLAMA_ERR_INVALID_ARG;
 }

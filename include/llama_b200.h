@@ -78,6 +78,9 @@ typedef struct llama_config {
     int32_t dtype;       /* llama_dtype */
     int32_t max_batch;   /* largest B passed to prefill / decode */
     int32_t max_seq;     /* prompt length + decode steps, per sequence */
+    int32_t n_kv_heads;  /* key/value heads (grouped keys and values); 0 => n_heads.
+                            n_heads % n_kv_heads == 0; query head h uses key/value
+                            head h / (n_heads / n_kv_heads) */
 } llama_config;
 
 typedef struct llama_model llama_model; /* opaque host handle */
@@ -85,7 +88,7 @@ typedef struct llama_model llama_model; /* opaque host handle */
 /* ------------------------------------------------------------------ model */
 
 /* Device bytes the model arena must hold for `cfg`: weights, RoPE table,
- * KV cache [L][2][max_batch][H][max_seq][head_dim], activations and
+ * KV cache [L][2][max_batch][n_kv_heads][max_seq][head_dim], activations and
  * workspace.  Host-only; queues nothing. */
 LLAMA_API int llama_model_bytes(const llama_config* cfg, uint64_t* bytes_out);
 
