@@ -480,15 +480,15 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
 // range leaves its (max, sum, output) in the workspace and the last range to
 // arrive merges them in range order.
 template <int BN, int HD>
-__device__ __forceinline__ void attn_issue(const StepArgs& a, int l, int b, int h, int kc, bool with_q, int len,
+// Chunk kc of query pair pr = b * H + h, whose keys and values are cache row
+// kvr = b * Hkv + h / (H / Hkv).
+__device__ __forceinline__ void attn_issue(const StepArgs& a, int l, int pr, int kvr, int kc, bool with_q, int len,
                                            uint32_t dst, uint32_t bar) {
     const int k0 = kc * ACH;
     const int nkeys = min(len - k0, ACH);
     const bf16* kc_ = a.kv + (size_t)(2 * l) * a.kv_layer;
     const bf16* vc = kc_ + a.kv_layer;
-    const int pr = b * a.H + h;                                        // query head h of sequence b ...
-    const size_t kvr = (size_t)b * a.Hkv + h / (a.H / a.Hkv);         // ... reads key/value head h / group
-    const size_t off = (kvr * a.smax + k0) * HD;
+    const size_t off = ((size_t)kvr * a.smax + k0) * HD;
     const uint32_t bytes = (uint32_t)(nkeys * HD * 2);
     // cache rows are read once per step (per query head of a group): first out of L2
     const uint64_t pol = l2_evict_first();
@@ -539,9 +539,11 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
     if (gw >= Wp) return true;
     const long long cs = Ctot * gw / Wp, ce = Ctot * (gw + 1) / Wp;
     auto owner = [&](long long i) { return (int)(((i + 1) * Wp - 1) / Ctot); };
-    // unit index -> (sequence b, head h, chunk kc) with b's length and chunk count
+    // unit index -> (sequence b, head h, chunk kc) with b's length and chunk
+    // count; the key/value row kvr = b * Hkv + h / G follows h without a division
+    const int G = a.H / a.Hkv;
     struct Pos {
-        int b, h, kc, len, nch;
+        int b, h, kc, len, nch, kvr, hg;
     };
     auto locate = [&](long long c) {
         Pos q;
@@ -551,11 +553,17 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
         const long long rem = c - (long long)a.H * __shfl_sync(0xffffffffu, excl, q.b);
         q.h = (int)(rem / q.nch);
         q.kc = (int)(rem - (long long)q.h * q.nch);
+        q.kvr = q.b * a.Hkv + q.h / G;
+        q.hg = q.h % G;
         return q;
     };
     auto advance = [&](Pos& q) {
         if (++q.kc < q.nch) return;
         q.kc = 0;
+        if (++q.hg == G) {        // the next key/value head (also across sequences: rows are b * Hkv + ...)
+            q.hg = 0;
+            ++q.kvr;
+        }
         if (++q.h < a.H) return;
         q.h = 0;
         ++q.b;
@@ -576,8 +584,8 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
     Pos iq = locate(cs);
     auto issue = [&](int buf) {
         if (lane == 0)
-            attn_issue<BN, HD>(a, l, iq.b, iq.h, iq.kc, ic == cs || iq.kc == 0, iq.len, wbuf + buf * C::ATT_BUF,
-                               wbar + 8 * buf);
+            attn_issue<BN, HD>(a, l, iq.b * a.H + iq.h, iq.kvr, iq.kc, ic == cs || iq.kc == 0, iq.len,
+                               wbuf + buf * C::ATT_BUF, wbar + 8 * buf);
         ++ic;
         advance(iq);
     };
