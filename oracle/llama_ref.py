@@ -26,6 +26,11 @@ Readings taken where the pages are silent (each also listed in the design doc):
   * RoPE acts per head (its d is the head dimension), on interleaved
     (even, odd) channel pairs, angle = position * base^(-2i/d_head).
   * Heads are contiguous blocks of d_head columns of Q, K, V.
+  * The bias variant (the page's bias=True count): every linear layer adds a
+    bias of its output width (Q, K, V before RoPE), and the two in-layer
+    norms add a shift after the gain, z = x / rms(x) * g + beta; the final
+    norm and the head have none (the count has none).  Biases and shifts are
+    drawn N(0, 0.02^2) like the weights and kept in fp32.
   * Grouped keys and values ([NAR] "GQA Was Not an Original LLaMA
     Feature"; LLaMA itself has one K/V head per query head): with n_kv
     key/value heads, K and V have n_kv heads of d_head columns and query
@@ -221,7 +226,16 @@ def layer_weights(shape, layer: int, seed: int = 0) -> dict:
          for name, (r, c) in dims.items()}
     W["g_attn"] = np.ones(d)
     W["g_ffn"] = np.ones(d)
+    if getattr(shape, "bias", False):
+        vec = {"bq": d, "bk": kvd, "bv": kvd, "bo": d, "bg": h, "bu": h, "bd": d, "beta_attn": d, "beta_ffn": d}
+        for name, n in vec.items():
+            W[name] = _draw(seed, synth.layer_tensor_id(layer, name), 1, n, "f32")[0]
     return W
+
+
+def _b(W, name):
+    """A bias or shift of the bias variant; 0 in the original model."""
+    return W.get(name, 0.0)
 
 
 def embed_table(shape, seed: int = 0) -> np.ndarray:
@@ -254,24 +268,24 @@ def attn_sublayer(z, W, positions, shape, kv_out=None, storage=None):
     st, st_kv = _storer(storage), _storer(storage, kv=True)
     H, Hkv = shape.n_heads, _kv_heads(shape)
     G = H // Hkv                                   # query heads per key/value head
-    q = split_heads(z @ W["wq"], H)
-    k = split_heads(z @ W["wk"], Hkv)
-    v = split_heads(z @ W["wv"], Hkv)
+    q = split_heads(z @ W["wq"] + _b(W, "bq"), H)
+    k = split_heads(z @ W["wk"] + _b(W, "bk"), Hkv)
+    v = split_heads(z @ W["wv"] + _b(W, "bv"), Hkv)
     q = st(rope(q, positions, shape.rope_theta))
     k = st_kv(rope(k, positions, shape.rope_theta))
     v = st_kv(v)
     if kv_out is not None:
         kv_out.append((k, v))
     o = np.stack([causal_attention(q[hh], k[hh // G], v[hh // G]) for hh in range(H)])
-    return st(merge_heads(o)) @ W["wo"]
+    return st(merge_heads(o)) @ W["wo"] + _b(W, "bo")
 
 
 def swiglu_ffn(z, W, storage=None):
     """(SiLU(z Wg) * (z Wu)) Wd, (n,d) -> (n,h) -> (n,d).  [PFD] SwiGLU;
     [NAR] SwiGLU(x) = SiLU(x W_g) (.) (x W_v)."""
-    gate = silu(z @ W["wg"])
-    up = z @ W["wu"]
-    return _storer(storage)(gate * up) @ W["wd"]
+    gate = silu(z @ W["wg"] + _b(W, "bg"))
+    up = z @ W["wu"] + _b(W, "bu")
+    return _storer(storage)(gate * up) @ W["wd"] + _b(W, "bd")
 
 
 def pre_norm_block(x, W, positions, shape, kv_out=None, storage=None):
@@ -281,8 +295,10 @@ def pre_norm_block(x, W, positions, shape, kv_out=None, storage=None):
     [PFD] "The one formula" and "Pre-norm: the norm goes on the branch, not
     the trunk"."""
     st = _storer(storage)
-    h = x + attn_sublayer(st(rms_norm(x, W["g_attn"], shape.norm_eps)), W, positions, shape, kv_out, storage)
-    y = h + swiglu_ffn(st(rms_norm(h, W["g_ffn"], shape.norm_eps)), W, storage)
+    z = rms_norm(x, W["g_attn"], shape.norm_eps) + _b(W, "beta_attn")
+    h = x + attn_sublayer(st(z), W, positions, shape, kv_out, storage)
+    z = rms_norm(h, W["g_ffn"], shape.norm_eps) + _b(W, "beta_ffn")
+    y = h + swiglu_ffn(st(z), W, storage)
     return y
 
 
@@ -358,10 +374,10 @@ def decode_step(shape, cache: list, tokens: np.ndarray, seed: int = 0, weights=N
     for l in range(shape.n_layers):
         W = get_w(l)
         Kc, Vc = cache[l]
-        z = rms_norm(x, W["g_attn"], shape.norm_eps)
-        q = (z @ W["wq"]).reshape(B, H, dh)
-        k = (z @ W["wk"]).reshape(B, Hkv, dh)
-        v = (z @ W["wv"]).reshape(B, Hkv, dh)
+        z = rms_norm(x, W["g_attn"], shape.norm_eps) + _b(W, "beta_attn")
+        q = (z @ W["wq"] + _b(W, "bq")).reshape(B, H, dh)
+        k = (z @ W["wk"] + _b(W, "bk")).reshape(B, Hkv, dh)
+        v = (z @ W["wv"] + _b(W, "bv")).reshape(B, Hkv, dh)
         pos = np.array([p])
         q = rope(q.reshape(B * H, 1, dh), pos, shape.rope_theta).reshape(B, H, dh)
         k = rope(k.reshape(B * Hkv, 1, dh), pos, shape.rope_theta).reshape(B, Hkv, dh)
@@ -373,9 +389,9 @@ def decode_step(shape, cache: list, tokens: np.ndarray, seed: int = 0, weights=N
                 s = Kc[b, hh // G] @ q[b, hh] / math.sqrt(dh)      # (p+1,)
                 w = np.exp(s - s.max())
                 o[b, hh] = (w / w.sum()) @ Vc[b, hh // G]
-        x = x + o.reshape(B, H * dh) @ W["wo"]
-        z = rms_norm(x, W["g_ffn"], shape.norm_eps)
-        x = x + (silu(z @ W["wg"]) * (z @ W["wu"])) @ W["wd"]
+        x = x + o.reshape(B, H * dh) @ W["wo"] + _b(W, "bo")
+        z = rms_norm(x, W["g_ffn"], shape.norm_eps) + _b(W, "beta_ffn")
+        x = x + (silu(z @ W["wg"] + _b(W, "bg")) * (z @ W["wu"] + _b(W, "bu"))) @ W["wd"] + _b(W, "bd")
         new_cache.append((Kc, Vc))
         del W
     logits = rms_norm(x, np.ones(shape.d_model), shape.norm_eps) @ head_matrix(shape, seed)

@@ -11,7 +11,10 @@ generator, and the tests check the two agree.
 Tensor ids (the generator key's second word):
     EMBED = 1, HEAD = 2, TOKENS = 3, TRUNK = 4,
     layer l, matrix m  ->  16 + 8*l + m  with m = wq 0, wk 1, wv 2, wo 3,
-                                              wg 4, wu 5, wd 6.
+                                              wg 4, wu 5, wd 6;
+    layer l, bias k    ->  2^20 + 16*l + k with k = bq 0, bk 1, bv 2, bo 3,
+                           bg 4, bu 5, bd 6, beta_attn 7, beta_ffn 8
+                           (the bias variant: linear biases, norm shifts).
 Element e of a matrix is its row-major index in the (d_in, d_out)
 orientation in which the forward pass multiplies ``x @ W``; the embedding
 table is (V, d) row-major.
@@ -36,7 +39,13 @@ _MATRIX = {"wq": 0, "wk": 1, "wv": 2, "wo": 3, "wg": 4, "wu": 5, "wd": 6}
 WEIGHT_STD = 0.02
 
 
+_BIAS = {"bq": 0, "bk": 1, "bv": 2, "bo": 3, "bg": 4, "bu": 5, "bd": 6, "beta_attn": 7, "beta_ffn": 8}
+BIAS_BASE = 1 << 20
+
+
 def layer_tensor_id(layer: int, name: str) -> int:
+    if name in _BIAS:
+        return BIAS_BASE + 16 * layer + _BIAS[name]
     return 16 + 8 * layer + _MATRIX[name]
 
 

@@ -23,6 +23,7 @@ class ModelShape:
     norm_eps: float = 1e-6
     rope_theta: float = 10000.0
     n_kv_heads: int = 0          # key/value heads (GQA / MQA); 0: one per query head
+    bias: bool = False           # the bias variant: linear biases and norm shifts
 
     @property
     def kv_heads(self) -> int:

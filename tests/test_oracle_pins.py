@@ -363,3 +363,67 @@ def test_grouped_kv_cache_size_and_decode(n_kv):
         logits, nxt, c7 = oracle.decode_step(s, c7, tok[:, t])
         assert np.allclose(logits, lg[:, t], atol=1e-12)
     assert c7[0][0].shape == (3, n_kv, 10, s.head_dim)
+
+
+# ---------------------------------------------------------------- the bias variant
+
+def _bias_shape():
+    return ModelShape("b", 1, 8, 2, 4, 16, 11, dtype="f32", bias=True)
+
+
+def _bias_weights(s, **nonzero):
+    """Every matrix zero except the named ones; biases and shifts from the generator."""
+    W = oracle.layer_weights(s, 0)
+    for name in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+        W[name] = nonzero.get(name, np.zeros_like(W[name]))
+    return W
+
+
+def test_bias_variant_closed_forms():
+    """The page's bias=True count ([PFD] "6.7B parameters, 1T tokens: the
+    arithmetic"): every linear layer adds a bias, each in-layer norm a shift.
+    With all matrices zero a block is y = x + b_o + b_d (V rows all equal
+    b_v average to b_v, which W_o = 0 drops); with W_o = I the value bias
+    passes, y = x + b_v + b_o + b_d; with W_q = W_k = 0 the causal weights
+    are uniform once b_q = 0, so W_v = W_o = I give h_t = x_t + mean_{j<=t}(rms(x_j) g +
+    beta_attn) + b_v + b_o; and W_u = W_d = identity blocks give
+    y = h + (SiLU(b_g) * (rms(h) g + beta_ffn + b_u))[:d] + b_d."""
+    s = _bias_shape()
+    d, h = s.d_model, s.ffn_hidden
+    x = np.random.default_rng(30).normal(size=(6, d))
+    pos = np.arange(6)
+    W = _bias_weights(s)
+    y = oracle.pre_norm_block(x, W, pos, s)
+    assert np.allclose(y, x + W["bo"] + W["bd"], atol=1e-13)
+    W = _bias_weights(s, wo=np.eye(d))
+    y = oracle.pre_norm_block(x, W, pos, s)
+    assert np.allclose(y, x + W["bv"] + W["bo"] + W["bd"], atol=1e-13)
+    eye_du = np.eye(d, h)
+    W = _bias_weights(s, wv=np.eye(d), wo=np.eye(d), wu=eye_du, wd=eye_du.T)
+    W["bq"] = np.zeros(d)       # q = 0: every score 0 (RoPE would turn b_q and b_k by position)
+    y = oracle.pre_norm_block(x, W, pos, s)
+    zn = oracle.rms_norm(x, np.ones(d), s.norm_eps) + W["beta_attn"]
+    hh = x + np.cumsum(zn, axis=0) / (pos + 1)[:, None] + W["bv"] + W["bo"]
+    z2 = oracle.rms_norm(hh, np.ones(d), s.norm_eps) + W["beta_ffn"]
+    act = oracle.silu(W["bg"])[None, :] * (z2 @ eye_du + W["bu"][None, :])
+    assert np.allclose(y, hh + act @ eye_du.T + W["bd"], atol=1e-12)
+
+
+def test_bias_variant_with_zero_biases_is_the_original_model():
+    s = _bias_shape()
+    W = oracle.layer_weights(s, 0)
+    for name in ("bq", "bk", "bv", "bo", "bg", "bu", "bd", "beta_attn", "beta_ffn"):
+        W[name] = np.zeros_like(W[name])
+    tok = np.random.default_rng(31).integers(0, s.vocab, size=(2, 7))
+    plain = s.with_(bias=False)
+    a = oracle.prefill(s, tok, weights=lambda l: W)
+    b = oracle.prefill(plain, tok, weights=lambda l: {k: v for k, v in W.items() if k.startswith(("w", "g"))})
+    assert np.allclose(a, b, rtol=0, atol=1e-13)
+    # and the biases move it
+    assert not np.allclose(a, oracle.prefill(s, tok), atol=1e-6)
+    # decode == prefill rows with biases
+    lg, cache = oracle.prefill(s, tok[:, :5], return_cache=True)
+    full = oracle.prefill(s, tok)
+    for t in range(5, 7):
+        logits, _, cache = oracle.decode_step(s, cache, tok[:, t])
+        assert np.allclose(logits, full[:, t], atol=1e-12)
