@@ -32,7 +32,8 @@ class LlamaConfig(ctypes.Structure):
     _fields_ = [("n_layers", ctypes.c_int32), ("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("ffn_hidden", ctypes.c_int32), ("vocab", ctypes.c_int32),
                 ("norm_eps", ctypes.c_float), ("rope_theta", ctypes.c_float), ("dtype", ctypes.c_int32),
-                ("max_batch", ctypes.c_int32), ("max_seq", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32)]
+                ("max_batch", ctypes.c_int32), ("max_seq", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("bias", ctypes.c_int32)]
 
 
 def _load():
@@ -118,7 +119,8 @@ def make_config(shape, max_batch: int, max_seq: int) -> LlamaConfig:
     ffn_hidden, vocab, dtype ('bf16' | 'f32'), norm_eps, rope_theta."""
     return LlamaConfig(shape.n_layers, shape.d_model, shape.n_heads, shape.head_dim, shape.ffn_hidden,
                        shape.vocab, shape.norm_eps, shape.rope_theta, BF16 if shape.dtype == "bf16" else F32,
-                       max_batch, max_seq, int(getattr(shape, "n_kv_heads", 0) or 0))
+                       max_batch, max_seq, int(getattr(shape, "n_kv_heads", 0) or 0),
+                       int(bool(getattr(shape, "bias", False))))
 
 
 def model_bytes(cfg: LlamaConfig) -> int:

@@ -400,11 +400,14 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
         float gs[BN], us[BN];
         splitk_sum<BN>(part + (size_t)(256 * j + et) * ns * Mp, nseg_of(2 * j), M, Mp, gs);
         splitk_sum<BN>(part + (size_t)(256 * j + 128 + et) * ns * Mp, nseg_of(2 * j + 1), M, Mp, us);
+        const float* cb = a.biases ? a.biases[4 * l + 2] : nullptr;   // folded gate / up biases
+        const float bg = cb ? cb[256 * j + et] : 0.f, bu = cb ? cb[256 * j + 128 + et] : 0.f;
 #pragma unroll
         for (int b = 0; b < BN; ++b)
             if (b < M) {
                 const float inv = sm.sinv[b];
-                a.act[(size_t)b * a.h + 128 * j + et] = __float2bfloat16_rn(silu_f(gs[b] * inv) * (us[b] * inv));
+                a.act[(size_t)b * a.h + 128 * j + et] =
+                    __float2bfloat16_rn(silu_f(gs[b] * inv + bg) * (us[b] * inv + bu));
             }
         esync();
         if (tid == 0) count_done(done_ctr(a, l, DK_GU));
@@ -427,12 +430,13 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
             // and the block's sum of squares per row
             const bool to_ffn = (type == PH_O);
             const float gn = (to_ffn ? a.gains[2 * l + 1] : a.gains[2 * (l + 1)])[n];
+            const float bn = a.biases ? a.biases[4 * l + (to_ffn ? 1 : 3)][n] : 0.f;   // b_o / b_d
             bf16* xg = to_ffn ? a.xg2 : a.xg;
 #pragma unroll
             for (int b = 0; b < BN; ++b)
                 if (b < M) {
                     float* o = a.trunk + (size_t)b * a.d + n;
-                    const float x = __ldcg(o) + sum[b];
+                    const float x = __ldcg(o) + sum[b] + bn;
                     *o = x;
                     xg[(size_t)b * a.d + n] = __float2bfloat16_rn(x * gn);
                     sm.xbuf[b * XLD + et] = x * x;
@@ -1154,6 +1158,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                 ep.d = a.d;
                 ep.smax = a.smax;
                 ep.Hkv = a.Hkv;
+                ep.bias = (type == PH_QKV && a.biases) ? a.biases[4 * l] : nullptr;   // folded QKV biases
                 for (int i = w.s; i < w.e;) {
                     const int mb = i / w.kbt;
                     const bool ok = mbar_wait(sm.tfull + 8 * acc, acc_ph, abort_flag, a.err);

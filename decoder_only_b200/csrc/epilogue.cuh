@@ -35,6 +35,7 @@ struct EpiArgs {
     int S;                // tokens per sequence in this call (prefill), 1 in decode
     int H, hd, d, smax;
     int Hkv;              // key/value heads: columns [d, d + Hkv hd) are K, then V
+    const float* bias;    // the bias variant: fp32 per output column (weight row order), or NULL
 };
 
 __device__ __forceinline__ float silu_f(float u) { return u / (1.0f + __expf(-u)); }
@@ -58,16 +59,36 @@ __device__ __forceinline__ void store32<bf16>(bf16* dst, const float (&v)[32]) {
                            pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
 }
 
-// Residual add of 32 columns (n0 % 32 == 0, n0 + 32 <= N).
+// 32 bias values starting at column n0 (zeros without the bias variant)
+__device__ __forceinline__ void bias32(const float* bias, int n0, float (&b)[32]) {
+    if (bias) {
+        const float4* p = reinterpret_cast<const float4*>(bias + n0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 t = p[j];
+            b[4 * j] = t.x;
+            b[4 * j + 1] = t.y;
+            b[4 * j + 2] = t.z;
+            b[4 * j + 3] = t.w;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) b[j] = 0.f;
+    }
+}
+
+// Residual add of 32 columns (n0 % 32 == 0, n0 + 32 <= N), plus the bias.
 __device__ __forceinline__ void epi_resid32(const EpiArgs& a, int m, int n0, const float (&v)[32]) {
     float4* p = reinterpret_cast<float4*>(a.out + (size_t)m * a.ld_out + n0);
+    float b[32];
+    bias32(a.bias, n0, b);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         float4 t = p[j];
-        t.x += v[4 * j];
-        t.y += v[4 * j + 1];
-        t.z += v[4 * j + 2];
-        t.w += v[4 * j + 3];
+        t.x += v[4 * j] + b[4 * j];
+        t.y += v[4 * j + 1] + b[4 * j + 1];
+        t.z += v[4 * j + 2] + b[4 * j + 2];
+        t.w += v[4 * j + 3] + b[4 * j + 3];
         p[j] = t;
     }
 }
@@ -84,13 +105,18 @@ __device__ __forceinline__ void epi_f32_32(const EpiArgs& a, int m, int n0, cons
     }
 }
 
-// SwiGLU: hidden units j0..j0+31 from their gate and up pre-activations.
+// SwiGLU: hidden units j0..j0+31 from their gate and up pre-activations
+// (weight rows (j0 / 128) * 256 + j0 % 128 .. and 128 rows further).
 template <typename T>
 __device__ __forceinline__ void epi_swiglu32(const EpiArgs& a, int m, int j0, const float (&g)[32],
                                              const float (&u)[32]) {
+    const int ng = (j0 / 128) * 256 + (j0 % 128);
+    float bg[32], bu[32];
+    bias32(a.bias, ng, bg);
+    bias32(a.bias, ng + 128, bu);
     float r[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) r[j] = silu_f(g[j]) * u[j];
+    for (int j = 0; j < 32; ++j) r[j] = silu_f(g[j] + bg[j]) * (u[j] + bu[j]);
     store32<T>(reinterpret_cast<T*>(a.act) + (size_t)m * a.hidden + j0, r);
 }
 
@@ -103,6 +129,8 @@ __device__ __forceinline__ void epi_qkv32(const EpiArgs& a, int m, int n0, const
     const int c = which == 0 ? n0 : n0 - a.d - (which - 1) * kvd;
     const int head = c / a.hd;           // query head (Q) or key/value head (K, V)
     const int i0 = c - head * a.hd;      // multiple of 32 within the head
+    float bq[32];
+    bias32(a.bias, n0, bq);
     int b, s, pos;
     if (a.d_pos) {                       // decode: one token per sequence at its own position
         b = m;
@@ -119,13 +147,13 @@ __device__ __forceinline__ void epi_qkv32(const EpiArgs& a, int m, int n0, const
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             float2 t = cs[j];
-            float x0 = v[2 * j], x1 = v[2 * j + 1];
+            float x0 = v[2 * j] + bq[2 * j], x1 = v[2 * j + 1] + bq[2 * j + 1];
             r[2 * j] = x0 * t.x - x1 * t.y;
             r[2 * j + 1] = x0 * t.y + x1 * t.x;
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = v[j];
+        for (int j = 0; j < 32; ++j) r[j] = v[j] + bq[j];
     }
     T* dst;
     if (which == 0) {

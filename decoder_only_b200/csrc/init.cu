@@ -104,3 +104,28 @@ int launch_fill_f32(float* dst, float v, int64_t n, cudaStream_t st) {
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }
+
+// c[r] = b[r] + sum_k W[r][k] beta[k] (fp32 accumulate), one warp per row:
+// the folded bias of a projection that consumes a shifted RMSNorm.
+template <typename T>
+__global__ void bias_fold_kernel(const T* __restrict__ W, int rows, int K, const float* __restrict__ beta,
+                                 const float* __restrict__ b, float* __restrict__ c) {
+    const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (r >= rows) return;
+    const T* w = W + (size_t)r * K;
+    float s = 0.f;
+    for (int k = lane; k < K; k += 32) s = fmaf(to_f32(w[k]), beta[k], s);
+    s = warp_sum(s);
+    if (lane == 0) c[r] = b[r] + s;
+}
+
+int launch_bias_fold(int dtype, const void* W, int rows, int K, const float* beta, const float* b, float* c,
+                     cudaStream_t st) {
+    const int blocks = (rows + 7) / 8;
+    if (dtype == LLAMA_BF16)
+        bias_fold_kernel<bf16><<<blocks, 256, 0, st>>>((const bf16*)W, rows, K, beta, b, c);
+    else
+        bias_fold_kernel<float><<<blocks, 256, 0, st>>>((const float*)W, rows, K, beta, b, c);
+    LLAMA_LAUNCH_CHECK();
+    return LLAMA_OK;
+}

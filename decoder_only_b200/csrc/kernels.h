@@ -15,10 +15,14 @@ struct EpiArgs;
 int launch_init_matrix(int dtype, void* dst, int K, int N_log, int blk, int blk_stride, int row_off,
                        int rowmajor_nk, uint32_t seed, uint32_t tensor_id, double scale, cudaStream_t st);
 int launch_fill_f32(float* dst, float v, int64_t n, cudaStream_t st);
+// c = b + W beta per row of W [rows, K] (the bias variant's folded bias)
+int launch_bias_fold(int dtype, const void* W, int rows, int K, const float* beta, const float* b, float* c,
+                     cudaStream_t st);
 
 // norm.cu
+// y = x / rms(x) * g (+ beta, the bias variant's shift, when beta is not NULL)
 int launch_rmsnorm(int dtype, const float* x, const float* g, void* y, int rows, int d, float eps,
-                   cudaStream_t st);
+                   cudaStream_t st, const float* beta = nullptr);
 int launch_embed(int dtype, const int32_t* tok, const void* E, float* x, int rows, int d, int vocab, int* err,
                  cudaStream_t st);
 int launch_argmax(const float* logits, int rows, int n, int64_t ld, int32_t* out, cudaStream_t st);
@@ -77,6 +81,8 @@ __host__ __device__ inline int step_slots(int mblk, int ctas) { return (ctas + m
 struct StepArgs {
     const CUtensorMap* maps;      // device table: 4 per layer (W_qkv, W_o, W_gu, W_d), head, xg, attn, act, xg2
     const float* const* gains;    // device table [2L + 1]: g_attn[l], g_ffn[l], ..., g_final
+    const float* const* biases;   // bias variant: device table [4L] (b_qkv + W_qkv beta_attn, b_o,
+                                  // b_gu + W_gu beta_ffn, b_d per layer), or NULL
     const __nv_bfloat16* embed;
     __nv_bfloat16* kv;            // layer l: K at kv + 2l * kv_layer, V at kv + (2l + 1) * kv_layer
     size_t kv_layer;

@@ -112,11 +112,18 @@ namespace {
 
 constexpr uint32_t TID_EMBED = 1, TID_HEAD = 2;
 inline uint32_t layer_tid(int l, int m) { return 16u + 8u * (uint32_t)l + (uint32_t)m; }
+// bias variant vectors: bq 0, bk 1, bv 2, bo 3, bg 4, bu 5, bd 6, beta_attn 7, beta_ffn 8
+inline uint32_t bias_tid(int l, int k) { return (1u << 20) + 16u * (uint32_t)l + (uint32_t)k; }
 constexpr int MAX_COUNTERS = 4096;
 
 struct Layer {
     void *wqkv, *wo, *wgu, *wd;
     float *g_attn, *g_ffn;
+    // the bias variant (NULL otherwise), fp32 in weight-row order: Q|K|V, O,
+    // gate/up interleaved like W_gu, down; the norm shifts; and the decode
+    // step's folded biases b + W beta of the projections that consume a norm
+    float *b_qkv = nullptr, *b_o = nullptr, *b_gu = nullptr, *b_d = nullptr;
+    float *beta_attn = nullptr, *beta_ffn = nullptr, *c_qkv = nullptr, *c_gu = nullptr;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -155,6 +162,7 @@ struct llama_model {
     int* attn_cnt;           // decode-attention arrival counters [max_batch * H]
     CUtensorMap* step_maps;  // decode-step tensor-map table (device) [4L + 5]
     const float** step_gains;  // decode-step gain table (device) [2L + 1]
+    const float** step_biases; // decode-step bias table (device) [4L], bias variant only
     unsigned int* step_bar;  // decode-step synchronisation words
     void* step_xg2;          // decode-step FFN-norm input g * x, bf16 [max_batch, d]
     float* step_ssq;         // decode-step block sums of squares [2][64][32]
@@ -244,6 +252,16 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
         ly.wd = take(d * h * esz);
         ly.g_attn = (float*)take(d * 4);
         ly.g_ffn = (float*)take(d * 4);
+        if (c->bias) {
+            ly.b_qkv = (float*)take((d + 2 * kvd) * 4);
+            ly.b_o = (float*)take(d * 4);
+            ly.b_gu = (float*)take(2 * h * 4);
+            ly.b_d = (float*)take(d * 4);
+            ly.beta_attn = (float*)take(d * 4);
+            ly.beta_ffn = (float*)take(d * 4);
+            ly.c_qkv = (float*)take((d + 2 * kvd) * 4);
+            ly.c_gu = (float*)take(2 * h * 4);
+        }
         if (m) m->layers[l] = ly;
     }
     float* g_final = (float*)take(d * 4);
@@ -269,6 +287,7 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     int* attn_cnt = (int*)take((size_t)c->max_batch * c->n_heads * 4);
     CUtensorMap* step_maps = (CUtensorMap*)take((size_t)(4 * L + 5) * sizeof(CUtensorMap));
     const float** step_gains = (const float**)take((size_t)(2 * L + 1) * sizeof(float*));
+    const float** step_biases = (const float**)take(c->bias ? (size_t)(4 * L) * sizeof(float*) : 0);
     unsigned int* step_bar = (unsigned int*)take(decode_step_sync_words((int)L) * 4);
     void* step_xg2 = take((size_t)c->max_batch * d * esz);
     float* step_ssq = (float*)take(2 * 64 * 32 * 4);
@@ -308,6 +327,7 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
         m->attn_cnt = attn_cnt;
         m->step_maps = step_maps;
         m->step_gains = step_gains;
+        m->step_biases = c->bias ? step_biases : nullptr;
         m->step_bar = step_bar;
         m->step_xg2 = step_xg2;
         m->step_ssq = step_ssq;
@@ -404,7 +424,7 @@ int project(llama_model* m, const char* name, int mode, const void* A, const voi
     }
     // fp32 storage: SIMT GEMM
     prof::Scope ps(st, region, in_bytes + out_bytes(mode, M, N, m->esz), flops);
-    if (mode == EPI_RESID) return launch_gemm_simt(dt, A, W, a.out, M, N, K, 1, st);
+    if (mode == EPI_RESID && !a.bias) return launch_gemm_simt(dt, A, W, a.out, M, N, K, 1, st);
     if (mode == EPI_F32) return launch_gemm_simt(dt, A, W, a.out, M, N, K, 0, st);
     int rc = launch_gemm_simt(dt, A, W, m->gemm_c, M, N, K, 0, st);
     if (rc) return rc;
@@ -426,7 +446,7 @@ int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
         // attention sublayer
         {
             prof::Scope ps(st, decode ? "decode_rmsnorm" : "prefill_rmsnorm", nb, 3.0 * n * d);
-            if ((rc = launch_rmsnorm(dt, m->trunk, ly.g_attn, m->xn, n, d, c.norm_eps, st))) return rc;
+            if ((rc = launch_rmsnorm(dt, m->trunk, ly.g_attn, m->xn, n, d, c.norm_eps, st, ly.beta_attn))) return rc;
         }
         EpiArgs qa = base_args(m, n, nq);
         qa.q = m->q;
@@ -434,6 +454,7 @@ int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
         qa.vc = vcache(m, l);
         qa.S = decode ? 1 : S;
         qa.d_pos = decode ? m->d_pos : nullptr;
+        qa.bias = ly.b_qkv;
         if ((rc = project(m, "qkv", EPI_QKV, m->xn, ly.wqkv, n, nq, d, m->splits_qkv, qa, decode, st))) return rc;
         if (decode) {
             double len = 0;   // keys read this step, averaged over the sequences
@@ -457,14 +478,17 @@ int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
         EpiArgs ra = base_args(m, n, d);
         ra.out = m->trunk;
         ra.ld_out = d;
+        ra.bias = ly.b_o;
         if ((rc = project(m, "o", EPI_RESID, m->attn, ly.wo, n, d, d, m->splits_o, ra, decode, st))) return rc;
         // feed-forward sublayer
         {
             prof::Scope ps(st, decode ? "decode_rmsnorm" : "prefill_rmsnorm", nb, 3.0 * n * d);
-            if ((rc = launch_rmsnorm(dt, m->trunk, ly.g_ffn, m->xn, n, d, c.norm_eps, st))) return rc;
+            if ((rc = launch_rmsnorm(dt, m->trunk, ly.g_ffn, m->xn, n, d, c.norm_eps, st, ly.beta_ffn))) return rc;
         }
         EpiArgs sa = base_args(m, n, 2 * h);
         sa.act = m->act;
+        sa.bias = ly.b_gu;
+        ra.bias = ly.b_d;
         if ((rc = project(m, "gateup", EPI_SWIGLU, m->xn, ly.wgu, n, 2 * h, d, m->splits_gu, sa, decode, st))) return rc;
         if ((rc = project(m, "down", EPI_RESID, m->act, ly.wd, n, d, h, m->splits_d, ra, decode, st))) return rc;
     }
@@ -494,6 +518,7 @@ StepArgs step_args(llama_model* m) {
     memset(&a, 0, sizeof(a));
     a.maps = m->step_maps;
     a.gains = m->step_gains;
+    a.biases = m->step_biases;
     a.embed = (const bf16*)m->embed;
     a.kv = (bf16*)m->kv;
     a.kv_layer = m->kv_layer_elems;
@@ -556,6 +581,16 @@ int step_tables(llama_model* m) {
     gains[2 * L] = m->g_final;
     LLAMA_CUDA_TRY(cudaMemcpy(m->step_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
     LLAMA_CUDA_TRY(cudaMemcpy(m->step_gains, gains.data(), gains.size() * sizeof(float*), cudaMemcpyHostToDevice));
+    if (m->step_biases) {
+        std::vector<const float*> bt((size_t)4 * L);
+        for (int l = 0; l < L; ++l) {
+            bt[4 * l + 0] = m->layers[l].c_qkv;
+            bt[4 * l + 1] = m->layers[l].b_o;
+            bt[4 * l + 2] = m->layers[l].c_gu;
+            bt[4 * l + 3] = m->layers[l].b_d;
+        }
+        LLAMA_CUDA_TRY(cudaMemcpy(m->step_biases, bt.data(), bt.size() * sizeof(float*), cudaMemcpyHostToDevice));
+    }
     return LLAMA_OK;
 }
 
@@ -723,6 +758,25 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
         TRY(launch_init_matrix(dt, ly.wd, h, d, d, 0, 0, 0, seed, layer_tid(l, 6), sc, st));
         TRY(launch_fill_f32(ly.g_attn, 1.0f, d, st));
         TRY(launch_fill_f32(ly.g_ffn, 1.0f, d, st));
+        if (cfg->bias) {
+            // vectors of the bias variant: the generator with K = 1 (element j of the vector)
+            auto vec = [&](float* dst, int n, int blk, int blk_stride, int row_off, int k) {
+                return launch_init_matrix(LLAMA_F32, dst, 1, n, blk, blk_stride, row_off, 0, seed, bias_tid(l, k), sc,
+                                          st);
+            };
+            TRY(vec(ly.b_qkv, d, d, 0, 0, 0));
+            TRY(vec(ly.b_qkv, kvd, kvd, 0, d, 1));
+            TRY(vec(ly.b_qkv, kvd, kvd, 0, d + kvd, 2));
+            TRY(vec(ly.b_o, d, d, 0, 0, 3));
+            TRY(vec(ly.b_gu, h, 128, 256, 0, 4));
+            TRY(vec(ly.b_gu, h, 128, 256, 128, 5));
+            TRY(vec(ly.b_d, d, d, 0, 0, 6));
+            TRY(vec(ly.beta_attn, d, d, 0, 0, 7));
+            TRY(vec(ly.beta_ffn, d, d, 0, 0, 8));
+            // decode step: W (g x / rms + beta) + b = W (g x) / rms + (b + W beta)
+            TRY(launch_bias_fold(dt, ly.wqkv, d + 2 * kvd, d, ly.beta_attn, ly.b_qkv, ly.c_qkv, st));
+            TRY(launch_bias_fold(dt, ly.wgu, 2 * h, d, ly.beta_ffn, ly.b_gu, ly.c_gu, st));
+        }
     }
     // RoPE table: angle = pos * theta^(-2i/hd), cos and sin in fp64, stored fp32
     const int hp = cfg->head_dim / 2;

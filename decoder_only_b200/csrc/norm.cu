@@ -40,7 +40,8 @@ constexpr int RMS_MAXV = 8;   // float4 per thread held in registers: d <= 8 * 4
 
 template <typename TO>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ g,
-                                                      TO* __restrict__ y, int d, float eps) {
+                                                      const float* __restrict__ beta, TO* __restrict__ y, int d,
+                                                      float eps) {
     pdl_launch_dependents();
     pdl_wait();
     const int r = blockIdx.x;
@@ -75,14 +76,15 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
         const int i = threadIdx.x + j * blockDim.x;
         if (i < nv) {
             const float4 gg = g4[i];
-            store4<TO>(yr + 4 * i, v[j].x * inv * gg.x, v[j].y * inv * gg.y, v[j].z * inv * gg.z,
-                       v[j].w * inv * gg.w);
+            const float4 bb = beta ? reinterpret_cast<const float4*>(beta)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+            store4<TO>(yr + 4 * i, v[j].x * inv * gg.x + bb.x, v[j].y * inv * gg.y + bb.y,
+                       v[j].z * inv * gg.z + bb.z, v[j].w * inv * gg.w + bb.w);
         }
     }
 }
 
 int launch_rmsnorm(int dtype, const float* x, const float* g, void* y, int rows, int d, float eps,
-                   cudaStream_t st) {
+                   cudaStream_t st, const float* beta) {
     if (rows <= 0) return LLAMA_OK;
     const int nv = d / 4;
     int threads = ((ceil_div(nv, 4) + 31) / 32) * 32;
@@ -90,9 +92,9 @@ int launch_rmsnorm(int dtype, const float* x, const float* g, void* y, int rows,
     if (threads > 256) threads = 256;
     if (nv > RMS_MAXV * threads) return LLAMA_ERR_INVALID_ARG;
     if (dtype == LLAMA_BF16)
-        launch_pdl(rmsnorm_kernel<bf16>, dim3(rows), dim3(threads), 0, st, x, g, (bf16*)y, d, eps);
+        launch_pdl(rmsnorm_kernel<bf16>, dim3(rows), dim3(threads), 0, st, x, g, beta, (bf16*)y, d, eps);
     else
-        launch_pdl(rmsnorm_kernel<float>, dim3(rows), dim3(threads), 0, st, x, g, (float*)y, d, eps);
+        launch_pdl(rmsnorm_kernel<float>, dim3(rows), dim3(threads), 0, st, x, g, beta, (float*)y, d, eps);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
 }

@@ -88,7 +88,8 @@ __global__ void epilogue_from_f32_kernel(const float* __restrict__ C, int ldc, E
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = row[c * 32 + j];
-        epi_qkv32<T>(a, m, c * 32, v);
+        if constexpr (MODE == EPI_RESID) epi_resid32(a, m, c * 32, v);
+        else epi_qkv32<T>(a, m, c * 32, v);
     }
 }
 
@@ -103,6 +104,8 @@ int launch_epilogue_from_f32(int dtype, int mode, const float* C, int ldc, const
     } else if (mode == EPI_QKV) {
         if (dtype == LLAMA_BF16) epilogue_from_f32_kernel<bf16, EPI_QKV><<<blocks, 128, 0, st>>>(C, ldc, a);
         else epilogue_from_f32_kernel<float, EPI_QKV><<<blocks, 128, 0, st>>>(C, ldc, a);
+    } else if (mode == EPI_RESID) {
+        epilogue_from_f32_kernel<float, EPI_RESID><<<blocks, 128, 0, st>>>(C, ldc, a);
     } else {
         return LLAMA_ERR_INVALID_ARG;
     }

@@ -81,6 +81,10 @@ typedef struct llama_config {
     int32_t n_kv_heads;  /* key/value heads (grouped keys and values); 0 => n_heads.
                             n_heads % n_kv_heads == 0; query head h uses key/value
                             head h / (n_heads / n_kv_heads) */
+    int32_t bias;        /* 1: the bias variant -- every linear layer adds a bias of its
+                            output width, each in-layer RMSNorm adds a shift after the
+                            gain (none on the final norm and head); fp32, drawn like
+                            the weights from tensor ids 2^20 + 16 l + k */
 } llama_config;
 
 typedef struct llama_model llama_model; /* opaque host handle */
