@@ -374,6 +374,14 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
     const int n = mb * BM + et;
     float* part = a.partial + a.part_off[w.g.kind];
     const bool direct = (nseg == 1) && !PAIR;
+    // a residual block's trunk values are final once the phase's input is
+    // (the previous residual phase finished before it): read them before the
+    // arrival, off the finishing range's critical path
+    float tv[BN];
+    if constexpr (MODE == EPI_RESID) {
+#pragma unroll
+        for (int b = 0; b < BN; ++b) tv[b] = (b < M) ? __ldcg(a.trunk + (size_t)b * a.d + n) : 0.f;
+    }
     if (!direct) {
         float* dst = part + ((size_t)n * ns + ((int)blockIdx.x - first_of(mb))) * Mp;
 #pragma unroll
@@ -436,7 +444,7 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
             for (int b = 0; b < BN; ++b)
                 if (b < M) {
                     float* o = a.trunk + (size_t)b * a.d + n;
-                    const float x = __ldcg(o) + sum[b] + bn;
+                    const float x = tv[b] + sum[b] + bn;
                     *o = x;
                     xg[(size_t)b * a.d + n] = __float2bfloat16_rn(x * gn);
                     sm.xbuf[b * XLD + et] = x * x;
