@@ -377,10 +377,13 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
     // a residual block's trunk values are final once the phase's input is
     // (the previous residual phase finished before it): read them before the
     // arrival, off the finishing range's critical path
-    float tv[BN];
+    float tv[BN], gn = 0.f, bn = 0.f;
     if constexpr (MODE == EPI_RESID) {
 #pragma unroll
         for (int b = 0; b < BN; ++b) tv[b] = (b < M) ? __ldcg(a.trunk + (size_t)b * a.d + n) : 0.f;
+        // and the next norm's gain, the projection's bias (b_o / b_d) of this column
+        gn = (type == PH_O ? a.gains[2 * l + 1] : a.gains[2 * (l + 1)])[n];
+        bn = a.biases ? a.biases[4 * l + (type == PH_O ? 1 : 3)][n] : 0.f;
     }
     if (!direct) {
         float* dst = part + ((size_t)n * ns + ((int)blockIdx.x - first_of(mb))) * Mp;
@@ -437,8 +440,6 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
             // trunk += the block's sum; then the next norm's inputs: bf16(g * x)
             // and the block's sum of squares per row
             const bool to_ffn = (type == PH_O);
-            const float gn = (to_ffn ? a.gains[2 * l + 1] : a.gains[2 * (l + 1)])[n];
-            const float bn = a.biases ? a.biases[4 * l + (to_ffn ? 1 : 3)][n] : 0.f;   // b_o / b_d
             bf16* xg = to_ffn ? a.xg2 : a.xg;
 #pragma unroll
             for (int b = 0; b < BN; ++b)
