@@ -174,20 +174,44 @@ TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "decode_step_llama7b_2layer_dra
 STEP_SOURCE = os.path.join(ROOT, "decoder_only_b200", "csrc", "decode_step.cu")
 
 
+def code_hash(path: str) -> str:
+    """sha256 (16 hex digits) of a C++/CUDA source with its comments and
+    whitespace removed: it changes when the code does, not its comments."""
+    import hashlib
+    with open(path) as f:
+        src = f.read()
+    out, i, n = [], 0, len(src)
+    while i < n:
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif src[i] == '"':                      # string literal: kept as is
+            j = i + 1
+            while j < n and src[j] != '"':
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(src[i])
+            i += 1
+    return hashlib.sha256("".join("".join(out).split()).encode()).hexdigest()[:16]
+
+
 def decode_step_traffic_ratio():
     """DRAM traffic / algorithmic bytes of the fused decode step from the
-    committed ncu summary, or None when the kernel source has changed since
+    committed ncu summary, or None when the kernel's code has changed since
     the counters were taken."""
-    import hashlib
     try:
         with open(TRAFFIC_PROFILE) as f:
             txt = f.read()
-        with open(STEP_SOURCE, "rb") as f:
-            h = hashlib.sha256(f.read()).hexdigest()[:16]
+        h = code_hash(STEP_SOURCE)
     except OSError:
         return None
     ratio = re.search(r"traffic_ratio:\s*([0-9.]+)", txt)
-    src = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", txt)
+    src = re.search(r"kernel_code_sha256_16:\s*([0-9a-f]+)", txt)
     if not ratio or not src or src.group(1) != h:
         return None
     return float(ratio.group(1))

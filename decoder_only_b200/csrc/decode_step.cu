@@ -5,19 +5,21 @@
 // Was Not an Original LLaMA Feature")) is a chain of small, HBM-bound
 // phases:
 //   embed (+ the first norm's inputs)
-//   per layer:  QKV projection (+RoPE, append K and V at the position)
+//   per layer:  QKV projection (+RoPE, append K and V at each sequence's position)
 //               attention over the cache
 //               O projection (+residual, + the FFN norm's inputs)
 //               gate/up projection (+SwiGLU)
 //               down projection (+residual, + the next norm's inputs)
-//   head projection (fp32 logits), greedy argmax, position + 1.
+//   head projection (fp32 logits), greedy argmax, positions + 1.
 // Launched one kernel per phase, fixed costs dominate (launch, set-up,
 // pipeline fill, tails).  Here one cooperative launch of one CTA per SM runs
-// all phases, separated by a grid-wide barrier; the weights -- which do not
-// depend on any phase -- stream continuously: the TMA producer keeps its
-// ring of weight tiles full across phase boundaries, and only the
-// activation tile of each stage waits for the barrier that makes that
-// activation visible.
+// all phases.  Phases are ordered by completion counts, not grid barriers:
+// every unit of work that a later phase reads (a finished 128-row block of a
+// projection, a finished attention pair) adds one to a count per (layer,
+// kind), and a consumer waits only for the count it depends on.  The
+// weights -- which depend on no phase -- stream continuously: the TMA
+// producer keeps its ring of weight tiles full across phase boundaries, and
+// only the activation tile of each stage waits for its phase's input.
 //
 // Work split of a projection: its (128-row block, 64-wide k-block)
 // iterations, block-major, are cut into gridDim.x equal contiguous ranges
@@ -33,18 +35,19 @@
 // bf16(g * x) and the block's sum of squares; the projection consuming the
 // norm multiplies its fp32 result by rsqrt(sum of the block sums / d + eps),
 // the block sums added in a fixed order.  No phase waits on a separate
-// normalisation pass over the whole trunk.
+// normalisation pass over the whole trunk.  (The bias variant's norm shift
+// beta enters the same way: W beta is folded into that projection's bias.)
 //
-// Warp roles (192 threads):
-//   warp 0     TMA producer, all projections of the step in order
-//   warp 1     TMEM owner and tcgen05.mma issuer (swap-AB: 128 weight rows on
+// Warp roles (256 threads):
+//   warps 0-3  projection epilogues, attention, greedy choice
+//   warp 4     TMA producer, all projections of the step in order
+//   warp 5     TMEM owner and tcgen05.mma issuer (swap-AB: 128 weight rows on
 //              the TMEM lanes, the B <= 32 tokens as N = 16 or 32 columns)
-//   warps 2-5  everything else: projection epilogues, attention, greedy
-//              choice, and the arrivals at the grid barrier.
+//   warps 6-7  attention
 // Every wait is bounded (2 s): a CTA that gives up records
-// LLAMA_DEVERR_TIMEOUT and leaves; the others then give up at the next grid
-// barrier.  Named barriers among the 128 epilogue threads follow a
-// collective OR of each thread's wait result, so they leave together.
+// LLAMA_DEVERR_TIMEOUT and leaves; the others then give up at their own next
+// wait.  Named barriers among the 128 epilogue threads follow a collective
+// OR of each thread's wait result, so they leave together.
 #include <cuda.h>
 
 #include <algorithm>
@@ -1201,9 +1204,10 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
     } else {
         // -------------------------------------------------------- attention warps 6, 7
         // They join the epilogue warps in each attention phase: wait for the
-        // barrier that opens it, take their share, and arrive at the named
-        // barrier the epilogue warps pass before they leave the phase (once
-        // per layer, also after a failure, so that nobody waits for them).
+        // QKV completion count that opens it, take their share, and arrive at
+        // the named barrier the epilogue warps pass before they leave the
+        // phase (once per layer, also after a failure, so that nobody waits
+        // for them).
         uint32_t uses[2] = {0u, 0u};
         int w = 1;
         if (lane == 0) w = wait_at_least(a.bar + SY_EMBED, E, abort_flag, a.err);
