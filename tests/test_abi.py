@@ -61,3 +61,55 @@ def test_bf16_batch_limit_and_tiny_fp32_accepted():
     assert lb.lib.llama_model_bytes(ctypes.byref(lb.make_config(LLAMA_7B, 33, 64)),
                                     ctypes.byref(ctypes.c_uint64())) == -1
     assert lb.model_bytes(lb.make_config(TINY, 1, 32)) > 0
+
+
+def _bytes(shape, B=4, S=128):
+    n = ctypes.c_uint64()
+    rc = lb.lib.llama_model_bytes(ctypes.byref(lb.make_config(shape, B, S)), ctypes.byref(n))
+    return rc, n.value
+
+
+def test_grouped_kv_heads_shrink_the_projection_and_the_cache_exactly():
+    """n_kv key/value heads: W_k and W_v lose 2 d (H - n_kv) hd values per
+    layer and the cache 2 L B S (H - n_kv) hd (the [NAR] KV-cache formula)."""
+    s = LLAMA_7B.with_(n_layers=2)
+    B, S = 4, 128
+    rc, full = _bytes(s, B, S)
+    rc8, gqa = _bytes(s.with_(n_kv_heads=8), B, S)
+    assert rc == rc8 == 0
+    hd, H, L, d = s.head_dim, s.n_heads, s.n_layers, s.d_model
+    saved = 2 * (L * 2 * d * (H - 8) * hd + 2 * L * B * S * (H - 8) * hd)   # bf16 bytes
+    # beyond that only the decode step's split-K partials of the narrower QKV
+    # projection change (fp32, [rows][slots][B]), plus 256-byte alignment
+    qkv_partials = 4 * 3 * d * 8 * B
+    assert saved - 256 * 64 <= full - gqa <= saved + qkv_partials
+
+
+@pytest.mark.parametrize("n_kv", [3, -1, 64])
+def test_grouped_kv_heads_must_divide_the_query_heads(n_kv):
+    assert _bytes(LLAMA_7B.with_(n_layers=1, n_kv_heads=n_kv))[0] == -1
+
+
+def test_bias_variant_adds_its_vectors():
+    """Per layer: b_qkv, b_o, b_gu, b_d, two shifts, and the decode step's two
+    folded biases, fp32 (the page's +1,622,016 values for 7B plus the folds)."""
+    s = LLAMA_7B.with_(n_layers=2)
+    rc0, plain = _bytes(s)
+    rc1, biased = _bytes(s.with_(bias=True))
+    assert rc0 == rc1 == 0
+    d, h, L = s.d_model, s.ffn_hidden, s.n_layers
+    per_layer = (3 * d + d + 2 * h + d + 2 * d) + (3 * d + 2 * h)
+    assert biased - plain >= 4 * L * per_layer
+    assert biased - plain < 4 * L * per_layer + 256 * 16 * L + 4096
+
+
+def test_code_hash_ignores_comments_not_code(tmp_path):
+    import bench
+    a = tmp_path / "a.cu"
+    a.write_text('int f(int x) {  // twice\n  return 2 * x; /* doubled */ }\nconst char* s = "// kept";\n')
+    b = tmp_path / "b.cu"
+    b.write_text('int f(int x) {\n  return 2 * x;\n}\nconst char* s = "// kept";  // other words\n')
+    c = tmp_path / "c.cu"
+    c.write_text('int f(int x) {\n  return 3 * x;\n}\nconst char* s = "// kept";\n')
+    assert bench.code_hash(str(a)) == bench.code_hash(str(b))
+    assert bench.code_hash(str(a)) != bench.code_hash(str(c))
