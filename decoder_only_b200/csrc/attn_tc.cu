@@ -8,8 +8,10 @@
 // knowledge note credits to the xFormers attention of the training system.
 //
 // One CTA per (128-query tile, head, sequence), longest tiles first.
-//   warp 0      TMA: Q once, then K_j and V_j tiles (2-stage ring).  3-D
-//               tensor maps (hd, position, head) make rows >= S read as 0.
+//   warp 0      TMA: lane 0 Q once, then the K_j tiles; lane 1 the V_j
+//               tiles (2-stage rings; K_j is free once S_j is computed, V_j
+//               once O_j is, so K runs ahead of V).  3-D tensor maps (hd,
+//               position, head) make rows >= S read as 0.
 //   warp 1      TMEM allocator + MMA issuer:
 //                 S_j = Q K_j^T   (M 128, N 128, K hd)  -> TMEM S[j % 2]
 //                 O_j = P_j V_j   (M 128, N hd, K 128)  -> TMEM O[j % 2]
@@ -74,12 +76,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t q_full = bars;
     const uint32_t k_full = bars + 8;        // [2]
     const uint32_t v_full = bars + 24;       // [2]
-    const uint32_t kv_empty = bars + 40;     // [2]
+    const uint32_t k_empty = bars + 40;      // [2]
     const uint32_t s_full = bars + 56;       // [2]
     const uint32_t s_empty = bars + 72;      // [2]
     const uint32_t p_full = bars + 88;       // [2]
     const uint32_t o_full = bars + 104;      // [2]
     const uint32_t o_empty = bars + 120;     // [2]
+    const uint32_t v_empty = bars + 136;     // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 160);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -97,7 +100,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(k_full + 8 * i, 1);
             mbar_init(v_full + 8 * i, 1);
-            mbar_init(kv_empty + 8 * i, 1);
+            mbar_init(k_empty + 8 * i, 1);
+            mbar_init(v_empty + 8 * i, 1);
             mbar_init(s_full + 8 * i, 1);
             mbar_init(s_empty + 8 * i, 128);
             mbar_init(p_full + 8 * i, 128);
@@ -121,35 +125,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
-        if (lane == 0) {
+        if (lane < 2) {
+            // lane 0: Q, then K_j; lane 1: V_j
+            const bool is_k = (lane == 0);
+            const uint32_t full = is_k ? k_full : v_full, empty = is_k ? k_empty : v_empty;
+            const uint32_t dst = is_k ? sK : sV;
+            const CUtensorMap* map = is_k ? &tmK : &tmV;
             bool ok = true;
-            mbar_expect_tx(q_full, C::TILE);
-            for (int r = 0; r < C::NREG; ++r) tma_load_3d(sQ + r * C::REG, &tmQ, q_full, 64 * r, q0, head);
+            if (is_k) {
+                mbar_expect_tx(q_full, C::TILE);
+                for (int r = 0; r < C::NREG; ++r) tma_load_3d(sQ + r * C::REG, &tmQ, q_full, 64 * r, q0, head);
+            }
             int issued = 0;
             for (int j = 0; j < n_kv && ok; ++j) {
                 const int st = j & 1;
-                if (!mbar_wait(kv_empty + 8 * st, ((j >> 1) & 1) ^ 1u, abort_flag, err)) {
+                if (!mbar_wait(empty + 8 * st, ((j >> 1) & 1) ^ 1u, abort_flag, err)) {
                     ok = false;
                     break;
                 }
-                mbar_expect_tx(k_full + 8 * st, C::TILE);
+                mbar_expect_tx(full + 8 * st, C::TILE);
                 for (int r = 0; r < C::NREG; ++r)
-                    tma_load_3d(sK + st * C::TILE + r * C::REG, &tmK, k_full + 8 * st, 64 * r, j * BKV, kv_head);
-                mbar_expect_tx(v_full + 8 * st, C::TILE);
-                for (int r = 0; r < C::NREG; ++r)
-                    tma_load_3d(sV + st * C::TILE + r * C::REG, &tmV, v_full + 8 * st, 64 * r, j * BKV, kv_head);
+                    tma_load_3d(dst + st * C::TILE + r * C::REG, map, full + 8 * st, 64 * r, j * BKV, kv_head);
                 issued = j + 1;
             }
             if (!ok) {
                 // drain (bounded) the copies this thread issued
                 const uint64_t t0 = global_timer();
-                while (!mbar_try_wait(q_full, 0) && global_timer() - t0 < WAIT_LIMIT_NS / 4) {
+                while (is_k && !mbar_try_wait(q_full, 0) && global_timer() - t0 < WAIT_LIMIT_NS / 4) {
                 }
                 for (int j = issued > 2 ? issued - 2 : 0; j < issued; ++j) {
-                    const int st = j & 1;
                     const uint32_t par = (j >> 1) & 1;
-                    while (!(mbar_try_wait(k_full + 8 * st, par) && mbar_try_wait(v_full + 8 * st, par)) &&
-                           global_timer() - t0 < WAIT_LIMIT_NS / 2) {
+                    while (!mbar_try_wait(full + 8 * (j & 1), par) && global_timer() - t0 < WAIT_LIMIT_NS / 2) {
                     }
                 }
             }
@@ -179,6 +185,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                   kk > 0 ? 1u : 0u);
                     }
                     umma_commit(s_full + 8 * st);
+                    umma_commit(k_empty + 8 * st);
                 }
                 if (j > 0) {
                     const int jj = j - 1, st = jj & 1;
@@ -200,7 +207,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         umma_bf16(d_o, sw128_desc(sP + st * C::P_TILE + poff), vd, IDESC_PV, kk > 0 ? 1u : 0u);
                     }
                     umma_commit(o_full + 8 * st);
-                    umma_commit(kv_empty + 8 * st);
+                    umma_commit(v_empty + 8 * st);
                 }
             }
         }
@@ -226,42 +233,50 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t s_addr = tmem + lane_addr + (uint32_t)(st * 128);
+                // only the diagonal tile masks: there key k is visible iff
+                // k <= min(q, S - 1) (a select per score, no branch)
                 const bool diag = (j == n_kv - 1);
-                const int k0 = j * BKV;
-                // pass 1: row maximum over the visible keys
-                float mx = -INFINITY;
+                const int lim = min(q, S - 1) - j * BKV;
+                // pass 1: row maximum, eight independent partial maxima
+                float mx8[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     float sv[32];
                     tmem_ld32(s_addr + c * 32, sv);
+                    if (diag) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int key = k0 + c * 32 + i;
-                        const bool vis = !diag || (key <= q && key < S);
-                        mx = fmaxf(mx, vis ? sv[i] : -INFINITY);
+                        for (int i = 0; i < 32; ++i) sv[i] = (c * 32 + i <= lim) ? sv[i] : -INFINITY;
                     }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
                 }
+                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
                 const float m_new = fmaxf(m, mx);
                 corr = (m == -INFINITY) ? 0.f : exp2f((m - m_new) * scale_log2);
                 const float mo = m_new * scale_log2;
-                // pass 2: probabilities (bf16) into the P tile, row sum from the rounded values
-                float rs = 0.f;
+                // pass 2: probabilities (bf16) into the P tile, row sum of the
+                // rounded values in four independent partial sums
+                float rs4[4] = {0.f, 0.f, 0.f, 0.f};
                 const uint32_t pbase = sP + st * C::P_TILE;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     float sv[32];
                     tmem_ld32(s_addr + c * 32, sv);
+                    if (diag) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) sv[i] = (c * 32 + i <= lim) ? sv[i] : -INFINITY;
+                    }
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const int key = k0 + c * 32 + 2 * i;
-                        const bool v0 = !diag || (key <= q && key < S);
-                        const bool v1 = !diag || (key + 1 <= q && key + 1 < S);
-                        const float p0 = v0 ? exp2f(fmaf(sv[2 * i], scale_log2, -mo)) : 0.f;
-                        const float p1 = v1 ? exp2f(fmaf(sv[2 * i + 1], scale_log2, -mo)) : 0.f;
+                        const float p0 = exp2f(fmaf(sv[2 * i], scale_log2, -mo));
+                        const float p1 = exp2f(fmaf(sv[2 * i + 1], scale_log2, -mo));
                         pk[i] = pack_bf16x2(p0, p1);
                         const float2 r = unpack_bf16x2(pk[i]);
-                        rs += r.x + r.y;
+                        rs4[i & 3] += r.x + r.y;
                     }
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
@@ -271,6 +286,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                      : "memory");
                     }
                 }
+                const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
                 tc_fence_before();
                 mbar_arrive(s_empty + 8 * st);
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
