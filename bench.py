@@ -496,6 +496,88 @@ def run_b200(args, wl, shape):
         dist.destroy_process_group()
 
 
+# ----------------------------------------------------------------------------- per-kernel sweep
+
+# (batch, sequence length) points of the per-kernel prefill sweep at the 65B
+# widths: seq in {512, 1024, 2048} x batch in {1, 8}
+SWEEP_POINTS = [(b, s) for b in (1, 8) for s in (512, 1024, 2048)]
+
+
+def sweep_table(prof, peaks):
+    """Per kernel family of one profiled prefill: device time, launches, and
+    the achieved rate against the measured peak that bounds it (tensor
+    FLOP/s for the projections and attention, HBM bytes/s for the rest)."""
+    fam = {}
+    for name, e in prof.items():
+        f = fam.setdefault(kernel_family(name), dict(ms=0.0, flops=0.0, bytes=0.0, launches=0))
+        f["ms"] += e["ms"]
+        f["flops"] += e["flops"]
+        f["bytes"] += e["bytes"]
+        f["launches"] += e["launches"]
+    out = {}
+    for k, f in sorted(fam.items(), key=lambda kv: -kv[1]["ms"]):
+        r = dict(ms=round(f["ms"], 3), launches=f["launches"])
+        if f["ms"] > 0 and f["flops"] > 0 and (k.startswith("gemm_tc prefill") or k == "prefill_attention"):
+            t = f["flops"] / (f["ms"] * 1e-3) / 1e12
+            r.update(tflops=round(t, 1), frac_bf16=round(t / peaks["bf16_tflops"], 4))
+        elif f["ms"] > 0 and f["bytes"] > 0:
+            g = f["bytes"] / (f["ms"] * 1e-3) / 1e9
+            r.update(gbs=round(g, 1), frac_hbm=round(g / peaks["hbm_gbs"], 4))
+        out[k] = r
+    return out
+
+
+def run_sweep(args, wl, shape):
+    """Prefill of every SWEEP_POINTS (batch, length) on one model: whole-
+    prefill time (CUDA events over --steps runs after --warmup) and one
+    profiled prefill split per kernel family.  One JSON line."""
+    import torch
+
+    import decoder_only_b200 as lb
+    import synth
+
+    torch.cuda.set_device(0)
+    bmax = max(b for b, _ in SWEEP_POINTS)
+    smax = max(s for _, s in SWEEP_POINTS)
+    model = lb.Model(shape, max_batch=bmax, max_seq=smax, seed=synth.workloads.SEED)
+    peaks, peak_src = load_peaks()
+    st = torch.cuda.current_stream()
+    points = []
+    for B, S in SWEEP_POINTS:
+        tok = torch.from_numpy(synth.tokens(synth.workloads.SEED, B * S, shape.vocab).reshape(B, S)).cuda()
+        logits = torch.empty(B, S, shape.vocab, dtype=torch.float32, device="cuda")
+        for _ in range(args.warmup):
+            model.prefill(tok, out=logits)
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(st)
+        for _ in range(args.steps):
+            model.prefill(tok, out=logits)
+        ev[1].record(st)
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[1]) / args.steps
+        lb.profile_reset()
+        lb.profile_enable(True)
+        model.prefill(tok, out=logits)
+        torch.cuda.synchronize()
+        prof = lb.profile_read()
+        lb.profile_enable(False)
+        flops, _ = algorithmic_work(shape, B, S, 0)
+        tf = flops / (ms * 1e-3) / 1e12
+        points.append(dict(batch=B, seq=S, prefill_ms=round(ms, 3), tokens_per_s=round(B * S / (ms * 1e-3), 1),
+                           tflops=round(tf, 1), frac_bf16=round(tf / peaks["bf16_tflops_sustained"], 4),
+                           kernels=sweep_table(prof, peaks)))
+        del logits
+    grid = "batch {%s} x length {%s}" % (", ".join(str(b) for b in sorted({b for b, _ in SWEEP_POINTS})),
+                                        ", ".join(str(s) for s in sorted({s for _, s in SWEEP_POINTS})))
+    print(json.dumps(dict(metric="per-kernel prefill sweep", unit="ms / TFLOP/s / GB/s",
+                          workload=wl["desc"].split(":")[0] + ": prefill at every point of " + grid,
+                          model=shape.name, steps=args.steps, warmup=args.warmup, peak_source=peak_src,
+                          data="synthetic (seeded token ids; random-init weights N(0, 0.02^2) drawn on device)",
+                          points=points)), flush=True)
+    model.close()
+
+
 def summarize_ncu(path):
     """Per-kernel launches, total device time and share from an ncu
     `--metrics gpu__time_duration.sum --csv` launch list."""
@@ -532,7 +614,11 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--workload", default="7b", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=sorted(WORKLOADS),
+                    help="default: 7b (65b-slice with --sweep)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="per-kernel prefill sweep over batch {1, 8} x length {512, 1024, 2048} "
+                         "(one JSON line; 1 GPU)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu", action="store_true",
                     help="only the warm-up and timed steps, each timed step in an NVTX range 'timed_step' "
@@ -546,11 +632,16 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from synth import workloads as wls
-    wl = dict(WORKLOADS[args.workload], name=args.workload)
+    name = args.workload or ("65b-slice" if args.sweep else "7b")
+    wl = dict(WORKLOADS[name], name=name)
     shape = getattr(wls, wl["model"])
     if "layers" in wl:
         shape = shape.with_(n_layers=wl["layers"], name=f"{shape.name}-{wl['layers']}layer")
-    if args.impl == "reference":
+    if args.sweep:
+        if args.impl == "reference" or int(os.environ.get("WORLD_SIZE", "1")) > 1:
+            ap.error("--sweep times this library on one GPU")
+        run_sweep(args, wl, shape)
+    elif args.impl == "reference":
         run_reference(args, wl, shape)
     else:
         run_b200(args, wl, shape)
