@@ -121,6 +121,8 @@ def _qkv(B, H, S, hd, kv_stride, dtype):
 @pytest.mark.parametrize("B,H,S,hd,dtype", [
     (1, 2, 1, 32, torch.float32), (1, 4, 37, 32, torch.float32), (2, 3, 130, 64, torch.float32),
     (1, 2, 200, 128, torch.bfloat16), (2, 2, 64, 64, torch.bfloat16),
+    # a single key; one valid row in the last query tile; a ragged tail at head_dim 64
+    (1, 2, 1, 128, torch.bfloat16), (1, 3, 129, 128, torch.bfloat16), (2, 2, 257, 64, torch.bfloat16),
 ])
 def test_attention_prefill(B, H, S, hd, dtype):
     kv_stride = S + 5
