@@ -38,7 +38,7 @@ class LlamaConfig(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built; run `python -m decoder_only_b200.build`")
+        raise ImportError(f"{LIB_PATH} is not built; run `python decoder_only_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, U64, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_float
     sig = {
@@ -178,8 +178,9 @@ class Model:
 
     def positions(self):
         """Each sequence's decode position (host ints)."""
-        buf = (ctypes.c_int32 * 64)()
-        n = lib.llama_positions(self.h, ctypes.cast(buf, ctypes.c_void_p), 64)
+        cap = max(int(self.cfg.max_batch), 1)
+        buf = (ctypes.c_int32 * cap)()
+        n = lib.llama_positions(self.h, ctypes.cast(buf, ctypes.c_void_p), cap)
         _check(min(n, 0), "llama_positions")
         return [buf[i] for i in range(n)]
 
