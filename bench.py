@@ -217,8 +217,20 @@ def decode_step_traffic_ratio():
     return float(ratio.group(1))
 
 
-def roofline(prof, decode_scale, peaks, peak_src):
-    """Dominant kernel over one step from the live per-region timing."""
+def roofline(prof, decode_scale, peaks, peak_src, graph_decode_ms=None, decode_steps=0, step_ms=None,
+             decode_bytes_per_step=None):
+    """Dominant kernel over one step.
+
+    Prefill kernels: the live per-region timing of one profiled (eager)
+    prefill.  The fused decode step (one kernel per step, replayed from a
+    CUDA graph in the timed region): with `graph_decode_ms` (the timed
+    steps' decode time, CUDA events around the graph replays) its time per
+    launch is graph_decode_ms / decode_steps and its algorithmic bytes per
+    launch `decode_bytes_per_step` (weights once + the K and V rows at the
+    mean cache length of the timed steps); the eager, stamped profiled steps
+    give only the other kernels' shares.  The block is
+    refused (returned as an error note) when the per-kernel times add up to
+    more than the timed step `step_ms`."""
     fam = {}
     for name, e in prof.items():
         scale = decode_scale if name.startswith("decode") else 1.0
@@ -228,7 +240,18 @@ def roofline(prof, decode_scale, peaks, peak_src):
         f["flops"] += e["flops"]
         f["launches"] += e["launches"]
         f["step_ms"] += e["ms"] * scale
+    timing = "eager per-region CUDA events (one profiled prefill)"
+    if graph_decode_ms is not None and "decode_step" in fam and decode_steps:
+        f = fam["decode_step"]
+        per = max(f["launches"], 1)
+        f["bytes"] = (decode_bytes_per_step if decode_bytes_per_step else f["bytes"] / per) * decode_steps
+        f["flops"] = f["flops"] / per * decode_steps
+        f["ms"], f["launches"], f["step_ms"] = graph_decode_ms, decode_steps, graph_decode_ms
+        timing += "; decode_step: CUDA events around the timed steps' graph replays"
     total = sum(f["step_ms"] for f in fam.values())
+    if step_ms is not None and total > 1.02 * step_ms:
+        return dict(error=f"per-kernel times add up to {total:.2f} ms, more than the timed step "
+                          f"({step_ms:.2f} ms): not reported")
     name, f = max(fam.items(), key=lambda kv: kv[1]["step_ms"])
     per_launch_ms = f["ms"] / max(f["launches"], 1)
     if name.startswith("gemm_tc prefill") or name == "prefill_attention":
@@ -245,7 +268,7 @@ def roofline(prof, decode_scale, peaks, peak_src):
         if r is not None:   # bytes per launch: measured ratio x this launch's algorithmic bytes
             traffic = round(r * f["bytes"] / max(f["launches"], 1))
     out.update(kernel=name, achieved=round(achieved, 1), peak=peak, frac=round(achieved / peak, 4),
-               peak_source=peak_src, traffic=traffic, launches_profiled=f["launches"],
+               peak_source=peak_src, traffic=traffic, timing=timing, launches_timed=f["launches"],
                avg_launch_us=round(per_launch_ms * 1e3, 2), share_of_step=round(f["step_ms"] / total, 4),
                shares={k: round(v["step_ms"] / total, 4) for k, v in sorted(fam.items(), key=lambda kv: -kv[1]["step_ms"])},
                est_ms_per_step={k: round(v["step_ms"], 2) for k, v in sorted(fam.items(), key=lambda kv: -kv[1]["step_ms"])})
@@ -390,40 +413,46 @@ def run_b200(args, wl, shape):
         return
 
     # ------------------------------------------------ timed region (device events)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    # events on the launching stream: one before the first step, and per step
+    # one after its prefill and one after its decode steps (graph replays),
+    # so that the prefill / decode split comes from the timed steps themselves
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev_mid = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def timed_step(i):
+        if decode_only:
+            model.rewind(S)
+            ev_mid[i].record(st)
+            model.generate(first, steps, out=gen)
+        else:
+            model.prefill(tok_dev, out=logits)
+            ev_mid[i].record(st)
+            if steps:
+                model.generate(None, steps, out=gen, batch=B)
+        ev_end[i].record(st)
+
     barrier()
     torch.cuda.synchronize()
     l0 = lb.kernel_launches()
     with ClockSampler(local) as clk:
-        ev[0].record(st)
-        for _ in range(args.steps):
-            step()
-        ev[1].record(st)
+        ev0.record(st)
+        for i in range(args.steps):
+            timed_step(i)
         torch.cuda.synchronize()
     barrier()
     launches = lb.kernel_launches() - l0
-    ms = max_over_ranks(ev[0].elapsed_time(ev[1]), world, "cuda")
+    ms = max_over_ranks(ev0.elapsed_time(ev_end[-1]), world, "cuda")
     clocks = clk.summary()
     tokens_step = (0 if decode_only else B * S) + B * steps
     value = replica_throughput(world, tokens_step, args.steps, ms)
 
-    # ------------------------------------------------ prefill / decode split
-    split = {}
-    if not decode_only:
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        pre, dec = [], []
-        for _ in range(2):
-            e[0].record(st)
-            model.prefill(tok_dev, out=logits)
-            e[1].record(st)
-            if steps:
-                model.generate(None, steps, out=gen, batch=B)
-            e[2].record(st)
-            torch.cuda.synchronize()
-            pre.append(e[0].elapsed_time(e[1]))
-            dec.append(e[1].elapsed_time(e[2]))
-        split["prefill_ms"] = min(pre)
-        split["decode_ms"] = min(dec) if steps else 0.0
+    # ------------------------------------------------ prefill / decode split (same events)
+    starts = [ev0] + ev_end[:-1]
+    pre = [a.elapsed_time(b) for a, b in zip(starts, ev_mid)]
+    dec = [a.elapsed_time(b) for a, b in zip(ev_mid, ev_end)]
+    split = dict(prefill_ms=0.0 if decode_only else statistics.median(pre),
+                 decode_ms=statistics.median(dec) if steps else 0.0)
 
     # ------------------------------------------------ end to end from host buffers
     out_host = torch.empty(max(steps, 1), B, dtype=torch.int32).pin_memory()
@@ -457,13 +486,15 @@ def run_b200(args, wl, shape):
     torch.cuda.synchronize()
     prof = lb.profile_read()
     lb.profile_enable(False)
-    roof = roofline(prof, steps / max(prof_steps, 1), peaks, peak_src)
+    flops_pre, bytes_dec = algorithmic_work(shape, B, S, steps)
+    roof = roofline(prof, steps / max(prof_steps, 1), peaks, peak_src,
+                    graph_decode_ms=split["decode_ms"] if steps and shape.dtype == "bf16" else None,
+                    decode_steps=steps, step_ms=ms / args.steps, decode_bytes_per_step=bytes_dec)
     phases = None
     if shape.dtype == "bf16" and steps:
         phases = step_phases(model.step_timeline(), shape.n_layers)
 
     if rank == 0:
-        flops_pre, bytes_dec = algorithmic_work(shape, B, S, steps)
         line = dict(
             metric=METRIC, value=round(value, 2), unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
             ms_per_step=round(ms / args.steps, 3), higher_is_better=True, scaling="weak", vs_baseline=None,
@@ -472,16 +503,17 @@ def run_b200(args, wl, shape):
                         decode_steps=steps, parallelism=f"replicas x{world}" if world > 1 else "single GPU",
                         l2="inputs larger than L2: every step streams all weights (13+ GB) from HBM"),
             gpu_launches=launches, clocks=clocks, roofline=roof)
-        if split:
-            pre_s, dec_s = split["prefill_ms"] * 1e-3, split["decode_ms"] * 1e-3
+        if split["prefill_ms"] > 0:
+            pre_s = split["prefill_ms"] * 1e-3
             line["prefill"] = dict(tokens_per_s=round(B * S / pre_s, 1), ms=round(split["prefill_ms"], 3),
                                    tflops=round(flops_pre / pre_s / 1e12, 1),
                                    frac_bf16=round(flops_pre / pre_s / 1e12 / peaks["bf16_tflops_sustained"], 4))
-            if steps:
-                line["decode"] = dict(tokens_per_s=round(B * steps / dec_s, 1),
-                                      ms_per_step=round(split["decode_ms"] / steps, 4),
-                                      gbs=round(bytes_dec * steps / dec_s / 1e9, 1),
-                                      frac_hbm=round(bytes_dec * steps / dec_s / 1e9 / peaks["hbm_gbs"], 4))
+        if steps:
+            dec_s = split["decode_ms"] * 1e-3
+            line["decode"] = dict(tokens_per_s=round(B * steps / dec_s, 1),
+                                  ms_per_step=round(split["decode_ms"] / steps, 4),
+                                  gbs=round(bytes_dec * steps / dec_s / 1e9, 1),
+                                  frac_hbm=round(bytes_dec * steps / dec_s / 1e9 / peaks["hbm_gbs"], 4))
         if phases:
             line["decode_step_phases_us"] = phases
         if e2e_ms is not None:

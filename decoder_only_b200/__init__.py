@@ -62,6 +62,7 @@ def _load():
         "llama_op_attention_decode_work_bytes": [I, I, I, I],
         "llama_op_attention_decode_noalloc": [I, P, P, P, P, I, I, I, I, I, P],
         "llama_op_argmax": [P, I, I, P, P],
+        "llama_op_last_error": [],
         "llama_rewind": [P, I, P],
         "llama_complete": [P, P, I, I, P, I, P, P],
         "llama_kernel_launches": [],
@@ -334,6 +335,12 @@ def attention_decode_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, 
                                                  _ptr(v.contiguous()), _ptr(o), B, H, length, hd, kv_stride,
                                                  _stream()), "llama_op_attention_decode_noalloc")
     return o
+
+
+def op_last_error() -> int:
+    """Reads and clears the single ops' device error word (synchronises the
+    current device): 0, or -4 when a bounded device wait expired."""
+    return int(lib.llama_op_last_error())
 
 
 def argmax(logits: torch.Tensor) -> torch.Tensor:

@@ -369,13 +369,12 @@ int make_head_map(CUtensorMap* map, const void* ptr, int hd, int rows, int strid
 
 template <int HD>
 int attn_attr() {
-    static bool done = false;
-    if (!done) {
+    static PerDeviceOnce once;
+    return once_per_device(once, []() -> int {
         LLAMA_CUDA_TRY(cudaFuncSetAttribute(attn_prefill_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             ACfg<HD>::SMEM));
-        done = true;
-    }
-    return LLAMA_OK;
+        return (int)LLAMA_OK;
+    });
 }
 
 }  // namespace

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "llama_b200.h"
 
 typedef __nv_bfloat16 bf16;
@@ -85,6 +87,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
     __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&w);
     return __bfloat1622float2(v);
+}
+
+// One-time set-up that acts on the current device only (a kernel's
+// shared-memory attribute, the address of a __device__ variable): f runs
+// once per device, under a lock, with that device current; a failed f is
+// retried on the next call.
+constexpr int LLAMA_MAX_DEVICES = 64;
+struct PerDeviceOnce {
+    std::mutex mu;
+    bool done[LLAMA_MAX_DEVICES] = {};
+};
+template <class F>
+inline int once_per_device(PerDeviceOnce& pd, F&& f) {
+    int dev = -1;
+    LLAMA_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= LLAMA_MAX_DEVICES) return LLAMA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(pd.mu);
+    if (pd.done[dev]) return LLAMA_OK;
+    const int rc = f();
+    if (rc == LLAMA_OK) pd.done[dev] = true;
+    return rc;
 }
 
 static inline int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }

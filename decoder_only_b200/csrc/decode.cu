@@ -108,13 +108,9 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) attn_decode_kernel(
     }
     __syncthreads();   // barrier initialised before anyone waits on it
     // bounded wait for both copies
-    bool ok = false;
-    {
-        const uint64_t t0 = [] {
-            uint64_t t;
-            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-            return t;
-        }();
+    auto wait_copies = [bar_a](uint64_t limit_ns) {
+        uint64_t t0;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
         while (true) {
             uint32_t done;
             asm volatile(
@@ -123,17 +119,20 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) attn_decode_kernel(
                 : "=r"(done)
                 : "r"(bar_a)
                 : "memory");
-            if (done) {
-                ok = true;
-                break;
-            }
+            if (done) return true;
             uint64_t t;
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-            if (t - t0 > 2000000000ull) {
-                if (threadIdx.x == 0) atomicOr(err, LLAMA_DEVERR_TIMEOUT);
-                break;
-            }
+            if (t - t0 > limit_ns) return false;
         }
+    };
+    const bool ok = wait_copies(2000000000ull);
+    if (!ok) {
+        // The chunk is dropped (its partial carries no keys) and the error
+        // word says so.  The copies may still be in flight into this CTA's
+        // shared memory: wait for them once more (bounded) so that they do
+        // not land in the next CTA placed on this SM, and read none of it.
+        if (threadIdx.x == 0) atomicOr(err, LLAMA_DEVERR_TIMEOUT);
+        wait_copies(2000000000ull);
     }
     float m = -INFINITY, l = 0.f, acc[DPL];
 #pragma unroll
@@ -244,13 +243,12 @@ int* attention_decode_counters(float* work, int B, int H, int max_len, int hd) {
 
 template <typename T, int HD>
 static int dec_attr() {
-    static bool attr = false;
-    if (!attr) {
+    static PerDeviceOnce once;
+    return once_per_device(once, []() -> int {
         LLAMA_CUDA_TRY(cudaFuncSetAttribute(attn_decode_kernel<T, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             (int)(2 * (size_t)DEC_CHUNK * HD * sizeof(T))));
-        attr = true;
-    }
-    return LLAMA_OK;
+        return (int)LLAMA_OK;
+    });
 }
 
 template <typename T, int HD>

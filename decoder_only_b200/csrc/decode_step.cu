@@ -1241,12 +1241,13 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
 template <int BN, int HD>
 int launch_step_t(const StepArgs& a, cudaStream_t st) {
     using C = SCfg<BN, HD>;
-    static bool attr = false;
-    if (!attr) {
+    static PerDeviceOnce once;
+    int rc = once_per_device(once, []() -> int {
         LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<BN, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             C::SMEM));
-        attr = true;
-    }
+        return (int)LLAMA_OK;
+    });
+    if (rc) return rc;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(decode_step_ctas());
     cfg.blockDim = dim3(NT);

@@ -320,13 +320,12 @@ int num_sms() {
 
 template <int BN, int MODE>
 int ensure_attr() {
-    static bool attr = false;
-    if (!attr) {
+    static PerDeviceOnce once;
+    return once_per_device(once, []() -> int {
         LLAMA_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, MODE>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::SMEM));
-        attr = true;
-    }
-    return LLAMA_OK;
+        return (int)LLAMA_OK;
+    });
 }
 
 template <int BN, int MODE>

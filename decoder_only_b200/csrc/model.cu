@@ -133,10 +133,25 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // Error word of the standalone ops (the model has its own in its arena).
 __device__ int g_op_err_word;
 
+// Its device address on the current device: in host code the variable's
+// name is only a host-side stand-in, so the address is looked up once per
+// device, with that device current.
 int op_error_word(int** p) {
-    static int* addr = nullptr;
-    if (!addr) LLAMA_CUDA_TRY(cudaGetSymbolAddress((void**)&addr, g_op_err_word));
-    *p = addr;
+    static PerDeviceOnce once;
+    static int* addr[LLAMA_MAX_DEVICES];
+    int dev = -1;
+    LLAMA_CUDA_TRY(cudaGetDevice(&dev));
+    int rc = once_per_device(once, [dev]() -> int {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_op_err_word) != cudaSuccess || !a) {
+            cudaGetLastError();
+            return (int)LLAMA_ERR_CUDA;
+        }
+        addr[dev] = static_cast<int*>(a);
+        return (int)LLAMA_OK;
+    });
+    if (rc) return rc;
+    *p = addr[dev];
     return LLAMA_OK;
 }
 
@@ -1129,6 +1144,20 @@ int llama_debug_gemm_timeout(void* stream) {
     LLAMA_CUDA_TRY(cudaStreamSynchronize(st));
     if (rc) return rc;
     return (e & LLAMA_DEVERR_TIMEOUT) ? LLAMA_ERR_TIMEOUT : LLAMA_OK;
+}
+
+int llama_op_last_error(void) {
+    int* err = nullptr;
+    int rc = op_error_word(&err);
+    if (rc) return rc;
+    LLAMA_CUDA_TRY(cudaDeviceSynchronize());
+    int e = 0;
+    LLAMA_CUDA_TRY(cudaMemcpy(&e, err, sizeof(int), cudaMemcpyDeviceToHost));
+    LLAMA_CUDA_TRY(cudaMemset(err, 0, sizeof(int)));
+    LLAMA_CUDA_TRY(cudaDeviceSynchronize());
+    if (e & LLAMA_DEVERR_TIMEOUT) return LLAMA_ERR_TIMEOUT;
+    if (e) return LLAMA_ERR_INVALID_ARG;
+    return LLAMA_OK;
 }
 
 int llama_op_argmax(const float* d_logits, int32_t rows, int32_t n, int32_t* d_out, void* stream) {

@@ -232,13 +232,12 @@ __global__ void __launch_bounds__(256) attn_prefill_simt_kernel(const T* __restr
 
 template <typename T, int HD>
 static int attn_simt_attr(size_t smem) {
-    static bool attr_set = false;
-    if (!attr_set) {
+    static PerDeviceOnce once;
+    return once_per_device(once, [smem]() -> int {
         LLAMA_CUDA_TRY(cudaFuncSetAttribute(attn_prefill_simt_kernel<T, HD>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        attr_set = true;
-    }
-    return LLAMA_OK;
+        return (int)LLAMA_OK;
+    });
 }
 
 template <typename T, int HD>

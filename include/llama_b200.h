@@ -24,8 +24,11 @@
  * Conventions for every entry point below
  *   - Pointers named d_* are DEVICE pointers; h_* are HOST pointers.  The
  *     caller owns every buffer it passes and keeps it alive until the work
- *     queued on `stream` has finished.  The library never calls cudaMalloc:
- *     the model lives in one caller-allocated device arena.
+ *     queued on `stream` has finished.  The model lives in one
+ *     caller-allocated device arena and the single ops work on caller
+ *     buffers: no entry point allocates device memory, except the
+ *     failure-detection self-test llama_debug_gemm_timeout, which allocates
+ *     and frees its own 80 KB operands.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     asynchronous on it unless stated otherwise; outputs are valid once the
  *     stream has been synchronised.
@@ -91,7 +94,8 @@ typedef struct llama_model llama_model; /* opaque host handle */
 
 /* ------------------------------------------------------------------ model */
 
-/* Device bytes the model arena must hold for `cfg`: weights, RoPE table,
+/* Device bytes the model arena must hold for `cfg`: weights ([PFD] "6.7B
+ * parameters, 1T tokens: the arithmetic" counts them), RoPE table,
  * KV cache [L][2][max_batch][n_kv_heads][max_seq][head_dim], activations and
  * workspace.  Host-only; queues nothing. */
 LLAMA_API int llama_model_bytes(const llama_config* cfg, uint64_t* bytes_out);
@@ -106,7 +110,10 @@ LLAMA_API int llama_model_bytes(const llama_config* cfg, uint64_t* bytes_out);
 LLAMA_API int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena,
                        uint64_t arena_bytes, void* stream, llama_model** out);
 
-/* Causal prefill of B sequences of S tokens each (B <= max_batch,
+/* [PFD] "The one formula": embedding, L pre-norm blocks, final RMSNorm and
+ * head, with the causal mask of "LLaMA is a pull request against the 2017
+ * transformer".
+ * Causal prefill of B sequences of S tokens each (B <= max_batch,
  * 1 <= S <= max_seq).  d_tokens: int32 [B*S], row b*S + s.  Resets the KV
  * cache and sets the decode position to S.  d_logits: fp32 [B*S, vocab]
  * logits of every position, or NULL to skip the final norm and head. */
@@ -124,13 +131,18 @@ LLAMA_API int llama_prefill(llama_model* m, const int32_t* d_tokens, int32_t B, 
 LLAMA_API int llama_prefill_ragged(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S,
                                    const int32_t* h_lens, float* d_logits, void* stream);
 
-/* The blocks alone, on a given fp32 trunk: d_x [B*S, d_model] in,
+/* [PFD] "The one formula" and "Pre-norm: the norm goes on the branch, not
+ * the trunk": h = x + Attn(RMSNorm(x)), y = h + FFN(RMSNorm(h)), per block.
+ * The blocks alone, on a given fp32 trunk: d_x [B*S, d_model] in,
  * d_y [B*S, d_model] out (the trunk after the last block, before the final
  * norm).  Positions 0..S-1 per sequence.  d_x and d_y may alias. */
 LLAMA_API int llama_prefill_trunk(llama_model* m, const float* d_x, int32_t B, int32_t S,
                         float* d_y, void* stream);
 
-/* One greedy decoding step for the B sequences of the last prefill: token
+/* [NAR] "GQA Was Not an Original LLaMA Feature": autoregressive decoding
+ * appends the new token's key and value to the cache and attends over all
+ * cached positions.
+ * One greedy decoding step for the B sequences of the last prefill: token
  * d_tokens[b] (int32 [B]) sits at its sequence's current position p_b; its
  * K and V are appended at p_b; attention spans 0..p_b.  d_next (int32 [B],
  * may be NULL): argmax of the logits, lowest id on ties.  d_logits: fp32
@@ -225,19 +237,33 @@ LLAMA_API int llama_debug_gemm_timeout(void* stream);
  * The kernels the model runs, exposed one by one on caller buffers.  dtype
  * selects fp32 or bf16 storage of the T-typed operands. */
 
+/* Standalone-op error word: the single ops below (and
+ * llama_op_attention_decode_noalloc) record an expired bounded device wait
+ * in one word per device, as the model does in its own.  This waits for all
+ * work queued on the current device (cudaDeviceSynchronize), then reads and
+ * clears that device's word: LLAMA_OK, or LLAMA_ERR_TIMEOUT when a call's
+ * result is incomplete (a decode-attention chunk whose keys never arrived
+ * is left out of its row's softmax). */
+LLAMA_API int llama_op_last_error(void);
+
 /* y[r, :] = x[r, :] / sqrt(mean(x[r, :]^2) + eps) * g, r < rows.
  * x fp32 [rows, d]; g fp32 [d]; y dtype-typed [rows, d]; d % 4 == 0,
  * d <= 8192.  [PFD] "RMSNorm: LayerNorm minus the mean". */
 LLAMA_API int llama_op_rmsnorm(int32_t dtype, const float* d_x, const float* d_g, void* d_y,
                      int32_t rows, int32_t d, float eps, void* stream);
 
-/* C = A W^T, or C += A W^T when accumulate != 0.  A dtype-typed [M, K],
+/* [PFD] "The code": every projection is x @ W; here W is stored (d_out,
+ * d_in), so the product is A W^T.
+ * C = A W^T, or C += A W^T when accumulate != 0.  A dtype-typed [M, K],
  * W dtype-typed [N, K] (K-major), C fp32 [M, N].  bf16: tcgen05 tensor-core
  * GEMM, K % 64 == 0, N % 16 == 0, pointers 16-byte aligned; fp32: SIMT. */
 LLAMA_API int llama_op_gemm(int32_t dtype, const void* d_A, const void* d_W, float* d_C,
                   int32_t M, int32_t N, int32_t K, int32_t accumulate, void* stream);
 
-/* Causal attention, heads independent.  q, k, v dtype-typed with layout
+/* [PFD] "LLaMA is a pull request against the 2017 transformer" (attention
+ * untouched, causal mask); "RoPE: rotate Q and K, leave V alone" (q and k
+ * arrive rotated).
+ * Causal attention, heads independent.  q, k, v dtype-typed with layout
  * [B][H][*][head_dim]; q has S rows per head, k/v have kv_stride rows per
  * head (>= S; the first S are used).  o dtype-typed [B*S, H*head_dim]:
  * row b*S + t, columns of head h at [h*head_dim, (h+1)*head_dim).
@@ -247,7 +273,9 @@ LLAMA_API int llama_op_attention_prefill(int32_t dtype, const void* d_q, const v
                                int32_t S, int32_t head_dim, int32_t kv_stride,
                                void* stream);
 
-/* Decode attention: one query per (b, h) against keys/values 0..len-1.
+/* [NAR] "GQA Was Not an Original LLaMA Feature": the decoding query reads
+ * the keys and values of every earlier position.
+ * Decode attention: one query per (b, h) against keys/values 0..len-1.
  * q dtype-typed [B, H*head_dim]; k, v [B][H][kv_stride][head_dim];
  * o dtype-typed [B, H*head_dim].  Split over the sequence into chunks of 128
  * keys whose partial results go to d_work (llama_op_attention_decode_work_bytes
@@ -284,7 +312,8 @@ LLAMA_API int llama_op_attention_decode_noalloc(int32_t dtype, const void* d_q, 
                                                 int32_t len, int32_t head_dim, int32_t kv_stride,
                                                 void* stream);
 
-/* out[r] = argmax_j logits[r, j] (lowest j on ties), r < rows. */
+/* Greedy choice over the (n, vocab) logits of [PFD] "The one formula".
+ * out[r] = argmax_j logits[r, j] (lowest j on ties), r < rows. */
 LLAMA_API int llama_op_argmax(const float* d_logits, int32_t rows, int32_t n, int32_t* d_out,
                     void* stream);
 

@@ -21,7 +21,7 @@ Sources (cited by page title and section):
         Invention Myth" (RMSNorm with gain g, SwiGLU, the RoPE relative-offset
         identity) and "GQA Was Not an Original LLaMA Feature" (KV cache).
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * RMSNorm carries the gain g of [NAR]; the gains are 1 in every workload.
   * RoPE acts per head (its d is the head dimension), on interleaved
     (even, odd) channel pairs, angle = position * base^(-2i/d_head).

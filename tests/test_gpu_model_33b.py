@@ -12,7 +12,7 @@ import decoder_only_b200 as lb
 import oracle
 import synth
 from synth.workloads import LLAMA_33B, SEED
-from _parity import argmax_agreement, storage_bar
+from _parity import greedy_bar, storage_bar
 
 pytestmark = pytest.mark.gpu
 
@@ -35,7 +35,7 @@ def test_33b_widths_prefill_and_decode_against_oracle():
         m.close()
         torch.cuda.empty_cache()
     exact, stored = oracle.prefill(SHAPE, toks, storage=(None, "bf16"))
-    storage_bar(pre, exact[:, :PROMPT], stored[:, :PROMPT])
-    storage_bar(dec, exact[:, PROMPT:], stored[:, PROMPT:])
-    assert argmax_agreement(pre, exact[:, :PROMPT])[1] >= 0.99
-    assert argmax_agreement(dec, exact[:, PROMPT:])[1] >= 0.99
+    storage_bar(pre, exact[:, :PROMPT], stored[:, :PROMPT], what="33B prefill")
+    storage_bar(dec, exact[:, PROMPT:], stored[:, PROMPT:], what="33B decode")
+    greedy_bar(pre, exact[:, :PROMPT], stored[:, :PROMPT], what="33B prefill")
+    greedy_bar(dec, exact[:, PROMPT:], stored[:, PROMPT:], what="33B decode")

@@ -313,6 +313,41 @@ def test_bf16_kv_cache_alone_moves_deep_logits_past_2e2():
     assert np.sqrt(np.mean((kv_only - exact) ** 2)) / rms < 2e-2
 
 
+def test_bf16_storage_alone_moves_one_7b_block_past_2e2():
+    """Why the stated 2e-2 max-norm bound is not asserted even for one block:
+    one 7B-shaped block on the 1 x 2048 N(0, 1) trunk, exact in fp64 except
+    that every value a bf16 workload stores in bf16 is rounded to bf16
+    (normalised projection inputs, Q, K, V, attention output, SwiGLU
+    activation), already moves both the block output y and its increment
+    y - x by more than 2e-2 of their RMS in max norm, while the RMS-norm
+    distance stays far below it."""
+    from synth.workloads import BLOCK_7B, SEED
+    import synth
+    S, d = 2048, BLOCK_7B.d_model
+    x = synth.normal_f32(SEED, synth.TRUNK, S * d, 1.0).reshape(S, d).astype(np.float64)
+    W = oracle.layer_weights(BLOCK_7B, 0)
+    exact = oracle.block_forward(BLOCK_7B, x, weights=W)
+    stored = oracle.block_forward(BLOCK_7B, x, weights=W, storage="bf16")
+    for a, b in ((stored, exact), (stored - x, exact - x)):
+        r = np.sqrt(np.mean(b ** 2))
+        assert np.max(np.abs(a - b)) / r > 2e-2
+        assert np.sqrt(np.mean((a - b) ** 2)) / r < 5e-3
+
+
+def test_bf16_storage_alone_flips_over_1pct_of_greedy_tokens_at_two_7b_layers():
+    """Why strict greedy agreement >= 99 % is not asserted at 7B widths: with
+    random-init weights the top two of 32000 logits are often close, and
+    bf16 storage alone (everything else exact) already changes the greedy
+    token at more than 1 % of the positions of a two-layer 7B-width model.
+    The GPU tests hold the GPU to the flip count of bf16 storage instead."""
+    from synth.workloads import LLAMA_7B, SEED
+    import synth
+    s = LLAMA_7B.with_(n_layers=2)
+    tok = synth.tokens(SEED, 2 * 256, s.vocab).reshape(2, 256)
+    exact, stored = oracle.prefill(s, tok, storage=(None, "bf16"))
+    assert np.mean(exact.argmax(-1) == stored.argmax(-1)) < 0.99
+
+
 # ---------------------------------------------------------------- grouped keys and values
 
 def _gqa_shape(n_kv):
