@@ -528,6 +528,72 @@ def run_b200(args, wl, shape):
         dist.destroy_process_group()
 
 
+# ----------------------------------------------------------------------------- tensor parallel
+
+def run_tp(args, wl, shape):
+    """--parallel tp under torchrun: one model split over the N ranks
+    (llama_config.tp_size = N), its prefill's two exchanges per block done by
+    NCCL all-reduce (torch.distributed) on the library's exchange stream.
+    Decoding is not sharded, so a step is the prefill alone (logits at every
+    position); total work is fixed as N grows (scaling "strong")."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import decoder_only_b200 as lb
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    B, S = wl["batch"], wl["seq"]
+    model = lb.Model(shape, max_batch=B, max_seq=S, seed=synth.workloads.SEED, tp=(rank, world))
+    model.set_allreduce(lb.dist_allreduce(), chunks=args.tp_chunks)
+    tok = torch.from_numpy(replica_tokens(shape, 0, B, S)).cuda()    # every shard sees the same batch
+    logits = torch.empty(B, S, shape.vocab, dtype=torch.float32, device="cuda")
+    st = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        model.prefill(tok, out=logits)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    l0 = lb.kernel_launches()
+    with ClockSampler(local) as clk:
+        ev[0].record(st)
+        for _ in range(args.steps):
+            model.prefill(tok, out=logits)
+        ev[1].record(st)
+        torch.cuda.synchronize()
+    dist.barrier()
+    launches = lb.kernel_launches() - l0
+    ms = max_over_ranks(ev[0].elapsed_time(ev[1]), world, "cuda")
+    flops, _ = algorithmic_work(shape, B, S, 0)
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        per_s = ms * 1e-3 / args.steps
+        print(json.dumps(dict(
+            metric=METRIC, value=round(B * S * args.steps / (ms * 1e-3), 2), unit=UNIT, n_gpus=world,
+            steps=args.steps, warmup=args.warmup, ms_per_step=round(ms / args.steps, 3), higher_is_better=True,
+            scaling="strong", vs_baseline=None, dtype="bf16",
+            data="synthetic (seeded token ids; random-init weights N(0, 0.02^2) drawn on device)",
+            config=dict(workload=f"{wl['desc'].split(':')[0]}: prefill {B} x {S} (logits at every position), "
+                                 f"tensor parallel over {world} GPUs", model=shape.name, global_batch=B, seq_len=S,
+                        parallelism=f"tp{world} (NCCL all-reduce after O and down, {args.tp_chunks} row blocks)",
+                        l2="inputs larger than L2: every step streams all weights from HBM"),
+            gpu_launches=launches, clocks=clk.summary(),
+            prefill=dict(tflops=round(flops / per_s / 1e12, 1),
+                         frac_bf16_per_gpu=round(flops / per_s / 1e12 / world / peaks["bf16_tflops_sustained"], 4),
+                         peak_source=peak_src))), flush=True)
+    model.close()
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 # ----------------------------------------------------------------------------- per-kernel sweep
 
 # (batch, sequence length) points of the per-kernel prefill sweep at the 65B
@@ -652,6 +718,13 @@ def main():
                     help="per-kernel prefill sweep over batch {1, 8} x length {512, 1024, 2048} "
                          "(one JSON line; 1 GPU)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-heads", type=int, default=0,
+                    help="grouped keys and values: the workload's model with this many key/value heads")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "tp"],
+                    help="N > 1: independent replicas (default) or one model split over the N GPUs "
+                         "(tensor parallel prefill, under torchrun)")
+    ap.add_argument("--tp-chunks", type=int, default=4, help="row blocks per exchange with --parallel tp")
     ap.add_argument("--ncu", action="store_true",
                     help="only the warm-up and timed steps, each timed step in an NVTX range 'timed_step' "
                          "(for: ncu --nvtx --nvtx-include timed_step/ ...); prints no JSON")
@@ -669,12 +742,23 @@ def main():
     shape = getattr(wls, wl["model"])
     if "layers" in wl:
         shape = shape.with_(n_layers=wl["layers"], name=f"{shape.name}-{wl['layers']}layer")
+    if args.kv_heads:
+        shape = shape.with_(n_kv_heads=args.kv_heads, name=f"{shape.name}-kv{args.kv_heads}")
+        wl["desc"] = wl["desc"].replace(":", f" ({args.kv_heads} key/value heads):", 1)
+    if args.batch:
+        wl["desc"] = wl["desc"].replace(f"{wl['batch']} x", f"{args.batch} x", 1).replace(
+            f"batch {wl['batch']}", f"batch {args.batch}", 1)
+        wl["batch"] = args.batch
     if args.sweep:
         if args.impl == "reference" or int(os.environ.get("WORLD_SIZE", "1")) > 1:
             ap.error("--sweep times this library on one GPU")
         run_sweep(args, wl, shape)
     elif args.impl == "reference":
         run_reference(args, wl, shape)
+    elif args.parallel == "tp":
+        if int(os.environ.get("WORLD_SIZE", "1")) < 2:
+            ap.error("--parallel tp needs torchrun with 2 or more ranks")
+        run_tp(args, wl, shape)
     else:
         run_b200(args, wl, shape)
 

@@ -10,6 +10,7 @@ from __future__ import annotations
 import ctypes
 import os
 import re
+import traceback
 
 import torch
 
@@ -33,7 +34,11 @@ class LlamaConfig(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("ffn_hidden", ctypes.c_int32), ("vocab", ctypes.c_int32),
                 ("norm_eps", ctypes.c_float), ("rope_theta", ctypes.c_float), ("dtype", ctypes.c_int32),
                 ("max_batch", ctypes.c_int32), ("max_seq", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
-                ("bias", ctypes.c_int32)]
+                ("bias", ctypes.c_int32), ("tp_size", ctypes.c_int32), ("tp_rank", ctypes.c_int32)]
+
+
+# int (*)(float* d_buf, uint64_t count, void* stream, void* ctx): the exchange of a shard
+ALLREDUCE_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p)
 
 
 def _load():
@@ -63,6 +68,8 @@ def _load():
         "llama_op_attention_decode_noalloc": [I, P, P, P, P, I, I, I, I, I, P],
         "llama_op_argmax": [P, I, I, P, P],
         "llama_op_last_error": [],
+        "llama_set_allreduce": [P, ALLREDUCE_FN, P, I],
+        "llama_tp_shard": [P, P],
         "llama_rewind": [P, I, P],
         "llama_complete": [P, P, I, I, P, I, P, P],
         "llama_kernel_launches": [],
@@ -115,13 +122,63 @@ def _dt(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def make_config(shape, max_batch: int, max_seq: int) -> LlamaConfig:
+def make_config(shape, max_batch: int, max_seq: int, tp=None) -> LlamaConfig:
     """`shape`: any object with n_layers, d_model, n_heads, head_dim,
-    ffn_hidden, vocab, dtype ('bf16' | 'f32'), norm_eps, rope_theta."""
+    ffn_hidden, vocab, dtype ('bf16' | 'f32'), norm_eps, rope_theta.
+    `tp`: (rank, size) of a tensor-parallel shard, or None."""
+    rank, size = tp if tp is not None else (0, 0)
     return LlamaConfig(shape.n_layers, shape.d_model, shape.n_heads, shape.head_dim, shape.ffn_hidden,
                        shape.vocab, shape.norm_eps, shape.rope_theta, BF16 if shape.dtype == "bf16" else F32,
                        max_batch, max_seq, int(getattr(shape, "n_kv_heads", 0) or 0),
-                       int(bool(getattr(shape, "bias", False))))
+                       int(bool(getattr(shape, "bias", False))), size, rank)
+
+
+def tp_shard(shape, rank: int, size: int) -> dict:
+    """The slices shard `rank` of `size` holds (llama_tp_shard)."""
+    cfg = make_config(shape, 1, 1, (rank, size))
+    out = (ctypes.c_int32 * 6)()
+    _check(lib.llama_tp_shard(ctypes.byref(cfg), ctypes.cast(out, ctypes.c_void_p)), "llama_tp_shard")
+    return dict(head0=out[0], heads=out[1], kv_head0=out[2], kv_heads=out[3], hidden0=out[4], hidden=out[5])
+
+
+def allreduce_callback(resolve, reduce):
+    """The C exchange (llama_allreduce_fn) around two Python callables:
+    resolve(ptr, count) -> the float32 tensor of `count` elements at `ptr`;
+    reduce(buf, stream) queues the sum over the shards of `buf` in place on
+    `stream` (a torch stream, or None for host tensors).  Exceptions are
+    printed and reported to the library as a failed exchange."""
+    streams = {}
+
+    def cb(ptr, count, stream, ctx):
+        try:
+            buf = resolve(ptr or 0, int(count))
+            st = None
+            if stream:
+                st = streams.get(stream)
+                if st is None:
+                    st = streams[stream] = torch.cuda.ExternalStream(stream)
+            reduce(buf, st)
+            return 0
+        except Exception:
+            traceback.print_exc()
+            return 1
+
+    return ALLREDUCE_FN(cb)
+
+
+def dist_allreduce(group=None):
+    """reduce(buf, stream) for allreduce_callback / Model.set_allreduce: one
+    torch.distributed sum all-reduce (NCCL between GPUs) queued on `stream`."""
+    import torch.distributed as dist
+
+    def reduce(buf, stream):
+        if stream is None:
+            dist.all_reduce(buf, group=group)
+        else:
+            with torch.cuda.stream(stream):
+                dist.all_reduce(buf, group=group)
+
+    return reduce
 
 
 def model_bytes(cfg: LlamaConfig) -> int:
@@ -133,9 +190,9 @@ def model_bytes(cfg: LlamaConfig) -> int:
 class Model:
     """One model in one device arena.  Weights are generated on the device."""
 
-    def __init__(self, shape, max_batch: int, max_seq: int, seed: int = 0):
+    def __init__(self, shape, max_batch: int, max_seq: int, seed: int = 0, tp=None):
         self.shape = shape
-        self.cfg = make_config(shape, max_batch, max_seq)
+        self.cfg = make_config(shape, max_batch, max_seq, tp)
         nbytes = model_bytes(self.cfg)
         self.arena = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
         h = ctypes.c_void_p()
@@ -148,6 +205,19 @@ class Model:
         if self.h:
             lib.llama_free(self.h)
             self.h = None
+
+    def set_allreduce(self, reduce, chunks: int = 4):
+        """Installs the exchange of a tensor-parallel shard (llama_set_allreduce):
+        reduce(buf, stream) sums `buf`, a float32 view of trunk rows in this
+        model's arena, over the shards in place on `stream`."""
+        arena = self.arena
+
+        def resolve(ptr, count):
+            off = ptr - arena.data_ptr()
+            return arena[off:off + 4 * count].view(torch.float32)
+
+        self._allreduce_cb = allreduce_callback(resolve, reduce)   # kept alive with the model
+        _check(lib.llama_set_allreduce(self.h, self._allreduce_cb, None, chunks), "llama_set_allreduce")
 
     def __del__(self):
         try:

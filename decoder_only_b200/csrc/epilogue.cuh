@@ -36,6 +36,7 @@ struct EpiArgs {
     int H, hd, d, smax;
     int Hkv;              // key/value heads: columns [d, d + Hkv hd) are K, then V
     const float* bias;    // the bias variant: fp32 per output column (weight row order), or NULL
+    int m0;               // EPI_QKV prefill: token row of the GEMM's first row (row blocks launched apart)
 };
 
 __device__ __forceinline__ float silu_f(float u) { return u / (1.0f + __expf(-u)); }
@@ -137,8 +138,8 @@ __device__ __forceinline__ void epi_qkv32(const EpiArgs& a, int m, int n0, const
         s = 0;
         pos = a.d_pos[m];
     } else {
-        b = m / a.S;
-        s = m - b * a.S;
+        b = (m + a.m0) / a.S;
+        s = (m + a.m0) - b * a.S;
         pos = s;
     }
     float r[32];

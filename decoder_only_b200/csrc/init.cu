@@ -60,22 +60,27 @@ template <typename T> __device__ __forceinline__ T round_store(double v);
 template <> __device__ __forceinline__ float round_store<float>(double v) { return __double2float_rn(v); }
 template <> __device__ __forceinline__ bf16 round_store<bf16>(double v) { return f64_to_bf16_rne(v); }
 
-// Fill the device rows of one logical matrix.
-//   logical output column n in [0, N_log), input index k in [0, K);
-//   device row = row_off + (n / blk) * blk_stride + (n % blk), row length K;
-//   element index e = rowmajor_nk ? n*K + k : k*N_log + n.
+// Fill the device rows of a block of one logical matrix.
+//   The logical matrix has output columns n in [0, N_full) and inputs
+//   k in [0, K_full); element index e = rowmajor_nk ? n*K_full + k
+//   : k*N_full + n.  The block held here is n in [n0, n0 + N_loc),
+//   k in [k0, k0 + K_loc) (a tensor-parallel shard; the whole matrix when
+//   n0 = k0 = 0 and the sizes are the full ones).  Local column nl = n - n0
+//   goes to device row row_off + (nl / blk) * blk_stride + (nl % blk), row
+//   length K_loc, at column k - k0.
 template <typename T>
-__global__ void init_matrix_kernel(T* __restrict__ dst, int K, int N_log, int blk, int blk_stride,
-                                   int row_off, int rowmajor_nk, uint32_t seed, uint32_t tensor_id,
-                                   double scale) {
-    const uint64_t total = (uint64_t)N_log * (uint64_t)K;
+__global__ void init_matrix_kernel(T* __restrict__ dst, int K_full, int N_full, int k0, int K_loc, int n0, int N_loc,
+                                   int blk, int blk_stride, int row_off, int rowmajor_nk, uint32_t seed,
+                                   uint32_t tensor_id, double scale) {
+    const uint64_t total = (uint64_t)N_loc * (uint64_t)K_loc;
     for (uint64_t idx = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; idx < total;
          idx += (uint64_t)gridDim.x * blockDim.x) {
-        const int n = (int)(idx / (uint64_t)K);
-        const int k = (int)(idx - (uint64_t)n * K);
-        const uint64_t e = rowmajor_nk ? idx : (uint64_t)k * N_log + n;
-        const int row = row_off + (n / blk) * blk_stride + (n % blk);
-        dst[(size_t)row * K + k] = round_store<T>(scale * normal_at(seed, tensor_id, e));
+        const int nl = (int)(idx / (uint64_t)K_loc);
+        const int kl = (int)(idx - (uint64_t)nl * K_loc);
+        const uint64_t n = (uint64_t)(n0 + nl), k = (uint64_t)(k0 + kl);
+        const uint64_t e = rowmajor_nk ? n * K_full + k : k * N_full + n;
+        const int row = row_off + (nl / blk) * blk_stride + (nl % blk);
+        dst[(size_t)row * K_loc + kl] = round_store<T>(scale * normal_at(seed, tensor_id, e));
     }
 }
 
@@ -84,19 +89,29 @@ __global__ void fill_f32_kernel(float* dst, float v, int64_t n) {
         dst[i] = v;
 }
 
-int launch_init_matrix(int dtype, void* dst, int K, int N_log, int blk, int blk_stride, int row_off,
-                       int rowmajor_nk, uint32_t seed, uint32_t tensor_id, double scale,
-                       cudaStream_t st) {
+int launch_init_shard(int dtype, void* dst, int K_full, int N_full, int k0, int K_loc, int n0, int N_loc, int blk,
+                      int blk_stride, int row_off, int rowmajor_nk, uint32_t seed, uint32_t tensor_id, double scale,
+                      cudaStream_t st) {
+    if (k0 < 0 || n0 < 0 || K_loc <= 0 || N_loc <= 0 || k0 + K_loc > K_full || n0 + N_loc > N_full || blk <= 0)
+        return LLAMA_ERR_INVALID_ARG;
     const int threads = 256;
     const int blocks = 148 * 16;
     if (dtype == LLAMA_BF16)
-        init_matrix_kernel<bf16><<<blocks, threads, 0, st>>>((bf16*)dst, K, N_log, blk, blk_stride, row_off,
-                                                             rowmajor_nk, seed, tensor_id, scale);
+        init_matrix_kernel<bf16><<<blocks, threads, 0, st>>>((bf16*)dst, K_full, N_full, k0, K_loc, n0, N_loc, blk,
+                                                             blk_stride, row_off, rowmajor_nk, seed, tensor_id, scale);
     else
-        init_matrix_kernel<float><<<blocks, threads, 0, st>>>((float*)dst, K, N_log, blk, blk_stride, row_off,
-                                                              rowmajor_nk, seed, tensor_id, scale);
+        init_matrix_kernel<float><<<blocks, threads, 0, st>>>((float*)dst, K_full, N_full, k0, K_loc, n0, N_loc,
+                                                              blk, blk_stride, row_off, rowmajor_nk, seed, tensor_id,
+                                                              scale);
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;
+}
+
+int launch_init_matrix(int dtype, void* dst, int K, int N_log, int blk, int blk_stride, int row_off,
+                       int rowmajor_nk, uint32_t seed, uint32_t tensor_id, double scale,
+                       cudaStream_t st) {
+    return launch_init_shard(dtype, dst, K, N_log, 0, K, 0, N_log, blk, blk_stride, row_off, rowmajor_nk, seed,
+                             tensor_id, scale, st);
 }
 
 int launch_fill_f32(float* dst, float v, int64_t n, cudaStream_t st) {

@@ -14,6 +14,10 @@ struct EpiArgs;
 // init.cu
 int launch_init_matrix(int dtype, void* dst, int K, int N_log, int blk, int blk_stride, int row_off,
                        int rowmajor_nk, uint32_t seed, uint32_t tensor_id, double scale, cudaStream_t st);
+// block n in [n0, n0 + N_loc), k in [k0, k0 + K_loc) of a (K_full, N_full) logical matrix
+int launch_init_shard(int dtype, void* dst, int K_full, int N_full, int k0, int K_loc, int n0, int N_loc, int blk,
+                      int blk_stride, int row_off, int rowmajor_nk, uint32_t seed, uint32_t tensor_id, double scale,
+                      cudaStream_t st);
 int launch_fill_f32(float* dst, float v, int64_t n, cudaStream_t st);
 // c = b + W beta per row of W [rows, K] (the bias variant's folded bias)
 int launch_bias_fold(int dtype, const void* W, int rows, int K, const float* beta, const float* b, float* c,

@@ -197,6 +197,15 @@ struct llama_model {
     int cur_len;             // largest position over the sequences (host)
     std::vector<int> pos_h;  // host mirror of d_pos: each sequence's position (ragged batches)
     int splits_qkv, splits_o, splits_gu, splits_d, splits_head;
+    // tensor parallelism (tp > 1): this shard's query heads, key/value heads
+    // and FFN hidden units (the full counts when tp == 1), the exchange and
+    // its stream, and the events ordering the row blocks between the streams
+    int tp, tp_rank, Hl, Hkvl, hl;
+    llama_allreduce_fn ar_fn;
+    void* ar_ctx;
+    int ar_chunks;
+    cudaStream_t comm;
+    std::vector<cudaEvent_t> tp_ev;   // [3][TP_MAX_CHUNKS]: ready, O exchanged, down exchanged
     cudaStream_t cap_stream;
     cudaGraphExec_t graph;
     int graph_B;
@@ -210,6 +219,13 @@ int hidden_of(const llama_config* c);
 // Key/value heads (grouped keys and values); 0 in the config means one per query head
 inline int kv_heads(const llama_config* c) { return c->n_kv_heads > 0 ? c->n_kv_heads : c->n_heads; }
 
+// Tensor parallelism: shards, and what one shard holds
+constexpr int TP_MAX_CHUNKS = 16;
+inline int tp_of(const llama_config* c) { return c->tp_size > 1 ? c->tp_size : 1; }
+inline int heads_local(const llama_config* c) { return c->n_heads / tp_of(c); }
+inline int kv_local(const llama_config* c) { return kv_heads(c) / tp_of(c); }
+inline int hidden_local(const llama_config* c) { return hidden_of(c) / tp_of(c); }
+
 int validate(const llama_config* c) {
     if (!c) return LLAMA_ERR_INVALID_ARG;
     if (c->n_layers < 0 || c->d_model <= 0 || c->n_heads <= 0 || c->vocab <= 0) return LLAMA_ERR_INVALID_ARG;
@@ -220,6 +236,16 @@ int validate(const llama_config* c) {
     if (!(c->norm_eps >= 0.f) || !(c->rope_theta > 0.f)) return LLAMA_ERR_INVALID_ARG;
     if (c->d_model % 32 != 0 || c->d_model > 8192) return LLAMA_ERR_INVALID_ARG;
     if (c->ffn_hidden < 0 || c->ffn_hidden % 128 != 0) return LLAMA_ERR_INVALID_ARG;
+    if (c->tp_size < 0 || c->tp_size > 64) return LLAMA_ERR_INVALID_ARG;
+    if (c->tp_size > 1) {
+        // whole heads, whole key/value heads and whole 128-unit SwiGLU blocks per shard
+        const int T = c->tp_size;
+        if (c->tp_rank < 0 || c->tp_rank >= T) return LLAMA_ERR_INVALID_ARG;
+        if (c->n_heads % T != 0 || kv_heads(c) % T != 0 || hidden_of(c) % (128 * T) != 0)
+            return LLAMA_ERR_INVALID_ARG;
+    } else if (c->tp_rank != 0) {
+        return LLAMA_ERR_INVALID_ARG;
+    }
     if (c->dtype == LLAMA_BF16) {
         if (c->head_dim != 64 && c->head_dim != 128) return LLAMA_ERR_INVALID_ARG;
         if (c->d_model % 256 != 0) return LLAMA_ERR_INVALID_ARG;
@@ -245,8 +271,10 @@ int hidden_of(const llama_config* c) {
 // Walks the arena layout; with m != NULL assigns the pointers.
 uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     const int esz = c->dtype == LLAMA_BF16 ? 2 : 4;
-    const size_t d = c->d_model, h = hidden_of(c), V = c->vocab, L = c->n_layers;
-    const size_t kvd = (size_t)kv_heads(c) * c->head_dim;
+    // per shard: dq query features, kvd key/value features, h hidden units
+    const size_t d = c->d_model, h = hidden_local(c), V = c->vocab, L = c->n_layers;
+    const size_t kvd = (size_t)kv_local(c) * c->head_dim;
+    const size_t dq = (size_t)heads_local(c) * c->head_dim;
     const size_t nmax = (size_t)c->max_batch * c->max_seq;
     size_t off = 0;
     auto take = [&](size_t bytes) -> void* {
@@ -261,20 +289,20 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     }
     for (size_t l = 0; l < L; ++l) {
         Layer ly;
-        ly.wqkv = take((d + 2 * kvd) * d * esz);
-        ly.wo = take(d * d * esz);
+        ly.wqkv = take((dq + 2 * kvd) * d * esz);
+        ly.wo = take(d * dq * esz);
         ly.wgu = take(2 * h * d * esz);
         ly.wd = take(d * h * esz);
         ly.g_attn = (float*)take(d * 4);
         ly.g_ffn = (float*)take(d * 4);
         if (c->bias) {
-            ly.b_qkv = (float*)take((d + 2 * kvd) * 4);
+            ly.b_qkv = (float*)take((dq + 2 * kvd) * 4);
             ly.b_o = (float*)take(d * 4);
             ly.b_gu = (float*)take(2 * h * 4);
             ly.b_d = (float*)take(d * 4);
             ly.beta_attn = (float*)take(d * 4);
             ly.beta_ffn = (float*)take(d * 4);
-            ly.c_qkv = (float*)take((d + 2 * kvd) * 4);
+            ly.c_qkv = (float*)take((dq + 2 * kvd) * 4);
             ly.c_gu = (float*)take(2 * h * 4);
         }
         if (m) m->layers[l] = ly;
@@ -282,14 +310,14 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     float* g_final = (float*)take(d * 4);
     void* head = take(V * d * esz);
     float2* rope = (float2*)take((size_t)c->max_seq * (c->head_dim / 2) * sizeof(float2));
-    const size_t kv_layer = (size_t)c->max_batch * kv_heads(c) * c->max_seq * c->head_dim;
+    const size_t kv_layer = (size_t)c->max_batch * kv_local(c) * c->max_seq * c->head_dim;
     void* kv = take(2 * L * kv_layer * esz);
     float* trunk = (float*)take(nmax * d * 4);
     void* xn = take(nmax * d * esz);
-    void* q = take(nmax * d * esz);
-    void* attn = take(nmax * d * esz);
+    void* q = take(nmax * dq * esz);
+    void* attn = take(nmax * dq * esz);
     void* act = take(nmax * h * esz);
-    const size_t cmax = std::max(3 * d, 2 * h);
+    const size_t cmax = std::max(dq + 2 * kvd, 2 * h);
     float* gemm_c = (float*)take(c->dtype == LLAMA_F32 ? nmax * std::max(cmax, V) * 4 : 0);
     float* logits_dec = (float*)take((size_t)c->max_batch * V * 4);
     long long part_off[5];
@@ -391,13 +419,13 @@ EpiArgs base_args(llama_model* m, int M, int N) {
     memset(&a, 0, sizeof(a));
     a.M = M;
     a.N = N;
-    a.H = m->cfg.n_heads;
-    a.Hkv = kv_heads(&m->cfg);
+    a.H = m->Hl;                       // this shard's heads (all of them without tensor parallelism)
+    a.Hkv = m->Hkvl;
     a.hd = m->cfg.head_dim;
-    a.d = m->cfg.d_model;
+    a.d = m->Hl * m->cfg.head_dim;     // Q columns of the QKV projection
     a.smax = m->cfg.max_seq;
     a.rope = m->rope;
-    a.hidden = hidden_of(&m->cfg);
+    a.hidden = m->hl;
     return a;
 }
 
@@ -508,6 +536,131 @@ int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
         if ((rc = project(m, "down", EPI_RESID, m->act, ly.wd, n, d, h, m->splits_d, ra, decode, st))) return rc;
     }
     return LLAMA_OK;
+}
+
+// ----------------------------------------------------------- tensor parallel
+// One projection on token rows [r0, r0 + rows) of A [n, K] (row-major): the
+// operand, the outputs and, for the QKV epilogue, the token index of its
+// first row move with the block.
+int project_rows(llama_model* m, const char* name, int mode, const void* A, const void* W, int r0, int rows,
+                 int N, int K, EpiArgs a, cudaStream_t st) {
+    const uint8_t* Ar = static_cast<const uint8_t*>(A) + (size_t)r0 * K * m->esz;
+    a.M = rows;
+    if (a.out) a.out += (size_t)r0 * a.ld_out;
+    if (a.act) a.act = static_cast<uint8_t*>(a.act) + (size_t)r0 * a.hidden * m->esz;
+    a.m0 = r0;
+    return project(m, name, mode, Ar, W, rows, N, K, 1, a, false, st);
+}
+
+// The L blocks of a shard ([KN] "Efficient Training Implementation": model
+// parallelism with the all-reduce hidden behind computation).  The token
+// rows after attention are cut into row blocks; per block, the O (and
+// later the down) projection writes this shard's partial into the trunk --
+// shard 0 adds it to the trunk and the output bias, the others store it --
+// and the exchange sums the block over the shards on the model's own
+// stream while the next block computes.  The FFN norm of a block (and, in
+// the next layer, the attention norm and QKV projection of a block) waits
+// only for that block's exchange.  Attention needs every row of a sequence
+// and runs once per layer, between the QKV and O row blocks.
+int run_blocks_tp(llama_model* m, int B, int S, cudaStream_t st) {
+    const llama_config& c = m->cfg;
+    const int d = c.d_model, dq = m->Hl * c.head_dim;
+    const int nq = dq + 2 * m->Hkvl * c.head_dim;
+    const int n = B * S, dt = c.dtype;
+    const int want = std::max(1, std::min(m->ar_chunks, TP_MAX_CHUNKS));
+    const int per = std::max(128, ((n + want - 1) / want + 127) / 128 * 128);
+    const int nch = (n + per - 1) / per;
+    cudaEvent_t* ready = m->tp_ev.data();
+    cudaEvent_t* done_o = ready + TP_MAX_CHUNKS;
+    cudaEvent_t* done_d = ready + 2 * TP_MAX_CHUNKS;
+    const bool lead = m->tp_rank == 0;
+    const int out_mode = lead ? EPI_RESID : EPI_F32;
+    auto rows_of = [&](int k) { return std::min(per, n - k * per); };
+    // queue the sum over the shards of trunk rows of block k after the work queued so far on st
+    auto exchange = [&](int k, cudaEvent_t done) -> int {
+        LLAMA_CUDA_TRY(cudaEventRecord(ready[k], st));
+        LLAMA_CUDA_TRY(cudaStreamWaitEvent(m->comm, ready[k], 0));
+        {
+            const double bytes = (double)rows_of(k) * d * 4;
+            prof::Scope ps(m->comm, "prefill_allreduce", 2.0 * bytes * (m->tp - 1) / m->tp, 0.0);
+            if (m->ar_fn(m->trunk + (size_t)k * per * d, (uint64_t)rows_of(k) * d, (void*)m->comm, m->ar_ctx) != 0)
+                return LLAMA_ERR_CUDA;
+        }
+        LLAMA_CUDA_TRY(cudaEventRecord(done, m->comm));
+        return LLAMA_OK;
+    };
+    int rc;
+    for (int l = 0; l < c.n_layers; ++l) {
+        const Layer& ly = m->layers[l];
+        // attention norm + QKV (+ RoPE, KV append) per row block
+        for (int k = 0; k < nch; ++k) {
+            const int r0 = k * per, rows = rows_of(k);
+            if (l > 0) LLAMA_CUDA_TRY(cudaStreamWaitEvent(st, done_d[k], 0));
+            {
+                prof::Scope ps(st, "prefill_rmsnorm", (double)rows * d * (4 + m->esz), 3.0 * rows * d);
+                if ((rc = launch_rmsnorm(dt, m->trunk + (size_t)r0 * d, ly.g_attn,
+                                         static_cast<uint8_t*>(m->xn) + (size_t)r0 * d * m->esz, rows, d, c.norm_eps,
+                                         st, ly.beta_attn)))
+                    return rc;
+            }
+            EpiArgs qa = base_args(m, rows, nq);
+            qa.q = m->q;
+            qa.kc = kcache(m, l);
+            qa.vc = vcache(m, l);
+            qa.S = S;
+            qa.bias = ly.b_qkv;
+            if ((rc = project_rows(m, "qkv", EPI_QKV, m->xn, ly.wqkv, r0, rows, nq, d, qa, st))) return rc;
+        }
+        {
+            prof::Scope ps(st, "prefill_attention", 4.0 * n * dq * m->esz, 2.0 * B * (double)S * (S + 1) * dq);
+            if (dt == LLAMA_BF16)
+                rc = launch_attention_prefill_tc(m->q, kcache(m, l), vcache(m, l), m->attn, B, m->Hl, m->Hkvl, S,
+                                                 c.head_dim, c.max_seq, m->d_err, st);
+            else
+                rc = launch_attention_prefill_simt(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, m->Hl, m->Hkvl,
+                                                   S, c.head_dim, c.max_seq, st);
+            if (rc) return rc;
+        }
+        // O projection: this shard's partial of each row block, then its exchange
+        for (int k = 0; k < nch; ++k) {
+            EpiArgs ra = base_args(m, rows_of(k), d);
+            ra.out = m->trunk;
+            ra.ld_out = d;
+            ra.bias = lead ? ly.b_o : nullptr;
+            if ((rc = project_rows(m, "o", out_mode, m->attn, ly.wo, k * per, rows_of(k), d, dq, ra, st))) return rc;
+            if ((rc = exchange(k, done_o[k]))) return rc;
+        }
+        // FFN per row block, once the block's attention output has been summed
+        for (int k = 0; k < nch; ++k) {
+            const int r0 = k * per, rows = rows_of(k);
+            LLAMA_CUDA_TRY(cudaStreamWaitEvent(st, done_o[k], 0));
+            {
+                prof::Scope ps(st, "prefill_rmsnorm", (double)rows * d * (4 + m->esz), 3.0 * rows * d);
+                if ((rc = launch_rmsnorm(dt, m->trunk + (size_t)r0 * d, ly.g_ffn,
+                                         static_cast<uint8_t*>(m->xn) + (size_t)r0 * d * m->esz, rows, d, c.norm_eps,
+                                         st, ly.beta_ffn)))
+                    return rc;
+            }
+            EpiArgs sa = base_args(m, rows, 2 * m->hl);
+            sa.act = m->act;
+            sa.bias = ly.b_gu;
+            if ((rc = project_rows(m, "gateup", EPI_SWIGLU, m->xn, ly.wgu, r0, rows, 2 * m->hl, d, sa, st))) return rc;
+            EpiArgs ra = base_args(m, rows, d);
+            ra.out = m->trunk;
+            ra.ld_out = d;
+            ra.bias = lead ? ly.b_d : nullptr;
+            if ((rc = project_rows(m, "down", out_mode, m->act, ly.wd, r0, rows, d, m->hl, ra, st))) return rc;
+            if ((rc = exchange(k, done_d[k]))) return rc;
+        }
+    }
+    for (int k = 0; k < nch; ++k) LLAMA_CUDA_TRY(cudaStreamWaitEvent(st, done_d[k], 0));
+    return LLAMA_OK;
+}
+
+// The blocks of a prefill: the shard schedule under tensor parallelism.
+int prefill_blocks(llama_model* m, int B, int S, cudaStream_t st) {
+    if (m->tp > 1) return run_blocks_tp(m, B, S, st);
+    return run_blocks(m, B, S, false, st);
 }
 
 int run_head(llama_model* m, const float* x, int n, float* logits, bool decode, cudaStream_t st) {
@@ -744,9 +897,28 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
     m->graph = nullptr;
     m->graph_B = 0;
     m->graph_kernels = 0;
+    m->tp = tp_of(cfg);
+    m->tp_rank = m->tp > 1 ? cfg->tp_rank : 0;
+    m->Hl = heads_local(cfg);
+    m->Hkvl = kv_local(cfg);
+    m->hl = hidden_local(cfg);
+    m->ar_fn = nullptr;
+    m->ar_ctx = nullptr;
+    m->ar_chunks = 1;
+    m->comm = nullptr;
+    m->cap_stream = nullptr;
     if (cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
         delete m;
         return LLAMA_ERR_CUDA;
+    }
+    if (m->tp > 1) {
+        bool ok = cudaStreamCreateWithFlags(&m->comm, cudaStreamNonBlocking) == cudaSuccess;
+        m->tp_ev.assign(3 * TP_MAX_CHUNKS, nullptr);
+        for (auto& e : m->tp_ev) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) {
+            llama_free(m);
+            return LLAMA_ERR_CUDA;
+        }
     }
     const int dt = cfg->dtype;
     const int d = cfg->d_model, h = m->cfg.ffn_hidden, V = cfg->vocab;
@@ -761,36 +933,47 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
     TRY(launch_init_matrix(dt, m->embed, d, V, V, 0, 0, 1, seed, TID_EMBED, sc, st));
     TRY(launch_init_matrix(dt, m->head, d, V, V, 0, 0, 0, seed, TID_HEAD, sc, st));
     TRY(launch_fill_f32(m->g_final, 1.0f, d, st));
+    // A shard holds slices of the full matrices: query / key / value
+    // columns of its heads, the matching input rows of Wo, and the gate / up
+    // columns and Wdown input rows of its hidden units (r = 0, T = 1: all).
+    const int r = m->tp_rank;
+    const int kvd = kv_heads(cfg) * cfg->head_dim;        // full key/value width
+    const int dql = m->Hl * cfg->head_dim;                // this shard's query, key/value and hidden widths
+    const int kvl = m->Hkvl * cfg->head_dim;
+    const int hl = m->hl;
     for (int l = 0; l < cfg->n_layers; ++l) {
         const Layer& ly = m->layers[l];
-        const int kvd = kv_heads(cfg) * cfg->head_dim;   // K and V rows follow the d rows of Q
-        TRY(launch_init_matrix(dt, ly.wqkv, d, d, d, 0, 0, 0, seed, layer_tid(l, 0), sc, st));
-        TRY(launch_init_matrix(dt, ly.wqkv, d, kvd, kvd, 0, d, 0, seed, layer_tid(l, 1), sc, st));
-        TRY(launch_init_matrix(dt, ly.wqkv, d, kvd, kvd, 0, d + kvd, 0, seed, layer_tid(l, 2), sc, st));
-        TRY(launch_init_matrix(dt, ly.wo, d, d, d, 0, 0, 0, seed, layer_tid(l, 3), sc, st));
-        TRY(launch_init_matrix(dt, ly.wgu, d, h, 128, 256, 0, 0, seed, layer_tid(l, 4), sc, st));
-        TRY(launch_init_matrix(dt, ly.wgu, d, h, 128, 256, 128, 0, seed, layer_tid(l, 5), sc, st));
-        TRY(launch_init_matrix(dt, ly.wd, h, d, d, 0, 0, 0, seed, layer_tid(l, 6), sc, st));
+        // W_qkv rows: the shard's Q columns, then its K, then its V
+        TRY(launch_init_shard(dt, ly.wqkv, d, d, 0, d, r * dql, dql, dql, 0, 0, 0, seed, layer_tid(l, 0), sc, st));
+        TRY(launch_init_shard(dt, ly.wqkv, d, kvd, 0, d, r * kvl, kvl, kvl, 0, dql, 0, seed, layer_tid(l, 1), sc,
+                              st));
+        TRY(launch_init_shard(dt, ly.wqkv, d, kvd, 0, d, r * kvl, kvl, kvl, 0, dql + kvl, 0, seed, layer_tid(l, 2),
+                              sc, st));
+        TRY(launch_init_shard(dt, ly.wo, d, d, r * dql, dql, 0, d, d, 0, 0, 0, seed, layer_tid(l, 3), sc, st));
+        TRY(launch_init_shard(dt, ly.wgu, d, h, 0, d, r * hl, hl, 128, 256, 0, 0, seed, layer_tid(l, 4), sc, st));
+        TRY(launch_init_shard(dt, ly.wgu, d, h, 0, d, r * hl, hl, 128, 256, 128, 0, seed, layer_tid(l, 5), sc, st));
+        TRY(launch_init_shard(dt, ly.wd, h, d, r * hl, hl, 0, d, d, 0, 0, 0, seed, layer_tid(l, 6), sc, st));
         TRY(launch_fill_f32(ly.g_attn, 1.0f, d, st));
         TRY(launch_fill_f32(ly.g_ffn, 1.0f, d, st));
         if (cfg->bias) {
-            // vectors of the bias variant: the generator with K = 1 (element j of the vector)
-            auto vec = [&](float* dst, int n, int blk, int blk_stride, int row_off, int k) {
-                return launch_init_matrix(LLAMA_F32, dst, 1, n, blk, blk_stride, row_off, 0, seed, bias_tid(l, k), sc,
-                                          st);
+            // vectors of the bias variant: the generator with K = 1 (element j of
+            // the vector); a shard holds the slice of the biases of its columns
+            auto vec = [&](float* dst, int n_full, int n0, int n_loc, int blk, int blk_stride, int row_off, int k) {
+                return launch_init_shard(LLAMA_F32, dst, 1, n_full, 0, 1, n0, n_loc, blk, blk_stride, row_off, 0, seed,
+                                         bias_tid(l, k), sc, st);
             };
-            TRY(vec(ly.b_qkv, d, d, 0, 0, 0));
-            TRY(vec(ly.b_qkv, kvd, kvd, 0, d, 1));
-            TRY(vec(ly.b_qkv, kvd, kvd, 0, d + kvd, 2));
-            TRY(vec(ly.b_o, d, d, 0, 0, 3));
-            TRY(vec(ly.b_gu, h, 128, 256, 0, 4));
-            TRY(vec(ly.b_gu, h, 128, 256, 128, 5));
-            TRY(vec(ly.b_d, d, d, 0, 0, 6));
-            TRY(vec(ly.beta_attn, d, d, 0, 0, 7));
-            TRY(vec(ly.beta_ffn, d, d, 0, 0, 8));
+            TRY(vec(ly.b_qkv, d, r * dql, dql, dql, 0, 0, 0));
+            TRY(vec(ly.b_qkv, kvd, r * kvl, kvl, kvl, 0, dql, 1));
+            TRY(vec(ly.b_qkv, kvd, r * kvl, kvl, kvl, 0, dql + kvl, 2));
+            TRY(vec(ly.b_o, d, 0, d, d, 0, 0, 3));
+            TRY(vec(ly.b_gu, h, r * hl, hl, 128, 256, 0, 4));
+            TRY(vec(ly.b_gu, h, r * hl, hl, 128, 256, 128, 5));
+            TRY(vec(ly.b_d, d, 0, d, d, 0, 0, 6));
+            TRY(vec(ly.beta_attn, d, 0, d, d, 0, 0, 7));
+            TRY(vec(ly.beta_ffn, d, 0, d, d, 0, 0, 8));
             // decode step: W (g x / rms + beta) + b = W (g x) / rms + (b + W beta)
-            TRY(launch_bias_fold(dt, ly.wqkv, d + 2 * kvd, d, ly.beta_attn, ly.b_qkv, ly.c_qkv, st));
-            TRY(launch_bias_fold(dt, ly.wgu, 2 * h, d, ly.beta_ffn, ly.b_gu, ly.c_gu, st));
+            TRY(launch_bias_fold(dt, ly.wqkv, dql + 2 * kvl, d, ly.beta_attn, ly.b_qkv, ly.c_qkv, st));
+            TRY(launch_bias_fold(dt, ly.wgu, 2 * hl, d, ly.beta_ffn, ly.b_gu, ly.c_gu, st));
         }
     }
     // RoPE table: angle = pos * theta^(-2i/hd), cos and sin in fp64, stored fp32
@@ -841,6 +1024,7 @@ static int prefill_impl(llama_model* m, const int32_t* d_tokens, int32_t B, int3
     if (h_lens)
         for (int b = 0; b < B; ++b)
             if (h_lens[b] < 1 || h_lens[b] > S) return LLAMA_ERR_INVALID_ARG;
+    if (m->tp > 1 && !m->ar_fn) return LLAMA_ERR_STATE;   // a shard needs its exchange
     const int n = B * S;
     const int V = m->cfg.vocab;
     int rc;
@@ -849,7 +1033,7 @@ static int prefill_impl(llama_model* m, const int32_t* d_tokens, int32_t B, int3
         rc = launch_embed(m->cfg.dtype, d_tokens, m->embed, m->trunk, n, m->cfg.d_model, V, m->d_err, st);
     }
     if (rc) return rc;
-    if ((rc = run_blocks(m, B, S, false, st))) return rc;
+    if ((rc = prefill_blocks(m, B, S, st))) return rc;
     // positions: where each sequence continues
     if (h_lens) {
         LLAMA_CUDA_TRY(cudaMemcpyAsync(m->d_pos, h_lens, (size_t)B * 4, cudaMemcpyHostToDevice, st));
@@ -895,8 +1079,9 @@ int llama_prefill_trunk(llama_model* m, const float* d_x, int32_t B, int32_t S, 
         return LLAMA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     const size_t bytes = (size_t)B * S * m->cfg.d_model * 4;
+    if (m->tp > 1 && !m->ar_fn) return LLAMA_ERR_STATE;
     if (d_x != m->trunk) LLAMA_CUDA_TRY(cudaMemcpyAsync(m->trunk, d_x, bytes, cudaMemcpyDeviceToDevice, st));
-    int rc = run_blocks(m, B, S, false, st);
+    int rc = prefill_blocks(m, B, S, st);
     if (rc) return rc;
     if (d_y != m->trunk) LLAMA_CUDA_TRY(cudaMemcpyAsync(d_y, m->trunk, bytes, cudaMemcpyDeviceToDevice, st));
     launch_pdl(pos_set_kernel, dim3(1), dim3(32), 0, st, m->d_pos, (int)S, (int)B);
@@ -908,7 +1093,7 @@ int llama_prefill_trunk(llama_model* m, const float* d_x, int32_t B, int32_t S, 
 }
 
 int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t* d_next, float* d_logits, void* stream) {
-    if (!m || !d_tokens) return LLAMA_ERR_INVALID_ARG;
+    if (!m || !d_tokens || m->tp > 1) return LLAMA_ERR_INVALID_ARG;
     if (m->B <= 0 || m->cur_len >= m->cfg.max_seq) return LLAMA_ERR_STATE;
     cudaStream_t st = (cudaStream_t)stream;
     int rc = ensure_graph(m);
@@ -925,7 +1110,7 @@ int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t* d_next, 
 }
 
 int llama_generate(llama_model* m, const int32_t* d_first, int32_t n_steps, int32_t* d_out, void* stream) {
-    if (!m || !d_out || n_steps < 0) return LLAMA_ERR_INVALID_ARG;
+    if (!m || !d_out || n_steps < 0 || m->tp > 1) return LLAMA_ERR_INVALID_ARG;
     if (m->B <= 0 || m->cur_len + n_steps > m->cfg.max_seq) return LLAMA_ERR_STATE;
     cudaStream_t st = (cudaStream_t)stream;
     int rc = ensure_graph(m);
@@ -939,6 +1124,28 @@ int llama_generate(llama_model* m, const int32_t* d_first, int32_t n_steps, int3
         m->cur_len += 1;
         for (int& p : m->pos_h) p += 1;
     }
+    return LLAMA_OK;
+}
+
+int llama_set_allreduce(llama_model* m, llama_allreduce_fn fn, void* ctx, int32_t chunks) {
+    if (!m || !fn || chunks < 1 || chunks > TP_MAX_CHUNKS || m->tp <= 1) return LLAMA_ERR_INVALID_ARG;
+    m->ar_fn = fn;
+    m->ar_ctx = ctx;
+    m->ar_chunks = chunks;
+    return LLAMA_OK;
+}
+
+int llama_tp_shard(const llama_config* cfg, int32_t* h_out) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if (!h_out) return LLAMA_ERR_INVALID_ARG;
+    const int r = tp_of(cfg) > 1 ? cfg->tp_rank : 0;
+    h_out[0] = r * heads_local(cfg);
+    h_out[1] = heads_local(cfg);
+    h_out[2] = r * kv_local(cfg);
+    h_out[3] = kv_local(cfg);
+    h_out[4] = r * hidden_local(cfg);
+    h_out[5] = hidden_local(cfg);
     return LLAMA_OK;
 }
 
@@ -965,7 +1172,7 @@ int llama_rewind(llama_model* m, int32_t position, void* stream) {
 int llama_complete(llama_model* m, const int32_t* h_tokens, int32_t B, int32_t S, float* d_logits, int32_t n_steps,
                    int32_t* h_out, void* stream) {
     if (!m || !h_tokens || !h_out || B <= 0 || S <= 0 || n_steps < 0 || B > m->cfg.max_batch ||
-        S + n_steps > m->cfg.max_seq)
+        S + n_steps > m->cfg.max_seq || m->tp > 1)
         return LLAMA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     const llama_config& c = m->cfg;
@@ -990,13 +1197,14 @@ int llama_complete(llama_model* m, const int32_t* h_tokens, int32_t B, int32_t S
 int llama_model_tensor(const llama_model* m, const char* name, int32_t layer, void** d_ptr, uint64_t* bytes) {
     if (!m || !name || !d_ptr || !bytes) return LLAMA_ERR_INVALID_ARG;
     const llama_config& c = m->cfg;
-    const size_t d = c.d_model, h = c.ffn_hidden, V = c.vocab, es = m->esz;
+    const size_t d = c.d_model, h = m->hl, V = c.vocab, es = m->esz;   // h, dq: this shard's widths
+    const size_t dq = (size_t)m->Hl * c.head_dim;
     const size_t nmax = (size_t)c.max_batch * c.max_seq;
     auto lay = [&](int l) -> const Layer* { return (l >= 0 && l < c.n_layers) ? &m->layers[l] : nullptr; };
     if (!strcmp(name, "kv")) { *d_ptr = m->kv; *bytes = 2 * (size_t)c.n_layers * m->kv_layer_elems * es; }
     else if (!strcmp(name, "trunk")) { *d_ptr = m->trunk; *bytes = nmax * d * 4; }
-    else if (!strcmp(name, "q")) { *d_ptr = m->q; *bytes = nmax * d * es; }
-    else if (!strcmp(name, "attn")) { *d_ptr = m->attn; *bytes = nmax * d * es; }
+    else if (!strcmp(name, "q")) { *d_ptr = m->q; *bytes = nmax * dq * es; }
+    else if (!strcmp(name, "attn")) { *d_ptr = m->attn; *bytes = nmax * dq * es; }
     else if (!strcmp(name, "xn")) { *d_ptr = m->xn; *bytes = nmax * d * es; }
     else if (!strcmp(name, "act")) { *d_ptr = m->act; *bytes = nmax * h * es; }
     else if (!strcmp(name, "embed")) { *d_ptr = m->embed; *bytes = V * d * es; }
@@ -1007,9 +1215,9 @@ int llama_model_tensor(const llama_model* m, const char* name, int32_t layer, vo
         if (!ly) return LLAMA_ERR_INVALID_ARG;
         if (!strcmp(name, "wqkv")) {
             *d_ptr = ly->wqkv;
-            *bytes = (d + 2 * (size_t)kv_heads(&c) * c.head_dim) * d * es;
+            *bytes = (dq + 2 * (size_t)m->Hkvl * c.head_dim) * d * es;
         }
-        else if (!strcmp(name, "wo")) { *d_ptr = ly->wo; *bytes = d * d * es; }
+        else if (!strcmp(name, "wo")) { *d_ptr = ly->wo; *bytes = d * dq * es; }
         else if (!strcmp(name, "wgu")) { *d_ptr = ly->wgu; *bytes = 2 * h * d * es; }
         else if (!strcmp(name, "wd")) { *d_ptr = ly->wd; *bytes = d * h * es; }
         else return LLAMA_ERR_INVALID_ARG;
@@ -1031,6 +1239,9 @@ void llama_free(llama_model* m) {
     if (!m) return;
     if (m->graph) cudaGraphExecDestroy(m->graph);
     if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
+    for (cudaEvent_t e : m->tp_ev)
+        if (e) cudaEventDestroy(e);
+    if (m->comm) cudaStreamDestroy(m->comm);
     delete m;
 }
 

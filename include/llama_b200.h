@@ -88,6 +88,10 @@ typedef struct llama_config {
                             output width, each in-layer RMSNorm adds a shift after the
                             gain (none on the final norm and head); fp32, drawn like
                             the weights from tensor ids 2^20 + 16 l + k */
+    int32_t tp_size;     /* tensor parallelism: 0 or 1 = off; T > 1 = this model is one of
+                            T shards (see llama_set_allreduce).  n_heads, n_kv_heads and
+                            ffn_hidden / 128 must divide by T. */
+    int32_t tp_rank;     /* this shard, 0 <= tp_rank < T */
 } llama_config;
 
 typedef struct llama_model llama_model; /* opaque host handle */
@@ -187,6 +191,49 @@ LLAMA_API int llama_complete(llama_model* m, const int32_t* h_tokens, int32_t B,
  * per-layer weights.  Layouts are those of the arena described above. */
 LLAMA_API int llama_model_tensor(const llama_model* m, const char* name, int32_t layer,
                        void** d_ptr, uint64_t* bytes);
+
+/* ------------------------------------------------------- tensor parallel
+ * [KN] "LLaMA: Open and Efficient Foundation Language Models" knowledge
+ * note, "Efficient Training Implementation": the model is split across GPUs
+ * (model parallelism) and the all-reduce is hidden behind computation.
+ *
+ * Shard r of T holds query heads [r H/T, (r+1) H/T) and key/value heads
+ * [r Hkv/T, (r+1) Hkv/T) -- their columns of Wq, Wk, Wv, their rows of Wo
+ * (the attention features they produce) and their KV cache -- and FFN
+ * hidden units [r h/T, (r+1) h/T): their columns of Wgate and Wup and rows
+ * of Wdown.  Embedding, norms, head and the fp32 trunk are replicated.  The
+ * weights a shard holds are exactly the slices of the full model's (same
+ * generator, same element indices).  In each block the O and down
+ * projections of a shard produce a partial sum of the full product; shard 0
+ * adds its partial (and the bias variant's output bias) to the trunk, the
+ * others write theirs in its place, and one all-reduce (sum) over the
+ * shards then leaves the new trunk on every shard:
+ *     x' = x + sum_r attn_r Wo_r,    y = x' + sum_r act_r Wdown_r.
+ * Prefill (llama_prefill, llama_prefill_ragged, llama_prefill_trunk) runs
+ * this way; decoding is not sharded (the decode entry points return
+ * LLAMA_ERR_INVALID_ARG on a shard). */
+
+/* Sum all-reduce of `count` floats at d_buf across the T shards, in place,
+ * queued on `stream` (a cudaStream_t): every shard's d_buf must hold the
+ * element-wise sum once the work queued on `stream` completes, identical on
+ * every shard.  Return 0, or non-zero to abort the calling entry point with
+ * LLAMA_ERR_CUDA.  Called from the host thread that made the entry-point
+ * call, once per row chunk and exchange point (2 per block). */
+typedef int (*llama_allreduce_fn)(float* d_buf, uint64_t count, void* stream, void* ctx);
+
+/* Installs the exchange of a shard (tp_size > 1): `fn` with `ctx` is called
+ * for each all-reduce.  `chunks` (1..16) splits the token rows of every
+ * projection after attention into that many blocks (multiples of 128 rows):
+ * the all-reduce of block c, queued on a stream of the model's own, runs
+ * while the projections of block c + 1 compute, and the next sublayer's
+ * norm and projection of block c start as soon as block c's all-reduce is
+ * done.  Host-only. */
+LLAMA_API int llama_set_allreduce(llama_model* m, llama_allreduce_fn fn, void* ctx, int32_t chunks);
+
+/* The slices shard cfg->tp_rank of cfg->tp_size holds, into h_out (host
+ * int32 [6]): first query head, query heads, first key/value head,
+ * key/value heads, first FFN hidden unit, FFN hidden units.  Host-only. */
+LLAMA_API int llama_tp_shard(const llama_config* cfg, int32_t* h_out);
 
 /* Reads (synchronously) and clears the sticky device error word that
  * bounded device waits set; returns LLAMA_OK or LLAMA_ERR_TIMEOUT. */

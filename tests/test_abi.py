@@ -7,7 +7,7 @@ import pytest
 
 import decoder_only_b200 as lb
 import oracle
-from synth.workloads import PRESETS, TINY, LLAMA_7B, LLAMA_13B
+from synth.workloads import PRESETS, TINY, LLAMA_7B, LLAMA_13B, LLAMA_65B_SLICE
 
 
 def test_every_declared_symbol_is_exported():
@@ -113,3 +113,45 @@ def test_code_hash_ignores_comments_not_code(tmp_path):
     c.write_text('int f(int x) {\n  return 3 * x;\n}\nconst char* s = "// kept";\n')
     assert bench.code_hash(str(a)) == bench.code_hash(str(b))
     assert bench.code_hash(str(a)) != bench.code_hash(str(c))
+
+
+# ------------------------------------------------------------------ tensor parallel (host logic)
+
+@pytest.mark.parametrize("shape,T", [(LLAMA_7B, 2), (LLAMA_13B, 2), (LLAMA_13B, 4), (LLAMA_7B.with_(n_kv_heads=8), 2),
+                                     (LLAMA_65B_SLICE, 4)])
+def test_tp_shards_partition_heads_and_hidden_units(shape, T):
+    """Every query head, key/value head and FFN hidden unit belongs to
+    exactly one shard, in contiguous rank-ordered slices."""
+    if True:
+        sh = [lb.tp_shard(shape, r, T) for r in range(T)]
+        for key0, key, total in (("head0", "heads", shape.n_heads), ("kv_head0", "kv_heads", shape.kv_heads),
+                                 ("hidden0", "hidden", shape.ffn_hidden)):
+            assert [s[key0] for s in sh] == [r * total // T for r in range(T)]
+            assert all(s[key] == total // T for s in sh)
+
+
+def test_tp_shard_holds_its_slice_of_the_weights_and_cache():
+    """A shard's arena is the unsharded one minus (T - 1) / T of the sharded
+    weights (Q, K, V, O, gate, up, down) and of the KV cache."""
+    s = LLAMA_7B.with_(n_layers=2)
+    B, S = 4, 128
+    full = lb.model_bytes(lb.make_config(s, B, S))
+    half = lb.model_bytes(lb.make_config(s, B, S, tp=(1, 2)))
+    d, h, L = s.d_model, s.ffn_hidden, s.n_layers
+    sharded = 2 * L * (4 * d * d + 3 * d * h) + 2 * 2 * L * B * S * d          # bf16 bytes
+    act = B * S * (2 * d + h) * 2                                              # q, attention output, SwiGLU act
+    saved = full - half
+    # beyond that: the decode step's split-K partial regions, sized by the widths the model holds
+    assert sharded // 2 <= saved <= sharded // 2 + act // 2 + (1 << 20)
+
+
+@pytest.mark.parametrize("tp", [(0, 3), (2, 2), (-1, 2), (1, 1), (0, 256), (0, 4)])
+def test_tp_configs_that_do_not_divide_are_rejected(tp):
+    # 7B: 32 heads, 11008 = 86 blocks of 128 hidden units: 4 shards would split a block
+    n = ctypes.c_uint64()
+    cfg = lb.make_config(LLAMA_7B.with_(n_layers=1), 4, 128, tp=tp)
+    assert lb.lib.llama_model_bytes(ctypes.byref(cfg), ctypes.byref(n)) == -1
+
+
+def test_tp_exchange_is_rejected_on_an_unsharded_model_handle():
+    assert lb.lib.llama_set_allreduce(None, lb.ALLREDUCE_FN(lambda *a: 0), None, 4) == -1
