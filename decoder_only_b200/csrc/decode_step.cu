@@ -69,16 +69,6 @@ static_assert(NAW == 6, "warp roles");
 constexpr int ACH = 16;      // keys per attention chunk (one bulk copy of K rows, one of V rows)
 constexpr int AMX = 2048;    // logits per greedy-choice item
 constexpr int SSQ_BLOCKS = 64;   // 128-feature blocks of one norm's sums of squares (d <= 8192)
-// L2 prefetch distances: weight tiles ahead of the ring's newest request, and
-// attention chunks ahead of a warp's newest chunk copy (0: none)
-#ifndef LLAMA_STEP_PF_W
-#define LLAMA_STEP_PF_W 0
-#endif
-#ifndef LLAMA_STEP_PF_A
-#define LLAMA_STEP_PF_A 0
-#endif
-constexpr int PF_W = LLAMA_STEP_PF_W;
-constexpr int PF_A = LLAMA_STEP_PF_A;
 
 enum PhaseType { PH_EMBED = 0, PH_QKV = 1, PH_ATTN = 2, PH_O = 3, PH_GU = 4, PH_DOWN = 5, PH_HEAD = 6, PH_ARGMAX = 7 };
 
@@ -536,17 +526,6 @@ __device__ __forceinline__ void attn_issue(const StepArgs& a, int l, int pr, int
                      : "memory");
 }
 
-// L2 prefetch of chunk kc's key and value rows (cache row kvr)
-template <int HD>
-__device__ __forceinline__ void attn_prefetch(const StepArgs& a, int l, int kvr, int kc, int len) {
-    const int k0 = kc * ACH;
-    const uint32_t bytes = (uint32_t)(min(len - k0, ACH) * HD * 2);
-    const bf16* kc_ = a.kv + (size_t)(2 * l) * a.kv_layer;
-    const size_t off = ((size_t)kvr * a.smax + k0) * HD;
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kc_ + off), "r"(bytes) : "memory");
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kc_ + a.kv_layer + off), "r"(bytes) : "memory");
-}
-
 // Attention of layer l for attention warp aw of this CTA (0..NAW-1).
 template <int BN, int HD>
 __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Smem<BN, HD>& sm, uint32_t* uses,
@@ -616,23 +595,15 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
     // stores wrote before
     if (lane == 0) asm volatile("fence.proxy.async.global;\n\tfence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
-    // issue cursor, and the prefetch cursor PF_A chunks ahead of it
+    // issue cursor
     long long ic = cs;
     Pos iq = locate(cs);
-    long long fc = cs + PF_A;
-    Pos fq = iq;
-    if (PF_A > 0 && fc < ce) fq = locate(fc);
     auto issue = [&](int buf) {
         if (lane == 0)
             attn_issue<BN, HD>(a, l, iq.b * a.H + iq.h, iq.kvr, iq.kc, ic == cs || iq.kc == 0, iq.len,
                                wbuf + buf * C::ATT_BUF, wbar + 8 * buf);
         ++ic;
         advance(iq);
-        if (PF_A > 0 && fc < ce) {
-            if (lane == 0) attn_prefetch<HD>(a, l, fq.kvr, fq.kc, fq.len);
-            ++fc;
-            advance(fq);
-        }
     };
     issue(0);
     if (ic < ce) issue(1);
@@ -983,11 +954,9 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
         // as soon as a ring slot frees; the activation tile of a stage only
         // once the completion count its phase reads after is complete.
         if (lane == 0) {
-            Cursor wc, xc, pc;
+            Cursor wc, xc;
             cursor_seek(a, P, wc, 0);
             xc = wc;
-            pc = wc;
-            for (int j = 0; j < PF_W && pc.valid; ++j) cursor_next(a, P, pc);   // PF_W tiles ahead
             int wn = 0, xn = 0, ready = -1;
             const uint64_t wpol = l2_evict_first();   // a weight tile is read once per step
             // the embedding (and the reset of the completion counts) first
@@ -1003,10 +972,6 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                                          wc.mb * BM, wpol);
                         ++wn;
                         cursor_next(a, P, wc);
-                        if (PF_W > 0 && pc.valid) {
-                            tma_prefetch_2d(a.maps + pc.map_a, pc.kb * BK, pc.mb * BM);
-                            cursor_next(a, P, pc);
-                        }
                         prog = true;
                     }
                 }
