@@ -13,16 +13,25 @@
 //               once O_j is, so K runs ahead of V).  3-D tensor maps (hd,
 //               position, head) make rows >= S read as 0.
 //   warp 1      TMEM allocator + MMA issuer:
-//                 S_j = Q K_j^T   (M 128, N 128, K hd)  -> TMEM S[j % 2]
-//                 O_j = P_j V_j   (M 128, N hd, K 128)  -> TMEM O[j % 2]
+//                 S_j = Q K_j^T        (M 128, N 128, K hd)  -> TMEM S[j % 2]
+//                 O  += P_j V_j        (M 128, N hd, K 128)  -> TMEM O (one
+//                                       accumulator for the whole row tile)
 //               V is the MN-major B operand (hd contiguous), so the cache
 //               layout [position][hd] is used as is.
 //   warps 2..5  one query row per thread: row max of S_j (pass 1), then
-//               p = 2^((s - m) log2e / sqrt(hd)) rounded to bf16 into the
+//               p = 2^(s log2e / sqrt(hd) - m) rounded to bf16 into the
 //               shared P tile (128-byte swizzled, K-major) and the row sum
-//               (pass 2); one tile later O_{j-1} is read from TMEM and
-//               folded into the fp32 running output with the online-softmax
-//               correction exp(m_old - m_new).
+//               (pass 2), both passes on the row's 128 scores held in
+//               registers (one TMEM read per tile).  The running maximum m
+//               (log2 units) moves only when a tile's maximum exceeds it by
+//               more than 8: p stays <= 2^8, exact in fp32 and bf16's range,
+//               and the output in TMEM is rescaled by 2^(m_old - m_new) (TMEM
+//               load, scale, store, after the previous P V product) only
+//               then -- a few times per row -- instead of folding every
+//               tile's product into registers.  The pass is bound by the
+//               instructions it issues per score (one warp per sub-
+//               partition): one FMA, one ex2, half a pack, one add.
+//               After the last tile: O / (row sum), bf16, to global.
 // All mbarrier waits are bounded (see tcgen05.cuh).
 #include <cudaTypedefs.h>
 
@@ -37,6 +46,15 @@ using namespace tc;
 constexpr int BQ = 128;         // queries per tile
 constexpr int BKV = 128;        // keys per tile
 constexpr int NTHREADS = 192;
+constexpr float RESCALE_LOG2 = 8.f;   // move the running maximum only by more than this (log2 units)
+
+// 2^x by the special-function unit's approximation (one instruction;
+// relative error far below bf16's 2^-9; 2^-inf = 0 for masked scores)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 template <int HD>
 struct ACfg {
@@ -50,7 +68,7 @@ struct ACfg {
     static constexpr int OFF_P = OFF_V + 2 * TILE;           // [2]
     static constexpr int OFF_BAR = OFF_P + 2 * P_TILE;
     static constexpr int SMEM = OFF_BAR + 256 + 1024;
-    static constexpr uint32_t TMEM_COLS = 512;               // S[2] at 0, 128; O[2] at 256, 384
+    static constexpr uint32_t TMEM_COLS = 512;               // S[2] at 0, 128; O at 256
 };
 
 // P tile position of 8 consecutive keys (one 16-byte chunk) of query row t:
@@ -80,8 +98,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t s_full = bars + 56;       // [2]
     const uint32_t s_empty = bars + 72;      // [2]
     const uint32_t p_full = bars + 88;       // [2]
-    const uint32_t o_full = bars + 104;      // [2]
-    const uint32_t o_empty = bars + 120;     // [2]
+    const uint32_t o_done = bars + 104;      // one phase per completed P V product
+    const uint32_t o_last = bars + 112;      // the last P V product
     const uint32_t v_empty = bars + 136;     // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 160);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -105,9 +123,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(s_full + 8 * i, 1);
             mbar_init(s_empty + 8 * i, 128);
             mbar_init(p_full + 8 * i, 128);
-            mbar_init(o_full + 8 * i, 1);
-            mbar_init(o_empty + 8 * i, 128);
         }
+        mbar_init(o_done, 1);
+        mbar_init(o_last, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -188,26 +206,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     umma_commit(k_empty + 8 * st);
                 }
                 if (j > 0) {
+                    // P_jj is complete (and O rescaled where a row's maximum moved)
                     const int jj = j - 1, st = jj & 1;
                     const uint32_t par = (jj >> 1) & 1;
                     if (!mbar_wait(p_full + 8 * st, par, abort_flag, err) ||
-                        !mbar_wait(v_full + 8 * st, par, abort_flag, err) ||
-                        !mbar_wait(o_empty + 8 * st, par ^ 1u, abort_flag, err)) {
+                        !mbar_wait(v_full + 8 * st, par, abort_flag, err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t d_o = tmem + 256u + (uint32_t)(st * 128);
+                    const uint32_t d_o = tmem + 256u;
 #pragma unroll
                     for (int kk = 0; kk < BKV / 16; ++kk) {
                         // A = P (K-major, keys contiguous); B = V (MN-major): 16 keys = 2 groups of 8 rows
                         const uint32_t poff = (kk >> 2) * C::REG + (kk & 3) * 32;
                         uint64_t vd = sw128_desc(sV + st * C::TILE + kk * 2048);
                         vd = (vd & ~(((uint64_t)0x3FFF) << 16)) | ((uint64_t)(C::REG >> 4) << 16);   // LBO: next 64 hd
-                        umma_bf16(d_o, sw128_desc(sP + st * C::P_TILE + poff), vd, IDESC_PV, kk > 0 ? 1u : 0u);
+                        umma_bf16(d_o, sw128_desc(sP + st * C::P_TILE + poff), vd, IDESC_PV,
+                                  (jj > 0 || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit(o_full + 8 * st);
+                    umma_commit(o_done);
                     umma_commit(v_empty + 8 * st);
+                    if (jj == n_kv - 1) umma_commit(o_last);
                 }
             }
         }
@@ -217,114 +237,121 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int t = quarter * 32 + lane;               // query row within the tile
         const int q = q0 + t;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        float o[HD];
-#pragma unroll
-        for (int i = 0; i < HD; ++i) o[i] = 0.f;
-        float m = -INFINITY, l = 0.f, corr_prev = 0.f;
+        const uint32_t o_addr = tmem + lane_addr + 256u;
+        float m = -INFINITY, l = 0.f;                    // running maximum (log2 units) and row sum
         bool ok = true;
-        for (int j = 0; j <= n_kv; ++j) {
-            float corr = 0.f;
-            if (j < n_kv) {
-                const int st = j & 1;
-                const uint32_t par = (j >> 1) & 1;
-                if (!mbar_wait(s_full + 8 * st, par, abort_flag, err)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t s_addr = tmem + lane_addr + (uint32_t)(st * 128);
-                // only the diagonal tile masks: there key k is visible iff
-                // k <= min(q, S - 1) (a select per score, no branch)
-                const bool diag = (j == n_kv - 1);
-                const int lim = min(q, S - 1) - j * BKV;
-                // pass 1: row maximum, eight independent partial maxima
-                float mx8[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float sv[32];
-                    tmem_ld32(s_addr + c * 32, sv);
-                    if (diag) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) sv[i] = (c * 32 + i <= lim) ? sv[i] : -INFINITY;
-                    }
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
-                }
-                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-                const float m_new = fmaxf(m, mx);
-                corr = (m == -INFINITY) ? 0.f : exp2f((m - m_new) * scale_log2);
-                const float mo = m_new * scale_log2;
-                // pass 2: probabilities (bf16) into the P tile, row sum of the
-                // rounded values in four independent partial sums
-                float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-                const uint32_t pbase = sP + st * C::P_TILE;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float sv[32];
-                    tmem_ld32(s_addr + c * 32, sv);
-                    if (diag) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) sv[i] = (c * 32 + i <= lim) ? sv[i] : -INFINITY;
-                    }
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float p0 = exp2f(fmaf(sv[2 * i], scale_log2, -mo));
-                        const float p1 = exp2f(fmaf(sv[2 * i + 1], scale_log2, -mo));
-                        pk[i] = pack_bf16x2(p0, p1);
-                        const float2 r = unpack_bf16x2(pk[i]);
-                        rs4[i & 3] += r.x + r.y;
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint32_t addr = p_chunk_addr(pbase, t, c * 4 + u);
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * u]),
-                                     "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
-                                     : "memory");
-                    }
-                }
-                const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-                tc_fence_before();
-                mbar_arrive(s_empty + 8 * st);
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                mbar_arrive(p_full + 8 * st);
-                l = l * corr + rs;
-                m = m_new;
+        for (int j = 0; j < n_kv; ++j) {
+            const int st = j & 1;
+            const uint32_t par = (j >> 1) & 1;
+            // warp-uniform decision: the TMEM loads below are warp-collective
+            if (!__all_sync(0xffffffffu, mbar_wait(s_full + 8 * st, par, abort_flag, err))) {
+                ok = false;
+                break;
             }
-            if (j > 0) {
-                const int jj = j - 1, st = jj & 1;
-                const uint32_t par = (jj >> 1) & 1;
-                if (!mbar_wait(o_full + 8 * st, par, abort_flag, err)) {
+            tc_fence_after();
+            const uint32_t s_addr = tmem + lane_addr + (uint32_t)(st * 128);
+            // the row's 128 scores, four TMEM loads in flight, one wait
+            float sv[128];
+            {
+                uint32_t* r = reinterpret_cast<uint32_t*>(sv);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) TMEM_LD_X32(s_addr + c * 32, (r + 32 * c));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            }
+            // only the diagonal tile masks: there key k is visible iff
+            // k <= min(q, S - 1) (a select per score, no branch)
+            if (j == n_kv - 1) {
+                const int lim = min(q, S - 1) - j * BKV;
+#pragma unroll
+                for (int i = 0; i < 128; ++i) sv[i] = (i <= lim) ? sv[i] : -INFINITY;
+            }
+            // pass 1: row maximum, eight independent partial maxima
+            float mx8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) mx8[u] = sv[u];
+#pragma unroll
+            for (int i = 8; i < 128; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            // the running maximum moves (and O is rescaled) only by more than RESCALE_LOG2
+            const float mt = mx * scale_log2;
+            float corr = 1.f;
+            bool rescale = false;
+            if (m == -INFINITY) {
+                m = mt;                                  // first tile: nothing accumulated yet
+            } else if (mt > m + RESCALE_LOG2) {
+                corr = ex2_approx(m - mt);
+                m = mt;
+                rescale = true;
+            }
+            // pass 2: probabilities (bf16) into the P tile; the row sum adds
+            // the fp32 values in four independent partial sums
+            float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint32_t pbase = sP + st * C::P_TILE;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {               // 16 chunks of 8 keys (16 bytes of P)
+                uint32_t pk[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float p0 = ex2_approx(fmaf(sv[8 * c + 2 * i], scale_log2, -m));
+                    const float p1 = ex2_approx(fmaf(sv[8 * c + 2 * i + 1], scale_log2, -m));
+                    pk[i] = pack_bf16x2(p0, p1);
+                    rs4[i] += p0 + p1;
+                }
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_chunk_addr(pbase, t, c)), "r"(pk[0]),
+                             "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                             : "memory");
+            }
+            const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+            tc_fence_before();
+            mbar_arrive(s_empty + 8 * st);
+            // a warp with a moved maximum rescales its 32 rows of O once the
+            // previous P V product is done.  Its completion is phase j - 1 of
+            // o_done: S_j's completion (waited for above) follows that of
+            // P_{j-2} V_{j-2}, and P_j V_j waits for this warp, so the
+            // barrier is in phase j - 1 or j here.
+            if (__any_sync(0xffffffffu, rescale)) {
+                bool w = mbar_wait(o_done, (uint32_t)((j - 1) & 1), abort_flag, err);
+                if (!__all_sync(0xffffffffu, w)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t o_addr = tmem + lane_addr + 256u + (uint32_t)(st * 128);
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < HD / 32; ++c) {
                     float ov[32];
                     tmem_ld32(o_addr + c * 32, ov);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], corr_prev, ov[i]);
+                    for (int i = 0; i < 32; ++i) ov[i] *= corr;
+                    tmem_st32(o_addr + c * 32, ov);
                 }
+                tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(o_empty + 8 * st);
             }
-            corr_prev = corr;
+            l = l * corr + rs;
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(p_full + 8 * st);
         }
-        if (ok && q < S) {
+        // the last P V product: O / l, bf16, to global
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_last, 0, abort_flag, err));
+        if (ok) {
+            tc_fence_after();
             const float inv = 1.f / l;
             bf16* dst = out + ((size_t)b * S + q) * ((size_t)H * HD) + (size_t)h * HD;
+#pragma unroll 1
+            for (int c = 0; c < HD / 32; ++c) {
+                float ov[32];
+                tmem_ld32(o_addr + c * 32, ov);
+                if (q < S) {
 #pragma unroll
-            for (int c = 0; c < HD / 8; ++c) {
-                uint4 w = make_uint4(pack_bf16x2(o[8 * c] * inv, o[8 * c + 1] * inv),
-                                     pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
-                                     pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
-                                     pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
-                *reinterpret_cast<uint4*>(dst + 8 * c) = w;
+                    for (int u = 0; u < 4; ++u) {
+                        uint4 w = make_uint4(pack_bf16x2(ov[8 * u] * inv, ov[8 * u + 1] * inv),
+                                             pack_bf16x2(ov[8 * u + 2] * inv, ov[8 * u + 3] * inv),
+                                             pack_bf16x2(ov[8 * u + 4] * inv, ov[8 * u + 5] * inv),
+                                             pack_bf16x2(ov[8 * u + 6] * inv, ov[8 * u + 7] * inv));
+                        *reinterpret_cast<uint4*>(dst + c * 32 + 8 * u) = w;
+                    }
+                }
             }
         }
     }
