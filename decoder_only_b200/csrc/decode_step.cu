@@ -268,11 +268,19 @@ __device__ bool wait_at_least(const unsigned* p, unsigned target, volatile int* 
     }
 }
 
-// One finished unit; the caller's fence makes the CTA's writes before it
-// (ordered by a CTA barrier) visible first
+// One finished unit: a release add, so the writes of the CTA (or warp) that
+// the caller's barrier ordered before it are visible to whoever acquires the
+// count (release is cumulative over what happened before it)
 __device__ __forceinline__ void count_done(unsigned* p) {
-    __threadfence();
-    atomicAdd(p, 1u);
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p) : "memory");
+}
+
+// Arrival at a split counter: releases the caller's (barrier-ordered) partial
+// writes and acquires the earlier arrivals', returns the previous value
+__device__ __forceinline__ int arrive_acq_rel(int* p) {
+    int prev;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(p) : "memory");
+    return prev;
 }
 
 // The completion count (and its complete value) that phase `type` of layer
@@ -330,6 +338,24 @@ __device__ __forceinline__ void splitk_sum(const float* p, int slots, int M, int
     constexpr int U = BN <= 16 ? 4 : 2;   // slots in flight per round (register budget)
 #pragma unroll
     for (int b = 0; b < BN; ++b) out[b] = 0.f;
+    if (M <= 4) {
+        // one float4 per slot: eight slots per round in flight, summed in slot order
+        for (int s0 = 0; s0 < slots; s0 += 8) {
+            float4 w[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                w[u] = (s0 + u < slots) ? __ldcg(reinterpret_cast<const float4*>(p + (size_t)(s0 + u) * Mp))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                out[0] += w[u].x;
+                out[1] += w[u].y;
+                out[2] += w[u].z;
+                out[3] += w[u].w;
+            }
+        }
+        return;
+    }
     int s = 0;
     for (; s + U <= slots; s += U) {
         float4 w[U][BN / 4];
@@ -398,13 +424,9 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
         if (tid == 0) {
             int* cnt = a.counters + a.cnt_off[w.g.kind] + (PAIR ? (mb >> 1) : mb);
             const int target = PAIR ? nseg_of(mb & ~1) + nseg_of(mb | 1) : nseg;
-            __threadfence();
-            const int prev = atomicAdd(cnt, 1);
+            const int prev = arrive_acq_rel(cnt);
             last = (prev == target - 1);
-            if (last) {
-                *cnt = 0;
-                __threadfence();
-            }
+            if (last) *cnt = 0;   // ready for the next step; published by this CTA's later release
         }
         if (!esync_any(last)) return;
     }
@@ -770,13 +792,9 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
         __syncwarp();
         int last = 0;
         if (lane == 0) {
-            __threadfence();
-            const int prev = atomicAdd(a.attn_cnt + pr, 1);
+            const int prev = arrive_acq_rel(a.attn_cnt + pr);
             last = (prev == nparts - 1);
-            if (last) {
-                a.attn_cnt[pr] = 0;
-                __threadfence();
-            }
+            if (last) a.attn_cnt[pr] = 0;   // published by this warp's later release
         }
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) continue;
