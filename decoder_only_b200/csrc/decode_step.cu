@@ -520,8 +520,8 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
 template <int BN, int HD>
 // Chunk kc of query pair pr = b * H + h, whose keys and values are cache row
 // kvr = b * Hkv + h / (H / Hkv).
-__device__ __forceinline__ void attn_issue(const StepArgs& a, int l, int pr, int kvr, int kc, bool with_q, int len,
-                                           uint32_t dst, uint32_t bar) {
+__device__ __forceinline__ void attn_issue_kv(const StepArgs& a, int l, int kvr, int kc, int len, uint32_t dst,
+                                              uint32_t bar, uint32_t extra_bytes, bool arrive) {
     const int k0 = kc * ACH;
     const int nkeys = min(len - k0, ACH);
     const bf16* kc_ = a.kv + (size_t)(2 * l) * a.kv_layer;
@@ -530,7 +530,11 @@ __device__ __forceinline__ void attn_issue(const StepArgs& a, int l, int pr, int
     const uint32_t bytes = (uint32_t)(nkeys * HD * 2);
     // cache rows are read once per step (per query head of a group): first out of L2
     const uint64_t pol = l2_evict_first();
-    mbar_expect_tx(bar, 2 * bytes + (with_q ? HD * 2 : 0));
+    if (arrive)
+        mbar_expect_tx(bar, 2 * bytes + extra_bytes);
+    else   // the barrier's one arrival comes later, with the query (or without it)
+        asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(2 * bytes)
+                     : "memory");
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
             "r"(dst),
@@ -541,11 +545,13 @@ __device__ __forceinline__ void attn_issue(const StepArgs& a, int l, int pr, int
             "r"(dst + ACH * HD * 2),
         "l"(vc + off), "r"(bytes), "r"(bar), "l"(pol)
         : "memory");
-    if (with_q)
-        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                         dst + SCfg<BN, HD>::ATT_Q),
-                     "l"(a.q + (size_t)pr * HD), "r"((uint32_t)(HD * 2)), "r"(bar)
-                     : "memory");
+}
+template <int BN, int HD>
+__device__ __forceinline__ void attn_issue_q(const StepArgs& a, int pr, uint32_t dst, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst + SCfg<BN, HD>::ATT_Q),
+                 "l"(a.q + (size_t)pr * HD), "r"((uint32_t)(HD * 2)), "r"(bar)
+                 : "memory");
 }
 
 // Attention of layer l for attention warp aw of this CTA (0..NAW-1).
@@ -574,7 +580,18 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
     const long long Ctot = (long long)a.H * __shfl_sync(0xffffffffu, incl, Bq - 1);
     const int Wp = (int)min((long long)gridDim.x * NAW, Ctot);
     const int gw = blockIdx.x * NAW + aw;
-    if (gw >= Wp) return true;
+    if (gw >= Wp) {
+        // no attention work here: still wait for this layer's QKV count, so
+        // that attention warps 6 and 7 arrive at the named barrier they share
+        // with the epilogue warps once per layer, never a layer ahead
+        int w = 1;
+        if (lane == 0) {
+            unsigned tgt = 0;
+            const unsigned* dp = dep_of(a, PH_ATTN, l, tgt);
+            w = wait_at_least(dp, tgt, abort_flag, a.err);
+        }
+        return __shfl_sync(0xffffffffu, w, 0) != 0;
+    }
     const long long cs = Ctot * gw / Wp, ce = Ctot * (gw + 1) / Wp;
     auto owner = [&](long long i) { return (int)(((i + 1) * Wp - 1) / Ctot); };
     // unit index -> (sequence b, head h, chunk kc) with b's length and chunk
@@ -611,24 +628,83 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
     };
     const uint32_t wbuf = smem_u32(sm.att) + aw * 2 * C::ATT_BUF;
     const uint32_t wbar = sm.abar + aw * 16;
-    // the cache rows and queries of this step were stored by other CTAs
-    // (generic proxy) before their completion counts; the bulk copies read
-    // them through the async proxy, and overwrite shared memory that generic
-    // stores wrote before
-    if (lane == 0) asm volatile("fence.proxy.async.global;\n\tfence.proxy.async.shared::cta;" ::: "memory");
-    __syncwarp();
     // issue cursor
     long long ic = cs;
     Pos iq = locate(cs);
     auto issue = [&](int buf) {
-        if (lane == 0)
-            attn_issue<BN, HD>(a, l, iq.b * a.H + iq.h, iq.kvr, iq.kc, ic == cs || iq.kc == 0, iq.len,
-                               wbuf + buf * C::ATT_BUF, wbar + 8 * buf);
+        if (lane == 0) {
+            const bool with_q = ic == cs || iq.kc == 0;
+            const uint32_t dst = wbuf + buf * C::ATT_BUF, bar = wbar + 8 * buf;
+            attn_issue_kv<BN, HD>(a, l, iq.kvr, iq.kc, iq.len, dst, bar, with_q ? HD * 2 : 0, true);
+            if (with_q) attn_issue_q<BN, HD>(a, iq.b * a.H + iq.h, dst, bar);
+        }
         ++ic;
         advance(iq);
     };
-    issue(0);
-    if (ic < ce) issue(1);
+    // The first two chunks' keys and values go out before this layer's QKV
+    // projection is complete, unless a chunk holds the position this step
+    // appends (its pair's last chunk): those rows were written by earlier
+    // steps.  Their query (and their one barrier arrival) follows once the
+    // QKV count is complete.  Shared memory first: its earlier generic
+    // writes (the epilogues' transpose buffer) before the async copies.
+    if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    bool early[2] = {false, false};
+    {
+        Pos eq = iq;
+        for (int k = 0; k < 2 && cs + k < ce; ++k) {
+            early[k] = eq.kc < eq.nch - 1;
+            if (early[k] && lane == 0)
+                attn_issue_kv<BN, HD>(a, l, eq.kvr, eq.kc, eq.len, wbuf + k * C::ATT_BUF, wbar + 8 * k, 0, false);
+            advance(eq);
+        }
+    }
+    // this layer's QKV projection complete (queries, and the newest keys and values)
+    {
+        int w = 1;
+        if (lane == 0) {
+            unsigned tgt = 0;
+            const unsigned* dp = dep_of(a, PH_ATTN, l, tgt);
+            w = wait_at_least(dp, tgt, abort_flag, a.err);
+        }
+        if (!__shfl_sync(0xffffffffu, w, 0)) {
+            // leave no early copy in flight: arrive, then wait (bounded) for the bytes
+            if (lane == 0)
+                for (int k = 0; k < 2; ++k)
+                    if (early[k]) {
+                        mbar_arrive(wbar + 8 * k);
+                        const uint64_t t0 = global_timer();
+                        while (!mbar_try_wait(wbar + 8 * k, uses[k] & 1u) &&
+                               global_timer() - t0 < WAIT_LIMIT_NS / 4) {
+                        }
+                        uses[k]++;
+                    }
+            __syncwarp();
+            return false;
+        }
+    }
+    // the queries and the newest cache rows of this step were stored by other
+    // CTAs (generic proxy) before their completion counts; the bulk copies
+    // read them through the async proxy
+    if (lane == 0) asm volatile("fence.proxy.async.global;" ::: "memory");
+    __syncwarp();
+    for (int k = 0; k < 2 && ic < ce; ++k) {
+        if (early[k]) {
+            if (lane == 0) {
+                const uint32_t dst = wbuf + k * C::ATT_BUF, bar = wbar + 8 * k;
+                if (ic == cs || iq.kc == 0) {
+                    mbar_expect_tx(bar, HD * 2);
+                    attn_issue_q<BN, HD>(a, iq.b * a.H + iq.h, dst, bar);
+                } else {
+                    mbar_arrive(bar);
+                }
+            }
+            ++ic;
+            advance(iq);
+        } else {
+            issue(k);
+        }
+    }
     const float scale = rsqrtf((float)HD);
     float m = -INFINITY, lsum = 0.f, acc[DPL], qv[DPL];
     Pos cq = locate(cs);
@@ -1104,7 +1180,8 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                 bool ok = true;
                 if (tid == 0) {
                     unsigned tgt = 0;
-                    const unsigned* dp = (type == PH_EMBED) ? nullptr : dep_of(a, type, l, tgt);
+                    // attention: each attention warp waits itself, after its first copies
+                    const unsigned* dp = (type == PH_EMBED || type == PH_ATTN) ? nullptr : dep_of(a, type, l, tgt);
                     if (dp) ok = wait_at_least(dp, tgt, abort_flag, a.err);
                     // the embedding (and the zeroed counts) before anything else
                     if (ok && p == 1) ok = wait_at_least(a.bar + SY_EMBED, E, abort_flag, a.err);
@@ -1231,16 +1308,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
         if (lane == 0) w = wait_at_least(a.bar + SY_EMBED, E, abort_flag, a.err);
         bool ok = __shfl_sync(0xffffffffu, w, 0) != 0;
         for (int l = 0; l < a.L; ++l) {
-            if (ok) {
-                w = 1;
-                if (lane == 0) {
-                    unsigned tgt = 0;
-                    const unsigned* dp = dep_of(a, PH_ATTN, l, tgt);
-                    w = wait_at_least(dp, tgt, abort_flag, a.err);
-                }
-                ok = __shfl_sync(0xffffffffu, w, 0) != 0;
-                if (ok) ok = phase_attn<BN, HD>(a, l, warp - 2, lane, sm, uses, abort_flag);
-            }
+            if (ok) ok = phase_attn<BN, HD>(a, l, warp - 2, lane, sm, uses, abort_flag);
             __syncwarp();
             asm volatile("bar.arrive 2, 192;" ::: "memory");
         }
