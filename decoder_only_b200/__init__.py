@@ -34,7 +34,8 @@ class LlamaConfig(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("ffn_hidden", ctypes.c_int32), ("vocab", ctypes.c_int32),
                 ("norm_eps", ctypes.c_float), ("rope_theta", ctypes.c_float), ("dtype", ctypes.c_int32),
                 ("max_batch", ctypes.c_int32), ("max_seq", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
-                ("bias", ctypes.c_int32), ("tp_size", ctypes.c_int32), ("tp_rank", ctypes.c_int32)]
+                ("bias", ctypes.c_int32), ("tp_size", ctypes.c_int32), ("tp_rank", ctypes.c_int32),
+                ("kv_pages", ctypes.c_int32)]
 
 
 # int (*)(float* d_buf, uint64_t count, void* stream, void* ctx): the exchange of a shard
@@ -70,6 +71,7 @@ def _load():
         "llama_op_last_error": [],
         "llama_set_allreduce": [P, ALLREDUCE_FN, P, I],
         "llama_tp_shard": [P, P],
+        "llama_set_pages": [P, P, I, I, P],
         "llama_rewind": [P, I, P],
         "llama_complete": [P, P, I, I, P, I, P, P],
         "llama_kernel_launches": [],
@@ -122,15 +124,16 @@ def _dt(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def make_config(shape, max_batch: int, max_seq: int, tp=None) -> LlamaConfig:
+def make_config(shape, max_batch: int, max_seq: int, tp=None, kv_pages: int = 0) -> LlamaConfig:
     """`shape`: any object with n_layers, d_model, n_heads, head_dim,
     ffn_hidden, vocab, dtype ('bf16' | 'f32'), norm_eps, rope_theta.
-    `tp`: (rank, size) of a tensor-parallel shard, or None."""
+    `tp`: (rank, size) of a tensor-parallel shard, or None.  `kv_pages`:
+    pages of 128 positions in a paged KV cache (0: contiguous)."""
     rank, size = tp if tp is not None else (0, 0)
     return LlamaConfig(shape.n_layers, shape.d_model, shape.n_heads, shape.head_dim, shape.ffn_hidden,
                        shape.vocab, shape.norm_eps, shape.rope_theta, BF16 if shape.dtype == "bf16" else F32,
                        max_batch, max_seq, int(getattr(shape, "n_kv_heads", 0) or 0),
-                       int(bool(getattr(shape, "bias", False))), size, rank)
+                       int(bool(getattr(shape, "bias", False))), size, rank, kv_pages)
 
 
 def tp_shard(shape, rank: int, size: int) -> dict:
@@ -190,9 +193,9 @@ def model_bytes(cfg: LlamaConfig) -> int:
 class Model:
     """One model in one device arena.  Weights are generated on the device."""
 
-    def __init__(self, shape, max_batch: int, max_seq: int, seed: int = 0, tp=None):
+    def __init__(self, shape, max_batch: int, max_seq: int, seed: int = 0, tp=None, kv_pages: int = 0):
         self.shape = shape
-        self.cfg = make_config(shape, max_batch, max_seq, tp)
+        self.cfg = make_config(shape, max_batch, max_seq, tp, kv_pages)
         nbytes = model_bytes(self.cfg)
         self.arena = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
         h = ctypes.c_void_p()
@@ -205,6 +208,14 @@ class Model:
         if self.h:
             lib.llama_free(self.h)
             self.h = None
+
+    def set_pages(self, table):
+        """Page table of a paged KV cache (llama_set_pages): table[b][p] is the
+        pool page of sequence b's positions 128 p .. 128 p + 127."""
+        rows = [list(map(int, r)) for r in table]
+        B, n = len(rows), len(rows[0])
+        flat = (ctypes.c_int32 * (B * n))(*[v for r in rows for v in r])
+        _check(lib.llama_set_pages(self.h, ctypes.cast(flat, ctypes.c_void_p), B, n, _stream()), "llama_set_pages")
 
     def set_allreduce(self, reduce, chunks: int = 4):
         """Installs the exchange of a tensor-parallel shard (llama_set_allreduce):

@@ -36,6 +36,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "kernels.h"
 #include "tcgen05.cuh"
 
@@ -83,7 +84,7 @@ template <int HD>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ out, int H, int S,
-                           int Hkv, float scale_log2, int* err) {
+                           int Hkv, float scale_log2, const int* __restrict__ pages, int pps, int* err) {
     using C = ACfg<HD>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -163,7 +164,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 mbar_expect_tx(full + 8 * st, C::TILE);
                 for (int r = 0; r < C::NREG; ++r)
-                    tma_load_3d(dst + st * C::TILE + r * C::REG, map, full + 8 * st, 64 * r, j * BKV, kv_head);
+                    // paged cache: key tile j is page pages[b][j] (KV_PAGE == BKV positions)
+                    tma_load_3d(dst + st * C::TILE + r * C::REG, map, full + 8 * st, 64 * r, pages ? 0 : j * BKV,
+                                pages ? __ldg(pages + b * pps + j) * Hkv + (kv_head - b * Hkv) : kv_head);
                 issued = j + 1;
             }
             if (!ok) {
@@ -414,7 +417,8 @@ int attention_tc_prepare() {
 }
 
 int launch_attention_prefill_tc(const void* q, const void* k, const void* v, void* o, int B, int H, int Hkv, int S,
-                                int hd, int kv_stride, int* err, cudaStream_t st) {
+                                int hd, int kv_stride, int* err, cudaStream_t st, const int* pages, int pps,
+                                int n_pages) {
     if (B <= 0 || S <= 0) return LLAMA_OK;
     if (hd != 64 && hd != 128) return LLAMA_ERR_INVALID_ARG;
     if (Hkv <= 0 || H % Hkv != 0) return LLAMA_ERR_INVALID_ARG;
@@ -424,18 +428,25 @@ int launch_attention_prefill_tc(const void* q, const void* k, const void* v, voi
     CUtensorMap mq, mk, mv;
     int rc;
     if ((rc = make_head_map(&mq, q, hd, S, S, B * H))) return rc;
-    if ((rc = make_head_map(&mk, k, hd, S, kv_stride, B * Hkv))) return rc;
-    if ((rc = make_head_map(&mv, v, hd, S, kv_stride, B * Hkv))) return rc;
+    if (pages) {
+        // the page pool [page][Hkv][KV_PAGE][hd]: one (page, head) slab per z coordinate
+        static_assert(KV_PAGE == BKV, "a key tile is one page");
+        if ((rc = make_head_map(&mk, k, hd, KV_PAGE, KV_PAGE, n_pages * Hkv))) return rc;
+        if ((rc = make_head_map(&mv, v, hd, KV_PAGE, KV_PAGE, n_pages * Hkv))) return rc;
+    } else {
+        if ((rc = make_head_map(&mk, k, hd, S, kv_stride, B * Hkv))) return rc;
+        if ((rc = make_head_map(&mv, v, hd, S, kv_stride, B * Hkv))) return rc;
+    }
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
     dim3 grid((S + BQ - 1) / BQ, H, B);
     if (hd == 128) {
         if ((rc = attn_attr<128>())) return rc;
         launch_pdl(attn_prefill_tc_kernel<128>, grid, dim3(NTHREADS), ACfg<128>::SMEM, st, mq, mk, mv, (bf16*)o, H, S,
-                   Hkv, scale_log2, err);
+                   Hkv, scale_log2, pages, pps, err);
     } else {
         if ((rc = attn_attr<64>())) return rc;
         launch_pdl(attn_prefill_tc_kernel<64>, grid, dim3(NTHREADS), ACfg<64>::SMEM, st, mq, mk, mv, (bf16*)o, H, S,
-                   Hkv, scale_log2, err);
+                   Hkv, scale_log2, pages, pps, err);
     }
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;

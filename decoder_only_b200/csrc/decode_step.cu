@@ -66,6 +66,7 @@ constexpr int BK = 64;       // K per stage (one 128-byte swizzle row)
 constexpr int NT = 256;      // warps 0-3 epilogue, 4 TMA producer, 5 MMA, 6-7 attention
 constexpr int NAW = STEP_ATTN_WARPS;   // attention warps per CTA: the four epilogue warps and warps 6, 7
 static_assert(NAW == 6, "warp roles");
+static_assert(KV_PAGE % 16 == 0, "an attention chunk stays inside one page");
 constexpr int ACH = 16;      // keys per attention chunk (one bulk copy of K rows, one of V rows)
 constexpr int AMX = 2048;    // logits per greedy-choice item
 constexpr int SSQ_BLOCKS = 64;   // 128-feature blocks of one norm's sums of squares (d <= 8192)
@@ -520,13 +521,14 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
 template <int BN, int HD>
 // Chunk kc of query pair pr = b * H + h, whose keys and values are cache row
 // kvr = b * Hkv + h / (H / Hkv).
-__device__ __forceinline__ void attn_issue_kv(const StepArgs& a, int l, int kvr, int kc, int len, uint32_t dst,
+__device__ __forceinline__ void attn_issue_kv(const StepArgs& a, int l, int b, int kvr, int kc, int len, uint32_t dst,
                                               uint32_t bar, uint32_t extra_bytes, bool arrive) {
     const int k0 = kc * ACH;
     const int nkeys = min(len - k0, ACH);
     const bf16* kc_ = a.kv + (size_t)(2 * l) * a.kv_layer;
     const bf16* vc = kc_ + a.kv_layer;
-    const size_t off = ((size_t)kvr * a.smax + k0) * HD;
+    // a chunk never crosses a page of a paged cache (ACH divides KV_PAGE)
+    const size_t off = kv_row_offset(a.pages, a.pps, b, a.Hkv, kvr - b * a.Hkv, a.smax, k0, HD);
     const uint32_t bytes = (uint32_t)(nkeys * HD * 2);
     // cache rows are read once per step (per query head of a group): first out of L2
     const uint64_t pol = l2_evict_first();
@@ -635,7 +637,7 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
         if (lane == 0) {
             const bool with_q = ic == cs || iq.kc == 0;
             const uint32_t dst = wbuf + buf * C::ATT_BUF, bar = wbar + 8 * buf;
-            attn_issue_kv<BN, HD>(a, l, iq.kvr, iq.kc, iq.len, dst, bar, with_q ? HD * 2 : 0, true);
+            attn_issue_kv<BN, HD>(a, l, iq.b, iq.kvr, iq.kc, iq.len, dst, bar, with_q ? HD * 2 : 0, true);
             if (with_q) attn_issue_q<BN, HD>(a, iq.b * a.H + iq.h, dst, bar);
         }
         ++ic;
@@ -655,7 +657,8 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
         for (int k = 0; k < 2 && cs + k < ce; ++k) {
             early[k] = eq.kc < eq.nch - 1;
             if (early[k] && lane == 0)
-                attn_issue_kv<BN, HD>(a, l, eq.kvr, eq.kc, eq.len, wbuf + k * C::ATT_BUF, wbar + 8 * k, 0, false);
+                attn_issue_kv<BN, HD>(a, l, eq.b, eq.kvr, eq.kc, eq.len, wbuf + k * C::ATT_BUF, wbar + 8 * k, 0,
+                                      false);
             advance(eq);
         }
     }
@@ -1265,6 +1268,8 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                 ep.d = a.d;
                 ep.smax = a.smax;
                 ep.Hkv = a.Hkv;
+                ep.pages = a.pages;
+                ep.pps = a.pps;
                 ep.bias = (type == PH_QKV && a.biases) ? a.biases[4 * l] : nullptr;   // folded QKV biases
                 for (int i = w.s; i < w.e;) {
                     const int mb = i / w.kbt;

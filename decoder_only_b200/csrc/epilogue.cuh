@@ -37,7 +37,22 @@ struct EpiArgs {
     int Hkv;              // key/value heads: columns [d, d + Hkv hd) are K, then V
     const float* bias;    // the bias variant: fp32 per output column (weight row order), or NULL
     int m0;               // EPI_QKV prefill: token row of the GEMM's first row (row blocks launched apart)
+    const int* pages;     // paged KV cache: page of (sequence b, logical page p) at pages[b * pps + p],
+    int pps;              // a page holding KV_PAGE positions of every key/value head; NULL: contiguous
 };
+
+constexpr int KV_PAGE = 128;   // positions per page of a paged KV cache
+
+// Element offset of cache row (sequence b, key/value head kvh, position pos):
+// contiguous [B][Hkv][smax][hd], or paged [page][Hkv][KV_PAGE][hd]
+__host__ __device__ __forceinline__ size_t kv_row_offset(const int* pages, int pps, int b, int Hkv, int kvh, int smax,
+                                                         int pos, int hd) {
+    if (pages) {
+        const int pg = pages[b * pps + pos / KV_PAGE];
+        return (((size_t)pg * Hkv + kvh) * KV_PAGE + pos % KV_PAGE) * hd;
+    }
+    return (((size_t)b * Hkv + kvh) * smax + pos) * hd;
+}
 
 __device__ __forceinline__ float silu_f(float u) { return u / (1.0f + __expf(-u)); }
 
@@ -161,7 +176,7 @@ __device__ __forceinline__ void epi_qkv32(const EpiArgs& a, int m, int n0, const
         dst = reinterpret_cast<T*>(a.q) + (((size_t)b * a.H + head) * a.S + s) * a.hd + i0;
     } else {
         T* base = reinterpret_cast<T*>(which == 1 ? a.kc : a.vc);
-        dst = base + (((size_t)b * a.Hkv + head) * a.smax + pos) * a.hd + i0;
+        dst = base + kv_row_offset(a.pages, a.pps, b, a.Hkv, head, a.smax, pos, a.hd) + i0;
     }
     store32<T>(dst, r);
 }

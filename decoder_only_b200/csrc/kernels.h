@@ -44,8 +44,10 @@ int launch_attention_prefill_simt(int dtype, const void* q, const void* k, const
 int attention_prepare();  // sets kernel attributes; call before any stream capture
 
 // attn_tc.cu  (bf16 tcgen05 causal flash attention, head_dim 64 or 128)
+// pages (device, [B][pps] page ids) != NULL: k and v are page pools of n_pages pages [Hkv][128][hd]
 int launch_attention_prefill_tc(const void* q, const void* k, const void* v, void* o, int B, int H, int Hkv, int S,
-                                int hd, int kv_stride, int* err, cudaStream_t st);
+                                int hd, int kv_stride, int* err, cudaStream_t st, const int* pages = nullptr,
+                                int pps = 0, int n_pages = 0);
 int attention_tc_prepare();
 
 // decode.cu
@@ -113,6 +115,8 @@ struct StepArgs {
     int L, d, h, V, H, hd, B, smax;
     int Hkv;                      // key/value heads (query head h uses h / (H / Hkv))
     float eps;
+    const int* pages;             // paged KV cache: page table [B][pps] (device), or NULL (contiguous)
+    int pps;
 };
 int decode_step_prepare();
 int launch_decode_step(const StepArgs& a, cudaStream_t st);

@@ -206,6 +206,12 @@ struct llama_model {
     int ar_chunks;
     cudaStream_t comm;
     std::vector<cudaEvent_t> tp_ev;   // [3][TP_MAX_CHUNKS]: ready, O exchanged, down exchanged
+    // paged KV cache (kv_pages > 0): the page table [max_batch][pps] on the
+    // device, whether it holds a valid table, and the positions it covers
+    int* pages;
+    int pps;
+    bool pages_ready;
+    int seq_cap;
     cudaStream_t cap_stream;
     cudaGraphExec_t graph;
     int graph_B;
@@ -237,6 +243,7 @@ int validate(const llama_config* c) {
     if (c->d_model % 32 != 0 || c->d_model > 8192) return LLAMA_ERR_INVALID_ARG;
     if (c->ffn_hidden < 0 || c->ffn_hidden % 128 != 0) return LLAMA_ERR_INVALID_ARG;
     if (c->tp_size < 0 || c->tp_size > 64) return LLAMA_ERR_INVALID_ARG;
+    if (c->kv_pages < 0 || (c->kv_pages > 0 && c->dtype != LLAMA_BF16)) return LLAMA_ERR_INVALID_ARG;
     if (c->tp_size > 1) {
         // whole heads, whole key/value heads and whole 128-unit SwiGLU blocks per shard
         const int T = c->tp_size;
@@ -310,8 +317,13 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
     float* g_final = (float*)take(d * 4);
     void* head = take(V * d * esz);
     float2* rope = (float2*)take((size_t)c->max_seq * (c->head_dim / 2) * sizeof(float2));
-    const size_t kv_layer = (size_t)c->max_batch * kv_local(c) * c->max_seq * c->head_dim;
+    // KV cache: contiguous [max_batch][n_kv][max_seq][hd] per layer and K / V, or a
+    // pool of kv_pages pages [n_kv][KV_PAGE][hd] with a page table [max_batch][pps]
+    const size_t pps = ((size_t)c->max_seq + KV_PAGE - 1) / KV_PAGE;
+    const size_t kv_layer = c->kv_pages > 0 ? (size_t)c->kv_pages * kv_local(c) * KV_PAGE * c->head_dim
+                                            : (size_t)c->max_batch * kv_local(c) * c->max_seq * c->head_dim;
     void* kv = take(2 * L * kv_layer * esz);
+    int* pages = (int*)take(c->kv_pages > 0 ? (size_t)c->max_batch * pps * 4 : 0);
     float* trunk = (float*)take(nmax * d * 4);
     void* xn = take(nmax * d * esz);
     void* q = take(nmax * dq * esz);
@@ -356,6 +368,8 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
         m->rope = rope;
         m->kv = kv;
         m->kv_layer_elems = kv_layer;
+        m->pages = c->kv_pages > 0 ? pages : nullptr;
+        m->pps = (int)pps;
         m->trunk = trunk;
         m->xn = xn;
         m->q = q;
@@ -426,6 +440,8 @@ EpiArgs base_args(llama_model* m, int M, int N) {
     a.smax = m->cfg.max_seq;
     a.rope = m->rope;
     a.hidden = m->hl;
+    a.pages = m->pages;
+    a.pps = m->pps;
     return a;
 }
 
@@ -512,7 +528,7 @@ int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
             prof::Scope ps(st, "prefill_attention", 4.0 * n * d * m->esz, 2.0 * B * (double)S * (S + 1) * d);
             if (dt == LLAMA_BF16)
                 rc = launch_attention_prefill_tc(m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, Hkv, S,
-                                                 c.head_dim, c.max_seq, m->d_err, st);
+                                                 c.head_dim, c.max_seq, m->d_err, st, m->pages, m->pps, c.kv_pages);
             else
                 rc = launch_attention_prefill_simt(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, Hkv, S,
                                                    c.head_dim, c.max_seq, st);
@@ -615,7 +631,7 @@ int run_blocks_tp(llama_model* m, int B, int S, cudaStream_t st) {
             prof::Scope ps(st, "prefill_attention", 4.0 * n * dq * m->esz, 2.0 * B * (double)S * (S + 1) * dq);
             if (dt == LLAMA_BF16)
                 rc = launch_attention_prefill_tc(m->q, kcache(m, l), vcache(m, l), m->attn, B, m->Hl, m->Hkvl, S,
-                                                 c.head_dim, c.max_seq, m->d_err, st);
+                                                 c.head_dim, c.max_seq, m->d_err, st, m->pages, m->pps, c.kv_pages);
             else
                 rc = launch_attention_prefill_simt(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, m->Hl, m->Hkvl,
                                                    S, c.head_dim, c.max_seq, st);
@@ -721,6 +737,8 @@ StepArgs step_args(llama_model* m) {
     a.B = m->B;
     a.smax = c.max_seq;
     a.eps = c.norm_eps;
+    a.pages = m->pages;
+    a.pps = m->pps;
     return a;
 }
 
@@ -907,6 +925,8 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
     m->ar_chunks = 1;
     m->comm = nullptr;
     m->cap_stream = nullptr;
+    m->pages_ready = m->pages == nullptr;
+    m->seq_cap = cfg->max_seq;
     if (cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
         delete m;
         return LLAMA_ERR_CUDA;
@@ -998,6 +1018,27 @@ int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d_arena, ui
         llama_free(m);
         return LLAMA_ERR_CUDA;
     }
+    if (m->pages) {
+        // pages start zeroed (a page's rows past its sequence's length are read, masked,
+        // by the prefill attention: they must be finite); the default table gives
+        // sequence b pages b * pps .. when the pool holds that many
+        if (cudaMemsetAsync(m->kv, 0, 2 * (size_t)cfg->n_layers * m->kv_layer_elems * m->esz, st) != cudaSuccess) {
+            llama_free(m);
+            return LLAMA_ERR_CUDA;
+        }
+        if ((int64_t)cfg->kv_pages >= (int64_t)cfg->max_batch * m->pps) {
+            std::vector<int> tab((size_t)cfg->max_batch * m->pps);
+            for (size_t i = 0; i < tab.size(); ++i) tab[i] = (int)i;
+            if (cudaMemcpyAsync(m->pages, tab.data(), tab.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+                cudaStreamSynchronize(st) != cudaSuccess) {
+                llama_free(m);
+                return LLAMA_ERR_CUDA;
+            }
+            m->pages_ready = true;
+        } else {
+            m->seq_cap = 0;   // positions need pages: llama_set_pages first
+        }
+    }
     pick_decode_splits(m);
     if ((rc = gemm_tc_prepare()) || (rc = attention_prepare()) || (rc = attention_tc_prepare()) ||
         (rc = attention_decode_prepare()) || (cfg->dtype == LLAMA_BF16 && (rc = decode_step_prepare()))) {
@@ -1025,6 +1066,8 @@ static int prefill_impl(llama_model* m, const int32_t* d_tokens, int32_t B, int3
         for (int b = 0; b < B; ++b)
             if (h_lens[b] < 1 || h_lens[b] > S) return LLAMA_ERR_INVALID_ARG;
     if (m->tp > 1 && !m->ar_fn) return LLAMA_ERR_STATE;   // a shard needs its exchange
+    if (!m->pages_ready) return LLAMA_ERR_STATE;         // a paged cache needs its page table
+    if (S > m->seq_cap) return LLAMA_ERR_INVALID_ARG;    // positions beyond the sequences' pages
     const int n = B * S;
     const int V = m->cfg.vocab;
     int rc;
@@ -1080,6 +1123,8 @@ int llama_prefill_trunk(llama_model* m, const float* d_x, int32_t B, int32_t S, 
     cudaStream_t st = (cudaStream_t)stream;
     const size_t bytes = (size_t)B * S * m->cfg.d_model * 4;
     if (m->tp > 1 && !m->ar_fn) return LLAMA_ERR_STATE;
+    if (!m->pages_ready) return LLAMA_ERR_STATE;
+    if (S > m->seq_cap) return LLAMA_ERR_INVALID_ARG;
     if (d_x != m->trunk) LLAMA_CUDA_TRY(cudaMemcpyAsync(m->trunk, d_x, bytes, cudaMemcpyDeviceToDevice, st));
     int rc = prefill_blocks(m, B, S, st);
     if (rc) return rc;
@@ -1094,7 +1139,7 @@ int llama_prefill_trunk(llama_model* m, const float* d_x, int32_t B, int32_t S, 
 
 int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t* d_next, float* d_logits, void* stream) {
     if (!m || !d_tokens || m->tp > 1) return LLAMA_ERR_INVALID_ARG;
-    if (m->B <= 0 || m->cur_len >= m->cfg.max_seq) return LLAMA_ERR_STATE;
+    if (m->B <= 0 || m->cur_len >= m->cfg.max_seq || m->cur_len >= m->seq_cap) return LLAMA_ERR_STATE;
     cudaStream_t st = (cudaStream_t)stream;
     int rc = ensure_graph(m);
     if (rc) return rc;
@@ -1111,7 +1156,8 @@ int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t* d_next, 
 
 int llama_generate(llama_model* m, const int32_t* d_first, int32_t n_steps, int32_t* d_out, void* stream) {
     if (!m || !d_out || n_steps < 0 || m->tp > 1) return LLAMA_ERR_INVALID_ARG;
-    if (m->B <= 0 || m->cur_len + n_steps > m->cfg.max_seq) return LLAMA_ERR_STATE;
+    if (m->B <= 0 || m->cur_len + n_steps > m->cfg.max_seq || m->cur_len + n_steps > m->seq_cap)
+        return LLAMA_ERR_STATE;
     cudaStream_t st = (cudaStream_t)stream;
     int rc = ensure_graph(m);
     if (rc) return rc;
@@ -1132,6 +1178,28 @@ int llama_set_allreduce(llama_model* m, llama_allreduce_fn fn, void* ctx, int32_
     m->ar_fn = fn;
     m->ar_ctx = ctx;
     m->ar_chunks = chunks;
+    return LLAMA_OK;
+}
+
+int llama_set_pages(llama_model* m, const int32_t* h_table, int32_t B, int32_t pages_per_seq, void* stream) {
+    if (!m || !m->pages || !h_table || B < 1 || B > m->cfg.max_batch || pages_per_seq < 1 ||
+        pages_per_seq > m->pps)
+        return LLAMA_ERR_INVALID_ARG;
+    // every page in range, and no page given to two (sequence, position) slots
+    std::vector<int> tab((size_t)m->cfg.max_batch * m->pps, 0);
+    std::vector<char> used((size_t)m->cfg.kv_pages, 0);
+    for (int b = 0; b < B; ++b)
+        for (int p = 0; p < pages_per_seq; ++p) {
+            const int pg = h_table[(size_t)b * pages_per_seq + p];
+            if (pg < 0 || pg >= m->cfg.kv_pages || used[pg]) return LLAMA_ERR_INVALID_ARG;
+            used[pg] = 1;
+            tab[(size_t)b * m->pps + p] = pg;
+        }
+    cudaStream_t st = (cudaStream_t)stream;
+    LLAMA_CUDA_TRY(cudaMemcpyAsync(m->pages, tab.data(), tab.size() * 4, cudaMemcpyHostToDevice, st));
+    LLAMA_CUDA_TRY(cudaStreamSynchronize(st));   // the host table is the caller's again on return
+    m->pages_ready = true;
+    m->seq_cap = std::min(m->cfg.max_seq, pages_per_seq * KV_PAGE);
     return LLAMA_OK;
 }
 

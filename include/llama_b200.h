@@ -92,6 +92,10 @@ typedef struct llama_config {
                             T shards (see llama_set_allreduce).  n_heads, n_kv_heads and
                             ffn_hidden / 128 must divide by T. */
     int32_t tp_rank;     /* this shard, 0 <= tp_rank < T */
+    int32_t kv_pages;    /* 0: contiguous KV cache [L][2][max_batch][n_kv][max_seq][head_dim];
+                            P > 0 (bf16 only): a pool of P pages of 128 positions,
+                            [L][2][P][n_kv][128][head_dim], mapped per sequence by a page
+                            table (llama_set_pages) */
 } llama_config;
 
 typedef struct llama_model llama_model; /* opaque host handle */
@@ -191,6 +195,21 @@ LLAMA_API int llama_complete(llama_model* m, const int32_t* h_tokens, int32_t B,
  * per-layer weights.  Layouts are those of the arena described above. */
 LLAMA_API int llama_model_tensor(const llama_model* m, const char* name, int32_t layer,
                        void** d_ptr, uint64_t* bytes);
+
+/* [NAR] "GQA Was Not an Original LLaMA Feature": decoding keeps the keys and
+ * values of every earlier position, per sequence.  With a paged cache
+ * (kv_pages > 0) they live in pages of 128 positions taken from one pool, so
+ * that sequences of different lengths need not each reserve max_seq
+ * positions.  h_table (host int32 [B][pages_per_seq]) gives sequence b's
+ * logical page p (positions 128 p .. 128 p + 127) as a pool page in
+ * [0, kv_pages); no page may appear twice.  Positions of each sequence are
+ * then limited to 128 * pages_per_seq (and max_seq).  Copies the table to
+ * the device on `stream` and synchronises it.  At init, when kv_pages >=
+ * max_batch * ceil(max_seq / 128), sequence b gets pages b * ceil(max_seq /
+ * 128) + p; otherwise the table must be set before the first prefill
+ * (LLAMA_ERR_STATE).  The pool starts zeroed. */
+LLAMA_API int llama_set_pages(llama_model* m, const int32_t* h_table, int32_t B, int32_t pages_per_seq,
+                              void* stream);
 
 /* ------------------------------------------------------- tensor parallel
  * [KN] "LLaMA: Open and Efficient Foundation Language Models" knowledge

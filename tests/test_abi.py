@@ -155,3 +155,23 @@ def test_tp_configs_that_do_not_divide_are_rejected(tp):
 
 def test_tp_exchange_is_rejected_on_an_unsharded_model_handle():
     assert lb.lib.llama_set_allreduce(None, lb.ALLREDUCE_FN(lambda *a: 0), None, 4) == -1
+
+
+# ------------------------------------------------------------------ paged KV cache (host logic)
+
+def test_paged_cache_arena_holds_the_pool_instead_of_the_slabs():
+    s = LLAMA_7B.with_(n_layers=2)
+    B, S = 4, 1000
+    contiguous = lb.model_bytes(lb.make_config(s, B, S))
+    paged = lb.model_bytes(lb.make_config(s, B, S, kv_pages=11))
+    kv = 2 * s.n_layers * B * S * s.d_model * 2
+    pool = 2 * s.n_layers * 11 * 128 * s.d_model * 2
+    table = B * 8 * 4
+    assert contiguous - kv == pytest.approx(paged - pool - table, abs=256 * 4)
+
+
+def test_paged_cache_needs_bf16():
+    n = ctypes.c_uint64()
+    assert lb.lib.llama_model_bytes(ctypes.byref(lb.make_config(TINY, 1, 32, kv_pages=2)), ctypes.byref(n)) == -1
+    assert lb.lib.llama_model_bytes(ctypes.byref(lb.make_config(LLAMA_7B, 1, 32, kv_pages=-1)),
+                                    ctypes.byref(n)) == -1
