@@ -518,9 +518,10 @@ __device__ void tile_epilogue(const StepArgs& a, const EpiArgs& ep, const Work& 
 // shuffles; a pair inside one range is written directly, otherwise each
 // range leaves its (max, sum, output) in the workspace and the last range to
 // arrive merges them in range order.
-template <int BN, int HD>
 // Chunk kc of query pair pr = b * H + h, whose keys and values are cache row
-// kvr = b * Hkv + h / (H / Hkv).
+// kvr = b * Hkv + h / (H / Hkv); PG: the cache is paged (the kernel is
+// instantiated apart for paged and contiguous caches).
+template <int BN, int HD, bool PG>
 __device__ __forceinline__ void attn_issue_kv(const StepArgs& a, int l, int b, int kvr, int kc, int len, uint32_t dst,
                                               uint32_t bar, uint32_t extra_bytes, bool arrive) {
     const int k0 = kc * ACH;
@@ -528,7 +529,7 @@ __device__ __forceinline__ void attn_issue_kv(const StepArgs& a, int l, int b, i
     const bf16* kc_ = a.kv + (size_t)(2 * l) * a.kv_layer;
     const bf16* vc = kc_ + a.kv_layer;
     // a chunk never crosses a page of a paged cache (ACH divides KV_PAGE)
-    const size_t off = kv_row_offset(a.pages, a.pps, b, a.Hkv, kvr - b * a.Hkv, a.smax, k0, HD);
+    const size_t off = kv_row_offset(PG ? a.pages : nullptr, a.pps, b, a.Hkv, kvr - b * a.Hkv, a.smax, k0, HD);
     const uint32_t bytes = (uint32_t)(nkeys * HD * 2);
     // cache rows are read once per step (per query head of a group): first out of L2
     const uint64_t pol = l2_evict_first();
@@ -557,7 +558,7 @@ __device__ __forceinline__ void attn_issue_q(const StepArgs& a, int pr, uint32_t
 }
 
 // Attention of layer l for attention warp aw of this CTA (0..NAW-1).
-template <int BN, int HD>
+template <int BN, int HD, bool PG>
 __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Smem<BN, HD>& sm, uint32_t* uses,
                            volatile int* abort_flag) {
     using C = SCfg<BN, HD>;
@@ -637,7 +638,7 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
         if (lane == 0) {
             const bool with_q = ic == cs || iq.kc == 0;
             const uint32_t dst = wbuf + buf * C::ATT_BUF, bar = wbar + 8 * buf;
-            attn_issue_kv<BN, HD>(a, l, iq.b, iq.kvr, iq.kc, iq.len, dst, bar, with_q ? HD * 2 : 0, true);
+            attn_issue_kv<BN, HD, PG>(a, l, iq.b, iq.kvr, iq.kc, iq.len, dst, bar, with_q ? HD * 2 : 0, true);
             if (with_q) attn_issue_q<BN, HD>(a, iq.b * a.H + iq.h, dst, bar);
         }
         ++ic;
@@ -657,7 +658,7 @@ __device__ bool phase_attn(const StepArgs& a, int l, int aw, int lane, const Sme
         for (int k = 0; k < 2 && cs + k < ce; ++k) {
             early[k] = eq.kc < eq.nch - 1;
             if (early[k] && lane == 0)
-                attn_issue_kv<BN, HD>(a, l, eq.b, eq.kvr, eq.kc, eq.len, wbuf + k * C::ATT_BUF, wbar + 8 * k, 0,
+                attn_issue_kv<BN, HD, PG>(a, l, eq.b, eq.kvr, eq.kc, eq.len, wbuf + k * C::ATT_BUF, wbar + 8 * k, 0,
                                       false);
             advance(eq);
         }
@@ -988,7 +989,7 @@ __device__ void phase_argmax(const StepArgs& a, int tid, const Smem<BN, HD>& sm,
 
 
 // ---------------------------------------------------------------- the kernel
-template <int BN, int HD>
+template <int BN, int HD, bool PG>
 __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
     using C = SCfg<BN, HD>;
     extern __shared__ uint8_t smem_raw[];
@@ -1238,7 +1239,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                     }
                 }
             } else if (type == PH_ATTN) {
-                fail = !phase_attn<BN, HD>(a, l, warp, lane, sm, uses, abort_flag);
+                fail = !phase_attn<BN, HD, PG>(a, l, warp, lane, sm, uses, abort_flag);
                 asm volatile("bar.sync 2, 192;" ::: "memory");   // with attention warps 6, 7
             } else if (type == PH_ARGMAX) {
                 phase_argmax<BN, HD>(a, tid, sm, E, abort_flag);
@@ -1268,7 +1269,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
                 ep.d = a.d;
                 ep.smax = a.smax;
                 ep.Hkv = a.Hkv;
-                ep.pages = a.pages;
+                ep.pages = PG ? a.pages : nullptr;
                 ep.pps = a.pps;
                 ep.bias = (type == PH_QKV && a.biases) ? a.biases[4 * l] : nullptr;   // folded QKV biases
                 for (int i = w.s; i < w.e;) {
@@ -1313,7 +1314,7 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
         if (lane == 0) w = wait_at_least(a.bar + SY_EMBED, E, abort_flag, a.err);
         bool ok = __shfl_sync(0xffffffffu, w, 0) != 0;
         for (int l = 0; l < a.L; ++l) {
-            if (ok) ok = phase_attn<BN, HD>(a, l, warp - 2, lane, sm, uses, abort_flag);
+            if (ok) ok = phase_attn<BN, HD, PG>(a, l, warp - 2, lane, sm, uses, abort_flag);
             __syncwarp();
             asm volatile("bar.arrive 2, 192;" ::: "memory");
         }
@@ -1329,13 +1330,13 @@ __global__ void __launch_bounds__(NT, 1) decode_step_kernel(StepArgs a) {
     }
 }
 
-template <int BN, int HD>
+template <int BN, int HD, bool PG>
 int launch_step_t(const StepArgs& a, cudaStream_t st) {
     using C = SCfg<BN, HD>;
     static PerDeviceOnce once;
     int rc = once_per_device(once, []() -> int {
-        LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<BN, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            C::SMEM));
+        LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<BN, HD, PG>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
         return (int)LLAMA_OK;
     });
     if (rc) return rc;
@@ -1349,7 +1350,7 @@ int launch_step_t(const StepArgs& a, cudaStream_t st) {
     attr_c[0].val.cooperative = 1;
     cfg.attrs = attr_c;
     cfg.numAttrs = 1;
-    LLAMA_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_step_kernel<BN, HD>, a));
+    LLAMA_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_step_kernel<BN, HD, PG>, a));
     llama_count_launches(1);
     return LLAMA_OK;
 }
@@ -1377,26 +1378,36 @@ long long decode_step_layout(int ctas, int qkv_rows, int d, int h, int V, int B,
     return off;
 }
 
+template <int BN, int HD>
+int step_prepare_t() {
+    LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<BN, HD, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        SCfg<BN, HD>::SMEM));
+    LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<BN, HD, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        SCfg<BN, HD>::SMEM));
+    return LLAMA_OK;
+}
+
 int decode_step_prepare() {
     int n = 0;
-    LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        SCfg<16, 128>::SMEM));
-    LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<32, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        SCfg<32, 128>::SMEM));
-    LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<16, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        SCfg<16, 64>::SMEM));
-    LLAMA_CUDA_TRY(cudaFuncSetAttribute(decode_step_kernel<32, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        SCfg<32, 64>::SMEM));
+    if (int rc = step_prepare_t<16, 128>()) return rc;
+    if (int rc = step_prepare_t<32, 128>()) return rc;
+    if (int rc = step_prepare_t<16, 64>()) return rc;
+    if (int rc = step_prepare_t<32, 64>()) return rc;
     // one CTA per SM must fit for the cooperative launch
-    LLAMA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_step_kernel<16, 128>, NT,
+    LLAMA_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_step_kernel<16, 128, false>, NT,
                                                                  SCfg<16, 128>::SMEM));
     return n >= 1 ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 int launch_decode_step(const StepArgs& a, cudaStream_t st) {
     if (a.B <= 0 || a.B > 32) return LLAMA_ERR_INVALID_ARG;
-    if (a.hd == 128) return a.B <= 16 ? launch_step_t<16, 128>(a, st) : launch_step_t<32, 128>(a, st);
-    if (a.hd == 64) return a.B <= 16 ? launch_step_t<16, 64>(a, st) : launch_step_t<32, 64>(a, st);
+    const bool pg = a.pages != nullptr;
+    if (a.hd == 128)
+        return a.B <= 16 ? (pg ? launch_step_t<16, 128, true>(a, st) : launch_step_t<16, 128, false>(a, st))
+                         : (pg ? launch_step_t<32, 128, true>(a, st) : launch_step_t<32, 128, false>(a, st));
+    if (a.hd == 64)
+        return a.B <= 16 ? (pg ? launch_step_t<16, 64, true>(a, st) : launch_step_t<16, 64, false>(a, st))
+                         : (pg ? launch_step_t<32, 64, true>(a, st) : launch_step_t<32, 64, false>(a, st));
     return LLAMA_ERR_INVALID_ARG;
 }
 
