@@ -8,38 +8,41 @@
 // knowledge note credits to the xFormers attention of the training system.
 //
 // Persistent CTAs, one per SM, each working through a list of work items
-// (128-query tile, head, sequence): longest items first, dealt in snake
-// order.  The tile rings and barriers run on over item boundaries, so the
-// next item's Q, K and first scores load and compute while the current
-// item's output is written.
-//   warp 0      TMA: lane 0 each item's Q (once the previous item's last
-//               Q K^T is done), then its K_j tiles; lane 1 the V_j tiles
-//               (2-stage rings; K_j is free once S_j is computed, V_j once
-//               O_j is, so K runs ahead of V).  3-D tensor maps (hd,
-//               position, head) make rows >= S read as 0.
+// (128-query tile, head, sequence) that it claims from a global counter;
+// the rings and barriers run on over item boundaries, so the next item's Q,
+// K and first scores load and compute while the current item's output is
+// written.
+//   warp 0      TMA: lane 0 claims the items, loads each item's Q (once the
+//               previous item's last Q K^T is done), then its K_j tiles;
+//               lane 1 the V_j tiles.  Three-stage rings: a tile is fetched
+//               three tiles ahead of its use, which covers the load latency
+//               from L2 (about 2 us for a 32 KB tile when all SMs stream
+//               keys and values).  3-D tensor maps (hd, position, head) make
+//               rows >= S read as 0.
 //   warp 1      TMEM allocator + MMA issuer:
-//                 S_j = Q K_j^T        (M 128, N 128, K hd)  -> TMEM S[j % 2]
-//                 O  += P_j V_j        (M 128, N hd, K 128)  -> TMEM O (one
-//                                       accumulator for the whole row tile)
-//               V is the MN-major B operand (hd contiguous), so the cache
-//               layout [position][hd] is used as is.
-//   warps 2..5  one query row per thread: row max of S_j (pass 1), then
-//               p = 2^(s log2e / sqrt(hd) - m) rounded to bf16 into the
-//               shared P tile (128-byte swizzled, K-major) and the row sum
-//               (pass 2), both passes on the row's 128 scores held in
-//               registers (one TMEM read per tile).  The running maximum m
-//               (log2 units) moves only when a tile's maximum exceeds it by
-//               more than 8: p stays <= 2^8, exact in fp32 and bf16's range,
-//               and the output in TMEM is rescaled by 2^(m_old - m_new) (TMEM
-//               load, scale, store, after the previous P V product) only
-//               then -- a few times per row -- instead of folding every
-//               tile's product into registers.  The pass is bound by the
-//               instructions it issues per score (one warp per sub-
-//               partition): one FMA, one ex2, half a pack, one add.
-//               After an item's last tile: O / (row sum), bf16, to
-//               global; the item's first P V product waits for that read.
+//                 S_j = Q K_j^T      (M 128, N 128, K hd)  -> TMEM stage j % 3
+//                 O  += P_j V_j      (M 128, N hd, K 128)  -> TMEM O (one
+//                                     accumulator per work item)
+//               P_j is the A operand read from tensor memory (written over
+//               S_j by the softmax), V the MN-major B operand (hd
+//               contiguous), so the cache layout [position][hd] is used as
+//               is.  A stage is free for S_{j+3} once P_j V_j is done.
+//   warps 2..5  one query row per thread: the row's 128 scores into
+//               registers (one TMEM read), row max (pass 1), then p =
+//               2^(s log2e / sqrt(hd) - m) rounded to bf16 into the row's
+//               TMEM lane and the row sum in fp32 (pass 2).  The running
+//               maximum m (log2 units) moves only when a tile's maximum
+//               exceeds it by more than 8: p stays <= 2^8, exact in fp32 and
+//               bf16's range, and the output in TMEM is rescaled by
+//               2^(m_old - m_new) (TMEM load, scale, store, after the
+//               previous P V product) only then -- a few times per row --
+//               instead of folding every tile's product into registers.
+//               After an item's last tile: O / (row sum), bf16, to global;
+//               the next item's first P V product waits for that read.
 // All mbarrier waits are bounded (see tcgen05.cuh).
 #include <cudaTypedefs.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "epilogue.cuh"
@@ -63,89 +66,126 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+constexpr int NST = 3;          // stages of the K, V and S / P rings
+
 template <int HD>
 struct ACfg {
     static constexpr int REG = 128 * 128;                    // one [128 rows][64 bf16] swizzled region, bytes
     static constexpr int NREG = HD / 64;                     // regions per Q / K / V tile
     static constexpr int TILE = NREG * REG;                  // Q, K or V tile bytes
-    static constexpr int P_TILE = 2 * REG;                   // P: [128 q][128 keys] bf16
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + TILE;               // [2]
-    static constexpr int OFF_V = OFF_K + 2 * TILE;           // [2]
-    static constexpr int OFF_P = OFF_V + 2 * TILE;           // [2]
-    static constexpr int OFF_BAR = OFF_P + 2 * P_TILE;
-    static constexpr int SMEM = OFF_BAR + 256 + 1024;
-    static constexpr uint32_t TMEM_COLS = 512;               // S[2] at 0, 128; O at 256
+    static constexpr int OFF_K = OFF_Q + TILE;               // [NST]
+    static constexpr int OFF_V = OFF_K + NST * TILE;         // [NST]
+    static constexpr int OFF_BAR = OFF_V + NST * TILE;
+    static constexpr int SMEM = OFF_BAR + 512 + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;               // S / P [NST] at 0, 128, 256; O at 384
+    static constexpr uint32_t O_COL = 128 * NST;
+    static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-// P tile position of 8 consecutive keys (one 16-byte chunk) of query row t:
-// region by key half, 128-byte row t, chunk index XOR (t % 8).
-__device__ __forceinline__ uint32_t p_chunk_addr(uint32_t base, int t, int chunk16) {
-    const int region = chunk16 >> 3;
-    const int c = chunk16 & 7;
-    return base + region * (128 * 128) + t * 128 + ((c ^ (t & 7)) << 4);
+// A x B with A (M x K, bf16) read from tensor memory: row m in lane m, K along
+// the columns, two values per 32-bit column; B from shared memory.
+__device__ __forceinline__ void umma_bf16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accum)
+        : "memory");
+}
+
+// 32 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+        "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+        "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
 }
 
 template <int HD>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ out, int H, int S,
-                           int Hkv, int B, float scale_log2, const int* __restrict__ pages, int pps, int* err) {
+                           int Hkv, int B, float scale_log2, const int* __restrict__ pages, int pps, int hblk,
+                           int* sched, int* err) {
     using C = ACfg<HD>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw);
-    const uint32_t sQ = base + C::OFF_Q, sK = base + C::OFF_K, sV = base + C::OFF_V, sP = base + C::OFF_P;
+    const uint32_t sQ = base + C::OFF_Q, sK = base + C::OFF_K, sV = base + C::OFF_V;
     const uint32_t bars = base + C::OFF_BAR;
     const uint32_t q_full = bars;
-    const uint32_t k_full = bars + 8;        // [2]
-    const uint32_t v_full = bars + 24;       // [2]
-    const uint32_t k_empty = bars + 40;      // [2]
-    const uint32_t s_full = bars + 56;       // [2]
-    const uint32_t s_empty = bars + 72;      // [2]
-    const uint32_t p_full = bars + 88;       // [2]
-    const uint32_t o_done = bars + 104;      // one phase per completed P V product
-    const uint32_t o_last = bars + 112;      // one phase per work item: its last P V product
-    const uint32_t q_empty = bars + 120;     // one phase per work item: its last Q K^T (Q free)
-    const uint32_t o_free = bars + 128;      // one phase per work item: its output read out of TMEM
-    const uint32_t v_empty = bars + 136;     // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 160);
+    const uint32_t q_empty = bars + 8;       // one phase per work item: its last Q K^T (Q free)
+    const uint32_t o_done = bars + 16;       // one phase per completed P V product
+    const uint32_t o_last = bars + 24;       // one phase per work item: its last P V product
+    const uint32_t o_free = bars + 32;       // one phase per work item: its output read out of TMEM
+    const uint32_t k_full = bars + 40;       // [NST]
+    const uint32_t k_empty = bars + 64;      // [NST] Q K_t^T done: K stage free
+    const uint32_t v_full = bars + 88;       // [NST]
+    const uint32_t pv_done = bars + 112;     // [NST] P_t V_t done: V stage and S / P stage free
+    const uint32_t s_full = bars + 136;      // [NST]
+    const uint32_t p_full = bars + 160;      // [NST] P_t in TMEM (and O rescaled)
+    const uint32_t item_full = bars + 184;   // [2] a work item's index published in item_ring
+    const uint32_t item_empty = bars + 200;  // [2] read by all six consumers (V lane, MMA, 4 softmax warps)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 256);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* item_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);   // [2]
 
-    // Work items (128-query tile, head, sequence), longest (most key tiles)
-    // first, dealt to the persistent CTAs in snake order (CTA c takes item
-    // c of the first G, item 2G - 1 - c of the next G, ...), which evens out
-    // the CTAs' key-tile totals.  Per-tile rings run on counters over all of
-    // a CTA's items, so one item's start overlaps the previous one's end.
+    // Work items (128-query tile, head, sequence) in blocks of hblk heads,
+    // longest (most key tiles) first within a block: the items running at
+    // one time share the key and value tiles of a few heads in L2.  Each
+    // CTA starts with item blockIdx.x and then takes the next unclaimed one
+    // from a global counter (sched[0]) whenever it is ready for another, so
+    // the CTAs finish together however the item lengths fall.  Lane 0 of
+    // warp 0 claims the items and publishes them to the other roles through
+    // a two-entry ring; the tile rings and barriers run on over item
+    // boundaries, so one item's start overlaps the previous one's end.
     const int n_qt = (S + BQ - 1) / BQ;
     const int total = n_qt * H * B;
-    const int G = (int)gridDim.x, cta = (int)blockIdx.x;
-    auto item_at = [&](int n) { return n * G + ((n & 1) ? G - 1 - cta : cta); };
+    const int G = (int)gridDim.x;
     auto item = [&](int it, int& qt, int& h, int& b) {
-        qt = n_qt - 1 - it / (H * B);
-        const int r = it - (n_qt - 1 - qt) * (H * B);
-        h = r % H;
-        b = r / H;
+        const int per = hblk * n_qt;
+        const int k = it / per;
+        const int r = it - k * per;
+        const int gg = min(hblk, H * B - k * hblk);
+        qt = n_qt - 1 - r / gg;
+        const int hb = k * hblk + r % gg;
+        h = hb % H;
+        b = hb / H;
+    };
+    // consumer side of the item ring: the index of this role's ni-th item
+    auto next_item = [&](int ni, bool& ok) -> int {
+        const int slot = ni & 1;
+        ok = mbar_wait(item_full + 8 * slot, (uint32_t)((ni >> 1) & 1), abort_flag, err);
+        return ok ? item_ring[slot] : total;
     };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NST; ++i) {
             mbar_init(k_full + 8 * i, 1);
-            mbar_init(v_full + 8 * i, 1);
             mbar_init(k_empty + 8 * i, 1);
-            mbar_init(v_empty + 8 * i, 1);
+            mbar_init(v_full + 8 * i, 1);
+            mbar_init(pv_done + 8 * i, 1);
             mbar_init(s_full + 8 * i, 1);
-            mbar_init(s_empty + 8 * i, 128);
             mbar_init(p_full + 8 * i, 128);
         }
         mbar_init(o_done, 1);
         mbar_init(o_last, 1);
         mbar_init(q_empty, 1);
         mbar_init(o_free, 128);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(item_full + 8 * i, 1);
+            mbar_init(item_empty + 8 * i, 6);
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -167,12 +207,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // lane 0: each item's Q (once the previous item's last Q K^T is done), then its K_j;
             // lane 1: the V_j
             const bool is_k = (lane == 0);
-            const uint32_t full = is_k ? k_full : v_full, empty = is_k ? k_empty : v_empty;
+            const uint32_t full = is_k ? k_full : v_full, empty = is_k ? k_empty : pv_done;
             const uint32_t dst = is_k ? sK : sV;
             const CUtensorMap* map = is_k ? &tmK : &tmV;
             bool ok = true;
             int kt = 0, ni = 0, q_loads = 0;
-            for (int it = item_at(0); it < total && ok; it = item_at(++ni)) {
+            int it = blockIdx.x;
+            for (;; ++ni) {
+                if (is_k) {
+                    // publish item ni (after all six consumers have read item ni - 2 from its slot)
+                    const int slot = ni & 1;
+                    if (ni >= 2 && !mbar_wait(item_empty + 8 * slot, (uint32_t)(((ni >> 1) - 1) & 1), abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    item_ring[slot] = it;
+                    mbar_arrive(item_full + 8 * slot);
+                } else {
+                    it = next_item(ni, ok);
+                    if (!ok) break;
+                    mbar_arrive(item_empty + 8 * (ni & 1));
+                }
+                if (it >= total) break;
                 int qt, h, b;
                 item(it, qt, h, b);
                 const int kv_head = b * Hkv + h / (H / Hkv);      // grouped keys and values
@@ -187,8 +243,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     ++q_loads;
                 }
                 for (int j = 0; j <= qt; ++j, ++kt) {
-                    const int st = kt & 1;
-                    if (!mbar_wait(empty + 8 * st, ((kt >> 1) & 1) ^ 1u, abort_flag, err)) {
+                    const int st = kt % NST;
+                    if (!mbar_wait(empty + 8 * st, ((kt / NST) & 1) ^ 1u, abort_flag, err)) {
                         ok = false;
                         break;
                     }
@@ -198,6 +254,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         tma_load_3d(dst + st * C::TILE + r * C::REG, map, full + 8 * st, 64 * r, pages ? 0 : j * BKV,
                                     pages ? __ldg(pages + b * pps + j) * Hkv + (kv_head - b * Hkv) : kv_head);
                 }
+                if (!ok) break;
+                if (is_k) it = G + atomicAdd(sched, 1);   // claim the next item
             }
             if (!ok) {
                 // drain (bounded) the copies this thread issued
@@ -205,9 +263,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 while (is_k && q_loads > 0 && !mbar_try_wait(q_full, (uint32_t)((q_loads - 1) & 1)) &&
                        global_timer() - t0 < WAIT_LIMIT_NS / 4) {
                 }
-                for (int t = kt > 2 ? kt - 2 : 0; t < kt; ++t) {
-                    const uint32_t par = (t >> 1) & 1;
-                    while (!mbar_try_wait(full + 8 * (t & 1), par) && global_timer() - t0 < WAIT_LIMIT_NS / 2) {
+                for (int t = kt > NST ? kt - NST : 0; t < kt; ++t) {
+                    const uint32_t par = (t / NST) & 1;
+                    while (!mbar_try_wait(full + 8 * (t % NST), par) && global_timer() - t0 < WAIT_LIMIT_NS / 2) {
                     }
                 }
             }
@@ -218,8 +276,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             constexpr uint32_t IDESC_QK = idesc_bf16(BKV);                 // K-major A and B
             constexpr uint32_t IDESC_PV = idesc_bf16(HD) | (1u << 16);      // B (V) MN-major
             bool ok = true;
-            int kt0 = 0, ni = 0;
-            for (int it = item_at(0); it < total && ok; it = item_at(++ni)) {
+            int kt0 = 0;
+            for (int ni = 0; ok; ++ni) {
+                const int it = next_item(ni, ok);
+                if (!ok) break;
+                mbar_arrive(item_empty + 8 * (ni & 1));
+                if (it >= total) break;
                 int qt, h, b;
                 item(it, qt, h, b);
                 const int n_kv = qt + 1;
@@ -227,10 +289,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc_fence_after();
                 for (int j = 0; j <= n_kv && ok; ++j) {
                     if (j < n_kv) {
-                        const int t = kt0 + j, st = t & 1;
-                        const uint32_t par = (t >> 1) & 1;
+                        // S_t into stage t % NST, once P_{t - NST} V_{t - NST} has read that stage
+                        const int t = kt0 + j, st = t % NST;
+                        const uint32_t par = (t / NST) & 1;
                         if (!mbar_wait(k_full + 8 * st, par, abort_flag, err) ||
-                            !mbar_wait(s_empty + 8 * st, par ^ 1u, abort_flag, err)) {
+                            !mbar_wait(pv_done + 8 * st, par ^ 1u, abort_flag, err)) {
                             ok = false;
                             break;
                         }
@@ -248,8 +311,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     if (j > 0) {
                         // P_jj is complete (and O rescaled where a row's maximum moved)
-                        const int jj = j - 1, t = kt0 + jj, st = t & 1;
-                        const uint32_t par = (t >> 1) & 1;
+                        const int jj = j - 1, t = kt0 + jj, st = t % NST;
+                        const uint32_t par = (t / NST) & 1;
                         if (!mbar_wait(p_full + 8 * st, par, abort_flag, err) ||
                             !mbar_wait(v_full + 8 * st, par, abort_flag, err) ||
                             (jj == 0 && ni > 0 && !mbar_wait(o_free, (uint32_t)((ni - 1) & 1), abort_flag, err))) {
@@ -257,18 +320,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t d_o = tmem + 256u;
+                        const uint32_t d_o = tmem + C::O_COL;
+                        const uint32_t p_t = tmem + (uint32_t)(st * 128);   // P_t over S_t's first 64 columns
 #pragma unroll
                         for (int kk = 0; kk < BKV / 16; ++kk) {
-                            // A = P (K-major, keys contiguous); B = V (MN-major): 16 keys = 2 groups of 8 rows
-                            const uint32_t poff = (kk >> 2) * C::REG + (kk & 3) * 32;
+                            // A = P from TMEM (16 keys = 8 columns); B = V (MN-major): 16 keys = 2 groups of 8 rows
                             uint64_t vd = sw128_desc(sV + st * C::TILE + kk * 2048);
                             vd = (vd & ~(((uint64_t)0x3FFF) << 16)) | ((uint64_t)(C::REG >> 4) << 16);   // LBO: next 64 hd
-                            umma_bf16(d_o, sw128_desc(sP + st * C::P_TILE + poff), vd, IDESC_PV,
-                                      (jj > 0 || kk > 0) ? 1u : 0u);
+                            umma_bf16_tmem_a(d_o, p_t + 8u * kk, vd, IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
                         }
                         umma_commit(o_done);
-                        umma_commit(v_empty + 8 * st);
+                        umma_commit(pv_done + 8 * st);
                         if (jj == n_kv - 1) umma_commit(o_last);
                     }
                 }
@@ -280,18 +342,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int quarter = warp & 3;
         const int t_row = quarter * 32 + lane;           // query row within the tile
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        const uint32_t o_addr = tmem + lane_addr + 256u;
+        const uint32_t o_addr = tmem + lane_addr + C::O_COL;
         bool ok = true;
-        int kt0 = 0, ni = 0;
-        for (int it = item_at(0); it < total && ok; it = item_at(++ni)) {
+        int kt0 = 0;
+        for (int ni = 0; ok; ++ni) {
+            bool got;
+            const int it = next_item(ni, got);
+            if (!__all_sync(0xffffffffu, got)) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(item_empty + 8 * (ni & 1));
+            if (it >= total) break;
             int qt, h, b;
             item(it, qt, h, b);
             const int n_kv = qt + 1;
             const int q = qt * BQ + t_row;
             float m = -INFINITY, l = 0.f;                // running maximum (log2 units) and row sum
             for (int j = 0; j < n_kv; ++j) {
-                const int t = kt0 + j, st = t & 1;
-                const uint32_t par = (t >> 1) & 1;
+                const int t = kt0 + j, st = t % NST;
+                const uint32_t par = (t / NST) & 1;
                 // warp-uniform decision: the TMEM loads below are warp-collective
                 if (!__all_sync(0xffffffffu, mbar_wait(s_full + 8 * st, par, abort_flag, err))) {
                     ok = false;
@@ -333,27 +401,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     m = mt;
                     rescale = true;
                 }
-                // pass 2: probabilities (bf16) into the P tile; the row sum adds
-                // the fp32 values in four independent partial sums
+                // pass 2: probabilities (bf16 pairs, key 2c in the low half of
+                // column c) into this row's TMEM lane over the first 64 columns
+                // of S_t (read out above); the row sum adds the fp32 values in
+                // four independent partial sums
                 float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-                const uint32_t pbase = sP + st * C::P_TILE;
+                const uint32_t p_addr = tmem + lane_addr + (uint32_t)(st * 128);
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {           // 16 chunks of 8 keys (16 bytes of P)
-                    uint32_t pk[4];
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[32];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float p0 = ex2_approx(fmaf(sv[8 * c + 2 * i], scale_log2, -m));
-                        const float p1 = ex2_approx(fmaf(sv[8 * c + 2 * i + 1], scale_log2, -m));
+                    for (int i = 0; i < 32; ++i) {
+                        const float p0 = ex2_approx(fmaf(sv[64 * half + 2 * i], scale_log2, -m));
+                        const float p1 = ex2_approx(fmaf(sv[64 * half + 2 * i + 1], scale_log2, -m));
                         pk[i] = pack_bf16x2(p0, p1);
-                        rs4[i] += p0 + p1;
+                        rs4[i & 3] += p0 + p1;
                     }
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_chunk_addr(pbase, t_row, c)),
-                                 "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
-                                 : "memory");
+                    tmem_st32u(p_addr + 32 * half, pk);
                 }
                 const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-                tc_fence_before();
-                mbar_arrive(s_empty + 8 * st);
+                tmem_st_wait();
                 // a warp with a moved maximum rescales its 32 rows of O once the
                 // previous P V product is done.  Its completion is phase t - 1 of
                 // o_done: S_t's completion (waited for above) follows that of
@@ -378,7 +445,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tc_fence_before();
                 }
                 l = l * corr + rs;
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                tc_fence_before();
                 mbar_arrive(p_full + 8 * st);
             }
             // the item's last product: O / l, bf16, to global; then O is free for the next item
@@ -415,6 +482,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
                      : "memory");
+    }
+    if (threadIdx.x == 0) {
+        // this CTA claims no more items; the last CTA to finish zeroes the
+        // counters for the next launch
+        __threadfence();
+        if (atomicAdd(sched + 1, 1) == G - 1) {
+            atomicExch(sched, 0);
+            atomicExch(sched + 1, 0);
+        }
     }
 }
 
@@ -466,9 +542,10 @@ int attention_tc_prepare() {
 }
 
 int launch_attention_prefill_tc(const void* q, const void* k, const void* v, void* o, int B, int H, int Hkv, int S,
-                                int hd, int kv_stride, int* err, cudaStream_t st, const int* pages, int pps,
+                                int hd, int kv_stride, int* err, int* sched, cudaStream_t st, const int* pages, int pps,
                                 int n_pages) {
     if (B <= 0 || S <= 0) return LLAMA_OK;
+    if (!sched) return LLAMA_ERR_INVALID_ARG;
     if (hd != 64 && hd != 128) return LLAMA_ERR_INVALID_ARG;
     if (Hkv <= 0 || H % Hkv != 0) return LLAMA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
@@ -492,14 +569,20 @@ int launch_attention_prefill_tc(const void* q, const void* k, const void* v, voi
     static int n_sm = 0;
     if (!n_sm) n_sm = tc_num_sms();
     dim3 grid(items < n_sm ? items : n_sm);
+    // heads per block of work items: the key and value bytes of a block's
+    // heads (all positions) about 32 MB, so two blocks in flight stay well
+    // inside L2; at least 8 heads, for the balance of the CTAs' loads
+    const double kv_head_bytes = 4.0 * S * hd / (H / Hkv);
+    int hblk = (int)(32.0 * (1 << 20) / kv_head_bytes);
+    hblk = std::max(8, std::min(hblk, H * B));
     if (hd == 128) {
         if ((rc = attn_attr<128>())) return rc;
         launch_pdl(attn_prefill_tc_kernel<128>, grid, dim3(NTHREADS), ACfg<128>::SMEM, st, mq, mk, mv, (bf16*)o, H, S,
-                   Hkv, B, scale_log2, pages, pps, err);
+                   Hkv, B, scale_log2, pages, pps, hblk, sched, err);
     } else {
         if ((rc = attn_attr<64>())) return rc;
         launch_pdl(attn_prefill_tc_kernel<64>, grid, dim3(NTHREADS), ACfg<64>::SMEM, st, mq, mk, mv, (bf16*)o, H, S,
-                   Hkv, B, scale_log2, pages, pps, err);
+                   Hkv, B, scale_log2, pages, pps, hblk, sched, err);
     }
     LLAMA_LAUNCH_CHECK();
     return LLAMA_OK;

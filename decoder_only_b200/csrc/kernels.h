@@ -45,9 +45,11 @@ int attention_prepare();  // sets kernel attributes; call before any stream capt
 
 // attn_tc.cu  (bf16 tcgen05 causal flash attention, head_dim 64 or 128)
 // pages (device, [B][pps] page ids) != NULL: k and v are page pools of n_pages pages [Hkv][128][hd]
+// sched: two device ints, zero before the first launch and left zero by each
+// launch (the work-item counter); launches sharing them must not overlap
 int launch_attention_prefill_tc(const void* q, const void* k, const void* v, void* o, int B, int H, int Hkv, int S,
-                                int hd, int kv_stride, int* err, cudaStream_t st, const int* pages = nullptr,
-                                int pps = 0, int n_pages = 0);
+                                int hd, int kv_stride, int* err, int* sched, cudaStream_t st,
+                                const int* pages = nullptr, int pps = 0, int n_pages = 0);
 int attention_tc_prepare();
 
 // decode.cu

@@ -132,6 +132,8 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Error word of the standalone ops (the model has its own in its arena).
 __device__ int g_op_err_word;
+// Work-item counters of the standalone prefill attention op.
+__device__ int g_op_attn_sched[2];
 
 // Its device address on the current device: in host code the variable's
 // name is only a host-side stand-in, so the address is looked up once per
@@ -144,6 +146,26 @@ int op_error_word(int** p) {
     int rc = once_per_device(once, [dev]() -> int {
         void* a = nullptr;
         if (cudaGetSymbolAddress(&a, g_op_err_word) != cudaSuccess || !a) {
+            cudaGetLastError();
+            return (int)LLAMA_ERR_CUDA;
+        }
+        addr[dev] = static_cast<int*>(a);
+        return (int)LLAMA_OK;
+    });
+    if (rc) return rc;
+    *p = addr[dev];
+    return LLAMA_OK;
+}
+
+// The same for the standalone attention op's work-item counters.
+int op_attn_sched(int** p) {
+    static PerDeviceOnce once;
+    static int* addr[LLAMA_MAX_DEVICES];
+    int dev = -1;
+    LLAMA_CUDA_TRY(cudaGetDevice(&dev));
+    int rc = once_per_device(once, [dev]() -> int {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_op_attn_sched) != cudaSuccess || !a) {
             cudaGetLastError();
             return (int)LLAMA_ERR_CUDA;
         }
@@ -193,6 +215,7 @@ struct llama_model {
     float* trunk_last;       // last-position trunk rows [max_batch, d]
     int* d_pos;              // decode position
     int* d_err;              // sticky device error word
+    int* attn_sched;         // prefill attention's work-item counters (2 ints, zero between launches)
     int B;                   // batch of the last prefill (0: none)
     int cur_len;             // largest position over the sequences (host)
     std::vector<int> pos_h;  // host mirror of d_pos: each sequence's position (ragged batches)
@@ -399,6 +422,7 @@ uint64_t layout(const llama_config* c, llama_model* m, uint8_t* base) {
         m->trunk_last = trunk_last;
         m->d_pos = d_posv;
         m->d_err = small + 1;
+        m->attn_sched = small + 8;
     }
     return off;
 }
@@ -528,7 +552,8 @@ int run_blocks(llama_model* m, int B, int S, bool decode, cudaStream_t st) {
             prof::Scope ps(st, "prefill_attention", 4.0 * n * d * m->esz, 2.0 * B * (double)S * (S + 1) * d);
             if (dt == LLAMA_BF16)
                 rc = launch_attention_prefill_tc(m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, Hkv, S,
-                                                 c.head_dim, c.max_seq, m->d_err, st, m->pages, m->pps, c.kv_pages);
+                                                 c.head_dim, c.max_seq, m->d_err, m->attn_sched, st, m->pages, m->pps,
+                                                 c.kv_pages);
             else
                 rc = launch_attention_prefill_simt(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, c.n_heads, Hkv, S,
                                                    c.head_dim, c.max_seq, st);
@@ -631,7 +656,8 @@ int run_blocks_tp(llama_model* m, int B, int S, cudaStream_t st) {
             prof::Scope ps(st, "prefill_attention", 4.0 * n * dq * m->esz, 2.0 * B * (double)S * (S + 1) * dq);
             if (dt == LLAMA_BF16)
                 rc = launch_attention_prefill_tc(m->q, kcache(m, l), vcache(m, l), m->attn, B, m->Hl, m->Hkvl, S,
-                                                 c.head_dim, c.max_seq, m->d_err, st, m->pages, m->pps, c.kv_pages);
+                                                 c.head_dim, c.max_seq, m->d_err, m->attn_sched, st, m->pages, m->pps,
+                                                 c.kv_pages);
             else
                 rc = launch_attention_prefill_simt(dt, m->q, kcache(m, l), vcache(m, l), m->attn, B, m->Hl, m->Hkvl,
                                                    S, c.head_dim, c.max_seq, st);
@@ -1360,7 +1386,9 @@ int llama_op_attention_prefill(int32_t dtype, const void* d_q, const void* d_k, 
     int* err = nullptr;
     int rc = op_error_word(&err);
     if (rc) return rc;
-    return launch_attention_prefill_tc(d_q, d_k, d_v, d_o, B, H, H, S, head_dim, kv_stride, err,
+    int* sched = nullptr;
+    if ((rc = op_attn_sched(&sched))) return rc;
+    return launch_attention_prefill_tc(d_q, d_k, d_v, d_o, B, H, H, S, head_dim, kv_stride, err, sched,
                                        (cudaStream_t)stream);
 }
 

@@ -333,7 +333,9 @@ LLAMA_API int llama_op_gemm(int32_t dtype, const void* d_A, const void* d_W, flo
  * [B][H][*][head_dim]; q has S rows per head, k/v have kv_stride rows per
  * head (>= S; the first S are used).  o dtype-typed [B*S, H*head_dim]:
  * row b*S + t, columns of head h at [h*head_dim, (h+1)*head_dim).
- * Scale 1/sqrt(head_dim); key j is visible to query t iff j <= t. */
+ * Scale 1/sqrt(head_dim); key j is visible to query t iff j <= t.
+ * The bf16 kernel's CTAs take work items from a counter that each call
+ * leaves zero: calls on one device run one at a time (stream-ordered). */
 LLAMA_API int llama_op_attention_prefill(int32_t dtype, const void* d_q, const void* d_k,
                                const void* d_v, void* d_o, int32_t B, int32_t H,
                                int32_t S, int32_t head_dim, int32_t kv_stride,
