@@ -8,37 +8,41 @@
 // knowledge note credits to the xFormers attention of the training system.
 //
 // Persistent CTAs, one per SM, each working through a list of work items
-// (128-query tile, head, sequence) that it claims from a global counter;
-// the rings and barriers run on over item boundaries, so the next item's Q,
-// K and first scores load and compute while the current item's output is
-// written.
-//   warp 0      TMA: lane 0 claims the items, loads each item's Q (once the
-//               previous item's last Q K^T is done), then its K_j tiles;
-//               lane 1 the V_j tiles.  Three-stage rings: a tile is fetched
-//               three tiles ahead of its use, which covers the load latency
-//               from L2 (about 2 us for a 32 KB tile when all SMs stream
-//               keys and values).  3-D tensor maps (hd, position, head) make
+// -- a pair of adjacent 128-query tiles a, b of one (head, sequence), which
+// share every key / value tile they read -- that it claims from a global
+// counter; the rings and barriers run on over item boundaries, so the next
+// item's Q, K and first scores load and compute while the current item's
+// output is written.  Sharing each key / value tile between two query tiles
+// halves the bytes streamed from L2 per product: with one query tile per
+// CTA the TMA delivery of K and V (about 23 B per clock per SM with the
+// products and the softmax running) bounded the kernel.
+//   warp 0      TMA: lane 0 claims the items, loads each item's Q tiles
+//               (once the previous item's last Q K^T products are done),
+//               then its K_j tiles (three-stage ring); lane 1 the V_j tiles
+//               (two stages).  3-D tensor maps (hd, position, head) make
 //               rows >= S read as 0.
-//   warp 1      TMEM allocator + MMA issuer:
-//                 S_j = Q K_j^T      (M 128, N 128, K hd)  -> TMEM stage j % 3
-//                 O  += P_j V_j      (M 128, N hd, K 128)  -> TMEM O (one
-//                                     accumulator per work item)
-//               P_j is the A operand read from tensor memory (written over
-//               S_j by the softmax), V the MN-major B operand (hd
+//   warp 1      TMEM allocator + MMA issuer, an event loop over x in {a, b}:
+//                 S_x = Q_x K_j^T    (M 128, N 128, K hd)  -> TMEM S_x
+//                 O_x += P_x V_j     (M 128, N hd, K 128)  -> TMEM O_x
+//               P_x is the A operand read from tensor memory (written over
+//               S_x by the softmax), V the MN-major B operand (hd
 //               contiguous), so the cache layout [position][hd] is used as
-//               is.  A stage is free for S_{j+3} once P_j V_j is done.
-//   warps 2..5  one query row per thread: the row's 128 scores into
-//               registers (one TMEM read), row max (pass 1), then p =
-//               2^(s log2e / sqrt(hd) - m) rounded to bf16 into the row's
-//               TMEM lane and the row sum in fp32 (pass 2).  The running
-//               maximum m (log2 units) moves only when a tile's maximum
-//               exceeds it by more than 8: p stays <= 2^8, exact in fp32 and
-//               bf16's range, and the output in TMEM is rescaled by
-//               2^(m_old - m_new) (TMEM load, scale, store, after the
-//               previous P V product) only then -- a few times per row --
-//               instead of folding every tile's product into registers.
-//               After an item's last tile: O / (row sum), bf16, to global;
-//               the next item's first P V product waits for that read.
+//               is.  S_x(j + 1) is computed once P_x(j) V_j has completed
+//               (it overwrites the P_x it read); meanwhile the other tile's
+//               products run, so one tile's softmax overlaps the other's
+//               MMAs.
+//   warps 2..5  softmax of tile a, warps 6..9 of tile b, one query row per
+//               thread: the row's 128 scores into registers (one TMEM read),
+//               row max (pass 1), then p = 2^(s log2e / sqrt(hd) - m) rounded
+//               to bf16 into the row's TMEM lane and the row sum in fp32
+//               (pass 2).  The running maximum m (log2 units) moves only when
+//               a tile's maximum exceeds it by more than 8: p stays <= 2^8,
+//               exact in fp32 and bf16's range, and the output in TMEM is
+//               rescaled by 2^(m_old - m_new) (TMEM load, scale, store) only
+//               then -- a few times per row -- instead of folding every
+//               tile's product into registers.  After an item's last tile:
+//               O_x / (row sum), bf16, to global; the next item's first
+//               P_x V product waits for that read.
 // All mbarrier waits are bounded (see tcgen05.cuh).
 #include <cudaTypedefs.h>
 
@@ -55,7 +59,7 @@ using namespace tc;
 
 constexpr int BQ = 128;         // queries per tile
 constexpr int BKV = 128;        // keys per tile
-constexpr int NTHREADS = 192;
+constexpr int NTHREADS = 320;   // warp 0 TMA, warp 1 MMA, warps 2..5 softmax of tile a, 6..9 of tile b
 constexpr float RESCALE_LOG2 = 8.f;   // move the running maximum only by more than this (log2 units)
 
 // 2^x by the special-function unit's approximation (one instruction;
@@ -66,22 +70,35 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-constexpr int NST = 3;          // stages of the K, V and S / P rings
+constexpr int NSK = 3;          // stages of the key ring
+constexpr int NSV = 2;          // stages of the value ring
 
 template <int HD>
 struct ACfg {
     static constexpr int REG = 128 * 128;                    // one [128 rows][64 bf16] swizzled region, bytes
     static constexpr int NREG = HD / 64;                     // regions per Q / K / V tile
     static constexpr int TILE = NREG * REG;                  // Q, K or V tile bytes
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + TILE;               // [NST]
-    static constexpr int OFF_V = OFF_K + NST * TILE;         // [NST]
-    static constexpr int OFF_BAR = OFF_V + NST * TILE;
+    static constexpr int OFF_Q = 0;                          // [2]: tiles a, b
+    static constexpr int OFF_K = OFF_Q + 2 * TILE;           // [NSK]
+    static constexpr int OFF_V = OFF_K + NSK * TILE;         // [NSV]
+    static constexpr int OFF_BAR = OFF_V + NSV * TILE;
     static constexpr int SMEM = OFF_BAR + 512 + 1024;
-    static constexpr uint32_t TMEM_COLS = 512;               // S / P [NST] at 0, 128, 256; O at 384
-    static constexpr uint32_t O_COL = 128 * NST;
+    static constexpr uint32_t TMEM_COLS = 512;               // S / P of tiles a, b at 0, 128; O at 256, 384
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
+
+// Non-blocking probe of an mbarrier phase (for the MMA issuer's event loop).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 
 // A x B with A (M x K, bf16) read from tensor memory: row m in lane m, K along
 // the columns, two values per 32-bit column; B from shared memory.
@@ -121,40 +138,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t sQ = base + C::OFF_Q, sK = base + C::OFF_K, sV = base + C::OFF_V;
     const uint32_t bars = base + C::OFF_BAR;
     const uint32_t q_full = bars;
-    const uint32_t q_empty = bars + 8;       // one phase per work item: its last Q K^T (Q free)
-    const uint32_t o_done = bars + 16;       // one phase per completed P V product
-    const uint32_t o_last = bars + 24;       // one phase per work item: its last P V product
-    const uint32_t o_free = bars + 32;       // one phase per work item: its output read out of TMEM
-    const uint32_t k_full = bars + 40;       // [NST]
-    const uint32_t k_empty = bars + 64;      // [NST] Q K_t^T done: K stage free
-    const uint32_t v_full = bars + 88;       // [NST]
-    const uint32_t pv_done = bars + 112;     // [NST] P_t V_t done: V stage and S / P stage free
-    const uint32_t s_full = bars + 136;      // [NST]
-    const uint32_t p_full = bars + 160;      // [NST] P_t in TMEM (and O rescaled)
-    const uint32_t item_full = bars + 184;   // [2] a work item's index published in item_ring
-    const uint32_t item_empty = bars + 200;  // [2] read by all six consumers (V lane, MMA, 4 softmax warps)
+    const uint32_t q_empty = bars + 8;       // one phase per work item: its last Q K^T products done
+    const uint32_t k_full = bars + 16;       // [NSK]
+    const uint32_t k_empty = bars + 40;      // [NSK] every Q K_j^T of the key tile done
+    const uint32_t v_full = bars + 64;       // [NSV]
+    const uint32_t v_empty = bars + 80;      // [NSV] every P V_j of the value tile done
+    const uint32_t s_full = bars + 96;       // [2] per query tile x: S_x(n) in TMEM
+    const uint32_t p_full = bars + 112;      // [2] per x: P_x(n) in TMEM (and O_x rescaled); 128 arrivals
+    const uint32_t pv_done = bars + 128;     // [2] per x: P_x(n) V done -- S_x / P_x free, O_x current
+    const uint32_t o_last = bars + 144;      // [2] per x: the item's last P_x V done
+    const uint32_t o_free = bars + 160;      // [2] per x: O_x read out of TMEM; 128 arrivals
+    const uint32_t item_full = bars + 176;   // [2] a work item's index published in item_ring
+    const uint32_t item_empty = bars + 192;  // [2] read by the ten consumers (V lane, MMA, 8 softmax warps)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 256);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* item_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);   // [2]
 
-    // Work items (128-query tile, head, sequence) in blocks of hblk heads,
-    // longest (most key tiles) first within a block: the items running at
-    // one time share the key and value tiles of a few heads in L2.  Each
-    // CTA starts with item blockIdx.x and then takes the next unclaimed one
-    // from a global counter (sched[0]) whenever it is ready for another, so
-    // the CTAs finish together however the item lengths fall.  Lane 0 of
-    // warp 0 claims the items and publishes them to the other roles through
-    // a two-entry ring; the tile rings and barriers run on over item
-    // boundaries, so one item's start overlaps the previous one's end.
+    // Work items: a pair of adjacent 128-query tiles a = 2p, b = 2p + 1 of one
+    // (head, sequence), which share every key / value tile they read (b reads
+    // one more).  Items come in blocks of hblk heads, longest (most key tiles)
+    // first within a block, so the items running at one time share the key
+    // and value tiles of a few heads in L2.  Each CTA starts with item
+    // blockIdx.x and then claims the next unclaimed one from a global counter
+    // (sched[0]) whenever it is ready for another; lane 0 of warp 0 claims and
+    // publishes them to the other roles through a two-entry ring.  All rings
+    // and barriers run on across items.
     const int n_qt = (S + BQ - 1) / BQ;
-    const int total = n_qt * H * B;
+    const int n_qp = (n_qt + 1) / 2;
+    const int total = n_qp * H * B;
     const int G = (int)gridDim.x;
-    auto item = [&](int it, int& qt, int& h, int& b) {
-        const int per = hblk * n_qt;
+    auto item = [&](int it, int& pr, int& h, int& b) {
+        const int per = hblk * n_qp;
         const int k = it / per;
         const int r = it - k * per;
         const int gg = min(hblk, H * B - k * hblk);
-        qt = n_qt - 1 - r / gg;
+        pr = n_qp - 1 - r / gg;
         const int hb = k * hblk + r % gg;
         h = hb % H;
         b = hb / H;
@@ -170,21 +188,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int i = 0; i < NST; ++i) {
+        mbar_init(q_empty, 1);
+        for (int i = 0; i < NSK; ++i) {
             mbar_init(k_full + 8 * i, 1);
             mbar_init(k_empty + 8 * i, 1);
-            mbar_init(v_full + 8 * i, 1);
-            mbar_init(pv_done + 8 * i, 1);
-            mbar_init(s_full + 8 * i, 1);
-            mbar_init(p_full + 8 * i, 128);
         }
-        mbar_init(o_done, 1);
-        mbar_init(o_last, 1);
-        mbar_init(q_empty, 1);
-        mbar_init(o_free, 128);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(item_full + 8 * i, 1);
-            mbar_init(item_empty + 8 * i, 6);
+        for (int i = 0; i < NSV; ++i) {
+            mbar_init(v_full + 8 * i, 1);
+            mbar_init(v_empty + 8 * i, 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(s_full + 8 * x, 1);
+            mbar_init(p_full + 8 * x, 128);
+            mbar_init(pv_done + 8 * x, 1);
+            mbar_init(o_last + 8 * x, 1);
+            mbar_init(o_free + 8 * x, 128);
+            mbar_init(item_full + 8 * x, 1);
+            mbar_init(item_empty + 8 * x, 10);
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -204,10 +224,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
         if (lane < 2) {
-            // lane 0: each item's Q (once the previous item's last Q K^T is done), then its K_j;
-            // lane 1: the V_j
+            // lane 0: claims and publishes the items; each item's Q tiles (once the
+            // previous item's last Q K^T products are done), then its K_j; lane 1: the V_j
             const bool is_k = (lane == 0);
-            const uint32_t full = is_k ? k_full : v_full, empty = is_k ? k_empty : pv_done;
+            const int ns = is_k ? NSK : NSV;
+            const uint32_t full = is_k ? k_full : v_full, empty = is_k ? k_empty : v_empty;
             const uint32_t dst = is_k ? sK : sV;
             const CUtensorMap* map = is_k ? &tmK : &tmV;
             bool ok = true;
@@ -215,7 +236,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int it = blockIdx.x;
             for (;; ++ni) {
                 if (is_k) {
-                    // publish item ni (after all six consumers have read item ni - 2 from its slot)
+                    // publish item ni (after all ten consumers have read item ni - 2 from its slot)
                     const int slot = ni & 1;
                     if (ni >= 2 && !mbar_wait(item_empty + 8 * slot, (uint32_t)(((ni >> 1) - 1) & 1), abort_flag, err)) {
                         ok = false;
@@ -229,22 +250,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     mbar_arrive(item_empty + 8 * (ni & 1));
                 }
                 if (it >= total) break;
-                int qt, h, b;
-                item(it, qt, h, b);
+                int pr, h, b;
+                item(it, pr, h, b);
+                const bool has_b = 2 * pr + 1 < n_qt;
+                const int nk = has_b ? 2 * pr + 2 : 2 * pr + 1;     // key tiles of the pair
                 const int kv_head = b * Hkv + h / (H / Hkv);      // grouped keys and values
                 if (is_k) {
                     if (ni > 0 && !mbar_wait(q_empty, (uint32_t)((ni - 1) & 1), abort_flag, err)) {
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(q_full, C::TILE);
-                    for (int r = 0; r < C::NREG; ++r)
-                        tma_load_3d(sQ + r * C::REG, &tmQ, q_full, 64 * r, qt * BQ, b * H + h);
+                    mbar_expect_tx(q_full, (has_b ? 2 : 1) * C::TILE);
+                    for (int r = 0; r < C::NREG; ++r) {
+                        tma_load_3d(sQ + r * C::REG, &tmQ, q_full, 64 * r, 2 * pr * BQ, b * H + h);
+                        if (has_b) tma_load_3d(sQ + C::TILE + r * C::REG, &tmQ, q_full, 64 * r, (2 * pr + 1) * BQ, b * H + h);
+                    }
                     ++q_loads;
                 }
-                for (int j = 0; j <= qt; ++j, ++kt) {
-                    const int st = kt % NST;
-                    if (!mbar_wait(empty + 8 * st, ((kt / NST) & 1) ^ 1u, abort_flag, err)) {
+                for (int j = 0; j < nk; ++j, ++kt) {
+                    const int st = kt % ns;
+                    if (!mbar_wait(empty + 8 * st, ((kt / ns) & 1) ^ 1u, abort_flag, err)) {
                         ok = false;
                         break;
                     }
@@ -263,88 +288,138 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 while (is_k && q_loads > 0 && !mbar_try_wait(q_full, (uint32_t)((q_loads - 1) & 1)) &&
                        global_timer() - t0 < WAIT_LIMIT_NS / 4) {
                 }
-                for (int t = kt > NST ? kt - NST : 0; t < kt; ++t) {
-                    const uint32_t par = (t / NST) & 1;
-                    while (!mbar_try_wait(full + 8 * (t % NST), par) && global_timer() - t0 < WAIT_LIMIT_NS / 2) {
+                for (int t = kt > ns ? kt - ns : 0; t < kt; ++t) {
+                    const uint32_t par = (t / ns) & 1;
+                    while (!mbar_try_wait(full + 8 * (t % ns), par) && global_timer() - t0 < WAIT_LIMIT_NS / 2) {
                     }
                 }
             }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
+        // An event loop over the two query tiles x: S_x(j) = Q_x K_j^T once K_j has
+        // landed and the previous P_x V product has completed (S_x(j) overwrites
+        // the P_x it read); O_x += P_x(j) V_j once the softmax has written P_x(j)
+        // and V_j has landed.  One tile's softmax overlaps the other tile's products.
         if (lane == 0) {
             constexpr uint32_t IDESC_QK = idesc_bf16(BKV);                 // K-major A and B
             constexpr uint32_t IDESC_PV = idesc_bf16(HD) | (1u << 16);      // B (V) MN-major
             bool ok = true;
-            int kt0 = 0;
+            int kv0 = 0;                                // key / value tiles of earlier items
+            int sc[2] = {0, 0}, pc[2] = {0, 0};         // S_x / P_x V products issued so far (all items)
+            int nix[2] = {0, 0};                        // items in which tile x took part
             for (int ni = 0; ok; ++ni) {
                 const int it = next_item(ni, ok);
                 if (!ok) break;
                 mbar_arrive(item_empty + 8 * (ni & 1));
                 if (it >= total) break;
-                int qt, h, b;
-                item(it, qt, h, b);
-                const int n_kv = qt + 1;
+                int pr, h, b;
+                item(it, pr, h, b);
+                const bool has_b = 2 * pr + 1 < n_qt;
+                const int nkx[2] = {2 * pr + 1, has_b ? 2 * pr + 2 : 0};
+                const int nk = has_b ? nkx[1] : nkx[0];
                 ok = mbar_wait(q_full, (uint32_t)(ni & 1), abort_flag, err);
                 tc_fence_after();
-                for (int j = 0; j <= n_kv && ok; ++j) {
-                    if (j < n_kv) {
-                        // S_t into stage t % NST, once P_{t - NST} V_{t - NST} has read that stage
-                        const int t = kt0 + j, st = t % NST;
-                        const uint32_t par = (t / NST) & 1;
-                        if (!mbar_wait(k_full + 8 * st, par, abort_flag, err) ||
-                            !mbar_wait(pv_done + 8 * st, par ^ 1u, abort_flag, err)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t d_s = tmem + (uint32_t)(st * 128);
+                int js[2] = {0, 0}, jp[2] = {0, 0};     // this item's next S_x / P_x V tile
+                int krel = 0, vrel = 0;
+                bool q_rel = false;
+                uint64_t t_last = global_timer();
+                while (ok && (krel < nk || vrel < nk || !q_rel)) {
+                    bool prog = false;
 #pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk) {
-                            const uint32_t off = (kk >> 2) * C::REG + (kk & 3) * 32;
-                            umma_bf16(d_s, sw128_desc(sQ + off), sw128_desc(sK + st * C::TILE + off), IDESC_QK,
-                                      kk > 0 ? 1u : 0u);
+                    for (int x = 0; x < 2; ++x) {
+                        // O_x += P_x(j) V_j
+                        const int j = jp[x];
+                        if (j < js[x] && mbar_test(p_full + 8 * x, (uint32_t)(pc[x] & 1)) &&
+                            mbar_test(v_full + 8 * ((kv0 + j) % NSV), (uint32_t)(((kv0 + j) / NSV) & 1)) &&
+                            (j > 0 || nix[x] == 0 || mbar_test(o_free + 8 * x, (uint32_t)((nix[x] - 1) & 1)))) {
+                            tc_fence_after();
+                            const uint32_t d_o = tmem + 256u + 128u * x;
+                            const uint32_t p_t = tmem + 128u * x;     // P_x over S_x's first 64 columns
+                            const uint32_t v_t = sV + ((kv0 + j) % NSV) * C::TILE;
+#pragma unroll
+                            for (int kk = 0; kk < BKV / 16; ++kk) {
+                                // A = P from TMEM (16 keys = 8 columns); B = V (MN-major): 16 keys = 2 groups of 8 rows
+                                uint64_t vd = sw128_desc(v_t + kk * 2048);
+                                vd = (vd & ~(((uint64_t)0x3FFF) << 16)) | ((uint64_t)(C::REG >> 4) << 16);   // LBO: next 64 hd
+                                umma_bf16_tmem_a(d_o, p_t + 8u * kk, vd, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+                            }
+                            umma_commit(pv_done + 8 * x);
+                            if (j == nkx[x] - 1) umma_commit(o_last + 8 * x);
+                            ++pc[x];
+                            jp[x] = j + 1;
+                            prog = true;
                         }
-                        umma_commit(s_full + 8 * st);
-                        umma_commit(k_empty + 8 * st);
-                        if (j == n_kv - 1) umma_commit(q_empty);   // Q free for the next item
                     }
-                    if (j > 0) {
-                        // P_jj is complete (and O rescaled where a row's maximum moved)
-                        const int jj = j - 1, t = kt0 + jj, st = t % NST;
-                        const uint32_t par = (t / NST) & 1;
-                        if (!mbar_wait(p_full + 8 * st, par, abort_flag, err) ||
-                            !mbar_wait(v_full + 8 * st, par, abort_flag, err) ||
-                            (jj == 0 && ni > 0 && !mbar_wait(o_free, (uint32_t)((ni - 1) & 1), abort_flag, err))) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t d_o = tmem + C::O_COL;
-                        const uint32_t p_t = tmem + (uint32_t)(st * 128);   // P_t over S_t's first 64 columns
 #pragma unroll
-                        for (int kk = 0; kk < BKV / 16; ++kk) {
-                            // A = P from TMEM (16 keys = 8 columns); B = V (MN-major): 16 keys = 2 groups of 8 rows
-                            uint64_t vd = sw128_desc(sV + st * C::TILE + kk * 2048);
-                            vd = (vd & ~(((uint64_t)0x3FFF) << 16)) | ((uint64_t)(C::REG >> 4) << 16);   // LBO: next 64 hd
-                            umma_bf16_tmem_a(d_o, p_t + 8u * kk, vd, IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+                    for (int x = 0; x < 2; ++x) {
+                        // S_x(j) = Q_x K_j^T
+                        const int j = js[x];
+                        if (j < nkx[x] && jp[x] == j &&
+                            mbar_test(k_full + 8 * ((kv0 + j) % NSK), (uint32_t)(((kv0 + j) / NSK) & 1)) &&
+                            (sc[x] == 0 || mbar_test(pv_done + 8 * x, (uint32_t)((sc[x] - 1) & 1)))) {
+                            tc_fence_after();
+                            const uint32_t d_s = tmem + 128u * x;
+                            const uint32_t q_t = sQ + x * C::TILE, k_t = sK + ((kv0 + j) % NSK) * C::TILE;
+#pragma unroll
+                            for (int kk = 0; kk < HD / 16; ++kk) {
+                                const uint32_t off = (kk >> 2) * C::REG + (kk & 3) * 32;
+                                umma_bf16(d_s, sw128_desc(q_t + off), sw128_desc(k_t + off), IDESC_QK,
+                                          kk > 0 ? 1u : 0u);
+                            }
+                            umma_commit(s_full + 8 * x);
+                            ++sc[x];
+                            js[x] = j + 1;
+                            prog = true;
                         }
-                        umma_commit(o_done);
-                        umma_commit(pv_done + 8 * st);
-                        if (jj == n_kv - 1) umma_commit(o_last);
+                    }
+                    // release key / value tiles once every product that reads them is issued,
+                    // and the Q tiles once both tiles' last Q K^T is
+                    while (krel < nk && (krel >= nkx[0] || js[0] > krel) && (krel >= nkx[1] || js[1] > krel)) {
+                        umma_commit(k_empty + 8 * ((kv0 + krel) % NSK));
+                        ++krel;
+                        prog = true;
+                    }
+                    while (vrel < nk && (vrel >= nkx[0] || jp[0] > vrel) && (vrel >= nkx[1] || jp[1] > vrel)) {
+                        umma_commit(v_empty + 8 * ((kv0 + vrel) % NSV));
+                        ++vrel;
+                        prog = true;
+                    }
+                    if (!q_rel && js[0] == nkx[0] && js[1] == nkx[1]) {
+                        umma_commit(q_empty);
+                        q_rel = true;
+                        prog = true;
+                    }
+                    if (prog) {
+                        t_last = global_timer();
+                        continue;
+                    }
+                    if (*abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    if (global_timer() - t_last > WAIT_LIMIT_NS) {
+                        *abort_flag = 1;
+                        atomicOr(err, LLAMA_DEVERR_TIMEOUT);
+                        ok = false;
+                        break;
                     }
                 }
-                kt0 += n_kv;
+                kv0 += nk;
+                nix[0] += 1;
+                if (has_b) nix[1] += 1;
             }
         }
     } else {
-        // ---------------------------------------------------------- softmax + output (warps 2..5)
+        // ---------------------------------------------------------- softmax + output (warps 2..9)
+        const int x = (warp - 2) >> 2;                   // query tile a (0) or b (1)
         const int quarter = warp & 3;
         const int t_row = quarter * 32 + lane;           // query row within the tile
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        const uint32_t o_addr = tmem + lane_addr + C::O_COL;
+        const uint32_t o_addr = tmem + lane_addr + 256u + 128u * x;
+        const uint32_t s_addr = tmem + lane_addr + 128u * x;
         bool ok = true;
-        int kt0 = 0;
+        int sc = 0, nix = 0;                             // S_x tiles and items of tile x so far
         for (int ni = 0; ok; ++ni) {
             bool got;
             const int it = next_item(ni, got);
@@ -352,21 +427,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(item_empty + 8 * (ni & 1));
             if (it >= total) break;
-            int qt, h, b;
-            item(it, qt, h, b);
+            int pr, h, b;
+            item(it, pr, h, b);
+            const int qt = 2 * pr + x;
+            if (qt >= n_qt) continue;                    // the pair's second tile lies past S
             const int n_kv = qt + 1;
             const int q = qt * BQ + t_row;
             float m = -INFINITY, l = 0.f;                // running maximum (log2 units) and row sum
-            for (int j = 0; j < n_kv; ++j) {
-                const int t = kt0 + j, st = t % NST;
-                const uint32_t par = (t / NST) & 1;
+            for (int j = 0; j < n_kv; ++j, ++sc) {
                 // warp-uniform decision: the TMEM loads below are warp-collective
-                if (!__all_sync(0xffffffffu, mbar_wait(s_full + 8 * st, par, abort_flag, err))) {
+                if (!__all_sync(0xffffffffu, mbar_wait(s_full + 8 * x, (uint32_t)(sc & 1), abort_flag, err))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t s_addr = tmem + lane_addr + (uint32_t)(st * 128);
                 // the row's 128 scores, four TMEM loads in flight, one wait
                 float sv[128];
                 {
@@ -403,10 +477,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 // pass 2: probabilities (bf16 pairs, key 2c in the low half of
                 // column c) into this row's TMEM lane over the first 64 columns
-                // of S_t (read out above); the row sum adds the fp32 values in
+                // of S_x (read out above); the row sum adds the fp32 values in
                 // four independent partial sums
                 float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-                const uint32_t p_addr = tmem + lane_addr + (uint32_t)(st * 128);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[32];
@@ -417,22 +490,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         pk[i] = pack_bf16x2(p0, p1);
                         rs4[i & 3] += p0 + p1;
                     }
-                    tmem_st32u(p_addr + 32 * half, pk);
+                    tmem_st32u(s_addr + 32 * half, pk);
                 }
                 const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
                 tmem_st_wait();
-                // a warp with a moved maximum rescales its 32 rows of O once the
-                // previous P V product is done.  Its completion is phase t - 1 of
-                // o_done: S_t's completion (waited for above) follows that of
-                // P_{t-2} V_{t-2}, and P_t V_t waits for this warp, so the
-                // barrier is in phase t - 1 or t here.
+                // a warp with a moved maximum rescales its 32 rows of O_x: the
+                // previous P_x V product has completed (S_x(j) was issued after it)
                 if (__any_sync(0xffffffffu, rescale)) {
-                    bool w = mbar_wait(o_done, (uint32_t)((t - 1) & 1), abort_flag, err);
-                    if (!__all_sync(0xffffffffu, w)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
 #pragma unroll 1
                     for (int c = 0; c < HD / 32; ++c) {
                         float ov[32];
@@ -442,14 +506,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         tmem_st32(o_addr + c * 32, ov);
                     }
                     tmem_st_wait();
-                    tc_fence_before();
                 }
                 l = l * corr + rs;
                 tc_fence_before();
-                mbar_arrive(p_full + 8 * st);
+                mbar_arrive(p_full + 8 * x);
             }
-            // the item's last product: O / l, bf16, to global; then O is free for the next item
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_last, (uint32_t)(ni & 1), abort_flag, err));
+            // the tile's last product: O_x / l, bf16, to global; then O_x is free for the next item
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_last + 8 * x, (uint32_t)(nix & 1), abort_flag, err));
             if (!ok) break;
             tc_fence_after();
             const float inv = 1.f / l;
@@ -470,8 +533,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(o_free);
-            kt0 += n_kv;
+            mbar_arrive(o_free + 8 * x);
+            ++nix;
         }
     }
 
@@ -565,7 +628,7 @@ int launch_attention_prefill_tc(const void* q, const void* k, const void* v, voi
     }
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
     // persistent CTAs: one per SM (or per work item, if fewer)
-    const int items = ((S + BQ - 1) / BQ) * H * B;
+    const int items = (((S + BQ - 1) / BQ + 1) / 2) * H * B;
     static int n_sm = 0;
     if (!n_sm) n_sm = tc_num_sms();
     dim3 grid(items < n_sm ? items : n_sm);
