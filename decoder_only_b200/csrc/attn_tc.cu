@@ -629,8 +629,7 @@ int launch_attention_prefill_tc(const void* q, const void* k, const void* v, voi
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
     // persistent CTAs: one per SM (or per work item, if fewer)
     const int items = (((S + BQ - 1) / BQ + 1) / 2) * H * B;
-    static int n_sm = 0;
-    if (!n_sm) n_sm = tc_num_sms();
+    const int n_sm = tc_num_sms();
     dim3 grid(items < n_sm ? items : n_sm);
     // heads per block of work items: the key and value bytes of a block's
     // heads (all positions) about 32 MB, so two blocks in flight stay well

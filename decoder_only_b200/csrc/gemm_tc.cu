@@ -23,6 +23,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "kernels.h"
@@ -307,13 +309,15 @@ int make_map(CUtensorMap* map, const void* ptr, int rows, int K, int box_rows) {
     return r == CUDA_SUCCESS ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
+// SM count of the current device (looked up once per device)
 int num_sms() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
+    static std::atomic<int> cached[LLAMA_MAX_DEVICES];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= LLAMA_MAX_DEVICES) return 148;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
     return n;
 }
