@@ -73,6 +73,16 @@ __device__ __forceinline__ float ex2_approx(float x) {
 constexpr int NSK = 3;          // stages of the key ring
 constexpr int NSV = 2;          // stages of the value ring
 
+// mbarrier byte offsets in the barrier region (derived from the ring depths,
+// so that changing a depth cannot make two barriers share a word)
+constexpr int B_QFULL = 0, B_QEMPTY = 8, B_KFULL = 16;
+constexpr int B_KEMPTY = B_KFULL + 8 * NSK, B_VFULL = B_KEMPTY + 8 * NSK;
+constexpr int B_VEMPTY = B_VFULL + 8 * NSV, B_SFULL = B_VEMPTY + 8 * NSV;
+constexpr int B_PFULL = B_SFULL + 16, B_PVDONE = B_PFULL + 16, B_OLAST = B_PVDONE + 16;
+constexpr int B_OFREE = B_OLAST + 16, B_IFULL = B_OFREE + 16, B_IEMPTY = B_IFULL + 16;
+constexpr int B_WORDS = 256;    // tensor-memory slot, abort flag, item ring after the barriers
+static_assert(B_IEMPTY + 16 <= B_WORDS, "mbarrier region");
+
 template <int HD>
 struct ACfg {
     static constexpr int REG = 128 * 128;                    // one [128 rows][64 bf16] swizzled region, bytes
@@ -137,20 +147,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint8_t* gbase = smem_raw + (base - raw);
     const uint32_t sQ = base + C::OFF_Q, sK = base + C::OFF_K, sV = base + C::OFF_V;
     const uint32_t bars = base + C::OFF_BAR;
-    const uint32_t q_full = bars;
-    const uint32_t q_empty = bars + 8;       // one phase per work item: its last Q K^T products done
-    const uint32_t k_full = bars + 16;       // [NSK]
-    const uint32_t k_empty = bars + 40;      // [NSK] every Q K_j^T of the key tile done
-    const uint32_t v_full = bars + 64;       // [NSV]
-    const uint32_t v_empty = bars + 80;      // [NSV] every P V_j of the value tile done
-    const uint32_t s_full = bars + 96;       // [2] per query tile x: S_x(n) in TMEM
-    const uint32_t p_full = bars + 112;      // [2] per x: P_x(n) in TMEM (and O_x rescaled); 128 arrivals
-    const uint32_t pv_done = bars + 128;     // [2] per x: P_x(n) V done -- S_x / P_x free, O_x current
-    const uint32_t o_last = bars + 144;      // [2] per x: the item's last P_x V done
-    const uint32_t o_free = bars + 160;      // [2] per x: O_x read out of TMEM; 128 arrivals
-    const uint32_t item_full = bars + 176;   // [2] a work item's index published in item_ring
-    const uint32_t item_empty = bars + 192;  // [2] read by the ten consumers (V lane, MMA, 8 softmax warps)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 256);
+    const uint32_t q_full = bars + B_QFULL;
+    const uint32_t q_empty = bars + B_QEMPTY;    // one phase per work item: its last Q K^T products done
+    const uint32_t k_full = bars + B_KFULL;      // [NSK]
+    const uint32_t k_empty = bars + B_KEMPTY;    // [NSK] every Q K_j^T of the key tile done
+    const uint32_t v_full = bars + B_VFULL;      // [NSV]
+    const uint32_t v_empty = bars + B_VEMPTY;    // [NSV] every P V_j of the value tile done
+    const uint32_t s_full = bars + B_SFULL;      // [2] per query tile x: S_x(n) in TMEM
+    const uint32_t p_full = bars + B_PFULL;      // [2] per x: P_x(n) in TMEM (and O_x rescaled); 128 arrivals
+    const uint32_t pv_done = bars + B_PVDONE;    // [2] per x: P_x(n) V done -- S_x / P_x free, O_x current
+    const uint32_t o_last = bars + B_OLAST;      // [2] per x: the item's last P_x V done
+    const uint32_t o_free = bars + B_OFREE;      // [2] per x: O_x read out of TMEM; 128 arrivals
+    const uint32_t item_full = bars + B_IFULL;   // [2] a work item's index published in item_ring
+    const uint32_t item_empty = bars + B_IEMPTY; // [2] read by the ten consumers (V lane, MMA, 8 softmax warps)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + B_WORDS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* item_ring = reinterpret_cast<volatile int*>(tmem_slot + 2);   // [2]
 
