@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t empty_bar = bars + 8 * C::STAGES;            // [STAGES]
     const uint32_t tfull_bar = bars + 16 * C::STAGES;           // [2]
     const uint32_t tempty_bar = tfull_bar + 16;                 // [2]
+    const uint32_t drain_bar = tfull_bar + 48;                  // the MMA issuer's last commit
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::STAGES * C::STAGE_BYTES + 16 * C::STAGES + 32);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -105,6 +106,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(tfull_bar + 8 * i, 1);
             mbar_init(tempty_bar + 8 * i, 128);
         }
+        mbar_init(drain_bar, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
@@ -199,7 +201,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
                 int mb, nb, sp, kb0, kb1;
                 ts.get(t, mb, nb, sp, kb0, kb1);
-                if (!mbar_wait(tempty_bar + 8 * acc, acc_phase ^ 1u, abort_flag, err)) break;
+                if (!mbar_wait(tempty_bar + 8 * acc, acc_phase ^ 1u, abort_flag, err)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
                 for (int kb = kb0; kb < kb1; ++kb) {
@@ -226,6 +231,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     acc_phase ^= 1u;
                 }
             }
+            // on the abort path the last products may still be running (on the normal
+            // path the epilogue has waited for every tile's products)
+            if (!ok) mma_drain(drain_bar);
         }
     } else {
         // ------------------------------------------------ epilogue warps 2..5

@@ -117,6 +117,18 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
 }
+
+// Before a CTA ends: wait (bounded) until every tcgen05 operation this thread
+// issued has completed -- a commit to an mbarrier of its own (count 1, used
+// once), then its first phase -- so that no product or commit arrival is
+// still in flight when the tensor memory is freed and the CTA exits, on the
+// abort paths too.
+__device__ __forceinline__ void mma_drain(uint32_t bar) {
+    umma_commit(bar);
+    const uint64_t t0 = global_timer();
+    while (!mbar_try_wait(bar, 0) && global_timer() - t0 < WAIT_LIMIT_NS / 4) {
+    }
+}
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
