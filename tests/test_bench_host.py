@@ -8,7 +8,10 @@
   up to more than the timed step.
 * The DRAM-traffic ratio is used only while the kernel's code (comments and
   layout aside) is the one the counters were taken on.
-* The ncu launch-list summary sums launches and device time per kernel."""
+* The ncu launch-list summary sums launches and device time per kernel.
+* The clock record (median SM clock, active throttle reasons), the decode
+  step's algorithmic bytes (weights once + K/V rows at the mean length) and
+  the per-phase spans of the decode-step timeline."""
 import pytest
 
 import bench
@@ -141,3 +144,54 @@ def test_summarize_ncu_sums_launches_per_kernel(tmp_path, capsys):
     norm = [l for l in out if l.startswith("rmsnorm_kernel")][0].split()
     assert norm[-4] == "1" and float(norm[-3]) == pytest.approx(2.0) and float(norm[-1]) == pytest.approx(0.2)
     assert rows["total"][1] == "3" and float(rows["total"][2]) == pytest.approx(10.0)
+
+
+# ----------------------------------------------------------------------------- clocks, bytes, phases
+
+def test_clock_summary_takes_the_median_and_collects_active_reasons():
+    cs = bench.ClockSampler(0)
+    cs.tmp.write("1965, 1965, 700.1, Not Active, Not Active, Not Active, Active\n"
+                 "1830, 1965, 980.0, Not Active, Not Active, Not Active, Active\n"
+                 "1965, 1965, 990.5, Active, Not Active, Not Active, Not Active\n"
+                 "[N/A], 1965, 0, Not Active, Not Active, Not Active, Not Active\n")
+    out = cs.summary()
+    assert out["sm_mhz"] == 1965.0 and out["sm_max_mhz"] == 1965.0 and out["samples"] == 3
+    assert out["reasons"] == ["hw_slowdown", "sw_power_cap"]
+
+
+def test_clock_summary_without_samples_says_unavailable():
+    cs = bench.ClockSampler(0)
+    assert cs.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+
+def test_decode_bytes_of_the_7b_workload():
+    """Weights once (2 (L (4 d^2 + 3 d h) + d V) bytes) plus K and V rows at the mean
+    length of 128 steps after a 2048-token prompt: 13.21 + 4.43 = 17.64 GB per step."""
+    from synth.workloads import LLAMA_7B
+    flops, step_bytes = bench.algorithmic_work(LLAMA_7B, 4, 2048, 128)
+    d, h, V, L = 4096, 11008, 32000, 32
+    weights = 2.0 * (L * (4 * d * d + 3 * d * h) + d * V)
+    kv = 2.0 * 2 * L * 4 * (2048 + 64.5) * d
+    assert step_bytes == pytest.approx(weights + kv)
+    assert weights / 1e9 == pytest.approx(13.21, abs=0.01) and kv / 1e9 == pytest.approx(4.43, abs=0.01)
+    n = 4 * 2048
+    assert flops == pytest.approx(2.0 * n * (4 * d * d + 3 * d * h) * L + 2.0 * n * d * V
+                                  + 2.0 * 4 * 2048 * 2049 * d * L)
+
+
+def test_step_phases_sum_each_phase_type_over_layers():
+    import numpy as np
+    L = 2
+    P = 3 + 5 * L
+    tl = np.zeros((2, P, 2), dtype=np.uint64)
+    t = 0
+    for p in range(P):          # CTA 0 starts each phase at t, CTA 1 ends it 1000 ns later
+        tl[0, p] = (t, t + 1000)
+        tl[1, p] = (t + 200, t + 2000)
+        t += 2500               # 500 ns gap after every phase
+    out = bench.step_phases(tl, L)
+    assert out["embed"] == 2.0 and out["head"] == 2.0 and out["argmax"] == 2.0
+    for name in ("qkv", "attention", "o_proj", "gate_up", "down"):
+        assert out[name] == 4.0           # 2 us per layer, 2 layers
+    assert out["barrier_gaps"] == pytest.approx(0.5 * (P - 1))
+    assert out["total"] == pytest.approx((2500 * (P - 1) + 2000) / 1e3)
