@@ -108,7 +108,10 @@ typedef struct llama_model llama_model; /* opaque host handle */
  * workspace.  Host-only; queues nothing. */
 LLAMA_API int llama_model_bytes(const llama_config* cfg, uint64_t* bytes_out);
 
-/* Carve the model out of `d_arena` (>= llama_model_bytes, 256-byte aligned)
+/* [PFD] "6.7B parameters, 1T tokens: the arithmetic" fixes the shapes; the
+ * pages give no initialisation (their models are trained), so the weights
+ * are a synthetic stand-in drawn the same way on the GPU and in the oracle.
+ * Carve the model out of `d_arena` (>= llama_model_bytes, 256-byte aligned)
  * and fill the weights on the device from the counter-based generator
  * (Philox4x32-10 keyed by (seed, tensor id), Box-Muller, N(0, 0.02^2),
  * rounded to nearest-even into the storage type; RMSNorm gains 1).  Builds
@@ -128,7 +131,9 @@ LLAMA_API int llama_init_weights(const llama_config* cfg, uint32_t seed, void* d
 LLAMA_API int llama_prefill(llama_model* m, const int32_t* d_tokens, int32_t B, int32_t S,
                   float* d_logits, void* stream);
 
-/* Ragged batch: the same [B, S] token block, but sequence b holds only its
+/* [PFD] "The one formula", causal: each sequence on its own (the pages do
+ * not discuss batching; positions restart at 0 in every sequence).
+ * Ragged batch: the same [B, S] token block, but sequence b holds only its
  * first h_lens[b] tokens (host int32 [B], 1 <= h_lens[b] <= S); the
  * remaining tokens are padding and must be valid ids (their rows are
  * computed and ignored: causal attention keeps them out of every valid
@@ -159,7 +164,10 @@ LLAMA_API int llama_prefill_trunk(llama_model* m, const float* d_x, int32_t B, i
 LLAMA_API int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t* d_next,
                       float* d_logits, void* stream);
 
-/* n_steps greedy steps fed back on the device: step 0 consumes
+/* [NAR] "GQA Was Not an Original LLaMA Feature": autoregressive decoding,
+ * one token per step; greedy (argmax, lowest id on ties) because the pages
+ * name no decoding strategy.
+ * n_steps greedy steps fed back on the device: step 0 consumes
  * d_first [B] (or, when d_first is NULL, the greedy choice at the last
  * position of the preceding llama_prefill that produced logits, or the
  * token the preceding step chose); step i consumes the token step i-1
@@ -168,19 +176,24 @@ LLAMA_API int llama_decode_step(llama_model* m, const int32_t* d_tokens, int32_t
 LLAMA_API int llama_generate(llama_model* m, const int32_t* d_first, int32_t n_steps,
                    int32_t* d_out, void* stream);
 
-/* Current decode position: the largest over the sequences (tokens held
+/* No passage (bookkeeping of the decode positions of llama_decode_step).
+ * Current decode position: the largest over the sequences (tokens held
  * per sequence in the KV cache; all equal unless the batch is ragged). */
 LLAMA_API int llama_position(const llama_model* m);
 
-/* Each sequence's position into h_out (host int32, n >= B); returns B. */
+/* No passage (bookkeeping).  Each sequence's position into h_out (host
+ * int32, n >= B); returns B. */
 LLAMA_API int llama_positions(const llama_model* m, int32_t* h_out, int32_t n);
 
-/* Move every sequence's position back to `position` (1 <= position <= the
+/* No passage (bookkeeping: re-run decoding from an earlier position).
+ * Move every sequence's position back to `position` (1 <= position <= the
  * smallest current position): cache entries below it are kept, later ones
  * are overwritten by the next steps.  Queued on `stream`. */
 LLAMA_API int llama_rewind(llama_model* m, int32_t position, void* stream);
 
-/* End to end from HOST buffers: copy h_tokens (int32 [B*S], host; pinned
+/* [PFD] "The one formula" (prefill) then [NAR] "GQA Was Not an Original
+ * LLaMA Feature" (decoding), as llama_prefill and llama_generate.
+ * End to end from HOST buffers: copy h_tokens (int32 [B*S], host; pinned
  * memory makes the copy asynchronous) to the device, prefill (logits of
  * every position into d_logits [B*S, vocab] when it is not NULL, else the
  * head runs on each sequence's last position only), then n_steps greedy
@@ -189,7 +202,8 @@ LLAMA_API int llama_rewind(llama_model* m, int32_t position, void* stream);
 LLAMA_API int llama_complete(llama_model* m, const int32_t* h_tokens, int32_t B, int32_t S,
                              float* d_logits, int32_t n_steps, int32_t* h_out, void* stream);
 
-/* Device pointer and byte size of an internal buffer, for inspection:
+/* No passage (inspection).
+ * Device pointer and byte size of an internal buffer, for inspection:
  * name in {"kv" (the whole cache), "trunk", "q", "attn", "act", "xn",
  * "embed", "head", "wqkv", "wo", "wgu", "wd"}; `layer` selects the layer for
  * per-layer weights.  Layouts are those of the arena described above. */
@@ -240,7 +254,9 @@ LLAMA_API int llama_set_pages(llama_model* m, const int32_t* h_table, int32_t B,
  * call, once per row chunk and exchange point (2 per block). */
 typedef int (*llama_allreduce_fn)(float* d_buf, uint64_t count, void* stream, void* ctx);
 
-/* Installs the exchange of a shard (tp_size > 1): `fn` with `ctx` is called
+/* [KN] "Efficient Training Implementation" (above): the all-reduce hidden
+ * behind computation.
+ * Installs the exchange of a shard (tp_size > 1): `fn` with `ctx` is called
  * for each all-reduce.  `chunks` (1..16) splits the token rows of every
  * projection after attention into that many blocks (multiples of 128 rows):
  * the all-reduce of block c, queued on a stream of the model's own, runs
@@ -249,28 +265,36 @@ typedef int (*llama_allreduce_fn)(float* d_buf, uint64_t count, void* stream, vo
  * done.  Host-only. */
 LLAMA_API int llama_set_allreduce(llama_model* m, llama_allreduce_fn fn, void* ctx, int32_t chunks);
 
-/* The slices shard cfg->tp_rank of cfg->tp_size holds, into h_out (host
+/* [KN] "Efficient Training Implementation" (above): the model split
+ * across GPUs.
+ * The slices shard cfg->tp_rank of cfg->tp_size holds, into h_out (host
  * int32 [6]): first query head, query heads, first key/value head,
  * key/value heads, first FFN hidden unit, FFN hidden units.  Host-only. */
 LLAMA_API int llama_tp_shard(const llama_config* cfg, int32_t* h_out);
 
-/* Reads (synchronously) and clears the sticky device error word that
+/* No passage (failure detection).
+ * Reads (synchronously) and clears the sticky device error word that
  * bounded device waits set; returns LLAMA_OK or LLAMA_ERR_TIMEOUT. */
 LLAMA_API int llama_last_error(llama_model* m);
 
-/* Releases the host handle (and its captured graphs).  The arena is the
+/* No passage (lifetime).
+ * Releases the host handle (and its captured graphs).  The arena is the
  * caller's to free afterwards. */
 LLAMA_API void llama_free(llama_model* m);
 
+/* No passage.  Static text naming a llama_status value; never NULL. */
 LLAMA_API const char* llama_status_str(int status);
 
-/* --------------------------------------------------------- instrumentation */
+/* --------------------------------------------------------- instrumentation
+ * No passage: measurement of the computation above, not a step of it. */
 
-/* Kernel launches this library has issued in this process; a replay of the
+/* No passage (instrumentation).
+ * Kernel launches this library has issued in this process; a replay of the
  * captured decode graph counts every kernel in it. */
 LLAMA_API int64_t llama_kernel_launches(void);
 
-/* Per-region device timing (process-wide, host-side state).  While enabled,
+/* No passage (instrumentation).
+ * Per-region device timing (process-wide, host-side state).  While enabled,
  * every region of the launch sequence (one GEMM, its reduction, a norm,
  * an attention pass ...) is bracketed by CUDA events on its stream and the
  * decode step runs eagerly instead of as a graph.  Entries accumulate the
@@ -283,7 +307,8 @@ LLAMA_API int llama_profile_count(void);
 LLAMA_API int llama_profile_entry(int32_t i, const char** name, double* ms, int64_t* launches,
                                   int64_t* calls, double* bytes, double* flops);
 
-/* Phase timestamps of the last bf16 decode step run while profiling was
+/* No passage (instrumentation).
+ * Phase timestamps of the last bf16 decode step run while profiling was
  * enabled: h_out (host) receives ctas * phases * 2 %globaltimer values
  * (ns), [cta][phase][start, end]; phases run embed, then per layer QKV,
  * attention, O, gate/up, down, then head and greedy choice.  With
@@ -291,7 +316,8 @@ LLAMA_API int llama_profile_entry(int32_t i, const char** name, double* ms, int6
 LLAMA_API int llama_step_timeline(llama_model* m, uint64_t* h_out, int64_t n, int32_t* ctas,
                                   int32_t* phases);
 
-/* Failure-detection self-test (synchronous): runs one small tensor-core
+/* No passage (failure detection).
+ * Failure-detection self-test (synchronous): runs one small tensor-core
  * GEMM whose activation tile is never requested, so the kernel's bounded
  * wait for it expires (about 2 s); the kernel records the timeout, frees
  * its tensor memory and exits.  Returns LLAMA_ERR_TIMEOUT when the
@@ -303,7 +329,8 @@ LLAMA_API int llama_debug_gemm_timeout(void* stream);
  * The kernels the model runs, exposed one by one on caller buffers.  dtype
  * selects fp32 or bf16 storage of the T-typed operands. */
 
-/* Standalone-op error word: the single ops below (and
+/* No passage (failure detection).
+ * Standalone-op error word: the single ops below (and
  * llama_op_attention_decode_noalloc) record an expired bounded device wait
  * in one word per device, as the model does in its own.  This waits for all
  * work queued on the current device (cudaDeviceSynchronize), then reads and
@@ -353,10 +380,14 @@ LLAMA_API int llama_op_attention_decode(int32_t dtype, const void* d_q, const vo
                               const void* d_v, void* d_o, int32_t B, int32_t H,
                               int32_t len, int32_t head_dim, int32_t kv_stride,
                               void* d_work, uint64_t work_bytes, void* stream);
+/* [NAR] "GQA Was Not an Original LLaMA Feature" (workspace of the decode
+ * attention above): bytes of d_work llama_op_attention_decode needs for
+ * B x H queries over up to max_len keys (host-only; 0 for invalid arguments). */
 LLAMA_API uint64_t llama_op_attention_decode_work_bytes(int32_t B, int32_t H, int32_t max_len,
                                               int32_t head_dim);
 
-/* The same decode attention for callers that cannot allocate device
+/* [NAR] "GQA Was Not an Original LLaMA Feature", as llama_op_attention_decode.
+ * The same decode attention for callers that cannot allocate device
  * memory when they call it (runtimes that plan all device memory up front,
  * code being captured into a CUDA graph that must not allocate, embedders
  * without a device allocator).  The pages have no counterpart: this is an

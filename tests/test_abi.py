@@ -175,3 +175,19 @@ def test_paged_cache_needs_bf16():
     assert lb.lib.llama_model_bytes(ctypes.byref(lb.make_config(TINY, 1, 32, kv_pages=2)), ctypes.byref(n)) == -1
     assert lb.lib.llama_model_bytes(ctypes.byref(lb.make_config(LLAMA_7B, 1, 32, kv_pages=-1)),
                                     ctypes.byref(n)) == -1
+
+
+def test_every_entry_point_cites_its_passage_or_says_it_has_none():
+    """Each declaration in the header comes after a comment that cites the page
+    passage defining its operation ([PFD], [NAR], [KN] tags) or states that
+    there is none (bookkeeping, inspection, instrumentation, failure detection)."""
+    import re
+    from pathlib import Path
+    src = (Path(__file__).resolve().parent.parent / "include" / "llama_b200.h").read_text()
+    missing = []
+    for m in re.finditer(r"^LLAMA_API[^(]*?(\w+)\s*\(", src, re.M):
+        before = src[:m.start()]
+        comment = before[before.rfind("/*"):before.rfind("*/")]
+        if not re.search(r"\[(PFD|NAR|KN)\]|No passage", comment):
+            missing.append(m.group(1))
+    assert not missing, missing
